@@ -26,10 +26,11 @@ Steps, in the order the pages give them:
    gamma * sqrt(pi/2) / m * S^T (2z - 1).
 6. int8 boundary-layer mode — [inferrs] "三个反直觉的关键发现" item 3
    (first and last layers kept at q8_0 precision).  Reading: per-vector
-   absmax scale = fp16(fp32(absmax) / 127), q_i = round-half-even of the
-   fp32 quotient x_i / scale, clamped to [-127, 127]; q = 0 when the
-   scale is 0.  These are the IEEE fp32 operations the kernel performs,
-   so both sides decide every q_i identically.
+   absmax scale = fp16(fp32(absmax) / 127), r = fp32(1 / scale) correctly
+   rounded, q_i = round-half-even of the fp32 product x_i * r, clamped to
+   [-127, 127]; q = 0 when the scale is 0 or infinite.  These are the IEEE
+   fp32 operations the kernel performs, so both sides decide every q_i
+   identically.
 """
 
 import math
@@ -123,9 +124,10 @@ def encode_int8(x):
     with np.errstate(over="ignore"):
         scale16 = (absmax / np.float32(127.0)).astype(np.float32).astype(np.float16)
     scale32 = scale16.astype(np.float32)
-    with np.errstate(divide="ignore", invalid="ignore"):
-        quot = x32 / scale32[..., None]
-    q = np.clip(np.rint(quot), -127, 127)
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+        recip = (np.float32(1.0) / scale32).astype(np.float32)
+        prod = (x32 * recip[..., None]).astype(np.float32)
+    q = np.clip(np.rint(prod), -127, 127)
     q = np.where((scale32 > 0)[..., None] & np.isfinite(scale32)[..., None], q, 0)
     return q.astype(np.int64), scale16
 
