@@ -1,0 +1,452 @@
+"""Benchmark: compressed decode attention over a TurboQuant KV cache.
+
+Default workload (one step): a Llama-3-8B-shaped decode step over 32
+attention layers, each with its own compressed cache -- batch 1, 32 query
+heads, 8 KV heads (GQA 4), d = 128, 32768 cached tokens, K 4-bit / V 2-bit.
+Per layer the step appends one new token (quantise-append of its K and V)
+and runs decode attention over the whole cache (32769+ tokens).  Inputs are
+seeded synthetic bf16 data (log-normal per-channel scales, sigma 1); the 32
+distinct caches (839 MB) are far larger than L2, so every layer's cache
+comes from HBM.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
+oracle on the same workload instead (bounded sample per step).
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+LAYERS, BATCH, HQ, HKV, D, CONTEXT = 32, 1, 32, 8, 128, 32768
+K_BITS, V_BITS = 4, 2
+SEED = 1234
+WORKLOAD = "llama3-8b-shaped decode step: 32 layers x (append 1 token + decode attention), B=1, Hq=32, Hkv=8, " \
+           "d=128, context 32768, K4/V2 packed cache"
+METRIC = "compressed decode-attn KV tokens/s"
+
+
+def bytes_per_token_head(k_bits=K_BITS, v_bits=V_BITS, d=D):
+    """Algorithmic bytes one decode step reads per cached token and kv head."""
+    return d * k_bits // 8 + 2 + d * v_bits // 8 + 2
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active," \
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown," \
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        with open(self.file.name) as fh:
+            rows = [r.split(",") for r in fh.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], [], set()
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip() == "Active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            j = json.load(fh)
+        return float(j["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ oracle leg
+class OracleDecode:
+    """The fp64 CPU oracle on a bounded sample of the decode step.  One unit
+    of work = one (kv head) of one layer: encode the appended token, dequantise
+    the unit's cached tokens and attend with its 4 query heads.  The cache
+    contents (prefill) are built once, untimed."""
+
+    def __init__(self, context=CONTEXT, units=2):
+        from oracle import codebook as ocb, quantize as oq, rng as orng
+        from bit_kv_cache_tq_b200 import inputs
+        self.oq = oq
+        self.context = context
+        self.kc, self.kt = ocb.lloyd_max(D, K_BITS)
+        self.vc, self.vt = ocb.lloyd_max(D, V_BITS)
+        self.signs = orng.rotation_signs(SEED, D)
+        k = inputs.lognormal_kv(1, context + 1, units, D, seed=SEED, layer=0, which=inputs.K).float().numpy()
+        v = inputs.lognormal_kv(1, context + 1, units, D, seed=SEED, layer=0, which=inputs.V).float().numpy()
+        self.q = inputs.queries(1, HQ, D, seed=SEED).float().numpy().astype(np.float64)
+        self.new = [(k[0, context:, h], v[0, context:, h]) for h in range(units)]
+        self.caches = [(oq.encode_turbo(k[0, :context, h], self.signs, self.kc, self.kt, K_BITS),
+                        oq.encode_turbo(v[0, :context, h], self.signs, self.vc, self.vt, V_BITS))
+                       for h in range(units)]
+        self.done = 0
+
+    def unit(self):
+        from oracle import attention as oatt
+        oq, h = self.oq, self.done % len(self.caches)
+        ek, ev = self.caches[h]
+        nk = oq.encode_turbo(self.new[h][0], self.signs, self.kc, self.kt, K_BITS)
+        nv = oq.encode_turbo(self.new[h][1], self.signs, self.vc, self.vt, V_BITS)
+        khat = oq.dequantize_turbo(np.concatenate([ek["codes"], nk["codes"]]),
+                                   np.concatenate([ek["norm16"], nk["norm16"]]), self.signs, self.kc)
+        vhat = oq.dequantize_turbo(np.concatenate([ev["codes"], nv["codes"]]),
+                                   np.concatenate([ev["norm16"], nv["norm16"]]), self.signs, self.vc)
+        g = HQ // HKV
+        oatt.decode_attention(self.q[:, h * g:(h + 1) * g], khat[None, None], vhat[None, None], [self.context + 1])
+        self.done += 1
+
+    def tokens_per_unit(self):
+        return (self.context + 1) / HKV  # a layer token spans all 8 kv heads
+
+    @staticmethod
+    def cores():
+        try:
+            from threadpoolctl import threadpool_info
+            return max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+        except Exception:
+            return os.cpu_count()
+
+
+def oracle_sample(seconds_target=12.0):
+    """(tokens/s, cpu_baseline dict) of the oracle over ~seconds_target of work."""
+    w = OracleDecode()
+    w.unit()  # warm-up
+    n = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds_target:
+        w.unit()
+        n += 1
+    dt = time.perf_counter() - t0
+    val = n * w.tokens_per_unit() / dt
+    return val, {"kind": "oracle", "cores": w.cores(), "value": val, "unit": "tokens/s",
+                 "sample": "%d (kv head) units of one layer, each: encode 1 appended token, dequantise %d cached "
+                           "tokens, 4-head attention (fp64 numpy); %.1f s; a layer token = 8 kv-head vectors"
+                           % (n, CONTEXT, dt)}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = OracleDecode()
+    for _ in range(args.warmup):
+        w.unit()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        w.unit()
+    dt = time.perf_counter() - t0
+    value = args.steps * w.tokens_per_unit() / dt
+    info = {"kind": "oracle", "cores": w.cores(), "value": value, "unit": "tokens/s",
+            "sample": "each step: one (kv head) unit of one layer (encode 1 appended token, dequantise 32768 "
+                      "cached tokens, 4-head attention), fp64 numpy; a layer token = 8 kv-head vectors"}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": BATCH, "seq_len": CONTEXT + 1, "parallelism": "none"},
+            "cpu_baseline": info,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU leg
+def run_tq(args, world, rank, local):
+    from bit_kv_cache_tq_b200 import inputs, tq
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    steps, warmup = args.steps, args.warmup
+    total_steps = steps + warmup
+    cap = CONTEXT + total_steps + 1
+    gen_seed = SEED + 7919 * rank
+    kcb, vcb = tq.tq_codebook_init(D, K_BITS), tq.tq_codebook_init(D, V_BITS)
+    params = [tq.make_params(D, HQ, HKV, K_BITS, V_BITS, seed=gen_seed + l) for l in range(LAYERS)]
+    caches = [tq.alloc_cache(p, BATCH, cap, device=dev) for p in params]
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    zero_pos = torch.zeros(BATCH, dtype=torch.int32, device=dev)
+    # prefill: quantise the 32768-token context of every layer on the GPU (set-up)
+    for l in range(LAYERS):
+        k = inputs.lognormal_kv(BATCH, CONTEXT, HKV, D, gen_seed, l, inputs.K, device=dev)
+        v = inputs.lognormal_kv(BATCH, CONTEXT, HKV, D, gen_seed, l, inputs.V, device=dev)
+        tq.tq_quantize_append(params[l], kcb, vcb, k, v, zero_pos, caches[l], err)
+        del k, v
+    # per-step inputs, resident in HBM: new K/V tokens and queries per layer
+    k_new = [inputs.lognormal_kv(BATCH, total_steps, HKV, D, gen_seed, l, inputs.K, device=dev, token_offset_seed=1)
+             for l in range(LAYERS)]
+    v_new = [inputs.lognormal_kv(BATCH, total_steps, HKV, D, gen_seed, l, inputs.V, device=dev, token_offset_seed=1)
+             for l in range(LAYERS)]
+    qs = [[inputs.queries(BATCH, HQ, D, gen_seed, layer=l, step=i, device=dev) for i in range(total_steps)]
+          for l in range(LAYERS)]
+    positions = torch.arange(CONTEXT, CONTEXT + total_steps, dtype=torch.int32, device=dev).view(total_steps, 1)
+    lens = positions + 1
+    outs = torch.empty(LAYERS, BATCH, HQ, D, dtype=torch.float32, device=dev)
+    ws = torch.zeros(tq.tq_decode_workspace_bytes(params[0], BATCH, cap), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    st, word = tq.tq_read_device_error(err)
+    assert st == tq.TQ_OK, ("prefill", st, word)
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def enqueue_step(i, decode_only=False):
+        for l in range(LAYERS):
+            if not decode_only:
+                tq.tq_quantize_append(params[l], kcb, vcb, k_new[l][:, i:i + 1], v_new[l][:, i:i + 1], positions[i],
+                                      caches[l], err, stream=stream)
+            tq.tq_decode_attention(params[l], kcb, vcb, qs[l][i], caches[l], lens[i], cap, outs[l], ws, err,
+                                   stream=stream)
+
+    # one CUDA graph per step (the pointers of step i are baked in)
+    graphs = []
+    with torch.cuda.stream(stream):
+        for i in range(total_steps):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                enqueue_step(i)
+            graphs.append(g)
+        g_decode = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_decode, stream=stream):
+            enqueue_step(total_steps - 1, decode_only=True)
+    torch.cuda.synchronize()
+
+    for i in range(warmup):
+        graphs[i].replay()
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for i in range(warmup, total_steps):
+                graphs[i].replay()
+            end.record(stream)
+        end.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = start.elapsed_time(end)
+    ms = max_over_ranks(ms, world)
+    tokens_per_step = sum(LAYERS * BATCH * (CONTEXT + i + 1) for i in range(warmup, total_steps)) / steps
+    value = world * tokens_per_step * steps / (ms / 1000.0)
+    st, word = tq.tq_read_device_error(err)
+    assert st == tq.TQ_OK, ("timed steps", st, word)
+
+    # dominant kernel: decode attention alone, 32 layers per graph replay
+    reps = 20
+    with torch.cuda.stream(stream):
+        g_decode.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g_decode.replay()
+        e1.record(stream)
+    e1.synchronize()
+    decode_us = 1000.0 * e0.elapsed_time(e1) / (reps * LAYERS)
+    seq = CONTEXT + total_steps
+    alg_bytes = BATCH * HKV * seq * bytes_per_token_head()
+    achieved = alg_bytes / (decode_us * 1e-6) / 1e9
+    peak, peak_kind = measured_peaks()
+
+    # end to end through the C ABI with host buffers: pinned inputs copied in,
+    # outputs copied out, every step
+    h_k = [torch.empty(BATCH, 1, HKV, D, dtype=torch.bfloat16).pin_memory() for _ in range(LAYERS)]
+    h_v = [torch.empty(BATCH, 1, HKV, D, dtype=torch.bfloat16).pin_memory() for _ in range(LAYERS)]
+    h_q = [torch.empty(BATCH, HQ, D, dtype=torch.bfloat16).pin_memory() for _ in range(LAYERS)]
+    for l in range(LAYERS):
+        h_k[l].copy_(k_new[l][:, -1:])
+        h_v[l].copy_(v_new[l][:, -1:])
+        h_q[l].copy_(qs[l][-1])
+    h_out = torch.empty(LAYERS, BATCH, HQ, D, dtype=torch.float32).pin_memory()
+    s_k = [torch.empty(BATCH, 1, HKV, D, dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
+    s_v = [torch.empty(BATCH, 1, HKV, D, dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
+    s_q = [torch.empty(BATCH, HQ, D, dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
+    last = total_steps - 1
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g_e2e, stream=stream):
+            for l in range(LAYERS):
+                tq.tq_quantize_append(params[l], kcb, vcb, s_k[l], s_v[l], positions[last], caches[l], err,
+                                      stream=stream)
+                tq.tq_decode_attention(params[l], kcb, vcb, s_q[l], caches[l], lens[last], cap, outs[l], ws, err,
+                                       stream=stream)
+    torch.cuda.synchronize()
+    h2d = sum(t.numel() * t.element_size() for t in h_k + h_v + h_q)
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_steps = steps
+    with torch.cuda.stream(stream):
+        for it in range(warmup + e2e_steps):
+            if it == warmup:
+                stream.synchronize()
+                t_e2e = time.perf_counter()
+                f0 = torch.cuda.Event(enable_timing=True)
+                f1 = torch.cuda.Event(enable_timing=True)
+                f0.record(stream)
+            for l in range(LAYERS):
+                s_k[l].copy_(h_k[l], non_blocking=True)
+                s_v[l].copy_(h_v[l], non_blocking=True)
+                s_q[l].copy_(h_q[l], non_blocking=True)
+            g_e2e.replay()
+            h_out.copy_(outs, non_blocking=True)
+        f1.record(stream)
+    f1.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
+    e2e_value = world * LAYERS * BATCH * (last + CONTEXT + 1) * e2e_steps / (e2e_ms / 1000.0)
+
+    launches_per_step = LAYERS * 2  # quantise-append, decode attention (splits and merge fused)
+    if rank == 0:
+        cpu_info = oracle_sample(seconds_target=12.0)[1] if (world == 1 and not args.no_cpu_baseline) else None
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": warmup, "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": BATCH * world, "seq_len": CONTEXT + 1,
+                       "layers": LAYERS, "parallelism": "replicas%d" % world if world > 1 else "none",
+                       "l2": "inputs larger than L2: 32 distinct layer caches, %.0f MB" %
+                             (LAYERS * HKV * seq * bytes_per_token_head() / 1e6),
+                       "graphs": "one CUDA graph per step (32 x append + decode)"},
+            "hbm_gbs": alg_bytes * LAYERS / (ms / steps * 1e-3) / 1e9,
+            "pct_of_8tbs": 100.0 * alg_bytes * LAYERS / (ms / steps * 1e-3) / 8e12,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "tq_decode_attention (one fused kernel), %.2f us per launch, %d B algorithmic"
+                                   % (decode_us, alg_bytes)},
+            "cpu_baseline": cpu_info,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    del graphs, g_decode, g_e2e
+
+
+def run_profile_case(args):
+    """A small case for ncu: one Llama-3-8B-shaped layer (26 MB cache) and a
+    few eager launches of one kernel; prints nothing worth timing."""
+    from bit_kv_cache_tq_b200 import inputs, tq
+    dev = torch.device("cuda", 0)
+    params = tq.make_params(D, HQ, HKV, K_BITS, V_BITS, seed=SEED)
+    kcb, vcb = tq.tq_codebook_init(D, K_BITS), tq.tq_codebook_init(D, V_BITS)
+    cap = CONTEXT + 8
+    cache = tq.alloc_cache(params, BATCH, cap, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    pos = torch.zeros(BATCH, dtype=torch.int32, device=dev)
+    k = inputs.lognormal_kv(BATCH, CONTEXT + 1, HKV, D, SEED, 0, inputs.K, device=dev)
+    v = inputs.lognormal_kv(BATCH, CONTEXT + 1, HKV, D, SEED, 0, inputs.V, device=dev)
+    if args.profile == "quantize":
+        for _ in range(args.warmup + args.steps):
+            tq.tq_quantize_append(params, kcb, vcb, k, v, pos, cache, err)
+    else:
+        tq.tq_quantize_append(params, kcb, vcb, k, v, pos, cache, err)
+        q = inputs.queries(BATCH, HQ, D, SEED, device=dev)
+        lens = torch.full((BATCH,), CONTEXT + 1, dtype=torch.int32, device=dev)
+        ws = torch.zeros(tq.tq_decode_workspace_bytes(params, BATCH, cap), dtype=torch.uint8, device=dev)
+        out = torch.empty(BATCH, HQ, D, dtype=torch.float32, device=dev)
+        for _ in range(args.warmup + args.steps):
+            tq.tq_decode_attention(params, kcb, vcb, q, cache, lens, cap, out, ws, err)
+    torch.cuda.synchronize()
+    st, word = tq.tq_read_device_error(err)
+    assert st == tq.TQ_OK, (st, word)
+    print(json.dumps({"profile_case": args.profile, "launches": args.warmup + args.steps + (args.profile != "quantize")}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["decode", "quantize"], default=None,
+                    help="run a small one-layer case for ncu instead of the benchmark")
+    args = ap.parse_args()
+    if args.profile:
+        run_profile_case(args)
+        return
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_tq(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,47 @@
+// Internal declarations shared by the host code and the kernel launchers.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "tq.h"
+
+namespace tq {
+
+// Decode split plan: the token axis of every (sequence, kv head) is cut into
+// n_split ranges of split_len tokens (the last one may be shorter or empty).
+struct DecodePlan {
+    int n_split = 1;
+    int split_len = 0;
+    size_t off_ml = 0;   // float2 (m, l) per (b, hq, split)
+    size_t off_acc = 0;  // float acc[d] per (b, hq, split)
+    size_t off_counters = 0;  // uint32 per (b, kv head): splits finished
+    size_t bytes = 0;
+};
+
+// Thread blocks aimed at per SM when choosing the split count.
+constexpr int kBlocksPerSm = 2;
+// Smallest token range worth a separate split.
+constexpr int kMinSplitTokens = 256;
+// Most splits per (sequence, kv head); bounds the merge scratch in shared memory.
+constexpr int kMaxSplits = 384;
+// Token granularity of split boundaries.
+constexpr int kSplitAlign = 64;
+
+tq_status validate_params(const tq_params* p);
+tq_status validate_codebook(const tq_codebook* cb, int head_dim, int bits);
+tq_status validate_cache(const tq_params& p, const tq_cache* c);
+bool aligned16(const void* ptr);
+// Bytes of one stored vector: d*bits/8 (TURBO) or d (INT8).
+int vector_bytes(int mode, int bits, int head_dim);
+DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_sms);
+// Tensor-core decode path (decode_mma.cu): d = 128, TURBO K and V.
+bool decode_mma_supported(const tq_params& p);
+// SM count of the current CUDA device (0 when it cannot be queried).
+int num_sms_current();
+// Centroid scale in [8, 16) minimising the largest relative fp16 rounding error.
+double best_fp16_scale(const double* c, int n);
+// Rotation signs as a bit mask: bit i set <=> s_i = -1.
+void rotation_sign_bits(uint64_t seed, int head_dim, uint32_t words[8]);
+
+}  // namespace tq

@@ -1,0 +1,475 @@
+// Quantise-append and dequantise kernels (sm_100a) and their C entry points.
+//
+// Pages (by title):
+//   [tqai]    "TurboQuant：让大模型本地推理内存占用降低80%的KV缓存压缩技术",
+//             section "TurboQuant的核心创新：极坐标量化与随机旋转"
+//   [inferrs] "inferrs & TurboQuant：本地 LLM 推理的内存革命", sections
+//             "核心技术", "压缩格式对比", "三个反直觉的关键发现"
+//   [fwht]    "TurboQuant：用Rust核心与FWHT预处理实现LLM推理的4-bit KV缓存量化",
+//             section "2. 快速Walsh-Hadamard变换（FWHT）预处理"
+//   [google]  "Google 最新極限壓縮算法，砸碎大模型本地部署的內存墻，8 倍提升！",
+//             section "第二步：QJL —— 1 bit 清理殘差"
+//
+// Work layout: a head vector of d coordinates is held by d/32 lanes, 32
+// coordinates each.  The vector is read as 16-byte chunks of 8 elements;
+// lane j of the vector's lane group holds chunks j, j + d/32, j + 2d/32,
+// j + 3d/32, so every load instruction of a warp covers whole 32-byte
+// sectors.  The Walsh-Hadamard transform then runs 5 butterfly stages in
+// registers and log2(d/32) stages across lanes (warp shuffles).
+
+#include <cuda_runtime.h>
+
+#include <chrono>
+#include <cmath>
+#include <thread>
+
+#include "device_common.cuh"
+#include "internal.h"
+
+namespace tq {
+
+struct QuantSide {
+    const void* src;        // [batch][n_new][Hkv][d]
+    uint8_t* codes;         // [batch][Hkv][capacity][vbytes]
+    uint16_t* norms;        // [batch][Hkv][capacity]
+    uint8_t* qjl;           // [batch][Hkv][capacity][m/8] or null
+    uint16_t* gamma;        // [batch][Hkv][capacity] or null
+    const float* sketch;    // [m][d] or null
+    int mode, bits, vbytes, m;
+    float centroids[16];
+    float pos_boundaries[8];  // boundaries above zero, ascending (2^(bits-1) - 1 of them)
+};
+
+struct QuantArgs {
+    QuantSide side[2];  // 0 = K, 1 = V
+    const int32_t* positions;
+    uint32_t* err;
+    int batch, n_new, hkv, capacity;
+    uint32_t signs[8];
+};
+
+// Code of a rotated unit coordinate y: the number of boundaries below it.
+// With an odd-symmetric table the middle boundary is 0, so the count is
+// 2^(b-1) + #{t_k > 0 : |y| > t_k} for y > 0 and 2^(b-1) - 1 - #{...} otherwise
+// (an exact tie |y| == t_k on the negative side lands one cell high, inside
+// the boundary window the codes are compared with).
+template <int BITS>
+__device__ __forceinline__ uint32_t code_of(float y, const float* tpos) {
+    constexpr int half = 1 << (BITS - 1);
+    const float a = fabsf(y);
+    int m = 0;
+#pragma unroll
+    for (int k = 0; k < half - 1; ++k) m += a > tpos[k];
+    return y > 0.0f ? static_cast<uint32_t>(half + m) : static_cast<uint32_t>(half - 1 - m);
+}
+
+template <int BITS>
+__device__ __forceinline__ void store_chunk_codes(uint8_t* row, int chunk, uint32_t packed) {
+    if constexpr (BITS == 4) {
+        *reinterpret_cast<uint32_t*>(row + 4 * chunk) = packed;
+    } else if constexpr (BITS == 2) {
+        *reinterpret_cast<uint16_t*>(row + 2 * chunk) = static_cast<uint16_t>(packed);
+    } else {
+        row[3 * chunk] = static_cast<uint8_t>(packed);
+        row[3 * chunk + 1] = static_cast<uint8_t>(packed >> 8);
+        row[3 * chunk + 2] = static_cast<uint8_t>(packed >> 16);
+    }
+}
+
+template <int D, int BITS>
+__device__ __forceinline__ void turbo_encode(const QuantSide& s, float (&x)[32], int sub, size_t slot, bool valid,
+                                             const uint32_t* signs) {
+    constexpr int LPV = D / 32;
+    float sumsq = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int i = 8 * (sub + LPV * k) + e;
+            sumsq = fmaf(x[8 * k + e], x[8 * k + e], sumsq);
+            x[8 * k + e] = flip_sign(x[8 * k + e], sign_bit(signs, i));
+        }
+    fwht_registers(x);
+    fwht_lanes<32, LPV>(x, sub);
+    sumsq = group_sum<LPV>(sumsq);
+    const float n = sqrtf(sumsq);
+    const float inv = n > 0.0f ? 1.0f / (sqrtf(static_cast<float>(D)) * n) : 0.0f;
+    uint32_t codes[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        x[i] *= inv;  // rotated unit-vector coordinate y_i
+        codes[i] = code_of<BITS>(x[i], s.pos_boundaries);
+    }
+    if (valid) {
+        uint8_t* row = s.codes + slot * static_cast<size_t>(s.vbytes);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            uint32_t packed = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) packed |= codes[8 * k + e] << (BITS * e);
+            store_chunk_codes<BITS>(row, sub + LPV * k, packed);
+        }
+        if (sub == 0) s.norms[slot] = float_to_half_bits(n);
+    }
+    if (s.m > 0) {  // QJL residual sketch (keys only)
+        float g2 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            x[i] -= s.centroids[codes[i]];  // residual r_i
+            g2 = fmaf(x[i], x[i], g2);
+        }
+        g2 = group_sum<LPV>(g2);
+        uint32_t word = 0;
+        for (int r = 0; r < s.m; ++r) {
+            const float* row = s.sketch + static_cast<size_t>(r) * D;
+            float acc = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float4 a = __ldg(reinterpret_cast<const float4*>(row + 8 * (sub + LPV * k)));
+                const float4 b = __ldg(reinterpret_cast<const float4*>(row + 8 * (sub + LPV * k) + 4));
+                acc = fmaf(a.x, x[8 * k + 0], acc); acc = fmaf(a.y, x[8 * k + 1], acc);
+                acc = fmaf(a.z, x[8 * k + 2], acc); acc = fmaf(a.w, x[8 * k + 3], acc);
+                acc = fmaf(b.x, x[8 * k + 4], acc); acc = fmaf(b.y, x[8 * k + 5], acc);
+                acc = fmaf(b.z, x[8 * k + 6], acc); acc = fmaf(b.w, x[8 * k + 7], acc);
+            }
+            acc = group_sum<LPV>(acc);
+            word |= static_cast<uint32_t>(acc >= 0.0f) << (r & 31);
+            if ((r & 31) == 31) {
+                if (valid && sub == 0)
+                    reinterpret_cast<uint32_t*>(s.qjl + slot * static_cast<size_t>(s.m / 8))[r >> 5] = word;
+                word = 0;
+            }
+        }
+        if (valid && sub == 0) s.gamma[slot] = float_to_half_bits(sqrtf(g2));
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void int8_encode(const QuantSide& s, const float (&x)[32], int sub, size_t slot,
+                                            bool valid) {
+    constexpr int LPV = D / 32;
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    amax = group_max<LPV>(amax);
+    const __half scale16 = __float2half_rn(__fdiv_rn(amax, 127.0f));
+    const float scale = __half2float(scale16);
+    const float recip = (scale > 0.0f && scale < INFINITY) ? __frcp_rn(scale) : 0.0f;
+    if (!valid) return;
+    uint8_t* row = s.codes + slot * static_cast<size_t>(D);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float q = fminf(fmaxf(rintf(__fmul_rn(x[8 * k + e], recip)), -127.0f), 127.0f);
+            const uint32_t byte = static_cast<uint32_t>(static_cast<int32_t>(q)) & 0xffu;
+            if (e < 4) lo |= byte << (8 * e);
+            else hi |= byte << (8 * (e - 4));
+        }
+        *reinterpret_cast<uint2*>(row + 8 * (sub + LPV * k)) = make_uint2(lo, hi);
+    }
+    if (sub == 0) s.norms[slot] = __half_as_ushort(scale16);
+}
+
+template <int D, int DTYPE>
+__global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_constant__ QuantArgs a) {
+    constexpr int LPV = D / 32;  // lanes per vector
+    constexpr int VPW = 32 / LPV;  // vectors per warp pass
+    const QuantSide& s = a.side[blockIdx.y];
+    const int lane = threadIdx.x & 31, sub = lane % LPV, grp = lane / LPV;
+    const long long total = static_cast<long long>(a.batch) * a.n_new * a.hkv;
+    const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+    for (long long base = (static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32) * VPW;
+         base < total; base += nwarps * VPW) {
+        const long long v = base + grp;
+        bool valid = v < total;
+        size_t slot = 0;
+        if (valid) {
+            const int h = static_cast<int>(v % a.hkv);
+            const long long bt = v / a.hkv;
+            const int t = static_cast<int>(bt % a.n_new);
+            const int b = static_cast<int>(bt / a.n_new);
+            const int pos = a.positions[b];
+            if (pos < 0 || pos > a.capacity - a.n_new) {
+                if (a.err && t == 0 && h == 0 && sub == 0 && blockIdx.y == 0) atomicOr(a.err, TQ_DEVERR_POSITION);
+                valid = false;
+            } else {
+                slot = (static_cast<size_t>(b) * a.hkv + h) * a.capacity + pos + t;
+            }
+        }
+        float x[32];
+        if (v < total) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                load8_stream<DTYPE>(s.src, static_cast<size_t>(v) * D + 8 * (sub + LPV * k), &x[8 * k]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = 0.0f;
+        }
+        if (s.mode == TQ_MODE_INT8) {
+            int8_encode<D>(s, x, sub, slot, valid);
+        } else if (s.bits == 4) {
+            turbo_encode<D, 4>(s, x, sub, slot, valid, a.signs);
+        } else if (s.bits == 3) {
+            turbo_encode<D, 3>(s, x, sub, slot, valid, a.signs);
+        } else {
+            turbo_encode<D, 2>(s, x, sub, slot, valid, a.signs);
+        }
+    }
+}
+
+// ------------------------------------------------------------- dequantise
+struct DequantArgs {
+    QuantSide side[2];
+    float* out[2];
+    int b, start, count, hkv, capacity;
+    uint32_t signs[8];
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) dequantize_kernel(const __grid_constant__ DequantArgs a) {
+    constexpr int LPV = D / 32;
+    constexpr int VPW = 32 / LPV;
+    const QuantSide& s = a.side[blockIdx.y];
+    float* out = a.out[blockIdx.y];
+    if (!out) return;
+    const int lane = threadIdx.x & 31, sub = lane % LPV, grp = lane / LPV;
+    const long long total = static_cast<long long>(a.count) * a.hkv;
+    const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+    for (long long base = (static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32) * VPW;
+         base < total; base += nwarps * VPW) {
+        const long long v = base + grp;
+        const bool valid = v < total;
+        const int h = valid ? static_cast<int>(v % a.hkv) : 0;
+        const int t = valid ? static_cast<int>(v / a.hkv) : 0;
+        const size_t slot = (static_cast<size_t>(a.b) * a.hkv + h) * a.capacity + a.start + t;
+        float x[32];
+        if (s.mode == TQ_MODE_INT8) {
+            const float scale = valid ? half_bits_to_float(s.norms[slot]) : 0.0f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint2 w = valid ? *reinterpret_cast<const uint2*>(s.codes + slot * D + 8 * (sub + LPV * k))
+                                      : make_uint2(0, 0);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const uint32_t word = e < 4 ? w.x : w.y;
+                    const int8_t q = static_cast<int8_t>((word >> (8 * (e & 3))) & 0xffu);
+                    x[8 * k + e] = scale * static_cast<float>(q);
+                }
+            }
+        } else {
+            const uint32_t* words = reinterpret_cast<const uint32_t*>(s.codes + slot * static_cast<size_t>(s.vbytes));
+            const int nwords = s.vbytes / 4;
+            const uint32_t mask = (1u << s.bits) - 1u;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t chunk = valid ? stream_bits(words, nwords, 8 * s.bits * (sub + LPV * k), 8 * s.bits) : 0u;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[8 * k + e] = s.centroids[(chunk >> (s.bits * e)) & mask];
+            }
+            if (s.m > 0 && valid) {
+                const float coef = half_bits_to_float(s.gamma[slot]) * sqrtf(0.5f * 3.14159265358979f) / s.m;
+                const uint32_t* z = reinterpret_cast<const uint32_t*>(s.qjl + slot * static_cast<size_t>(s.m / 8));
+                for (int r = 0; r < s.m; ++r) {
+                    const float w = (z[r >> 5] >> (r & 31)) & 1u ? coef : -coef;
+                    const float* row = s.sketch + static_cast<size_t>(r) * D;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[8 * k + e] = fmaf(w, __ldg(row + 8 * (sub + LPV * k) + e), x[8 * k + e]);
+                }
+            }
+            fwht_registers(x);
+            fwht_lanes<32, LPV>(x, sub);
+            const float scale = (valid ? half_bits_to_float(s.norms[slot]) : 0.0f) / sqrtf(static_cast<float>(D));
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int i = 8 * (sub + LPV * k) + e;
+                    x[8 * k + e] = flip_sign(x[8 * k + e] * scale, sign_bit(a.signs, i));
+                }
+        }
+        if (valid) {
+            float* dst = out + static_cast<size_t>(v) * D;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float4* p = reinterpret_cast<float4*>(dst + 8 * (sub + LPV * k));
+                p[0] = make_float4(x[8 * k + 0], x[8 * k + 1], x[8 * k + 2], x[8 * k + 3]);
+                p[1] = make_float4(x[8 * k + 4], x[8 * k + 5], x[8 * k + 6], x[8 * k + 7]);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- launchers
+static void fill_side(QuantSide& s, int mode, int bits, int d, const tq_codebook* cb) {
+    s.mode = mode;
+    s.bits = mode == TQ_MODE_INT8 ? 8 : bits;
+    s.vbytes = vector_bytes(mode, bits, d);
+    for (int j = 0; j < 16; ++j) s.centroids[j] = 0.0f;
+    for (int j = 0; j < 8; ++j) s.pos_boundaries[j] = INFINITY;
+    if (mode == TQ_MODE_TURBO) {
+        const int n = 1 << bits, half = n / 2;
+        for (int j = 0; j < n; ++j) s.centroids[j] = static_cast<float>(cb->centroids[j]);
+        for (int k = 0; k < half - 1; ++k) s.pos_boundaries[k] = static_cast<float>(cb->boundaries[half + k]);
+    }
+}
+
+int num_sms_current() {  // SM count of the current device, 0 if unknown
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return sms;
+}
+
+template <int D, int DTYPE>
+static cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t stream) {
+    constexpr int VPW = 32 / (D / 32);
+    const long long total = static_cast<long long>(a.batch) * a.n_new * a.hkv;
+    const long long warps_needed = (total + VPW - 1) / VPW;
+    const int sms = num_sms_current();
+    long long blocks = (warps_needed + 7) / 8;
+    const long long cap = static_cast<long long>(sms > 0 ? sms : 148) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    quantize_append_kernel<D, DTYPE><<<dim3(static_cast<unsigned>(blocks), 2), 256, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_quantize_dtype(const QuantArgs& a, int dtype, cudaStream_t stream) {
+    switch (dtype) {
+        case TQ_F32: return launch_quantize<D, 0>(a, stream);
+        case TQ_BF16: return launch_quantize<D, 1>(a, stream);
+        default: return launch_quantize<D, 2>(a, stream);
+    }
+}
+
+}  // namespace tq
+
+// =================================================================== C ABI
+extern "C" {
+
+tq_status tq_quantize_append(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                             const void* k_new, const void* v_new, tq_dtype dtype, int32_t n_new,
+                             const int32_t* d_positions, const tq_cache* cache, uint32_t* d_error,
+                             void* stream) {
+    using namespace tq;
+    tq_status st = validate_params(params);
+    if (st != TQ_OK) return st;
+    const tq_params& p = *params;
+    if ((st = validate_cache(p, cache)) != TQ_OK) return st;
+    if (!k_new || !v_new || !d_positions || n_new < 1) return TQ_ERR_INVALID_ARG;
+    if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new)) return TQ_ERR_ALIGNMENT;
+    if (n_new > cache->capacity) return TQ_ERR_CAPACITY;
+    if (p.k_mode == TQ_MODE_TURBO && (st = validate_codebook(kcb, p.head_dim, p.k_bits)) != TQ_OK) return st;
+    if (p.v_mode == TQ_MODE_TURBO && (st = validate_codebook(vcb, p.head_dim, p.v_bits)) != TQ_OK) return st;
+    QuantArgs a{};
+    fill_side(a.side[0], p.k_mode, p.k_bits, p.head_dim, kcb);
+    fill_side(a.side[1], p.v_mode, p.v_bits, p.head_dim, vcb);
+    a.side[0].src = k_new;
+    a.side[0].codes = cache->k_codes;
+    a.side[0].norms = cache->k_norms;
+    a.side[0].qjl = cache->k_qjl;
+    a.side[0].gamma = cache->k_gamma;
+    a.side[0].sketch = cache->qjl_matrix;
+    a.side[0].m = p.qjl_dims;
+    a.side[1].src = v_new;
+    a.side[1].codes = cache->v_codes;
+    a.side[1].norms = cache->v_norms;
+    a.side[1].m = 0;
+    a.positions = d_positions;
+    a.err = d_error;
+    a.batch = cache->batch;
+    a.n_new = n_new;
+    a.hkv = p.num_kv_heads;
+    a.capacity = cache->capacity;
+    rotation_sign_bits(p.seed, p.head_dim, a.signs);
+    cudaError_t e;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    switch (p.head_dim) {
+        case 64: e = launch_quantize_dtype<64>(a, dtype, s); break;
+        case 128: e = launch_quantize_dtype<128>(a, dtype, s); break;
+        default: e = launch_quantize_dtype<256>(a, dtype, s); break;
+    }
+    return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+tq_status tq_dequantize(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                        const tq_cache* cache, int32_t b, int32_t start, int32_t count, float* d_k_out,
+                        float* d_v_out, void* stream) {
+    using namespace tq;
+    tq_status st = validate_params(params);
+    if (st != TQ_OK) return st;
+    const tq_params& p = *params;
+    if ((st = validate_cache(p, cache)) != TQ_OK) return st;
+    if (b < 0 || b >= cache->batch || start < 0 || count < 1 || start > cache->capacity - count)
+        return TQ_ERR_INVALID_ARG;
+    if (!d_k_out && !d_v_out) return TQ_ERR_INVALID_ARG;
+    if ((d_k_out && !aligned16(d_k_out)) || (d_v_out && !aligned16(d_v_out))) return TQ_ERR_ALIGNMENT;
+    if (p.k_mode == TQ_MODE_TURBO && (st = validate_codebook(kcb, p.head_dim, p.k_bits)) != TQ_OK) return st;
+    if (p.v_mode == TQ_MODE_TURBO && (st = validate_codebook(vcb, p.head_dim, p.v_bits)) != TQ_OK) return st;
+    DequantArgs a{};
+    fill_side(a.side[0], p.k_mode, p.k_bits, p.head_dim, kcb);
+    fill_side(a.side[1], p.v_mode, p.v_bits, p.head_dim, vcb);
+    a.side[0].codes = cache->k_codes;
+    a.side[0].norms = cache->k_norms;
+    a.side[0].qjl = cache->k_qjl;
+    a.side[0].gamma = cache->k_gamma;
+    a.side[0].sketch = cache->qjl_matrix;
+    a.side[0].m = p.qjl_dims;
+    a.side[1].codes = cache->v_codes;
+    a.side[1].norms = cache->v_norms;
+    a.out[0] = d_k_out;
+    a.out[1] = d_v_out;
+    a.b = b;
+    a.start = start;
+    a.count = count;
+    a.hkv = p.num_kv_heads;
+    a.capacity = cache->capacity;
+    rotation_sign_bits(p.seed, p.head_dim, a.signs);
+    const int lpv = p.head_dim / 32;
+    const long long warps = (static_cast<long long>(count) * p.num_kv_heads * lpv + 31) / 32;
+    long long blocks = (warps + 7) / 8;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const dim3 grid(static_cast<unsigned>(blocks), 2);
+    switch (p.head_dim) {
+        case 64: dequantize_kernel<64><<<grid, 256, 0, s>>>(a); break;
+        case 128: dequantize_kernel<128><<<grid, 256, 0, s>>>(a); break;
+        default: dequantize_kernel<256><<<grid, 256, 0, s>>>(a); break;
+    }
+    return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+tq_status tq_read_device_error(const uint32_t* d_error, uint32_t* out, void* stream, int32_t timeout_ms) {
+    if (!d_error || !out || timeout_ms < 0) return TQ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaEvent_t ev;
+    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return TQ_ERR_CUDA;
+    if (cudaEventRecord(ev, s) != cudaSuccess) {
+        cudaEventDestroy(ev);
+        return TQ_ERR_CUDA;
+    }
+    const auto deadline = std::chrono::steady_clock::now() + std::chrono::milliseconds(timeout_ms);
+    cudaError_t q;
+    while ((q = cudaEventQuery(ev)) == cudaErrorNotReady) {
+        if (std::chrono::steady_clock::now() > deadline) {
+            cudaEventDestroy(ev);
+            return TQ_ERR_TIMEOUT;
+        }
+        std::this_thread::sleep_for(std::chrono::microseconds(50));
+    }
+    cudaEventDestroy(ev);
+    if (q != cudaSuccess) return TQ_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, d_error, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess) return TQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TQ_ERR_CUDA;
+    *out = word;
+    return word ? TQ_ERR_DEVICE : TQ_OK;
+}
+
+}  // extern "C"

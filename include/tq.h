@@ -1,0 +1,286 @@
+/*
+ * tq.h — C ABI of the TurboQuant KV-cache library for NVIDIA B200 (sm_100a).
+ *
+ * The library compresses attention keys and values online and computes
+ * decode attention straight from the compressed cache.  Every entry point
+ * takes plain pointers and sizes; device pointers are CUDA device memory
+ * owned by the caller, host pointers are ordinary process memory.  The
+ * library allocates no device memory and keeps no global state: all caches,
+ * inputs, outputs and workspaces are provided by the caller.
+ *
+ * Pages the operations follow (cited by title and section):
+ *   [inferrs] "inferrs & TurboQuant：本地 LLM 推理的内存革命"
+ *   [tqai]    "TurboQuant：让大模型本地推理内存占用降低80%的KV缓存压缩技术"
+ *   [fwht]    "TurboQuant：用Rust核心与FWHT预处理实现LLM推理的4-bit KV缓存量化"
+ *   [google]  "Google 最新極限壓縮算法，砸碎大模型本地部署的內存墻，8 倍提升！"
+ *
+ * Conventions
+ * -----------
+ * - Every function returns a tq_status.  Arguments are validated on the host
+ *   before anything is launched; an invalid call launches nothing and
+ *   returns TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_ALIGNMENT or
+ *   TQ_ERR_CAPACITY.  No C++ exception crosses the ABI.
+ * - Device work is enqueued asynchronously on `stream` (a cudaStream_t
+ *   passed as void*; NULL means the legacy default stream).  A failed launch
+ *   returns TQ_ERR_CUDA.
+ * - Conditions only the device can see (an append position or sequence
+ *   length out of range) are never trapped: the kernel skips the offending
+ *   work and ORs a TQ_DEVERR_* bit into the caller's `d_error` word (device
+ *   uint32, may be NULL to disable reporting).  Read it with
+ *   tq_read_device_error.
+ * - Functions are reentrant and thread-safe; calls on different streams may
+ *   run concurrently as long as they do not write the same cache slots.
+ * - fp16 values are IEEE binary16 bit patterns stored as uint16_t.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TQ_ABI_VERSION 1
+
+typedef enum tq_status {
+    TQ_OK = 0,
+    TQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size, inconsistent params      */
+    TQ_ERR_UNSUPPORTED = 2,  /* valid in principle but not built (e.g. d = 512)   */
+    TQ_ERR_CAPACITY = 3,     /* workspace or cache too small for the request      */
+    TQ_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed              */
+    TQ_ERR_TIMEOUT = 5,      /* a bounded host wait ran out                       */
+    TQ_ERR_DEVICE = 6,       /* the device error word is non-zero                 */
+    TQ_ERR_ALIGNMENT = 7     /* a pointer is not 16-byte aligned                  */
+} tq_status;
+
+/* Storage mode of one side (K or V) of a cache. */
+typedef enum tq_mode {
+    TQ_MODE_TURBO = 0,  /* rotation + fp16 norm + Lloyd-Max b-bit codes         */
+    TQ_MODE_INT8 = 1    /* per-vector absmax int8 ("q8_0"-style boundary layers) */
+} tq_mode;
+
+/* Element type of raw K/V inputs and queries. */
+typedef enum tq_dtype { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
+
+/* Bits ORed into the caller's device error word. */
+#define TQ_DEVERR_POSITION 0x1u /* append: positions[b] < 0 or > capacity - n_new  */
+#define TQ_DEVERR_SEQLEN 0x2u   /* decode: seq_lens[b] < 1, > capacity or > max_seq_len */
+#define TQ_DEVERR_TIMEOUT 0x4u  /* decode: a bounded wait inside a kernel ran out (about 1 s);
+                                   the output is not valid and the workspace must be zeroed again */
+
+/*
+ * Lloyd-Max codebook for one (head_dim, bits) pair.  [tqai] section
+ * "TurboQuant的核心创新：极坐标量化与随机旋转": after the rotation each
+ * coordinate of the unit direction follows the density
+ *     f_d(x) = C_d (1 - x^2)^((d-3)/2),  |x| <= 1,
+ * and the optimal scalar quantiser for it is computed once, from the
+ * density alone.  centroids[0 .. 2^bits-1] ascend; boundaries[j] is the
+ * midpoint of centroids j and j+1.  Plain data, owned by the caller.
+ */
+typedef struct tq_codebook {
+    int32_t head_dim;
+    int32_t bits;
+    double centroids[16];
+    double boundaries[15];
+    /* Scale the tensor-core kernels apply to the centroids before rounding
+     * them to fp16 (their operand type); tq_codebook_init picks the value in
+     * [8, 16) that minimises the largest relative rounding error of the table.
+     * A representation detail, not part of the method: 0 selects sqrt(d). */
+    double fp16_scale;
+} tq_codebook;
+
+/*
+ * Cache configuration.  One tq_params describes one attention layer.
+ *   head_dim            d; 64, 128 or 256.
+ *   num_q_heads         Hq; a multiple of num_kv_heads.  Query head h reads
+ *                       kv head h / (Hq / Hkv) (contiguous GQA groups); the
+ *                       group size Hq / Hkv must be at most 16.
+ *   num_kv_heads        Hkv >= 1.
+ *   k_mode, v_mode      tq_mode of each side.  Asymmetric K/V bit widths:
+ *                       [inferrs] "三个反直觉的关键发现", [tqai] "配置策略与质量权衡".
+ *   k_bits, v_bits      2, 3 or 4 for TQ_MODE_TURBO; ignored for INT8.
+ *   qjl_dims            m, the QJL sketch size for K ([google] "第二步：QJL"):
+ *                       0 disables it; otherwise a multiple of 32 not above d,
+ *                       and only with k_mode == TQ_MODE_TURBO.
+ *   seed                selects the rotation signs and the QJL matrix
+ *                       (tq_rotation_signs, tq_qjl_matrix).  Keys, values and
+ *                       queries of one layer share the rotation.
+ *   sm_scale            softmax scale; 0 selects 1/sqrt(d).
+ *   sparse_v_threshold  Sparse V ([inferrs] "Sparse V：速度加成"): 0 disables;
+ *                       otherwise positions whose softmax weight is provably
+ *                       below it may be left out of the V sum (see
+ *                       tq_decode_attention).
+ */
+typedef struct tq_params {
+    int32_t head_dim;
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t k_mode;
+    int32_t v_mode;
+    int32_t k_bits;
+    int32_t v_bits;
+    int32_t qjl_dims;
+    uint64_t seed;
+    float sm_scale;
+    float sparse_v_threshold;
+} tq_params;
+
+/*
+ * Device-resident compressed cache of one layer (all pointers are device
+ * memory owned by the caller, each 16-byte aligned).  Layout is
+ * structure-of-arrays, per (batch entry, kv head), token-contiguous:
+ *   k_codes   [batch][Hkv][capacity][kb]   kb = d*k_bits/8 bytes (TURBO) or d (INT8)
+ *   k_norms   [batch][Hkv][capacity]       fp16 norm (TURBO) or fp16 scale (INT8)
+ *   k_qjl     [batch][Hkv][capacity][m/8]  QJL sign bits (NULL when qjl_dims == 0)
+ *   k_gamma   [batch][Hkv][capacity]       fp16 residual norm (NULL when qjl_dims == 0)
+ *   v_codes, v_norms                       as for K
+ *   qjl_matrix [m][d] fp32, row-major      the sketch S (NULL when qjl_dims == 0)
+ * Codes of one vector are one LSB-first bitstream: code i occupies bits
+ * [b*i, b*i+b), bit k of the stream is bit k%8 of byte k/8, so 3-bit codes
+ * cross byte boundaries ([inferrs] "压缩格式对比", turbo2/3/4).  INT8 codes
+ * are the d signed bytes of the vector.
+ */
+typedef struct tq_cache {
+    int32_t batch;
+    int32_t capacity;
+    uint8_t* k_codes;
+    uint16_t* k_norms;
+    uint8_t* k_qjl;
+    uint16_t* k_gamma;
+    uint8_t* v_codes;
+    uint16_t* v_norms;
+    const float* qjl_matrix;
+} tq_cache;
+
+/* Human-readable name of a status. Never NULL. */
+const char* tq_status_string(tq_status status);
+
+/* TQ_ABI_VERSION of the loaded library. */
+int32_t tq_abi_version(void);
+
+/*
+ * Host only.  Solve the Lloyd-Max conditions for f_d at `bits` bits
+ * (1 <= bits <= 4, 3 <= head_dim <= 4096) in fp64 and write the table to
+ * *out (caller-owned).  Deterministic: the result depends only on
+ * (head_dim, bits).  [tqai] "TurboQuant的核心创新" (precomputed,
+ * data-independent codebook).
+ */
+tq_status tq_codebook_init(int32_t head_dim, int32_t bits, tq_codebook* out);
+
+/*
+ * Host only.  The rotation of a layer is y = H diag(s) x / sqrt(d) with H
+ * the Sylvester-order Walsh-Hadamard matrix ([inferrs] "核心技术", [fwht]
+ * "2. 快速Walsh-Hadamard变换（FWHT）预处理").  Writes s (+1.0 / -1.0) for
+ * `seed` into out[0 .. head_dim-1] (caller-owned host array).  s_i is -1
+ * when bit 63 of the i-th SplitMix64 output from state `seed` is set.
+ */
+tq_status tq_rotation_signs(uint64_t seed, int32_t head_dim, float* out);
+
+/*
+ * Host only.  Writes the QJL sketch S (m x head_dim, row-major, iid N(0,1)
+ * rounded to fp32) for `seed` into out (caller-owned host array of
+ * m*head_dim floats).  The caller copies it to device memory and sets
+ * tq_cache.qjl_matrix.  Entries come from Box-Muller pairs on the
+ * SplitMix64 stream with state seed ^ 0x5155414E544A4C00.
+ */
+tq_status tq_qjl_matrix(uint64_t seed, int32_t m, int32_t head_dim, float* out);
+
+/*
+ * Host only.  Byte sizes of the six cache arrays, in tq_cache order
+ * (k_codes, k_norms, k_qjl, k_gamma, v_codes, v_norms), for `batch` entries
+ * of `capacity` tokens.  Unused arrays report 0.
+ */
+tq_status tq_cache_bytes(const tq_params* params, int32_t batch, int32_t capacity, size_t sizes_out[6]);
+
+/*
+ * Host only.  Bytes of device workspace tq_decode_attention needs for
+ * `batch` sequences of at most `max_seq_len` tokens on any device.  The
+ * workspace must be zero-filled once before its first use; every call that
+ * completes leaves it ready for the next one.
+ */
+tq_status tq_decode_workspace_bytes(const tq_params* params, int32_t batch, int32_t max_seq_len,
+                                    size_t* bytes_out);
+
+/*
+ * Quantise n_new new tokens per sequence and append them to the cache.
+ * [tqai] "TurboQuant的核心创新" (rotation, fp16 norm, Lloyd-Max codes),
+ * [google] "第二步：QJL" (1-bit residual sketch on K, when qjl_dims > 0),
+ * [inferrs] "三个反直觉的关键发现" item 3 (INT8 boundary layers).
+ *   k_new, v_new   device, [batch][n_new][Hkv][d] in `dtype`, 16-byte aligned.
+ *   n_new          >= 1.
+ *   d_positions    device int32 [batch]: sequence b's tokens go to cache
+ *                  slots positions[b] .. positions[b]+n_new-1.
+ *   kcb, vcb       codebooks matching (d, k_bits) and (d, v_bits); ignored
+ *                  (may be NULL) for an INT8 side.
+ * TURBO: norm n = ||x|| (fp32) stored as fp16 (round to nearest even);
+ * direction y = R(x)/n; code_i = number of boundaries below y_i; with QJL,
+ * r = y - c[code], gamma = ||r|| as fp16, sign bits of S r (1 when >= 0).
+ * INT8: scale = fp16(absmax/127), q_i = rint(x_i * fp32(1/scale)) clamped
+ * to [-127, 127].  A sequence whose position is out of range is skipped and
+ * sets TQ_DEVERR_POSITION.
+ */
+tq_status tq_quantize_append(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                             const void* k_new, const void* v_new, tq_dtype dtype, int32_t n_new,
+                             const int32_t* d_positions, const tq_cache* cache, uint32_t* d_error,
+                             void* stream);
+
+/*
+ * Reconstruct cache slots [start, start+count) of sequence b as fp32:
+ *   d_k_out, d_v_out  device, [count][Hkv][d] fp32 (either may be NULL).
+ * TURBO: x_hat = n16 * R^-1(c[code] + gamma16 sqrt(pi/2)/m S^T(2z-1)) (the
+ * QJL term only for K with qjl_dims > 0).  INT8: x_hat = scale16 * q.
+ */
+tq_status tq_dequantize(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                        const tq_cache* cache, int32_t b, int32_t start, int32_t count, float* d_k_out,
+                        float* d_v_out, void* stream);
+
+/*
+ * One decode-attention step read straight from the compressed cache.
+ * [google] "再看速度" (attention from 4-bit TurboQuant keys), [inferrs]
+ * "Sparse V：速度加成".  For every batch entry b and query head h, with kv
+ * head h / (Hq/Hkv) and L = seq_lens[b]:
+ *     s_i = sm_scale * <q, k_hat_i>,  p = softmax(s_0 .. s_{L-1}),
+ *     out = sum_i p_i v_hat_i
+ * where k_hat, v_hat are the reconstructions tq_dequantize defines.  The
+ * kernels never form k_hat: the query is rotated once, scores are
+ * n_k * <R q, c[code]> (+ the QJL term), the V sum runs in the rotated
+ * domain and one inverse rotation ends it.  The token axis is split across
+ * thread blocks and the partial results are merged by log-sum-exp.
+ *   d_q            device, [batch][Hq][d] in q_dtype.
+ *   d_seq_lens     device int32 [batch], each in [1, min(capacity, max_seq_len)].
+ *   max_seq_len    host upper bound on seq_lens (sizes the token split).
+ *   d_out          device, [batch][Hq][d] fp32.
+ *   d_workspace    device scratch of at least tq_decode_workspace_bytes
+ *                  bytes (16-byte aligned), zero-filled before its first use
+ *                  (it holds per-(sequence, kv head) split counters that each
+ *                  call returns to zero).  Calls sharing a workspace must not
+ *                  overlap on the device.
+ * Sparse V (sparse_v_threshold = tau > 0): position i is dropped from the V
+ * sum of head h only when exp(s_i - m)/l < tau for running softmax
+ * statistics m, l over a subset of the positions that includes i; since
+ * the full denominator is at least l e^m, every dropped position has exact
+ * weight p_i < tau.  Dropped positions stay in the denominator.  Which
+ * positions are dropped depends on the launch configuration.
+ * An out-of-range seq_len sets TQ_DEVERR_SEQLEN and yields zeros for b.
+ */
+tq_status tq_decode_attention(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                              const void* d_q, tq_dtype q_dtype, const tq_cache* cache,
+                              const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
+                              void* d_workspace, size_t workspace_bytes, uint32_t* d_error, void* stream);
+
+/*
+ * Copy the device error word to *out after the work queued on `stream` so
+ * far, waiting at most timeout_ms milliseconds (polling, never blocking
+ * indefinitely).  Returns TQ_ERR_TIMEOUT when the wait runs out,
+ * TQ_ERR_DEVICE when the word is non-zero (still written to *out), TQ_OK
+ * otherwise.
+ */
+tq_status tq_read_device_error(const uint32_t* d_error, uint32_t* out, void* stream, int32_t timeout_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */
