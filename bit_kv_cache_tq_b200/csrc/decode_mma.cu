@@ -10,33 +10,39 @@
 //
 // What is computed is the same as decode_split_kernel in decode.cu:
 //   s_i = sm_scale ||k_i|| (<q~, c[code_i]> + gamma_i sqrt(pi/2)/m <S q~, 2z_i - 1>),
-//   online softmax, acc = sum_i p_i ||v_i|| c[code_i] (rotated domain), then a
-//   log-sum-exp merge of the token splits and one inverse rotation.
+//   softmax over the sequence, acc = sum_i p_i ||v_i|| c[code_i] in the rotated
+//   domain, and one inverse rotation of acc / sum_i p_i.
 //
 // How (one persistent thread block per SM):
-//  * a producer warp streams the packed K and V codes of 128-token chunks into
-//    a ring of shared-memory stages with 1-D bulk async copies (TMA engine, no
-//    multicast), completion tracked by mbarriers; eight consumer warps take one
-//    16-token tile of every chunk;
-//  * the dequantised tiles of a GQA group form real dense products, so both
+//  * Work items are (sequence, kv head, token split).  A producer warp takes
+//    items from a global atomic counter (so ragged batches balance), and for
+//    each one streams the packed K and V codes (plus norms, QJL words and the
+//    queries) of 256-token chunks into a ring of shared-memory stages with 1-D
+//    bulk async copies (TMA engine, no multicast).  Each stage starts with a
+//    header naming its item and token range; completion is tracked by
+//    mbarriers.  Eight consumer warps take two 16-token tiles of every chunk.
+//  * The dequantised tiles of a GQA group form real dense products, so both
 //    contractions run on the tensor cores with warp-level m16n8k16 fp16 MMA
 //    (fp32 accumulate):  S^T[16 tok x 8 heads] = K~[16 x 128] Q~^T and
 //    O^T[128 x 8 heads] += V~^T[128 x 16 tok] P^T.  The A operands are built
-//    in registers straight from the codes: a 256-entry (per-lane replicated)
-//    shared-memory table maps one byte of 4-bit key codes to the fp16 pair of
+//    in registers straight from the codes: a 256-entry, per-lane replicated
+//    shared-memory table maps one byte of 4-bit key codes to a pair of fp16
 //    centroids, and a register byte-permute table maps 2-bit value codes.
-//    Because sum_c q~_c c[code_c] does not depend on the order of c, channels
-//    are assigned to fragment slots so that each lane's 16-byte load of a key
-//    row feeds its fragments directly (the query uses the same order).  Tokens
-//    of a tile are permuted the same way on both sides (tau below) so that the
-//    value words each lane needs are bank-conflict free.
-//  * the score fragment is turned into the second MMA's operand with one
-//    movmatrix transpose per 8x8 block; no shared-memory round trip.
-//  * split results are merged by the last block to finish a (sequence, kv
-//    head), found with an atomic counter (no spin-wait), which also applies the
+//    Since sum_c q~_c c[code_c] does not depend on the order of c, channels are
+//    assigned to fragment slots so that each lane's 16-byte load of a key row
+//    feeds its fragments directly (the query uses the same order); tokens of a
+//    tile are permuted the same way on both sides (tau) so that the value
+//    words each lane needs are bank-conflict free.
+//  * The score fragment becomes the second MMA's operand through one movmatrix
+//    transpose per 8x8 block.  The softmax rescales lazily: the running max
+//    used for exp2 only moves (with a warp-wide reduction) when a score exceeds
+//    it by more than 2^8, decided by one warp vote per chunk.
+//  * Split results are merged by the last block to finish a (sequence, kv
+//    head), found with an atomic counter (no spin-wait); it also applies the
 //    inverse rotation and writes the output.
 //  Every wait on an mbarrier is bounded (about a second); a wait that runs out
-//  sets TQ_DEVERR_TIMEOUT and the block leaves after draining its copies.
+//  sets TQ_DEVERR_TIMEOUT, all consumer warps agree on it at the next named
+//  barrier, and the block leaves after draining its copies.
 
 #include <cuda_runtime.h>
 
@@ -51,12 +57,21 @@ namespace mmadec {
 
 constexpr int D = 128;
 constexpr int CW = 8;                        // consumer warps
+constexpr int TPW = 2;                       // 16-token tiles per warp and chunk
 constexpr int NUM_THREADS = (CW + 1) * 32;   // + one producer warp
 constexpr int NUM_CONSUMERS = CW * 32;
-constexpr int CHUNK = CW * 16;               // tokens per stage
+constexpr int CHUNK = CW * TPW * 16;         // tokens per stage
 constexpr uint32_t LUT_BYTES = 65536;        // 256 entries x 256 B
+constexpr uint32_t QSLOT_BYTES = 16 * D * 4; // one item's queries, up to 16 heads in fp32
 constexpr long long WAIT_LIMIT = 2000000000ll;  // clock cycles (~1 s)
 constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LAZY = 8.0f;                 // log2 headroom before the running max moves
+constexpr float VRANGE = 64.0f;              // bound on ||v|| * vscale
+
+// stage header flags
+constexpr int F_FIRST = 1, F_LAST = 2, F_EMPTY = 4, F_END = 8;
+// global counters after the per-(sequence, kv head) split counters
+constexpr int C_ITEM = 0, C_DONE = 1;
 
 struct Args {
     const uint8_t* k_codes;
@@ -70,45 +85,44 @@ struct Args {
     const int32_t* seq_lens;
     float2* ws_ml;
     float* ws_acc;
-    uint32_t* counters;
+    uint32_t* counters;  // [units] split counters, then [2] global counters
     float* out;
     uint32_t* err;
-    int q_dtype, batch, hq, hkv, group, capacity, n_split, split_len, max_len, n_items, stages, m;
+    int q_dtype, q_bytes, batch, hq, hkv, group, capacity, n_split, split_len, max_len, n_items, units, stages, m;
     float sm_scale_log2;  // sm_scale * log2(e)
     float tau;
     float inv_alpha_k, inv_alpha_v;  // 1 / (centroid scale applied before fp16 rounding)
-    int staged_norms;     // capacity % 8 == 0: norms (and QJL words) ride in the TMA stages
+    int staged_norms;     // capacity % 8 == 0: norms and QJL words ride in the stages
     uint32_t signs[4];
     uint16_t kcent[16];  // fp16 bits of alpha_k * key centroid
     uint16_t vcent[16];  // fp16 bits of alpha_v * value centroid
 };
 
-// Shared-memory map (offsets in bytes from the dynamic base).
+// Shared-memory map (byte offsets from the dynamic base).  A stage is
+// [header | K codes | V codes | K norms | V norms | QJL words | gammas].
 struct Layout {
-    uint32_t ring, stage_bytes, kbytes_stage, vbytes_stage, kn_off, vn_off, z_off, gam_off;
-    uint32_t qh, sq, fac, merge, ml, bars, flags, total;
+    uint32_t ring, stage_bytes, k_off, v_off, kn_off, vn_off, z_off, gam_off;
+    uint32_t qring, qh, sq, fac, merge, ml, bars, flags, total;
 };
 
-// One stage: [K codes | V codes | K norms | V norms | QJL words | gammas] for
-// CHUNK tokens, every part 16-byte aligned.
 __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int m) {
     Layout L{};
-    const uint32_t vbk = 16 * kb, vbv = 16 * vb;
     L.ring = LUT_BYTES;
-    L.kbytes_stage = CHUNK * vbk;
-    L.vbytes_stage = CHUNK * vbv;
-    L.kn_off = L.kbytes_stage + L.vbytes_stage;
+    L.k_off = 16;
+    L.v_off = L.k_off + CHUNK * 16 * kb;
+    L.kn_off = L.v_off + CHUNK * 16 * vb;
     L.vn_off = L.kn_off + CHUNK * 2;
     L.z_off = L.vn_off + CHUNK * 2;
     L.gam_off = L.z_off + CHUNK * (m / 8);
     L.stage_bytes = L.gam_off + (m > 0 ? CHUNK * 2 : 0);
-    L.qh = L.ring + stages * L.stage_bytes;          // fp16 [16][128]
+    L.qring = L.ring + stages * L.stage_bytes;        // 2 query slots
+    L.qh = L.qring + 2 * QSLOT_BYTES;                  // fp16 [16][128]
     L.sq = L.qh + 16 * D * 2;                          // fp16 [16][64]
     L.fac = L.sq + 16 * 64 * 2;                        // float F1[16], F2[16]
     L.merge = L.fac + 32 * 4;                          // float [CW][8*nt][128]
     L.ml = L.merge + CW * 8 * nt * D * 4;              // float2 [CW][16]
-    L.bars = L.ml + CW * 16 * 8;                       // u64 full[8], empty[8]
-    L.flags = L.bars + 16 * 8;                         // int abort, last
+    L.bars = L.ml + CW * 16 * 8;                       // u64 full[8], empty[8], qfull[2], qempty[2]
+    L.flags = L.bars + 20 * 8;                         // int abort, last
     L.total = L.flags + 16;
     return L;
 }
@@ -139,54 +153,100 @@ __device__ __forceinline__ Item item_of(const Args& a, int item) {
 template <int KB, int VB, bool QJL>
 __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
     const uint32_t base = ptx::smem_addr(smem);
-    const uint32_t full0 = base + L.bars, empty0 = full0 + 64;
+    const uint32_t full0 = base + L.bars, empty0 = full0 + 64, qfull0 = full0 + 128, qempty0 = full0 + 144;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.flags);
     constexpr int VBK = 16 * KB, VBV = 16 * VB;
-    int it = 0;
+    const int zb = QJL ? a.m / 8 : 0;
+    const int G = a.group;
+    int seq = 0, qseq = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
-        const Item w = item_of(a, item);
-        for (int t0 = w.s0; t0 < w.s1; t0 += CHUNK) {
-            const int slot = it % a.stages, use = it / a.stages;
-            if (use > 0 && !ptx::mbar_wait_bounded(empty0 + 8 * slot, (use - 1) & 1, WAIT_LIMIT)) {
-                if (a.err) atomicOr(a.err, TQ_DEVERR_TIMEOUT);
-                *abort_flag = 1;
-                ok = false;
+    auto fail = [&]() {
+        if (!*abort_flag && a.err) atomicOr(a.err, TQ_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+        ok = false;
+    };
+    // claim a free stage slot (bounded wait); false on abort
+    auto claim = [&](uint32_t& full, uint8_t*& st) -> bool {
+        const int slot = seq % a.stages, use = seq / a.stages;
+        if (use > 0 && !ptx::mbar_wait_bounded(empty0 + 8 * slot, (use - 1) & 1, WAIT_LIMIT)) {
+            fail();
+            return false;
+        }
+        if (*abort_flag) {
+            ok = false;
+            return false;
+        }
+        full = full0 + 8 * slot;
+        st = smem + L.ring + slot * L.stage_bytes;
+        return true;
+    };
+    while (ok) {
+        const int i = static_cast<int>(atomicAdd(a.counters + a.units + C_ITEM, 1u));
+        if (i >= a.n_items) break;
+        const Item w = item_of(a, i);
+        const bool empty = w.s0 >= w.s1;
+        if (!empty) {  // the item's queries, into the next query slot
+            const int qs = qseq & 1;
+            if (qseq >= 2 && !ptx::mbar_wait_bounded(qempty0 + 8 * qs, ((qseq - 2) >> 1) & 1, WAIT_LIMIT)) {
+                fail();
                 break;
             }
-            if (*abort_flag) {
-                ok = false;
-                break;
-            }
-            int n = min(CHUNK, w.s1 - t0);
+            const uint32_t qbytes = G * D * a.q_bytes;
+            ptx::mbar_arrive_expect_tx(qfull0 + 8 * qs, qbytes);
+            ptx::bulk_copy_g2s(base + L.qring + qs * QSLOT_BYTES,
+                               static_cast<const uint8_t*>(a.q) +
+                                   (static_cast<size_t>(w.b) * a.hq + w.kv * G) * D * a.q_bytes,
+                               qbytes, qfull0 + 8 * qs);
+            ++qseq;
+        }
+        int t0 = w.s0;
+        do {
+            uint32_t full;
+            uint8_t* st;
+            if (!claim(full, st)) break;
+            const int n = empty ? 0 : min(CHUNK, w.s1 - t0);
+            const int flags = (t0 == w.s0 ? F_FIRST : 0) | ((empty || t0 + CHUNK >= w.s1) ? F_LAST : 0) |
+                              (empty ? F_EMPTY : 0);
+            *reinterpret_cast<int4*>(st) = make_int4(i, t0, n, flags);
+            const uint32_t dst = ptx::smem_addr(st);
             const size_t row = static_cast<size_t>(w.unit) * a.capacity + t0;
-            const uint32_t full = full0 + 8 * slot;
-            const uint32_t dst = base + L.ring + slot * L.stage_bytes;
-            if (a.staged_norms) {
+            if (n == 0) {
+                ptx::mbar_arrive_expect_tx(full, 0);
+            } else if (a.staged_norms) {
                 // capacity and t0 are multiples of 8, so rounding n up to 8 tokens
                 // stays inside the cache and keeps every 2-byte array 16-byte sized
-                n = (n + 7) & ~7;
-                const int zb = QJL ? a.m / 8 : 0;
-                ptx::mbar_arrive_expect_tx(full, n * (VBK + VBV + 4 + (QJL ? zb + 2 : 0)));
-                ptx::bulk_copy_g2s(dst, a.k_codes + row * VBK, n * VBK, full);
-                ptx::bulk_copy_g2s(dst + L.kbytes_stage, a.v_codes + row * VBV, n * VBV, full);
-                ptx::bulk_copy_g2s(dst + L.kn_off, a.k_norms + row, n * 2, full);
-                ptx::bulk_copy_g2s(dst + L.vn_off, a.v_norms + row, n * 2, full);
+                const int n8 = (n + 7) & ~7;
+                ptx::mbar_arrive_expect_tx(full, n8 * (VBK + VBV + 4 + (QJL ? zb + 2 : 0)));
+                ptx::bulk_copy_g2s(dst + L.k_off, a.k_codes + row * VBK, n8 * VBK, full);
+                ptx::bulk_copy_g2s(dst + L.v_off, a.v_codes + row * VBV, n8 * VBV, full);
+                ptx::bulk_copy_g2s(dst + L.kn_off, a.k_norms + row, n8 * 2, full);
+                ptx::bulk_copy_g2s(dst + L.vn_off, a.v_norms + row, n8 * 2, full);
                 if constexpr (QJL) {
-                    ptx::bulk_copy_g2s(dst + L.z_off, a.k_qjl + row * zb, n * zb, full);
-                    ptx::bulk_copy_g2s(dst + L.gam_off, a.k_gamma + row, n * 2, full);
+                    ptx::bulk_copy_g2s(dst + L.z_off, a.k_qjl + row * zb, n8 * zb, full);
+                    ptx::bulk_copy_g2s(dst + L.gam_off, a.k_gamma + row, n8 * 2, full);
                 }
             } else {
                 ptx::mbar_arrive_expect_tx(full, n * (VBK + VBV));
-                ptx::bulk_copy_g2s(dst, a.k_codes + row * VBK, n * VBK, full);
-                ptx::bulk_copy_g2s(dst + L.kbytes_stage, a.v_codes + row * VBV, n * VBV, full);
+                ptx::bulk_copy_g2s(dst + L.k_off, a.k_codes + row * VBK, n * VBK, full);
+                ptx::bulk_copy_g2s(dst + L.v_off, a.v_codes + row * VBV, n * VBV, full);
             }
-            ++it;
+            ++seq;
+            t0 += CHUNK;
+        } while (!empty && t0 < w.s1);
+    }
+    if (ok) {  // end-of-work sentinel
+        uint32_t full;
+        uint8_t* st;
+        if (claim(full, st)) {
+            *reinterpret_cast<int4*>(st) = make_int4(-1, 0, 0, F_END);
+            ptx::mbar_arrive_expect_tx(full, 0);
+            ++seq;
         }
     }
     // every copy issued must have landed before the block may exit
-    for (int j = max(0, it - a.stages); j < it; ++j)
+    for (int j = max(0, seq - a.stages); j < seq; ++j)
         ptx::mbar_wait_bounded(full0 + 8 * (j % a.stages), (j / a.stages) & 1, WAIT_LIMIT);
+    for (int j = max(0, qseq - 2); j < qseq; ++j) ptx::mbar_wait_bounded(qfull0 + 8 * (j & 1), (j >> 1) & 1, WAIT_LIMIT);
 }
 
 // ----------------------------------------------------------------- consumers
@@ -208,40 +268,138 @@ __device__ __forceinline__ uint32_t key_lut_addr(const uint32_t (&seg)[4], int j
     }
 }
 
+// Value fragments A[m-tile i][reg] of one 16-token tile for lane group g.
+template <int VB>
+__device__ __forceinline__ void value_fragments(uint32_t vst, uint32_t base, int g, int t, uint32_t laneoff,
+                                                uint32_t vl0, uint32_t vl1, uint32_t (&A)[8][4]) {
+    constexpr int VBV = 16 * VB;
+    if constexpr (VB == 2) {
+        // word g of physical tokens t, 4+t, 8+t, 12+t (logical k = 2t, 2t+1, 2t+8, 2t+9)
+        const uint32_t w0 = ptx::lds32(vst + t * VBV + 4 * g);
+        const uint32_t w1 = ptx::lds32(vst + (4 + t) * VBV + 4 * g);
+        const uint32_t w2 = ptx::lds32(vst + (8 + t) * VBV + 4 * g);
+        const uint32_t w3 = ptx::lds32(vst + (12 + t) * VBV + 4 * g);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const uint32_t wa0 = half ? w2 : w0, wb0 = half ? w3 : w1;
+            // interleave the bytes of the two tokens: fields at equal offsets pair up
+            const uint32_t P = __byte_perm(wa0, wb0, 0x5140), Q = __byte_perm(wa0, wb0, 0x7362);
+#pragma unroll
+            for (int src = 0; src < 2; ++src) {
+                const uint32_t x = src ? Q : P;
+#pragma unroll
+                for (int sh = 0; sh < 8; sh += 2) {
+                    // 2-bit codes (u0, u1) -> byte selector {2u0, 2u0+1, 2u1, 2u1+1}
+                    const uint32_t sel = ((x >> sh) & 0x03030303u) * 0x22u + 0x10101010u;
+                    const int f = (sh >> 1) & 1, hb = sh >> 2;
+                    A[2 * (2 * src) + hb][2 * half + f] = __byte_perm(vl0, vl1, sel);
+                    A[2 * (2 * src + 1) + hb][2 * half + f] = __byte_perm(vl0, vl1, sel >> 16);
+                }
+            }
+        }
+    } else {
+        // 16 * VB bits per lane group and token (2*VB bytes at byte 2*VB*g),
+        // realigned to two words; code pairs read through the value table
+        uint32_t seg[4][2];
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+            const int tok = 4 * k4 + t;
+            const uint32_t byte_off = 2 * VB * g;
+            const uint32_t wbase = byte_off >> 2, wsh = (byte_off & 3) * 8;
+            const uint32_t lo = ptx::lds32(vst + tok * VBV + 4 * wbase);
+            const uint32_t hi = (4 * wbase + 4 < VBV) ? ptx::lds32(vst + tok * VBV + 4 * wbase + 4) : 0u;
+            const uint32_t hi2 = (4 * wbase + 8 < VBV) ? ptx::lds32(vst + tok * VBV + 4 * wbase + 8) : 0u;
+            seg[k4][0] = __funnelshift_r(lo, hi, wsh);
+            seg[k4][1] = __funnelshift_r(hi, hi2, wsh);
+        }
+        constexpr uint32_t vm = (1u << VB) - 1u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int f = 0; f < 2; ++f) {
+                const int bit = VB * (2 * i + f);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const uint32_t* sx = seg[2 * half];
+                    const uint32_t* sy = seg[2 * half + 1];
+                    const uint32_t cx = bit >= 32 ? (sx[1] >> (bit - 32)) & vm
+                                                  : (bit + VB <= 32 ? (sx[0] >> bit) & vm
+                                                                    : __funnelshift_r(sx[0], sx[1], bit) & vm);
+                    const uint32_t cy = bit >= 32 ? (sy[1] >> (bit - 32)) & vm
+                                                  : (bit + VB <= 32 ? (sy[0] >> bit) & vm
+                                                                    : __funnelshift_r(sy[0], sy[1], bit) & vm);
+                    A[i][2 * half + f] = ptx::lds32(base + (((cx | (cy << VB)) << 8) | 128u | laneoff));
+                }
+            }
+    }
+}
+
+template <int NT>
+struct SoftState {
+    float m[NT][2];  // exp2 reference of heads 2t, 2t+1 (uniform over the lane group)
+    float l[NT][2];  // this lane's partial sum of exp2(s - m)
+    float acc[NT][8][4];
+    float vscale;    // power of two keeping p * ||v|| inside fp16 range; 0 = not set
+
+    __device__ void reset() {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            m[nt][0] = m[nt][1] = -INFINITY;
+            l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[nt][i][0] = acc[nt][i][1] = acc[nt][i][2] = acc[nt][i][3] = 0.f;
+        }
+        vscale = 0.f;
+    }
+};
+
 template <int KB, int VB, int NT, bool QJL>
-__device__ void consumer(const Args& a, uint8_t* smem, const Layout& L) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    const uint32_t base = ptx::smem_addr(smem);
-    const uint32_t full0 = base + L.bars, empty0 = full0 + 64;
-    const uint32_t laneoff = lane * 4;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.flags);
-    __half* qh = reinterpret_cast<__half*>(smem + L.qh);
-    __half* sq = reinterpret_cast<__half*>(smem + L.sq);
-    float* fac = reinterpret_cast<float*>(smem + L.fac);
-    float* merge = reinterpret_cast<float*>(smem + L.merge);
-    float2* ml = reinterpret_cast<float2*>(smem + L.ml);
-    int* last_flag = reinterpret_cast<int*>(smem + L.flags + 4);
-    constexpr int VBK = 16 * KB, VBV = 16 * VB;
-    const int G = a.group;
-    const float inv_sqrt_d = 0.08838834764831845f;
+struct Consumer {
+    const Args& a;
+    uint8_t* smem;
+    const Layout& L;
+    int tid, warp, lane, g, t;
+    uint32_t base, laneoff, vl0, vl1;
 
-    // value centroid pairs for the 2-bit byte-permute table
-    const uint32_t vl0 = a.vcent[0] | (static_cast<uint32_t>(a.vcent[1]) << 16);
-    const uint32_t vl1 = a.vcent[2] | (static_cast<uint32_t>(a.vcent[3]) << 16);
+    __device__ Consumer(const Args& a_, uint8_t* s_, const Layout& L_) : a(a_), smem(s_), L(L_) {
+        tid = threadIdx.x;
+        warp = tid >> 5;
+        lane = tid & 31;
+        g = lane >> 2;
+        t = lane & 3;
+        base = ptx::smem_addr(smem);
+        laneoff = lane * 4;
+        vl0 = a.vcent[0] | (static_cast<uint32_t>(a.vcent[1]) << 16);
+        vl1 = a.vcent[2] | (static_cast<uint32_t>(a.vcent[3]) << 16);
+    }
 
-    int it = 0;
-    for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
-        const Item w = item_of(a, item);
-        if (w.bad && a.err && w.split == 0 && w.kv == 0 && tid == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
+    __device__ bool aborted() const { return *reinterpret_cast<volatile int*>(smem + L.flags) != 0; }
+    __device__ void set_abort() {
+        if (!aborted() && a.err) atomicOr(a.err, TQ_DEVERR_TIMEOUT);
+        *reinterpret_cast<volatile int*>(smem + L.flags) = 1;
+    }
 
-        // ---- rotated queries of the kv head (fp16, scaled to max |q~| = 1)
+    // Rotated queries of the item (fp16, scaled to max |q~| = 1) and the scale
+    // factors of the scores; false on abort.
+    __device__ bool prologue(int qseq, uint32_t (&bq)[NT][8][2], uint32_t (&bz)[NT][4][2], float (&f1)[NT][2],
+                             float (&f2)[NT][2]) {
+        const uint32_t qfull = base + L.bars + 128 + 8 * (qseq & 1);
+        if (!ptx::mbar_wait_bounded(qfull, (qseq >> 1) & 1, WAIT_LIMIT)) set_abort();
+        ptx::named_barrier(1, NUM_CONSUMERS);
+        if (aborted()) return false;
+        const int G = a.group;
+        const uint8_t* qsrc = smem + L.qring + (qseq & 1) * QSLOT_BYTES;
+        __half* qh = reinterpret_cast<__half*>(smem + L.qh);
+        __half* sq = reinterpret_cast<__half*>(smem + L.sq);
+        float* fac = reinterpret_cast<float*>(smem + L.fac);
+        float* merge = reinterpret_cast<float*>(smem + L.merge);
+        const float inv_sqrt_d = 0.08838834764831845f;
         for (int h = warp; h < NT * 8; h += CW) {
             float x[4] = {0.f, 0.f, 0.f, 0.f};
             if (h < G) {
-                const size_t off = (static_cast<size_t>(w.b) * a.hq + w.kv * G + h) * D + lane * 4;
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    x[e] = flip_sign(load_scalar(a.q, off + e, a.q_dtype), sign_bit(a.signs, lane * 4 + e));
+                    x[e] = flip_sign(load_scalar(qsrc, h * D + lane * 4 + e, a.q_dtype), sign_bit(a.signs, lane * 4 + e));
                 fwht_registers(x);
                 fwht_lanes<4, 32>(x, lane);
 #pragma unroll
@@ -255,7 +413,7 @@ __device__ void consumer(const Args& a, uint8_t* smem, const Layout& L) {
             float smax = 1.f;
             if constexpr (QJL) {
                 // S q~ for sketch rows lane and lane + 32 (m <= 64); q~ staged in
-                // the merge buffer, which is free until the end of the item
+                // the merge buffer, which is free until the item's end
                 float* qf = merge + h * D;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) qf[lane * 4 + e] = x[e];
@@ -273,7 +431,7 @@ __device__ void consumer(const Args& a, uint8_t* smem, const Layout& L) {
                         }
                     }
                 }
-                float sm = group_max<32>(fmaxf(fabsf(sv[0]), fabsf(sv[1])));
+                const float sm = group_max<32>(fmaxf(fabsf(sv[0]), fabsf(sv[1])));
                 smax = sm > 0.f ? sm : 1.f;
                 sq[h * 64 + lane] = __float2half_rn(sv[0] / smax);
                 sq[h * 64 + lane + 32] = __float2half_rn(sv[1] / smax);
@@ -284,11 +442,7 @@ __device__ void consumer(const Args& a, uint8_t* smem, const Layout& L) {
             }
         }
         ptx::named_barrier(1, NUM_CONSUMERS);
-
-        // ---- per-lane operand fragments of the queries
-        uint32_t bq[NT][8][2];
-        uint32_t bz[NT][4][2];
-        float f1[NT][2], f2[NT][2];
+        if (tid == 0) ptx::mbar_arrive(base + L.bars + 144 + 8 * (qseq & 1));  // query slot free
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const __half* qrow = qh + (nt * 8 + g) * D + 32 * t;
@@ -310,303 +464,262 @@ __device__ void consumer(const Args& a, uint8_t* smem, const Layout& L) {
             f2[nt][0] = fac[16 + nt * 8 + 2 * t];
             f2[nt][1] = fac[16 + nt * 8 + 2 * t + 1];
         }
+        return true;
+    }
 
-        // ---- stream the split
-        float m_run[NT][2], l_run[NT][2], acc[NT][8][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            m_run[nt][0] = m_run[nt][1] = -INFINITY;
-            l_run[nt][0] = l_run[nt][1] = 0.f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[nt][i][0] = acc[nt][i][1] = acc[nt][i][2] = acc[nt][i][3] = 0.f;
-        }
-        float vscale = 0.f;  // power of two keeping p*||v|| inside fp16 range; 0 = not set yet
+    // One chunk: this warp's two tiles.  MASK: the chunk may end before CHUNK tokens.
+    template <bool MASK>
+    __device__ void chunk(const Item& w, const uint8_t* st, int t0, const uint32_t (&bq)[NT][8][2],
+                          const uint32_t (&bz)[NT][4][2], const float (&f1)[NT][2], const float (&f2)[NT][2],
+                          SoftState<NT>& S) {
+        constexpr int VBK = 16 * KB, VBV = 16 * VB;
+        const int lb = 32 * warp;  // first chunk-local token of this warp
+        if (MASK && t0 + lb >= w.s1) return;  // nothing of this warp's range is valid
+        const uint32_t sbase = ptx::smem_addr(st);
         const int ra = tau_row(g), rb = tau_row(g + 8);
+        const int zw = a.m / 16;
+        const bool zt = 16 * t < a.m;
         const size_t unit_row = static_cast<size_t>(w.unit) * a.capacity;
-        for (int t0 = w.s0; t0 < w.s1; t0 += CHUNK) {
-            const int slot = it % a.stages, use = it / a.stages;
-            const int tile0 = t0 + 16 * warp;
-            const int tok_a = tile0 + ra, tok_b = tile0 + rb;
-            const bool va = tok_a < w.s1, vb = tok_b < w.s1;
-            const bool zt = 16 * t < a.m;  // lanes past the sketch size carry no QJL bits
-            const int zw = a.m / 16;       // 16-bit QJL words per token
-            float kna = 0.f, knb = 0.f, vna = 0.f, vnb = 0.f, ga = 0.f, gb = 0.f;
-            uint32_t za = 0, zb = 0;
-            if (!a.staged_norms) {  // straight from global memory, issued before the wait
-                kna = va ? half_bits_to_float(a.k_norms[unit_row + tok_a]) : 0.f;
-                knb = vb ? half_bits_to_float(a.k_norms[unit_row + tok_b]) : 0.f;
-                vna = va ? half_bits_to_float(a.v_norms[unit_row + tok_a]) : 0.f;
-                vnb = vb ? half_bits_to_float(a.v_norms[unit_row + tok_b]) : 0.f;
-                if constexpr (QJL) {
-                    const uint16_t* zr = reinterpret_cast<const uint16_t*>(a.k_qjl);
-                    za = (va && zt) ? zr[(unit_row + tok_a) * zw + t] : 0u;
-                    zb = (vb && zt) ? zr[(unit_row + tok_b) * zw + t] : 0u;
-                    ga = va ? half_bits_to_float(a.k_gamma[unit_row + tok_a]) : 0.f;
-                    gb = vb ? half_bits_to_float(a.k_gamma[unit_row + tok_b]) : 0.f;
-                }
-            }
-            if (*abort_flag || !ptx::mbar_wait_bounded(full0 + 8 * slot, use & 1, WAIT_LIMIT)) {
-                if (!*abort_flag && a.err) atomicOr(a.err, TQ_DEVERR_TIMEOUT);
-                *abort_flag = 1;
-                break;  // every consumer warp still reaches the barrier below
-            }
+        float s[TPW][NT][4];
+        float vn[TPW][2];
+#pragma unroll
+        for (int k = 0; k < TPW; ++k) {
+            const int la = lb + 16 * k + ra, lbb = lb + 16 * k + rb;  // chunk-local tokens of rows g, g+8
+            const bool va = !MASK || t0 + la < w.s1, vb = !MASK || t0 + lbb < w.s1;
+            float kna, knb, ga = 0.f, gb = 0.f;
+            uint32_t za = 0, zb2 = 0;
             if (a.staged_norms) {
-                const uint8_t* st = smem + L.ring + slot * L.stage_bytes;
-                const int la = 16 * warp + ra, lb = 16 * warp + rb;
                 const __half* skn = reinterpret_cast<const __half*>(st + L.kn_off);
                 const __half* svn = reinterpret_cast<const __half*>(st + L.vn_off);
-                kna = va ? __half2float(skn[la]) : 0.f;
-                knb = vb ? __half2float(skn[lb]) : 0.f;
-                vna = va ? __half2float(svn[la]) : 0.f;
-                vnb = vb ? __half2float(svn[lb]) : 0.f;
+                kna = __half2float(skn[la]);
+                knb = __half2float(skn[lbb]);
+                vn[k][0] = va ? __half2float(svn[la]) : 0.f;
+                vn[k][1] = vb ? __half2float(svn[lbb]) : 0.f;
                 if constexpr (QJL) {
                     const uint16_t* sz = reinterpret_cast<const uint16_t*>(st + L.z_off);
                     const __half* sg = reinterpret_cast<const __half*>(st + L.gam_off);
-                    za = (va && zt) ? sz[la * zw + t] : 0u;
-                    zb = (vb && zt) ? sz[lb * zw + t] : 0u;
-                    ga = va ? __half2float(sg[la]) : 0.f;
-                    gb = vb ? __half2float(sg[lb]) : 0.f;
+                    za = zt ? sz[la * zw + t] : 0u;
+                    zb2 = zt ? sz[lbb * zw + t] : 0u;
+                    ga = __half2float(sg[la]);
+                    gb = __half2float(sg[lbb]);
+                }
+            } else {
+                kna = va ? half_bits_to_float(a.k_norms[unit_row + t0 + la]) : 0.f;
+                knb = vb ? half_bits_to_float(a.k_norms[unit_row + t0 + lbb]) : 0.f;
+                vn[k][0] = va ? half_bits_to_float(a.v_norms[unit_row + t0 + la]) : 0.f;
+                vn[k][1] = vb ? half_bits_to_float(a.v_norms[unit_row + t0 + lbb]) : 0.f;
+                if constexpr (QJL) {
+                    const uint16_t* zr = reinterpret_cast<const uint16_t*>(a.k_qjl);
+                    za = (va && zt) ? zr[(unit_row + t0 + la) * zw + t] : 0u;
+                    zb2 = (vb && zt) ? zr[(unit_row + t0 + lbb) * zw + t] : 0u;
+                    ga = va ? half_bits_to_float(a.k_gamma[unit_row + t0 + la]) : 0.f;
+                    gb = vb ? half_bits_to_float(a.k_gamma[unit_row + t0 + lbb]) : 0.f;
                 }
             }
-            if (tile0 < w.s1) {
-                const uint32_t kst = base + L.ring + slot * L.stage_bytes + (16 * warp) * VBK;
-                const uint32_t vst = base + L.ring + slot * L.stage_bytes + L.kbytes_stage + (16 * warp) * VBV;
-                // ---- keys: 16 bytes (KB words) of rows tau(g) and tau(g+8)
-                uint32_t sa[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
-                if constexpr (KB == 4) {
-                    const uint4 x = ptx::lds128(kst + ra * VBK + 16 * t);
-                    const uint4 y = ptx::lds128(kst + rb * VBK + 16 * t);
-                    sa[0] = x.x; sa[1] = x.y; sa[2] = x.z; sa[3] = x.w;
-                    sb[0] = y.x; sb[1] = y.y; sb[2] = y.z; sb[3] = y.w;
-                } else {
+            // ---- keys: the lane's 4*KB bytes of rows tau(g) and tau(g+8)
+            const uint32_t kst = sbase + L.k_off + (lb + 16 * k) * VBK;
+            uint32_t sa[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
+            if constexpr (KB == 4) {
+                const uint4 x = ptx::lds128(kst + ra * VBK + 16 * t);
+                const uint4 y = ptx::lds128(kst + rb * VBK + 16 * t);
+                sa[0] = x.x; sa[1] = x.y; sa[2] = x.z; sa[3] = x.w;
+                sb[0] = y.x; sb[1] = y.y; sb[2] = y.z; sb[3] = y.w;
+            } else {
 #pragma unroll
-                    for (int q = 0; q < KB; ++q) {
-                        sa[q] = ptx::lds32(kst + ra * VBK + 4 * KB * t + 4 * q);
-                        sb[q] = ptx::lds32(kst + rb * VBK + 4 * KB * t + 4 * q);
-                    }
+                for (int q = 0; q < KB; ++q) {
+                    sa[q] = ptx::lds32(kst + ra * VBK + 4 * KB * t + 4 * q);
+                    sb[q] = ptx::lds32(kst + rb * VBK + 4 * KB * t + 4 * q);
                 }
-                float cs[NT][4], cs2[NT][4];
+            }
+            float cs[NT][4], cs2[NT][4], cz[NT][4];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) cs[nt][e] = cs2[nt][e] = 0.f;
+                for (int e = 0; e < 4; ++e) cs[nt][e] = cs2[nt][e] = cz[nt][e] = 0.f;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t a0 = ptx::lds32(base + key_lut_addr<KB>(sa, j, 0, laneoff));
-                    const uint32_t a1 = ptx::lds32(base + key_lut_addr<KB>(sb, j, 0, laneoff));
-                    const uint32_t a2 = ptx::lds32(base + key_lut_addr<KB>(sa, j, 1, laneoff));
-                    const uint32_t a3 = ptx::lds32(base + key_lut_addr<KB>(sb, j, 1, laneoff));
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        if (j & 1) ptx::mma_16816(cs2[nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
-                        else ptx::mma_16816(cs[nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
-                    }
-                }
-                float cz[NT][4];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) cz[nt][0] = cz[nt][1] = cz[nt][2] = cz[nt][3] = 0.f;
-                if constexpr (QJL) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        // +-1 pairs from sign bits (bit set -> +1)
-                        const uint32_t xa = za >> (4 * j), xb = zb >> (4 * j);
-                        const uint32_t a0 = 0xBC00BC00u ^ ((xa & 1u) << 15) ^ ((xa & 2u) << 30);
-                        const uint32_t a2 = 0xBC00BC00u ^ ((xa & 4u) << 13) ^ ((xa & 8u) << 28);
-                        const uint32_t a1 = 0xBC00BC00u ^ ((xb & 1u) << 15) ^ ((xb & 2u) << 30);
-                        const uint32_t a3 = 0xBC00BC00u ^ ((xb & 4u) << 13) ^ ((xb & 8u) << 28);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) ptx::mma_16816(cz[nt], a0, a1, a2, a3, bz[nt][j][0], bz[nt][j][1]);
-                    }
-                }
-                // ---- scores (log2 domain), online softmax
-                float s[NT][4];
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t a0 = ptx::lds32(base + key_lut_addr<KB>(sa, j, 0, laneoff));
+                const uint32_t a1 = ptx::lds32(base + key_lut_addr<KB>(sb, j, 0, laneoff));
+                const uint32_t a2 = ptx::lds32(base + key_lut_addr<KB>(sa, j, 1, laneoff));
+                const uint32_t a3 = ptx::lds32(base + key_lut_addr<KB>(sb, j, 1, laneoff));
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float kn = e < 2 ? kna : knb;
-                        const float gm = e < 2 ? ga : gb;
-                        float v = (cs[nt][e] + cs2[nt][e]) * f1[nt][e & 1];
-                        if constexpr (QJL) v = fmaf(gm * cz[nt][e], f2[nt][e & 1], v);
-                        s[nt][e] = (e < 2 ? va : vb) ? v * kn : -INFINITY;
-                    }
+                    if (j & 1) ptx::mma_16816(cs2[nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
+                    else ptx::mma_16816(cs[nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
                 }
-                float pv[NT][4];
-                bool any_v = false;
+            }
+            if constexpr (QJL) {
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    float mx0 = fmaxf(s[nt][0], s[nt][2]), mx1 = fmaxf(s[nt][1], s[nt][3]);
+                for (int j = 0; j < 4; ++j) {
+                    // +-1 pairs from sign bits (bit set -> +1)
+                    const uint32_t xa = za >> (4 * j), xb = zb2 >> (4 * j);
+                    const uint32_t a0 = 0xBC00BC00u ^ ((xa & 1u) << 15) ^ ((xa & 2u) << 30);
+                    const uint32_t a2 = 0xBC00BC00u ^ ((xa & 4u) << 13) ^ ((xa & 8u) << 28);
+                    const uint32_t a1 = 0xBC00BC00u ^ ((xb & 1u) << 15) ^ ((xb & 2u) << 30);
+                    const uint32_t a3 = 0xBC00BC00u ^ ((xb & 4u) << 13) ^ ((xb & 8u) << 28);
 #pragma unroll
-                    for (int o = 4; o < 32; o <<= 1) {
-                        mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, o));
-                        mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, o));
-                    }
-                    const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-                    const float c0 = ptx::ex2(m_run[nt][0] - mn0), c1 = ptx::ex2(m_run[nt][1] - mn1);
-                    m_run[nt][0] = mn0;
-                    m_run[nt][1] = mn1;
-                    const float p0 = ptx::ex2(s[nt][0] - mn0), p1 = ptx::ex2(s[nt][1] - mn1);
-                    const float p2 = ptx::ex2(s[nt][2] - mn0), p3 = ptx::ex2(s[nt][3] - mn1);
-                    l_run[nt][0] = fmaf(l_run[nt][0], c0, p0 + p2);
-                    l_run[nt][1] = fmaf(l_run[nt][1], c1, p1 + p3);
-                    if (c0 != 1.f || c1 != 1.f) {
+                    for (int nt = 0; nt < NT; ++nt) ptx::mma_16816(cz[nt], a0, a1, a2, a3, bz[nt][j][0], bz[nt][j][1]);
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float v = (cs[nt][e] + cs2[nt][e]) * f1[nt][e & 1];
+                    if constexpr (QJL) v = fmaf((e < 2 ? ga : gb) * cz[nt][e], f2[nt][e & 1], v);
+                    v *= e < 2 ? kna : knb;
+                    if (MASK) v = (e < 2 ? va : vb) ? v : -INFINITY;
+                    s[k][nt][e] = v;
+                }
+        }
+
+        // ---- softmax: the reference max moves only when a score exceeds it by 2^LAZY
+        bool need = false;
+        float lm[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            lm[nt][0] = lm[nt][1] = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < TPW; ++k) {
+                lm[nt][0] = fmaxf(lm[nt][0], fmaxf(s[k][nt][0], s[k][nt][2]));
+                lm[nt][1] = fmaxf(lm[nt][1], fmaxf(s[k][nt][1], s[k][nt][3]));
+            }
+            need |= lm[nt][0] > S.m[nt][0] + LAZY || lm[nt][1] > S.m[nt][1] + LAZY;
+        }
+        float vmax = 0.f;
+#pragma unroll
+        for (int k = 0; k < TPW; ++k) vmax = fmaxf(vmax, fmaxf(vn[k][0], vn[k][1]));
+        need |= (S.vscale == 0.f && vmax > 0.f) || vmax * S.vscale > VRANGE;
+        if (__any_sync(kFullMask, need)) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) {
+                    lm[nt][0] = fmaxf(lm[nt][0], __shfl_xor_sync(kFullMask, lm[nt][0], o));
+                    lm[nt][1] = fmaxf(lm[nt][1], __shfl_xor_sync(kFullMask, lm[nt][1], o));
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float mn = fmaxf(S.m[nt][h], lm[nt][h]);
+                    if (mn > S.m[nt][h]) {
+                        const float c = ptx::ex2(S.m[nt][h] - mn);
+                        S.l[nt][h] *= c;
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            acc[nt][i][0] *= c0;
-                            acc[nt][i][2] *= c0;
-                            acc[nt][i][1] *= c1;
-                            acc[nt][i][3] *= c1;
+                            S.acc[nt][i][h] *= c;
+                            S.acc[nt][i][h + 2] *= c;
                         }
+                        S.m[nt][h] = mn;
                     }
-                    pv[nt][0] = p0;
-                    pv[nt][1] = p1;
-                    pv[nt][2] = p2;
-                    pv[nt][3] = p3;
-                    if (a.tau > 0.f) {
-                        // Sparse V: the exact denominator (relative to m_run) is at least
-                        // 1 (the token that set the running max) and at least this lane's
-                        // partial sum, so p / max(1, l) bounds the exact weight from above
-                        const float t0v = a.tau * fmaxf(1.f, l_run[nt][0]);
-                        const float t1v = a.tau * fmaxf(1.f, l_run[nt][1]);
-                        if (p0 < t0v) pv[nt][0] = 0.f;
-                        if (p2 < t0v) pv[nt][2] = 0.f;
-                        if (p1 < t1v) pv[nt][1] = 0.f;
-                        if (p3 < t1v) pv[nt][3] = 0.f;
-                    }
-                    any_v |= (pv[nt][0] + pv[nt][1] + pv[nt][2] + pv[nt][3]) > 0.f;
                 }
-                // keep p * ||v|| * vscale inside fp16 range (power-of-two rescale)
-                float vmax = fmaxf(vna, vnb);
+            }
 #pragma unroll
-                for (int o = 4; o < 32; o <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFullMask, vmax, o));
-                if (vscale == 0.f) {
-                    vscale = vmax > 0.f ? exp2f(8.0f - ceilf(log2f(vmax))) : 0.f;
-                } else if (vmax * vscale > 16384.f) {
-                    const float shrink = exp2f(8.0f - ceilf(log2f(vmax * vscale)));
+            for (int o = 4; o < 32; o <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFullMask, vmax, o));
+            if (vmax > 0.f && (S.vscale == 0.f || vmax * S.vscale > VRANGE)) {
+                const float target = exp2f(-ceilf(log2f(vmax)));  // vmax * target in (0.5, 1]
+                if (S.vscale > 0.f) {
+                    const float f = target / S.vscale;
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) acc[nt][i][e] *= shrink;
-                    vscale *= shrink;
+                            for (int e = 0; e < 4; ++e) S.acc[nt][i][e] *= f;
                 }
-                if (__any_sync(kFullMask, any_v) && vscale > 0.f) {
-                    const float wa = vna * vscale, wb = vnb * vscale;
-                    uint32_t bv[NT][2];
+                S.vscale = target;
+            }
+        }
+
+        // ---- values, tile by tile
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        bv[nt][0] = ptx::movmatrix_trans(ptx::pack_half2(pv[nt][0] * wa, pv[nt][1] * wa));
-                        bv[nt][1] = ptx::movmatrix_trans(ptx::pack_half2(pv[nt][2] * wb, pv[nt][3] * wb));
-                    }
-                    // ---- values: word(s) of lane group g from physical tokens t, 4+t, 8+t, 12+t
-                    uint32_t A[8][4];
-                    if constexpr (VB == 2) {
-                        const uint32_t w0 = ptx::lds32(vst + (t) * VBV + 4 * g);
-                        const uint32_t w1 = ptx::lds32(vst + (4 + t) * VBV + 4 * g);
-                        const uint32_t w2 = ptx::lds32(vst + (8 + t) * VBV + 4 * g);
-                        const uint32_t w3 = ptx::lds32(vst + (12 + t) * VBV + 4 * g);
+        for (int k = 0; k < TPW; ++k) {
+            if (MASK && t0 + lb + 16 * k >= w.s1) break;  // warp-uniform
+            float pv[NT][4];
+            bool any_v = false;
 #pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            const uint32_t wa0 = half ? w2 : w0, wb0 = half ? w3 : w1;
-                            const uint32_t P = __byte_perm(wa0, wb0, 0x5140), Q = __byte_perm(wa0, wb0, 0x7362);
+            for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-                            for (int src = 0; src < 2; ++src) {
-                                const uint32_t x = src ? Q : P;
-#pragma unroll
-                                for (int sh = 0; sh < 8; sh += 2) {
-                                    const uint32_t sel = ((x >> sh) & 0x03030303u) * 0x22u + 0x10101010u;
-                                    const int f = (sh >> 1) & 1, hb = sh >> 2;
-                                    A[2 * (2 * src) + hb][2 * half + f] = __byte_perm(vl0, vl1, sel);
-                                    A[2 * (2 * src + 1) + hb][2 * half + f] = __byte_perm(vl0, vl1, sel >> 16);
-                                }
-                            }
-                        }
-                    } else {
-                        // 16 * VB bits per lane group and token (2*VB bytes at byte 2*VB*g),
-                        // realigned to two words; codes read through the value table
-                        uint32_t seg[4][2];
-#pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            const int tok = 4 * k4 + t;  // physical tokens t, 4+t, 8+t, 12+t
-                            const uint32_t byte_off = 2 * VB * g;  // 16*VB bits = 2*VB bytes per group
-                            const uint32_t wbase = byte_off >> 2, wsh = (byte_off & 3) * 8;
-                            const uint32_t lo = ptx::lds32(vst + tok * VBV + 4 * wbase);
-                            const uint32_t hi = (4 * wbase + 4 < VBV) ? ptx::lds32(vst + tok * VBV + 4 * wbase + 4) : 0u;
-                            const uint32_t hi2 = (4 * wbase + 8 < VBV) ? ptx::lds32(vst + tok * VBV + 4 * wbase + 8) : 0u;
-                            seg[k4][0] = __funnelshift_r(lo, hi, wsh);
-                            seg[k4][1] = __funnelshift_r(hi, hi2, wsh);
-                        }
-                        constexpr uint32_t vm = (1u << VB) - 1u;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-#pragma unroll
-                            for (int f = 0; f < 2; ++f) {
-                                const int bit = VB * (2 * i + f);
-#pragma unroll
-                                for (int half = 0; half < 2; ++half) {
-                                    const uint32_t* sx = seg[2 * half];
-                                    const uint32_t* sy = seg[2 * half + 1];
-                                    const uint32_t cx = bit >= 32 ? (sx[1] >> (bit - 32)) & vm
-                                                        : (bit + VB <= 32 ? (sx[0] >> bit) & vm
-                                                                          : __funnelshift_r(sx[0], sx[1], bit) & vm);
-                                    const uint32_t cy = bit >= 32 ? (sy[1] >> (bit - 32)) & vm
-                                                        : (bit + VB <= 32 ? (sy[0] >> bit) & vm
-                                                                          : __funnelshift_r(sy[0], sy[1], bit) & vm);
-                                    const uint32_t idx = cx | (cy << VB);
-                                    A[i][2 * half + f] = ptx::lds32(base + ((idx << 8) | 128u | laneoff));
-                                }
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-                            ptx::mma_16816(acc[nt][i], A[i][0], A[i][1], A[i][2], A[i][3], bv[nt][0], bv[nt][1]);
+                for (int e = 0; e < 4; ++e) pv[nt][e] = ptx::ex2(s[k][nt][e] - S.m[nt][e & 1]);
+                S.l[nt][0] += pv[nt][0] + pv[nt][2];
+                S.l[nt][1] += pv[nt][1] + pv[nt][3];
+                if (a.tau > 0.f) {
+                    // Sparse V: the exact denominator relative to the reference is at
+                    // least 1 (the reference is a seen score) and at least this lane's
+                    // partial sum, so p / max(1, l) bounds the exact weight
+                    const float th0 = a.tau * fmaxf(1.f, S.l[nt][0]), th1 = a.tau * fmaxf(1.f, S.l[nt][1]);
+                    if (pv[nt][0] < th0) pv[nt][0] = 0.f;
+                    if (pv[nt][2] < th0) pv[nt][2] = 0.f;
+                    if (pv[nt][1] < th1) pv[nt][1] = 0.f;
+                    if (pv[nt][3] < th1) pv[nt][3] = 0.f;
+                    any_v |= (pv[nt][0] + pv[nt][1] + pv[nt][2] + pv[nt][3]) > 0.f;
                 }
             }
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(empty0 + 8 * slot);
-            ++it;
+            if (a.tau > 0.f && !__any_sync(kFullMask, any_v)) continue;
+            if (S.vscale == 0.f) continue;  // every value norm so far is zero
+            const float wa = vn[k][0] * S.vscale, wb = vn[k][1] * S.vscale;
+            uint32_t bv[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                bv[nt][0] = ptx::movmatrix_trans(ptx::pack_half2(pv[nt][0] * wa, pv[nt][1] * wa));
+                bv[nt][1] = ptx::movmatrix_trans(ptx::pack_half2(pv[nt][2] * wb, pv[nt][3] * wb));
+            }
+            uint32_t A[8][4];
+            value_fragments<VB>(sbase + L.v_off + (lb + 16 * k) * VBV, base, g, t, laneoff, vl0, vl1, A);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    ptx::mma_16816(S.acc[nt][i], A[i][0], A[i][1], A[i][2], A[i][3], bv[nt][0], bv[nt][1]);
         }
-        // ---- merge the eight warps of the block
+    }
+
+    __device__ float group_sum_g(float x) const {  // sum over the 8 lanes sharing t
+        x += __shfl_xor_sync(kFullMask, x, 4);
+        x += __shfl_xor_sync(kFullMask, x, 8);
+        x += __shfl_xor_sync(kFullMask, x, 16);
+        return x;
+    }
+
+    // End of an item: merge the warps, publish the split's partial, and merge
+    // all splits when this is the last one of its (sequence, kv head).
+    __device__ void epilogue(const Item& w, SoftState<NT>& S) {
+        const int G = a.group;
+        float* merge = reinterpret_cast<float*>(smem + L.merge);
+        float2* ml = reinterpret_cast<float2*>(smem + L.ml);
+        int* last_flag = reinterpret_cast<int*>(smem + L.flags + 4);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                float l = l_run[nt][h];
-                l += __shfl_xor_sync(kFullMask, l, 4);
-                l += __shfl_xor_sync(kFullMask, l, 8);
-                l += __shfl_xor_sync(kFullMask, l, 16);
-                if (g == 0) ml[warp * 16 + nt * 8 + 2 * t + h] = make_float2(m_run[nt][h], l);
+                const float l = group_sum_g(S.l[nt][h]);
+                if (g == 0) ml[warp * 16 + nt * 8 + 2 * t + h] = make_float2(S.m[nt][h], l);
             }
-        const float unscale = vscale > 0.f ? 1.0f / vscale : 0.f;
+        const float unscale = S.vscale > 0.f ? 1.0f / S.vscale : 0.f;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 float* mw = merge + (warp * 8 * NT + nt * 8) * D;
                 const int c_lo = 16 * g + 2 * i, c_hi = c_lo + 1;
-                mw[(2 * t) * D + c_lo] = acc[nt][i][0] * unscale;
-                mw[(2 * t + 1) * D + c_lo] = acc[nt][i][1] * unscale;
-                mw[(2 * t) * D + c_hi] = acc[nt][i][2] * unscale;
-                mw[(2 * t + 1) * D + c_hi] = acc[nt][i][3] * unscale;
+                mw[(2 * t) * D + c_lo] = S.acc[nt][i][0] * unscale;
+                mw[(2 * t + 1) * D + c_lo] = S.acc[nt][i][1] * unscale;
+                mw[(2 * t) * D + c_hi] = S.acc[nt][i][2] * unscale;
+                mw[(2 * t + 1) * D + c_hi] = S.acc[nt][i][3] * unscale;
             }
         ptx::named_barrier(1, NUM_CONSUMERS);
-        if (*abort_flag) return;  // read after the barrier: every consumer leaves together
         const size_t pbase = (static_cast<size_t>(w.unit) * a.n_split + w.split) * G;
         for (int idx = tid; idx < G * D; idx += NUM_CONSUMERS) {
             const int h = idx / D, c = idx % D;
             float mx = -INFINITY;
 #pragma unroll
-            for (int ww = 0; ww < CW; ++ww) mx = fmaxf(mx, ml[ww * 16 + h].x);
+            for (int ww = 0; ww < CW; ++ww)
+                if (ml[ww * 16 + h].y > 0.f) mx = fmaxf(mx, ml[ww * 16 + h].x);
             float l = 0.f, s = 0.f;
             if (mx > -INFINITY) {
 #pragma unroll
                 for (int ww = 0; ww < CW; ++ww) {
                     const float2 v = ml[ww * 16 + h];
-                    if (v.x == -INFINITY) continue;
+                    if (!(v.y > 0.f)) continue;
                     const float f = ptx::ex2(v.x - mx);
                     l = fmaf(v.y, f, l);
                     s = fmaf(merge[(ww * 8 * NT + h) * D + c], f, s);
@@ -621,12 +734,11 @@ __device__ void consumer(const Args& a, uint8_t* smem, const Layout& L) {
         ptx::named_barrier(1, NUM_CONSUMERS);
         if (*last_flag) {
             __threadfence();
-            // ---- last block of this (sequence, kv head): merge the splits.
             // Split weights 2^(m_s - M) / L per (split, head) go to shared memory
-            // first (one warp per head), then every output channel is a weighted
+            // first (one warp per head); every output channel is then a weighted
             // sum of coalesced partial rows.
-            float* o_s = merge;             // [G][D]
-            float* wts = merge + 16 * D;    // [n_split][G]
+            float* o_s = merge;           // [G][D]
+            float* wts = merge + 16 * D;  // [n_split][G]
             const size_t ubase = static_cast<size_t>(w.unit) * a.n_split * G;
             for (int h = warp; h < G; h += CW) {
                 float mx = -INFINITY;
@@ -651,18 +763,20 @@ __device__ void consumer(const Args& a, uint8_t* smem, const Layout& L) {
             for (int idx = tid; idx < G * D; idx += NUM_CONSUMERS) {
                 const int h = idx / D, c = idx % D;
                 const float* src = a.ws_acc + (ubase + h) * D + c;
+                const size_t stride = static_cast<size_t>(G) * D;
                 float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
                 int sp = 0;
                 for (; sp + 4 <= a.n_split; sp += 4) {
-                    s0 = fmaf(__ldcg(src + static_cast<size_t>(sp) * G * D), wts[sp * G + h], s0);
-                    s1 = fmaf(__ldcg(src + static_cast<size_t>(sp + 1) * G * D), wts[(sp + 1) * G + h], s1);
-                    s2 = fmaf(__ldcg(src + static_cast<size_t>(sp + 2) * G * D), wts[(sp + 2) * G + h], s2);
-                    s3 = fmaf(__ldcg(src + static_cast<size_t>(sp + 3) * G * D), wts[(sp + 3) * G + h], s3);
+                    s0 = fmaf(__ldcg(src + sp * stride), wts[sp * G + h], s0);
+                    s1 = fmaf(__ldcg(src + (sp + 1) * stride), wts[(sp + 1) * G + h], s1);
+                    s2 = fmaf(__ldcg(src + (sp + 2) * stride), wts[(sp + 2) * G + h], s2);
+                    s3 = fmaf(__ldcg(src + (sp + 3) * stride), wts[(sp + 3) * G + h], s3);
                 }
-                for (; sp < a.n_split; ++sp) s0 = fmaf(__ldcg(src + static_cast<size_t>(sp) * G * D), wts[sp * G + h], s0);
+                for (; sp < a.n_split; ++sp) s0 = fmaf(__ldcg(src + sp * stride), wts[sp * G + h], s0);
                 o_s[h * D + c] = (s0 + s1) + (s2 + s3);
             }
             ptx::named_barrier(1, NUM_CONSUMERS);
+            const float inv_sqrt_d = 0.08838834764831845f;
             for (int h = warp; h < G; h += CW) {
                 float x[4];
 #pragma unroll
@@ -677,7 +791,56 @@ __device__ void consumer(const Args& a, uint8_t* smem, const Layout& L) {
         }
         ptx::named_barrier(1, NUM_CONSUMERS);
     }
-}
+
+    __device__ void run() {
+        const uint32_t full0 = base + L.bars, empty0 = full0 + 64;
+        uint32_t bq[NT][8][2];
+        uint32_t bz[NT][4][2];
+        float f1[NT][2], f2[NT][2];
+        SoftState<NT> S;
+        S.reset();
+        int seq = 0, qseq = 0;
+        bool done_ok = false;
+        while (true) {
+            const int slot = seq % a.stages, use = seq / a.stages;
+            if (!ptx::mbar_wait_bounded(full0 + 8 * slot, use & 1, WAIT_LIMIT)) set_abort();
+            ptx::named_barrier(1, NUM_CONSUMERS);  // every consumer warp sees the same abort state
+            if (aborted()) break;
+            const uint8_t* st = smem + L.ring + slot * L.stage_bytes;
+            const int4 hdr = *reinterpret_cast<const int4*>(st);
+            if (hdr.w & F_END) {
+                done_ok = true;
+                break;
+            }
+            const Item w = item_of(a, hdr.x);
+            if (w.bad && a.err && w.split == 0 && w.kv == 0 && tid == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
+            const bool empty = hdr.w & F_EMPTY;
+            if (hdr.w & F_FIRST) {
+                S.reset();
+                if (!empty) {
+                    if (!prologue(qseq, bq, bz, f1, f2)) break;
+                    ++qseq;
+                }
+            }
+            if (!empty) {
+                if (hdr.w & F_LAST) chunk<true>(w, st, hdr.y, bq, bz, f1, f2, S);
+                else chunk<false>(w, st, hdr.y, bq, bz, f1, f2, S);
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(empty0 + 8 * slot);
+            if (hdr.w & F_LAST) epilogue(w, S);
+            ++seq;
+        }
+        if (done_ok && tid == 0) {
+            // the last block to finish re-arms the global counters for the next call
+            __threadfence();
+            if (atomicAdd(a.counters + a.units + C_DONE, 1u) == gridDim.x - 1) {
+                a.counters[a.units + C_ITEM] = 0;
+                a.counters[a.units + C_DONE] = 0;
+            }
+        }
+    }
+};
 
 template <int KB, int VB, int NT, bool QJL>
 __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid_constant__ Args a) {
@@ -706,6 +869,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid
             ptx::mbar_init(bars + 8 * s, 1);
             ptx::mbar_init(bars + 64 + 8 * s, CW);
         }
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(bars + 128 + 8 * s, 1);
+            ptx::mbar_init(bars + 144 + 8 * s, 1);
+        }
         *reinterpret_cast<int*>(smem + L.flags) = 0;
         ptx::fence_mbar_init();
     }
@@ -713,7 +880,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid
     if (threadIdx.x >= NUM_CONSUMERS) {
         if (threadIdx.x == NUM_CONSUMERS) producer<KB, VB, QJL>(a, smem, L);
     } else {
-        consumer<KB, VB, NT, QJL>(a, smem, L);
+        Consumer<KB, VB, NT, QJL> c(a, smem, L);
+        c.run();
     }
 }
 
@@ -767,6 +935,7 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     a.sketch = c.qjl_matrix;
     a.q = q;
     a.q_dtype = q_dtype;
+    a.q_bytes = q_dtype == TQ_F32 ? 4 : 2;
     a.seq_lens = seq_lens;
     a.ws_ml = reinterpret_cast<float2*>(ws + plan.off_ml);
     a.ws_acc = reinterpret_cast<float*>(ws + plan.off_acc);
@@ -781,14 +950,12 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     a.n_split = plan.n_split;
     a.split_len = plan.split_len;
     a.max_len = max_len;
-    a.n_items = c.batch * p.num_kv_heads * plan.n_split;
+    a.units = c.batch * p.num_kv_heads;
+    a.n_items = a.units * plan.n_split;
     a.m = p.qjl_dims;
     const float sm = p.sm_scale > 0.0f ? p.sm_scale : 1.0f / std::sqrt(128.0f);
     a.sm_scale_log2 = sm * LOG2E;
     a.tau = p.sparse_v_threshold;
-    uint32_t words[8];
-    rotation_sign_bits(p.seed, 128, words);
-    for (int i = 0; i < 4; ++i) a.signs[i] = words[i];
     const double sd = std::sqrt(128.0);
     const double ak = kcb->fp16_scale > 0.0 ? kcb->fp16_scale : sd;
     const double av = vcb->fp16_scale > 0.0 ? vcb->fp16_scale : sd;
@@ -799,12 +966,14 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
         a.vcent[j] = j < (1 << p.v_bits) ? half_bits(vcb->centroids[j] * av) : 0;
     }
     a.staged_norms = (c.capacity % 8) == 0;
+    uint32_t words[8];
+    rotation_sign_bits(p.seed, 128, words);
+    for (int i = 0; i < 4; ++i) a.signs[i] = words[i];
     const int nt = a.group <= 8 ? 1 : 2;
     const int kb = p.k_bits, vb = p.v_bits;
-    // as many stages as fit in 227 KB next to the table and the merge buffers
+    // as many stages as fit in 227 KB next to the tables and the merge buffers
     const Layout fixed = layout(kb, vb, nt, 0, p.qjl_dims);
-    const uint32_t stage = fixed.stage_bytes;
-    int stages = static_cast<int>((232448u - fixed.total) / stage);
+    int stages = static_cast<int>((232448u - fixed.total) / fixed.stage_bytes);
     if (stages > 8) stages = 8;
     if (stages < 2) return cudaErrorInvalidConfiguration;
     a.stages = stages;

@@ -246,18 +246,29 @@ static long long gcd_ll(long long a, long long b) {
 }
 
 DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_sms) {
-    // Split count: at least kBlocksPerSm blocks' worth of (unit, split) items per
-    // SM, rounded up so that the item count is a multiple of the SM count when
-    // possible (every persistent block then gets the same number of items),
-    // and never splits shorter than kMinSplitTokens.
+    // Split count.  Few long sequences: one wave of equal items, one per SM,
+    // when that keeps at least 85% of the SMs busy (every item then carries
+    // one prologue and one merge); otherwise a multiple of the SM count where
+    // possible.  Many sequences (a batch, possibly ragged): about four items
+    // per SM, which the kernel's dynamic scheduling balances.  Splits are never
+    // shorter than kMinSplitTokens nor more than kMaxSplits.
     DecodePlan plan;
     const long long units = static_cast<long long>(batch) * p.num_kv_heads;
-    const long long want = (static_cast<long long>(num_sms) * kBlocksPerSm + units - 1) / units;
-    const long long step = num_sms / gcd_ll(units, num_sms);
-    long long n = (want + step - 1) / step * step;
     long long most = (max_seq_len + kMinSplitTokens - 1) / kMinSplitTokens;
     if (most > kMaxSplits) most = kMaxSplits;
-    if (n > most) n = want < most ? want : most;
+    long long n;
+    const long long one_wave = num_sms / units;
+    if (units * 4 >= num_sms) {
+        n = (4ll * num_sms + units - 1) / units;
+    } else if (one_wave >= 1 && one_wave * units * 100 >= 85ll * num_sms) {
+        n = one_wave;
+    } else {
+        const long long want = (static_cast<long long>(num_sms) * kBlocksPerSm + units - 1) / units;
+        const long long step = num_sms / gcd_ll(units, num_sms);
+        n = (want + step - 1) / step * step;
+        if (n > most) n = want;
+    }
+    if (n > most) n = most;
     if (n < 1) n = 1;
     long long len = (max_seq_len + n - 1) / n;
     len = (len + kSplitAlign - 1) / kSplitAlign * kSplitAlign;
@@ -268,7 +279,7 @@ DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_s
     plan.off_ml = 0;
     plan.off_acc = (slots * 2 * sizeof(float) + 255) / 256 * 256;
     plan.off_counters = (plan.off_acc + slots * p.head_dim * sizeof(float) + 255) / 256 * 256;
-    plan.bytes = plan.off_counters + static_cast<size_t>(units) * sizeof(uint32_t);
+    plan.bytes = plan.off_counters + static_cast<size_t>(units + kGlobalCounters) * sizeof(uint32_t);
     return plan;
 }
 
@@ -283,7 +294,7 @@ static DecodePlan plan_bound(const tq_params& p, int batch, int max_seq_len) {
     const long long units = static_cast<long long>(batch) * p.num_kv_heads;
     plan.off_acc = (slots * 2 * sizeof(float) + 255) / 256 * 256;
     plan.off_counters = (plan.off_acc + slots * p.head_dim * sizeof(float) + 255) / 256 * 256;
-    plan.bytes = plan.off_counters + static_cast<size_t>(units) * sizeof(uint32_t);
+    plan.bytes = plan.off_counters + static_cast<size_t>(units + kGlobalCounters) * sizeof(uint32_t);
     return plan;
 }
 

@@ -15,7 +15,7 @@ struct DecodePlan {
     int split_len = 0;
     size_t off_ml = 0;   // float2 (m, l) per (b, hq, split)
     size_t off_acc = 0;  // float acc[d] per (b, hq, split)
-    size_t off_counters = 0;  // uint32 per (b, kv head): splits finished
+    size_t off_counters = 0;  // uint32 per (b, kv head): splits finished; then kGlobalCounters
     size_t bytes = 0;
 };
 
@@ -25,6 +25,8 @@ constexpr int kBlocksPerSm = 2;
 constexpr int kMinSplitTokens = 256;
 // Most splits per (sequence, kv head); bounds the merge scratch in shared memory.
 constexpr int kMaxSplits = 384;
+// Work-distribution counters after the per-(sequence, kv head) ones.
+constexpr int kGlobalCounters = 2;
 // Token granularity of split boundaries.
 constexpr int kSplitAlign = 64;
 
