@@ -321,7 +321,8 @@ extern "C" tq_status tq_decode_attention(const tq_params* params, const tq_codeb
     if (decode_mma_supported(p)) {
         const cudaError_t e = launch_decode_mma(p, kcb, vcb, *cache, d_q, q_dtype, d_seq_lens, max_seq_len, d_out, plan,
                                                 static_cast<char*>(d_workspace), d_error, sms, s);
-        return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+        if (e != cudaErrorNotSupported) return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+        // otherwise (a device whose shared-memory window differs) take the general path
     }
     DecodeArgs a{};
     fill_decode_side(a.k, p.k_mode, p.k_bits, p.head_dim, kcb, cache->k_codes, cache->k_norms);

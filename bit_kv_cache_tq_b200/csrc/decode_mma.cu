@@ -62,6 +62,10 @@ constexpr int NUM_THREADS = (CW + 1) * 32;   // + one producer warp
 constexpr int NUM_CONSUMERS = CW * 32;
 constexpr int CHUNK = CW * TPW * 16;         // tokens per stage
 constexpr uint32_t LUT_BYTES = 65536;        // 256 entries x 256 B
+// Shared-window address of the dynamic shared memory (the per-block reserved
+// shared memory precedes it); the host checks it before choosing this kernel,
+// and table lookups carry it as an immediate offset.
+constexpr uint32_t WINDOW = 1024;
 constexpr uint32_t QSLOT_BYTES = 16 * D * 4; // one item's queries, up to 16 heads in fp32
 constexpr long long WAIT_LIMIT = 2000000000ll;  // clock cycles (~1 s)
 constexpr float LOG2E = 1.4426950408889634f;
@@ -180,8 +184,8 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         st = smem + L.ring + slot * L.stage_bytes;
         return true;
     };
+    int i = blockIdx.x;  // the first item of every block is static; later ones come from the counter
     while (ok) {
-        const int i = static_cast<int>(atomicAdd(a.counters + a.units + C_ITEM, 1u));
         if (i >= a.n_items) break;
         const Item w = item_of(a, i);
         const bool empty = w.s0 >= w.s1;
@@ -233,6 +237,7 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
             ++seq;
             t0 += CHUNK;
         } while (!empty && t0 < w.s1);
+        i = static_cast<int>(gridDim.x + atomicAdd(a.counters + a.units + C_ITEM, 1u));
     }
     if (ok) {  // end-of-work sentinel
         uint32_t full;
@@ -271,7 +276,7 @@ __device__ __forceinline__ uint32_t key_lut_addr(const uint32_t (&seg)[4], int j
 // Value fragments A[m-tile i][reg] of one 16-token tile for lane group g.
 template <int VB>
 __device__ __forceinline__ void value_fragments(uint32_t vst, uint32_t base, int g, int t, uint32_t laneoff,
-                                                uint32_t vl0, uint32_t vl1, uint32_t (&A)[8][4]) {
+                                                uint32_t (&A)[8][4]) {
     constexpr int VBV = 16 * VB;
     if constexpr (VB == 2) {
         // word g of physical tokens t, 4+t, 8+t, 12+t (logical k = 2t, 2t+1, 2t+8, 2t+9)
@@ -279,22 +284,25 @@ __device__ __forceinline__ void value_fragments(uint32_t vst, uint32_t base, int
         const uint32_t w1 = ptx::lds32(vst + (4 + t) * VBV + 4 * g);
         const uint32_t w2 = ptx::lds32(vst + (8 + t) * VBV + 4 * g);
         const uint32_t w3 = ptx::lds32(vst + (12 + t) * VBV + 4 * g);
+        // Nibble n of a word holds channels 16g+2n (bits 0-1) and 16g+2n+1
+        // (bits 2-3), i.e. rows g and g+8 of m-tile n.  Interleaving the nibbles
+        // of the two tokens gives bytes (token a nibble | token b nibble << 4);
+        // each byte indexes the 64-bit table entry {(c[a0], c[b0]), (c[a1], c[b1])}
+        // = the row-g and row-(g+8) registers of that m-tile.
+        const uint32_t voff = 128u | ((laneoff & 60u) << 1);  // half-warp replica (lane & 15) * 8
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-            const uint32_t wa0 = half ? w2 : w0, wb0 = half ? w3 : w1;
-            // interleave the bytes of the two tokens: fields at equal offsets pair up
-            const uint32_t P = __byte_perm(wa0, wb0, 0x5140), Q = __byte_perm(wa0, wb0, 0x7362);
+            const uint32_t wa = half ? w2 : w0, wb = half ? w3 : w1;
+            const uint32_t even = (wa & 0x0F0F0F0Fu) | ((wb << 4) & 0xF0F0F0F0u);  // nibbles 0, 2, 4, 6
+            const uint32_t odd = ((wa >> 4) & 0x0F0F0F0Fu) | (wb & 0xF0F0F0F0u);   // nibbles 1, 3, 5, 7
 #pragma unroll
-            for (int src = 0; src < 2; ++src) {
-                const uint32_t x = src ? Q : P;
-#pragma unroll
-                for (int sh = 0; sh < 8; sh += 2) {
-                    // 2-bit codes (u0, u1) -> byte selector {2u0, 2u0+1, 2u1, 2u1+1}
-                    const uint32_t sel = ((x >> sh) & 0x03030303u) * 0x22u + 0x10101010u;
-                    const int f = (sh >> 1) & 1, hb = sh >> 2;
-                    A[2 * (2 * src) + hb][2 * half + f] = __byte_perm(vl0, vl1, sel);
-                    A[2 * (2 * src + 1) + hb][2 * half + f] = __byte_perm(vl0, vl1, sel >> 16);
-                }
+            for (int k = 0; k < 4; ++k) {
+                const uint2 re = ptx::lds64_imm<WINDOW>(__byte_perm(even, voff, 0x6504 | (k << 4)));
+                const uint2 ro = ptx::lds64_imm<WINDOW>(__byte_perm(odd, voff, 0x6504 | (k << 4)));
+                A[2 * k][2 * half] = re.x;
+                A[2 * k][2 * half + 1] = re.y;
+                A[2 * k + 1][2 * half] = ro.x;
+                A[2 * k + 1][2 * half + 1] = ro.y;
             }
         }
     } else {
@@ -328,7 +336,7 @@ __device__ __forceinline__ void value_fragments(uint32_t vst, uint32_t base, int
                     const uint32_t cy = bit >= 32 ? (sy[1] >> (bit - 32)) & vm
                                                   : (bit + VB <= 32 ? (sy[0] >> bit) & vm
                                                                     : __funnelshift_r(sy[0], sy[1], bit) & vm);
-                    A[i][2 * half + f] = ptx::lds32(base + (((cx | (cy << VB)) << 8) | 128u | laneoff));
+                    A[i][2 * half + f] = ptx::lds32_imm<WINDOW>(((cx | (cy << VB)) << 8) | 128u | laneoff);
                 }
             }
     }
@@ -359,7 +367,7 @@ struct Consumer {
     uint8_t* smem;
     const Layout& L;
     int tid, warp, lane, g, t;
-    uint32_t base, laneoff, vl0, vl1;
+    uint32_t base, laneoff;
 
     __device__ Consumer(const Args& a_, uint8_t* s_, const Layout& L_) : a(a_), smem(s_), L(L_) {
         tid = threadIdx.x;
@@ -369,8 +377,6 @@ struct Consumer {
         t = lane & 3;
         base = ptx::smem_addr(smem);
         laneoff = lane * 4;
-        vl0 = a.vcent[0] | (static_cast<uint32_t>(a.vcent[1]) << 16);
-        vl1 = a.vcent[2] | (static_cast<uint32_t>(a.vcent[3]) << 16);
     }
 
     __device__ bool aborted() const { return *reinterpret_cast<volatile int*>(smem + L.flags) != 0; }
@@ -531,22 +537,19 @@ struct Consumer {
                     sb[q] = ptx::lds32(kst + rb * VBK + 4 * KB * t + 4 * q);
                 }
             }
-            float cs[NT][4], cs2[NT][4], cz[NT][4];
+            float cs[NT][4], cz[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) cs[nt][e] = cs2[nt][e] = cz[nt][e] = 0.f;
+                for (int e = 0; e < 4; ++e) cs[nt][e] = cz[nt][e] = 0.f;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const uint32_t a0 = ptx::lds32(base + key_lut_addr<KB>(sa, j, 0, laneoff));
-                const uint32_t a1 = ptx::lds32(base + key_lut_addr<KB>(sb, j, 0, laneoff));
-                const uint32_t a2 = ptx::lds32(base + key_lut_addr<KB>(sa, j, 1, laneoff));
-                const uint32_t a3 = ptx::lds32(base + key_lut_addr<KB>(sb, j, 1, laneoff));
+                const uint32_t a0 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sa, j, 0, laneoff));
+                const uint32_t a1 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sb, j, 0, laneoff));
+                const uint32_t a2 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sa, j, 1, laneoff));
+                const uint32_t a3 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sb, j, 1, laneoff));
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    if (j & 1) ptx::mma_16816(cs2[nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
-                    else ptx::mma_16816(cs[nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
-                }
+                for (int nt = 0; nt < NT; ++nt) ptx::mma_16816(cs[nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
             }
             if constexpr (QJL) {
 #pragma unroll
@@ -565,7 +568,7 @@ struct Consumer {
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    float v = (cs[nt][e] + cs2[nt][e]) * f1[nt][e & 1];
+                    float v = cs[nt][e] * f1[nt][e & 1];
                     if constexpr (QJL) v = fmaf((e < 2 ? ga : gb) * cz[nt][e], f2[nt][e & 1], v);
                     v *= e < 2 ? kna : knb;
                     if (MASK) v = (e < 2 ? va : vb) ? v : -INFINITY;
@@ -664,7 +667,7 @@ struct Consumer {
                 bv[nt][1] = ptx::movmatrix_trans(ptx::pack_half2(pv[nt][2] * wb, pv[nt][3] * wb));
             }
             uint32_t A[8][4];
-            value_fragments<VB>(sbase + L.v_off + (lb + 16 * k) * VBV, base, g, t, laneoff, vl0, vl1, A);
+            value_fragments<VB>(sbase + L.v_off + (lb + 16 * k) * VBV, base, g, t, laneoff, A);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -734,46 +737,35 @@ struct Consumer {
         ptx::named_barrier(1, NUM_CONSUMERS);
         if (*last_flag) {
             __threadfence();
-            // Split weights 2^(m_s - M) / L per (split, head) go to shared memory
-            // first (one warp per head); every output channel is then a weighted
-            // sum of coalesced partial rows.
-            float* o_s = merge;           // [G][D]
-            float* wts = merge + 16 * D;  // [n_split][G]
+            // Merge the splits: every thread owns (head, channel) pairs and folds
+            // the splits in with a running max, loading SB splits at a time so
+            // their L2 reads overlap.
+            float* o_s = merge;  // [G][D]
             const size_t ubase = static_cast<size_t>(w.unit) * a.n_split * G;
-            for (int h = warp; h < G; h += CW) {
-                float mx = -INFINITY;
-                for (int sp = lane; sp < a.n_split; sp += 32) {
-                    const float2 v = __ldcg(a.ws_ml + ubase + sp * G + h);
-                    if (v.y > 0.f) mx = fmaxf(mx, v.x);
-                }
-                mx = group_max<32>(mx);
-                float l = 0.f;
-                for (int sp = lane; sp < a.n_split; sp += 32) {
-                    const float2 v = __ldcg(a.ws_ml + ubase + sp * G + h);
-                    const float wgt = (v.y > 0.f && mx > -INFINITY) ? ptx::ex2(v.x - mx) : 0.f;
-                    wts[sp * G + h] = wgt;
-                    l = fmaf(v.y, wgt, l);
-                }
-                l = group_sum<32>(l);
-                const float inv_l = l > 0.f ? 1.f / l : 0.f;
-                __syncwarp();
-                for (int sp = lane; sp < a.n_split; sp += 32) wts[sp * G + h] *= inv_l;
-            }
-            ptx::named_barrier(1, NUM_CONSUMERS);
+            constexpr int SB = 16;
             for (int idx = tid; idx < G * D; idx += NUM_CONSUMERS) {
                 const int h = idx / D, c = idx % D;
-                const float* src = a.ws_acc + (ubase + h) * D + c;
-                const size_t stride = static_cast<size_t>(G) * D;
-                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-                int sp = 0;
-                for (; sp + 4 <= a.n_split; sp += 4) {
-                    s0 = fmaf(__ldcg(src + sp * stride), wts[sp * G + h], s0);
-                    s1 = fmaf(__ldcg(src + (sp + 1) * stride), wts[(sp + 1) * G + h], s1);
-                    s2 = fmaf(__ldcg(src + (sp + 2) * stride), wts[(sp + 2) * G + h], s2);
-                    s3 = fmaf(__ldcg(src + (sp + 3) * stride), wts[(sp + 3) * G + h], s3);
+                float M = -INFINITY, Lsum = 0.f, acc = 0.f;
+                for (int s0 = 0; s0 < a.n_split; s0 += SB) {
+                    float2 mlv[SB];
+                    float av[SB];
+#pragma unroll
+                    for (int j = 0; j < SB; ++j) {
+                        const int sp = s0 + j;
+                        mlv[j] = sp < a.n_split ? __ldcg(a.ws_ml + ubase + sp * G + h) : make_float2(-INFINITY, 0.f);
+                        av[j] = sp < a.n_split ? __ldcg(a.ws_acc + (ubase + sp * G + h) * D + c) : 0.f;
+                    }
+#pragma unroll
+                    for (int j = 0; j < SB; ++j) {
+                        if (!(mlv[j].y > 0.f)) continue;
+                        const float mn = fmaxf(M, mlv[j].x);
+                        const float f_old = ptx::ex2(M - mn), f_new = ptx::ex2(mlv[j].x - mn);
+                        Lsum = fmaf(Lsum, f_old, mlv[j].y * f_new);
+                        acc = fmaf(acc, f_old, av[j] * f_new);
+                        M = mn;
+                    }
                 }
-                for (; sp < a.n_split; ++sp) s0 = fmaf(__ldcg(src + sp * stride), wts[sp * G + h], s0);
-                o_s[h * D + c] = (s0 + s1) + (s2 + s3);
+                o_s[h * D + c] = Lsum > 0.f ? acc / Lsum : 0.f;
             }
             ptx::named_barrier(1, NUM_CONSUMERS);
             const float inv_sqrt_d = 0.08838834764831845f;
@@ -799,6 +791,7 @@ struct Consumer {
         float f1[NT][2], f2[NT][2];
         SoftState<NT> S;
         S.reset();
+        Item w{};
         int seq = 0, qseq = 0;
         bool done_ok = false;
         while (true) {
@@ -812,10 +805,10 @@ struct Consumer {
                 done_ok = true;
                 break;
             }
-            const Item w = item_of(a, hdr.x);
-            if (w.bad && a.err && w.split == 0 && w.kv == 0 && tid == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
             const bool empty = hdr.w & F_EMPTY;
             if (hdr.w & F_FIRST) {
+                w = item_of(a, hdr.x);
+                if (w.bad && a.err && w.split == 0 && w.kv == 0 && tid == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
                 S.reset();
                 if (!empty) {
                     if (!prologue(qseq, bq, bz, f1, f2)) break;
@@ -846,24 +839,8 @@ template <int KB, int VB, int NT, bool QJL>
 __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid_constant__ Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const Layout L = layout(KB, VB, NT, a.stages, QJL ? a.m : 0);
-    // per-lane replicated centroid-pair tables: key pairs in bytes [0,128) of
-    // each 256-byte entry, value pairs (3- and 4-bit values) in [128, 256)
-    uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-    const __half* kc = reinterpret_cast<const __half*>(a.kcent);
-    const __half* vc = reinterpret_cast<const __half*>(a.vcent);
-    constexpr int nk = 1 << (2 * KB), nv = VB >= 3 ? 1 << (2 * VB) : 0;
-    for (int idx = threadIdx.x; idx < (nk + nv) * 32; idx += NUM_THREADS) {
-        const int e = idx >> 5, r = idx & 31;
-        if (e < nk) {
-            const __half2 v = __halves2half2(kc[e & ((1 << KB) - 1)], kc[e >> KB]);
-            lut[e * 64 + r] = *reinterpret_cast<const uint32_t*>(&v);
-        } else {
-            const int ev = e - nk;
-            const __half2 v = __halves2half2(vc[ev & ((1 << VB) - 1)], vc[ev >> VB]);
-            lut[ev * 64 + 32 + r] = *reinterpret_cast<const uint32_t*>(&v);
-        }
-    }
-    if (threadIdx.x == 0) {
+    ptx::launch_dependents();  // the next kernel may start launching; it waits for this one to finish
+    if (threadIdx.x == NUM_CONSUMERS) {
         const uint32_t bars = ptx::smem_addr(smem + L.bars);
         for (int s = 0; s < a.stages; ++s) {
             ptx::mbar_init(bars + 8 * s, 1);
@@ -876,13 +853,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid
         *reinterpret_cast<int*>(smem + L.flags) = 0;
         ptx::fence_mbar_init();
     }
-    __syncthreads();
+    __syncthreads();  // mbarriers initialised
     if (threadIdx.x >= NUM_CONSUMERS) {
-        if (threadIdx.x == NUM_CONSUMERS) producer<KB, VB, QJL>(a, smem, L);
-    } else {
-        Consumer<KB, VB, NT, QJL> c(a, smem, L);
-        c.run();
+        if (threadIdx.x == NUM_CONSUMERS) {
+            ptx::wait_prerequisites();  // the cache and queries may come from the previous kernel
+            producer<KB, VB, QJL>(a, smem, L);
+        }
+        return;
     }
+    // per-lane replicated centroid-pair tables, built while the first copies fly:
+    // key pairs in bytes [0,128) of each 256-byte entry, value pairs (3- and
+    // 4-bit values) in [128, 256)
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
+    const __half* kc = reinterpret_cast<const __half*>(a.kcent);
+    const __half* vc = reinterpret_cast<const __half*>(a.vcent);
+    constexpr int nk = 1 << (2 * KB), nv = VB >= 3 ? 1 << (2 * VB) : 256;
+    for (int idx = threadIdx.x; idx < (nk + nv) * 32; idx += NUM_CONSUMERS) {
+        const int e = idx >> 5, r = idx & 31;
+        if (e < nk) {
+            const __half2 v = __halves2half2(kc[e & ((1 << KB) - 1)], kc[e >> KB]);
+            lut[e * 64 + r] = *reinterpret_cast<const uint32_t*>(&v);
+        } else if (VB >= 3) {
+            const int ev = e - nk;
+            const __half2 v = __halves2half2(vc[ev & ((1 << VB) - 1)], vc[ev >> VB]);
+            lut[ev * 64 + 32 + r] = *reinterpret_cast<const uint32_t*>(&v);
+        } else {
+            // byte ev = (token a: two 2-bit codes) | (token b: two codes) << 4;
+            // word 2*replica: first channel (a, b), word 2*replica + 1: second channel
+            const int ev = e - nk, rep = r >> 1;
+            const int ca = (r & 1) ? (ev >> 2) & 3 : ev & 3;
+            const int cb = (r & 1) ? (ev >> 6) & 3 : (ev >> 4) & 3;
+            const __half2 v = __halves2half2(vc[ca], vc[cb]);
+            lut[ev * 64 + 32 + 2 * rep + (r & 1)] = *reinterpret_cast<const uint32_t*>(&v);
+        }
+    }
+    if (ptx::smem_addr(smem) != WINDOW) {  // the host checked the reserved size; never expected
+        if (threadIdx.x == 0) {
+            if (a.err) atomicOr(a.err, TQ_DEVERR_TIMEOUT);
+            *reinterpret_cast<volatile int*>(smem + L.flags) = 1;
+        }
+    }
+    ptx::wait_prerequisites();
+    ptx::named_barrier(1, NUM_CONSUMERS);  // tables complete
+    Consumer<KB, VB, NT, QJL> c(a, smem, L);
+    c.run();
 }
 
 template <int KB, int VB, int NT, bool QJL>
@@ -890,7 +904,18 @@ static cudaError_t launch_typed(const Args& a, int grid, size_t smem, cudaStream
     cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<KB, VB, NT, QJL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    decode_mma_kernel<KB, VB, NT, QJL><<<grid, NUM_THREADS, smem, stream>>>(a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_mma_kernel<KB, VB, NT, QJL>, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -969,6 +994,11 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     uint32_t words[8];
     rotation_sign_bits(p.seed, 128, words);
     for (int i = 0; i < 4; ++i) a.signs[i] = words[i];
+    int reserved = 0, dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+        static_cast<uint32_t>(reserved) != WINDOW)
+        return cudaErrorNotSupported;
     const int nt = a.group <= 8 ? 1 : 2;
     const int kb = p.k_bits, vb = p.v_bits;
     // as many stages as fit in 227 KB next to the tables and the merge buffers

@@ -59,6 +59,12 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
         : "memory");
 }
 
+// Programmatic dependent launch: let the next kernel in the stream begin
+// launching, and wait until every kernel this one depends on has finished and
+// its writes are visible (a no-op when not launched as a dependent).
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void named_barrier(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -90,6 +96,22 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+// Loads at (register + compile-time offset): the offset folds into the
+// instruction, so a table at a fixed shared-window address needs no add.
+template <uint32_t OFF>
+__device__ __forceinline__ uint32_t lds32_imm(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF));
+    return v;
+}
+
+template <uint32_t OFF>
+__device__ __forceinline__ uint2 lds64_imm(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0,%1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(addr), "n"(OFF));
     return v;
 }
 

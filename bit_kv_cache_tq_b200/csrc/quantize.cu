@@ -25,6 +25,7 @@
 
 #include "device_common.cuh"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace tq {
 
@@ -177,6 +178,8 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
     constexpr int LPV = D / 32;  // lanes per vector
     constexpr int VPW = 32 / LPV;  // vectors per warp pass
     const QuantSide& s = a.side[blockIdx.y];
+    ptx::launch_dependents();    // the next kernel may start launching
+    ptx::wait_prerequisites();   // inputs and cache may come from the previous kernel
     const int lane = threadIdx.x & 31, sub = lane % LPV, grp = lane / LPV;
     const long long total = static_cast<long long>(a.batch) * a.n_new * a.hkv;
     const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
@@ -334,7 +337,17 @@ static cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t stream) {
     const long long cap = static_cast<long long>(sms > 0 ? sms : 148) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    quantize_append_kernel<D, DTYPE><<<dim3(static_cast<unsigned>(blocks), 2), 256, 0, stream>>>(a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 2);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_append_kernel<D, DTYPE>, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
