@@ -737,35 +737,55 @@ struct Consumer {
         ptx::named_barrier(1, NUM_CONSUMERS);
         if (*last_flag) {
             __threadfence();
-            // Merge the splits: every thread owns (head, channel) pairs and folds
-            // the splits in with a running max, loading SB splits at a time so
-            // their L2 reads overlap.
-            float* o_s = merge;  // [G][D]
+            // Merge the splits: one warp per head, lane = float4 column.  The
+            // first batch of partial rows is requested before the split weights
+            // 2^(m_s - M) / L are reduced, so both reads overlap; the weighted sum
+            // runs in split order, so the result does not depend on timing.
+            float* o_s = merge;           // [G][D]
+            float* wts = merge + 16 * D;  // [n_split][G]
             const size_t ubase = static_cast<size_t>(w.unit) * a.n_split * G;
-            constexpr int SB = 16;
-            for (int idx = tid; idx < G * D; idx += NUM_CONSUMERS) {
-                const int h = idx / D, c = idx % D;
-                float M = -INFINITY, Lsum = 0.f, acc = 0.f;
-                for (int s0 = 0; s0 < a.n_split; s0 += SB) {
-                    float2 mlv[SB];
-                    float av[SB];
+            const float4* src4 = reinterpret_cast<const float4*>(a.ws_acc + ubase * D);
+            constexpr int PB = 16;  // splits per batch of loads
+            for (int h = warp; h < G; h += CW) {
+                float4 v[PB];
 #pragma unroll
-                    for (int j = 0; j < SB; ++j) {
-                        const int sp = s0 + j;
-                        mlv[j] = sp < a.n_split ? __ldcg(a.ws_ml + ubase + sp * G + h) : make_float2(-INFINITY, 0.f);
-                        av[j] = sp < a.n_split ? __ldcg(a.ws_acc + (ubase + sp * G + h) * D + c) : 0.f;
+                for (int j = 0; j < PB; ++j)
+                    v[j] = j < a.n_split ? __ldcg(src4 + (j * G + h) * (D / 4) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+                float mx = -INFINITY;
+                for (int sp = lane; sp < a.n_split; sp += 32) {
+                    const float2 m2 = __ldcg(a.ws_ml + ubase + sp * G + h);
+                    if (m2.y > 0.f) mx = fmaxf(mx, m2.x);
+                }
+                mx = group_max<32>(mx);
+                float l = 0.f;
+                for (int sp = lane; sp < a.n_split; sp += 32) {
+                    const float2 m2 = __ldcg(a.ws_ml + ubase + sp * G + h);
+                    const float wgt = (m2.y > 0.f && mx > -INFINITY) ? ptx::ex2(m2.x - mx) : 0.f;
+                    wts[sp * G + h] = wgt;
+                    l = fmaf(m2.y, wgt, l);
+                }
+                l = group_sum<32>(l);
+                const float inv_l = l > 0.f ? 1.f / l : 0.f;
+                __syncwarp();
+                float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int s0 = 0; s0 < a.n_split; s0 += PB) {
+                    if (s0 > 0) {
+#pragma unroll
+                        for (int j = 0; j < PB; ++j)
+                            v[j] = s0 + j < a.n_split ? __ldcg(src4 + ((s0 + j) * G + h) * (D / 4) + lane)
+                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
 #pragma unroll
-                    for (int j = 0; j < SB; ++j) {
-                        if (!(mlv[j].y > 0.f)) continue;
-                        const float mn = fmaxf(M, mlv[j].x);
-                        const float f_old = ptx::ex2(M - mn), f_new = ptx::ex2(mlv[j].x - mn);
-                        Lsum = fmaf(Lsum, f_old, mlv[j].y * f_new);
-                        acc = fmaf(acc, f_old, av[j] * f_new);
-                        M = mn;
+                    for (int j = 0; j < PB; ++j) {
+                        const float wgt = s0 + j < a.n_split ? wts[(s0 + j) * G + h] : 0.f;
+                        acc4.x = fmaf(v[j].x, wgt, acc4.x);
+                        acc4.y = fmaf(v[j].y, wgt, acc4.y);
+                        acc4.z = fmaf(v[j].z, wgt, acc4.z);
+                        acc4.w = fmaf(v[j].w, wgt, acc4.w);
                     }
                 }
-                o_s[h * D + c] = Lsum > 0.f ? acc / Lsum : 0.f;
+                *reinterpret_cast<float4*>(o_s + h * D + 4 * lane) =
+                    make_float4(acc4.x * inv_l, acc4.y * inv_l, acc4.z * inv_l, acc4.w * inv_l);
             }
             ptx::named_barrier(1, NUM_CONSUMERS);
             const float inv_sqrt_d = 0.08838834764831845f;
