@@ -314,7 +314,7 @@ extern "C" tq_status tq_decode_attention(const tq_params* params, const tq_codeb
     if (p.v_mode == TQ_MODE_TURBO && (st = validate_codebook(vcb, p.head_dim, p.v_bits)) != TQ_OK) return st;
     const int sms = num_sms_current();
     if (sms <= 0) return TQ_ERR_CUDA;
-    const DecodePlan plan = plan_decode(p, cache->batch, max_seq_len, sms);
+    const DecodePlan plan = plan_decode(p, cache->batch, max_seq_len, sms, workspace_bytes);
     if (workspace_bytes < plan.bytes) return TQ_ERR_CAPACITY;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);

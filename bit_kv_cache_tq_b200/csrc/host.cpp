@@ -245,7 +245,20 @@ static long long gcd_ll(long long a, long long b) {
     return a;
 }
 
-DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_sms) {
+size_t counter_region_bytes(size_t workspace_bytes) {
+    const size_t words = workspace_bytes / kMinUnitBytes + kGlobalCounters;
+    return (words * sizeof(uint32_t) + 255) / 256 * 256;
+}
+
+// Partials (m, l) then acc, after the counter region.
+static void place_partials(DecodePlan& plan, size_t slots, int head_dim, size_t counters) {
+    plan.off_counters = 0;
+    plan.off_ml = counters;
+    plan.off_acc = plan.off_ml + (slots * 2 * sizeof(float) + 255) / 256 * 256;
+    plan.bytes = plan.off_acc + slots * head_dim * sizeof(float);
+}
+
+DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_sms, size_t workspace_bytes) {
     // Split count.  Few long sequences: one wave of equal items, one per SM,
     // when that keeps at least 85% of the SMs busy (every item then carries
     // one prologue and one merge); otherwise a multiple of the SM count where
@@ -276,26 +289,27 @@ DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_s
     plan.n_split = static_cast<int>(n);
     plan.split_len = static_cast<int>(len);
     const size_t slots = static_cast<size_t>(batch) * p.num_q_heads * plan.n_split;
-    plan.off_ml = 0;
-    plan.off_acc = (slots * 2 * sizeof(float) + 255) / 256 * 256;
-    plan.off_counters = (plan.off_acc + slots * p.head_dim * sizeof(float) + 255) / 256 * 256;
-    plan.bytes = plan.off_counters + static_cast<size_t>(units + kGlobalCounters) * sizeof(uint32_t);
+    place_partials(plan, slots, p.head_dim, counter_region_bytes(workspace_bytes));
     return plan;
 }
 
 // Workspace bound valid for every device: the split count never exceeds
-// ceil(max_seq_len / kMinSplitTokens).
-static DecodePlan plan_bound(const tq_params& p, int batch, int max_seq_len) {
-    tq_params q = p;
-    DecodePlan plan = plan_decode(q, batch, max_seq_len, 1);
+// ceil(max_seq_len / kMinSplitTokens).  The counter region grows with the
+// workspace, so the size is the least fixed point of
+// bytes = counter_region_bytes(bytes) + partials.
+static size_t workspace_bound(const tq_params& p, int batch, int max_seq_len) {
     long long most = (max_seq_len + kMinSplitTokens - 1) / kMinSplitTokens;
     if (most > kMaxSplits) most = kMaxSplits;
     const size_t slots = static_cast<size_t>(batch) * p.num_q_heads * most;
-    const long long units = static_cast<long long>(batch) * p.num_kv_heads;
-    plan.off_acc = (slots * 2 * sizeof(float) + 255) / 256 * 256;
-    plan.off_counters = (plan.off_acc + slots * p.head_dim * sizeof(float) + 255) / 256 * 256;
-    plan.bytes = plan.off_counters + static_cast<size_t>(units + kGlobalCounters) * sizeof(uint32_t);
-    return plan;
+    DecodePlan plan;
+    place_partials(plan, slots, p.head_dim, 0);
+    const size_t partials = plan.bytes;
+    size_t bytes = partials;
+    for (;;) {
+        const size_t next = partials + counter_region_bytes(bytes);
+        if (next == bytes) return bytes;
+        bytes = next;
+    }
 }
 
 }  // namespace tq
@@ -369,7 +383,7 @@ tq_status tq_decode_workspace_bytes(const tq_params* params, int32_t batch, int3
     tq_status st = tq::validate_params(params);
     if (st != TQ_OK) return st;
     if (!bytes_out || batch < 1 || max_seq_len < 1) return TQ_ERR_INVALID_ARG;
-    *bytes_out = tq::plan_bound(*params, batch, max_seq_len).bytes;
+    *bytes_out = tq::workspace_bound(*params, batch, max_seq_len);
     return TQ_OK;
 }
 

@@ -10,13 +10,16 @@ namespace tq {
 
 // Decode split plan: the token axis of every (sequence, kv head) is cut into
 // n_split ranges of split_len tokens (the last one may be shorter or empty).
+// Workspace layout: the counter region comes first and its size depends only
+// on the workspace size, so counters sit at the same addresses whatever the
+// batch and lengths of a call; partial results follow it.
 struct DecodePlan {
     int n_split = 1;
     int split_len = 0;
-    size_t off_ml = 0;   // float2 (m, l) per (b, hq, split)
-    size_t off_acc = 0;  // float acc[d] per (b, hq, split)
     size_t off_counters = 0;  // uint32 per (b, kv head): splits finished; then kGlobalCounters
-    size_t bytes = 0;
+    size_t off_ml = 0;        // float2 (m, l) per (b, hq, split)
+    size_t off_acc = 0;       // float acc[d] per (b, hq, split)
+    size_t bytes = 0;         // end of the partials
 };
 
 // Thread blocks aimed at per SM when choosing the split count.
@@ -29,6 +32,10 @@ constexpr int kMaxSplits = 384;
 constexpr int kGlobalCounters = 2;
 // Token granularity of split boundaries.
 constexpr int kSplitAlign = 64;
+// Fewest partial bytes one (sequence, kv head) takes: one split of one query
+// head, (m, l) and acc[d] with d >= 64, is 8 + 4 d >= 264 bytes.  A workspace
+// of W bytes therefore never serves more than W / kMinUnitBytes of them.
+constexpr size_t kMinUnitBytes = 256;
 
 tq_status validate_params(const tq_params* p);
 tq_status validate_codebook(const tq_codebook* cb, int head_dim, int bits);
@@ -36,7 +43,9 @@ tq_status validate_cache(const tq_params& p, const tq_cache* c);
 bool aligned16(const void* ptr);
 // Bytes of one stored vector: d*bits/8 (TURBO) or d (INT8).
 int vector_bytes(int mode, int bits, int head_dim);
-DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_sms);
+// Bytes of the counter region at the front of a workspace of this size.
+size_t counter_region_bytes(size_t workspace_bytes);
+DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_sms, size_t workspace_bytes);
 // Tensor-core decode path (decode_mma.cu): d = 128, TURBO K and V.
 bool decode_mma_supported(const tq_params& p);
 // SM count of the current CUDA device (0 when it cannot be queried).

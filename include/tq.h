@@ -198,7 +198,9 @@ tq_status tq_cache_bytes(const tq_params* params, int32_t batch, int32_t capacit
  * Host only.  Bytes of device workspace tq_decode_attention needs for
  * `batch` sequences of at most `max_seq_len` tokens on any device.  The
  * workspace must be zero-filled once before its first use; every call that
- * completes leaves it ready for the next one.
+ * completes leaves it ready for the next one, whatever its batch and lengths,
+ * provided every call on it passes the same workspace_bytes (the size fixes
+ * where its counters live).
  */
 tq_status tq_decode_workspace_bytes(const tq_params* params, int32_t batch, int32_t max_seq_len,
                                     size_t* bytes_out);
@@ -254,8 +256,9 @@ tq_status tq_dequantize(const tq_params* params, const tq_codebook* kcb, const t
  *   d_out          device, [batch][Hq][d] fp32.
  *   d_workspace    device scratch of at least tq_decode_workspace_bytes
  *                  bytes (16-byte aligned), zero-filled before its first use
- *                  (it holds per-(sequence, kv head) split counters that each
- *                  call returns to zero).  Calls sharing a workspace must not
+ *                  (its front holds per-(sequence, kv head) split counters
+ *                  that each call returns to zero).  Calls sharing a
+ *                  workspace pass the same workspace_bytes and must not
  *                  overlap on the device.
  * Sparse V (sparse_v_threshold = tau > 0): position i is dropped from the V
  * sum of head h only when exp(s_i - m)/l < tau for running softmax

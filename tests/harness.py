@@ -175,11 +175,13 @@ def gpu_quantize(layer, k, v, capacity, positions=None, cache=None):
     return cache, st, word
 
 
-def gpu_decode(layer, q, cache, lens, max_len=None):
+def gpu_decode(layer, q, cache, lens, max_len=None, ws=None):
+    """Decode attention through the C ABI; a fresh zeroed workspace unless `ws` is given."""
     bsz = q.shape[0]
     lens_t = torch.as_tensor(np.asarray(lens), dtype=torch.int32).cuda()
     max_len = int(max(lens)) if max_len is None else max_len
-    ws = torch.zeros(tq.tq_decode_workspace_bytes(layer.params, bsz, max_len), dtype=torch.uint8, device="cuda")
+    if ws is None:
+        ws = torch.zeros(tq.tq_decode_workspace_bytes(layer.params, bsz, max_len), dtype=torch.uint8, device="cuda")
     out = torch.empty(bsz, layer.hq, layer.d, dtype=torch.float32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     tq.tq_decode_attention(layer.params, layer.kcb, layer.vcb, q.cuda().contiguous(), cache, lens_t, max_len, out, ws,

@@ -299,3 +299,23 @@ def test_decode_is_deterministic():
     a, _, _ = H.gpu_decode(layer, q, cache, [t])
     b, _, _ = H.gpu_decode(layer, q, cache, [t])
     assert np.array_equal(a, b)
+
+
+def test_workspace_reused_across_batches_and_lengths():
+    """One workspace, zeroed once, serves calls of different batch sizes and
+    lengths in any order; each result equals that of a fresh workspace."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=22)
+    t = 3000
+    k = inputs.lognormal_kv(4, t, 8, 128, seed=13, layer=22, which=inputs.K)
+    v = inputs.lognormal_kv(4, t, 8, 128, seed=13, layer=22, which=inputs.V)
+    q = inputs.queries(4, 32, 128, seed=13, layer=22)
+    wide, _, _ = H.gpu_quantize(layer, k, v, t)
+    narrow, _, _ = H.gpu_quantize(layer, k[:1], v[:1], t)
+    ws = torch.zeros(tq.tq_decode_workspace_bytes(layer.params, 4, t), dtype=torch.uint8, device="cuda")
+    calls = [(wide, q, [t, 2500, 1777, 64]), (narrow, q[:1], [700]), (wide, q, [2000, 1, 999, 1500]),
+             (narrow, q[:1], [t]), (wide, q, [t, t, t, t]), (narrow, q[:1], [257])]
+    for cache, qq, lens in calls:
+        got, st, word = H.gpu_decode(layer, qq, cache, lens, ws=ws)
+        assert st == tq.TQ_OK and word == 0
+        fresh, _, _ = H.gpu_decode(layer, qq, cache, lens)
+        assert np.array_equal(got, fresh), lens
