@@ -24,6 +24,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <mutex>
 
 #include "device_common.cuh"
 #include "internal.h"
@@ -357,4 +358,68 @@ extern "C" tq_status tq_decode_attention(const tq_params* params, const tq_codeb
         default: e = launch_decode_dim<256>(a, s); break;
     }
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Decode attention with library-owned scratch.  Some callers cannot allocate
+// device memory at the point of the call: an allocator hook that must not
+// recurse into allocation, a runtime whose memory pool is fixed before
+// serving starts, or code that runs while another component holds the
+// allocator.  For them the split partials and counters live in one fixed
+// device array of this library, so a call allocates nothing.  The array is
+// shared by every call on a device: it keeps the last call's partials (only
+// its counter words must be zero when a call starts, and every completed call
+// leaves them so), and calls that overlap on the device race on it.
+
+namespace tq {
+namespace {
+
+__device__ __align__(256) unsigned char g_static_scratch[TQ_DECODE_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_scratch_mutex;
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+// Address of this device's scratch.  The first call on a device looks the
+// symbol up and zero-fills the array on `stream`, ahead of the call's kernels.
+cudaError_t static_scratch(void** out, cudaStream_t stream) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+    if (!g_static_scratch_ptr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+        if (e != cudaSuccess) return e;
+        e = cudaMemsetAsync(ptr, 0, TQ_DECODE_STATIC_SCRATCH_BYTES, stream);
+        if (e != cudaSuccess) return e;
+        g_static_scratch_ptr[dev] = ptr;
+    }
+    *out = g_static_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace tq
+
+extern "C" tq_status tq_decode_attention_static(const tq_params* params, const tq_codebook* kcb,
+                                                const tq_codebook* vcb, const void* d_q, tq_dtype q_dtype,
+                                                const tq_cache* cache, const int32_t* d_seq_lens,
+                                                int32_t max_seq_len, float* d_out, uint32_t* d_error, void* stream) {
+    using namespace tq;
+    tq_status st = validate_params(params);
+    if (st != TQ_OK) return st;
+    if ((st = validate_cache(*params, cache)) != TQ_OK) return st;
+    if (max_seq_len < 1) return TQ_ERR_INVALID_ARG;
+    // Reject calls whose partials cannot fit before touching the device.
+    const int sms = num_sms_current();
+    if (sms <= 0) return TQ_ERR_CUDA;
+    if (plan_decode(*params, cache->batch, max_seq_len, sms, TQ_DECODE_STATIC_SCRATCH_BYTES).bytes >
+        TQ_DECODE_STATIC_SCRATCH_BYTES)
+        return TQ_ERR_CAPACITY;
+    void* scratch = nullptr;
+    if (static_scratch(&scratch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return TQ_ERR_CUDA;
+    return tq_decode_attention(params, kcb, vcb, d_q, q_dtype, cache, d_seq_lens, max_seq_len, d_out, scratch,
+                               TQ_DECODE_STATIC_SCRATCH_BYTES, d_error, stream);
 }

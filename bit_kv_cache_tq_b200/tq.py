@@ -29,8 +29,11 @@ TQ_DEVERR_POSITION, TQ_DEVERR_SEQLEN = 0x1, 0x2
 EXPORTED = (
     "tq_status_string", "tq_abi_version", "tq_codebook_init", "tq_rotation_signs", "tq_qjl_matrix",
     "tq_cache_bytes", "tq_decode_workspace_bytes", "tq_quantize_append", "tq_dequantize",
-    "tq_decode_attention", "tq_read_device_error",
+    "tq_decode_attention", "tq_decode_attention_static", "tq_read_device_error",
 )
+
+# Bytes of the library's own decode scratch per device (tq_decode_attention_static).
+TQ_DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class tq_codebook(ctypes.Structure):
@@ -79,6 +82,9 @@ _lib.tq_dequantize.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), 
 _lib.tq_decode_attention.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p, ctypes.c_int,
                                      _P(tq_cache), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+_lib.tq_decode_attention_static.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
+                                            ctypes.c_int, _P(tq_cache), ctypes.c_void_p, ctypes.c_int32,
+                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
 _lib.tq_read_device_error.argtypes = [ctypes.c_void_p, _P(ctypes.c_uint32), ctypes.c_void_p, ctypes.c_int32]
 for _name in EXPORTED:
     if _name not in ("tq_status_string", "tq_abi_version"):
@@ -242,6 +248,17 @@ def tq_decode_attention(params, kcb, vcb, q, cache, seq_lens, max_seq_len, out, 
                                   _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(error),
                                   _stream(stream))
     _check(st, "tq_decode_attention")
+
+
+def tq_decode_attention_static(params, kcb, vcb, q, cache, seq_lens, max_seq_len, out, error=None, stream=None):
+    """tq_decode_attention on the library's own per-device scratch (no workspace argument)."""
+    assert q.is_contiguous() and out.is_contiguous() and out.dtype == torch.float32
+    assert seq_lens.dtype == torch.int32 and seq_lens.is_cuda
+    c = cache.struct()
+    st = _lib.tq_decode_attention_static(ctypes.byref(params), kcb and ctypes.byref(kcb), vcb and ctypes.byref(vcb),
+                                         _ptr(q), _dtype_code(q), ctypes.byref(c), _ptr(seq_lens), max_seq_len,
+                                         _ptr(out), _ptr(error), _stream(stream))
+    _check(st, "tq_decode_attention_static")
 
 
 def tq_read_device_error(error, stream=None, timeout_ms=2000):

@@ -273,6 +273,34 @@ tq_status tq_decode_attention(const tq_params* params, const tq_codebook* kcb, c
                               const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
                               void* d_workspace, size_t workspace_bytes, uint32_t* d_error, void* stream);
 
+/* Bytes of the library's own decode scratch on each device. */
+#define TQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/*
+ * tq_decode_attention without a caller workspace; the pages have no
+ * counterpart (the method says nothing about where scratch lives).  It is
+ * for callers that must not allocate device memory when they decode: the
+ * split partials and counters go to one fixed 16 MiB device array of the
+ * library (TQ_DECODE_STATIC_SCRATCH_BYTES per device), and the call
+ * allocates nothing.  Arguments as for tq_decode_attention.
+ *   - Returns TQ_ERR_CAPACITY, before any device work, when the call needs
+ *     more scratch than the array holds (the launch plan for batch and
+ *     max_seq_len on the current device decides; a workspace bound from
+ *     tq_decode_workspace_bytes at or below the limit always fits).
+ *   - The first call on a device looks up the array's address and queues a
+ *     zero fill of it on `stream` ahead of its own kernels; make that first
+ *     call before any stream capture.
+ *   - The array is shared by all calls on the device and keeps the last
+ *     call's partials; only its counter words must be zero when a call
+ *     starts, and every completed call leaves them zero.  Calls that overlap
+ *     on the device (other streams, other threads) race on it: serialise
+ *     them.
+ */
+tq_status tq_decode_attention_static(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                                     const void* d_q, tq_dtype q_dtype, const tq_cache* cache,
+                                     const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
+                                     uint32_t* d_error, void* stream);
+
 /*
  * Copy the device error word to *out after the work queued on `stream` so
  * far, waiting at most timeout_ms milliseconds (polling, never blocking

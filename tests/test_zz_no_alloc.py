@@ -1,0 +1,56 @@
+"""tq_decode_attention_static (library-owned scratch, no allocation) against
+tq_decode_attention on a caller workspace.  Collected last on purpose: it must
+pass both alone and after every other GPU test has used the device."""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import harness as H
+from bit_kv_cache_tq_b200 import inputs, tq
+
+pytestmark = pytest.mark.gpu
+
+
+def _static(layer, q, cache, lens):
+    lens_t = torch.as_tensor(np.asarray(lens), dtype=torch.int32).cuda()
+    out = torch.empty(q.shape[0], layer.hq, layer.d, dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.tq_decode_attention_static(layer.params, layer.kcb, layer.vcb, q.cuda().contiguous(), cache, lens_t,
+                                  int(max(lens)), out, err)
+    st, word = tq.tq_read_device_error(err)
+    assert st == tq.TQ_OK and word == 0
+    return out.cpu().numpy()
+
+
+def test_static_scratch_matches_workspace_entry_point():
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=31)
+    t = 3000
+    k = inputs.lognormal_kv(3, t, 8, 128, seed=31, layer=31, which=inputs.K)
+    v = inputs.lognormal_kv(3, t, 8, 128, seed=31, layer=31, which=inputs.V)
+    q = inputs.queries(3, 32, 128, seed=31, layer=31)
+    wide, _, _ = H.gpu_quantize(layer, k, v, t)
+    narrow, _, _ = H.gpu_quantize(layer, k[:1], v[:1], t)
+    # two calls in a row on one shape, then other batch sizes and lengths
+    for cache, qq, lens in [(wide, q, [t, 1999, 700]), (wide, q, [t, 1999, 700]), (narrow, q[:1], [t]),
+                            (wide, q, [64, t, 1])]:
+        want, st, word = H.gpu_decode(layer, qq, cache, lens)
+        assert st == tq.TQ_OK and word == 0
+        got = _static(layer, qq, cache, lens)
+        assert H.rel_l2_per_vector(got, want).max() <= H.ATTN_TOL, lens
+
+
+def test_static_scratch_rejects_calls_beyond_its_size():
+    """1024 sequences x 64 query heads need more partials than the array holds;
+    the call fails before any device work (the cache pointers are never read)."""
+    p = tq.make_params(128, 64, 8)
+    kcb, vcb = tq.tq_codebook_init(128, 4), tq.tq_codebook_init(128, 2)
+    fake = 1 << 20
+    cache = tq.tq_cache(1024, 16, fake, fake, None, None, fake, fake, None)
+    st = tq.library().tq_decode_attention_static(ctypes.byref(p), ctypes.byref(kcb), ctypes.byref(vcb), fake,
+                                                 tq.TQ_BF16, ctypes.byref(cache), fake, 16, fake, None, None)
+    assert st == tq.TQ_ERR_CAPACITY
+    need = tq.tq_decode_workspace_bytes(p, 1024, 16)
+    assert need > tq.TQ_DECODE_STATIC_SCRATCH_BYTES
