@@ -134,6 +134,39 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+# DRAM traffic of the decode kernel, taken from the committed ncu summary; it
+# applies only while the kernel's sources are the ones that were profiled.
+DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_mma_kernel_llama8b_layer_32k.md")
+DECODE_SOURCES = ("decode_mma.cu", "device_common.cuh", "ptx.cuh")
+
+
+def decode_source_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "bit_kv_cache_tq_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(tokens):
+    """DRAM bytes (read + write) of one decode launch over `tokens` tokens per
+    kv head, scaled from the profiled launch; None when the summary is missing
+    or the kernel changed since it was taken."""
+    fields = {}
+    try:
+        with open(DECODE_PROFILE, encoding="utf-8") as fh:
+            for line in fh:
+                if line.startswith("- ") and ": " in line:
+                    key, val = line[2:].split(": ", 1)
+                    fields[key.strip()] = val.strip().strip("`")
+        if fields.get("kernel sources sha256") != decode_source_sha256():
+            return None
+        return float(fields["dram bytes per launch"]) * tokens / float(fields["tokens per kv head"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 # ------------------------------------------------------------------ oracle leg
 class OracleDecode:
     """The fp64 CPU oracle on a bounded sample of the decode step.  One unit
@@ -380,7 +413,7 @@ def run_tq(args, world, rank, local):
             "hbm_gbs": alg_bytes * LAYERS / (ms / steps * 1e-3) / 1e9,
             "pct_of_8tbs": 100.0 * alg_bytes * LAYERS / (ms / steps * 1e-3) / 8e12,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                         "frac": achieved / peak, "traffic": profiled_traffic(seq), "peak_kind": peak_kind,
                          "kernel": "tq_decode_attention (one fused kernel), %.2f us per launch, %d B algorithmic"
                                    % (decode_us, alg_bytes)},
             "cpu_baseline": cpu_info,
