@@ -42,6 +42,11 @@ def bytes_per_token_head(k_bits=K_BITS, v_bits=V_BITS, d=D):
     return d * k_bits // 8 + 2 + d * v_bits // 8 + 2
 
 
+def rank_seed(rank):
+    """Input seed of one replica: every rank draws its own layers and queries."""
+    return SEED + 7919 * rank
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -265,7 +270,7 @@ def run_tq(args, world, rank, local):
     steps, warmup = args.steps, args.warmup
     total_steps = steps + warmup
     cap = CONTEXT + total_steps + 1
-    gen_seed = SEED + 7919 * rank
+    gen_seed = rank_seed(rank)
     kcb, vcb = tq.tq_codebook_init(D, K_BITS), tq.tq_codebook_init(D, V_BITS)
     params = [tq.make_params(D, HQ, HKV, K_BITS, V_BITS, seed=gen_seed + l) for l in range(LAYERS)]
     caches = [tq.alloc_cache(p, BATCH, cap, device=dev) for p in params]
