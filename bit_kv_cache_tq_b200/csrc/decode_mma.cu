@@ -106,7 +106,7 @@ struct Args {
 // [header | K codes | V codes | K norms | V norms | QJL words | gammas].
 struct Layout {
     uint32_t ring, stage_bytes, k_off, v_off, kn_off, vn_off, z_off, gam_off;
-    uint32_t qring, qh, sq, fac, merge, ml, bars, flags, total;
+    uint32_t qring, qh, qlo, sq, fac, merge, ml, bars, flags, total;
 };
 
 __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int m) {
@@ -120,8 +120,9 @@ __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int
     L.gam_off = L.z_off + CHUNK * (m / 8);
     L.stage_bytes = L.gam_off + (m > 0 ? CHUNK * 2 : 0);
     L.qring = L.ring + stages * L.stage_bytes;        // 2 query slots
-    L.qh = L.qring + 2 * QSLOT_BYTES;                  // fp16 [16][128]
-    L.sq = L.qh + 16 * D * 2;                          // fp16 [16][64]
+    L.qh = L.qring + 2 * QSLOT_BYTES;                  // fp16 [16][128], rounded q~
+    L.qlo = L.qh + 16 * D * 2;                         // fp16 [16][128], q~ minus the rounded part
+    L.sq = L.qlo + 16 * D * 2;                         // fp16 [16][64]
     L.fac = L.sq + 16 * 64 * 2;                        // float F1[16], F2[16]
     L.merge = L.fac + 32 * 4;                          // float [CW][8*nt][128]
     L.ml = L.merge + CW * 8 * nt * D * 4;              // float2 [CW][16]
@@ -385,9 +386,9 @@ struct Consumer {
         *reinterpret_cast<volatile int*>(smem + L.flags) = 1;
     }
 
-    // Rotated queries of the item (fp16, scaled to max |q~| = 1) and the scale
+    // Rotated queries of the item (fp16 hi + lo pair, scaled to max |q~| = 1) and the scale
     // factors of the scores; false on abort.
-    __device__ bool prologue(int qseq, uint32_t (&bq)[NT][8][2], uint32_t (&bz)[NT][4][2], float (&f1)[NT][2],
+    __device__ bool prologue(int qseq, uint32_t (&bq)[NT][8][4], uint32_t (&bz)[NT][4][2], float (&f1)[NT][2],
                              float (&f2)[NT][2]) {
         const uint32_t qfull = base + L.bars + 128 + 8 * (qseq & 1);
         if (!ptx::mbar_wait_bounded(qfull, (qseq >> 1) & 1, WAIT_LIMIT)) set_abort();
@@ -396,6 +397,7 @@ struct Consumer {
         const int G = a.group;
         const uint8_t* qsrc = smem + L.qring + (qseq & 1) * QSLOT_BYTES;
         __half* qh = reinterpret_cast<__half*>(smem + L.qh);
+        __half* ql = reinterpret_cast<__half*>(smem + L.qlo);
         __half* sq = reinterpret_cast<__half*>(smem + L.sq);
         float* fac = reinterpret_cast<float*>(smem + L.fac);
         float* merge = reinterpret_cast<float*>(smem + L.merge);
@@ -415,7 +417,13 @@ struct Consumer {
             amax = group_max<32>(amax);
             const float qmax = amax > 0.f ? amax : 1.f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) qh[h * D + lane * 4 + e] = __float2half_rn(x[e] / qmax);
+            for (int e = 0; e < 4; ++e) {
+                // two fp16 terms: the scores keep about 22 bits of q~
+                const float u = x[e] / qmax;
+                const __half hi = __float2half_rn(u);
+                qh[h * D + lane * 4 + e] = hi;
+                ql[h * D + lane * 4 + e] = __float2half_rn(u - __half2float(hi));
+            }
             float smax = 1.f;
             if constexpr (QJL) {
                 // S q~ for sketch rows lane and lane + 32 (m <= 64); q~ staged in
@@ -452,10 +460,13 @@ struct Consumer {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const __half* qrow = qh + (nt * 8 + g) * D + 32 * t;
+            const __half* lrow = ql + (nt * 8 + g) * D + 32 * t;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 bq[nt][j][0] = *reinterpret_cast<const uint32_t*>(qrow + 4 * j);
                 bq[nt][j][1] = *reinterpret_cast<const uint32_t*>(qrow + 4 * j + 2);
+                bq[nt][j][2] = *reinterpret_cast<const uint32_t*>(lrow + 4 * j);
+                bq[nt][j][3] = *reinterpret_cast<const uint32_t*>(lrow + 4 * j + 2);
             }
             if constexpr (QJL) {
                 const __half* srow = sq + (nt * 8 + g) * 64 + 16 * t;
@@ -475,7 +486,7 @@ struct Consumer {
 
     // One chunk: this warp's two tiles.  MASK: the chunk may end before CHUNK tokens.
     template <bool MASK>
-    __device__ void chunk(const Item& w, const uint8_t* st, int t0, const uint32_t (&bq)[NT][8][2],
+    __device__ void chunk(const Item& w, const uint8_t* st, int t0, const uint32_t (&bq)[NT][8][4],
                           const uint32_t (&bz)[NT][4][2], const float (&f1)[NT][2], const float (&f2)[NT][2],
                           SoftState<NT>& S) {
         constexpr int VBK = 16 * KB, VBV = 16 * VB;
@@ -537,11 +548,12 @@ struct Consumer {
                     sb[q] = ptx::lds32(kst + rb * VBK + 4 * KB * t + 4 * q);
                 }
             }
-            float cs[NT][4], cz[NT][4];
+            // hi and lo query parts accumulate in separate chains
+            float cs[NT][4], cl[NT][4], cz[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) cs[nt][e] = cz[nt][e] = 0.f;
+                for (int e = 0; e < 4; ++e) cs[nt][e] = cl[nt][e] = cz[nt][e] = 0.f;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const uint32_t a0 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sa, j, 0, laneoff));
@@ -549,7 +561,10 @@ struct Consumer {
                 const uint32_t a2 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sa, j, 1, laneoff));
                 const uint32_t a3 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sb, j, 1, laneoff));
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) ptx::mma_16816(cs[nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
+                for (int nt = 0; nt < NT; ++nt) {
+                    ptx::mma_16816(cs[nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
+                    ptx::mma_16816(cl[nt], a0, a1, a2, a3, bq[nt][j][2], bq[nt][j][3]);
+                }
             }
             if constexpr (QJL) {
 #pragma unroll
@@ -568,7 +583,7 @@ struct Consumer {
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    float v = cs[nt][e] * f1[nt][e & 1];
+                    float v = (cs[nt][e] + cl[nt][e]) * f1[nt][e & 1];
                     if constexpr (QJL) v = fmaf((e < 2 ? ga : gb) * cz[nt][e], f2[nt][e & 1], v);
                     v *= e < 2 ? kna : knb;
                     if (MASK) v = (e < 2 ? va : vb) ? v : -INFINITY;
@@ -806,7 +821,7 @@ struct Consumer {
 
     __device__ void run() {
         const uint32_t full0 = base + L.bars, empty0 = full0 + 64;
-        uint32_t bq[NT][8][2];
+        uint32_t bq[NT][8][4];
         uint32_t bz[NT][4][2];
         float f1[NT][2], f2[NT][2];
         SoftState<NT> S;

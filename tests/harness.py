@@ -190,6 +190,27 @@ def gpu_decode(layer, q, cache, lens, max_len=None, ws=None):
     return out.cpu().numpy(), st, word
 
 
+def stored_hat(layer, cache, b, h, n, which):
+    """The oracle's reconstruction of the GPU's own stored bytes (codes, norms,
+    QJL bits, gamma) for tokens [0, n) of sequence b, kv head h: attention
+    parity is judged on the same codes, after code parity has passed."""
+    mode, bits = layer.side(which)
+    if which == 0:
+        raw, nrm = cache.k_codes[b, h, :n].cpu().numpy(), cache.k_norms[b, h, :n].cpu().numpy()
+    else:
+        raw, nrm = cache.v_codes[b, h, :n].cpu().numpy(), cache.v_norms[b, h, :n].cpu().numpy()
+    norm16 = nrm.view(np.float16)
+    if mode == tq.TQ_MODE_INT8:
+        return layer.oracle_decode({"q": raw.view(np.int8).astype(np.int64), "norm16": norm16}, which)
+    enc = {"codes": unpack_codes(raw, bits, layer.d), "norm16": norm16}
+    if which == 0 and layer.params.qjl_dims:
+        m = layer.params.qjl_dims
+        z = cache.k_qjl[b, h, :n].cpu().numpy()
+        enc["qjl_bits"] = np.unpackbits(z, axis=-1, bitorder="little")[:, :m]
+        enc["gamma16"] = cache.k_gamma[b, h, :n].cpu().numpy().view(np.float16)
+    return layer.oracle_decode(enc, which)
+
+
 def oracle_attention(layer, q, khat, vhat, lens, tau=0.0):
     """q [B, Hq, d]; khat/vhat [B, Hkv, L, d] fp64."""
     return oatt.decode_attention(np.asarray(q, dtype=np.float64), khat, vhat, lens,

@@ -59,7 +59,8 @@ def _oracle_hat(layer, enc, which, shape):
 
 def _attention_case(layer, kx, vx, q, lens, tau=0.0):
     """Quantise on the GPU, check codes; attend on the GPU over (a) its own
-    cache and (b) the oracle's codes uploaded; both against the oracle."""
+    cache, against the oracle's attention on those stored codes, and (b) the
+    oracle's codes uploaded, against the oracle's attention on its codes."""
     bsz, t, hkv, d = kx.shape
     cache, st, word = H.gpu_quantize(layer, kx, vx, t)
     assert st == tq.TQ_OK and word == 0
@@ -67,11 +68,14 @@ def _attention_case(layer, kx, vx, q, lens, tau=0.0):
     khat = _oracle_hat(layer, enc[0], 0, (bsz, hkv, t, d))
     vhat = _oracle_hat(layer, enc[1], 1, (bsz, hkv, t, d))
     ref = H.oracle_attention(layer, _to_np(q), khat, vhat, lens, tau)
-    # (a) end to end
+    want = ref["out"] if tau == 0 else ref["exact_sparse"]
+    # (a) end to end, judged on the GPU's own stored codes (code parity passed above)
     got, st, word = H.gpu_decode(layer, q, cache, lens)
     assert st == tq.TQ_OK and word == 0
-    want = ref["out"] if tau == 0 else ref["exact_sparse"]
-    err_e2e = H.rel_l2_per_vector(got, want)
+    ks = np.stack([np.stack([H.stored_hat(layer, cache, b, h, t, 0) for h in range(hkv)]) for b in range(bsz)])
+    vs = np.stack([np.stack([H.stored_hat(layer, cache, b, h, t, 1) for h in range(hkv)]) for b in range(bsz)])
+    ref_e2e = H.oracle_attention(layer, _to_np(q), ks, vs, lens, tau)
+    err_e2e = H.rel_l2_per_vector(got, ref_e2e["out"] if tau == 0 else ref_e2e["exact_sparse"])
     # (b) on the oracle's own codes
     cache2 = tq.alloc_cache(layer.params, bsz, t)
     for b in range(bsz):
