@@ -301,11 +301,12 @@ def run_tq(args, world, rank, local):
 
     def enqueue_step(i, decode_only=False):
         for l in range(LAYERS):
-            if not decode_only:
-                tq.tq_quantize_append(params[l], kcb, vcb, k_new[l][:, i:i + 1], v_new[l][:, i:i + 1], positions[i],
-                                      caches[l], err, stream=stream)
-            tq.tq_decode_attention(params[l], kcb, vcb, qs[l][i], caches[l], lens[i], cap, outs[l], ws, err,
-                                   stream=stream)
+            if decode_only:
+                tq.tq_decode_attention(params[l], kcb, vcb, qs[l][i], caches[l], lens[i], cap, outs[l], ws, err,
+                                       stream=stream)
+            else:  # append the step's token and attend, one launch per layer
+                tq.tq_append_decode_attention(params[l], kcb, vcb, k_new[l][:, i:i + 1], v_new[l][:, i:i + 1],
+                                              qs[l][i], caches[l], lens[i], cap, outs[l], ws, err, stream=stream)
 
     # one CUDA graph per step (the pointers of step i are baked in)
     graphs = []
@@ -376,10 +377,8 @@ def run_tq(args, world, rank, local):
     with torch.cuda.stream(stream):
         with torch.cuda.graph(g_e2e, stream=stream):
             for l in range(LAYERS):
-                tq.tq_quantize_append(params[l], kcb, vcb, s_k[l], s_v[l], positions[last], caches[l], err,
-                                      stream=stream)
-                tq.tq_decode_attention(params[l], kcb, vcb, s_q[l], caches[l], lens[last], cap, outs[l], ws, err,
-                                       stream=stream)
+                tq.tq_append_decode_attention(params[l], kcb, vcb, s_k[l], s_v[l], s_q[l], caches[l], lens[last], cap,
+                                              outs[l], ws, err, stream=stream)
     torch.cuda.synchronize()
     h2d = sum(t.numel() * t.element_size() for t in h_k + h_v + h_q)
     d2h = h_out.numel() * h_out.element_size()
@@ -403,7 +402,7 @@ def run_tq(args, world, rank, local):
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
     e2e_value = world * LAYERS * BATCH * (last + CONTEXT + 1) * e2e_steps / (e2e_ms / 1000.0)
 
-    launches_per_step = LAYERS * 2  # quantise-append, decode attention (splits and merge fused)
+    launches_per_step = LAYERS  # one fused append + decode-attention kernel per layer
     if rank == 0:
         cpu_info = oracle_sample(seconds_target=12.0)[1] if (world == 1 and not args.no_cpu_baseline) else None
         line = {
@@ -414,12 +413,12 @@ def run_tq(args, world, rank, local):
                        "layers": LAYERS, "parallelism": "replicas%d" % world if world > 1 else "none",
                        "l2": "inputs larger than L2: 32 distinct layer caches, %.0f MB" %
                              (LAYERS * HKV * seq * bytes_per_token_head() / 1e6),
-                       "graphs": "one CUDA graph per step (32 x append + decode)"},
+                       "graphs": "one CUDA graph per step: 32 x tq_append_decode_attention (append + attend, one kernel per layer)"},
             "hbm_gbs": alg_bytes * LAYERS / (ms / steps * 1e-3) / 1e9,
             "pct_of_8tbs": 100.0 * alg_bytes * LAYERS / (ms / steps * 1e-3) / 8e12,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(seq), "peak_kind": peak_kind,
-                         "kernel": "tq_decode_attention (one fused kernel), %.2f us per launch, %d B algorithmic"
+                         "kernel": "decode kernel timed alone (tq_decode_attention, no append), %.2f us per launch, %d B algorithmic"
                                    % (decode_us, alg_bytes)},
             "cpu_baseline": cpu_info,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

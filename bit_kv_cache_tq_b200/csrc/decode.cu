@@ -292,18 +292,22 @@ static cudaError_t launch_decode_dim(const DecodeArgs& a, cudaStream_t stream) {
     return launch_decode_general<D, 16>(a, stream);
 }
 
+// k_new / v_new non-null: append mode (one new token per sequence at seq_len - 1).
 cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const tq_codebook* vcb, const tq_cache& c,
                               const void* q, int q_dtype, const int32_t* seq_lens, int max_len, float* out,
-                              const DecodePlan& plan, char* ws, uint32_t* err, int num_sms, cudaStream_t stream);
+                              const DecodePlan& plan, char* ws, uint32_t* err, int num_sms, cudaStream_t stream,
+                              const void* k_new = nullptr, const void* v_new = nullptr, int new_dtype = 0);
 
 }  // namespace tq
 
-extern "C" tq_status tq_decode_attention(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
-                                         const void* d_q, tq_dtype q_dtype, const tq_cache* cache,
-                                         const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
-                                         void* d_workspace, size_t workspace_bytes, uint32_t* d_error,
-                                         void* stream) {
-    using namespace tq;
+namespace tq {
+// Decode attention; with k_new / v_new set, the step's new token of every
+// sequence is first written at position seq_len - 1 (append mode).
+static tq_status decode_impl(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                             const void* d_q, tq_dtype q_dtype, const tq_cache* cache, const int32_t* d_seq_lens,
+                             int32_t max_seq_len, float* d_out, void* d_workspace, size_t workspace_bytes,
+                             uint32_t* d_error, void* stream, const void* k_new, const void* v_new,
+                             tq_dtype kv_dtype) {
     tq_status st = validate_params(params);
     if (st != TQ_OK) return st;
     const tq_params& p = *params;
@@ -313,6 +317,12 @@ extern "C" tq_status tq_decode_attention(const tq_params* params, const tq_codeb
     if (!aligned16(d_q) || !aligned16(d_out) || !aligned16(d_workspace)) return TQ_ERR_ALIGNMENT;
     if (p.k_mode == TQ_MODE_TURBO && (st = validate_codebook(kcb, p.head_dim, p.k_bits)) != TQ_OK) return st;
     if (p.v_mode == TQ_MODE_TURBO && (st = validate_codebook(vcb, p.head_dim, p.v_bits)) != TQ_OK) return st;
+    const bool append = k_new != nullptr;
+    if (append) {
+        if (!v_new) return TQ_ERR_INVALID_ARG;
+        if (kv_dtype != TQ_F32 && kv_dtype != TQ_BF16 && kv_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
+        if (!aligned16(k_new) || !aligned16(v_new)) return TQ_ERR_ALIGNMENT;
+    }
     const int sms = num_sms_current();
     if (sms <= 0) return TQ_ERR_CUDA;
     const DecodePlan plan = plan_decode(p, cache->batch, max_seq_len, sms, workspace_bytes);
@@ -321,9 +331,15 @@ extern "C" tq_status tq_decode_attention(const tq_params* params, const tq_codeb
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (decode_mma_supported(p)) {
         const cudaError_t e = launch_decode_mma(p, kcb, vcb, *cache, d_q, q_dtype, d_seq_lens, max_seq_len, d_out, plan,
-                                                static_cast<char*>(d_workspace), d_error, sms, s);
+                                                static_cast<char*>(d_workspace), d_error, sms, s, k_new, v_new,
+                                                kv_dtype);
         if (e != cudaErrorNotSupported) return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
         // otherwise (a device whose shared-memory window differs) take the general path
+    }
+    if (append) {  // two launches: append, then attend
+        st = quantize_append_impl(params, kcb, vcb, k_new, v_new, kv_dtype, 1, d_seq_lens, true, cache, d_error,
+                                  stream);
+        if (st != TQ_OK) return st;
     }
     DecodeArgs a{};
     fill_decode_side(a.k, p.k_mode, p.k_bits, p.head_dim, kcb, cache->k_codes, cache->k_norms);
@@ -358,6 +374,27 @@ extern "C" tq_status tq_decode_attention(const tq_params* params, const tq_codeb
         default: e = launch_decode_dim<256>(a, s); break;
     }
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+}  // namespace tq
+
+extern "C" tq_status tq_decode_attention(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                                         const void* d_q, tq_dtype q_dtype, const tq_cache* cache,
+                                         const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
+                                         void* d_workspace, size_t workspace_bytes, uint32_t* d_error,
+                                         void* stream) {
+    return tq::decode_impl(params, kcb, vcb, d_q, q_dtype, cache, d_seq_lens, max_seq_len, d_out, d_workspace,
+                           workspace_bytes, d_error, stream, nullptr, nullptr, TQ_BF16);
+}
+
+extern "C" tq_status tq_append_decode_attention(const tq_params* params, const tq_codebook* kcb,
+                                                const tq_codebook* vcb, const void* k_new, const void* v_new,
+                                                tq_dtype kv_dtype, const void* d_q, tq_dtype q_dtype,
+                                                const tq_cache* cache, const int32_t* d_seq_lens,
+                                                int32_t max_seq_len, float* d_out, void* d_workspace,
+                                                size_t workspace_bytes, uint32_t* d_error, void* stream) {
+    if (!k_new || !v_new) return TQ_ERR_INVALID_ARG;
+    return tq::decode_impl(params, kcb, vcb, d_q, q_dtype, cache, d_seq_lens, max_seq_len, d_out, d_workspace,
+                           workspace_bytes, d_error, stream, k_new, v_new, kv_dtype);
 }
 
 // ---------------------------------------------------------------------------

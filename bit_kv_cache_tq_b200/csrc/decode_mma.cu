@@ -66,7 +66,10 @@ constexpr uint32_t LUT_BYTES = 65536;        // 256 entries x 256 B
 // shared memory precedes it); the host checks it before choosing this kernel,
 // and table lookups carry it as an immediate offset.
 constexpr uint32_t WINDOW = 1024;
-constexpr uint32_t QSLOT_BYTES = 16 * D * 4; // one item's queries, up to 16 heads in fp32
+constexpr uint32_t Q_BYTES = 16 * D * 4;     // one item's queries, up to 16 heads in fp32
+constexpr uint32_t NEW_ROW = D * 4;           // one appended key or value row, up to fp32
+constexpr uint32_t QSLOT_BYTES = Q_BYTES + 2 * NEW_ROW;  // queries, then the new key and value rows
+constexpr uint32_t APP_BYTES = 1024;          // the appended token's codes and scratch
 constexpr long long WAIT_LIMIT = 2000000000ll;  // clock cycles (~1 s)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LAZY = 8.0f;                 // log2 headroom before the running max moves
@@ -100,13 +103,20 @@ struct Args {
     uint32_t signs[4];
     uint16_t kcent[16];  // fp16 bits of alpha_k * key centroid
     uint16_t vcent[16];  // fp16 bits of alpha_v * value centroid
+    // append mode: one new token per sequence, written at position seq_len - 1
+    int append, new_dtype, new_bytes;
+    const void* k_new;   // [batch][1][Hkv][d]
+    const void* v_new;
+    float kbound[8];     // positive decision boundaries, ascending (unused ones +inf)
+    float vbound[8];
+    float kc32[16];      // fp32 key centroids (QJL residual)
 };
 
 // Shared-memory map (byte offsets from the dynamic base).  A stage is
 // [header | K codes | V codes | K norms | V norms | QJL words | gammas].
 struct Layout {
     uint32_t ring, stage_bytes, k_off, v_off, kn_off, vn_off, z_off, gam_off;
-    uint32_t qring, qh, qlo, sq, fac, merge, ml, bars, flags, total;
+    uint32_t qring, qh, qlo, sq, app, fac, merge, ml, bars, flags, total;
 };
 
 __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int m) {
@@ -123,7 +133,8 @@ __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int
     L.qh = L.qring + 2 * QSLOT_BYTES;                  // fp16 [16][128], rounded q~
     L.qlo = L.qh + 16 * D * 2;                         // fp16 [16][128], q~ minus the rounded part
     L.sq = L.qlo + 16 * D * 2;                         // fp16 [16][64]
-    L.fac = L.sq + 16 * 64 * 2;                        // float F1[16], F2[16]
+    L.app = L.sq + 16 * 64 * 2;                        // appended token: packed rows, norms, scratch
+    L.fac = L.app + APP_BYTES;                         // float F1[16], F2[16]
     L.merge = L.fac + 32 * 4;                          // float [CW][8*nt][128]
     L.ml = L.merge + CW * 8 * nt * D * 4;              // float2 [CW][16]
     L.bars = L.ml + CW * 16 * 8;                       // u64 full[8], empty[8], qfull[2], qempty[2]
@@ -136,7 +147,7 @@ __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int
 __device__ __forceinline__ int tau_row(int r) { return (r & 8) + (r & 1) * 4 + ((r & 7) >> 1); }
 
 struct Item {
-    int unit, split, b, kv, s0, s1;
+    int unit, split, b, kv, s0, s1, len;
     bool bad;  // seq_len out of range: the sequence is treated as empty
 };
 
@@ -151,6 +162,7 @@ __device__ __forceinline__ Item item_of(const Args& a, int item) {
     if (it.bad) len = 0;
     it.s0 = it.split * a.split_len;
     it.s1 = min(len, it.s0 + a.split_len);
+    it.len = len;
     return it;
 }
 
@@ -197,11 +209,21 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
                 break;
             }
             const uint32_t qbytes = G * D * a.q_bytes;
-            ptx::mbar_arrive_expect_tx(qfull0 + 8 * qs, qbytes);
+            // the item holding a sequence's last token also brings the token's new key and value
+            const bool app = a.append && w.s1 == w.len;
+            const uint32_t rbytes = D * a.new_bytes;
+            ptx::mbar_arrive_expect_tx(qfull0 + 8 * qs, qbytes + (app ? 2 * rbytes : 0u));
             ptx::bulk_copy_g2s(base + L.qring + qs * QSLOT_BYTES,
                                static_cast<const uint8_t*>(a.q) +
                                    (static_cast<size_t>(w.b) * a.hq + w.kv * G) * D * a.q_bytes,
                                qbytes, qfull0 + 8 * qs);
+            if (app) {
+                const size_t row = (static_cast<size_t>(w.b) * a.hkv + w.kv) * rbytes;
+                ptx::bulk_copy_g2s(base + L.qring + qs * QSLOT_BYTES + Q_BYTES,
+                                   static_cast<const uint8_t*>(a.k_new) + row, rbytes, qfull0 + 8 * qs);
+                ptx::bulk_copy_g2s(base + L.qring + qs * QSLOT_BYTES + Q_BYTES + NEW_ROW,
+                                   static_cast<const uint8_t*>(a.v_new) + row, rbytes, qfull0 + 8 * qs);
+            }
             ++qseq;
         }
         int t0 = w.s0;
@@ -388,8 +410,118 @@ struct Consumer {
 
     // Rotated queries of the item (fp16 hi + lo pair, scaled to max |q~| = 1) and the scale
     // factors of the scores; false on abort.
-    __device__ bool prologue(int qseq, uint32_t (&bq)[NT][8][4], uint32_t (&bz)[NT][4][2], float (&f1)[NT][2],
-                             float (&f2)[NT][2]) {
+    // The appended token of the item's sequence (append mode): warp 0 encodes
+    // the new key, warp 1 the new value, from the rows staged beside the
+    // queries, exactly as the quantise-append kernel does (norm, rotation,
+    // codes, packing, and for keys the QJL sign sketch of the residual).  The
+    // result goes to the cache slot and to the patch area, from which the
+    // stage holding the token is updated before it is consumed.
+    template <int BITS, bool SKETCH>
+    __device__ void encode_new(const uint8_t* src, uint8_t* codes, uint16_t* norms, const float* bounds, size_t slot,
+                               uint8_t* prow, uint16_t* pnorm, uint8_t* cbytes, float* rbuf) {
+        float x[4];
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[e] = load_scalar(src, lane * 4 + e, a.new_dtype);
+            ss = fmaf(x[e], x[e], ss);
+            x[e] = flip_sign(x[e], sign_bit(a.signs, lane * 4 + e));
+        }
+        fwht_registers(x);
+        fwht_lanes<4, 32>(x, lane);
+        ss = group_sum<32>(ss);
+        const float n = sqrtf(ss);
+        const float inv = n > 0.0f ? 1.0f / (sqrtf(static_cast<float>(D)) * n) : 0.0f;
+        uint32_t code[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[e] *= inv;  // rotated unit-vector coordinate
+            code[e] = code_of<BITS>(x[e], bounds);
+            cbytes[lane * 4 + e] = static_cast<uint8_t>(code[e]);
+        }
+        __syncwarp();
+        if (lane < 4 * BITS) {  // word `lane` of the LSB-first bitstream
+            const int c0 = (32 * lane) / BITS, c1 = (32 * lane + 31) / BITS;
+            uint32_t word = 0;
+            for (int c = c0; c <= c1; ++c) {
+                const int sh = c * BITS - 32 * lane;
+                const uint32_t v = cbytes[c];
+                word |= sh >= 0 ? (v << sh) : (v >> -sh);
+            }
+            reinterpret_cast<uint32_t*>(codes + slot * (16 * BITS))[lane] = word;
+            reinterpret_cast<uint32_t*>(prow)[lane] = word;
+        }
+        if (lane == 0) {
+            const uint16_t n16 = float_to_half_bits(n);
+            norms[slot] = n16;
+            *pnorm = n16;
+        }
+        if constexpr (SKETCH) {
+            float g2 = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float r = x[e] - a.kc32[code[e]];
+                g2 = fmaf(r, r, g2);
+                rbuf[lane * 4 + e] = r;
+            }
+            g2 = group_sum<32>(g2);
+            __syncwarp();
+            float acc0 = 0.f, acc1 = 0.f;
+            if (lane < a.m) {
+                const float* srow = a.sketch + static_cast<size_t>(lane) * D;
+                for (int c = 0; c < D; ++c) acc0 = fmaf(__ldg(srow + c), rbuf[c], acc0);
+            }
+            if (lane + 32 < a.m) {
+                const float* srow = a.sketch + static_cast<size_t>(lane + 32) * D;
+                for (int c = 0; c < D; ++c) acc1 = fmaf(__ldg(srow + c), rbuf[c], acc1);
+            }
+            const uint32_t z0 = __ballot_sync(kFullMask, lane < a.m && acc0 >= 0.f);
+            const uint32_t z1 = __ballot_sync(kFullMask, lane + 32 < a.m && acc1 >= 0.f);
+            uint8_t* pz = smem + L.app + 136;
+            uint32_t* qjl = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.k_qjl) + slot * (a.m / 8));
+            if (lane == 0) {
+                const uint16_t g16 = float_to_half_bits(sqrtf(g2));
+                const_cast<uint16_t*>(a.k_gamma)[slot] = g16;
+                *reinterpret_cast<uint16_t*>(smem + L.app + 132) = g16;
+                qjl[0] = z0;
+                reinterpret_cast<uint32_t*>(pz)[0] = z0;
+                if (a.m > 32) {
+                    qjl[1] = z1;
+                    reinterpret_cast<uint32_t*>(pz)[1] = z1;
+                }
+            }
+        }
+    }
+
+    // Copy the appended token from the patch area into the stage that holds it
+    // (chunk-local index p); warps 0 (key side) and 1 (value side).
+    __device__ void patch_stage(uint8_t* st, int p) {
+        const uint8_t* ap = smem + L.app;
+        if (warp == 0) {
+            if (lane < 4 * KB)
+                reinterpret_cast<uint32_t*>(st + L.k_off + p * (16 * KB))[lane] = reinterpret_cast<const uint32_t*>(ap)[lane];
+            if (a.staged_norms && lane == 0) {
+                reinterpret_cast<uint16_t*>(st + L.kn_off)[p] = *reinterpret_cast<const uint16_t*>(ap + 128);
+                if constexpr (QJL) {
+                    reinterpret_cast<uint16_t*>(st + L.gam_off)[p] = *reinterpret_cast<const uint16_t*>(ap + 132);
+                    const int zb = a.m / 8;
+                    for (int i = 0; i < zb / 4; ++i)
+                        reinterpret_cast<uint32_t*>(st + L.z_off + p * zb)[i] = reinterpret_cast<const uint32_t*>(ap + 136)[i];
+                }
+            }
+        } else if (warp == 1) {
+            if (lane < 4 * VB)
+                reinterpret_cast<uint32_t*>(st + L.v_off + p * (16 * VB))[lane] =
+                    reinterpret_cast<const uint32_t*>(ap + 64)[lane];
+            if (a.staged_norms && lane == 0)
+                reinterpret_cast<uint16_t*>(st + L.vn_off)[p] = *reinterpret_cast<const uint16_t*>(ap + 130);
+        }
+        // the stage is refilled later by the copy engine: order these writes first
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+
+    __device__ bool prologue(int qseq, const Item& w, bool app, uint32_t (&bq)[NT][8][4], uint32_t (&bz)[NT][4][2],
+                             float (&f1)[NT][2], float (&f2)[NT][2]) {
         const uint32_t qfull = base + L.bars + 128 + 8 * (qseq & 1);
         if (!ptx::mbar_wait_bounded(qfull, (qseq >> 1) & 1, WAIT_LIMIT)) set_abort();
         ptx::named_barrier(1, NUM_CONSUMERS);
@@ -454,6 +586,19 @@ struct Consumer {
                 fac[h] = h < G ? a.sm_scale_log2 * qmax * a.inv_alpha_k : 0.f;
                 fac[16 + h] = (QJL && h < G) ? a.sm_scale_log2 * 1.2533141373155003f / a.m * smax : 0.f;
             }
+        }
+        if (app && warp < 2) {
+            const size_t slot = static_cast<size_t>(w.unit) * a.capacity + (w.len - 1);
+            const uint8_t* rows = smem + L.qring + (qseq & 1) * QSLOT_BYTES + Q_BYTES;
+            uint8_t* ap = smem + L.app;
+            if (warp == 0)
+                encode_new<KB, QJL>(rows, const_cast<uint8_t*>(a.k_codes), const_cast<uint16_t*>(a.k_norms), a.kbound,
+                                    slot, ap, reinterpret_cast<uint16_t*>(ap + 128), ap + 256,
+                                    reinterpret_cast<float*>(ap + 512));
+            else
+                encode_new<VB, false>(rows + NEW_ROW, const_cast<uint8_t*>(a.v_codes), const_cast<uint16_t*>(a.v_norms),
+                                      a.vbound, slot, ap + 64, reinterpret_cast<uint16_t*>(ap + 130), ap + 384,
+                                      reinterpret_cast<float*>(ap + 512));
         }
         ptx::named_barrier(1, NUM_CONSUMERS);
         if (tid == 0) ptx::mbar_arrive(base + L.bars + 144 + 8 * (qseq & 1));  // query slot free
@@ -828,7 +973,7 @@ struct Consumer {
         S.reset();
         Item w{};
         int seq = 0, qseq = 0;
-        bool done_ok = false;
+        bool done_ok = false, app = false;
         while (true) {
             const int slot = seq % a.stages, use = seq / a.stages;
             if (!ptx::mbar_wait_bounded(full0 + 8 * slot, use & 1, WAIT_LIMIT)) set_abort();
@@ -845,10 +990,15 @@ struct Consumer {
                 w = item_of(a, hdr.x);
                 if (w.bad && a.err && w.split == 0 && w.kv == 0 && tid == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
                 S.reset();
+                app = a.append && !empty && w.s1 == w.len;
                 if (!empty) {
-                    if (!prologue(qseq, bq, bz, f1, f2)) break;
+                    if (!prologue(qseq, w, app, bq, bz, f1, f2)) break;
                     ++qseq;
                 }
+            }
+            if (app && (hdr.w & F_LAST)) {  // the stage holding the appended token
+                patch_stage(const_cast<uint8_t*>(st), w.len - 1 - hdr.y);
+                ptx::named_barrier(1, NUM_CONSUMERS);
             }
             if (!empty) {
                 if (hdr.w & F_LAST) chunk<true>(w, st, hdr.y, bq, bz, f1, f2, S);
@@ -983,9 +1133,23 @@ static uint16_t half_bits(double v) {
 
 cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const tq_codebook* vcb, const tq_cache& c,
                               const void* q, int q_dtype, const int32_t* seq_lens, int max_len, float* out,
-                              const DecodePlan& plan, char* ws, uint32_t* err, int num_sms, cudaStream_t stream) {
+                              const DecodePlan& plan, char* ws, uint32_t* err, int num_sms, cudaStream_t stream,
+                              const void* k_new, const void* v_new, int new_dtype) {
     using namespace mmadec;
     Args a{};
+    a.append = k_new != nullptr;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.new_dtype = new_dtype;
+    a.new_bytes = new_dtype == TQ_F32 ? 4 : 2;
+    {
+        const int hk = 1 << (p.k_bits - 1), hv = 1 << (p.v_bits - 1);
+        for (int k = 0; k < 8; ++k) {
+            a.kbound[k] = k < hk - 1 ? static_cast<float>(kcb->boundaries[hk + k]) : INFINITY;
+            a.vbound[k] = k < hv - 1 ? static_cast<float>(vcb->boundaries[hv + k]) : INFINITY;
+        }
+        for (int j = 0; j < 16; ++j) a.kc32[j] = j < (1 << p.k_bits) ? static_cast<float>(kcb->centroids[j]) : 0.f;
+    }
     a.k_codes = c.k_codes;
     a.v_codes = c.v_codes;
     a.k_norms = c.k_norms;

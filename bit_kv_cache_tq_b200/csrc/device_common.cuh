@@ -103,6 +103,21 @@ __device__ __forceinline__ float group_max(float x) {
     return x;
 }
 
+// Code of a rotated unit coordinate y: the number of boundaries below it.
+// With an odd-symmetric table the middle boundary is 0, so the count is
+// 2^(b-1) + #{t_k > 0 : |y| > t_k} for y > 0 and 2^(b-1) - 1 - #{...} otherwise
+// (an exact tie |y| == t_k on the negative side lands one cell high, inside
+// the boundary window the codes are compared with).
+template <int BITS>
+__device__ __forceinline__ uint32_t code_of(float y, const float* tpos) {
+    constexpr int half = 1 << (BITS - 1);
+    const float a = fabsf(y);
+    int m = 0;
+#pragma unroll
+    for (int k = 0; k < half - 1; ++k) m += a > tpos[k];
+    return y > 0.0f ? static_cast<uint32_t>(half + m) : static_cast<uint32_t>(half - 1 - m);
+}
+
 // `nbits` (<= 32) bits of a packed little-endian bitstream starting at bit
 // `bitoff`; `words` is the stream as 32-bit words and `nwords` its length
 // (never read past).

@@ -52,6 +52,12 @@ bool decode_mma_supported(const tq_params& p);
 int num_sms_current();
 // Centroid scale in [8, 16) minimising the largest relative fp16 rounding error.
 double best_fp16_scale(const double* c, int n);
+// tq_quantize_append; with pos_from_lens, d_positions holds each sequence's
+// length after the append and the new tokens go to its last n_new slots.
+tq_status quantize_append_impl(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                               const void* k_new, const void* v_new, int dtype, int32_t n_new,
+                               const int32_t* d_positions, bool pos_from_lens, const tq_cache* cache,
+                               uint32_t* d_error, void* stream);
 // Rotation signs as a bit mask: bit i set <=> s_i = -1.
 void rotation_sign_bits(uint64_t seed, int head_dim, uint32_t words[8]);
 

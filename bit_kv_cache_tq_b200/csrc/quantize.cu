@@ -43,26 +43,11 @@ struct QuantSide {
 
 struct QuantArgs {
     QuantSide side[2];  // 0 = K, 1 = V
-    const int32_t* positions;
+    const int32_t* positions;  // per sequence: first slot written, or (pos_from_lens) the length after the append
     uint32_t* err;
-    int batch, n_new, hkv, capacity;
+    int batch, n_new, hkv, capacity, pos_from_lens;
     uint32_t signs[8];
 };
-
-// Code of a rotated unit coordinate y: the number of boundaries below it.
-// With an odd-symmetric table the middle boundary is 0, so the count is
-// 2^(b-1) + #{t_k > 0 : |y| > t_k} for y > 0 and 2^(b-1) - 1 - #{...} otherwise
-// (an exact tie |y| == t_k on the negative side lands one cell high, inside
-// the boundary window the codes are compared with).
-template <int BITS>
-__device__ __forceinline__ uint32_t code_of(float y, const float* tpos) {
-    constexpr int half = 1 << (BITS - 1);
-    const float a = fabsf(y);
-    int m = 0;
-#pragma unroll
-    for (int k = 0; k < half - 1; ++k) m += a > tpos[k];
-    return y > 0.0f ? static_cast<uint32_t>(half + m) : static_cast<uint32_t>(half - 1 - m);
-}
 
 template <int BITS>
 __device__ __forceinline__ void store_chunk_codes(uint8_t* row, int chunk, uint32_t packed) {
@@ -193,7 +178,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
             const long long bt = v / a.hkv;
             const int t = static_cast<int>(bt % a.n_new);
             const int b = static_cast<int>(bt / a.n_new);
-            const int pos = a.positions[b];
+            const int pos = a.positions[b] - (a.pos_from_lens ? a.n_new : 0);
             if (pos < 0 || pos > a.capacity - a.n_new) {
                 if (a.err && t == 0 && h == 0 && sub == 0 && blockIdx.y == 0) atomicOr(a.err, TQ_DEVERR_POSITION);
                 valid = false;
@@ -369,6 +354,16 @@ tq_status tq_quantize_append(const tq_params* params, const tq_codebook* kcb, co
                              const void* k_new, const void* v_new, tq_dtype dtype, int32_t n_new,
                              const int32_t* d_positions, const tq_cache* cache, uint32_t* d_error,
                              void* stream) {
+    return tq::quantize_append_impl(params, kcb, vcb, k_new, v_new, dtype, n_new, d_positions, false, cache, d_error,
+                                    stream);
+}
+
+}  // extern "C"
+
+tq_status tq::quantize_append_impl(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                                   const void* k_new, const void* v_new, int dtype, int32_t n_new,
+                                   const int32_t* d_positions, bool pos_from_lens, const tq_cache* cache,
+                                   uint32_t* d_error, void* stream) {
     using namespace tq;
     tq_status st = validate_params(params);
     if (st != TQ_OK) return st;
@@ -395,6 +390,7 @@ tq_status tq_quantize_append(const tq_params* params, const tq_codebook* kcb, co
     a.side[1].norms = cache->v_norms;
     a.side[1].m = 0;
     a.positions = d_positions;
+    a.pos_from_lens = pos_from_lens ? 1 : 0;
     a.err = d_error;
     a.batch = cache->batch;
     a.n_new = n_new;
@@ -410,6 +406,8 @@ tq_status tq_quantize_append(const tq_params* params, const tq_codebook* kcb, co
     }
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
+
+extern "C" {
 
 tq_status tq_dequantize(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
                         const tq_cache* cache, int32_t b, int32_t start, int32_t count, float* d_k_out,

@@ -29,7 +29,7 @@ TQ_DEVERR_POSITION, TQ_DEVERR_SEQLEN = 0x1, 0x2
 EXPORTED = (
     "tq_status_string", "tq_abi_version", "tq_codebook_init", "tq_rotation_signs", "tq_qjl_matrix",
     "tq_cache_bytes", "tq_decode_workspace_bytes", "tq_quantize_append", "tq_dequantize",
-    "tq_decode_attention", "tq_decode_attention_static", "tq_read_device_error",
+    "tq_decode_attention", "tq_append_decode_attention", "tq_decode_attention_static", "tq_read_device_error",
 )
 
 # Bytes of the library's own decode scratch per device (tq_decode_attention_static).
@@ -82,6 +82,10 @@ _lib.tq_dequantize.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), 
 _lib.tq_decode_attention.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p, ctypes.c_int,
                                      _P(tq_cache), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+_lib.tq_append_decode_attention.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
+                                            _P(tq_cache), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
 _lib.tq_decode_attention_static.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
                                             ctypes.c_int, _P(tq_cache), ctypes.c_void_p, ctypes.c_int32,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
@@ -248,6 +252,20 @@ def tq_decode_attention(params, kcb, vcb, q, cache, seq_lens, max_seq_len, out, 
                                   _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(error),
                                   _stream(stream))
     _check(st, "tq_decode_attention")
+
+
+def tq_append_decode_attention(params, kcb, vcb, k_new, v_new, q, cache, seq_lens, max_seq_len, out, workspace,
+                               error=None, stream=None):
+    """Append k_new/v_new ([batch, 1, Hkv, d]) at slot seq_lens-1, then decode attention over seq_lens tokens."""
+    assert q.is_contiguous() and out.is_contiguous() and out.dtype == torch.float32
+    assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.dtype == v_new.dtype
+    assert seq_lens.dtype == torch.int32 and seq_lens.is_cuda
+    c = cache.struct()
+    st = _lib.tq_append_decode_attention(ctypes.byref(params), kcb and ctypes.byref(kcb), vcb and ctypes.byref(vcb),
+                                         _ptr(k_new), _ptr(v_new), _dtype_code(k_new), _ptr(q), _dtype_code(q), ctypes.byref(c),
+                                         _ptr(seq_lens), max_seq_len, _ptr(out), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _ptr(error), _stream(stream))
+    _check(st, "tq_append_decode_attention")
 
 
 def tq_decode_attention_static(params, kcb, vcb, q, cache, seq_lens, max_seq_len, out, error=None, stream=None):

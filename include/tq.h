@@ -273,6 +273,31 @@ tq_status tq_decode_attention(const tq_params* params, const tq_codebook* kcb, c
                               const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
                               void* d_workspace, size_t workspace_bytes, uint32_t* d_error, void* stream);
 
+/*
+ * One decode step of a layer in one call: append the step's new token of
+ * every sequence to the cache, then tq_decode_attention over the cache that
+ * includes it ([tqai] "TurboQuant的核心创新" for the encoding, [google]
+ * "再看速度" for the attention; the pages run the two one after the other).
+ *   k_new, v_new  device, [batch][1][Hkv][d] in kv_dtype, 16-byte aligned.
+ *   d_seq_lens    lengths AFTER the append: sequence b's new token goes to
+ *                 slot seq_lens[b] - 1 and attention covers seq_lens[b]
+ *                 tokens.
+ *   Other arguments as for tq_decode_attention (same workspace rules).
+ * The new token is encoded exactly as tq_quantize_append encodes it (the
+ * cache afterwards holds what tq_quantize_append would have written, up to
+ * codes within the boundary window).  On the tensor-core path (d = 128,
+ * turbo K and V) this is one kernel: the block that owns a sequence's last
+ * token split encodes the token while the cache streams in.  Other
+ * configurations run tq_quantize_append's kernel and then the attention
+ * kernels.  A seq_len outside [1, capacity] skips that sequence's append and
+ * sets TQ_DEVERR_SEQLEN (or TQ_DEVERR_POSITION on the two-kernel path).
+ */
+tq_status tq_append_decode_attention(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                                     const void* k_new, const void* v_new, tq_dtype kv_dtype, const void* d_q,
+                                     tq_dtype q_dtype, const tq_cache* cache, const int32_t* d_seq_lens,
+                                     int32_t max_seq_len, float* d_out, void* d_workspace, size_t workspace_bytes,
+                                     uint32_t* d_error, void* stream);
+
 /* Bytes of the library's own decode scratch on each device. */
 #define TQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
 

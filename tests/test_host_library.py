@@ -191,3 +191,17 @@ def test_entry_points_reject_bad_arguments_before_launch():
     # error-word reader
     word = ctypes.c_uint32()
     assert lib.tq_read_device_error(None, ctypes.byref(word), None, 10) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_append_decode_rejects_bad_arguments_before_launch():
+    lib = tq.library()
+    p = tq.make_params(128, 32, 8)
+    kcb, vcb = tq.tq_codebook_init(128, 4), tq.tq_codebook_init(128, 2)
+    fake = 1 << 20
+    cache = tq.tq_cache(1, 64, fake, fake, None, None, fake, fake, None)
+    args = (ctypes.byref(p), ctypes.byref(kcb), ctypes.byref(vcb))
+    tail = (fake, tq.TQ_BF16, ctypes.byref(cache), fake, 64, fake, fake, 1 << 20, None, None)
+    assert lib.tq_append_decode_attention(*args, None, fake, tq.TQ_BF16, *tail) == tq.TQ_ERR_INVALID_ARG
+    assert lib.tq_append_decode_attention(*args, fake, None, tq.TQ_BF16, *tail) == tq.TQ_ERR_INVALID_ARG
+    assert lib.tq_append_decode_attention(*args, fake + 4, fake, tq.TQ_BF16, *tail) == tq.TQ_ERR_ALIGNMENT
+    assert lib.tq_append_decode_attention(*args, fake, fake, 7, *tail) == tq.TQ_ERR_INVALID_ARG
