@@ -68,15 +68,16 @@ constexpr uint32_t LUT_BYTES = 65536;        // 256 entries x 256 B
 constexpr uint32_t WINDOW = 1024;
 constexpr uint32_t Q_BYTES = 16 * D * 4;     // one item's queries, up to 16 heads in fp32
 constexpr uint32_t NEW_ROW = D * 4;           // one appended key or value row, up to fp32
-constexpr uint32_t QSLOT_BYTES = Q_BYTES + 2 * NEW_ROW;  // queries, then the new key and value rows
+constexpr uint32_t QHDR = 32;                 // item header at the front of a query slot
+constexpr uint32_t QSLOT_BYTES = QHDR + Q_BYTES + 2 * NEW_ROW;  // header, queries, new key and value rows
 constexpr uint32_t APP_BYTES = 1024;          // the appended token's codes and scratch
 constexpr long long WAIT_LIMIT = 2000000000ll;  // clock cycles (~1 s)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LAZY = 8.0f;                 // log2 headroom before the running max moves
 constexpr float VRANGE = 64.0f;              // bound on ||v|| * vscale
 
-// stage header flags
-constexpr int F_FIRST = 1, F_LAST = 2, F_EMPTY = 4, F_END = 8;
+// header flags: item (query slot) EMPTY / END / APPEND, chunk (stage) LAST
+constexpr int F_LAST = 2, F_EMPTY = 4, F_END = 8, F_APPEND = 16;
 // global counters after the per-(sequence, kv head) split counters
 constexpr int C_ITEM = 0, C_DONE = 1;
 
@@ -189,6 +190,13 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
             fail();
             return false;
         }
+        // Every block asks for its first stage at the same moment; the other
+        // stages follow once it has landed, so first bytes do not queue behind
+        // the whole grid's prefetch.
+        if (seq == 1 && !ptx::mbar_wait_bounded(full0, 0, WAIT_LIMIT)) {
+            fail();
+            return false;
+        }
         if (*abort_flag) {
             ok = false;
             return false;
@@ -197,49 +205,65 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         st = smem + L.ring + slot * L.stage_bytes;
         return true;
     };
+    // Every item starts with a header in the next query slot (the queries and,
+    // for a sequence's last split in append mode, the new key and value rows
+    // follow it), so consumers can prepare the item while its chunks fly.
+    // Empty items take a query slot but no stage.
+    auto claim_q = [&](uint8_t*& slot, uint32_t& qfull) -> bool {
+        const int qs = qseq & 1;
+        if (qseq >= 2 && !ptx::mbar_wait_bounded(qempty0 + 8 * qs, ((qseq - 2) >> 1) & 1, WAIT_LIMIT)) {
+            fail();
+            return false;
+        }
+        if (*abort_flag) {
+            ok = false;
+            return false;
+        }
+        slot = smem + L.qring + qs * QSLOT_BYTES;
+        qfull = qfull0 + 8 * qs;
+        ++qseq;
+        return true;
+    };
     int i = blockIdx.x;  // the first item of every block is static; later ones come from the counter
     while (ok) {
         if (i >= a.n_items) break;
         const Item w = item_of(a, i);
+        if (w.bad && a.err && w.split == 0 && w.kv == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
         const bool empty = w.s0 >= w.s1;
-        if (!empty) {  // the item's queries, into the next query slot
-            const int qs = qseq & 1;
-            if (qseq >= 2 && !ptx::mbar_wait_bounded(qempty0 + 8 * qs, ((qseq - 2) >> 1) & 1, WAIT_LIMIT)) {
-                fail();
-                break;
-            }
+        const bool app = a.append && !empty && w.s1 == w.len;
+        uint8_t* qslot;
+        uint32_t qfull;
+        if (!claim_q(qslot, qfull)) break;
+        int4* hdr = reinterpret_cast<int4*>(qslot);
+        hdr[0] = make_int4(i, w.s0, w.s1, w.len);
+        hdr[1] = make_int4((empty ? F_EMPTY : 0) | (app ? F_APPEND : 0), w.unit, w.b, w.kv);
+        if (empty) {
+            ptx::mbar_arrive_expect_tx(qfull, 0);
+        } else {
             const uint32_t qbytes = G * D * a.q_bytes;
-            // the item holding a sequence's last token also brings the token's new key and value
-            const bool app = a.append && w.s1 == w.len;
             const uint32_t rbytes = D * a.new_bytes;
-            ptx::mbar_arrive_expect_tx(qfull0 + 8 * qs, qbytes + (app ? 2 * rbytes : 0u));
-            ptx::bulk_copy_g2s(base + L.qring + qs * QSLOT_BYTES,
+            const uint32_t qdst = ptx::smem_addr(qslot) + QHDR;
+            ptx::mbar_arrive_expect_tx(qfull, qbytes + (app ? 2 * rbytes : 0u));
+            ptx::bulk_copy_g2s(qdst,
                                static_cast<const uint8_t*>(a.q) +
                                    (static_cast<size_t>(w.b) * a.hq + w.kv * G) * D * a.q_bytes,
-                               qbytes, qfull0 + 8 * qs);
+                               qbytes, qfull);
             if (app) {
                 const size_t row = (static_cast<size_t>(w.b) * a.hkv + w.kv) * rbytes;
-                ptx::bulk_copy_g2s(base + L.qring + qs * QSLOT_BYTES + Q_BYTES,
-                                   static_cast<const uint8_t*>(a.k_new) + row, rbytes, qfull0 + 8 * qs);
-                ptx::bulk_copy_g2s(base + L.qring + qs * QSLOT_BYTES + Q_BYTES + NEW_ROW,
-                                   static_cast<const uint8_t*>(a.v_new) + row, rbytes, qfull0 + 8 * qs);
+                ptx::bulk_copy_g2s(qdst + Q_BYTES, static_cast<const uint8_t*>(a.k_new) + row, rbytes, qfull);
+                ptx::bulk_copy_g2s(qdst + Q_BYTES + NEW_ROW, static_cast<const uint8_t*>(a.v_new) + row, rbytes,
+                                   qfull);
             }
-            ++qseq;
         }
-        int t0 = w.s0;
-        do {
+        for (int t0 = w.s0; t0 < w.s1; t0 += CHUNK) {
             uint32_t full;
             uint8_t* st;
             if (!claim(full, st)) break;
-            const int n = empty ? 0 : min(CHUNK, w.s1 - t0);
-            const int flags = (t0 == w.s0 ? F_FIRST : 0) | ((empty || t0 + CHUNK >= w.s1) ? F_LAST : 0) |
-                              (empty ? F_EMPTY : 0);
-            *reinterpret_cast<int4*>(st) = make_int4(i, t0, n, flags);
+            const int n = min(CHUNK, w.s1 - t0);
+            *reinterpret_cast<int4*>(st) = make_int4(i, t0, n, t0 + CHUNK >= w.s1 ? F_LAST : 0);
             const uint32_t dst = ptx::smem_addr(st);
             const size_t row = static_cast<size_t>(w.unit) * a.capacity + t0;
-            if (n == 0) {
-                ptx::mbar_arrive_expect_tx(full, 0);
-            } else if (a.staged_norms) {
+            if (a.staged_norms) {
                 // capacity and t0 are multiples of 8, so rounding n up to 8 tokens
                 // stays inside the cache and keeps every 2-byte array 16-byte sized
                 const int n8 = (n + 7) & ~7;
@@ -258,17 +282,16 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
                 ptx::bulk_copy_g2s(dst + L.v_off, a.v_codes + row * VBV, n * VBV, full);
             }
             ++seq;
-            t0 += CHUNK;
-        } while (!empty && t0 < w.s1);
+        }
+        if (!ok) break;
         i = static_cast<int>(gridDim.x + atomicAdd(a.counters + a.units + C_ITEM, 1u));
     }
-    if (ok) {  // end-of-work sentinel
-        uint32_t full;
-        uint8_t* st;
-        if (claim(full, st)) {
-            *reinterpret_cast<int4*>(st) = make_int4(-1, 0, 0, F_END);
-            ptx::mbar_arrive_expect_tx(full, 0);
-            ++seq;
+    if (ok) {  // end-of-work sentinel, in the next query slot
+        uint8_t* qslot;
+        uint32_t qfull;
+        if (claim_q(qslot, qfull)) {
+            reinterpret_cast<int4*>(qslot)[1] = make_int4(F_END, 0, 0, 0);
+            ptx::mbar_arrive_expect_tx(qfull, 0);
         }
     }
     // every copy issued must have landed before the block may exit
@@ -390,7 +413,7 @@ struct Consumer {
     uint8_t* smem;
     const Layout& L;
     int tid, warp, lane, g, t;
-    uint32_t base, laneoff;
+    uint32_t base, laneoff, sgn4;
 
     __device__ Consumer(const Args& a_, uint8_t* s_, const Layout& L_) : a(a_), smem(s_), L(L_) {
         tid = threadIdx.x;
@@ -400,6 +423,12 @@ struct Consumer {
         t = lane & 3;
         base = ptx::smem_addr(smem);
         laneoff = lane * 4;
+        // rotation signs of coordinates 4 lane .. 4 lane + 3 (word lane / 8),
+        // read with constant indices: a per-lane index into the parameters
+        // would serialise
+        const int wsel = lane >> 3;
+        const uint32_t sw = wsel == 0 ? a.signs[0] : wsel == 1 ? a.signs[1] : wsel == 2 ? a.signs[2] : a.signs[3];
+        sgn4 = (sw >> (4 * (lane & 7))) & 0xFu;
     }
 
     __device__ bool aborted() const { return *reinterpret_cast<volatile int*>(smem + L.flags) != 0; }
@@ -425,7 +454,7 @@ struct Consumer {
         for (int e = 0; e < 4; ++e) {
             x[e] = load_scalar(src, lane * 4 + e, a.new_dtype);
             ss = fmaf(x[e], x[e], ss);
-            x[e] = flip_sign(x[e], sign_bit(a.signs, lane * 4 + e));
+            x[e] = flip_sign(x[e], (sgn4 >> e) & 1u);
         }
         fwht_registers(x);
         fwht_lanes<4, 32>(x, lane);
@@ -520,14 +549,11 @@ struct Consumer {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
 
-    __device__ bool prologue(int qseq, const Item& w, bool app, uint32_t (&bq)[NT][8][4], uint32_t (&bz)[NT][4][2],
+    // The item's queries are in query slot `qseq` (already waited for).
+    __device__ void prologue(int qseq, const Item& w, bool app, uint32_t (&bq)[NT][8][4], uint32_t (&bz)[NT][4][2],
                              float (&f1)[NT][2], float (&f2)[NT][2]) {
-        const uint32_t qfull = base + L.bars + 128 + 8 * (qseq & 1);
-        if (!ptx::mbar_wait_bounded(qfull, (qseq >> 1) & 1, WAIT_LIMIT)) set_abort();
-        ptx::named_barrier(1, NUM_CONSUMERS);
-        if (aborted()) return false;
         const int G = a.group;
-        const uint8_t* qsrc = smem + L.qring + (qseq & 1) * QSLOT_BYTES;
+        const uint8_t* qsrc = smem + L.qring + (qseq & 1) * QSLOT_BYTES + QHDR;
         __half* qh = reinterpret_cast<__half*>(smem + L.qh);
         __half* ql = reinterpret_cast<__half*>(smem + L.qlo);
         __half* sq = reinterpret_cast<__half*>(smem + L.sq);
@@ -539,7 +565,7 @@ struct Consumer {
             if (h < G) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    x[e] = flip_sign(load_scalar(qsrc, h * D + lane * 4 + e, a.q_dtype), sign_bit(a.signs, lane * 4 + e));
+                    x[e] = flip_sign(load_scalar(qsrc, h * D + lane * 4 + e, a.q_dtype), (sgn4 >> e) & 1u);
                 fwht_registers(x);
                 fwht_lanes<4, 32>(x, lane);
 #pragma unroll
@@ -548,10 +574,11 @@ struct Consumer {
             float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
             amax = group_max<32>(amax);
             const float qmax = amax > 0.f ? amax : 1.f;
+            const float rq = 1.0f / qmax;  // F1 undoes the scale (to one fp32 ulp)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 // two fp16 terms: the scores keep about 22 bits of q~
-                const float u = x[e] / qmax;
+                const float u = x[e] * rq;
                 const __half hi = __float2half_rn(u);
                 qh[h * D + lane * 4 + e] = hi;
                 ql[h * D + lane * 4 + e] = __float2half_rn(u - __half2float(hi));
@@ -589,7 +616,7 @@ struct Consumer {
         }
         if (app && warp < 2) {
             const size_t slot = static_cast<size_t>(w.unit) * a.capacity + (w.len - 1);
-            const uint8_t* rows = smem + L.qring + (qseq & 1) * QSLOT_BYTES + Q_BYTES;
+            const uint8_t* rows = smem + L.qring + (qseq & 1) * QSLOT_BYTES + QHDR + Q_BYTES;
             uint8_t* ap = smem + L.app;
             if (warp == 0)
                 encode_new<KB, QJL>(rows, const_cast<uint8_t*>(a.k_codes), const_cast<uint16_t*>(a.k_norms), a.kbound,
@@ -600,18 +627,19 @@ struct Consumer {
                                       a.vbound, slot, ap + 64, reinterpret_cast<uint16_t*>(ap + 130), ap + 384,
                                       reinterpret_cast<float*>(ap + 512));
         }
-        ptx::named_barrier(1, NUM_CONSUMERS);
-        if (tid == 0) ptx::mbar_arrive(base + L.bars + 144 + 8 * (qseq & 1));  // query slot free
+        ptx::named_barrier(1, NUM_CONSUMERS);  // every warp is done with the query slot
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const __half* qrow = qh + (nt * 8 + g) * D + 32 * t;
             const __half* lrow = ql + (nt * 8 + g) * D + 32 * t;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                bq[nt][j][0] = *reinterpret_cast<const uint32_t*>(qrow + 4 * j);
-                bq[nt][j][1] = *reinterpret_cast<const uint32_t*>(qrow + 4 * j + 2);
-                bq[nt][j][2] = *reinterpret_cast<const uint32_t*>(lrow + 4 * j);
-                bq[nt][j][3] = *reinterpret_cast<const uint32_t*>(lrow + 4 * j + 2);
+                const uint2 hv = *reinterpret_cast<const uint2*>(qrow + 4 * j);
+                const uint2 lv = *reinterpret_cast<const uint2*>(lrow + 4 * j);
+                bq[nt][j][0] = hv.x;
+                bq[nt][j][1] = hv.y;
+                bq[nt][j][2] = lv.x;
+                bq[nt][j][3] = lv.y;
             }
             if constexpr (QJL) {
                 const __half* srow = sq + (nt * 8 + g) * 64 + 16 * t;
@@ -626,7 +654,6 @@ struct Consumer {
             f2[nt][0] = fac[16 + nt * 8 + 2 * t];
             f2[nt][1] = fac[16 + nt * 8 + 2 * t + 1];
         }
-        return true;
     }
 
     // One chunk: this warp's two tiles.  MASK: the chunk may end before CHUNK tokens.
@@ -891,26 +918,30 @@ struct Consumer {
             a.ws_acc[(pbase + h) * D + c] = s * a.inv_alpha_v;  // undo the centroid scale
             if (c == 0) a.ws_ml[pbase + h] = make_float2(mx, l);
         }
-        __threadfence();
+        // publish the partial: the barrier orders every thread's writes before
+        // thread 0's release, and its acquire orders the merge's reads after
+        // the other blocks' partials
         ptx::named_barrier(1, NUM_CONSUMERS);
-        if (tid == 0) *last_flag = atomicAdd(a.counters + w.unit, 1u) == static_cast<uint32_t>(a.n_split - 1);
+        if (tid == 0) *last_flag = ptx::atom_add_acq_rel_gpu(a.counters + w.unit, 1u) ==
+                                   static_cast<uint32_t>(a.n_split - 1);
         ptx::named_barrier(1, NUM_CONSUMERS);
         if (*last_flag) {
-            __threadfence();
-            // Merge the splits: one warp per head, lane = float4 column.  The
-            // first batch of partial rows is requested before the split weights
-            // 2^(m_s - M) / L are reduced, so both reads overlap; the weighted sum
-            // runs in split order, so the result does not depend on timing.
-            float* o_s = merge;           // [G][D]
-            float* wts = merge + 16 * D;  // [n_split][G]
+            // Merge the splits: two warps per head, each lane two channels.  A
+            // warp's first batch of partial rows is requested before its split
+            // weights 2^(m_s - M) are formed (its own row of shared memory), so
+            // both reads overlap; the weighted sum runs in split order, so the
+            // result does not depend on timing.
+            float* o_s = merge;  // [G][D]
             const size_t ubase = static_cast<size_t>(w.unit) * a.n_split * G;
-            const float4* src4 = reinterpret_cast<const float4*>(a.ws_acc + ubase * D);
-            constexpr int PB = 16;  // splits per batch of loads
-            for (int h = warp; h < G; h += CW) {
-                float4 v[PB];
+            const float2* src2 = reinterpret_cast<const float2*>(a.ws_acc + ubase * D);
+            float* wts = merge + 16 * D + warp * kMaxSplits;
+            constexpr int PB = 24;  // splits per batch of loads
+            for (int u = warp; u < 2 * G; u += CW) {
+                const int h = u >> 1, c2 = (u & 1) * 32 + lane;  // float2 column
+                float2 v[PB];
 #pragma unroll
                 for (int j = 0; j < PB; ++j)
-                    v[j] = j < a.n_split ? __ldcg(src4 + (j * G + h) * (D / 4) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[j] = j < a.n_split ? __ldcg(src2 + (j * G + h) * (D / 2) + c2) : make_float2(0.f, 0.f);
                 float mx = -INFINITY;
                 for (int sp = lane; sp < a.n_split; sp += 32) {
                     const float2 m2 = __ldcg(a.ws_ml + ubase + sp * G + h);
@@ -921,31 +952,29 @@ struct Consumer {
                 for (int sp = lane; sp < a.n_split; sp += 32) {
                     const float2 m2 = __ldcg(a.ws_ml + ubase + sp * G + h);
                     const float wgt = (m2.y > 0.f && mx > -INFINITY) ? ptx::ex2(m2.x - mx) : 0.f;
-                    wts[sp * G + h] = wgt;
+                    wts[sp] = wgt;
                     l = fmaf(m2.y, wgt, l);
                 }
                 l = group_sum<32>(l);
                 const float inv_l = l > 0.f ? 1.f / l : 0.f;
                 __syncwarp();
-                float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                float2 acc = make_float2(0.f, 0.f);
                 for (int s0 = 0; s0 < a.n_split; s0 += PB) {
                     if (s0 > 0) {
 #pragma unroll
                         for (int j = 0; j < PB; ++j)
-                            v[j] = s0 + j < a.n_split ? __ldcg(src4 + ((s0 + j) * G + h) * (D / 4) + lane)
-                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                            v[j] = s0 + j < a.n_split ? __ldcg(src2 + ((s0 + j) * G + h) * (D / 2) + c2)
+                                                      : make_float2(0.f, 0.f);
                     }
 #pragma unroll
                     for (int j = 0; j < PB; ++j) {
-                        const float wgt = s0 + j < a.n_split ? wts[(s0 + j) * G + h] : 0.f;
-                        acc4.x = fmaf(v[j].x, wgt, acc4.x);
-                        acc4.y = fmaf(v[j].y, wgt, acc4.y);
-                        acc4.z = fmaf(v[j].z, wgt, acc4.z);
-                        acc4.w = fmaf(v[j].w, wgt, acc4.w);
+                        const float wgt = s0 + j < a.n_split ? wts[s0 + j] : 0.f;
+                        acc.x = fmaf(v[j].x, wgt, acc.x);
+                        acc.y = fmaf(v[j].y, wgt, acc.y);
                     }
                 }
-                *reinterpret_cast<float4*>(o_s + h * D + 4 * lane) =
-                    make_float4(acc4.x * inv_l, acc4.y * inv_l, acc4.z * inv_l, acc4.w * inv_l);
+                __syncwarp();  // the weights row is rewritten by this warp's next unit
+                *reinterpret_cast<float2*>(o_s + h * D + 2 * c2) = make_float2(acc.x * inv_l, acc.y * inv_l);
             }
             ptx::named_barrier(1, NUM_CONSUMERS);
             const float inv_sqrt_d = 0.08838834764831845f;
@@ -957,7 +986,7 @@ struct Consumer {
                 fwht_lanes<4, 32>(x, lane);
                 float* dst = a.out + (static_cast<size_t>(w.b) * a.hq + w.kv * G + h) * D + lane * 4;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) dst[e] = flip_sign(x[e] * inv_sqrt_d, sign_bit(a.signs, lane * 4 + e));
+                for (int e = 0; e < 4; ++e) dst[e] = flip_sign(x[e] * inv_sqrt_d, (sgn4 >> e) & 1u);
             }
             if (tid == 0) a.counters[w.unit] = 0;
         }
@@ -965,49 +994,58 @@ struct Consumer {
     }
 
     __device__ void run() {
-        const uint32_t full0 = base + L.bars, empty0 = full0 + 64;
+        const uint32_t full0 = base + L.bars, empty0 = full0 + 64, qfull0 = full0 + 128, qempty0 = full0 + 144;
         uint32_t bq[NT][8][4];
         uint32_t bz[NT][4][2];
         float f1[NT][2], f2[NT][2];
         SoftState<NT> S;
-        S.reset();
-        Item w{};
         int seq = 0, qseq = 0;
-        bool done_ok = false, app = false;
+        bool done_ok = false;
         while (true) {
-            const int slot = seq % a.stages, use = seq / a.stages;
-            if (!ptx::mbar_wait_bounded(full0 + 8 * slot, use & 1, WAIT_LIMIT)) set_abort();
+            // next item: its header (and queries) in query slot qseq
+            if (!ptx::mbar_wait_bounded(qfull0 + 8 * (qseq & 1), (qseq >> 1) & 1, WAIT_LIMIT)) set_abort();
             ptx::named_barrier(1, NUM_CONSUMERS);  // every consumer warp sees the same abort state
             if (aborted()) break;
-            const uint8_t* st = smem + L.ring + slot * L.stage_bytes;
-            const int4 hdr = *reinterpret_cast<const int4*>(st);
-            if (hdr.w & F_END) {
+            const int4* qh = reinterpret_cast<const int4*>(smem + L.qring + (qseq & 1) * QSLOT_BYTES);
+            const int4 h0 = qh[0], h1 = qh[1];
+            if (h1.x & F_END) {
                 done_ok = true;
                 break;
             }
-            const bool empty = hdr.w & F_EMPTY;
-            if (hdr.w & F_FIRST) {
-                w = item_of(a, hdr.x);
-                if (w.bad && a.err && w.split == 0 && w.kv == 0 && tid == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
-                S.reset();
-                app = a.append && !empty && w.s1 == w.len;
-                if (!empty) {
-                    if (!prologue(qseq, w, app, bq, bz, f1, f2)) break;
-                    ++qseq;
-                }
-            }
-            if (app && (hdr.w & F_LAST)) {  // the stage holding the appended token
-                patch_stage(const_cast<uint8_t*>(st), w.len - 1 - hdr.y);
+            Item w;
+            w.split = h0.x % a.n_split;
+            w.s0 = h0.y;
+            w.s1 = h0.z;
+            w.len = h0.w;
+            w.unit = h1.y;
+            w.b = h1.z;
+            w.kv = h1.w;
+            w.bad = false;
+            const bool empty = h1.x & F_EMPTY, app = h1.x & F_APPEND;
+            S.reset();
+            if (!empty) prologue(qseq, w, app, bq, bz, f1, f2);  // its named barrier ends the slot's use
+            else ptx::named_barrier(1, NUM_CONSUMERS);           // every warp has read the header
+            if (tid == 0) ptx::mbar_arrive(qempty0 + 8 * (qseq & 1));  // query slot free
+            ++qseq;
+            for (int t0 = w.s0; t0 < w.s1; t0 += CHUNK) {
+                const int slot = seq % a.stages, use = seq / a.stages;
+                if (!ptx::mbar_wait_bounded(full0 + 8 * slot, use & 1, WAIT_LIMIT)) set_abort();
                 ptx::named_barrier(1, NUM_CONSUMERS);
+                if (aborted()) break;
+                const uint8_t* st = smem + L.ring + slot * L.stage_bytes;
+                const bool last = t0 + CHUNK >= w.s1;
+                if (app && last) {  // the stage holding the appended token
+                    patch_stage(const_cast<uint8_t*>(st), w.len - 1 - t0);
+                    ptx::named_barrier(1, NUM_CONSUMERS);
+                }
+                if (last) chunk<true>(w, st, t0, bq, bz, f1, f2, S);
+                else chunk<false>(w, st, t0, bq, bz, f1, f2, S);
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(empty0 + 8 * slot);
+                ++seq;
             }
-            if (!empty) {
-                if (hdr.w & F_LAST) chunk<true>(w, st, hdr.y, bq, bz, f1, f2, S);
-                else chunk<false>(w, st, hdr.y, bq, bz, f1, f2, S);
-            }
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(empty0 + 8 * slot);
-            if (hdr.w & F_LAST) epilogue(w, S);
-            ++seq;
+            if (aborted()) break;
+            epilogue(w, S);
         }
         if (done_ok && tid == 0) {
             // the last block to finish re-arms the global counters for the next call
@@ -1046,30 +1084,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid
         }
         return;
     }
-    // per-lane replicated centroid-pair tables, built while the first copies fly:
-    // key pairs in bytes [0,128) of each 256-byte entry, value pairs (3- and
-    // 4-bit values) in [128, 256)
-    uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-    const __half* kc = reinterpret_cast<const __half*>(a.kcent);
-    const __half* vc = reinterpret_cast<const __half*>(a.vcent);
-    constexpr int nk = 1 << (2 * KB), nv = VB >= 3 ? 1 << (2 * VB) : 256;
-    for (int idx = threadIdx.x; idx < (nk + nv) * 32; idx += NUM_CONSUMERS) {
-        const int e = idx >> 5, r = idx & 31;
-        if (e < nk) {
-            const __half2 v = __halves2half2(kc[e & ((1 << KB) - 1)], kc[e >> KB]);
-            lut[e * 64 + r] = *reinterpret_cast<const uint32_t*>(&v);
-        } else if (VB >= 3) {
-            const int ev = e - nk;
-            const __half2 v = __halves2half2(vc[ev & ((1 << VB) - 1)], vc[ev >> VB]);
-            lut[ev * 64 + 32 + r] = *reinterpret_cast<const uint32_t*>(&v);
-        } else {
-            // byte ev = (token a: two 2-bit codes) | (token b: two codes) << 4;
-            // word 2*replica: first channel (a, b), word 2*replica + 1: second channel
-            const int ev = e - nk, rep = r >> 1;
-            const int ca = (r & 1) ? (ev >> 2) & 3 : ev & 3;
-            const int cb = (r & 1) ? (ev >> 6) & 3 : (ev >> 4) & 3;
-            const __half2 v = __halves2half2(vc[ca], vc[cb]);
-            lut[ev * 64 + 32 + 2 * rep + (r & 1)] = *reinterpret_cast<const uint32_t*>(&v);
+    // Per-lane replicated centroid-pair tables, built while the first copies
+    // fly: row e (256 bytes) holds the key pair for code byte e in its first
+    // 32 words and the value pair(s) in the last 32.  Step 1: thread e forms
+    // row e's words once (from centroids staged in shared memory: a per-thread
+    // index into the kernel parameters would serialise).  Step 2: the
+    // threads replicate them in address order, 16 bytes per store (a warp
+    // covers 512 contiguous bytes), with independent reads.
+    {
+        __half* cen = reinterpret_cast<__half*>(smem + L.app);  // [16] key, [16] value
+        uint32_t* compact = reinterpret_cast<uint32_t*>(smem + L.merge);  // [256] key, [256][2] value
+        if (threadIdx.x == 0) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                cen[j] = __ushort_as_half(a.kcent[j]);
+                cen[16 + j] = __ushort_as_half(a.vcent[j]);
+            }
+        }
+        ptx::named_barrier(1, NUM_CONSUMERS);
+        {
+            const int e = threadIdx.x;
+            const __half* kc = cen;
+            const __half* vc = cen + 16;
+            const __half2 k2 = __halves2half2(kc[e & ((1 << KB) - 1)], kc[(e >> KB) & ((1 << KB) - 1)]);
+            __half2 v0, v1;
+            if constexpr (VB >= 3) {
+                v0 = v1 = __halves2half2(vc[e & ((1 << VB) - 1)], vc[(e >> VB) & ((1 << VB) - 1)]);
+            } else {
+                // byte e = (token a: two 2-bit codes) | (token b: two codes) << 4; the
+                // first word holds channel 1 of (a, b), the second channel 2
+                v0 = __halves2half2(vc[e & 3], vc[(e >> 4) & 3]);
+                v1 = __halves2half2(vc[(e >> 2) & 3], vc[(e >> 6) & 3]);
+            }
+            compact[e] = *reinterpret_cast<const uint32_t*>(&k2);
+            compact[256 + 2 * e] = *reinterpret_cast<const uint32_t*>(&v0);
+            compact[256 + 2 * e + 1] = *reinterpret_cast<const uint32_t*>(&v1);
+        }
+        ptx::named_barrier(1, NUM_CONSUMERS);
+        uint4* lut4 = reinterpret_cast<uint4*>(smem);
+        const int part = threadIdx.x & 15;  // the same 16-byte column of every row this thread writes
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int e = (threadIdx.x >> 4) + 16 * k;
+            uint4 v;
+            if (part < 8) {
+                const uint32_t w = compact[e];
+                v = make_uint4(w, w, w, w);
+            } else {
+                const uint2 w = *reinterpret_cast<const uint2*>(compact + 256 + 2 * e);
+                v = make_uint4(w.x, w.y, w.x, w.y);
+            }
+            lut4[threadIdx.x + 256 * k] = v;
         }
     }
     if (ptx::smem_addr(smem) != WINDOW) {  // the host checked the reserved size; never expected
