@@ -56,7 +56,7 @@ namespace tq {
 namespace mmadec {
 
 constexpr int D = 128;
-constexpr int CW = 8;                        // consumer warps
+constexpr int CW = 11;                       // consumer warps (3 warps per scheduler with the producer)
 constexpr int TPW = 2;                       // 16-token tiles per warp and chunk
 constexpr int NUM_THREADS = (CW + 1) * 32;   // + one producer warp
 constexpr int NUM_CONSUMERS = CW * 32;
@@ -66,10 +66,7 @@ constexpr uint32_t LUT_BYTES = 65536;        // 256 entries x 256 B
 // shared memory precedes it); the host checks it before choosing this kernel,
 // and table lookups carry it as an immediate offset.
 constexpr uint32_t WINDOW = 1024;
-constexpr uint32_t Q_BYTES = 16 * D * 4;     // one item's queries, up to 16 heads in fp32
-constexpr uint32_t NEW_ROW = D * 4;           // one appended key or value row, up to fp32
 constexpr uint32_t QHDR = 32;                 // item header at the front of a query slot
-constexpr uint32_t QSLOT_BYTES = QHDR + Q_BYTES + 2 * NEW_ROW;  // header, queries, new key and value rows
 constexpr uint32_t APP_BYTES = 1024;          // the appended token's codes and scratch
 constexpr long long WAIT_LIMIT = 2000000000ll;  // clock cycles (~1 s)
 constexpr float LOG2E = 1.4426950408889634f;
@@ -117,10 +114,16 @@ struct Args {
 // [header | K codes | V codes | K norms | V norms | QJL words | gammas].
 struct Layout {
     uint32_t ring, stage_bytes, k_off, v_off, kn_off, vn_off, z_off, gam_off;
-    uint32_t qring, qh, qlo, sq, app, fac, merge, ml, bars, flags, total;
+    uint32_t qslot, qrows, qring, qh, qlo, sq, app, fac, merge, ml, bars, flags, total;
 };
 
-__host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int m) {
+__host__ __device__ inline uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
+
+// g: query heads per kv head; q_bytes, new_bytes: element sizes of the
+// queries and of the appended rows (0: no append); n_split: splits per
+// (sequence, kv head).
+__host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int m, int g, int q_bytes, int new_bytes,
+                                         int n_split) {
     Layout L{};
     L.ring = LUT_BYTES;
     L.k_off = 16;
@@ -130,14 +133,25 @@ __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int
     L.z_off = L.vn_off + CHUNK * 2;
     L.gam_off = L.z_off + CHUNK * (m / 8);
     L.stage_bytes = L.gam_off + (m > 0 ? CHUNK * 2 : 0);
+    // query slot: header, the item's g query rows, the appended key and value rows
+    L.qrows = QHDR + align16(g * D * q_bytes);
+    L.qslot = align16(L.qrows + 2 * D * new_bytes);
     L.qring = L.ring + stages * L.stage_bytes;        // 2 query slots
-    L.qh = L.qring + 2 * QSLOT_BYTES;                  // fp16 [16][128], rounded q~
-    L.qlo = L.qh + 16 * D * 2;                         // fp16 [16][128], q~ minus the rounded part
-    L.sq = L.qlo + 16 * D * 2;                         // fp16 [16][64]
-    L.app = L.sq + 16 * 64 * 2;                        // appended token: packed rows, norms, scratch
+    L.qh = L.qring + 2 * L.qslot;                      // fp16 [8 nt][128], rounded q~
+    L.qlo = L.qh + 8 * nt * D * 2;                     // fp16 [8 nt][128], q~ minus the rounded part
+    L.sq = L.qlo + 8 * nt * D * 2;                     // fp16 [8 nt][64]
+    L.app = L.sq + 8 * nt * 64 * 2;                    // appended token: packed rows, norms, scratch
     L.fac = L.app + APP_BYTES;                         // float F1[16], F2[16]
-    L.merge = L.fac + 32 * 4;                          // float [CW][8*nt][128]
-    L.ml = L.merge + CW * 8 * nt * D * 4;              // float2 [CW][16]
+    L.merge = L.fac + 32 * 4;
+    // merge area, reused: per-warp partials [CW][g][128]; the final merge's
+    // [g][128] outputs and [CW][n_split] weights; the prologue's [8 nt][128]
+    // sketch staging; the table build's 768 compact words
+    uint32_t merge = CW * g * D * 4;
+    const uint32_t fin = (g * D + CW * n_split) * 4;
+    if (fin > merge) merge = fin;
+    if (8u * nt * D * 4 > merge) merge = 8 * nt * D * 4;
+    if (768u * 4 > merge) merge = 768 * 4;
+    L.ml = L.merge + align16(merge);                   // float2 [CW][16]
     L.bars = L.ml + CW * 16 * 8;                       // u64 full[8], empty[8], qfull[2], qempty[2]
     L.flags = L.bars + 20 * 8;                         // int abort, last
     L.total = L.flags + 16;
@@ -219,7 +233,7 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
             ok = false;
             return false;
         }
-        slot = smem + L.qring + qs * QSLOT_BYTES;
+        slot = smem + L.qring + qs * L.qslot;
         qfull = qfull0 + 8 * qs;
         ++qseq;
         return true;
@@ -250,9 +264,9 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
                                qbytes, qfull);
             if (app) {
                 const size_t row = (static_cast<size_t>(w.b) * a.hkv + w.kv) * rbytes;
-                ptx::bulk_copy_g2s(qdst + Q_BYTES, static_cast<const uint8_t*>(a.k_new) + row, rbytes, qfull);
-                ptx::bulk_copy_g2s(qdst + Q_BYTES + NEW_ROW, static_cast<const uint8_t*>(a.v_new) + row, rbytes,
-                                   qfull);
+                const uint32_t rdst = ptx::smem_addr(qslot) + L.qrows;
+                ptx::bulk_copy_g2s(rdst, static_cast<const uint8_t*>(a.k_new) + row, rbytes, qfull);
+                ptx::bulk_copy_g2s(rdst + rbytes, static_cast<const uint8_t*>(a.v_new) + row, rbytes, qfull);
             }
         }
         for (int t0 = w.s0; t0 < w.s1; t0 += CHUNK) {
@@ -553,7 +567,7 @@ struct Consumer {
     __device__ void prologue(int qseq, const Item& w, bool app, uint32_t (&bq)[NT][8][4], uint32_t (&bz)[NT][4][2],
                              float (&f1)[NT][2], float (&f2)[NT][2]) {
         const int G = a.group;
-        const uint8_t* qsrc = smem + L.qring + (qseq & 1) * QSLOT_BYTES + QHDR;
+        const uint8_t* qsrc = smem + L.qring + (qseq & 1) * L.qslot + QHDR;
         __half* qh = reinterpret_cast<__half*>(smem + L.qh);
         __half* ql = reinterpret_cast<__half*>(smem + L.qlo);
         __half* sq = reinterpret_cast<__half*>(smem + L.sq);
@@ -616,14 +630,14 @@ struct Consumer {
         }
         if (app && warp < 2) {
             const size_t slot = static_cast<size_t>(w.unit) * a.capacity + (w.len - 1);
-            const uint8_t* rows = smem + L.qring + (qseq & 1) * QSLOT_BYTES + QHDR + Q_BYTES;
+            const uint8_t* rows = smem + L.qring + (qseq & 1) * L.qslot + L.qrows;
             uint8_t* ap = smem + L.app;
             if (warp == 0)
                 encode_new<KB, QJL>(rows, const_cast<uint8_t*>(a.k_codes), const_cast<uint16_t*>(a.k_norms), a.kbound,
                                     slot, ap, reinterpret_cast<uint16_t*>(ap + 128), ap + 256,
                                     reinterpret_cast<float*>(ap + 512));
             else
-                encode_new<VB, false>(rows + NEW_ROW, const_cast<uint8_t*>(a.v_codes), const_cast<uint16_t*>(a.v_norms),
+                encode_new<VB, false>(rows + D * a.new_bytes, const_cast<uint8_t*>(a.v_codes), const_cast<uint16_t*>(a.v_norms),
                                       a.vbound, slot, ap + 64, reinterpret_cast<uint16_t*>(ap + 130), ap + 384,
                                       reinterpret_cast<float*>(ap + 512));
         }
@@ -889,12 +903,17 @@ struct Consumer {
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                float* mw = merge + (warp * 8 * NT + nt * 8) * D;
+                const int h0 = nt * 8 + 2 * t;  // heads h0, h0 + 1 of this lane's columns
+                float* mw = merge + (warp * G + h0) * D;
                 const int c_lo = 16 * g + 2 * i, c_hi = c_lo + 1;
-                mw[(2 * t) * D + c_lo] = S.acc[nt][i][0] * unscale;
-                mw[(2 * t + 1) * D + c_lo] = S.acc[nt][i][1] * unscale;
-                mw[(2 * t) * D + c_hi] = S.acc[nt][i][2] * unscale;
-                mw[(2 * t + 1) * D + c_hi] = S.acc[nt][i][3] * unscale;
+                if (h0 < G) {
+                    mw[c_lo] = S.acc[nt][i][0] * unscale;
+                    mw[c_hi] = S.acc[nt][i][2] * unscale;
+                }
+                if (h0 + 1 < G) {
+                    mw[D + c_lo] = S.acc[nt][i][1] * unscale;
+                    mw[D + c_hi] = S.acc[nt][i][3] * unscale;
+                }
             }
         ptx::named_barrier(1, NUM_CONSUMERS);
         const size_t pbase = (static_cast<size_t>(w.unit) * a.n_split + w.split) * G;
@@ -912,7 +931,7 @@ struct Consumer {
                     if (!(v.y > 0.f)) continue;
                     const float f = ptx::ex2(v.x - mx);
                     l = fmaf(v.y, f, l);
-                    s = fmaf(merge[(ww * 8 * NT + h) * D + c], f, s);
+                    s = fmaf(merge[(ww * G + h) * D + c], f, s);
                 }
             }
             a.ws_acc[(pbase + h) * D + c] = s * a.inv_alpha_v;  // undo the centroid scale
@@ -934,7 +953,7 @@ struct Consumer {
             float* o_s = merge;  // [G][D]
             const size_t ubase = static_cast<size_t>(w.unit) * a.n_split * G;
             const float2* src2 = reinterpret_cast<const float2*>(a.ws_acc + ubase * D);
-            float* wts = merge + 16 * D + warp * kMaxSplits;
+            float* wts = merge + G * D + warp * a.n_split;
             constexpr int PB = 24;  // splits per batch of loads
             for (int u = warp; u < 2 * G; u += CW) {
                 const int h = u >> 1, c2 = (u & 1) * 32 + lane;  // float2 column
@@ -1004,9 +1023,10 @@ struct Consumer {
         while (true) {
             // next item: its header (and queries) in query slot qseq
             if (!ptx::mbar_wait_bounded(qfull0 + 8 * (qseq & 1), (qseq >> 1) & 1, WAIT_LIMIT)) set_abort();
-            ptx::named_barrier(1, NUM_CONSUMERS);  // every consumer warp sees the same abort state
-            if (aborted()) break;
-            const int4* qh = reinterpret_cast<const int4*>(smem + L.qring + (qseq & 1) * QSLOT_BYTES);
+            // every consumer warp takes the same decision (the producer may set
+            // the flag at any moment, so each thread's own read could differ)
+            if (ptx::named_barrier_or(1, NUM_CONSUMERS, aborted())) break;
+            const int4* qh = reinterpret_cast<const int4*>(smem + L.qring + (qseq & 1) * L.qslot);
             const int4 h0 = qh[0], h1 = qh[1];
             if (h1.x & F_END) {
                 done_ok = true;
@@ -1027,25 +1047,30 @@ struct Consumer {
             else ptx::named_barrier(1, NUM_CONSUMERS);           // every warp has read the header
             if (tid == 0) ptx::mbar_arrive(qempty0 + 8 * (qseq & 1));  // query slot free
             ++qseq;
+            // Warps wait for each stage on their own.  A wait that runs out sets
+            // the abort flag and later waits are skipped, but every warp still
+            // walks the item's stages and meets the others at the item's named
+            // barriers (the patch below, the epilogue), so none is left behind.
             for (int t0 = w.s0; t0 < w.s1; t0 += CHUNK) {
                 const int slot = seq % a.stages, use = seq / a.stages;
-                if (!ptx::mbar_wait_bounded(full0 + 8 * slot, use & 1, WAIT_LIMIT)) set_abort();
-                ptx::named_barrier(1, NUM_CONSUMERS);
-                if (aborted()) break;
+                if (!aborted() && !ptx::mbar_wait_bounded(full0 + 8 * slot, use & 1, WAIT_LIMIT)) set_abort();
+                const bool ok = !aborted();
                 const uint8_t* st = smem + L.ring + slot * L.stage_bytes;
                 const bool last = t0 + CHUNK >= w.s1;
                 if (app && last) {  // the stage holding the appended token
-                    patch_stage(const_cast<uint8_t*>(st), w.len - 1 - t0);
+                    if (ok) patch_stage(const_cast<uint8_t*>(st), w.len - 1 - t0);
                     ptx::named_barrier(1, NUM_CONSUMERS);
                 }
-                if (last) chunk<true>(w, st, t0, bq, bz, f1, f2, S);
-                else chunk<false>(w, st, t0, bq, bz, f1, f2, S);
+                if (ok) {
+                    if (last) chunk<true>(w, st, t0, bq, bz, f1, f2, S);
+                    else chunk<false>(w, st, t0, bq, bz, f1, f2, S);
+                }
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(empty0 + 8 * slot);
                 ++seq;
             }
-            if (aborted()) break;
             epilogue(w, S);
+            if (ptx::named_barrier_or(1, NUM_CONSUMERS, aborted())) break;
         }
         if (done_ok && tid == 0) {
             // the last block to finish re-arms the global counters for the next call
@@ -1061,7 +1086,8 @@ struct Consumer {
 template <int KB, int VB, int NT, bool QJL>
 __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid_constant__ Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const Layout L = layout(KB, VB, NT, a.stages, QJL ? a.m : 0);
+    const Layout L = layout(KB, VB, NT, a.stages, QJL ? a.m : 0, a.group, a.q_bytes, a.append ? a.new_bytes : 0,
+                            a.n_split);
     ptx::launch_dependents();  // the next kernel may start launching; it waits for this one to finish
     if (threadIdx.x == NUM_CONSUMERS) {
         const uint32_t bars = ptx::smem_addr(smem + L.bars);
@@ -1102,7 +1128,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid
             }
         }
         ptx::named_barrier(1, NUM_CONSUMERS);
-        {
+        if (threadIdx.x < 256) {
             const int e = threadIdx.x;
             const __half* kc = cen;
             const __half* vc = cen + 16;
@@ -1122,10 +1148,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid
         }
         ptx::named_barrier(1, NUM_CONSUMERS);
         uint4* lut4 = reinterpret_cast<uint4*>(smem);
+        static_assert(NUM_CONSUMERS % 16 == 0, "each thread writes one 16-byte column of the rows");
         const int part = threadIdx.x & 15;  // the same 16-byte column of every row this thread writes
+        constexpr int REP = (256 * 16 + NUM_CONSUMERS - 1) / NUM_CONSUMERS;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const int e = (threadIdx.x >> 4) + 16 * k;
+        for (int k = 0; k < REP; ++k) {
+            const int c = threadIdx.x + NUM_CONSUMERS * k;
+            if (c >= 256 * 16) break;
+            const int e = c >> 4;
             uint4 v;
             if (part < 8) {
                 const uint32_t w = compact[e];
@@ -1134,7 +1164,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid
                 const uint2 w = *reinterpret_cast<const uint2*>(compact + 256 + 2 * e);
                 v = make_uint4(w.x, w.y, w.x, w.y);
             }
-            lut4[threadIdx.x + 256 * k] = v;
+            lut4[c] = v;
         }
     }
     if (ptx::smem_addr(smem) != WINDOW) {  // the host checked the reserved size; never expected
@@ -1266,12 +1296,13 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     const int nt = a.group <= 8 ? 1 : 2;
     const int kb = p.k_bits, vb = p.v_bits;
     // as many stages as fit in 227 KB next to the tables and the merge buffers
-    const Layout fixed = layout(kb, vb, nt, 0, p.qjl_dims);
+    const Layout fixed = layout(kb, vb, nt, 0, p.qjl_dims, a.group, a.q_bytes, a.append ? a.new_bytes : 0, a.n_split);
     int stages = static_cast<int>((232448u - fixed.total) / fixed.stage_bytes);
     if (stages > 8) stages = 8;
     if (stages < 2) return cudaErrorInvalidConfiguration;
     a.stages = stages;
-    const size_t smem = layout(kb, vb, nt, stages, p.qjl_dims).total;
+    const size_t smem =
+        layout(kb, vb, nt, stages, p.qjl_dims, a.group, a.q_bytes, a.append ? a.new_bytes : 0, a.n_split).total;
     int grid = num_sms;
     if (grid > a.n_items) grid = a.n_items;
     const bool qjl = p.qjl_dims > 0;
