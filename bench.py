@@ -323,6 +323,41 @@ def bulk_quantize(dev, d, reps=3):
     return {key: round(val, 2) for key, val in res.items()}
 
 
+def bf16_sdpa_baseline(dev, reps=20):
+    """Uncompressed comparison arm (library code, not this path): torch's
+    scaled_dot_product_attention over bf16 K/V of the same decode shape (B=1,
+    Hq=32, Hkv=8, d=128, 32769 tokens), 32 distinct layer caches (4.3 GB,
+    larger than L2), timed with CUDA events; 512 B per token and kv head."""
+    import torch.nn.functional as F
+    from bit_kv_cache_tq_b200 import inputs
+    seq = CONTEXT + 1
+    ks = [inputs.lognormal_kv(BATCH, seq, HKV, D, SEED, l, inputs.K, device=dev).transpose(1, 2).contiguous()
+          for l in range(LAYERS)]
+    vs = [inputs.lognormal_kv(BATCH, seq, HKV, D, SEED, l, inputs.V, device=dev).transpose(1, 2).contiguous()
+          for l in range(LAYERS)]
+    q = inputs.queries(BATCH, HQ, D, SEED, device=dev).view(BATCH, HQ, 1, D)
+
+    def sweep():
+        for l in range(LAYERS):
+            F.scaled_dot_product_attention(q, ks[l], vs[l], enable_gqa=True)
+
+    for _ in range(3):
+        sweep()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        sweep()
+    e1.record()
+    e1.synchronize()
+    us = 1000.0 * e0.elapsed_time(e1) / (reps * LAYERS)
+    bytes_layer = 2 * BATCH * HKV * seq * D * 2
+    del ks, vs
+    torch.cuda.empty_cache()
+    return {"kernel": "torch.nn.functional.scaled_dot_product_attention (bf16, enable_gqa, default backend)",
+            "us_per_layer": round(us, 2), "kv_tokens_per_s": round(BATCH * seq / (us * 1e-6)),
+            "gbs": round(bytes_layer / (us * 1e-6) / 1e9, 1), "bytes_per_layer": bytes_layer}
+
+
 def run_tq(args, world, rank, local):
     from bit_kv_cache_tq_b200 import inputs, tq
     dev = torch.device("cuda", local)
@@ -485,7 +520,8 @@ def run_tq(args, world, rank, local):
             "gpu_launches": launches_per_step * steps,
             "clocks": clocks.summary(),
         }
-        if not args.no_quantize:
+        if not args.quick:
+            line["bf16_baseline"] = bf16_sdpa_baseline(dev)
             peak_gbs = measured_peaks()[0]
             q = {"workload": "bulk prefill quantise: 262144 tokens x 8 kv heads, bf16, 32 layers (0, 1, 30, 31 "
                              "int8 per-vector absmax, others K4/V3 turbo), one input slab, 32 distinct outputs",
@@ -535,7 +571,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-quantize", action="store_true", help="skip the bulk prefill quantise measurement")
+    ap.add_argument("--quick", action="store_true",
+                    help="skip the bf16 baseline and the bulk prefill quantise measurement")
     ap.add_argument("--profile", choices=["decode", "quantize"], default=None,
                     help="run a small one-layer case for ncu instead of the benchmark")
     args = ap.parse_args()

@@ -62,30 +62,66 @@ __device__ __forceinline__ void store_chunk_codes(uint8_t* row, int chunk, uint3
     }
 }
 
+// Code of the rotated coordinate x = y * sqrt(d) * ||x|| against the
+// boundaries scaled the same way (ts[k] = t_k sqrt(d) ||x||, ascending): the
+// count of boundaries below y, found with a binary search over the positive
+// half (the table is odd-symmetric, its middle boundary is 0).  Deciding on x
+// against scaled boundaries instead of on y = x / (sqrt(d) ||x||) moves a
+// decision only when y is within a few ulp of a boundary.
+template <int BITS>
+__device__ __forceinline__ uint32_t code_scaled(float x, const float (&ts)[7]) {
+    constexpr int half = 1 << (BITS - 1);
+    const float a = fabsf(x);
+    int m;
+    if constexpr (BITS == 4) {
+        const bool p2 = a > ts[3];
+        const bool p1 = a > (p2 ? ts[5] : ts[1]);
+        const float w = p1 ? (p2 ? ts[6] : ts[2]) : (p2 ? ts[4] : ts[0]);
+        m = 4 * p2 + 2 * p1 + (a > w);
+    } else if constexpr (BITS == 3) {
+        const bool p1 = a > ts[1];
+        m = 2 * p1 + (a > (p1 ? ts[2] : ts[0]));
+    } else {
+        m = a > ts[0];
+    }
+    return x > 0.0f ? static_cast<uint32_t>(half + m) : static_cast<uint32_t>(half - 1 - m);
+}
+
+// Rotation signs of this lane's 32 coordinates 8 (sub + LPV k) + e, as bit
+// 8 k + e of one word (built once per thread).
+template <int D>
+__device__ __forceinline__ uint32_t lane_sign_mask(const uint32_t* signs, int sub) {
+    constexpr int LPV = D / 32;
+    uint32_t m = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int i0 = 8 * (sub + LPV * k);
+        m |= ((signs[i0 >> 5] >> (i0 & 31)) & 0xFFu) << (8 * k);
+    }
+    return m;
+}
+
 template <int D, int BITS>
 __device__ __forceinline__ void turbo_encode(const QuantSide& s, float (&x)[32], int sub, size_t slot, bool valid,
-                                             const uint32_t* signs) {
+                                             uint32_t smask) {
     constexpr int LPV = D / 32;
     float sumsq = 0.0f;
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int i = 8 * (sub + LPV * k) + e;
-            sumsq = fmaf(x[8 * k + e], x[8 * k + e], sumsq);
-            x[8 * k + e] = flip_sign(x[8 * k + e], sign_bit(signs, i));
-        }
+    for (int j = 0; j < 32; ++j) {
+        sumsq = fmaf(x[j], x[j], sumsq);
+        x[j] = __uint_as_float(__float_as_uint(x[j]) ^ ((smask << (31 - j)) & 0x80000000u));
+    }
     fwht_registers(x);
     fwht_lanes<32, LPV>(x, sub);
     sumsq = group_sum<LPV>(sumsq);
     const float n = sqrtf(sumsq);
-    const float inv = n > 0.0f ? 1.0f / (sqrtf(static_cast<float>(D)) * n) : 0.0f;
+    const float scale = sqrtf(static_cast<float>(D)) * n;  // y_i = x_i / scale
+    float ts[7];
+#pragma unroll
+    for (int k = 0; k < 7; ++k) ts[k] = s.pos_boundaries[k] * scale;
     uint32_t codes[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        x[i] *= inv;  // rotated unit-vector coordinate y_i
-        codes[i] = code_of<BITS>(x[i], s.pos_boundaries);
-    }
+    for (int i = 0; i < 32; ++i) codes[i] = code_scaled<BITS>(x[i], ts);
     if (valid) {
         uint8_t* row = s.codes + slot * static_cast<size_t>(s.vbytes);
 #pragma unroll
@@ -98,10 +134,11 @@ __device__ __forceinline__ void turbo_encode(const QuantSide& s, float (&x)[32],
         if (sub == 0) s.norms[slot] = float_to_half_bits(n);
     }
     if (s.m > 0) {  // QJL residual sketch (keys only)
+        const float inv = n > 0.0f ? 1.0f / scale : 0.0f;
         float g2 = 0.0f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            x[i] -= s.centroids[codes[i]];  // residual r_i
+            x[i] = x[i] * inv - s.centroids[codes[i]];  // residual r_i = y_i - c[code_i]
             g2 = fmaf(x[i], x[i], g2);
         }
         g2 = group_sum<LPV>(g2);
@@ -159,13 +196,14 @@ __device__ __forceinline__ void int8_encode(const QuantSide& s, const float (&x)
 }
 
 template <int D, int DTYPE>
-__global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_constant__ QuantArgs a) {
+__global__ void __launch_bounds__(256, 2) quantize_append_kernel(const __grid_constant__ QuantArgs a) {
     constexpr int LPV = D / 32;  // lanes per vector
     constexpr int VPW = 32 / LPV;  // vectors per warp pass
     const QuantSide& s = a.side[blockIdx.y];
     ptx::launch_dependents();    // the next kernel may start launching
     ptx::wait_prerequisites();   // inputs and cache may come from the previous kernel
     const int lane = threadIdx.x & 31, sub = lane % LPV, grp = lane / LPV;
+    const uint32_t smask = lane_sign_mask<D>(a.signs, sub);
     const long long total = static_cast<long long>(a.batch) * a.n_new * a.hkv;
     const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
     for (long long base = (static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32) * VPW;
@@ -198,11 +236,11 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
         if (s.mode == TQ_MODE_INT8) {
             int8_encode<D>(s, x, sub, slot, valid);
         } else if (s.bits == 4) {
-            turbo_encode<D, 4>(s, x, sub, slot, valid, a.signs);
+            turbo_encode<D, 4>(s, x, sub, slot, valid, smask);
         } else if (s.bits == 3) {
-            turbo_encode<D, 3>(s, x, sub, slot, valid, a.signs);
+            turbo_encode<D, 3>(s, x, sub, slot, valid, smask);
         } else {
-            turbo_encode<D, 2>(s, x, sub, slot, valid, a.signs);
+            turbo_encode<D, 2>(s, x, sub, slot, valid, smask);
         }
     }
 }
