@@ -73,8 +73,9 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LAZY = 8.0f;                 // log2 headroom before the running max moves
 constexpr float VRANGE = 64.0f;              // bound on ||v|| * vscale
 
-// header flags: item (query slot) EMPTY / END / APPEND, chunk (stage) LAST
-constexpr int F_LAST = 2, F_EMPTY = 4, F_END = 8, F_APPEND = 16;
+// header flags: item (query slot) EMPTY / END / APPEND / DRAIN (one stage to
+// consume unread), chunk (stage) LAST
+constexpr int F_LAST = 2, F_EMPTY = 4, F_END = 8, F_APPEND = 16, F_DRAIN = 32;
 // global counters after the per-(sequence, kv head) split counters
 constexpr int C_ITEM = 0, C_DONE = 1;
 
@@ -238,7 +239,52 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         ++qseq;
         return true;
     };
-    int i = blockIdx.x;  // the first item of every block is static; later ones come from the counter
+    // issue the copies of chunk [t0, t0 + n) of a unit into the next stage
+    auto issue_chunk = [&](int unit, int t0, int n) -> bool {
+        uint32_t full;
+        uint8_t* st;
+        if (!claim(full, st)) return false;
+        const uint32_t dst = ptx::smem_addr(st);
+        const size_t row = static_cast<size_t>(unit) * a.capacity + t0;
+        if (a.staged_norms) {
+            // capacity and t0 are multiples of 8, so rounding n up to 8 tokens
+            // stays inside the cache and keeps every 2-byte array 16-byte sized
+            const int n8 = (n + 7) & ~7;
+            ptx::mbar_arrive_expect_tx(full, n8 * (VBK + VBV + 4 + (QJL ? zb + 2 : 0)));
+            ptx::bulk_copy_g2s(dst + L.k_off, a.k_codes + row * VBK, n8 * VBK, full);
+            ptx::bulk_copy_g2s(dst + L.v_off, a.v_codes + row * VBV, n8 * VBV, full);
+            ptx::bulk_copy_g2s(dst + L.kn_off, a.k_norms + row, n8 * 2, full);
+            ptx::bulk_copy_g2s(dst + L.vn_off, a.v_norms + row, n8 * 2, full);
+            if constexpr (QJL) {
+                ptx::bulk_copy_g2s(dst + L.z_off, a.k_qjl + row * zb, n8 * zb, full);
+                ptx::bulk_copy_g2s(dst + L.gam_off, a.k_gamma + row, n8 * 2, full);
+            }
+        } else {
+            ptx::mbar_arrive_expect_tx(full, n * (VBK + VBV));
+            ptx::bulk_copy_g2s(dst + L.k_off, a.k_codes + row * VBK, n * VBK, full);
+            ptx::bulk_copy_g2s(dst + L.v_off, a.v_codes + row * VBV, n * VBV, full);
+        }
+        ++seq;
+        return true;
+    };
+    const uint32_t qbytes = G * D * a.q_bytes;
+    // The block's first item is static: its queries and first chunk (as many
+    // tokens as the cache could hold there) are requested before the sequence
+    // length is read, so the first bytes arrive a DRAM round trip sooner.  If
+    // the item turns out empty, its header tells the consumers to drain that
+    // stage; if shorter, they only read its valid part.
+    int i = blockIdx.x;
+    bool first = true, spec = false;
+    if (i < a.n_items && !*abort_flag) {
+        const int unit = i / a.n_split, split = i % a.n_split;
+        const int b = unit / a.hkv, kv = unit % a.hkv, s0 = split * a.split_len;
+        const uint32_t qf = qfull0;  // query slot 0
+        ptx::mbar_expect_tx(qf, qbytes);
+        ptx::bulk_copy_g2s(ptx::smem_addr(smem + L.qring) + QHDR,
+                           static_cast<const uint8_t*>(a.q) + (static_cast<size_t>(b) * a.hq + kv * G) * D * a.q_bytes,
+                           qbytes, qf);
+        spec = issue_chunk(unit, s0, min(CHUNK, a.capacity - s0));
+    }
     while (ok) {
         if (i >= a.n_items) break;
         const Item w = item_of(a, i);
@@ -250,53 +296,31 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         if (!claim_q(qslot, qfull)) break;
         int4* hdr = reinterpret_cast<int4*>(qslot);
         hdr[0] = make_int4(i, w.s0, w.s1, w.len);
-        hdr[1] = make_int4((empty ? F_EMPTY : 0) | (app ? F_APPEND : 0), w.unit, w.b, w.kv);
-        if (empty) {
-            ptx::mbar_arrive_expect_tx(qfull, 0);
-        } else {
-            const uint32_t qbytes = G * D * a.q_bytes;
-            const uint32_t rbytes = D * a.new_bytes;
-            const uint32_t qdst = ptx::smem_addr(qslot) + QHDR;
-            ptx::mbar_arrive_expect_tx(qfull, qbytes + (app ? 2 * rbytes : 0u));
-            ptx::bulk_copy_g2s(qdst,
+        hdr[1] = make_int4((empty ? F_EMPTY : 0) | (app ? F_APPEND : 0) | (first && spec && empty ? F_DRAIN : 0),
+                           w.unit, w.b, w.kv);
+        const uint32_t rbytes = D * a.new_bytes;
+        const uint32_t extra = app ? 2 * rbytes : 0u;  // append rows
+        if (first) {  // queries already requested; add the append rows, then arrive
+            if (app) ptx::mbar_expect_tx(qfull, extra);
+        } else if (!empty) {
+            ptx::mbar_expect_tx(qfull, qbytes + extra);
+            ptx::bulk_copy_g2s(ptx::smem_addr(qslot) + QHDR,
                                static_cast<const uint8_t*>(a.q) +
                                    (static_cast<size_t>(w.b) * a.hq + w.kv * G) * D * a.q_bytes,
                                qbytes, qfull);
-            if (app) {
-                const size_t row = (static_cast<size_t>(w.b) * a.hkv + w.kv) * rbytes;
-                const uint32_t rdst = ptx::smem_addr(qslot) + L.qrows;
-                ptx::bulk_copy_g2s(rdst, static_cast<const uint8_t*>(a.k_new) + row, rbytes, qfull);
-                ptx::bulk_copy_g2s(rdst + rbytes, static_cast<const uint8_t*>(a.v_new) + row, rbytes, qfull);
-            }
         }
-        for (int t0 = w.s0; t0 < w.s1; t0 += CHUNK) {
-            uint32_t full;
-            uint8_t* st;
-            if (!claim(full, st)) break;
-            const int n = min(CHUNK, w.s1 - t0);
-            *reinterpret_cast<int4*>(st) = make_int4(i, t0, n, t0 + CHUNK >= w.s1 ? F_LAST : 0);
-            const uint32_t dst = ptx::smem_addr(st);
-            const size_t row = static_cast<size_t>(w.unit) * a.capacity + t0;
-            if (a.staged_norms) {
-                // capacity and t0 are multiples of 8, so rounding n up to 8 tokens
-                // stays inside the cache and keeps every 2-byte array 16-byte sized
-                const int n8 = (n + 7) & ~7;
-                ptx::mbar_arrive_expect_tx(full, n8 * (VBK + VBV + 4 + (QJL ? zb + 2 : 0)));
-                ptx::bulk_copy_g2s(dst + L.k_off, a.k_codes + row * VBK, n8 * VBK, full);
-                ptx::bulk_copy_g2s(dst + L.v_off, a.v_codes + row * VBV, n8 * VBV, full);
-                ptx::bulk_copy_g2s(dst + L.kn_off, a.k_norms + row, n8 * 2, full);
-                ptx::bulk_copy_g2s(dst + L.vn_off, a.v_norms + row, n8 * 2, full);
-                if constexpr (QJL) {
-                    ptx::bulk_copy_g2s(dst + L.z_off, a.k_qjl + row * zb, n8 * zb, full);
-                    ptx::bulk_copy_g2s(dst + L.gam_off, a.k_gamma + row, n8 * 2, full);
-                }
-            } else {
-                ptx::mbar_arrive_expect_tx(full, n * (VBK + VBV));
-                ptx::bulk_copy_g2s(dst + L.k_off, a.k_codes + row * VBK, n * VBK, full);
-                ptx::bulk_copy_g2s(dst + L.v_off, a.v_codes + row * VBV, n * VBV, full);
-            }
-            ++seq;
+        if (app) {
+            const size_t row = (static_cast<size_t>(w.b) * a.hkv + w.kv) * rbytes;
+            const uint32_t rdst = ptx::smem_addr(qslot) + L.qrows;
+            ptx::bulk_copy_g2s(rdst, static_cast<const uint8_t*>(a.k_new) + row, rbytes, qfull);
+            ptx::bulk_copy_g2s(rdst + rbytes, static_cast<const uint8_t*>(a.v_new) + row, rbytes, qfull);
         }
+        ptx::mbar_arrive(qfull);  // header written, every copy of the slot accounted for
+        int t0 = w.s0;
+        if (first && spec) t0 += CHUNK;  // the speculative stage holds the first chunk
+        for (; t0 < w.s1; t0 += CHUNK)
+            if (!issue_chunk(w.unit, t0, min(CHUNK, w.s1 - t0))) break;
+        first = false;
         if (!ok) break;
         i = static_cast<int>(gridDim.x + atomicAdd(a.counters + a.units + C_ITEM, 1u));
     }
@@ -917,25 +941,43 @@ struct Consumer {
             }
         ptx::named_barrier(1, NUM_CONSUMERS);
         const size_t pbase = (static_cast<size_t>(w.unit) * a.n_split + w.split) * G;
-        for (int idx = tid; idx < G * D; idx += NUM_CONSUMERS) {
-            const int h = idx / D, c = idx % D;
+        // per head: the warps' weights 2^(m_w - M) (in place of m_w) and the
+        // split's (M, L); then every output column is one weighted sum
+        if (tid < G) {
+            const int h = tid;
             float mx = -INFINITY;
 #pragma unroll
             for (int ww = 0; ww < CW; ++ww)
                 if (ml[ww * 16 + h].y > 0.f) mx = fmaxf(mx, ml[ww * 16 + h].x);
-            float l = 0.f, s = 0.f;
-            if (mx > -INFINITY) {
+            float l = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < CW; ++ww) {
+                const float2 v = ml[ww * 16 + h];
+                const float f = (v.y > 0.f && mx > -INFINITY) ? ptx::ex2(v.x - mx) : 0.f;
+                l = fmaf(v.y, f, l);
+                ml[ww * 16 + h].x = f;
+            }
+            a.ws_ml[pbase + h] = make_float2(mx, l);
+        }
+        ptx::named_barrier(1, NUM_CONSUMERS);
+        {
+            const float4* m4 = reinterpret_cast<const float4*>(merge);
+            float4* dst4 = reinterpret_cast<float4*>(a.ws_acc + pbase * D);
+            for (int idx = tid; idx < G * (D / 4); idx += NUM_CONSUMERS) {
+                const int h = idx / (D / 4), c4 = idx % (D / 4);
+                float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int ww = 0; ww < CW; ++ww) {
-                    const float2 v = ml[ww * 16 + h];
-                    if (!(v.y > 0.f)) continue;
-                    const float f = ptx::ex2(v.x - mx);
-                    l = fmaf(v.y, f, l);
-                    s = fmaf(merge[(ww * G + h) * D + c], f, s);
+                    const float f = ml[ww * 16 + h].x;
+                    const float4 v = m4[(ww * G + h) * (D / 4) + c4];
+                    acc4.x = fmaf(v.x, f, acc4.x);
+                    acc4.y = fmaf(v.y, f, acc4.y);
+                    acc4.z = fmaf(v.z, f, acc4.z);
+                    acc4.w = fmaf(v.w, f, acc4.w);
                 }
+                const float iv = a.inv_alpha_v;  // undo the centroid scale
+                dst4[h * (D / 4) + c4] = make_float4(acc4.x * iv, acc4.y * iv, acc4.z * iv, acc4.w * iv);
             }
-            a.ws_acc[(pbase + h) * D + c] = s * a.inv_alpha_v;  // undo the centroid scale
-            if (c == 0) a.ws_ml[pbase + h] = make_float2(mx, l);
         }
         // publish the partial: the barrier orders every thread's writes before
         // thread 0's release, and its acquire orders the merge's reads after
@@ -1043,6 +1085,13 @@ struct Consumer {
             w.bad = false;
             const bool empty = h1.x & F_EMPTY, app = h1.x & F_APPEND;
             S.reset();
+            if (h1.x & F_DRAIN) {  // a stage filled before the item was known to be empty
+                const int slot = seq % a.stages, use = seq / a.stages;
+                if (!aborted() && !ptx::mbar_wait_bounded(full0 + 8 * slot, use & 1, WAIT_LIMIT)) set_abort();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(empty0 + 8 * slot);
+                ++seq;
+            }
             if (!empty) prologue(qseq, w, app, bq, bz, f1, f2);  // its named barrier ends the slot's use
             else ptx::named_barrier(1, NUM_CONSUMERS);           // every warp has read the header
             if (tid == 0) ptx::mbar_arrive(qempty0 + 8 * (qseq & 1));  // query slot free
