@@ -67,6 +67,11 @@ constexpr uint32_t LUT_BYTES = 65536;        // 256 entries x 256 B
 // and table lookups carry it as an immediate offset.
 constexpr uint32_t WINDOW = 1024;
 constexpr uint32_t QHDR = 32;                 // item header at the front of a query slot
+// Row strides (halves) of the fp16 query and sketch buffers: 2 words past a
+// multiple of 32 banks, so the 8-byte fragment loads of a half-warp (lane
+// groups g = 0..3 at rows g, columns 16 t) hit 32 distinct banks.
+constexpr int QH_STRIDE = D + 4;
+constexpr int SQ_STRIDE = 64 + 4;
 constexpr uint32_t APP_BYTES = 1024;          // the appended token's codes and scratch
 constexpr long long WAIT_LIMIT = 2000000000ll;  // clock cycles (~1 s)
 constexpr float LOG2E = 1.4426950408889634f;
@@ -138,10 +143,10 @@ __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int
     L.qrows = QHDR + align16(g * D * q_bytes);
     L.qslot = align16(L.qrows + 2 * D * new_bytes);
     L.qring = L.ring + stages * L.stage_bytes;        // 2 query slots
-    L.qh = L.qring + 2 * L.qslot;                      // fp16 [8 nt][128], rounded q~
-    L.qlo = L.qh + 8 * nt * D * 2;                     // fp16 [8 nt][128], q~ minus the rounded part
-    L.sq = L.qlo + 8 * nt * D * 2;                     // fp16 [8 nt][64]
-    L.app = L.sq + 8 * nt * 64 * 2;                    // appended token: packed rows, norms, scratch
+    L.qh = L.qring + 2 * L.qslot;                      // fp16 [8 nt][QH_STRIDE], rounded q~
+    L.qlo = L.qh + 8 * nt * QH_STRIDE * 2;             // fp16 [8 nt][QH_STRIDE], q~ minus the rounded part
+    L.sq = L.qlo + 8 * nt * QH_STRIDE * 2;             // fp16 [8 nt][SQ_STRIDE]
+    L.app = align16(L.sq + 8 * nt * SQ_STRIDE * 2);    // appended token: packed rows, norms, scratch
     L.fac = L.app + APP_BYTES;                         // float F1[16], F2[16]
     L.merge = L.fac + 32 * 4;
     // merge area, reused: per-warp partials [CW][g][128]; the final merge's
@@ -601,9 +606,9 @@ struct Consumer {
         for (int h = warp; h < NT * 8; h += CW) {
             float x[4] = {0.f, 0.f, 0.f, 0.f};
             if (h < G) {
+                load4(qsrc, h * D + lane * 4, a.q_dtype, x);
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    x[e] = flip_sign(load_scalar(qsrc, h * D + lane * 4 + e, a.q_dtype), (sgn4 >> e) & 1u);
+                for (int e = 0; e < 4; ++e) x[e] = flip_sign(x[e], (sgn4 >> e) & 1u);
                 fwht_registers(x);
                 fwht_lanes<4, 32>(x, lane);
 #pragma unroll
@@ -613,14 +618,19 @@ struct Consumer {
             amax = group_max<32>(amax);
             const float qmax = amax > 0.f ? amax : 1.f;
             const float rq = 1.0f / qmax;  // F1 undoes the scale (to one fp32 ulp)
+            // two fp16 terms: the scores keep about 22 bits of q~
+            uint32_t hw[2], lw[2];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                // two fp16 terms: the scores keep about 22 bits of q~
-                const float u = x[e] * rq;
-                const __half hi = __float2half_rn(u);
-                qh[h * D + lane * 4 + e] = hi;
-                ql[h * D + lane * 4 + e] = __float2half_rn(u - __half2float(hi));
+            for (int e2 = 0; e2 < 2; ++e2) {
+                const float u0 = x[2 * e2] * rq, u1 = x[2 * e2 + 1] * rq;
+                const __half2 hi = __floats2half2_rn(u0, u1);
+                const float2 hf = __half22float2(hi);
+                const __half2 lo = __floats2half2_rn(u0 - hf.x, u1 - hf.y);
+                hw[e2] = *reinterpret_cast<const uint32_t*>(&hi);
+                lw[e2] = *reinterpret_cast<const uint32_t*>(&lo);
             }
+            *reinterpret_cast<uint2*>(qh + h * QH_STRIDE + lane * 4) = make_uint2(hw[0], hw[1]);
+            *reinterpret_cast<uint2*>(ql + h * QH_STRIDE + lane * 4) = make_uint2(lw[0], lw[1]);
             float smax = 1.f;
             if constexpr (QJL) {
                 // S q~ for sketch rows lane and lane + 32 (m <= 64); q~ staged in
@@ -644,8 +654,8 @@ struct Consumer {
                 }
                 const float sm = group_max<32>(fmaxf(fabsf(sv[0]), fabsf(sv[1])));
                 smax = sm > 0.f ? sm : 1.f;
-                sq[h * 64 + lane] = __float2half_rn(sv[0] / smax);
-                sq[h * 64 + lane + 32] = __float2half_rn(sv[1] / smax);
+                sq[h * SQ_STRIDE + lane] = __float2half_rn(sv[0] / smax);
+                sq[h * SQ_STRIDE + lane + 32] = __float2half_rn(sv[1] / smax);
             }
             if (lane == 0) {
                 fac[h] = h < G ? a.sm_scale_log2 * qmax * a.inv_alpha_k : 0.f;
@@ -668,8 +678,8 @@ struct Consumer {
         ptx::named_barrier(1, NUM_CONSUMERS);  // every warp is done with the query slot
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const __half* qrow = qh + (nt * 8 + g) * D + 32 * t;
-            const __half* lrow = ql + (nt * 8 + g) * D + 32 * t;
+            const __half* qrow = qh + (nt * 8 + g) * QH_STRIDE + 32 * t;
+            const __half* lrow = ql + (nt * 8 + g) * QH_STRIDE + 32 * t;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const uint2 hv = *reinterpret_cast<const uint2*>(qrow + 4 * j);
@@ -680,7 +690,7 @@ struct Consumer {
                 bq[nt][j][3] = lv.y;
             }
             if constexpr (QJL) {
-                const __half* srow = sq + (nt * 8 + g) * 64 + 16 * t;
+                const __half* srow = sq + (nt * 8 + g) * SQ_STRIDE + 16 * t;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     bz[nt][j][0] = *reinterpret_cast<const uint32_t*>(srow + 4 * j);

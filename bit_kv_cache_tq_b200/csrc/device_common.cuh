@@ -47,6 +47,27 @@ __device__ __forceinline__ void load8_stream(const void* base, size_t elem_off, 
     }
 }
 
+// Four consecutive elements (16-byte aligned for fp32, 8-byte otherwise) in
+// any of the three dtypes, as fp32.
+__device__ __forceinline__ void load4(const void* base, size_t off, int dtype, float (&out)[4]) {
+    if (dtype == 0) {
+        const float4 v = *reinterpret_cast<const float4*>(static_cast<const float*>(base) + off);
+        out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+        return;
+    }
+    const uint2 w = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(base) + off);
+    if (dtype == 1) {  // bf16: the upper half of an fp32
+        out[0] = __uint_as_float(w.x << 16);
+        out[1] = __uint_as_float(w.x & 0xffff0000u);
+        out[2] = __uint_as_float(w.y << 16);
+        out[3] = __uint_as_float(w.y & 0xffff0000u);
+    } else {
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+        out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
+    }
+}
+
 // One scalar of a query in any of the three dtypes.
 __device__ __forceinline__ float load_scalar(const void* base, size_t off, int dtype) {
     if (dtype == 0) return static_cast<const float*>(base)[off];
