@@ -367,7 +367,10 @@ def run_tq(args, world, rank, local):
     cap = CONTEXT + total_steps + 1
     gen_seed = rank_seed(rank)
     kcb, vcb = tq.tq_codebook_init(D, K_BITS), tq.tq_codebook_init(D, V_BITS)
-    params = [tq.make_params(D, HQ, HKV, K_BITS, V_BITS, seed=gen_seed + l) for l in range(LAYERS)]
+    # each layer's kernel follows another layer's on the stream, which never
+    # writes this layer's cache: the decode may start streaming it early
+    params = [tq.make_params(D, HQ, HKV, K_BITS, V_BITS, seed=gen_seed + l, flags=tq.TQ_PARAM_PREFETCH_EARLY)
+              for l in range(LAYERS)]
     caches = [tq.alloc_cache(p, BATCH, cap, device=dev) for p in params]
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     zero_pos = torch.zeros(BATCH, dtype=torch.int32, device=dev)

@@ -31,8 +31,8 @@
 //    Since sum_c q~_c c[code_c] does not depend on the order of c, channels are
 //    assigned to fragment slots so that each lane's 16-byte load of a key row
 //    feeds its fragments directly (the query uses the same order); tokens of a
-//    tile are permuted the same way on both sides (tau) so that the value
-//    words each lane needs are bank-conflict free.
+//    tile are permuted the same way on both sides (tau) so that neither the
+//    key rows nor the value words a warp reads have bank conflicts.
 //  * The score fragment becomes the second MMA's operand through one movmatrix
 //    transpose per 8x8 block.  The softmax rescales lazily: the running max
 //    used for exp2 only moves (with a warp-wide reduction) when a score exceeds
@@ -109,6 +109,7 @@ struct Args {
     uint16_t vcent[16];  // fp16 bits of alpha_v * value centroid
     // append mode: one new token per sequence, written at position seq_len - 1
     int append, new_dtype, new_bytes;
+    int early;           // TQ_PARAM_PREFETCH_EARLY: the first chunk may be read before the previous kernel ends
     const void* k_new;   // [batch][1][Hkv][d]
     const void* v_new;
     float kbound[8];     // positive decision boundaries, ascending (unused ones +inf)
@@ -158,14 +159,22 @@ __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int
     if (8u * nt * D * 4 > merge) merge = 8 * nt * D * 4;
     if (768u * 4 > merge) merge = 768 * 4;
     L.ml = L.merge + align16(merge);                   // float2 [CW][16]
-    L.bars = L.ml + CW * 16 * 8;                       // u64 full[8], empty[8], qfull[2], qempty[2]
-    L.flags = L.bars + 20 * 8;                         // int abort, last
+    L.bars = L.ml + CW * 16 * 8;                       // u64 full[8], empty[8], qfull[2], qempty[2], q0
+    L.flags = L.bars + 21 * 8;                         // int abort, last
     L.total = L.flags + 16;
     return L;
 }
 
-// Physical token (within a 16-token tile) of logical MMA row r.
-__device__ __forceinline__ int tau_row(int r) { return (r & 8) + (r & 1) * 4 + ((r & 7) >> 1); }
+// Physical token (within a 16-token tile) of logical MMA row r: even rows
+// 2i -> i, odd rows 2i+1 -> 4 + (i ^ 1), plus 8 for rows 8..15.  The value
+// words a lane reads (rows 2t, 2t+1, 2t+8, 2t+9: tokens t, 4 + (t ^ 1), 8 + t,
+// 12 + (t ^ 1)) fall in four distinct bank groups, and the two key rows a
+// quarter-warp reads (rows 2q, 2q+1) lie an odd number of 64-byte rows apart,
+// so neither read has bank conflicts.
+__device__ __forceinline__ int tau_row(int r) {
+    const int i = (r & 7) >> 1;
+    return (r & 8) + ((r & 1) ? 4 + (i ^ 1) : i);
+}
 
 struct Item {
     int unit, split, b, kv, s0, s1, len;
@@ -278,17 +287,27 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
     // length is read, so the first bytes arrive a DRAM round trip sooner.  If
     // the item turns out empty, its header tells the consumers to drain that
     // stage; if shorter, they only read its valid part.
+    // With TQ_PARAM_PREFETCH_EARLY the first chunk is even requested before
+    // the previous kernel on the stream has finished (the caller promises it
+    // does not write this cache; in append mode the step's own new token is
+    // patched in from its staged rows), so it streams in while the previous
+    // layer's blocks drain.  Queries, lengths and everything else wait.
     int i = blockIdx.x;
-    bool first = true, spec = false;
-    if (i < a.n_items && !*abort_flag) {
-        const int unit = i / a.n_split, split = i % a.n_split;
-        const int b = unit / a.hkv, kv = unit % a.hkv, s0 = split * a.split_len;
-        const uint32_t qf = qfull0;  // query slot 0
-        ptx::mbar_expect_tx(qf, qbytes);
+    bool first = true, spec = false, q0_issued = false;
+    const bool have_first = i < a.n_items;
+    const int unit0 = i / a.n_split, split0 = i % a.n_split;
+    const int s00 = split0 * a.split_len;
+    if (have_first && a.early && !*abort_flag) spec = issue_chunk(unit0, s00, min(CHUNK, a.capacity - s00));
+    ptx::wait_prerequisites();
+    if (have_first && !*abort_flag) {
+        const int b = unit0 / a.hkv, kv = unit0 % a.hkv;
+        const uint32_t q0 = full0 + 160;  // its own barrier: consumers rotate before the header lands
+        ptx::mbar_arrive_expect_tx(q0, qbytes);
         ptx::bulk_copy_g2s(ptx::smem_addr(smem + L.qring) + QHDR,
                            static_cast<const uint8_t*>(a.q) + (static_cast<size_t>(b) * a.hq + kv * G) * D * a.q_bytes,
-                           qbytes, qf);
-        spec = issue_chunk(unit, s0, min(CHUNK, a.capacity - s0));
+                           qbytes, q0);
+        q0_issued = true;
+        if (!a.early) spec = issue_chunk(unit0, s00, min(CHUNK, a.capacity - s00));
     }
     while (ok) {
         if (i >= a.n_items) break;
@@ -341,6 +360,7 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
     for (int j = max(0, seq - a.stages); j < seq; ++j)
         ptx::mbar_wait_bounded(full0 + 8 * (j % a.stages), (j / a.stages) & 1, WAIT_LIMIT);
     for (int j = max(0, qseq - 2); j < qseq; ++j) ptx::mbar_wait_bounded(qfull0 + 8 * (j & 1), (j >> 1) & 1, WAIT_LIMIT);
+    if (q0_issued) ptx::mbar_wait_bounded(full0 + 160, 0, WAIT_LIMIT);
 }
 
 // ----------------------------------------------------------------- consumers
@@ -368,11 +388,12 @@ __device__ __forceinline__ void value_fragments(uint32_t vst, uint32_t base, int
                                                 uint32_t (&A)[8][4]) {
     constexpr int VBV = 16 * VB;
     if constexpr (VB == 2) {
-        // word g of physical tokens t, 4+t, 8+t, 12+t (logical k = 2t, 2t+1, 2t+8, 2t+9)
+        // word g of physical tokens t, 4 + (t ^ 1), 8 + t, 12 + (t ^ 1)
+        // (logical k = 2t, 2t+1, 2t+8, 2t+9)
         const uint32_t w0 = ptx::lds32(vst + t * VBV + 4 * g);
-        const uint32_t w1 = ptx::lds32(vst + (4 + t) * VBV + 4 * g);
+        const uint32_t w1 = ptx::lds32(vst + (4 + (t ^ 1)) * VBV + 4 * g);
         const uint32_t w2 = ptx::lds32(vst + (8 + t) * VBV + 4 * g);
-        const uint32_t w3 = ptx::lds32(vst + (12 + t) * VBV + 4 * g);
+        const uint32_t w3 = ptx::lds32(vst + (12 + (t ^ 1)) * VBV + 4 * g);
         // Nibble n of a word holds channels 16g+2n (bits 0-1) and 16g+2n+1
         // (bits 2-3), i.e. rows g and g+8 of m-tile n.  Interleaving the nibbles
         // of the two tokens gives bytes (token a nibble | token b nibble << 4);
@@ -400,7 +421,7 @@ __device__ __forceinline__ void value_fragments(uint32_t vst, uint32_t base, int
         uint32_t seg[4][2];
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
-            const int tok = 4 * k4 + t;
+            const int tok = 4 * k4 + ((k4 & 1) ? (t ^ 1) : t);  // tau of logical k = 2t, 2t+1, 2t+8, 2t+9
             const uint32_t byte_off = 2 * VB * g;
             const uint32_t wbase = byte_off >> 2, wsh = (byte_off & 3) * 8;
             const uint32_t lo = ptx::lds32(vst + tok * VBV + 4 * wbase);
@@ -593,8 +614,9 @@ struct Consumer {
     }
 
     // The item's queries are in query slot `qseq` (already waited for).
-    __device__ void prologue(int qseq, const Item& w, bool app, uint32_t (&bq)[NT][8][4], uint32_t (&bz)[NT][4][2],
-                             float (&f1)[NT][2], float (&f2)[NT][2]) {
+    // Rotate the queries in query slot `qseq` into the fp16 fragment buffers
+    // and the score factors (no barrier; the prologue's barrier publishes them).
+    __device__ void rotate(int qseq) {
         const int G = a.group;
         const uint8_t* qsrc = smem + L.qring + (qseq & 1) * L.qslot + QHDR;
         __half* qh = reinterpret_cast<__half*>(smem + L.qh);
@@ -662,6 +684,17 @@ struct Consumer {
                 fac[16 + h] = (QJL && h < G) ? a.sm_scale_log2 * 1.2533141373155003f / a.m * smax : 0.f;
             }
         }
+    }
+
+    // Item start: the queries (rotated here unless `rotated`), the appended
+    // token's encoding (append mode), then every warp's query fragments.
+    __device__ void prologue(int qseq, bool rotated, const Item& w, bool app, uint32_t (&bq)[NT][8][4],
+                             uint32_t (&bz)[NT][4][2], float (&f1)[NT][2], float (&f2)[NT][2]) {
+        if (!rotated) rotate(qseq);
+        __half* qh = reinterpret_cast<__half*>(smem + L.qh);
+        __half* ql = reinterpret_cast<__half*>(smem + L.qlo);
+        __half* sq = reinterpret_cast<__half*>(smem + L.sq);
+        float* fac = reinterpret_cast<float*>(smem + L.fac);
         if (app && warp < 2) {
             const size_t slot = static_cast<size_t>(w.unit) * a.capacity + (w.len - 1);
             const uint8_t* rows = smem + L.qring + (qseq & 1) * L.qslot + L.qrows;
@@ -1071,7 +1104,17 @@ struct Consumer {
         float f1[NT][2], f2[NT][2];
         SoftState<NT> S;
         int seq = 0, qseq = 0;
-        bool done_ok = false;
+        bool done_ok = false, first_rotated = false;
+        // The block's first item: its queries were requested before anything
+        // else and complete on their own barrier, so they are rotated before
+        // the item's header (which waits for the sequence length) arrives.
+        if (static_cast<int>(blockIdx.x) < a.n_items) {
+            if (!ptx::mbar_wait_bounded(base + L.bars + 160, 0, WAIT_LIMIT)) set_abort();
+            if (!aborted()) {
+                rotate(0);
+                first_rotated = true;
+            }
+        }
         while (true) {
             // next item: its header (and queries) in query slot qseq
             if (!ptx::mbar_wait_bounded(qfull0 + 8 * (qseq & 1), (qseq >> 1) & 1, WAIT_LIMIT)) set_abort();
@@ -1102,7 +1145,7 @@ struct Consumer {
                 if (lane == 0) ptx::mbar_arrive(empty0 + 8 * slot);
                 ++seq;
             }
-            if (!empty) prologue(qseq, w, app, bq, bz, f1, f2);  // its named barrier ends the slot's use
+            if (!empty) prologue(qseq, qseq == 0 && first_rotated, w, app, bq, bz, f1, f2);  // ends the slot's use
             else ptx::named_barrier(1, NUM_CONSUMERS);           // every warp has read the header
             if (tid == 0) ptx::mbar_arrive(qempty0 + 8 * (qseq & 1));  // query slot free
             ++qseq;
@@ -1158,14 +1201,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid
             ptx::mbar_init(bars + 128 + 8 * s, 1);
             ptx::mbar_init(bars + 144 + 8 * s, 1);
         }
+        {
+            ptx::mbar_init(bars + 160, 1);  // the first item's queries
+        }
         *reinterpret_cast<int*>(smem + L.flags) = 0;
         ptx::fence_mbar_init();
     }
     __syncthreads();  // mbarriers initialised
     if (threadIdx.x >= NUM_CONSUMERS) {
         if (threadIdx.x == NUM_CONSUMERS) {
-            ptx::wait_prerequisites();  // the cache and queries may come from the previous kernel
-            producer<KB, VB, QJL>(a, smem, L);
+            producer<KB, VB, QJL>(a, smem, L);  // waits for the previous kernel itself
         }
         return;
     }
@@ -1292,6 +1337,7 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     using namespace mmadec;
     Args a{};
     a.append = k_new != nullptr;
+    a.early = (p.flags & TQ_PARAM_PREFETCH_EARLY) ? 1 : 0;
     a.k_new = k_new;
     a.v_new = v_new;
     a.new_dtype = new_dtype;

@@ -202,6 +202,7 @@ tq_status validate_params(const tq_params* p) {
     if (!(std::isfinite(p->sm_scale) && p->sm_scale >= 0.0f)) return TQ_ERR_INVALID_ARG;
     if (!(std::isfinite(p->sparse_v_threshold) && p->sparse_v_threshold >= 0.0f && p->sparse_v_threshold < 1.0f))
         return TQ_ERR_INVALID_ARG;
+    if ((p->flags & ~TQ_PARAM_PREFETCH_EARLY) != 0 || p->reserved != 0) return TQ_ERR_INVALID_ARG;
     return TQ_OK;
 }
 

@@ -24,6 +24,7 @@ TQ_ERR_CUDA, TQ_ERR_TIMEOUT, TQ_ERR_DEVICE, TQ_ERR_ALIGNMENT = 4, 5, 6, 7
 TQ_MODE_TURBO, TQ_MODE_INT8 = 0, 1
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 TQ_DEVERR_POSITION, TQ_DEVERR_SEQLEN = 0x1, 0x2
+TQ_PARAM_PREFETCH_EARLY = 0x1
 
 # every symbol include/tq.h declares
 EXPORTED = (
@@ -54,7 +55,8 @@ class tq_params(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
                 ("k_mode", ctypes.c_int32), ("v_mode", ctypes.c_int32), ("k_bits", ctypes.c_int32),
                 ("v_bits", ctypes.c_int32), ("qjl_dims", ctypes.c_int32), ("seed", ctypes.c_uint64),
-                ("sm_scale", ctypes.c_float), ("sparse_v_threshold", ctypes.c_float)]
+                ("sm_scale", ctypes.c_float), ("sparse_v_threshold", ctypes.c_float),
+                ("flags", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
 
 
 class tq_cache(ctypes.Structure):
@@ -157,9 +159,9 @@ def tq_qjl_matrix(seed, m, head_dim):
 
 
 def make_params(head_dim, num_q_heads, num_kv_heads, k_bits=4, v_bits=2, k_mode=TQ_MODE_TURBO,
-                v_mode=TQ_MODE_TURBO, qjl_dims=0, seed=0, sm_scale=0.0, sparse_v_threshold=0.0):
+                v_mode=TQ_MODE_TURBO, qjl_dims=0, seed=0, sm_scale=0.0, sparse_v_threshold=0.0, flags=0):
     return tq_params(head_dim, num_q_heads, num_kv_heads, k_mode, v_mode, k_bits, v_bits, qjl_dims, seed,
-                     sm_scale, sparse_v_threshold)
+                     sm_scale, sparse_v_threshold, flags, 0)
 
 
 def tq_cache_bytes(params, batch, capacity):

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 1
+#define TQ_ABI_VERSION 2
 
 typedef enum tq_status {
     TQ_OK = 0,
@@ -112,7 +112,18 @@ typedef struct tq_codebook {
  *                       otherwise positions whose softmax weight is provably
  *                       below it may be left out of the V sum (see
  *                       tq_decode_attention).
+ *   flags               TQ_PARAM_* bits; 0 for none.
+ *
+ * TQ_PARAM_PREFETCH_EARLY: the caller promises that the kernel launched just
+ * before a decode call on the same stream does not write this layer's cache
+ * (nor does anything else still running).  Decode kernels are launched as
+ * programmatic dependents of that kernel; with this flag they start streaming
+ * the cache before it has finished (queries, new rows, lengths and every
+ * write still wait for it), which hides most of their start-up behind the
+ * previous layer's tail.  Without the flag nothing is read early.
  */
+#define TQ_PARAM_PREFETCH_EARLY 0x1u
+
 typedef struct tq_params {
     int32_t head_dim;
     int32_t num_q_heads;
@@ -125,6 +136,8 @@ typedef struct tq_params {
     uint64_t seed;
     float sm_scale;
     float sparse_v_threshold;
+    uint32_t flags;
+    uint32_t reserved;  /* 0 */
 } tq_params;
 
 /*

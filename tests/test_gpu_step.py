@@ -131,3 +131,37 @@ def test_step_bad_length_is_reported():
     layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=49)
     cache, got, st, word, _ = _step_case(layer, 256, [256, 0, 999], seed=49)
     assert st == tq.TQ_ERR_DEVICE and word & tq.TQ_DEVERR_SEQLEN
+
+
+def test_early_prefetch_flag_same_results():
+    """TQ_PARAM_PREFETCH_EARLY: two layers' steps alternate on one stream (the
+    kernel before each call writes the other layer's cache, as the flag
+    requires); every output equals the same sequence run without the flag."""
+    t, steps = 1500, 3
+    outs = {}
+    for flags in (0, tq.TQ_PARAM_PREFETCH_EARLY):
+        layers = [H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=60 + l) for l in range(2)]
+        for layer in layers:
+            layer.params.flags = flags
+        ks = [inputs.lognormal_kv(1, t, 8, 128, seed=61, layer=l, which=inputs.K) for l in range(2)]
+        vs = [inputs.lognormal_kv(1, t, 8, 128, seed=61, layer=l, which=inputs.V) for l in range(2)]
+        caches = [H.gpu_quantize(layers[l], ks[l][:, : t - steps], vs[l][:, : t - steps], t)[0] for l in range(2)]
+        torch.cuda.synchronize()
+        ws = torch.zeros(tq.tq_decode_workspace_bytes(layers[0].params, 1, t), dtype=torch.uint8, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        res = []
+        for i in range(steps):
+            n = t - steps + i + 1
+            lens = torch.tensor([n], dtype=torch.int32, device="cuda")
+            for l in range(2):
+                q = inputs.queries(1, 32, 128, seed=62, layer=l, step=i).cuda()
+                out = torch.empty(1, 32, 128, dtype=torch.float32, device="cuda")
+                tq.tq_append_decode_attention(layers[l].params, layers[l].kcb, layers[l].vcb,
+                                              ks[l][:, n - 1:n].cuda(), vs[l][:, n - 1:n].cuda(), q, caches[l],
+                                              lens, t, out, ws, err)
+                res.append(out)
+        st, word = tq.tq_read_device_error(err)
+        assert st == tq.TQ_OK and word == 0
+        outs[flags] = [r.cpu().numpy() for r in res]
+    for a, b in zip(outs[0], outs[tq.TQ_PARAM_PREFETCH_EARLY]):
+        assert np.array_equal(a, b)

@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert tq.tq_abi_version() == 1
+    assert tq.tq_abi_version() == 2
     for st in range(8):
         assert tq.tq_status_string(st)
     assert tq.tq_status_string(99) == "unknown status"
@@ -134,7 +134,8 @@ def test_workspace_bound_grows_with_length_and_batch():
     ("k_bits", 5, tq.TQ_ERR_INVALID_ARG), ("v_bits", 1, tq.TQ_ERR_INVALID_ARG),
     ("qjl_dims", 48, tq.TQ_ERR_INVALID_ARG), ("qjl_dims", 512, tq.TQ_ERR_INVALID_ARG),
     ("k_mode", 3, tq.TQ_ERR_INVALID_ARG), ("sm_scale", -1.0, tq.TQ_ERR_INVALID_ARG),
-    ("sparse_v_threshold", 1.5, tq.TQ_ERR_INVALID_ARG),
+    ("sparse_v_threshold", 1.5, tq.TQ_ERR_INVALID_ARG), ("flags", 0x2, tq.TQ_ERR_INVALID_ARG),
+    ("reserved", 1, tq.TQ_ERR_INVALID_ARG),
 ])
 def test_params_validation(field, value, status):
     p = tq.make_params(128, 32, 8)
