@@ -743,8 +743,11 @@ struct Consumer {
                           const uint32_t (&bz)[NT][4][2], const float (&f1)[NT][2], const float (&f2)[NT][2],
                           SoftState<NT>& S) {
         constexpr int VBK = 16 * KB, VBV = 16 * VB;
-        const int lb = 32 * warp;  // first chunk-local token of this warp
-        if (MASK && t0 + lb >= w.s1) return;  // nothing of this warp's range is valid
+        // this warp's tiles are k * CW + warp (k < TPW): a short last chunk
+        // spreads over many warps instead of keeping two tiles on a few
+        const int lb = 16 * warp;  // first chunk-local token of this warp's first tile
+        constexpr int TS = 16 * CW;  // token distance between a warp's tiles
+        if (MASK && t0 + lb >= w.s1) return;  // nothing of this warp's tiles is valid
         const uint32_t sbase = ptx::smem_addr(st);
         const int ra = tau_row(g), rb = tau_row(g + 8);
         const int zw = a.m / 16;
@@ -754,7 +757,15 @@ struct Consumer {
         float vn[TPW][2];
 #pragma unroll
         for (int k = 0; k < TPW; ++k) {
-            const int la = lb + 16 * k + ra, lbb = lb + 16 * k + rb;  // chunk-local tokens of rows g, g+8
+            if (MASK && t0 + lb + TS * k >= w.s1) {  // tile past the item's end (warp-uniform)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) s[k][nt][e] = -INFINITY;
+                vn[k][0] = vn[k][1] = 0.f;
+                continue;
+            }
+            const int la = lb + TS * k + ra, lbb = lb + TS * k + rb;  // chunk-local tokens of rows g, g+8
             const bool va = !MASK || t0 + la < w.s1, vb = !MASK || t0 + lbb < w.s1;
             float kna, knb, ga = 0.f, gb = 0.f;
             uint32_t za = 0, zb2 = 0;
@@ -787,7 +798,7 @@ struct Consumer {
                 }
             }
             // ---- keys: the lane's 4*KB bytes of rows tau(g) and tau(g+8)
-            const uint32_t kst = sbase + L.k_off + (lb + 16 * k) * VBK;
+            const uint32_t kst = sbase + L.k_off + (lb + TS * k) * VBK;
             uint32_t sa[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
             if constexpr (KB == 4) {
                 const uint4 x = ptx::lds128(kst + ra * VBK + 16 * t);
@@ -904,7 +915,7 @@ struct Consumer {
         // ---- values, tile by tile
 #pragma unroll
         for (int k = 0; k < TPW; ++k) {
-            if (MASK && t0 + lb + 16 * k >= w.s1) break;  // warp-uniform
+            if (MASK && t0 + lb + TS * k >= w.s1) break;  // warp-uniform
             float pv[NT][4];
             bool any_v = false;
 #pragma unroll
@@ -935,7 +946,7 @@ struct Consumer {
                 bv[nt][1] = ptx::movmatrix_trans(ptx::pack_half2(pv[nt][2] * wb, pv[nt][3] * wb));
             }
             uint32_t A[8][4];
-            value_fragments<VB>(sbase + L.v_off + (lb + 16 * k) * VBV, base, g, t, laneoff, A);
+            value_fragments<VB>(sbase + L.v_off + (lb + TS * k) * VBV, base, g, t, laneoff, A);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
