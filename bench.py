@@ -358,6 +358,58 @@ def bf16_sdpa_baseline(dev, reps=20):
             "gbs": round(bytes_layer / (us * 1e-6) / 1e9, 1), "bytes_per_layer": bytes_layer}
 
 
+def decode_configs(dev, reps=10):
+    """The decode kernel on the other full-size decode workloads, timed with
+    CUDA events over `reps` calls (caches larger than L2, or cycled copies):
+    batched ragged (B=16, Hq=32, Hkv=8, lengths uniform in [2048, 8192], K3/V2,
+    4 cache copies) and 70B-shaped long context (B=4, Hq=64, Hkv=8, 131072
+    tokens, K3 + 64-bit QJL / V2, Sparse V at 1e-6)."""
+    from bit_kv_cache_tq_b200 import inputs, tq
+    res = {}
+    cases = [("batched_ragged_b16_k3v2", 16, 32, 8192, 3, 0, 0.0, 4),
+             ("long_context_b4_hq64_128k_k3qjl_v2_sparse", 4, 64, 131072, 3, 64, 1e-6, 1)]
+    for name, bsz, hq, tmax, kb, m, tau, copies in cases:
+        p = tq.make_params(D, hq, HKV, k_bits=kb, v_bits=2, qjl_dims=m, seed=SEED, sparse_v_threshold=tau)
+        kcb, vcb = tq.tq_codebook_init(D, kb), tq.tq_codebook_init(D, 2)
+        if bsz == 16:
+            lens = inputs.ragged_lengths(bsz, 2048, 8192, seed=0).tolist()
+        else:
+            lens = [tmax] * bsz
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        pos = torch.zeros(bsz, dtype=torch.int32, device=dev)
+        caches = []
+        for c in range(copies):
+            cache = tq.alloc_cache(p, bsz, tmax, device=dev)
+            k = inputs.lognormal_kv(bsz, tmax, HKV, D, SEED, 40 + c, inputs.K, device=dev)
+            v = inputs.lognormal_kv(bsz, tmax, HKV, D, SEED, 40 + c, inputs.V, device=dev)
+            tq.tq_quantize_append(p, kcb, vcb, k, v, pos, cache, err)
+            del k, v
+            caches.append(cache)
+        q = inputs.queries(bsz, hq, D, SEED, device=dev)
+        lens_t = torch.tensor(lens, dtype=torch.int32, device=dev)
+        ws = torch.zeros(tq.tq_decode_workspace_bytes(p, bsz, tmax), dtype=torch.uint8, device=dev)
+        out = torch.empty(bsz, hq, D, dtype=torch.float32, device=dev)
+        for c in range(copies):
+            tq.tq_decode_attention(p, kcb, vcb, q, caches[c], lens_t, tmax, out, ws, err)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for r in range(reps):
+            tq.tq_decode_attention(p, kcb, vcb, q, caches[r % copies], lens_t, tmax, out, ws, err)
+        e1.record()
+        e1.synchronize()
+        st, word = tq.tq_read_device_error(err)
+        assert st == tq.TQ_OK, (name, st, word)
+        us = 1000.0 * e0.elapsed_time(e1) / reps
+        per_tok = D * kb // 8 + 2 + (m // 8 + 2 if m else 0) + D * 2 // 8 + 2
+        nbytes = sum(lens) * HKV * per_tok
+        res[name] = {"us_per_call": round(us, 2), "kv_tokens_per_s": round(sum(lens) / (us * 1e-6)),
+                     "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "algorithmic_bytes": nbytes,
+                     "bytes_per_token_kv_head": per_tok}
+        del caches, ws
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_tq(args, world, rank, local):
     from bit_kv_cache_tq_b200 import inputs, tq
     dev = torch.device("cuda", local)
@@ -525,6 +577,7 @@ def run_tq(args, world, rank, local):
         }
         if not args.quick:
             line["bf16_baseline"] = bf16_sdpa_baseline(dev)
+            line["decode_configs"] = decode_configs(dev)
             peak_gbs = measured_peaks()[0]
             q = {"workload": "bulk prefill quantise: 262144 tokens x 8 kv heads, bf16, 32 layers (0, 1, 30, 31 "
                              "int8 per-vector absmax, others K4/V3 turbo), one input slab, 32 distinct outputs",

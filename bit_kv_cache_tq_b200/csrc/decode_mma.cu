@@ -79,8 +79,8 @@ constexpr float LAZY = 8.0f;                 // log2 headroom before the running
 constexpr float VRANGE = 64.0f;              // bound on ||v|| * vscale
 
 // header flags: item (query slot) EMPTY / END / APPEND / DRAIN (one stage to
-// consume unread), chunk (stage) LAST
-constexpr int F_LAST = 2, F_EMPTY = 4, F_END = 8, F_APPEND = 16, F_DRAIN = 32;
+// consume unread) / SKIP (no work: only the drain), chunk (stage) LAST
+constexpr int F_LAST = 2, F_EMPTY = 4, F_END = 8, F_APPEND = 16, F_DRAIN = 32, F_SKIP = 64;
 // global counters after the per-(sequence, kv head) split counters
 constexpr int C_ITEM = 0, C_DONE = 1;
 
@@ -180,6 +180,14 @@ struct Item {
     int unit, split, b, kv, s0, s1, len;
     bool bad;  // seq_len out of range: the sequence is treated as empty
 };
+
+// Splits of a unit that hold tokens (at least 1, so an empty sequence still
+// gets its zero output): the merge waits for exactly these; the others are
+// skipped without any work.
+__device__ __forceinline__ int live_splits(const Args& a, int len) {
+    const int n = (len + a.split_len - 1) / a.split_len;
+    return n > 1 ? n : 1;
+}
 
 __device__ __forceinline__ Item item_of(const Args& a, int item) {
     Item it;
@@ -313,6 +321,15 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         if (i >= a.n_items) break;
         const Item w = item_of(a, i);
         if (w.bad && a.err && w.split == 0 && w.kv == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
+        // a dead split holds no token and the merge does not wait for it: skip
+        // it, unless it is the block's first item (its queries and speculative
+        // chunk already fill query slot 0 and a stage; the header then tells
+        // the consumers to release them and do nothing else)
+        const bool dead = w.split >= live_splits(a, w.len);
+        if (dead && !first) {
+            i = static_cast<int>(gridDim.x + atomicAdd(a.counters + a.units + C_ITEM, 1u));
+            continue;
+        }
         const bool empty = w.s0 >= w.s1;
         const bool app = a.append && !empty && w.s1 == w.len;
         uint8_t* qslot;
@@ -320,7 +337,8 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         if (!claim_q(qslot, qfull)) break;
         int4* hdr = reinterpret_cast<int4*>(qslot);
         hdr[0] = make_int4(i, w.s0, w.s1, w.len);
-        hdr[1] = make_int4((empty ? F_EMPTY : 0) | (app ? F_APPEND : 0) | (first && spec && empty ? F_DRAIN : 0),
+        hdr[1] = make_int4((empty ? F_EMPTY : 0) | (app ? F_APPEND : 0) | (first && spec && empty ? F_DRAIN : 0) |
+                               (dead ? F_SKIP : 0),
                            w.unit, w.b, w.kv);
         const uint32_t rbytes = D * a.new_bytes;
         const uint32_t extra = app ? 2 * rbytes : 0u;  // append rows
@@ -1037,8 +1055,9 @@ struct Consumer {
         // thread 0's release, and its acquire orders the merge's reads after
         // the other blocks' partials
         ptx::named_barrier(1, NUM_CONSUMERS);
+        const int nlive = live_splits(a, w.len);  // the splits the merge waits for
         if (tid == 0) *last_flag = ptx::atom_add_acq_rel_gpu(a.counters + w.unit, 1u) ==
-                                   static_cast<uint32_t>(a.n_split - 1);
+                                   static_cast<uint32_t>(nlive - 1);
         ptx::named_barrier(1, NUM_CONSUMERS);
         if (*last_flag) {
             // Merge the splits: two warps per head, each lane two channels.  A
@@ -1056,15 +1075,15 @@ struct Consumer {
                 float2 v[PB];
 #pragma unroll
                 for (int j = 0; j < PB; ++j)
-                    v[j] = j < a.n_split ? __ldcg(src2 + (j * G + h) * (D / 2) + c2) : make_float2(0.f, 0.f);
+                    v[j] = j < nlive ? __ldcg(src2 + (j * G + h) * (D / 2) + c2) : make_float2(0.f, 0.f);
                 float mx = -INFINITY;
-                for (int sp = lane; sp < a.n_split; sp += 32) {
+                for (int sp = lane; sp < nlive; sp += 32) {
                     const float2 m2 = __ldcg(a.ws_ml + ubase + sp * G + h);
                     if (m2.y > 0.f) mx = fmaxf(mx, m2.x);
                 }
                 mx = group_max<32>(mx);
                 float l = 0.f;
-                for (int sp = lane; sp < a.n_split; sp += 32) {
+                for (int sp = lane; sp < nlive; sp += 32) {
                     const float2 m2 = __ldcg(a.ws_ml + ubase + sp * G + h);
                     const float wgt = (m2.y > 0.f && mx > -INFINITY) ? ptx::ex2(m2.x - mx) : 0.f;
                     wts[sp] = wgt;
@@ -1074,16 +1093,16 @@ struct Consumer {
                 const float inv_l = l > 0.f ? 1.f / l : 0.f;
                 __syncwarp();
                 float2 acc = make_float2(0.f, 0.f);
-                for (int s0 = 0; s0 < a.n_split; s0 += PB) {
+                for (int s0 = 0; s0 < nlive; s0 += PB) {
                     if (s0 > 0) {
 #pragma unroll
                         for (int j = 0; j < PB; ++j)
-                            v[j] = s0 + j < a.n_split ? __ldcg(src2 + ((s0 + j) * G + h) * (D / 2) + c2)
+                            v[j] = s0 + j < nlive ? __ldcg(src2 + ((s0 + j) * G + h) * (D / 2) + c2)
                                                       : make_float2(0.f, 0.f);
                     }
 #pragma unroll
                     for (int j = 0; j < PB; ++j) {
-                        const float wgt = s0 + j < a.n_split ? wts[s0 + j] : 0.f;
+                        const float wgt = s0 + j < nlive ? wts[s0 + j] : 0.f;
                         acc.x = fmaf(v[j].x, wgt, acc.x);
                         acc.y = fmaf(v[j].y, wgt, acc.y);
                     }
@@ -1182,7 +1201,7 @@ struct Consumer {
                 if (lane == 0) ptx::mbar_arrive(empty0 + 8 * slot);
                 ++seq;
             }
-            epilogue(w, S);
+            if (!(h1.x & F_SKIP)) epilogue(w, S);
             if (ptx::named_barrier_or(1, NUM_CONSUMERS, aborted())) break;
         }
         if (done_ok && tid == 0) {

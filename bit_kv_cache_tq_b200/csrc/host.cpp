@@ -263,8 +263,9 @@ DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_s
     // Split count.  Few long sequences: one wave of equal items, one per SM,
     // when that keeps at least 85% of the SMs busy (every item then carries
     // one prologue and one merge); otherwise a multiple of the SM count where
-    // possible.  Many sequences (a batch, possibly ragged): about four items
-    // per SM, which the kernel's dynamic scheduling balances.  Splits are never
+    // possible.  Many sequences (a batch, possibly ragged): about two items
+    // per SM, which the kernel's dynamic scheduling balances (splits past a
+    // sequence's end cost nothing).  Splits are never
     // shorter than kMinSplitTokens nor more than kMaxSplits.
     DecodePlan plan;
     const long long units = static_cast<long long>(batch) * p.num_kv_heads;
@@ -273,7 +274,7 @@ DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_s
     long long n;
     const long long one_wave = num_sms / units;
     if (units * 4 >= num_sms) {
-        n = (4ll * num_sms + units - 1) / units;
+        n = (2ll * num_sms + units - 1) / units;
     } else if (one_wave >= 1 && one_wave * units * 100 >= 85ll * num_sms) {
         n = one_wave;
     } else {
