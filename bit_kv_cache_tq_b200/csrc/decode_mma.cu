@@ -223,7 +223,7 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
     // claim a free stage slot (bounded wait); false on abort
     auto claim = [&](uint32_t& full, uint8_t*& st) -> bool {
         const int slot = seq % a.stages, use = seq / a.stages;
-        if (use > 0 && !ptx::mbar_wait_bounded(empty0 + 8 * slot, (use - 1) & 1, WAIT_LIMIT)) {
+        if (use > 0 && !ptx::mbar_wait_bounded_sleep(empty0 + 8 * slot, (use - 1) & 1, WAIT_LIMIT, 100)) {
             fail();
             return false;
         }
@@ -248,7 +248,7 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
     // Empty items take a query slot but no stage.
     auto claim_q = [&](uint8_t*& slot, uint32_t& qfull) -> bool {
         const int qs = qseq & 1;
-        if (qseq >= 2 && !ptx::mbar_wait_bounded(qempty0 + 8 * qs, ((qseq - 2) >> 1) & 1, WAIT_LIMIT)) {
+        if (qseq >= 2 && !ptx::mbar_wait_bounded_sleep(qempty0 + 8 * qs, ((qseq - 2) >> 1) & 1, WAIT_LIMIT, 100)) {
             fail();
             return false;
         }

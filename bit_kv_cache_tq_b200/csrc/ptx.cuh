@@ -55,6 +55,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     return true;
 }
 
+// As mbar_wait_bounded, sleeping `ns` nanoseconds between polls: for a thread
+// that waits most of the time and should leave its scheduler to other warps.
+__device__ __forceinline__ bool mbar_wait_bounded_sleep(uint32_t bar, uint32_t parity, long long limit, unsigned ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long start = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - start > limit) return false;
+        __nanosleep(ns);
+    }
+    return true;
+}
+
 // 1-D bulk copy global -> shared (this CTA), completion counted on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
