@@ -1434,7 +1434,9 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     const Layout fixed = layout(kb, vb, nt, 0, p.qjl_dims, a.group, a.q_bytes, a.append ? a.new_bytes : 0, a.n_split);
     int stages = static_cast<int>((232448u - fixed.total) / fixed.stage_bytes);
     if (stages > 8) stages = 8;
-    if (stages < 2) return cudaErrorInvalidConfiguration;
+    // large groups (16 query heads per kv head) leave no room for two stages
+    // beside the per-warp merge buffers: the caller takes the general kernels
+    if (stages < 2) return cudaErrorNotSupported;
     a.stages = stages;
     const size_t smem =
         layout(kb, vb, nt, stages, p.qjl_dims, a.group, a.q_bytes, a.append ? a.new_bytes : 0, a.n_split).total;

@@ -323,3 +323,16 @@ def test_workspace_reused_across_batches_and_lengths():
         assert st == tq.TQ_OK and word == 0
         fresh, _, _ = H.gpu_decode(layer, qq, cache, lens)
         assert np.array_equal(got, fresh), lens
+
+
+def test_group16_d128():
+    """d = 128 with 16 query heads per kv head (the tensor-core kernel's merge
+    buffers leave no room for its stages, so the general kernels serve it),
+    fp32 queries, ragged lengths, K4/V3."""
+    layer = H.Layer(128, 32, 2, k_bits=4, v_bits=3, seed=23)
+    t = 1100
+    k = inputs.lognormal_kv(2, t, 2, 128, seed=14, layer=23, which=inputs.K)
+    v = inputs.lognormal_kv(2, t, 2, 128, seed=14, layer=23, which=inputs.V)
+    q = inputs.queries(2, 32, 128, seed=14, layer=23, dtype=torch.float32)
+    e2e, same, _, _, _ = _attention_case(layer, k, v, q, [t, 517])
+    assert same.max() < H.ATTN_TOL and e2e.max() < H.ATTN_TOL, (same.max(), e2e.max())
