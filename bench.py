@@ -416,7 +416,8 @@ def run_tq(args, world, rank, local):
     torch.cuda.set_device(dev)
     steps, warmup = args.steps, args.warmup
     total_steps = steps + warmup
-    cap = CONTEXT + total_steps + 1
+    # a capacity that is a multiple of 8 lets the kernel stage norms beside the codes
+    cap = (CONTEXT + total_steps + 1 + 7) // 8 * 8
     gen_seed = rank_seed(rank)
     kcb, vcb = tq.tq_codebook_init(D, K_BITS), tq.tq_codebook_init(D, V_BITS)
     # each layer's kernel follows another layer's on the stream, which never

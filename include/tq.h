@@ -150,6 +150,9 @@ typedef struct tq_params {
  *   k_gamma   [batch][Hkv][capacity]       fp16 residual norm (NULL when qjl_dims == 0)
  *   v_codes, v_norms                       as for K
  *   qjl_matrix [m][d] fp32, row-major      the sketch S (NULL when qjl_dims == 0)
+ * A capacity that is a multiple of 8 lets the decode kernels move the
+ * norms, QJL words and gammas with the codes in their bulk copies; with any
+ * other capacity they read them from global memory in the inner loop.
  * Codes of one vector are one LSB-first bitstream: code i occupies bits
  * [b*i, b*i+b), bit k of the stream is bit k%8 of byte k/8, so 3-bit codes
  * cross byte boundaries ([inferrs] "压缩格式对比", turbo2/3/4).  INT8 codes
