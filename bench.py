@@ -400,11 +400,25 @@ def decode_configs(dev, reps=10):
         st, word = tq.tq_read_device_error(err)
         assert st == tq.TQ_OK, (name, st, word)
         us = 1000.0 * e0.elapsed_time(e1) / reps
+        extra = {}
+        if tau > 0:  # Sparse V's effect: the same call without skipping
+            dense = tq.make_params(D, hq, HKV, k_bits=kb, v_bits=2, qjl_dims=m, seed=SEED)
+            out_d = torch.empty_like(out)
+            tq.tq_decode_attention(p, kcb, vcb, q, caches[0], lens_t, tmax, out, ws, err)
+            tq.tq_decode_attention(dense, kcb, vcb, q, caches[0], lens_t, tmax, out_d, ws, err)
+            rel = ((out - out_d).norm(dim=-1) / out_d.norm(dim=-1)).max().item()
+            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            d0.record()
+            for r in range(reps):
+                tq.tq_decode_attention(dense, kcb, vcb, q, caches[r % copies], lens_t, tmax, out_d, ws, err)
+            d1.record()
+            d1.synchronize()
+            extra = {"max_rel_l2_vs_no_skip": rel, "us_without_sparse_v": round(1000.0 * d0.elapsed_time(d1) / reps, 2)}
         per_tok = D * kb // 8 + 2 + (m // 8 + 2 if m else 0) + D * 2 // 8 + 2
         nbytes = sum(lens) * HKV * per_tok
         res[name] = {"us_per_call": round(us, 2), "kv_tokens_per_s": round(sum(lens) / (us * 1e-6)),
                      "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "algorithmic_bytes": nbytes,
-                     "bytes_per_token_kv_head": per_tok}
+                     "bytes_per_token_kv_head": per_tok, **extra}
         del caches, ws
         torch.cuda.empty_cache()
     return res

@@ -101,11 +101,11 @@ template <int N, int SPAN>
 __device__ __forceinline__ void fwht_lanes(float (&v)[N], int sub) {
 #pragma unroll
     for (int m = 1; m < SPAN; m <<= 1) {
-        const bool upper = sub & m;
+        const float sg = (sub & m) ? -1.0f : 1.0f;  // upper lane: p - v, lower lane: v + p (one rounding)
 #pragma unroll
         for (int i = 0; i < N; ++i) {
             const float p = __shfl_xor_sync(kFullMask, v[i], m);
-            v[i] = upper ? (p - v[i]) : (v[i] + p);
+            v[i] = fmaf(v[i], sg, p);
         }
     }
 }
