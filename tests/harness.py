@@ -193,7 +193,7 @@ def gpu_decode(layer, q, cache, lens, max_len=None, ws=None):
 def stored_hat(layer, cache, b, h, n, which):
     """The oracle's reconstruction of the GPU's own stored bytes (codes, norms,
     QJL bits, gamma) for tokens [0, n) of sequence b, kv head h: attention
-    parity is judged on the same codes, after code parity has passed."""
+    parity is measured on the same codes, after code parity has passed."""
     mode, bits = layer.side(which)
     if which == 0:
         raw, nrm = cache.k_codes[b, h, :n].cpu().numpy(), cache.k_norms[b, h, :n].cpu().numpy()

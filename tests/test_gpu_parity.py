@@ -69,7 +69,7 @@ def _attention_case(layer, kx, vx, q, lens, tau=0.0):
     vhat = _oracle_hat(layer, enc[1], 1, (bsz, hkv, t, d))
     ref = H.oracle_attention(layer, _to_np(q), khat, vhat, lens, tau)
     want = ref["out"] if tau == 0 else ref["exact_sparse"]
-    # (a) end to end, judged on the GPU's own stored codes (code parity passed above)
+    # (a) end to end, compared on the GPU's own stored codes (code parity passed above)
     got, st, word = H.gpu_decode(layer, q, cache, lens)
     assert st == tq.TQ_OK and word == 0
     ks = np.stack([np.stack([H.stored_hat(layer, cache, b, h, t, 0) for h in range(hkv)]) for b in range(bsz)])
