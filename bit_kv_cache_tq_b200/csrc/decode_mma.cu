@@ -1013,34 +1013,25 @@ struct Consumer {
             }
         ptx::named_barrier(1, NUM_CONSUMERS);
         const size_t pbase = (static_cast<size_t>(w.unit) * a.n_split + w.split) * G;
-        // per head: the warps' weights 2^(m_w - M) (in place of m_w) and the
-        // split's (M, L); then every output column is one weighted sum
-        if (tid < G) {
-            const int h = tid;
-            float mx = -INFINITY;
-#pragma unroll
-            for (int ww = 0; ww < CW; ++ww)
-                if (ml[ww * 16 + h].y > 0.f) mx = fmaxf(mx, ml[ww * 16 + h].x);
-            float l = 0.f;
-#pragma unroll
-            for (int ww = 0; ww < CW; ++ww) {
-                const float2 v = ml[ww * 16 + h];
-                const float f = (v.y > 0.f && mx > -INFINITY) ? ptx::ex2(v.x - mx) : 0.f;
-                l = fmaf(v.y, f, l);
-                ml[ww * 16 + h].x = f;
-            }
-            a.ws_ml[pbase + h] = make_float2(mx, l);
-        }
-        ptx::named_barrier(1, NUM_CONSUMERS);
+        // every output column is one weighted sum over the warps, with the
+        // weights 2^(m_w - M) of its head (each thread forms them; the thread
+        // of a head's first column also writes the split's (M, L))
         {
             const float4* m4 = reinterpret_cast<const float4*>(merge);
             float4* dst4 = reinterpret_cast<float4*>(a.ws_acc + pbase * D);
             for (int idx = tid; idx < G * (D / 4); idx += NUM_CONSUMERS) {
                 const int h = idx / (D / 4), c4 = idx % (D / 4);
+                float mx = -INFINITY;
+#pragma unroll
+                for (int ww = 0; ww < CW; ++ww)
+                    if (ml[ww * 16 + h].y > 0.f) mx = fmaxf(mx, ml[ww * 16 + h].x);
                 float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                float l = 0.f;
 #pragma unroll
                 for (int ww = 0; ww < CW; ++ww) {
-                    const float f = ml[ww * 16 + h].x;
+                    const float2 mlw = ml[ww * 16 + h];
+                    const float f = (mlw.y > 0.f && mx > -INFINITY) ? ptx::ex2(mlw.x - mx) : 0.f;
+                    l = fmaf(mlw.y, f, l);
                     const float4 v = m4[(ww * G + h) * (D / 4) + c4];
                     acc4.x = fmaf(v.x, f, acc4.x);
                     acc4.y = fmaf(v.y, f, acc4.y);
@@ -1049,6 +1040,7 @@ struct Consumer {
                 }
                 const float iv = a.inv_alpha_v;  // undo the centroid scale
                 dst4[h * (D / 4) + c4] = make_float4(acc4.x * iv, acc4.y * iv, acc4.z * iv, acc4.w * iv);
+                if (c4 == 0) a.ws_ml[pbase + h] = make_float2(mx, l);
             }
         }
         // publish the partial: the barrier orders every thread's writes before
