@@ -14,20 +14,28 @@
 //   domain, and one inverse rotation of acc / sum_i p_i.
 //
 // How (one persistent thread block per SM):
-//  * Work items are (sequence, kv head, token split).  A producer warp takes
-//    items from a global atomic counter (so ragged batches balance), and for
-//    each one streams the packed K and V codes (plus norms, QJL words and the
-//    queries) of 256-token chunks into a ring of shared-memory stages with 1-D
-//    bulk async copies (TMA engine, no multicast).  Each stage starts with a
-//    header naming its item and token range; completion is tracked by
-//    mbarriers.  Eight consumer warps take two 16-token tiles of every chunk.
+//  * Work items are (sequence, kv head, token split).  A producer thread takes
+//    items (the block's first one statically, the rest from a global atomic
+//    counter, so ragged batches balance; splits past a sequence's end are
+//    skipped).  For each item it writes a header (range, length, flags) into
+//    the next of two query slots and bulk-copies the item's queries behind it
+//    (plus, in append mode, the step's new key and value rows), then streams
+//    the packed K and V codes, norms and QJL words of 352-token chunks into a
+//    ring of shared-memory stages with 1-D bulk async copies (TMA engine, no
+//    multicast), completion tracked by mbarriers.  The block's first chunk and
+//    queries are requested before the sequence lengths are read.
+//  * Eleven consumer warps each take two 16-token tiles of every chunk (tiles
+//    CW apart, so a short last chunk spreads over many warps); each warp waits
+//    for a stage on its own, with no block barrier per chunk.
 //  * The dequantised tiles of a GQA group form real dense products, so both
 //    contractions run on the tensor cores with warp-level m16n8k16 fp16 MMA
 //    (fp32 accumulate):  S^T[16 tok x 8 heads] = K~[16 x 128] Q~^T and
-//    O^T[128 x 8 heads] += V~^T[128 x 16 tok] P^T.  The A operands are built
-//    in registers straight from the codes: a 256-entry, per-lane replicated
-//    shared-memory table maps one byte of 4-bit key codes to a pair of fp16
-//    centroids, and a register byte-permute table maps 2-bit value codes.
+//    O^T[128 x 8 heads] += V~^T[128 x 16 tok] P^T.  The query enters as two
+//    fp16 terms (hi + lo), so the scores keep about 22 bits of it.  The A
+//    operands are built in registers straight from the codes through a
+//    per-lane replicated shared-memory table: one byte of 4-bit key codes
+//    gives a pair of fp16 centroids, one byte of 2-bit value codes (two
+//    tokens, two channels) gives two pairs.
 //    Since sum_c q~_c c[code_c] does not depend on the order of c, channels are
 //    assigned to fragment slots so that each lane's 16-byte load of a key row
 //    feeds its fragments directly (the query uses the same order); tokens of a
@@ -38,11 +46,12 @@
 //    used for exp2 only moves (with a warp-wide reduction) when a score exceeds
 //    it by more than 2^8, decided by one warp vote per chunk.
 //  * Split results are merged by the last block to finish a (sequence, kv
-//    head), found with an atomic counter (no spin-wait); it also applies the
-//    inverse rotation and writes the output.
+//    head), found with one acquire-release atomic per split (no spin-wait);
+//    it also applies the inverse rotation and writes the output.
 //  Every wait on an mbarrier is bounded (about a second); a wait that runs out
-//  sets TQ_DEVERR_TIMEOUT, all consumer warps agree on it at the next named
-//  barrier, and the block leaves after draining its copies.
+//  sets TQ_DEVERR_TIMEOUT and later waits are skipped; the consumer warps take
+//  the same abort decision at the item boundaries (a barrier with an OR
+//  reduction), and the block leaves after draining its copies.
 
 #include <cuda_runtime.h>
 
