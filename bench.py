@@ -362,15 +362,23 @@ def decode_configs(dev, reps=10):
     """The decode kernel on the other full-size decode workloads, timed with
     CUDA events over `reps` calls (caches larger than L2, or cycled copies):
     batched ragged (B=16, Hq=32, Hkv=8, lengths uniform in [2048, 8192], K3/V2,
-    4 cache copies) and 70B-shaped long context (B=4, Hq=64, Hkv=8, 131072
-    tokens, K3 + 64-bit QJL / V2, Sparse V at 1e-6)."""
+    4 cache copies), 70B-shaped long context (B=4, Hq=64, Hkv=8, 131072
+    tokens, K3 + 64-bit QJL / V2, Sparse V at 1e-6), and the Llama-3-8B-shaped
+    layer (B=1, 32768 tokens, 4 cache copies) with int8 keys and 2-bit values
+    (the mixed setting) and as an int8 boundary layer (int8 keys and values).
+    A kb of 8 below stands for int8 (one byte per channel, fp16 scale)."""
     from bit_kv_cache_tq_b200 import inputs, tq
     res = {}
-    cases = [("batched_ragged_b16_k3v2", 16, 32, 8192, 3, 0, 0.0, 4),
-             ("long_context_b4_hq64_128k_k3qjl_v2_sparse", 4, 64, 131072, 3, 64, 1e-6, 1)]
-    for name, bsz, hq, tmax, kb, m, tau, copies in cases:
-        p = tq.make_params(D, hq, HKV, k_bits=kb, v_bits=2, qjl_dims=m, seed=SEED, sparse_v_threshold=tau)
-        kcb, vcb = tq.tq_codebook_init(D, kb), tq.tq_codebook_init(D, 2)
+    cases = [("batched_ragged_b16_k3v2", 16, 32, 8192, 3, 2, 0, 0.0, 4),
+             ("long_context_b4_hq64_128k_k3qjl_v2_sparse", 4, 64, 131072, 3, 2, 64, 1e-6, 1),
+             ("llama8b_32k_int8k_v2", 1, 32, 32768, 8, 2, 0, 0.0, 4),
+             ("llama8b_32k_int8k_int8v", 1, 32, 32768, 8, 8, 0, 0.0, 4)]
+    for name, bsz, hq, tmax, kb, vb, m, tau, copies in cases:
+        modes = dict(k_mode=tq.TQ_MODE_INT8 if kb == 8 else tq.TQ_MODE_TURBO,
+                     v_mode=tq.TQ_MODE_INT8 if vb == 8 else tq.TQ_MODE_TURBO,
+                     k_bits=4 if kb == 8 else kb, v_bits=2 if vb == 8 else vb)
+        p = tq.make_params(D, hq, HKV, qjl_dims=m, seed=SEED, sparse_v_threshold=tau, **modes)
+        kcb, vcb = tq.tq_codebook_init(D, modes["k_bits"]), tq.tq_codebook_init(D, modes["v_bits"])
         if bsz == 16:
             lens = inputs.ragged_lengths(bsz, 2048, 8192, seed=0).tolist()
         else:
@@ -402,7 +410,7 @@ def decode_configs(dev, reps=10):
         us = 1000.0 * e0.elapsed_time(e1) / reps
         extra = {}
         if tau > 0:  # Sparse V's effect: the same call without skipping
-            dense = tq.make_params(D, hq, HKV, k_bits=kb, v_bits=2, qjl_dims=m, seed=SEED)
+            dense = tq.make_params(D, hq, HKV, qjl_dims=m, seed=SEED, **modes)
             out_d = torch.empty_like(out)
             tq.tq_decode_attention(p, kcb, vcb, q, caches[0], lens_t, tmax, out, ws, err)
             tq.tq_decode_attention(dense, kcb, vcb, q, caches[0], lens_t, tmax, out_d, ws, err)
@@ -414,7 +422,7 @@ def decode_configs(dev, reps=10):
             d1.record()
             d1.synchronize()
             extra = {"max_rel_l2_vs_no_skip": rel, "us_without_sparse_v": round(1000.0 * d0.elapsed_time(d1) / reps, 2)}
-        per_tok = D * kb // 8 + 2 + (m // 8 + 2 if m else 0) + D * 2 // 8 + 2
+        per_tok = D * kb // 8 + 2 + (m // 8 + 2 if m else 0) + D * vb // 8 + 2
         nbytes = sum(lens) * HKV * per_tok
         res[name] = {"us_per_call": round(us, 2), "kv_tokens_per_s": round(sum(lens) / (us * 1e-6)),
                      "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "algorithmic_bytes": nbytes,

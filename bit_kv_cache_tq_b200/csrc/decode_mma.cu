@@ -81,7 +81,15 @@ constexpr uint32_t QHDR = 32;                 // item header at the front of a q
 // groups g = 0..3 at rows g, columns 16 t) hit 32 distinct banks.
 constexpr int QH_STRIDE = D + 4;
 constexpr int SQ_STRIDE = 64 + 4;
-constexpr uint32_t APP_BYTES = 1024;          // the appended token's codes and scratch
+// the appended token's patch area: packed key row (up to 128 B: int8 keys),
+// packed value row, key norm, value norm, gamma, sketch words, then the
+// encoders' scratch (code bytes of each side, the key residual)
+constexpr uint32_t AP_K = 0, AP_V = 128, AP_KN = 256, AP_VN = 258, AP_GAM = 260, AP_Z = 264, AP_KC = 288,
+                   AP_VC = 416, AP_R = 544;
+constexpr uint32_t APP_BYTES = AP_R + 4 * D;
+// key side in int8 mode (one byte per channel, fp16 scale in the norm slot):
+// the kernel's KB template parameter takes this value
+constexpr int KB_INT8 = 8;
 constexpr long long WAIT_LIMIT = 2000000000ll;  // clock cycles (~1 s)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LAZY = 8.0f;                 // log2 headroom before the running max moves
@@ -409,6 +417,20 @@ __device__ __forceinline__ uint32_t key_lut_addr(const uint32_t (&seg)[4], int j
     }
 }
 
+// Four int8 channels (one word, byte i = channel i) as two fp16 pairs, exactly:
+// byte b ^ 0x80 = b + 128 becomes the mantissa of 1024 + (b + 128), and
+// subtracting 1152 leaves b.
+__device__ __forceinline__ void int8_pairs(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    const uint32_t pl = __byte_perm(u, 0x64646464u, 0x5140);  // channels 0, 1
+    const uint32_t ph = __byte_perm(u, 0x64646464u, 0x7362);  // channels 2, 3
+    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+    const __half2 l2 = __hsub2(*reinterpret_cast<const __half2*>(&pl), bias);
+    const __half2 h2 = __hsub2(*reinterpret_cast<const __half2*>(&ph), bias);
+    lo = *reinterpret_cast<const uint32_t*>(&l2);
+    hi = *reinterpret_cast<const uint32_t*>(&h2);
+}
+
 // Value fragments A[m-tile i][reg] of one 16-token tile for lane group g.
 template <int VB>
 __device__ __forceinline__ void value_fragments(uint32_t vst, uint32_t base, int g, int t, uint32_t laneoff,
@@ -539,6 +561,44 @@ struct Consumer {
     template <int BITS, bool SKETCH>
     __device__ void encode_new(const uint8_t* src, uint8_t* codes, uint16_t* norms, const float* bounds, size_t slot,
                                uint8_t* prow, uint16_t* pnorm, uint8_t* cbytes, float* rbuf) {
+        if constexpr (BITS == KB_INT8)
+            encode_int8(src, codes, norms, slot, prow, pnorm);
+        else
+            encode_turbo<BITS, SKETCH>(src, codes, norms, bounds, slot, prow, pnorm, cbytes, rbuf);
+    }
+
+    // int8 row (the quantise kernel's arithmetic): fp16 scale = absmax / 127,
+    // bytes rint(x / scale) clamped to +-127, one per channel in natural order
+    __device__ void encode_int8(const uint8_t* src, uint8_t* codes, uint16_t* norms, size_t slot, uint8_t* prow,
+                                uint16_t* pnorm) {
+        float x[4];
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[e] = load_scalar(src, lane * 4 + e, a.new_dtype);
+            amax = fmaxf(amax, fabsf(x[e]));
+        }
+        amax = group_max<32>(amax);
+        const __half scale16 = __float2half_rn(__fdiv_rn(amax, 127.0f));
+        const float scale = __half2float(scale16);
+        const float recip = (scale > 0.0f && scale < INFINITY) ? __frcp_rn(scale) : 0.0f;
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float q = fminf(fmaxf(rintf(__fmul_rn(x[e], recip)), -127.0f), 127.0f);
+            word |= (static_cast<uint32_t>(static_cast<int32_t>(q)) & 0xffu) << (8 * e);
+        }
+        reinterpret_cast<uint32_t*>(codes + slot * D)[lane] = word;
+        reinterpret_cast<uint32_t*>(prow)[lane] = word;
+        if (lane == 0) {
+            norms[slot] = __half_as_ushort(scale16);
+            *pnorm = __half_as_ushort(scale16);
+        }
+    }
+
+    template <int BITS, bool SKETCH>
+    __device__ void encode_turbo(const uint8_t* src, uint8_t* codes, uint16_t* norms, const float* bounds, size_t slot,
+                                 uint8_t* prow, uint16_t* pnorm, uint8_t* cbytes, float* rbuf) {
         float x[4];
         float ss = 0.f;
 #pragma unroll
@@ -597,12 +657,12 @@ struct Consumer {
             }
             const uint32_t z0 = __ballot_sync(kFullMask, lane < a.m && acc0 >= 0.f);
             const uint32_t z1 = __ballot_sync(kFullMask, lane + 32 < a.m && acc1 >= 0.f);
-            uint8_t* pz = smem + L.app + 136;
+            uint8_t* pz = smem + L.app + AP_Z;
             uint32_t* qjl = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.k_qjl) + slot * (a.m / 8));
             if (lane == 0) {
                 const uint16_t g16 = float_to_half_bits(sqrtf(g2));
                 const_cast<uint16_t*>(a.k_gamma)[slot] = g16;
-                *reinterpret_cast<uint16_t*>(smem + L.app + 132) = g16;
+                *reinterpret_cast<uint16_t*>(smem + L.app + AP_GAM) = g16;
                 qjl[0] = z0;
                 reinterpret_cast<uint32_t*>(pz)[0] = z0;
                 if (a.m > 32) {
@@ -619,22 +679,22 @@ struct Consumer {
         const uint8_t* ap = smem + L.app;
         if (warp == 0) {
             if (lane < 4 * KB)
-                reinterpret_cast<uint32_t*>(st + L.k_off + p * (16 * KB))[lane] = reinterpret_cast<const uint32_t*>(ap)[lane];
+                reinterpret_cast<uint32_t*>(st + L.k_off + p * (16 * KB))[lane] = reinterpret_cast<const uint32_t*>(ap + AP_K)[lane];
             if (a.staged_norms && lane == 0) {
-                reinterpret_cast<uint16_t*>(st + L.kn_off)[p] = *reinterpret_cast<const uint16_t*>(ap + 128);
+                reinterpret_cast<uint16_t*>(st + L.kn_off)[p] = *reinterpret_cast<const uint16_t*>(ap + AP_KN);
                 if constexpr (QJL) {
-                    reinterpret_cast<uint16_t*>(st + L.gam_off)[p] = *reinterpret_cast<const uint16_t*>(ap + 132);
+                    reinterpret_cast<uint16_t*>(st + L.gam_off)[p] = *reinterpret_cast<const uint16_t*>(ap + AP_GAM);
                     const int zb = a.m / 8;
                     for (int i = 0; i < zb / 4; ++i)
-                        reinterpret_cast<uint32_t*>(st + L.z_off + p * zb)[i] = reinterpret_cast<const uint32_t*>(ap + 136)[i];
+                        reinterpret_cast<uint32_t*>(st + L.z_off + p * zb)[i] = reinterpret_cast<const uint32_t*>(ap + AP_Z)[i];
                 }
             }
         } else if (warp == 1) {
             if (lane < 4 * VB)
                 reinterpret_cast<uint32_t*>(st + L.v_off + p * (16 * VB))[lane] =
-                    reinterpret_cast<const uint32_t*>(ap + 64)[lane];
+                    reinterpret_cast<const uint32_t*>(ap + AP_V)[lane];
             if (a.staged_norms && lane == 0)
-                reinterpret_cast<uint16_t*>(st + L.vn_off)[p] = *reinterpret_cast<const uint16_t*>(ap + 130);
+                reinterpret_cast<uint16_t*>(st + L.vn_off)[p] = *reinterpret_cast<const uint16_t*>(ap + AP_VN);
         }
         // the stage is refilled later by the copy engine: order these writes first
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -656,12 +716,14 @@ struct Consumer {
             float x[4] = {0.f, 0.f, 0.f, 0.f};
             if (h < G) {
                 load4(qsrc, h * D + lane * 4, a.q_dtype, x);
+                if constexpr (KB != KB_INT8) {  // int8 keys live in the original domain
 #pragma unroll
-                for (int e = 0; e < 4; ++e) x[e] = flip_sign(x[e], (sgn4 >> e) & 1u);
-                fwht_registers(x);
-                fwht_lanes<4, 32>(x, lane);
+                    for (int e = 0; e < 4; ++e) x[e] = flip_sign(x[e], (sgn4 >> e) & 1u);
+                    fwht_registers(x);
+                    fwht_lanes<4, 32>(x, lane);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) x[e] *= inv_sqrt_d;
+                    for (int e = 0; e < 4; ++e) x[e] *= inv_sqrt_d;
+                }
             }
             float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
             amax = group_max<32>(amax);
@@ -728,12 +790,12 @@ struct Consumer {
             uint8_t* ap = smem + L.app;
             if (warp == 0)
                 encode_new<KB, QJL>(rows, const_cast<uint8_t*>(a.k_codes), const_cast<uint16_t*>(a.k_norms), a.kbound,
-                                    slot, ap, reinterpret_cast<uint16_t*>(ap + 128), ap + 256,
-                                    reinterpret_cast<float*>(ap + 512));
+                                    slot, ap + AP_K, reinterpret_cast<uint16_t*>(ap + AP_KN), ap + AP_KC,
+                                    reinterpret_cast<float*>(ap + AP_R));
             else
                 encode_new<VB, false>(rows + D * a.new_bytes, const_cast<uint8_t*>(a.v_codes), const_cast<uint16_t*>(a.v_norms),
-                                      a.vbound, slot, ap + 64, reinterpret_cast<uint16_t*>(ap + 130), ap + 384,
-                                      reinterpret_cast<float*>(ap + 512));
+                                      a.vbound, slot, ap + AP_V, reinterpret_cast<uint16_t*>(ap + AP_VN), ap + AP_VC,
+                                      reinterpret_cast<float*>(ap + AP_R));
         }
         ptx::named_barrier(1, NUM_CONSUMERS);  // every warp is done with the query slot
 #pragma unroll
@@ -827,7 +889,22 @@ struct Consumer {
             // ---- keys: the lane's 4*KB bytes of rows tau(g) and tau(g+8)
             const uint32_t kst = sbase + L.k_off + (lb + TS * k) * VBK;
             uint32_t sa[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
-            if constexpr (KB == 4) {
+            uint32_t ka[8], kb8[8];  // int8 keys: channels 32 t .. 32 t + 31 of rows tau(g), tau(g + 8)
+            if constexpr (KB == KB_INT8) {
+                // 128-byte rows all start at bank 0: lanes of odd g read their
+                // second 16 bytes first, so a quarter-warp (g = 2q, 2q + 1) hits
+                // 32 distinct banks
+                const uint32_t sw = (g & 1) * 16;
+                const uint4 x0 = ptx::lds128(kst + ra * VBK + 32 * t + sw);
+                const uint4 x1 = ptx::lds128(kst + ra * VBK + 32 * t + (sw ^ 16));
+                const uint4 y0 = ptx::lds128(kst + rb * VBK + 32 * t + sw);
+                const uint4 y1 = ptx::lds128(kst + rb * VBK + 32 * t + (sw ^ 16));
+                const bool odd = g & 1;
+                ka[0] = odd ? x1.x : x0.x; ka[1] = odd ? x1.y : x0.y; ka[2] = odd ? x1.z : x0.z; ka[3] = odd ? x1.w : x0.w;
+                ka[4] = odd ? x0.x : x1.x; ka[5] = odd ? x0.y : x1.y; ka[6] = odd ? x0.z : x1.z; ka[7] = odd ? x0.w : x1.w;
+                kb8[0] = odd ? y1.x : y0.x; kb8[1] = odd ? y1.y : y0.y; kb8[2] = odd ? y1.z : y0.z; kb8[3] = odd ? y1.w : y0.w;
+                kb8[4] = odd ? y0.x : y1.x; kb8[5] = odd ? y0.y : y1.y; kb8[6] = odd ? y0.z : y1.z; kb8[7] = odd ? y0.w : y1.w;
+            } else if constexpr (KB == 4) {
                 const uint4 x = ptx::lds128(kst + ra * VBK + 16 * t);
                 const uint4 y = ptx::lds128(kst + rb * VBK + 16 * t);
                 sa[0] = x.x; sa[1] = x.y; sa[2] = x.z; sa[3] = x.w;
@@ -847,10 +924,16 @@ struct Consumer {
                 for (int e = 0; e < 4; ++e) cs[nt][e] = cl[nt][e] = cz[nt][e] = 0.f;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const uint32_t a0 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sa, j, 0, laneoff));
-                const uint32_t a1 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sb, j, 0, laneoff));
-                const uint32_t a2 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sa, j, 1, laneoff));
-                const uint32_t a3 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sb, j, 1, laneoff));
+                uint32_t a0, a1, a2, a3;
+                if constexpr (KB == KB_INT8) {
+                    int8_pairs(ka[j], a0, a2);
+                    int8_pairs(kb8[j], a1, a3);
+                } else {
+                    a0 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sa, j, 0, laneoff));
+                    a1 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sb, j, 0, laneoff));
+                    a2 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sa, j, 1, laneoff));
+                    a3 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sb, j, 1, laneoff));
+                }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     ptx::mma_16816(cs[nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
@@ -1267,7 +1350,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid
             const int e = threadIdx.x;
             const __half* kc = cen;
             const __half* vc = cen + 16;
-            const __half2 k2 = __halves2half2(kc[e & ((1 << KB) - 1)], kc[(e >> KB) & ((1 << KB) - 1)]);
+            constexpr int KM = KB == KB_INT8 ? 0 : (1 << KB) - 1;  // int8 keys use no table
+            const __half2 k2 = __halves2half2(kc[e & KM], kc[(e >> (KB & 7)) & KM]);
             __half2 v0, v1;
             if constexpr (VB >= 3) {
                 v0 = v1 = __halves2half2(vc[e & ((1 << VB) - 1)], vc[(e >> VB) & ((1 << VB) - 1)]);
@@ -1336,8 +1420,14 @@ static cudaError_t launch_typed(const Args& a, int grid, size_t smem, cudaStream
 
 template <int KB, int VB>
 static cudaError_t launch_kv(const Args& a, int nt, bool qjl, int grid, size_t smem, cudaStream_t s) {
-    if (nt == 1) return qjl ? launch_typed<KB, VB, 1, true>(a, grid, smem, s) : launch_typed<KB, VB, 1, false>(a, grid, smem, s);
-    return qjl ? launch_typed<KB, VB, 2, true>(a, grid, smem, s) : launch_typed<KB, VB, 2, false>(a, grid, smem, s);
+    if constexpr (KB == KB_INT8) {  // no sketch on int8 keys
+        if (qjl) return cudaErrorNotSupported;
+        return nt == 1 ? launch_typed<KB, VB, 1, false>(a, grid, smem, s) : launch_typed<KB, VB, 2, false>(a, grid, smem, s);
+    } else {
+        if (nt == 1)
+            return qjl ? launch_typed<KB, VB, 1, true>(a, grid, smem, s) : launch_typed<KB, VB, 1, false>(a, grid, smem, s);
+        return qjl ? launch_typed<KB, VB, 2, true>(a, grid, smem, s) : launch_typed<KB, VB, 2, false>(a, grid, smem, s);
+    }
 }
 
 template <int KB>
@@ -1352,8 +1442,9 @@ static cudaError_t launch_k(const Args& a, int vb, int nt, bool qjl, int grid, s
 }  // namespace mmadec
 
 bool decode_mma_supported(const tq_params& p) {
-    return p.head_dim == 128 && p.k_mode == TQ_MODE_TURBO && p.v_mode == TQ_MODE_TURBO &&
-           p.num_q_heads / p.num_kv_heads <= 16 && p.qjl_dims <= 64;
+    // turbo keys (any bits, optional sketch) or int8 keys (no sketch); turbo values
+    const bool keys = p.k_mode == TQ_MODE_TURBO ? p.qjl_dims <= 64 : (p.k_mode == TQ_MODE_INT8 && p.qjl_dims == 0);
+    return p.head_dim == 128 && keys && p.v_mode == TQ_MODE_TURBO && p.num_q_heads / p.num_kv_heads <= 16;
 }
 
 static uint16_t half_bits(double v) {
@@ -1366,6 +1457,7 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
                               const DecodePlan& plan, char* ws, uint32_t* err, int num_sms, cudaStream_t stream,
                               const void* k_new, const void* v_new, int new_dtype) {
     using namespace mmadec;
+    const bool k_int8 = p.k_mode == TQ_MODE_INT8;
     Args a{};
     a.append = k_new != nullptr;
     a.early = (p.flags & TQ_PARAM_PREFETCH_EARLY) ? 1 : 0;
@@ -1374,12 +1466,14 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     a.new_dtype = new_dtype;
     a.new_bytes = new_dtype == TQ_F32 ? 4 : 2;
     {
-        const int hk = 1 << (p.k_bits - 1), hv = 1 << (p.v_bits - 1);
+        // int8 keys: no boundaries, centroids or table entries
+        const int hk = k_int8 ? 1 : 1 << (p.k_bits - 1), hv = 1 << (p.v_bits - 1);
         for (int k = 0; k < 8; ++k) {
             a.kbound[k] = k < hk - 1 ? static_cast<float>(kcb->boundaries[hk + k]) : INFINITY;
             a.vbound[k] = k < hv - 1 ? static_cast<float>(vcb->boundaries[hv + k]) : INFINITY;
         }
-        for (int j = 0; j < 16; ++j) a.kc32[j] = j < (1 << p.k_bits) ? static_cast<float>(kcb->centroids[j]) : 0.f;
+        for (int j = 0; j < 16; ++j)
+            a.kc32[j] = (!k_int8 && j < (1 << p.k_bits)) ? static_cast<float>(kcb->centroids[j]) : 0.f;
     }
     a.k_codes = c.k_codes;
     a.v_codes = c.v_codes;
@@ -1412,12 +1506,13 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     a.sm_scale_log2 = sm * LOG2E;
     a.tau = p.sparse_v_threshold;
     const double sd = std::sqrt(128.0);
-    const double ak = kcb->fp16_scale > 0.0 ? kcb->fp16_scale : sd;
+    // int8 keys enter the products as exact integers (the scale rides in the norm)
+    const double ak = k_int8 ? 1.0 : kcb->fp16_scale > 0.0 ? kcb->fp16_scale : sd;
     const double av = vcb->fp16_scale > 0.0 ? vcb->fp16_scale : sd;
     a.inv_alpha_k = static_cast<float>(1.0 / ak);
     a.inv_alpha_v = static_cast<float>(1.0 / av);
     for (int j = 0; j < 16; ++j) {
-        a.kcent[j] = j < (1 << p.k_bits) ? half_bits(kcb->centroids[j] * ak) : 0;
+        a.kcent[j] = (!k_int8 && j < (1 << p.k_bits)) ? half_bits(kcb->centroids[j] * ak) : 0;
         a.vcent[j] = j < (1 << p.v_bits) ? half_bits(vcb->centroids[j] * av) : 0;
     }
     a.staged_norms = (c.capacity % 8) == 0;
@@ -1430,7 +1525,7 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
         static_cast<uint32_t>(reserved) != WINDOW)
         return cudaErrorNotSupported;
     const int nt = a.group <= 8 ? 1 : 2;
-    const int kb = p.k_bits, vb = p.v_bits;
+    const int kb = k_int8 ? KB_INT8 : p.k_bits, vb = p.v_bits;
     // as many stages as fit in 227 KB next to the tables and the merge buffers
     const Layout fixed = layout(kb, vb, nt, 0, p.qjl_dims, a.group, a.q_bytes, a.append ? a.new_bytes : 0, a.n_split);
     int stages = static_cast<int>((232448u - fixed.total) / fixed.stage_bytes);
@@ -1445,6 +1540,7 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     if (grid > a.n_items) grid = a.n_items;
     const bool qjl = p.qjl_dims > 0;
     switch (kb) {
+        case KB_INT8: return launch_k<KB_INT8>(a, vb, nt, qjl, grid, smem, stream);
         case 2: return launch_k<2>(a, vb, nt, qjl, grid, smem, stream);
         case 3: return launch_k<3>(a, vb, nt, qjl, grid, smem, stream);
         default: return launch_k<4>(a, vb, nt, qjl, grid, smem, stream);

@@ -3,6 +3,8 @@
 * Llama-3-8B-shaped layer (B=1, Hq=32, Hkv=8, d=128, 32768-token prefill plus
   one appended token, K4/V2), decoded with the benchmark's launch plan: every
   code, norm and output compared.
+* The same layer with int8 keys and 2-bit values, prefilled and then one
+  fused append-and-attend step: every code, scale, norm and output compared.
 * Batched ragged decode (B=16, lengths uniform in [2048, 8192], K3/V2): every
   code, norm and output compared.
 * 70B-shaped long context (B=4, Hq=64, Hkv=8, 131072 tokens, K3 + 64-bit QJL,
@@ -80,6 +82,38 @@ def test_llama8b_layer_full_context():
     assert st == tq.TQ_OK and word == 0
     got, st, word = H.gpu_decode(layer, q, cache, [t], max_len=cap)
     assert st == tq.TQ_OK and word == 0
+    kn, vn = _np64(k), _np64(v)
+    khat = np.empty((1, 8, t, 128))
+    vhat = np.empty((1, 8, t, 128))
+    for h in range(8):
+        khat[0, h], vhat[0, h] = _oracle_unit(layer, kn[0, :, h], vn[0, :, h], cache, 0, h, t)
+    ref = H.oracle_attention(layer, _np64(q), khat, vhat, [t])
+    err = H.rel_l2_per_vector(got, ref["out"])
+    assert err.max() < H.ATTN_TOL, err.max()
+
+
+def test_llama8b_int8_keys_full_context():
+    """The Llama-3-8B-shaped layer with int8 keys and 2-bit values: 32768
+    tokens prefilled, then one fused append-and-attend step; every code, scale,
+    norm and output compared."""
+    layer = H.Layer(128, 32, 8, k_mode=tq.TQ_MODE_INT8, v_bits=2, seed=4321)
+    ctx = 32768
+    t = ctx + 1
+    cap = ctx + 8
+    k = inputs.lognormal_kv(1, t, 8, 128, seed=4321, layer=0, which=inputs.K)
+    v = inputs.lognormal_kv(1, t, 8, 128, seed=4321, layer=0, which=inputs.V)
+    q = inputs.queries(1, 32, 128, seed=4321)
+    cache = tq.alloc_cache(layer.params, 1, cap)
+    cache, st, word = H.gpu_quantize(layer, k[:, :ctx], v[:, :ctx], cap, cache=cache)
+    assert st == tq.TQ_OK and word == 0
+    ws = torch.zeros(tq.tq_decode_workspace_bytes(layer.params, 1, cap), dtype=torch.uint8, device="cuda")
+    out = torch.empty(1, 32, 128, dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.tq_append_decode_attention(layer.params, layer.kcb, layer.vcb, k[:, ctx:].cuda(), v[:, ctx:].cuda(), q.cuda(),
+                                  cache, torch.tensor([t], dtype=torch.int32, device="cuda"), cap, out, ws, err)
+    st, word = tq.tq_read_device_error(err)
+    assert st == tq.TQ_OK and word == 0
+    got = out.cpu().numpy()
     kn, vn = _np64(k), _np64(v)
     khat = np.empty((1, 8, t, 128))
     vhat = np.empty((1, 8, t, 128))

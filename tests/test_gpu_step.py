@@ -89,16 +89,29 @@ def test_step_qjl_group8_ragged():
     _check_attention(layer, cache, lens, q, got)
 
 
-@pytest.mark.parametrize("cfg", ["d64", "int8_k"])
+@pytest.mark.parametrize("cfg", ["d64", "int8_v"])
 def test_step_two_kernel_path(cfg):
     """Configurations outside the tensor-core kernel append with the quantise
     kernel and attend with the general kernels."""
     if cfg == "d64":
         layer = H.Layer(64, 8, 2, k_bits=4, v_bits=3, seed=45)
     else:
-        layer = H.Layer(128, 16, 4, k_mode=tq.TQ_MODE_INT8, v_bits=2, seed=45)
+        layer = H.Layer(128, 16, 4, k_bits=4, v_mode=tq.TQ_MODE_INT8, seed=45)
     lens = [700, 350, 1]
     cache, got, st, word, (k, v, kn, vn, q) = _step_case(layer, 700, lens, seed=45)
+    assert st == tq.TQ_OK and word == 0
+    _check_appended(layer, cache, lens, kn, vn)
+    _check_attention(layer, cache, lens, q, got)
+
+
+@pytest.mark.parametrize("hq,v_bits", [(32, 2), (64, 3)])
+def test_step_int8_keys(hq, v_bits):
+    """int8 keys with turbo values (the mixed setting) in the fused kernel: the
+    appended key is written as int8 bytes and an fp16 scale, bit-exact with the
+    oracle, and attention over the stored cache matches."""
+    layer = H.Layer(128, hq, 8, k_mode=tq.TQ_MODE_INT8, v_bits=v_bits, seed=51)
+    lens = [2100, 1333, 5]
+    cache, got, st, word, (k, v, kn, vn, q) = _step_case(layer, 2100, lens, seed=51)
     assert st == tq.TQ_OK and word == 0
     _check_appended(layer, cache, lens, kn, vn)
     _check_attention(layer, cache, lens, q, got)
