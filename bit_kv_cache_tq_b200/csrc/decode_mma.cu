@@ -87,17 +87,19 @@ constexpr int SQ_STRIDE = 64 + 4;
 constexpr uint32_t AP_K = 0, AP_V = 128, AP_KN = 256, AP_VN = 258, AP_GAM = 260, AP_Z = 264, AP_KC = 288,
                    AP_VC = 416, AP_R = 544;
 constexpr uint32_t APP_BYTES = AP_R + 4 * D;
-// key side in int8 mode (one byte per channel, fp16 scale in the norm slot):
-// the kernel's KB template parameter takes this value
-constexpr int KB_INT8 = 8;
+// a side in int8 mode (one byte per channel, fp16 scale in the norm slot):
+// the kernel's KB / VB template parameters take this value.  Int8 values come
+// only with int8 keys (an all-int8 layer), which need no centroid tables.
+constexpr int INT8_BITS = 8;
+__host__ __device__ constexpr bool uses_tables(int kb, int vb) { return !(kb == INT8_BITS && vb == INT8_BITS); }
 constexpr long long WAIT_LIMIT = 2000000000ll;  // clock cycles (~1 s)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LAZY = 8.0f;                 // log2 headroom before the running max moves
 constexpr float VRANGE = 64.0f;              // bound on ||v|| * vscale
 
-// header flags: item (query slot) EMPTY / END / APPEND / DRAIN (one stage to
-// consume unread) / SKIP (no work: only the drain), chunk (stage) LAST
-constexpr int F_LAST = 2, F_EMPTY = 4, F_END = 8, F_APPEND = 16, F_DRAIN = 32, F_SKIP = 64;
+// item header flags (query slot): EMPTY / END / APPEND / DRAIN (one stage to
+// consume unread) / SKIP (no work: only the drain)
+constexpr int F_EMPTY = 4, F_END = 8, F_APPEND = 16, F_DRAIN = 32, F_SKIP = 64;
 // global counters after the per-(sequence, kv head) split counters
 constexpr int C_ITEM = 0, C_DONE = 1;
 
@@ -149,7 +151,7 @@ __host__ __device__ inline uint32_t align16(uint32_t x) { return (x + 15u) & ~15
 __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int m, int g, int q_bytes, int new_bytes,
                                          int n_split) {
     Layout L{};
-    L.ring = LUT_BYTES;
+    L.ring = uses_tables(kb, vb) ? LUT_BYTES : 0;
     L.k_off = 16;
     L.v_off = L.k_off + CHUNK * 16 * kb;
     L.kn_off = L.v_off + CHUNK * 16 * vb;
@@ -417,8 +419,8 @@ __device__ __forceinline__ uint32_t key_lut_addr(const uint32_t (&seg)[4], int j
     }
 }
 
-// Four int8 channels (one word, byte i = channel i) as two fp16 pairs, exactly:
-// byte b ^ 0x80 = b + 128 becomes the mantissa of 1024 + (b + 128), and
+// Four int8 bytes of one word as two fp16 pairs (bytes 0, 1 and bytes 2, 3),
+// exactly: b ^ 0x80 = b + 128 becomes the mantissa of 1024 + (b + 128), and
 // subtracting 1152 leaves b.
 __device__ __forceinline__ void int8_pairs(uint32_t w, uint32_t& lo, uint32_t& hi) {
     const uint32_t u = w ^ 0x80808080u;
@@ -436,7 +438,26 @@ template <int VB>
 __device__ __forceinline__ void value_fragments(uint32_t vst, uint32_t base, int g, int t, uint32_t laneoff,
                                                 uint32_t (&A)[8][4]) {
     constexpr int VBV = 16 * VB;
-    if constexpr (VB == 2) {
+    if constexpr (VB == INT8_BITS) {
+        // channels 16 g .. 16 g + 15 (16 bytes) of physical tokens t, 4 + (t ^ 1),
+        // 8 + t, 12 + (t ^ 1) (logical k = 2t, 2t+1, 2t+8, 2t+9); row g of m-tile
+        // i is channel 16 g + 2 i, row g + 8 channel 16 g + 2 i + 1
+        const uint4 xa = ptx::lds128(vst + t * VBV + 16 * g);
+        const uint4 xb = ptx::lds128(vst + (4 + (t ^ 1)) * VBV + 16 * g);
+        const uint4 xc = ptx::lds128(vst + (8 + t) * VBV + 16 * g);
+        const uint4 xd = ptx::lds128(vst + (12 + (t ^ 1)) * VBV + 16 * g);
+        const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w}, wb[4] = {xb.x, xb.y, xb.z, xb.w};
+        const uint32_t wc[4] = {xc.x, xc.y, xc.z, xc.w}, wd[4] = {xd.x, xd.y, xd.z, xd.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int w = i >> 1;
+            const uint32_t sel = (i & 1) ? 0x7362u : 0x5140u;  // bytes 2p, 2p + 1 of both words, interleaved
+            const uint32_t ab = __byte_perm(wa[w], wb[w], sel);
+            const uint32_t cd = __byte_perm(wc[w], wd[w], sel);
+            int8_pairs(ab, A[i][0], A[i][1]);
+            int8_pairs(cd, A[i][2], A[i][3]);
+        }
+    } else if constexpr (VB == 2) {
         // word g of physical tokens t, 4 + (t ^ 1), 8 + t, 12 + (t ^ 1)
         // (logical k = 2t, 2t+1, 2t+8, 2t+9)
         const uint32_t w0 = ptx::lds32(vst + t * VBV + 4 * g);
@@ -561,7 +582,7 @@ struct Consumer {
     template <int BITS, bool SKETCH>
     __device__ void encode_new(const uint8_t* src, uint8_t* codes, uint16_t* norms, const float* bounds, size_t slot,
                                uint8_t* prow, uint16_t* pnorm, uint8_t* cbytes, float* rbuf) {
-        if constexpr (BITS == KB_INT8)
+        if constexpr (BITS == INT8_BITS)
             encode_int8(src, codes, norms, slot, prow, pnorm);
         else
             encode_turbo<BITS, SKETCH>(src, codes, norms, bounds, slot, prow, pnorm, cbytes, rbuf);
@@ -716,7 +737,7 @@ struct Consumer {
             float x[4] = {0.f, 0.f, 0.f, 0.f};
             if (h < G) {
                 load4(qsrc, h * D + lane * 4, a.q_dtype, x);
-                if constexpr (KB != KB_INT8) {  // int8 keys live in the original domain
+                if constexpr (KB != INT8_BITS) {  // int8 keys live in the original domain
 #pragma unroll
                     for (int e = 0; e < 4; ++e) x[e] = flip_sign(x[e], (sgn4 >> e) & 1u);
                     fwht_registers(x);
@@ -890,7 +911,7 @@ struct Consumer {
             const uint32_t kst = sbase + L.k_off + (lb + TS * k) * VBK;
             uint32_t sa[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
             uint32_t ka[8], kb8[8];  // int8 keys: channels 32 t .. 32 t + 31 of rows tau(g), tau(g + 8)
-            if constexpr (KB == KB_INT8) {
+            if constexpr (KB == INT8_BITS) {
                 // 128-byte rows all start at bank 0: lanes of odd g read their
                 // second 16 bytes first, so a quarter-warp (g = 2q, 2q + 1) hits
                 // 32 distinct banks
@@ -925,7 +946,7 @@ struct Consumer {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 uint32_t a0, a1, a2, a3;
-                if constexpr (KB == KB_INT8) {
+                if constexpr (KB == INT8_BITS) {
                     int8_pairs(ka[j], a0, a2);
                     int8_pairs(kb8[j], a1, a3);
                 } else {
@@ -1200,11 +1221,16 @@ struct Consumer {
                 float x[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) x[e] = o_s[h * D + lane * 4 + e];
-                fwht_registers(x);
-                fwht_lanes<4, 32>(x, lane);
                 float* dst = a.out + (static_cast<size_t>(w.b) * a.hq + w.kv * G + h) * D + lane * 4;
+                if constexpr (VB == INT8_BITS) {  // int8 values: already in the original domain
 #pragma unroll
-                for (int e = 0; e < 4; ++e) dst[e] = flip_sign(x[e] * inv_sqrt_d, (sgn4 >> e) & 1u);
+                    for (int e = 0; e < 4; ++e) dst[e] = x[e];
+                } else {
+                    fwht_registers(x);
+                    fwht_lanes<4, 32>(x, lane);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = flip_sign(x[e] * inv_sqrt_d, (sgn4 >> e) & 1u);
+                }
             }
             if (tid == 0) a.counters[w.unit] = 0;
         }
@@ -1335,7 +1361,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid
     // index into the kernel parameters would serialise).  Step 2: the
     // threads replicate them in address order, 16 bytes per store (a warp
     // covers 512 contiguous bytes), with independent reads.
-    {
+    if constexpr (uses_tables(KB, VB)) {
         __half* cen = reinterpret_cast<__half*>(smem + L.app);  // [16] key, [16] value
         uint32_t* compact = reinterpret_cast<uint32_t*>(smem + L.merge);  // [256] key, [256][2] value
         if (threadIdx.x == 0) {
@@ -1350,11 +1376,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_mma_kernel(const __grid
             const int e = threadIdx.x;
             const __half* kc = cen;
             const __half* vc = cen + 16;
-            constexpr int KM = KB == KB_INT8 ? 0 : (1 << KB) - 1;  // int8 keys use no table
+            constexpr int KM = KB == INT8_BITS ? 0 : (1 << KB) - 1;  // int8 keys use no table
             const __half2 k2 = __halves2half2(kc[e & KM], kc[(e >> (KB & 7)) & KM]);
             __half2 v0, v1;
             if constexpr (VB >= 3) {
-                v0 = v1 = __halves2half2(vc[e & ((1 << VB) - 1)], vc[(e >> VB) & ((1 << VB) - 1)]);
+                constexpr int VM = VB == INT8_BITS ? 0 : (1 << VB) - 1;
+                v0 = v1 = __halves2half2(vc[e & VM], vc[(e >> (VB & 7)) & VM]);
             } else {
                 // byte e = (token a: two 2-bit codes) | (token b: two codes) << 4; the
                 // first word holds channel 1 of (a, b), the second channel 2
@@ -1420,7 +1447,7 @@ static cudaError_t launch_typed(const Args& a, int grid, size_t smem, cudaStream
 
 template <int KB, int VB>
 static cudaError_t launch_kv(const Args& a, int nt, bool qjl, int grid, size_t smem, cudaStream_t s) {
-    if constexpr (KB == KB_INT8) {  // no sketch on int8 keys
+    if constexpr (KB == INT8_BITS) {  // no sketch on int8 keys
         if (qjl) return cudaErrorNotSupported;
         return nt == 1 ? launch_typed<KB, VB, 1, false>(a, grid, smem, s) : launch_typed<KB, VB, 2, false>(a, grid, smem, s);
     } else {
@@ -1433,6 +1460,9 @@ static cudaError_t launch_kv(const Args& a, int nt, bool qjl, int grid, size_t s
 template <int KB>
 static cudaError_t launch_k(const Args& a, int vb, int nt, bool qjl, int grid, size_t smem, cudaStream_t s) {
     switch (vb) {
+        case INT8_BITS:
+            if constexpr (KB == INT8_BITS) return launch_kv<KB, INT8_BITS>(a, nt, qjl, grid, smem, s);
+            return cudaErrorNotSupported;
         case 2: return launch_kv<KB, 2>(a, nt, qjl, grid, smem, s);
         case 3: return launch_kv<KB, 3>(a, nt, qjl, grid, smem, s);
         default: return launch_kv<KB, 4>(a, nt, qjl, grid, smem, s);
@@ -1442,9 +1472,11 @@ static cudaError_t launch_k(const Args& a, int vb, int nt, bool qjl, int grid, s
 }  // namespace mmadec
 
 bool decode_mma_supported(const tq_params& p) {
-    // turbo keys (any bits, optional sketch) or int8 keys (no sketch); turbo values
+    // turbo keys (any bits, optional sketch) or int8 keys (no sketch); turbo
+    // values, or int8 values beside int8 keys
     const bool keys = p.k_mode == TQ_MODE_TURBO ? p.qjl_dims <= 64 : (p.k_mode == TQ_MODE_INT8 && p.qjl_dims == 0);
-    return p.head_dim == 128 && keys && p.v_mode == TQ_MODE_TURBO && p.num_q_heads / p.num_kv_heads <= 16;
+    const bool values = p.v_mode == TQ_MODE_TURBO || (p.v_mode == TQ_MODE_INT8 && p.k_mode == TQ_MODE_INT8);
+    return p.head_dim == 128 && keys && values && p.num_q_heads / p.num_kv_heads <= 16;
 }
 
 static uint16_t half_bits(double v) {
@@ -1457,7 +1489,7 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
                               const DecodePlan& plan, char* ws, uint32_t* err, int num_sms, cudaStream_t stream,
                               const void* k_new, const void* v_new, int new_dtype) {
     using namespace mmadec;
-    const bool k_int8 = p.k_mode == TQ_MODE_INT8;
+    const bool k_int8 = p.k_mode == TQ_MODE_INT8, v_int8 = p.v_mode == TQ_MODE_INT8;
     Args a{};
     a.append = k_new != nullptr;
     a.early = (p.flags & TQ_PARAM_PREFETCH_EARLY) ? 1 : 0;
@@ -1467,7 +1499,7 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     a.new_bytes = new_dtype == TQ_F32 ? 4 : 2;
     {
         // int8 keys: no boundaries, centroids or table entries
-        const int hk = k_int8 ? 1 : 1 << (p.k_bits - 1), hv = 1 << (p.v_bits - 1);
+        const int hk = k_int8 ? 1 : 1 << (p.k_bits - 1), hv = v_int8 ? 1 : 1 << (p.v_bits - 1);
         for (int k = 0; k < 8; ++k) {
             a.kbound[k] = k < hk - 1 ? static_cast<float>(kcb->boundaries[hk + k]) : INFINITY;
             a.vbound[k] = k < hv - 1 ? static_cast<float>(vcb->boundaries[hv + k]) : INFINITY;
@@ -1508,12 +1540,12 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     const double sd = std::sqrt(128.0);
     // int8 keys enter the products as exact integers (the scale rides in the norm)
     const double ak = k_int8 ? 1.0 : kcb->fp16_scale > 0.0 ? kcb->fp16_scale : sd;
-    const double av = vcb->fp16_scale > 0.0 ? vcb->fp16_scale : sd;
+    const double av = v_int8 ? 1.0 : vcb->fp16_scale > 0.0 ? vcb->fp16_scale : sd;
     a.inv_alpha_k = static_cast<float>(1.0 / ak);
     a.inv_alpha_v = static_cast<float>(1.0 / av);
     for (int j = 0; j < 16; ++j) {
         a.kcent[j] = (!k_int8 && j < (1 << p.k_bits)) ? half_bits(kcb->centroids[j] * ak) : 0;
-        a.vcent[j] = j < (1 << p.v_bits) ? half_bits(vcb->centroids[j] * av) : 0;
+        a.vcent[j] = (!v_int8 && j < (1 << p.v_bits)) ? half_bits(vcb->centroids[j] * av) : 0;
     }
     a.staged_norms = (c.capacity % 8) == 0;
     uint32_t words[8];
@@ -1525,7 +1557,7 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
         static_cast<uint32_t>(reserved) != WINDOW)
         return cudaErrorNotSupported;
     const int nt = a.group <= 8 ? 1 : 2;
-    const int kb = k_int8 ? KB_INT8 : p.k_bits, vb = p.v_bits;
+    const int kb = k_int8 ? INT8_BITS : p.k_bits, vb = v_int8 ? INT8_BITS : p.v_bits;
     // as many stages as fit in 227 KB next to the tables and the merge buffers
     const Layout fixed = layout(kb, vb, nt, 0, p.qjl_dims, a.group, a.q_bytes, a.append ? a.new_bytes : 0, a.n_split);
     int stages = static_cast<int>((232448u - fixed.total) / fixed.stage_bytes);
@@ -1540,7 +1572,7 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     if (grid > a.n_items) grid = a.n_items;
     const bool qjl = p.qjl_dims > 0;
     switch (kb) {
-        case KB_INT8: return launch_k<KB_INT8>(a, vb, nt, qjl, grid, smem, stream);
+        case INT8_BITS: return launch_k<INT8_BITS>(a, vb, nt, qjl, grid, smem, stream);
         case 2: return launch_k<2>(a, vb, nt, qjl, grid, smem, stream);
         case 3: return launch_k<3>(a, vb, nt, qjl, grid, smem, stream);
         default: return launch_k<4>(a, vb, nt, qjl, grid, smem, stream);

@@ -3,8 +3,9 @@
 * Llama-3-8B-shaped layer (B=1, Hq=32, Hkv=8, d=128, 32768-token prefill plus
   one appended token, K4/V2), decoded with the benchmark's launch plan: every
   code, norm and output compared.
-* The same layer with int8 keys and 2-bit values, prefilled and then one
-  fused append-and-attend step: every code, scale, norm and output compared.
+* The same layer with int8 keys and 2-bit values, and as an all-int8
+  boundary layer, prefilled and then one fused append-and-attend step: every
+  code, scale, norm and output compared.
 * Batched ragged decode (B=16, lengths uniform in [2048, 8192], K3/V2): every
   code, norm and output compared.
 * 70B-shaped long context (B=4, Hq=64, Hkv=8, 131072 tokens, K3 + 64-bit QJL,
@@ -92,11 +93,12 @@ def test_llama8b_layer_full_context():
     assert err.max() < H.ATTN_TOL, err.max()
 
 
-def test_llama8b_int8_keys_full_context():
-    """The Llama-3-8B-shaped layer with int8 keys and 2-bit values: 32768
-    tokens prefilled, then one fused append-and-attend step; every code, scale,
-    norm and output compared."""
-    layer = H.Layer(128, 32, 8, k_mode=tq.TQ_MODE_INT8, v_bits=2, seed=4321)
+@pytest.mark.parametrize("v_mode", [tq.TQ_MODE_TURBO, tq.TQ_MODE_INT8])
+def test_llama8b_int8_keys_full_context(v_mode):
+    """The Llama-3-8B-shaped layer with int8 keys and 2-bit values (or int8
+    values: a boundary layer): 32768 tokens prefilled, then one fused
+    append-and-attend step; every code, scale, norm and output compared."""
+    layer = H.Layer(128, 32, 8, k_mode=tq.TQ_MODE_INT8, v_mode=v_mode, v_bits=2, seed=4321)
     ctx = 32768
     t = ctx + 1
     cap = ctx + 8

@@ -253,11 +253,16 @@ def test_attention_over_int8_sides(k_mode, v_mode):
     assert same.max() < H.ATTN_TOL and e2e.max() < H.ATTN_TOL, (same.max(), e2e.max())
 
 
-@pytest.mark.parametrize("hq,v_bits,lens", [(32, 2, [3001, 1700]), (64, 4, [1200, 1]), (16, 3, [777])])
+@pytest.mark.parametrize("hq,v_bits,lens", [(32, 2, [3001, 1700]), (64, 4, [1200, 1]), (16, 3, [777]),
+                                           (32, "int8", [3001, 1700]), (64, "int8", [1200, 1]), (16, "int8", [777])])
 def test_int8_keys_turbo_values_ragged(hq, v_bits, lens):
-    """int8 keys beside turbo values in the tensor-core kernel: several chunks,
-    ragged tails, a one-token sequence, GQA groups of 2, 4 and 8."""
-    layer = H.Layer(128, hq, 8, k_mode=tq.TQ_MODE_INT8, v_bits=v_bits, seed=19)
+    """int8 keys beside turbo values (or int8 values: a boundary layer) in the
+    tensor-core kernel: several chunks, ragged tails, a one-token sequence,
+    GQA groups of 2, 4 and 8."""
+    if v_bits == "int8":
+        layer = H.Layer(128, hq, 8, k_mode=tq.TQ_MODE_INT8, v_mode=tq.TQ_MODE_INT8, seed=19)
+    else:
+        layer = H.Layer(128, hq, 8, k_mode=tq.TQ_MODE_INT8, v_bits=v_bits, seed=19)
     t = max(lens)
     k = inputs.lognormal_kv(len(lens), t, 8, 128, seed=19, layer=3, which=inputs.K)
     v = inputs.lognormal_kv(len(lens), t, 8, 128, seed=19, layer=3, which=inputs.V)

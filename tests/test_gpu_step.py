@@ -104,12 +104,16 @@ def test_step_two_kernel_path(cfg):
     _check_attention(layer, cache, lens, q, got)
 
 
-@pytest.mark.parametrize("hq,v_bits", [(32, 2), (64, 3)])
+@pytest.mark.parametrize("hq,v_bits", [(32, 2), (64, 3), (32, "int8")])
 def test_step_int8_keys(hq, v_bits):
-    """int8 keys with turbo values (the mixed setting) in the fused kernel: the
-    appended key is written as int8 bytes and an fp16 scale, bit-exact with the
-    oracle, and attention over the stored cache matches."""
-    layer = H.Layer(128, hq, 8, k_mode=tq.TQ_MODE_INT8, v_bits=v_bits, seed=51)
+    """int8 keys with turbo values (the mixed setting), or with int8 values (a
+    boundary layer), in the fused kernel: the appended rows are written as
+    int8 bytes and fp16 scales, bit-exact with the oracle, and attention over
+    the stored cache matches."""
+    if v_bits == "int8":
+        layer = H.Layer(128, hq, 8, k_mode=tq.TQ_MODE_INT8, v_mode=tq.TQ_MODE_INT8, seed=51)
+    else:
+        layer = H.Layer(128, hq, 8, k_mode=tq.TQ_MODE_INT8, v_bits=v_bits, seed=51)
     lens = [2100, 1333, 5]
     cache, got, st, word, (k, v, kn, vn, q) = _step_case(layer, 2100, lens, seed=51)
     assert st == tq.TQ_OK and word == 0
