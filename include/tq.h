@@ -301,9 +301,10 @@ tq_status tq_decode_attention(const tq_params* params, const tq_codebook* kcb, c
  *   Other arguments as for tq_decode_attention (same workspace rules).
  * The new token is encoded exactly as tq_quantize_append encodes it (the
  * cache afterwards holds what tq_quantize_append would have written, up to
- * codes within the boundary window).  On the tensor-core path (d = 128,
- * turbo K and V) this is one kernel: the block that owns a sequence's last
- * token split encodes the token while the cache streams in.  Other
+ * codes within the boundary window).  On the tensor-core path (d = 128;
+ * turbo or int8 K; turbo V, or int8 V beside int8 K with at most 4 query
+ * heads per kv head) this is one kernel: the block that owns a sequence's
+ * last token split encodes the token while the cache streams in.  Other
  * configurations run tq_quantize_append's kernel and then the attention
  * kernels.  A seq_len outside [1, capacity] skips that sequence's append and
  * sets TQ_DEVERR_SEQLEN (or TQ_DEVERR_POSITION on the two-kernel path).
