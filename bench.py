@@ -432,6 +432,54 @@ def decode_configs(dev, reps=10):
     return res
 
 
+def paged_decode(dev, reps=10, copies=4):
+    """The Llama-3-8B-shaped layer (B=1, 32768 tokens, K4/V2) read through a
+    block table (blocks in a random order over the pool), block sizes 16 and
+    256 tokens; 4 pools cycled so the reads come from HBM."""
+    from bit_kv_cache_tq_b200 import inputs, tq
+    p = tq.make_params(D, HQ, HKV, K_BITS, V_BITS, seed=SEED)
+    kcb, vcb = tq.tq_codebook_init(D, K_BITS), tq.tq_codebook_init(D, V_BITS)
+    n = CONTEXT
+    res = {}
+    for bs in (16, 256):
+        max_blocks = (n + bs - 1) // bs
+        gen = torch.Generator().manual_seed(SEED + bs)
+        pools, tables = [], []
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        for c in range(copies):
+            pool = tq.alloc_cache(p, max_blocks, bs, device=dev)
+            table = torch.randperm(max_blocks, generator=gen).to(torch.int32).view(1, max_blocks).to(dev)
+            k = inputs.lognormal_kv(1, n, HKV, D, SEED, 60 + c, inputs.K, device=dev)
+            v = inputs.lognormal_kv(1, n, HKV, D, SEED, 60 + c, inputs.V, device=dev)
+            tq.tq_quantize_append_paged(p, kcb, vcb, k, v, torch.zeros(1, dtype=torch.int32, device=dev), pool,
+                                        table, err)
+            del k, v
+            pools.append(pool)
+            tables.append(table)
+        q = inputs.queries(1, HQ, D, SEED, device=dev)
+        lens_t = torch.tensor([n], dtype=torch.int32, device=dev)
+        ws = torch.zeros(tq.tq_decode_workspace_bytes(p, 1, n), dtype=torch.uint8, device=dev)
+        out = torch.empty(1, HQ, D, dtype=torch.float32, device=dev)
+        for c in range(copies):
+            tq.tq_decode_attention_paged(p, kcb, vcb, q, pools[c], tables[c], lens_t, n, out, ws, err)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for r in range(reps):
+            tq.tq_decode_attention_paged(p, kcb, vcb, q, pools[r % copies], tables[r % copies], lens_t, n, out, ws,
+                                         err)
+        e1.record()
+        e1.synchronize()
+        st, word = tq.tq_read_device_error(err)
+        assert st == tq.TQ_OK, (bs, st, word)
+        us = 1000.0 * e0.elapsed_time(e1) / reps
+        nbytes = n * HKV * bytes_per_token_head()
+        res["block_%d" % bs] = {"us_per_call": round(us, 2), "kv_tokens_per_s": round(n / (us * 1e-6)),
+                                "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "algorithmic_bytes": nbytes}
+        del pools, tables, ws
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_tq(args, world, rank, local):
     from bit_kv_cache_tq_b200 import inputs, tq
     dev = torch.device("cuda", local)
@@ -532,19 +580,30 @@ def run_tq(args, world, rank, local):
     achieved = alg_bytes / (decode_us * 1e-6) / 1e9
     peak, peak_kind = measured_peaks()
 
-    # end to end through the C ABI with host buffers: pinned inputs copied in,
-    # outputs copied out, every step
-    h_k = [torch.empty(BATCH, 1, HKV, D, dtype=torch.bfloat16).pin_memory() for _ in range(LAYERS)]
-    h_v = [torch.empty(BATCH, 1, HKV, D, dtype=torch.bfloat16).pin_memory() for _ in range(LAYERS)]
-    h_q = [torch.empty(BATCH, HQ, D, dtype=torch.bfloat16).pin_memory() for _ in range(LAYERS)]
+    # end to end through the C ABI with host buffers: every step, the step's
+    # inputs (each layer's new K and V rows and queries, staged in one pinned
+    # slab) go in with one copy, and the outputs come back with one copy
+    kv_elems, q_elems = BATCH * HKV * D, BATCH * HQ * D
+    per_layer = 2 * kv_elems + q_elems  # bf16 elements: k row, v row, queries
+
+    def layer_views(slab):
+        ks, vs, qv = [], [], []
+        for l in range(LAYERS):
+            o = l * per_layer
+            ks.append(slab[o:o + kv_elems].view(BATCH, 1, HKV, D))
+            vs.append(slab[o + kv_elems:o + 2 * kv_elems].view(BATCH, 1, HKV, D))
+            qv.append(slab[o + 2 * kv_elems:o + per_layer].view(BATCH, HQ, D))
+        return ks, vs, qv
+
+    h_in = torch.empty(LAYERS * per_layer, dtype=torch.bfloat16).pin_memory()
+    h_k, h_v, h_q = layer_views(h_in)
     for l in range(LAYERS):
         h_k[l].copy_(k_new[l][:, -1:])
         h_v[l].copy_(v_new[l][:, -1:])
         h_q[l].copy_(qs[l][-1])
     h_out = torch.empty(LAYERS, BATCH, HQ, D, dtype=torch.float32).pin_memory()
-    s_k = [torch.empty(BATCH, 1, HKV, D, dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
-    s_v = [torch.empty(BATCH, 1, HKV, D, dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
-    s_q = [torch.empty(BATCH, HQ, D, dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
+    s_in = torch.empty(LAYERS * per_layer, dtype=torch.bfloat16, device=dev)
+    s_k, s_v, s_q = layer_views(s_in)
     last = total_steps - 1
     g_e2e = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
@@ -553,21 +612,17 @@ def run_tq(args, world, rank, local):
                 tq.tq_append_decode_attention(params[l], kcb, vcb, s_k[l], s_v[l], s_q[l], caches[l], lens[last], cap,
                                               outs[l], ws, err, stream=stream)
     torch.cuda.synchronize()
-    h2d = sum(t.numel() * t.element_size() for t in h_k + h_v + h_q)
+    h2d = h_in.numel() * h_in.element_size()
     d2h = h_out.numel() * h_out.element_size()
     e2e_steps = steps
     with torch.cuda.stream(stream):
         for it in range(warmup + e2e_steps):
             if it == warmup:
                 stream.synchronize()
-                t_e2e = time.perf_counter()
                 f0 = torch.cuda.Event(enable_timing=True)
                 f1 = torch.cuda.Event(enable_timing=True)
                 f0.record(stream)
-            for l in range(LAYERS):
-                s_k[l].copy_(h_k[l], non_blocking=True)
-                s_v[l].copy_(h_v[l], non_blocking=True)
-                s_q[l].copy_(h_q[l], non_blocking=True)
+            s_in.copy_(h_in, non_blocking=True)
             g_e2e.replay()
             h_out.copy_(outs, non_blocking=True)
         f1.record(stream)
@@ -601,6 +656,8 @@ def run_tq(args, world, rank, local):
         if not args.quick:
             line["bf16_baseline"] = bf16_sdpa_baseline(dev)
             line["decode_configs"] = decode_configs(dev)
+            line["paged_decode"] = {"workload": "llama3-8b-shaped layer, 32768 tokens, K4/V2, through a block "
+                                                "table (blocks in random order)", **paged_decode(dev)}
             peak_gbs = measured_peaks()[0]
             q = {"workload": "bulk prefill quantise: 262144 tokens x 8 kv heads, bf16, 32 layers (0, 1, 30, 31 "
                              "int8 per-vector absmax, others K4/V3 turbo), one input slab, 32 distinct outputs",

@@ -293,25 +293,36 @@ static cudaError_t launch_decode_dim(const DecodeArgs& a, cudaStream_t stream) {
 }
 
 // k_new / v_new non-null: append mode (one new token per sequence at seq_len - 1).
+// pm non-null: c is the pool of a paged cache.
 cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const tq_codebook* vcb, const tq_cache& c,
                               const void* q, int q_dtype, const int32_t* seq_lens, int max_len, float* out,
                               const DecodePlan& plan, char* ws, uint32_t* err, int num_sms, cudaStream_t stream,
-                              const void* k_new = nullptr, const void* v_new = nullptr, int new_dtype = 0);
+                              const void* k_new = nullptr, const void* v_new = nullptr, int new_dtype = 0,
+                              const PageMap* pm = nullptr);
 
 }  // namespace tq
 
 namespace tq {
 // Decode attention; with k_new / v_new set, the step's new token of every
-// sequence is first written at position seq_len - 1 (append mode).
+// sequence is first written at position seq_len - 1 (append mode).  With a
+// block table, `cache` is the pool of a paged cache (tensor-core path only).
 static tq_status decode_impl(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
                              const void* d_q, tq_dtype q_dtype, const tq_cache* cache, const int32_t* d_seq_lens,
                              int32_t max_seq_len, float* d_out, void* d_workspace, size_t workspace_bytes,
                              uint32_t* d_error, void* stream, const void* k_new, const void* v_new,
-                             tq_dtype kv_dtype) {
+                             tq_dtype kv_dtype, const tq_block_table* table = nullptr) {
     tq_status st = validate_params(params);
     if (st != TQ_OK) return st;
     const tq_params& p = *params;
-    if ((st = validate_cache(p, cache)) != TQ_OK) return st;
+    PageMap pages;
+    const PageMap* pm = nullptr;
+    if (table) {
+        if ((st = validate_pages(p, cache, table, &pages)) != TQ_OK) return st;
+        pm = &pages;
+    } else if ((st = validate_cache(p, cache)) != TQ_OK) {
+        return st;
+    }
+    const int batch = pm ? pm->batch : cache->batch;
     if (!d_q || !d_seq_lens || !d_out || !d_workspace || max_seq_len < 1) return TQ_ERR_INVALID_ARG;
     if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
     if (!aligned16(d_q) || !aligned16(d_out) || !aligned16(d_workspace)) return TQ_ERR_ALIGNMENT;
@@ -325,17 +336,19 @@ static tq_status decode_impl(const tq_params* params, const tq_codebook* kcb, co
     }
     const int sms = num_sms_current();
     if (sms <= 0) return TQ_ERR_CUDA;
-    const DecodePlan plan = plan_decode(p, cache->batch, max_seq_len, sms, workspace_bytes);
+    const DecodePlan plan = plan_decode(p, batch, max_seq_len, sms, workspace_bytes);
     if (workspace_bytes < plan.bytes) return TQ_ERR_CAPACITY;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (decode_mma_supported(p)) {
         const cudaError_t e = launch_decode_mma(p, kcb, vcb, *cache, d_q, q_dtype, d_seq_lens, max_seq_len, d_out, plan,
                                                 static_cast<char*>(d_workspace), d_error, sms, s, k_new, v_new,
-                                                kv_dtype);
+                                                kv_dtype, pm);
         if (e != cudaErrorNotSupported) return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
-        // otherwise (a device whose shared-memory window differs) take the general path
+        // otherwise (shared memory too small for two stages, or a device whose
+        // shared-memory window differs) take the general path
     }
+    if (pm) return TQ_ERR_UNSUPPORTED;  // the general kernels read contiguous caches only
     if (append) {  // two launches: append, then attend
         st = quantize_append_impl(params, kcb, vcb, k_new, v_new, kv_dtype, 1, d_seq_lens, true, cache, d_error,
                                   stream);
@@ -384,6 +397,29 @@ extern "C" tq_status tq_decode_attention(const tq_params* params, const tq_codeb
                                          void* stream) {
     return tq::decode_impl(params, kcb, vcb, d_q, q_dtype, cache, d_seq_lens, max_seq_len, d_out, d_workspace,
                            workspace_bytes, d_error, stream, nullptr, nullptr, TQ_BF16);
+}
+
+extern "C" tq_status tq_decode_attention_paged(const tq_params* params, const tq_codebook* kcb,
+                                               const tq_codebook* vcb, const void* d_q, tq_dtype q_dtype,
+                                               const tq_cache* pool, const tq_block_table* table,
+                                               const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
+                                               void* d_workspace, size_t workspace_bytes, uint32_t* d_error,
+                                               void* stream) {
+    if (!table) return TQ_ERR_INVALID_ARG;
+    return tq::decode_impl(params, kcb, vcb, d_q, q_dtype, pool, d_seq_lens, max_seq_len, d_out, d_workspace,
+                           workspace_bytes, d_error, stream, nullptr, nullptr, TQ_BF16, table);
+}
+
+extern "C" tq_status tq_append_decode_attention_paged(const tq_params* params, const tq_codebook* kcb,
+                                                      const tq_codebook* vcb, const void* k_new, const void* v_new,
+                                                      tq_dtype kv_dtype, const void* d_q, tq_dtype q_dtype,
+                                                      const tq_cache* pool, const tq_block_table* table,
+                                                      const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
+                                                      void* d_workspace, size_t workspace_bytes, uint32_t* d_error,
+                                                      void* stream) {
+    if (!k_new || !v_new || !table) return TQ_ERR_INVALID_ARG;
+    return tq::decode_impl(params, kcb, vcb, d_q, q_dtype, pool, d_seq_lens, max_seq_len, d_out, d_workspace,
+                           workspace_bytes, d_error, stream, k_new, v_new, kv_dtype, table);
 }
 
 extern "C" tq_status tq_append_decode_attention(const tq_params* params, const tq_codebook* kcb,

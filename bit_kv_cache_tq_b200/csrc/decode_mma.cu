@@ -131,6 +131,11 @@ struct Args {
     int early;           // TQ_PARAM_PREFETCH_EARLY: the first chunk may be read before the previous kernel ends
     const void* k_new;   // [batch][1][Hkv][d]
     const void* v_new;
+    // paged cache (table non-null): token t of (sequence b, kv head h) is row
+    // (table[b * max_blocks + t / block_size] * hkv + h) * block_size + t % block_size;
+    // `capacity` is then max_blocks * block_size
+    const int32_t* table;
+    int max_blocks, block_size, num_blocks;
     float kbound[8];     // positive decision boundaries, ascending (unused ones +inf)
     float vbound[8];
     float kc32[16];      // fp32 key centroids (QJL residual)
@@ -280,14 +285,60 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         ++qseq;
         return true;
     };
-    // issue the copies of chunk [t0, t0 + n) of a unit into the next stage
-    auto issue_chunk = [&](int unit, int t0, int n) -> bool {
+    // issue the copies of chunk [t0, t0 + n) of a unit into the next stage;
+    // `needed`: every token of the range lies below the sequence's length
+    auto issue_chunk = [&](int unit, int t0, int n, bool needed) -> bool {
         uint32_t full;
         uint8_t* st;
         if (!claim(full, st)) return false;
         const uint32_t dst = ptx::smem_addr(st);
         const size_t row = static_cast<size_t>(unit) * a.capacity + t0;
-        if (a.staged_norms) {
+        if (a.table) {
+            // paged: one copy per block and array.  Block sizes are multiples of
+            // 16 and t0 a multiple of 8, so every piece but the chunk's last
+            // covers a multiple of 8 tokens, and rounding the last up to 8 stays
+            // inside its block (norms then stay 16-byte sized).  A block outside
+            // the pool is not read.
+            // The chunk's table entries (at most MAXB: blocks hold >= 16
+            // tokens) are loaded together, so their latencies overlap.
+            constexpr int MAXB = CHUNK / 16 + 1;
+            const int b = unit / a.hkv, kv = unit % a.hkv, bs = a.block_size;
+            const int end = t0 + ((n + 7) & ~7);
+            const int j0 = t0 / bs, nb = (end - 1) / bs - j0 + 1;
+            const int32_t* trow = a.table + static_cast<size_t>(b) * a.max_blocks + j0;
+            int blk[MAXB];
+#pragma unroll
+            for (int j = 0; j < MAXB; ++j) blk[j] = j < nb ? __ldg(trow + j) : -1;
+            const uint32_t per = VBK + VBV + 4 + (QJL ? zb + 2 : 0);
+            uint32_t bytes = 0;
+            bool bad = false;
+#pragma unroll
+            for (int j = 0; j < MAXB; ++j) {
+                if (j < nb) {
+                    const int ts = max(t0, (j0 + j) * bs), te = min(end, (j0 + j + 1) * bs);
+                    if (blk[j] >= 0 && blk[j] < a.num_blocks) bytes += (te - ts) * per;
+                    else bad = true;
+                }
+            }
+            if (bad && needed && a.err) atomicOr(a.err, TQ_DEVERR_PAGE);
+            ptx::mbar_arrive_expect_tx(full, bytes);
+#pragma unroll
+            for (int j = 0; j < MAXB; ++j) {
+                if (j < nb && blk[j] >= 0 && blk[j] < a.num_blocks) {
+                    const int ts = max(t0, (j0 + j) * bs), cnt = min(end, (j0 + j + 1) * bs) - ts;
+                    const size_t r = (static_cast<size_t>(blk[j]) * a.hkv + kv) * bs + ts % bs;
+                    const uint32_t o = ts - t0;
+                    ptx::bulk_copy_g2s(dst + L.k_off + o * VBK, a.k_codes + r * VBK, cnt * VBK, full);
+                    ptx::bulk_copy_g2s(dst + L.v_off + o * VBV, a.v_codes + r * VBV, cnt * VBV, full);
+                    ptx::bulk_copy_g2s(dst + L.kn_off + o * 2, a.k_norms + r, cnt * 2, full);
+                    ptx::bulk_copy_g2s(dst + L.vn_off + o * 2, a.v_norms + r, cnt * 2, full);
+                    if constexpr (QJL) {
+                        ptx::bulk_copy_g2s(dst + L.z_off + o * zb, a.k_qjl + r * zb, cnt * zb, full);
+                        ptx::bulk_copy_g2s(dst + L.gam_off + o * 2, a.k_gamma + r, cnt * 2, full);
+                    }
+                }
+            }
+        } else if (a.staged_norms) {
             // capacity and t0 are multiples of 8, so rounding n up to 8 tokens
             // stays inside the cache and keeps every 2-byte array 16-byte sized
             const int n8 = (n + 7) & ~7;
@@ -324,7 +375,10 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
     const bool have_first = i < a.n_items;
     const int unit0 = i / a.n_split, split0 = i % a.n_split;
     const int s00 = split0 * a.split_len;
-    if (have_first && a.early && !*abort_flag) spec = issue_chunk(unit0, s00, min(CHUNK, a.capacity - s00));
+    // a split may start past the cache's end when max_seq_len exceeds the
+    // capacity: nothing to fetch speculatively there
+    const bool spec_ok = have_first && s00 < a.capacity;
+    if (spec_ok && a.early && !*abort_flag) spec = issue_chunk(unit0, s00, min(CHUNK, a.capacity - s00), false);
     ptx::wait_prerequisites();
     if (have_first && !*abort_flag) {
         const int b = unit0 / a.hkv, kv = unit0 % a.hkv;
@@ -334,7 +388,7 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
                            static_cast<const uint8_t*>(a.q) + (static_cast<size_t>(b) * a.hq + kv * G) * D * a.q_bytes,
                            qbytes, q0);
         q0_issued = true;
-        if (!a.early) spec = issue_chunk(unit0, s00, min(CHUNK, a.capacity - s00));
+        if (!a.early && spec_ok) spec = issue_chunk(unit0, s00, min(CHUNK, a.capacity - s00), false);
     }
     while (ok) {
         if (i >= a.n_items) break;
@@ -351,6 +405,19 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         }
         const bool empty = w.s0 >= w.s1;
         const bool app = a.append && !empty && w.s1 == w.len;
+        if (first && spec && a.table && !empty) {
+            // the speculative chunk was fetched before the length was known:
+            // report an unmapped block among its valid tokens now
+            const int32_t* trow = a.table + static_cast<size_t>(w.b) * a.max_blocks;
+            const int e = min(w.s1, w.s0 + CHUNK);
+            for (int t = w.s0; t < e; t += a.block_size - t % a.block_size) {
+                const int blk = __ldg(trow + t / a.block_size);
+                if (blk < 0 || blk >= a.num_blocks) {
+                    if (a.err) atomicOr(a.err, TQ_DEVERR_PAGE);
+                    break;
+                }
+            }
+        }
         uint8_t* qslot;
         uint32_t qfull;
         if (!claim_q(qslot, qfull)) break;
@@ -380,7 +447,7 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         int t0 = w.s0;
         if (first && spec) t0 += CHUNK;  // the speculative stage holds the first chunk
         for (; t0 < w.s1; t0 += CHUNK)
-            if (!issue_chunk(w.unit, t0, min(CHUNK, w.s1 - t0))) break;
+            if (!issue_chunk(w.unit, t0, min(CHUNK, w.s1 - t0), true)) break;
         first = false;
         if (!ok) break;
         i = static_cast<int>(gridDim.x + atomicAdd(a.counters + a.units + C_ITEM, 1u));
@@ -579,6 +646,7 @@ struct Consumer {
     // codes, packing, and for keys the QJL sign sketch of the residual).  The
     // result goes to the cache slot and to the patch area, from which the
     // stage holding the token is updated before it is consumed.
+    // (codes == nullptr: fill the patch area only, write nothing to the cache)
     template <int BITS, bool SKETCH>
     __device__ void encode_new(const uint8_t* src, uint8_t* codes, uint16_t* norms, const float* bounds, size_t slot,
                                uint8_t* prow, uint16_t* pnorm, uint8_t* cbytes, float* rbuf) {
@@ -609,10 +677,10 @@ struct Consumer {
             const float q = fminf(fmaxf(rintf(__fmul_rn(x[e], recip)), -127.0f), 127.0f);
             word |= (static_cast<uint32_t>(static_cast<int32_t>(q)) & 0xffu) << (8 * e);
         }
-        reinterpret_cast<uint32_t*>(codes + slot * D)[lane] = word;
+        if (codes) reinterpret_cast<uint32_t*>(codes + slot * D)[lane] = word;
         reinterpret_cast<uint32_t*>(prow)[lane] = word;
         if (lane == 0) {
-            norms[slot] = __half_as_ushort(scale16);
+            if (codes) norms[slot] = __half_as_ushort(scale16);
             *pnorm = __half_as_ushort(scale16);
         }
     }
@@ -649,12 +717,12 @@ struct Consumer {
                 const uint32_t v = cbytes[c];
                 word |= sh >= 0 ? (v << sh) : (v >> -sh);
             }
-            reinterpret_cast<uint32_t*>(codes + slot * (16 * BITS))[lane] = word;
+            if (codes) reinterpret_cast<uint32_t*>(codes + slot * (16 * BITS))[lane] = word;
             reinterpret_cast<uint32_t*>(prow)[lane] = word;
         }
         if (lane == 0) {
             const uint16_t n16 = float_to_half_bits(n);
-            norms[slot] = n16;
+            if (codes) norms[slot] = n16;
             *pnorm = n16;
         }
         if constexpr (SKETCH) {
@@ -682,12 +750,12 @@ struct Consumer {
             uint32_t* qjl = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.k_qjl) + slot * (a.m / 8));
             if (lane == 0) {
                 const uint16_t g16 = float_to_half_bits(sqrtf(g2));
-                const_cast<uint16_t*>(a.k_gamma)[slot] = g16;
+                if (codes) const_cast<uint16_t*>(a.k_gamma)[slot] = g16;
                 *reinterpret_cast<uint16_t*>(smem + L.app + AP_GAM) = g16;
-                qjl[0] = z0;
+                if (codes) qjl[0] = z0;
                 reinterpret_cast<uint32_t*>(pz)[0] = z0;
                 if (a.m > 32) {
-                    qjl[1] = z1;
+                    if (codes) qjl[1] = z1;
                     reinterpret_cast<uint32_t*>(pz)[1] = z1;
                 }
             }
@@ -806,16 +874,28 @@ struct Consumer {
         __half* sq = reinterpret_cast<__half*>(smem + L.sq);
         float* fac = reinterpret_cast<float*>(smem + L.fac);
         if (app && warp < 2) {
-            const size_t slot = static_cast<size_t>(w.unit) * a.capacity + (w.len - 1);
+            // the new token's cache row; a paged cache whose block is outside
+            // the pool gets no write (the token still joins this attention)
+            size_t slot = static_cast<size_t>(w.unit) * a.capacity + (w.len - 1);
+            bool store = true;
+            if (a.table) {
+                const int tok = w.len - 1;
+                const int blk = __ldg(a.table + static_cast<size_t>(w.b) * a.max_blocks + tok / a.block_size);
+                store = blk >= 0 && blk < a.num_blocks;
+                slot = store ? (static_cast<size_t>(blk) * a.hkv + w.kv) * a.block_size + tok % a.block_size : 0;
+                if (!store && warp == 0 && lane == 0 && a.err) atomicOr(a.err, TQ_DEVERR_PAGE);
+            }
             const uint8_t* rows = smem + L.qring + (qseq & 1) * L.qslot + L.qrows;
             uint8_t* ap = smem + L.app;
             if (warp == 0)
-                encode_new<KB, QJL>(rows, const_cast<uint8_t*>(a.k_codes), const_cast<uint16_t*>(a.k_norms), a.kbound,
-                                    slot, ap + AP_K, reinterpret_cast<uint16_t*>(ap + AP_KN), ap + AP_KC,
+                encode_new<KB, QJL>(rows, store ? const_cast<uint8_t*>(a.k_codes) : nullptr,
+                                    const_cast<uint16_t*>(a.k_norms), a.kbound, slot, ap + AP_K,
+                                    reinterpret_cast<uint16_t*>(ap + AP_KN), ap + AP_KC,
                                     reinterpret_cast<float*>(ap + AP_R));
             else
-                encode_new<VB, false>(rows + D * a.new_bytes, const_cast<uint8_t*>(a.v_codes), const_cast<uint16_t*>(a.v_norms),
-                                      a.vbound, slot, ap + AP_V, reinterpret_cast<uint16_t*>(ap + AP_VN), ap + AP_VC,
+                encode_new<VB, false>(rows + D * a.new_bytes, store ? const_cast<uint8_t*>(a.v_codes) : nullptr,
+                                      const_cast<uint16_t*>(a.v_norms), a.vbound, slot, ap + AP_V,
+                                      reinterpret_cast<uint16_t*>(ap + AP_VN), ap + AP_VC,
                                       reinterpret_cast<float*>(ap + AP_R));
         }
         ptx::named_barrier(1, NUM_CONSUMERS);  // every warp is done with the query slot
@@ -1487,7 +1567,7 @@ static uint16_t half_bits(double v) {
 cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const tq_codebook* vcb, const tq_cache& c,
                               const void* q, int q_dtype, const int32_t* seq_lens, int max_len, float* out,
                               const DecodePlan& plan, char* ws, uint32_t* err, int num_sms, cudaStream_t stream,
-                              const void* k_new, const void* v_new, int new_dtype) {
+                              const void* k_new, const void* v_new, int new_dtype, const PageMap* pm) {
     using namespace mmadec;
     const bool k_int8 = p.k_mode == TQ_MODE_INT8, v_int8 = p.v_mode == TQ_MODE_INT8;
     Args a{};
@@ -1547,7 +1627,18 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
         a.kcent[j] = (!k_int8 && j < (1 << p.k_bits)) ? half_bits(kcb->centroids[j] * ak) : 0;
         a.vcent[j] = (!v_int8 && j < (1 << p.v_bits)) ? half_bits(vcb->centroids[j] * av) : 0;
     }
-    a.staged_norms = (c.capacity % 8) == 0;
+    a.staged_norms = (c.capacity % 8) == 0;  // a paged pool's capacity is its block size, a multiple of 16
+    if (pm) {
+        a.table = pm->table;
+        a.max_blocks = pm->max_blocks;
+        a.block_size = pm->block_size;
+        a.num_blocks = pm->num_blocks;
+        a.batch = pm->batch;
+        a.capacity = pm->max_blocks * pm->block_size;
+        a.units = a.batch * p.num_kv_heads;
+        a.n_items = a.units * plan.n_split;
+        a.early = 0;  // the table itself may come from the previous kernel
+    }
     uint32_t words[8];
     rotation_sign_bits(p.seed, 128, words);
     for (int i = 0; i < 4; ++i) a.signs[i] = words[i];

@@ -237,6 +237,21 @@ tq_status validate_cache(const tq_params& p, const tq_cache* c) {
     return TQ_OK;
 }
 
+tq_status validate_pages(const tq_params& p, const tq_cache* pool, const tq_block_table* table, PageMap* pm) {
+    tq_status st = validate_cache(p, pool);
+    if (st != TQ_OK) return st;
+    if (!table || !table->d_table || table->batch < 1 || table->max_blocks < 1) return TQ_ERR_INVALID_ARG;
+    // blocks of whole 16-token tiles keep every per-block copy 16-byte sized
+    if (pool->capacity % 16 != 0) return TQ_ERR_INVALID_ARG;
+    if (static_cast<long long>(table->max_blocks) * pool->capacity > INT32_MAX) return TQ_ERR_INVALID_ARG;
+    pm->table = table->d_table;
+    pm->batch = table->batch;
+    pm->max_blocks = table->max_blocks;
+    pm->block_size = pool->capacity;
+    pm->num_blocks = pool->batch;
+    return TQ_OK;
+}
+
 static long long gcd_ll(long long a, long long b) {
     while (b) {
         const long long r = a % b;

@@ -45,7 +45,11 @@ struct QuantArgs {
     QuantSide side[2];  // 0 = K, 1 = V
     const int32_t* positions;  // per sequence: first slot written, or (pos_from_lens) the length after the append
     uint32_t* err;
-    int batch, n_new, hkv, capacity, pos_from_lens;
+    int batch, n_new, hkv, capacity, pos_from_lens;  // capacity: tokens a sequence may hold
+    // paged cache (table non-null): token t of sequence b is in block
+    // table[b * max_blocks + t / block_size] of the pool
+    const int32_t* table;
+    int max_blocks, block_size, num_blocks;
     uint32_t signs[8];
 };
 
@@ -220,6 +224,15 @@ __global__ void __launch_bounds__(256, 2) quantize_append_kernel(const __grid_co
             if (pos < 0 || pos > a.capacity - a.n_new) {
                 if (a.err && t == 0 && h == 0 && sub == 0 && blockIdx.y == 0) atomicOr(a.err, TQ_DEVERR_POSITION);
                 valid = false;
+            } else if (a.table) {
+                const int tok = pos + t;
+                const int blk = __ldg(a.table + static_cast<size_t>(b) * a.max_blocks + tok / a.block_size);
+                if (blk < 0 || blk >= a.num_blocks) {
+                    if (a.err && sub == 0 && blockIdx.y == 0) atomicOr(a.err, TQ_DEVERR_PAGE);
+                    valid = false;
+                } else {
+                    slot = (static_cast<size_t>(blk) * a.hkv + h) * a.block_size + tok % a.block_size;
+                }
             } else {
                 slot = (static_cast<size_t>(b) * a.hkv + h) * a.capacity + pos + t;
             }
@@ -396,12 +409,24 @@ tq_status tq_quantize_append(const tq_params* params, const tq_codebook* kcb, co
                                     stream);
 }
 
+tq_status tq_quantize_append_paged(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                                   const void* k_new, const void* v_new, tq_dtype dtype, int32_t n_new,
+                                   const int32_t* d_positions, const tq_cache* pool, const tq_block_table* table,
+                                   uint32_t* d_error, void* stream) {
+    if (!params) return TQ_ERR_INVALID_ARG;
+    tq::PageMap pm;
+    const tq_status st = tq::validate_pages(*params, pool, table, &pm);
+    if (st != TQ_OK) return st;
+    return tq::quantize_append_impl(params, kcb, vcb, k_new, v_new, dtype, n_new, d_positions, false, pool, d_error,
+                                    stream, &pm);
+}
+
 }  // extern "C"
 
 tq_status tq::quantize_append_impl(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
                                    const void* k_new, const void* v_new, int dtype, int32_t n_new,
                                    const int32_t* d_positions, bool pos_from_lens, const tq_cache* cache,
-                                   uint32_t* d_error, void* stream) {
+                                   uint32_t* d_error, void* stream, const PageMap* pm) {
     using namespace tq;
     tq_status st = validate_params(params);
     if (st != TQ_OK) return st;
@@ -410,7 +435,8 @@ tq_status tq::quantize_append_impl(const tq_params* params, const tq_codebook* k
     if (!k_new || !v_new || !d_positions || n_new < 1) return TQ_ERR_INVALID_ARG;
     if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
     if (!aligned16(k_new) || !aligned16(v_new)) return TQ_ERR_ALIGNMENT;
-    if (n_new > cache->capacity) return TQ_ERR_CAPACITY;
+    const int capacity = pm ? pm->max_blocks * pm->block_size : cache->capacity;  // tokens per sequence
+    if (n_new > capacity) return TQ_ERR_CAPACITY;
     if (p.k_mode == TQ_MODE_TURBO && (st = validate_codebook(kcb, p.head_dim, p.k_bits)) != TQ_OK) return st;
     if (p.v_mode == TQ_MODE_TURBO && (st = validate_codebook(vcb, p.head_dim, p.v_bits)) != TQ_OK) return st;
     QuantArgs a{};
@@ -430,10 +456,16 @@ tq_status tq::quantize_append_impl(const tq_params* params, const tq_codebook* k
     a.positions = d_positions;
     a.pos_from_lens = pos_from_lens ? 1 : 0;
     a.err = d_error;
-    a.batch = cache->batch;
+    a.batch = pm ? pm->batch : cache->batch;
     a.n_new = n_new;
     a.hkv = p.num_kv_heads;
-    a.capacity = cache->capacity;
+    a.capacity = capacity;
+    if (pm) {
+        a.table = pm->table;
+        a.max_blocks = pm->max_blocks;
+        a.block_size = pm->block_size;
+        a.num_blocks = pm->num_blocks;
+    }
     rotation_sign_bits(p.seed, p.head_dim, a.signs);
     cudaError_t e;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

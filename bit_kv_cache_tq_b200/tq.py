@@ -23,7 +23,7 @@ TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CAPACITY = 0, 1, 2, 3
 TQ_ERR_CUDA, TQ_ERR_TIMEOUT, TQ_ERR_DEVICE, TQ_ERR_ALIGNMENT = 4, 5, 6, 7
 TQ_MODE_TURBO, TQ_MODE_INT8 = 0, 1
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
-TQ_DEVERR_POSITION, TQ_DEVERR_SEQLEN = 0x1, 0x2
+TQ_DEVERR_POSITION, TQ_DEVERR_SEQLEN, TQ_DEVERR_TIMEOUT, TQ_DEVERR_PAGE = 0x1, 0x2, 0x4, 0x8
 TQ_PARAM_PREFETCH_EARLY = 0x1
 
 # every symbol include/tq.h declares
@@ -31,6 +31,7 @@ EXPORTED = (
     "tq_status_string", "tq_abi_version", "tq_codebook_init", "tq_rotation_signs", "tq_qjl_matrix",
     "tq_cache_bytes", "tq_decode_workspace_bytes", "tq_quantize_append", "tq_dequantize",
     "tq_decode_attention", "tq_append_decode_attention", "tq_decode_attention_static", "tq_read_device_error",
+    "tq_quantize_append_paged", "tq_decode_attention_paged", "tq_append_decode_attention_paged",
 )
 
 # Bytes of the library's own decode scratch per device (tq_decode_attention_static).
@@ -67,10 +68,15 @@ class tq_cache(ctypes.Structure):
                 ("qjl_matrix", ctypes.c_void_p)]
 
 
+class tq_block_table(ctypes.Structure):
+    _fields_ = [("d_table", ctypes.c_void_p), ("batch", ctypes.c_int32), ("max_blocks", ctypes.c_int32)]
+
+
 _P = ctypes.POINTER
 _lib.tq_status_string.restype = ctypes.c_char_p
 _lib.tq_status_string.argtypes = [ctypes.c_int]
 _lib.tq_abi_version.restype = ctypes.c_int32
+_lib.tq_abi_version.argtypes = []
 _lib.tq_codebook_init.argtypes = [ctypes.c_int32, ctypes.c_int32, _P(tq_codebook)]
 _lib.tq_rotation_signs.argtypes = [ctypes.c_uint64, ctypes.c_int32, ctypes.c_void_p]
 _lib.tq_qjl_matrix.argtypes = [ctypes.c_uint64, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]
@@ -92,6 +98,18 @@ _lib.tq_decode_attention_static.argtypes = [_P(tq_params), _P(tq_codebook), _P(t
                                             ctypes.c_int, _P(tq_cache), ctypes.c_void_p, ctypes.c_int32,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
 _lib.tq_read_device_error.argtypes = [ctypes.c_void_p, _P(ctypes.c_uint32), ctypes.c_void_p, ctypes.c_int32]
+_lib.tq_quantize_append_paged.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_int, ctypes.c_int32, ctypes.c_void_p,
+                                          _P(tq_cache), _P(tq_block_table), ctypes.c_void_p, ctypes.c_void_p]
+_lib.tq_decode_attention_paged.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
+                                           ctypes.c_int, _P(tq_cache), _P(tq_block_table), ctypes.c_void_p,
+                                           ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                           ctypes.c_void_p, ctypes.c_void_p]
+_lib.tq_append_decode_attention_paged.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
+                                                  ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
+                                                  _P(tq_cache), _P(tq_block_table), ctypes.c_void_p, ctypes.c_int32,
+                                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                                  ctypes.c_void_p]
 for _name in EXPORTED:
     if _name not in ("tq_status_string", "tq_abi_version"):
         getattr(_lib, _name).restype = ctypes.c_int
@@ -175,6 +193,12 @@ def tq_decode_workspace_bytes(params, batch, max_seq_len):
     _check(_lib.tq_decode_workspace_bytes(ctypes.byref(params), batch, max_seq_len, ctypes.byref(n)),
            "tq_decode_workspace_bytes")
     return int(n.value)
+
+
+def block_table(table):
+    """tq_block_table over an int32 CUDA tensor [batch, max_blocks] (kept alive by the caller)."""
+    assert table.dtype == torch.int32 and table.is_cuda and table.is_contiguous() and table.dim() == 2
+    return tq_block_table(_ptr(table), table.shape[0], table.shape[1])
 
 
 # -------------------------------------------------------------- cache storage
@@ -279,6 +303,48 @@ def tq_decode_attention_static(params, kcb, vcb, q, cache, seq_lens, max_seq_len
                                          _ptr(q), _dtype_code(q), ctypes.byref(c), _ptr(seq_lens), max_seq_len,
                                          _ptr(out), _ptr(error), _stream(stream))
     _check(st, "tq_decode_attention_static")
+
+
+def tq_quantize_append_paged(params, kcb, vcb, k_new, v_new, positions, pool, table, error=None, stream=None):
+    """tq_quantize_append on a paged cache: pool from alloc_cache(params, num_blocks, block_size),
+    table an int32 CUDA tensor [batch, max_blocks] of block indices."""
+    assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.dtype == v_new.dtype
+    assert positions.dtype == torch.int32 and positions.is_cuda
+    c, bt = pool.struct(), block_table(table)
+    st = _lib.tq_quantize_append_paged(ctypes.byref(params), kcb and ctypes.byref(kcb), vcb and ctypes.byref(vcb),
+                                       _ptr(k_new), _ptr(v_new), _dtype_code(k_new), k_new.shape[1],
+                                       _ptr(positions), ctypes.byref(c), ctypes.byref(bt), _ptr(error),
+                                       _stream(stream))
+    _check(st, "tq_quantize_append_paged")
+
+
+def tq_decode_attention_paged(params, kcb, vcb, q, pool, table, seq_lens, max_seq_len, out, workspace, error=None,
+                              stream=None):
+    """tq_decode_attention on a paged cache (see tq_quantize_append_paged)."""
+    assert q.is_contiguous() and out.is_contiguous() and out.dtype == torch.float32
+    assert seq_lens.dtype == torch.int32 and seq_lens.is_cuda
+    c, bt = pool.struct(), block_table(table)
+    st = _lib.tq_decode_attention_paged(ctypes.byref(params), kcb and ctypes.byref(kcb), vcb and ctypes.byref(vcb),
+                                        _ptr(q), _dtype_code(q), ctypes.byref(c), ctypes.byref(bt), _ptr(seq_lens),
+                                        max_seq_len, _ptr(out), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _ptr(error), _stream(stream))
+    _check(st, "tq_decode_attention_paged")
+
+
+def tq_append_decode_attention_paged(params, kcb, vcb, k_new, v_new, q, pool, table, seq_lens, max_seq_len, out,
+                                     workspace, error=None, stream=None):
+    """tq_append_decode_attention on a paged cache (see tq_quantize_append_paged)."""
+    assert q.is_contiguous() and out.is_contiguous() and out.dtype == torch.float32
+    assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.dtype == v_new.dtype
+    assert seq_lens.dtype == torch.int32 and seq_lens.is_cuda
+    c, bt = pool.struct(), block_table(table)
+    st = _lib.tq_append_decode_attention_paged(ctypes.byref(params), kcb and ctypes.byref(kcb),
+                                               vcb and ctypes.byref(vcb), _ptr(k_new), _ptr(v_new),
+                                               _dtype_code(k_new), _ptr(q), _dtype_code(q), ctypes.byref(c),
+                                               ctypes.byref(bt), _ptr(seq_lens), max_seq_len, _ptr(out),
+                                               _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                               _ptr(error), _stream(stream))
+    _check(st, "tq_append_decode_attention_paged")
 
 
 def tq_read_device_error(error, stream=None, timeout_ms=2000):

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 2
+#define TQ_ABI_VERSION 3
 
 typedef enum tq_status {
     TQ_OK = 0,
@@ -69,6 +69,8 @@ typedef enum tq_dtype { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
 #define TQ_DEVERR_SEQLEN 0x2u   /* decode: seq_lens[b] < 1, > capacity or > max_seq_len */
 #define TQ_DEVERR_TIMEOUT 0x4u  /* decode: a bounded wait inside a kernel ran out (about 1 s);
                                    the output is not valid and the workspace must be zeroed again */
+#define TQ_DEVERR_PAGE 0x8u     /* paged cache: a block-table entry a kernel needed lies outside
+                                   the pool; that access was skipped */
 
 /*
  * Lloyd-Max codebook for one (head_dim, bits) pair.  [tqai] section
@@ -314,6 +316,62 @@ tq_status tq_append_decode_attention(const tq_params* params, const tq_codebook*
                                      tq_dtype q_dtype, const tq_cache* cache, const int32_t* d_seq_lens,
                                      int32_t max_seq_len, float* d_out, void* d_workspace, size_t workspace_bytes,
                                      uint32_t* d_error, void* stream);
+
+/*
+ * Paged cache.  [inferrs] manages its compressed cache with PagedAttention
+ * ("二、inferrs：TurboQuant 轻量推理服务器"); the pages give no page format,
+ * so this one follows the usual block-table scheme.  The pool is a tq_cache whose
+ * `batch` counts physical blocks and whose `capacity` is the block size in
+ * tokens, a multiple of 16: every array keeps the layout above,
+ * [block][Hkv][block_size][...].  Token t of sequence b lives in block
+ * d_table[b * max_blocks + t / block_size], row t % block_size.
+ *   d_table     device int32 [batch][max_blocks]; entries of the blocks
+ *               below a sequence's length (and those an append writes)
+ *               must lie in [0, pool.batch).  A kernel that meets an entry
+ *               outside the pool skips the access and sets TQ_DEVERR_PAGE
+ *               (the decode may read entries past a sequence's length and
+ *               ignores the ones outside the pool).
+ *   batch       sequences.
+ *   max_blocks  entries per sequence: a sequence holds at most
+ *               max_blocks * block_size tokens.
+ */
+typedef struct tq_block_table {
+    const int32_t* d_table;
+    int32_t batch;
+    int32_t max_blocks;
+} tq_block_table;
+
+/*
+ * tq_quantize_append on a paged cache: positions count tokens of each
+ * sequence (0 .. max_blocks * block_size - n_new) as before, and every token
+ * goes to the block the table names.
+ */
+tq_status tq_quantize_append_paged(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                                   const void* k_new, const void* v_new, tq_dtype dtype, int32_t n_new,
+                                   const int32_t* d_positions, const tq_cache* pool, const tq_block_table* table,
+                                   uint32_t* d_error, void* stream);
+
+/*
+ * tq_decode_attention and tq_append_decode_attention on a paged cache.  The
+ * workspace is sized by tq_decode_workspace_bytes(params, table->batch,
+ * max_seq_len).  Only the tensor-core path reads a paged cache (d = 128 and
+ * the modes it takes, see tq_append_decode_attention); other configurations
+ * return TQ_ERR_UNSUPPORTED.  The kernel copies each chunk of a sequence
+ * block by block, so blocks of 64 or more tokens keep the copies large.
+ * TQ_PARAM_PREFETCH_EARLY is ignored here.
+ */
+tq_status tq_decode_attention_paged(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                                    const void* d_q, tq_dtype q_dtype, const tq_cache* pool,
+                                    const tq_block_table* table, const int32_t* d_seq_lens, int32_t max_seq_len,
+                                    float* d_out, void* d_workspace, size_t workspace_bytes, uint32_t* d_error,
+                                    void* stream);
+tq_status tq_append_decode_attention_paged(const tq_params* params, const tq_codebook* kcb,
+                                           const tq_codebook* vcb, const void* k_new, const void* v_new,
+                                           tq_dtype kv_dtype, const void* d_q, tq_dtype q_dtype,
+                                           const tq_cache* pool, const tq_block_table* table,
+                                           const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
+                                           void* d_workspace, size_t workspace_bytes, uint32_t* d_error,
+                                           void* stream);
 
 /* Bytes of the library's own decode scratch on each device. */
 #define TQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)16 << 20)

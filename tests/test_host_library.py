@@ -29,8 +29,31 @@ def test_library_exports_every_declared_symbol():
     assert set(tq.EXPORTED) <= set(declared)
 
 
+def _declared_arities():
+    """Parameter count of every function declared in include/tq.h."""
+    with open(os.path.join(ROOT, "include", "tq.h"), encoding="utf-8") as fh:
+        text = fh.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(tq_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text):
+        args = m.group(2).strip()
+        out[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_declares_every_argument_type():
+    """ctypes passes an undeclared integer argument as a 32-bit int: every
+    exported call must declare its argument types, one per C parameter (a
+    size_t passed as int reads garbage in its upper half)."""
+    arity = _declared_arities()
+    for name in tq.EXPORTED:
+        f = getattr(tq.library(), name)
+        assert f.argtypes is not None, name
+        assert len(f.argtypes) == arity[name], (name, len(f.argtypes), arity[name])
+
+
 def test_abi_version_and_status_strings():
-    assert tq.tq_abi_version() == 2
+    assert tq.tq_abi_version() == 3
     for st in range(8):
         assert tq.tq_status_string(st)
     assert tq.tq_status_string(99) == "unknown status"
@@ -206,3 +229,38 @@ def test_append_decode_rejects_bad_arguments_before_launch():
     assert lib.tq_append_decode_attention(*args, fake, None, tq.TQ_BF16, *tail) == tq.TQ_ERR_INVALID_ARG
     assert lib.tq_append_decode_attention(*args, fake + 4, fake, tq.TQ_BF16, *tail) == tq.TQ_ERR_ALIGNMENT
     assert lib.tq_append_decode_attention(*args, fake, fake, 7, *tail) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_paged_entry_points_reject_bad_arguments_before_launch():
+    """Block-table checks (block size a multiple of 16, a table, at least one
+    sequence and block) and the paged capacity run before any CUDA call."""
+    lib = tq.library()
+    p = tq.make_params(128, 32, 8)
+    kcb, vcb = tq.tq_codebook_init(128, 4), tq.tq_codebook_init(128, 2)
+    fake = 1 << 20
+    pool = tq.tq_cache(8, 64, fake, fake, None, None, fake, fake, None)  # 8 blocks of 64 tokens
+    table = tq.tq_block_table(fake, 2, 4)                                  # 2 sequences x 4 blocks
+    args = (ctypes.byref(p), ctypes.byref(kcb), ctypes.byref(vcb))
+
+    def append(pool_, table_, n_new=1):
+        return lib.tq_quantize_append_paged(*args, fake, fake, tq.TQ_BF16, n_new, fake, ctypes.byref(pool_),
+                                            table_ and ctypes.byref(table_), None, None)
+
+    def decode(pool_, table_):
+        return lib.tq_decode_attention_paged(*args, fake, tq.TQ_BF16, ctypes.byref(pool_),
+                                             table_ and ctypes.byref(table_), fake, 64, fake, None, 0, None, None)
+
+    assert append(pool, None) == tq.TQ_ERR_INVALID_ARG
+    assert append(pool, tq.tq_block_table(None, 2, 4)) == tq.TQ_ERR_INVALID_ARG
+    assert append(pool, tq.tq_block_table(fake, 0, 4)) == tq.TQ_ERR_INVALID_ARG
+    assert append(pool, tq.tq_block_table(fake, 2, 0)) == tq.TQ_ERR_INVALID_ARG
+    assert append(tq.tq_cache(8, 24, fake, fake, None, None, fake, fake, None), table) == tq.TQ_ERR_INVALID_ARG
+    # a sequence holds max_blocks * block_size = 256 tokens
+    assert append(pool, table, n_new=257) == tq.TQ_ERR_CAPACITY
+    assert decode(pool, None) == tq.TQ_ERR_INVALID_ARG
+    assert decode(tq.tq_cache(8, 8, fake, fake, None, None, fake, fake, None), table) == tq.TQ_ERR_INVALID_ARG
+    # null workspace
+    assert decode(pool, table) == tq.TQ_ERR_INVALID_ARG
+    assert lib.tq_append_decode_attention_paged(*args, None, fake, tq.TQ_BF16, fake, tq.TQ_BF16,
+                                                ctypes.byref(pool), ctypes.byref(table), fake, 64, fake, fake,
+                                                1 << 20, None, None) == tq.TQ_ERR_INVALID_ARG
