@@ -312,19 +312,19 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
             const uint32_t per = VBK + VBV + 4 + (QJL ? zb + 2 : 0);
             uint32_t bytes = 0;
             bool bad = false;
-#pragma unroll
-            for (int j = 0; j < MAXB; ++j) {
-                if (j < nb) {
-                    const int ts = max(t0, (j0 + j) * bs), te = min(end, (j0 + j + 1) * bs);
-                    if (blk[j] >= 0 && blk[j] < a.num_blocks) bytes += (te - ts) * per;
-                    else bad = true;
-                }
+            // (the loops below stay rolled: unrolled, their copies bloat the
+            // kernel's code and slow every configuration)
+#pragma unroll 1
+            for (int j = 0; j < nb; ++j) {
+                const int ts = max(t0, (j0 + j) * bs), te = min(end, (j0 + j + 1) * bs);
+                if (blk[j] >= 0 && blk[j] < a.num_blocks) bytes += (te - ts) * per;
+                else bad = true;
             }
             if (bad && needed && a.err) atomicOr(a.err, TQ_DEVERR_PAGE);
             ptx::mbar_arrive_expect_tx(full, bytes);
-#pragma unroll
-            for (int j = 0; j < MAXB; ++j) {
-                if (j < nb && blk[j] >= 0 && blk[j] < a.num_blocks) {
+#pragma unroll 1
+            for (int j = 0; j < nb; ++j) {
+                if (blk[j] >= 0 && blk[j] < a.num_blocks) {
                     const int ts = max(t0, (j0 + j) * bs), cnt = min(end, (j0 + j + 1) * bs) - ts;
                     const size_t r = (static_cast<size_t>(blk[j]) * a.hkv + kv) * bs + ts % bs;
                     const uint32_t o = ts - t0;
