@@ -365,14 +365,16 @@ def decode_configs(dev, reps=10):
     4 cache copies), 70B-shaped long context (B=4, Hq=64, Hkv=8, 131072
     tokens, K3 + 64-bit QJL / V2, Sparse V at 1e-6), and the Llama-3-8B-shaped
     layer (B=1, 32768 tokens, 4 cache copies) with int8 keys and 2-bit values
-    (the mixed setting) and as an int8 boundary layer (int8 keys and values).
+    (the mixed setting) and as an int8 boundary layer (int8 keys and values),
+    the latter also with 64 query heads (groups of 8).
     A kb of 8 below stands for int8 (one byte per channel, fp16 scale)."""
     from bit_kv_cache_tq_b200 import inputs, tq
     res = {}
     cases = [("batched_ragged_b16_k3v2", 16, 32, 8192, 3, 2, 0, 0.0, 4),
              ("long_context_b4_hq64_128k_k3qjl_v2_sparse", 4, 64, 131072, 3, 2, 64, 1e-6, 1),
              ("llama8b_32k_int8k_v2", 1, 32, 32768, 8, 2, 0, 0.0, 4),
-             ("llama8b_32k_int8k_int8v", 1, 32, 32768, 8, 8, 0, 0.0, 4)]
+             ("llama8b_32k_int8k_int8v", 1, 32, 32768, 8, 8, 0, 0.0, 4),
+             ("hq64_32k_int8k_int8v", 1, 64, 32768, 8, 8, 0, 0.0, 4)]
     for name, bsz, hq, tmax, kb, vb, m, tau, copies in cases:
         modes = dict(k_mode=tq.TQ_MODE_INT8 if kb == 8 else tq.TQ_MODE_TURBO,
                      v_mode=tq.TQ_MODE_INT8 if vb == 8 else tq.TQ_MODE_TURBO,

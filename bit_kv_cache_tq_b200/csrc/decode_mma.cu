@@ -76,6 +76,10 @@ constexpr uint32_t LUT_BYTES = 65536;        // 256 entries x 256 B
 // and table lookups carry it as an immediate offset.
 constexpr uint32_t WINDOW = 1024;
 constexpr uint32_t QHDR = 32;                 // item header at the front of a query slot
+// The warps' partials are combined this many query heads at a time, so the
+// combine buffer stays at 22.5 KB for any GQA group (8 or 16 heads would
+// otherwise crowd out the second stage).
+constexpr int MERGE_HEADS = 4;
 // Row strides (halves) of the fp16 query and sketch buffers: 2 words past a
 // multiple of 32 banks, so the 8-byte fragment loads of a half-warp (lane
 // groups g = 0..3 at rows g, columns 16 t) hit 32 distinct banks.
@@ -174,10 +178,11 @@ __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int
     L.app = align16(L.sq + 8 * nt * SQ_STRIDE * 2);    // appended token: packed rows, norms, scratch
     L.fac = L.app + APP_BYTES;                         // float F1[16], F2[16]
     L.merge = L.fac + 32 * 4;
-    // merge area, reused: per-warp partials [CW][g][128]; the final merge's
-    // [g][128] outputs and [CW][n_split] weights; the prologue's [8 nt][128]
-    // sketch staging; the table build's 768 compact words
-    uint32_t merge = CW * g * D * 4;
+    // merge area, reused: per-warp partials of up to MERGE_HEADS heads at a
+    // time [CW][MERGE_HEADS][128]; the final merge's [g][128] outputs and
+    // [CW][n_split] weights; the prologue's [8 nt][128] sketch staging; the
+    // table build's 768 compact words
+    uint32_t merge = CW * (g < MERGE_HEADS ? g : MERGE_HEADS) * D * 4;
     const uint32_t fin = (g * D + CW * n_split) * 4;
     if (fin > merge) merge = fin;
     if (8u * nt * D * 4 > merge) merge = 8 * nt * D * 4;
@@ -1188,32 +1193,35 @@ struct Consumer {
                 if (g == 0) ml[warp * 16 + nt * 8 + 2 * t + h] = make_float2(S.m[nt][h], l);
             }
         const float unscale = S.vscale > 0.f ? 1.0f / S.vscale : 0.f;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int h0 = nt * 8 + 2 * t;  // heads h0, h0 + 1 of this lane's columns
-                float* mw = merge + (warp * G + h0) * D;
-                const int c_lo = 16 * g + 2 * i, c_hi = c_lo + 1;
-                if (h0 < G) {
-                    mw[c_lo] = S.acc[nt][i][0] * unscale;
-                    mw[c_hi] = S.acc[nt][i][2] * unscale;
-                }
-                if (h0 + 1 < G) {
-                    mw[D + c_lo] = S.acc[nt][i][1] * unscale;
-                    mw[D + c_hi] = S.acc[nt][i][3] * unscale;
-                }
-            }
-        ptx::named_barrier(1, NUM_CONSUMERS);
         const size_t pbase = (static_cast<size_t>(w.unit) * a.n_split + w.split) * G;
-        // every output column is one weighted sum over the warps, with the
-        // weights 2^(m_w - M) of its head (each thread forms them; the thread
-        // of a head's first column also writes the split's (M, L))
-        {
+        const int GM = G < MERGE_HEADS ? G : MERGE_HEADS;  // heads per combine pass
+        for (int hb = 0; hb < G; hb += GM) {
+            if (hb > 0) ptx::named_barrier(1, NUM_CONSUMERS);  // the previous pass has read the buffer
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int h0 = nt * 8 + 2 * t;  // heads h0, h0 + 1 of this lane's columns (same pass)
+                    if (h0 < hb || h0 >= hb + GM) continue;
+                    float* mw = merge + (warp * GM + h0 - hb) * D;
+                    const int c_lo = 16 * g + 2 * i, c_hi = c_lo + 1;
+                    if (h0 < G) {
+                        mw[c_lo] = S.acc[nt][i][0] * unscale;
+                        mw[c_hi] = S.acc[nt][i][2] * unscale;
+                    }
+                    if (h0 + 1 < G) {
+                        mw[D + c_lo] = S.acc[nt][i][1] * unscale;
+                        mw[D + c_hi] = S.acc[nt][i][3] * unscale;
+                    }
+                }
+            ptx::named_barrier(1, NUM_CONSUMERS);
+            // every output column is one weighted sum over the warps, with the
+            // weights 2^(m_w - M) of its head (each thread forms them; the
+            // thread of a head's first column also writes the split's (M, L))
             const float4* m4 = reinterpret_cast<const float4*>(merge);
             float4* dst4 = reinterpret_cast<float4*>(a.ws_acc + pbase * D);
-            for (int idx = tid; idx < G * (D / 4); idx += NUM_CONSUMERS) {
-                const int h = idx / (D / 4), c4 = idx % (D / 4);
+            for (int idx = tid; idx < GM * (D / 4); idx += NUM_CONSUMERS) {
+                const int hl = idx / (D / 4), h = hb + hl, c4 = idx % (D / 4);
                 float mx = -INFINITY;
 #pragma unroll
                 for (int ww = 0; ww < CW; ++ww)
@@ -1225,7 +1233,7 @@ struct Consumer {
                     const float2 mlw = ml[ww * 16 + h];
                     const float f = (mlw.y > 0.f && mx > -INFINITY) ? ptx::ex2(mlw.x - mx) : 0.f;
                     l = fmaf(mlw.y, f, l);
-                    const float4 v = m4[(ww * G + h) * (D / 4) + c4];
+                    const float4 v = m4[(ww * GM + hl) * (D / 4) + c4];
                     acc4.x = fmaf(v.x, f, acc4.x);
                     acc4.y = fmaf(v.y, f, acc4.y);
                     acc4.z = fmaf(v.z, f, acc4.z);

@@ -254,11 +254,12 @@ def test_attention_over_int8_sides(k_mode, v_mode):
 
 
 @pytest.mark.parametrize("hq,v_bits,lens", [(32, 2, [3001, 1700]), (64, 4, [1200, 1]), (16, 3, [777]),
-                                           (32, "int8", [3001, 1700]), (64, "int8", [1200, 1]), (16, "int8", [777])])
+                                           (32, "int8", [3001, 1700]), (64, "int8", [1200, 1]), (16, "int8", [777]),
+                                           (128, 2, [900, 333]), (128, "int8", [900, 333])])
 def test_int8_keys_turbo_values_ragged(hq, v_bits, lens):
     """int8 keys beside turbo values (or int8 values: a boundary layer) in the
     tensor-core kernel: several chunks, ragged tails, a one-token sequence,
-    GQA groups of 2, 4 and 8."""
+    GQA groups of 2, 4, 8 and 16 (16 combines the warps in four passes)."""
     if v_bits == "int8":
         layer = H.Layer(128, hq, 8, k_mode=tq.TQ_MODE_INT8, v_mode=tq.TQ_MODE_INT8, seed=19)
     else:
@@ -344,9 +345,9 @@ def test_workspace_reused_across_batches_and_lengths():
 
 
 def test_group16_d128():
-    """d = 128 with 16 query heads per kv head (the tensor-core kernel's merge
-    buffers leave no room for its stages, so the general kernels serve it),
-    fp32 queries, ragged lengths, K4/V3."""
+    """d = 128 with 16 query heads per kv head (the tensor-core kernel with two
+    8-head column tiles, its warps combined in four passes), fp32 queries,
+    ragged lengths, K4/V3."""
     layer = H.Layer(128, 32, 2, k_bits=4, v_bits=3, seed=23)
     t = 1100
     k = inputs.lognormal_kv(2, t, 2, 128, seed=14, layer=23, which=inputs.K)
