@@ -1,17 +1,23 @@
 // Decode attention from the compressed cache on the tensor cores (sm_100a),
-// head dimension 128, TURBO keys and values, GQA groups of up to 16.
+// head dimension 128, GQA groups of up to 16: TURBO keys (optionally with the
+// QJL sketch) or int8 keys, TURBO values or (beside int8 keys) int8 values;
+// contiguous or paged (block-table) caches.
 //
 // Pages (by title):
 //   [google]  "Google 最新極限壓縮算法，砸碎大模型本地部署的內存墻，8 倍提升！",
 //             sections "再看速度" and "第二步：QJL —— 1 bit 清理殘差"
-//   [inferrs] "inferrs & TurboQuant：本地 LLM 推理的内存革命", section "Sparse V：速度加成"
+//   [inferrs] "inferrs & TurboQuant：本地 LLM 推理的内存革命", sections "Sparse V：速度加成",
+//             "三个反直觉的关键发现" (int8 boundary layers, int8 keys with 2-bit
+//             values) and "二、inferrs：TurboQuant 轻量推理服务器" (PagedAttention)
 //   [tqai]    "TurboQuant：让大模型本地推理内存占用降低80%的KV缓存压缩技术", section
 //             "TurboQuant的核心创新"
 //
 // What is computed is the same as decode_split_kernel in decode.cu:
 //   s_i = sm_scale ||k_i|| (<q~, c[code_i]> + gamma_i sqrt(pi/2)/m <S q~, 2z_i - 1>),
 //   softmax over the sequence, acc = sum_i p_i ||v_i|| c[code_i] in the rotated
-//   domain, and one inverse rotation of acc / sum_i p_i.
+//   domain, and one inverse rotation of acc / sum_i p_i.  An int8 side uses
+//   its scale for the norm and its bytes for the centroids, in the original
+//   domain (unrotated query for int8 keys; no inverse rotation for int8 values).
 //
 // How (one persistent thread block per SM):
 //  * Work items are (sequence, kv head, token split).  A producer thread takes
