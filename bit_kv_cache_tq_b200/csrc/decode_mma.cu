@@ -1667,8 +1667,9 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
     const Layout fixed = layout(kb, vb, nt, 0, p.qjl_dims, a.group, a.q_bytes, a.append ? a.new_bytes : 0, a.n_split);
     int stages = static_cast<int>((232448u - fixed.total) / fixed.stage_bytes);
     if (stages > 8) stages = 8;
-    // large groups (16 query heads per kv head) leave no room for two stages
-    // beside the per-warp merge buffers: the caller takes the general kernels
+    // fewer than two stages (an all-int8 layer with 16-head groups of fp32
+    // queries: its 92 KB stages and query slots do not fit twice): the caller
+    // takes the general kernels
     if (stages < 2) return cudaErrorNotSupported;
     a.stages = stages;
     const size_t smem =

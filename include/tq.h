@@ -304,8 +304,9 @@ tq_status tq_decode_attention(const tq_params* params, const tq_codebook* kcb, c
  * The new token is encoded exactly as tq_quantize_append encodes it (the
  * cache afterwards holds what tq_quantize_append would have written, up to
  * codes within the boundary window).  On the tensor-core path (d = 128;
- * turbo or int8 K; turbo V, or int8 V beside int8 K with at most 4 query
- * heads per kv head) this is one kernel: the block that owns a sequence's
+ * turbo or int8 K; turbo V, or int8 V beside int8 K; up to 16 query heads
+ * per kv head, except 16 fp32 queries per kv head on an all-int8 layer) this
+ * is one kernel: the block that owns a sequence's
  * last token split encodes the token while the cache streams in.  Other
  * configurations run tq_quantize_append's kernel and then the attention
  * kernels.  A seq_len outside [1, capacity] skips that sequence's append and
