@@ -1226,7 +1226,8 @@ struct Consumer {
             // thread of a head's first column also writes the split's (M, L))
             const float4* m4 = reinterpret_cast<const float4*>(merge);
             float4* dst4 = reinterpret_cast<float4*>(a.ws_acc + pbase * D);
-            for (int idx = tid; idx < GM * (D / 4); idx += NUM_CONSUMERS) {
+            const int np = G - hb < GM ? G - hb : GM;  // heads of this pass (the last may hold fewer)
+            for (int idx = tid; idx < np * (D / 4); idx += NUM_CONSUMERS) {
                 const int hl = idx / (D / 4), h = hb + hl, c4 = idx % (D / 4);
                 float mx = -INFINITY;
 #pragma unroll

@@ -255,11 +255,13 @@ def test_attention_over_int8_sides(k_mode, v_mode):
 
 @pytest.mark.parametrize("hq,v_bits,lens", [(32, 2, [3001, 1700]), (64, 4, [1200, 1]), (16, 3, [777]),
                                            (32, "int8", [3001, 1700]), (64, "int8", [1200, 1]), (16, "int8", [777]),
-                                           (128, 2, [900, 333]), (128, "int8", [900, 333])])
+                                           (128, 2, [900, 333]), (128, "int8", [900, 333]),
+                                           (48, 2, [1000, 17]), (104, "int8", [700])])
 def test_int8_keys_turbo_values_ragged(hq, v_bits, lens):
     """int8 keys beside turbo values (or int8 values: a boundary layer) in the
     tensor-core kernel: several chunks, ragged tails, a one-token sequence,
-    GQA groups of 2, 4, 8 and 16 (16 combines the warps in four passes)."""
+    GQA groups of 2, 4, 6, 8, 13 and 16 (groups above 4 combine the warps in
+    passes of four heads, the last pass of 6 and 13 a partial one)."""
     if v_bits == "int8":
         layer = H.Layer(128, hq, 8, k_mode=tq.TQ_MODE_INT8, v_mode=tq.TQ_MODE_INT8, seed=19)
     else:
