@@ -264,3 +264,19 @@ def test_paged_entry_points_reject_bad_arguments_before_launch():
     assert lib.tq_append_decode_attention_paged(*args, None, fake, tq.TQ_BF16, fake, tq.TQ_BF16,
                                                 ctypes.byref(pool), ctypes.byref(table), fake, 64, fake, fake,
                                                 1 << 20, None, None) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_binding_constants_match_the_header():
+    """Status codes, modes, dtypes, device-error bits and flags: the binding's
+    numbers are the header's."""
+    with open(os.path.join(ROOT, "include", "tq.h"), encoding="utf-8") as fh:
+        text = fh.read()
+    defines = {m.group(1): int(m.group(2), 16) for m in re.finditer(r"#define (TQ_[A-Z_]+) (0x[0-9a-fA-F]+)u", text)}
+    enums = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(TQ_[A-Z0-9_]+) = (\d+)", text)}
+    for name in ("TQ_DEVERR_POSITION", "TQ_DEVERR_SEQLEN", "TQ_DEVERR_TIMEOUT", "TQ_DEVERR_PAGE",
+                 "TQ_PARAM_PREFETCH_EARLY"):
+        assert getattr(tq, name) == defines[name], name
+    for name in ("TQ_OK", "TQ_ERR_INVALID_ARG", "TQ_ERR_UNSUPPORTED", "TQ_ERR_CAPACITY", "TQ_ERR_CUDA",
+                 "TQ_ERR_TIMEOUT", "TQ_ERR_DEVICE", "TQ_ERR_ALIGNMENT", "TQ_MODE_TURBO", "TQ_MODE_INT8",
+                 "TQ_F32", "TQ_BF16", "TQ_F16"):
+        assert getattr(tq, name) == enums[name], name
