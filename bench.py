@@ -655,7 +655,7 @@ def run_tq(args, world, rank, local):
             "gpu_launches": launches_per_step * steps,
             "clocks": clocks.summary(),
         }
-        if not args.quick:
+        if not args.quick and world == 1:  # the other workloads: single-GPU runs only (N GPUs stay held meanwhile)
             line["bf16_baseline"] = bf16_sdpa_baseline(dev)
             line["decode_configs"] = decode_configs(dev)
             line["paged_decode"] = {"workload": "llama3-8b-shaped layer, 32768 tokens, K4/V2, through a block "
