@@ -30,6 +30,7 @@ codebook   Lloyd-Max codebook for the rotated-coordinate density, and the
 quantize   norm, codes, bit packing, QJL residual bits, int8 mode,
            dequantisation.
 attention  decode attention over dequantised vectors, Sparse-V bounds.
+paging     the paged cache layout: which block row holds a token.
 """
 
-from . import rng, rotation, codebook, quantize, attention  # noqa: F401
+from . import rng, rotation, codebook, quantize, attention, paging  # noqa: F401
