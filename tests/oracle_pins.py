@@ -8,8 +8,9 @@ that some pin fails.
 
 What pins what (none of them retypes the oracle's own formula):
 * SplitMix64: published first outputs from state 0 (golden file).
-* signs / QJL matrix: sign balance; Kolmogorov-Smirnov against scipy's
-  normal CDF.
+* signs / QJL matrix: the first signs and the first Box-Muller pair derived
+  by hand from the published SplitMix64 words (golden file); sign balance;
+  Kolmogorov-Smirnov against scipy's normal CDF.
 * rotation: scipy.linalg.hadamard; H H^T = d I in integers; norm
   preservation and exact inversion (page: the transform is orthogonal and
   invertible); closed form of the image of a basis vector.
@@ -53,6 +54,25 @@ def pin_sign_balance(rng):
     assert abs(np.mean(s)) < 4.0 / math.sqrt(8192)
     # signs of different seeds are not the same vector
     assert not np.array_equal(rng.rotation_signs(1, 256), rng.rotation_signs(2, 256))
+
+
+def pin_first_signs(rng):
+    """Seed 0: signs from bit 63 of the published SplitMix64 outputs (golden)."""
+    gold = read_golden("qjl_first_pair.txt")
+    want = np.array([float(x) for x in gold["signs_seed0"]])
+    assert np.array_equal(rng.rotation_signs(0, len(want)), want)
+
+
+def pin_first_qjl_pair(rng):
+    """The sketch stream of seed 0x5155414E544A4C00 starts at state 0, so its
+    first Box-Muller pair follows by hand from the published words (golden):
+    u1 from the first word, cos term first, row-major fill."""
+    gold = read_golden("qjl_first_pair.txt")
+    seed = int(gold["qjl_seed"][0], 16)
+    s = rng.qjl_matrix(seed, 64, 128)
+    want = np.array([float(gold["qjl_s00"][0]), float(gold["qjl_s01"][0])]).astype(np.float32)
+    assert np.array_equal(s[0, :2], want.astype(np.float64)), (s[0, :2], want)
+    assert abs(s[0, 0] - float(gold["qjl_s00"][0])) < 1e-6 and abs(s[0, 1] - float(gold["qjl_s01"][0])) < 1e-6
 
 
 def pin_qjl_gaussian(rng):

@@ -159,3 +159,49 @@ def test_rotated_path_without_key_norm(monkeypatch):
 def test_splitmix_wrong_increment(monkeypatch):
     monkeypatch.setattr(rng, "GOLDEN_GAMMA", 0x9E3779B97F4A7C13)
     _fails(P.pin_splitmix64, rng)
+
+
+# ----------------------------------------------- random-number readings
+def test_sign_from_bit_zero(monkeypatch):
+    def bad_signs(seed, d):
+        words = rng.splitmix64(seed, d)
+        return np.array([-1.0 if w & 1 else 1.0 for w in words], dtype=np.float64)
+    monkeypatch.setattr(rng, "rotation_signs", bad_signs)
+    _fails(P.pin_first_signs, rng)
+
+
+def test_sign_inverted(monkeypatch):
+    real = rng.rotation_signs
+    monkeypatch.setattr(rng, "rotation_signs", lambda seed, d: -real(seed, d))
+    _fails(P.pin_first_signs, rng)
+
+
+def _box_muller(seed, m, d, swap_u=False, sin_first=False, column_major=False):
+    n = m * d
+    words = rng.splitmix64(seed ^ rng.QJL_STREAM_XOR, n + 1)
+    vals = []
+    for k in range((n + 1) // 2):
+        u1 = (words[2 * k] >> 11) * 2.0 ** -53
+        u2 = (words[2 * k + 1] >> 11) * 2.0 ** -53
+        if swap_u:
+            u1, u2 = u2, u1
+        r = math.sqrt(-2.0 * math.log(1.0 - u1))
+        c, s = r * math.cos(2.0 * math.pi * u2), r * math.sin(2.0 * math.pi * u2)
+        vals += [s, c] if sin_first else [c, s]
+    a = np.array(vals[:n], dtype=np.float64).astype(np.float32).astype(np.float64)
+    return a.reshape(d, m).T.copy() if column_major else a.reshape(m, d)
+
+
+@pytest.mark.parametrize("kind", ["swap_u", "sin_first", "column_major"])
+def test_box_muller_readings(monkeypatch, kind):
+    monkeypatch.setattr(rng, "qjl_matrix", lambda seed, m, d: _box_muller(seed, m, d, **{kind: True}))
+    _fails(P.pin_first_qjl_pair, rng)
+
+
+def test_box_muller_control():
+    # the helper above, with no mistake planted, passes the pin
+    class R:
+        pass
+    r = R()
+    r.qjl_matrix = lambda seed, m, d: _box_muller(seed, m, d)
+    P.pin_first_qjl_pair(r)

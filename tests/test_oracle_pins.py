@@ -13,6 +13,14 @@ def test_sign_balance():
     P.pin_sign_balance(rng)
 
 
+def test_first_rotation_signs():
+    P.pin_first_signs(rng)
+
+
+def test_first_qjl_pair():
+    P.pin_first_qjl_pair(rng)
+
+
 def test_qjl_matrix_is_gaussian():
     P.pin_qjl_gaussian(rng)
 
