@@ -30,8 +30,7 @@ def sources():
 def _stale():
     if not os.path.exists(LIB):
         return True
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
-        glob.glob(os.path.join(INCLUDE, "*.h"))
+    deps = sources() + _headers()
     built = os.path.getmtime(LIB)
     return any(os.path.getmtime(p) > built for p in deps)
 
@@ -41,22 +40,31 @@ def nvcc():
     return cand if os.path.exists(cand) else "nvcc"
 
 
+def _headers():
+    return glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
+        glob.glob(os.path.join(INCLUDE, "*.h"))
+
+
 def build(force=False, verbose=False):
-    """Compile every CUDA/C++ source into libtq.so; return its path."""
+    """Compile every CUDA/C++ source into libtq.so; return its path.  An object
+    is recompiled when its source or any header is newer than it."""
     if not force and not _stale():
         return LIB
     objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
+    newest_header = max([os.path.getmtime(h) for h in _headers()] + [0.0])
     objs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        objs.append(obj)
+        if not force and os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(src), newest_header):
+            continue
         cmd = [nvcc(), "-c", src, "-o", obj, "-I", INCLUDE, "-I", CSRC] + NVCC_FLAGS
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError("nvcc failed for %s:\n%s\n%s" % (src, res.stdout, res.stderr))
         if verbose:
             sys.stderr.write(res.stderr)
-        objs.append(obj)
     tmp = LIB + ".tmp"
     cmd = [nvcc(), "-shared", "-o", tmp] + objs + ["-gencode", "arch=compute_100a,code=sm_100a", "-lcudart_static",
                                                    "-ldl", "-lrt", "-lpthread"]

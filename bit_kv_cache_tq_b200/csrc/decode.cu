@@ -24,7 +24,6 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
-#include <mutex>
 
 #include "device_common.cuh"
 #include "internal.h"
@@ -440,36 +439,28 @@ extern "C" tq_status tq_append_decode_attention(const tq_params* params, const t
 // serving starts, or code that runs while another component holds the
 // allocator.  For them the split partials and counters live in one fixed
 // device array of this library, so a call allocates nothing.  The array is
-// shared by every call on a device: it keeps the last call's partials (only
-// its counter words must be zero when a call starts, and every completed call
-// leaves them so), and calls that overlap on the device race on it.
+// shared by every call on a device and keeps the last call's partials; calls
+// that overlap on the device race on it.
 
 namespace tq {
 namespace {
 
 __device__ __align__(256) unsigned char g_static_scratch[TQ_DECODE_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_static_scratch_mutex;
-void* g_static_scratch_ptr[kMaxDevices] = {};
-
-// Address of this device's scratch.  The first call on a device looks the
-// symbol up and zero-fills the array on `stream`, ahead of the call's kernels.
-cudaError_t static_scratch(void** out, cudaStream_t stream) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+// Address of the current device's scratch array, looked up on every call (a
+// host query that allocates nothing; nothing cached survives a device reset),
+// and a zero fill of the counter words a call over `units` (sequence, kv
+// head) pairs uses, queued on `stream` ahead of the call's kernels.  Every
+// call therefore starts from zeroed counters, whatever the previous call on
+// the array left behind (one that ended with TQ_DEVERR_TIMEOUT included).
+cudaError_t static_scratch(void** out, long long units, cudaStream_t stream) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
-    if (!g_static_scratch_ptr[dev]) {
-        void* ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_static_scratch);
-        if (e != cudaSuccess) return e;
-        e = cudaMemsetAsync(ptr, 0, TQ_DECODE_STATIC_SCRATCH_BYTES, stream);
-        if (e != cudaSuccess) return e;
-        g_static_scratch_ptr[dev] = ptr;
-    }
-    *out = g_static_scratch_ptr[dev];
+    const size_t counter_bytes = static_cast<size_t>(units + kGlobalCounters) * sizeof(uint32_t);
+    e = cudaMemsetAsync(ptr, 0, counter_bytes, stream);
+    if (e != cudaSuccess) return e;
+    *out = ptr;
     return cudaSuccess;
 }
 
@@ -492,7 +483,8 @@ extern "C" tq_status tq_decode_attention_static(const tq_params* params, const t
         TQ_DECODE_STATIC_SCRATCH_BYTES)
         return TQ_ERR_CAPACITY;
     void* scratch = nullptr;
-    if (static_scratch(&scratch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return TQ_ERR_CUDA;
+    const long long units = static_cast<long long>(cache->batch) * params->num_kv_heads;
+    if (static_scratch(&scratch, units, static_cast<cudaStream_t>(stream)) != cudaSuccess) return TQ_ERR_CUDA;
     return tq_decode_attention(params, kcb, vcb, d_q, q_dtype, cache, d_seq_lens, max_seq_len, d_out, scratch,
                                TQ_DECODE_STATIC_SCRATCH_BYTES, d_error, stream);
 }

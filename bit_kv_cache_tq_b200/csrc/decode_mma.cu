@@ -86,6 +86,13 @@ constexpr uint32_t QHDR = 32;                 // item header at the front of a q
 // combine buffer stays at 22.5 KB for any GQA group (8 or 16 heads would
 // otherwise crowd out the second stage).
 constexpr int MERGE_HEADS = 4;
+// A warp's partial of one head in the combine buffer: eight 16-channel blocks
+// of 20 floats (4 of padding), so the eight lane groups g writing channels
+// 16 g + 2 i at once hit eight distinct banks (a 128-float row would put every
+// other g on the same bank); blocks stay 16-byte aligned for float4 reads.
+constexpr int MBLK = 20;
+constexpr int MSTRIDE = 8 * MBLK;
+__device__ __forceinline__ int mslot(int c) { return (c >> 4) * MBLK + (c & 15); }
 // Row strides (halves) of the fp16 query and sketch buffers: 2 words past a
 // multiple of 32 banks, so the 8-byte fragment loads of a half-warp (lane
 // groups g = 0..3 at rows g, columns 16 t) hit 32 distinct banks.
@@ -107,9 +114,10 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LAZY = 8.0f;                 // log2 headroom before the running max moves
 constexpr float VRANGE = 64.0f;              // bound on ||v|| * vscale
 
-// item header flags (query slot): EMPTY / END / APPEND / DRAIN (one stage to
-// consume unread) / SKIP (no work: only the drain)
-constexpr int F_EMPTY = 4, F_END = 8, F_APPEND = 16, F_DRAIN = 32, F_SKIP = 64;
+// item header flags (query slot): EMPTY / END / APPEND / SKIP (no work: only the
+// drain); bits DRAIN_SHIFT and up count the stages the consumers release unread
+// after the item's chunks (speculative stages past the sequence's end)
+constexpr int F_EMPTY = 4, F_END = 8, F_APPEND = 16, F_SKIP = 64, DRAIN_SHIFT = 8;
 // global counters after the per-(sequence, kv head) split counters
 constexpr int C_ITEM = 0, C_DONE = 1;
 
@@ -185,10 +193,10 @@ __host__ __device__ inline Layout layout(int kb, int vb, int nt, int stages, int
     L.fac = L.app + APP_BYTES;                         // float F1[16], F2[16]
     L.merge = L.fac + 32 * 4;
     // merge area, reused: per-warp partials of up to MERGE_HEADS heads at a
-    // time [CW][MERGE_HEADS][128]; the final merge's [g][128] outputs and
+    // time [CW][MERGE_HEADS][MSTRIDE]; the final merge's [g][128] outputs and
     // [CW][n_split] weights; the prologue's [8 nt][128] sketch staging; the
     // table build's 768 compact words
-    uint32_t merge = CW * (g < MERGE_HEADS ? g : MERGE_HEADS) * D * 4;
+    uint32_t merge = CW * (g < MERGE_HEADS ? g : MERGE_HEADS) * MSTRIDE * 4;
     const uint32_t fin = (g * D + CW * n_split) * 4;
     if (fin > merge) merge = fin;
     if (8u * nt * D * 4 > merge) merge = 8 * nt * D * 4;
@@ -264,8 +272,9 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         }
         // Every block asks for its first stage at the same moment; the other
         // stages follow once it has landed, so first bytes do not queue behind
-        // the whole grid's prefetch.
-        if (seq == 1 && !ptx::mbar_wait_bounded(full0, 0, WAIT_LIMIT)) {
+        // the whole grid's prefetch.  (With the early prefetch the blocks start
+        // at staggered times, while the previous kernel drains: no such wait.)
+        if (seq == 1 && !a.early && !ptx::mbar_wait_bounded(full0, 0, WAIT_LIMIT)) {
             fail();
             return false;
         }
@@ -382,14 +391,26 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
     // patched in from its staged rows), so it streams in while the previous
     // layer's blocks drain.  Queries, lengths and everything else wait.
     int i = blockIdx.x;
-    bool first = true, spec = false, q0_issued = false;
+    bool first = true, q0_issued = false;
+    int nspec = 0;  // stages of the first item requested before its length was known
     const bool have_first = i < a.n_items;
     const int unit0 = i / a.n_split, split0 = i % a.n_split;
     const int s00 = split0 * a.split_len;
-    // a split may start past the cache's end when max_seq_len exceeds the
-    // capacity: nothing to fetch speculatively there
-    const bool spec_ok = have_first && s00 < a.capacity;
-    if (spec_ok && a.early && !*abort_flag) spec = issue_chunk(unit0, s00, min(CHUNK, a.capacity - s00), false);
+    // the first item's tokens as far as the cache reaches (a split may start
+    // past the cache's end when max_seq_len exceeds the capacity: nothing to
+    // fetch speculatively there)
+    const int spec_end = min(a.capacity, s00 + a.split_len);
+    // The length is read first thing after the wait; bring its line into L2
+    // now (L2 is coherent with any write of the previous kernel), so that read
+    // does not queue behind the grid's first copies in DRAM.
+    if (have_first) ptx::prefetch_l2(a.seq_lens + unit0 / a.hkv);
+    // With the early prefetch, as many of the first item's chunks as the
+    // stages hold stream in before the previous kernel ends.
+    if (have_first && a.early)
+        for (int t = s00; t < spec_end && nspec < a.stages && !*abort_flag; t += CHUNK) {
+            if (!issue_chunk(unit0, t, min(CHUNK, spec_end - t), false)) break;
+            ++nspec;
+        }
     ptx::wait_prerequisites();
     if (have_first && !*abort_flag) {
         const int b = unit0 / a.hkv, kv = unit0 % a.hkv;
@@ -399,7 +420,7 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
                            static_cast<const uint8_t*>(a.q) + (static_cast<size_t>(b) * a.hq + kv * G) * D * a.q_bytes,
                            qbytes, q0);
         q0_issued = true;
-        if (!a.early && spec_ok) spec = issue_chunk(unit0, s00, min(CHUNK, a.capacity - s00), false);
+        if (!a.early && s00 < spec_end && issue_chunk(unit0, s00, min(CHUNK, spec_end - s00), false)) nspec = 1;
     }
     while (ok) {
         if (i >= a.n_items) break;
@@ -416,11 +437,11 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         }
         const bool empty = w.s0 >= w.s1;
         const bool app = a.append && !empty && w.s1 == w.len;
-        if (first && spec && a.table && !empty) {
-            // the speculative chunk was fetched before the length was known:
-            // report an unmapped block among its valid tokens now
+        if (first && nspec > 0 && a.table && !empty) {
+            // the speculative chunks were fetched before the length was known:
+            // report an unmapped block among their valid tokens now
             const int32_t* trow = a.table + static_cast<size_t>(w.b) * a.max_blocks;
-            const int e = min(w.s1, w.s0 + CHUNK);
+            const int e = min(w.s1, w.s0 + nspec * CHUNK);
             for (int t = w.s0; t < e; t += a.block_size - t % a.block_size) {
                 const int blk = __ldg(trow + t / a.block_size);
                 if (blk < 0 || blk >= a.num_blocks) {
@@ -432,10 +453,13 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         uint8_t* qslot;
         uint32_t qfull;
         if (!claim_q(qslot, qfull)) break;
+        // chunks the consumers take for this item; speculative stages past
+        // them are released unread
+        const int nchunks = empty ? 0 : (w.s1 - w.s0 + CHUNK - 1) / CHUNK;
+        const int ndrain = first && nspec > nchunks ? nspec - nchunks : 0;
         int4* hdr = reinterpret_cast<int4*>(qslot);
         hdr[0] = make_int4(i, w.s0, w.s1, w.len);
-        hdr[1] = make_int4((empty ? F_EMPTY : 0) | (app ? F_APPEND : 0) | (first && spec && empty ? F_DRAIN : 0) |
-                               (dead ? F_SKIP : 0),
+        hdr[1] = make_int4((empty ? F_EMPTY : 0) | (app ? F_APPEND : 0) | (dead ? F_SKIP : 0) | (ndrain << DRAIN_SHIFT),
                            w.unit, w.b, w.kv);
         const uint32_t rbytes = D * a.new_bytes;
         const uint32_t extra = app ? 2 * rbytes : 0u;  // append rows
@@ -456,7 +480,7 @@ __device__ void producer(const Args& a, uint8_t* smem, const Layout& L) {
         }
         ptx::mbar_arrive(qfull);  // header written, every copy of the slot accounted for
         int t0 = w.s0;
-        if (first && spec) t0 += CHUNK;  // the speculative stage holds the first chunk
+        if (first) t0 += nspec * CHUNK;  // the speculative stages hold the first chunks
         for (; t0 < w.s1; t0 += CHUNK)
             if (!issue_chunk(w.unit, t0, min(CHUNK, w.s1 - t0), true)) break;
         first = false;
@@ -938,9 +962,288 @@ struct Consumer {
         }
     }
 
-    // One chunk: this warp's two tiles.  MASK: the chunk may end before CHUNK tokens.
+    // One chunk: this warp's TPW tiles.  MASK: the chunk may end before CHUNK
+    // tokens.  Each phase handles all of the warp's tiles in one branch-free
+    // stretch (the tiles are independent, so their load, lookup and MMA chains
+    // interleave); tokens past the item's end are computed on whatever the
+    // stage holds (finite table values) and masked afterwards.
     template <bool MASK>
-    __device__ void chunk(const Item& w, const uint8_t* st, int t0, const uint32_t (&bq)[NT][8][4],
+    __device__ void chunk_il(const Item& w, const uint8_t* st, int t0, const uint32_t (&bq)[NT][8][4],
+                          const uint32_t (&bz)[NT][4][2], const float (&f1)[NT][2], const float (&f2)[NT][2],
+                          SoftState<NT>& S) {
+        constexpr int VBK = 16 * KB, VBV = 16 * VB;
+        // this warp's tiles are k * CW + warp (k < TPW): a short last chunk
+        // spreads over many warps instead of keeping two tiles on a few
+        const int lb = 16 * warp;  // first chunk-local token of this warp's first tile
+        constexpr int TS = 16 * CW;  // token distance between a warp's tiles
+        if (MASK && t0 + lb >= w.s1) return;  // nothing of this warp's tiles is valid
+        const uint32_t sbase = ptx::smem_addr(st);
+        const int ra = tau_row(g), rb = tau_row(g + 8);
+        const int zw = a.m / 16;
+        const bool zt = 16 * t < a.m;
+        const size_t unit_row = static_cast<size_t>(w.unit) * a.capacity;
+        // chunk-local tokens of rows g, g + 8 of each tile, and their validity
+        int la[TPW], lbb[TPW];
+        bool va[TPW], vb[TPW];
+#pragma unroll
+        for (int k = 0; k < TPW; ++k) {
+            la[k] = lb + TS * k + ra;
+            lbb[k] = lb + TS * k + rb;
+            va[k] = !MASK || t0 + la[k] < w.s1;
+            vb[k] = !MASK || t0 + lbb[k] < w.s1;
+        }
+        // ---- norms (and QJL words and gammas) of every tile
+        float kna[TPW], knb[TPW], vn[TPW][2], ga[TPW], gb[TPW];
+        uint32_t za[TPW], zb2[TPW];
+        if (a.staged_norms) {
+            const __half* skn = reinterpret_cast<const __half*>(st + L.kn_off);
+            const __half* svn = reinterpret_cast<const __half*>(st + L.vn_off);
+#pragma unroll
+            for (int k = 0; k < TPW; ++k) {
+                kna[k] = __half2float(skn[la[k]]);
+                knb[k] = __half2float(skn[lbb[k]]);
+                vn[k][0] = va[k] ? __half2float(svn[la[k]]) : 0.f;
+                vn[k][1] = vb[k] ? __half2float(svn[lbb[k]]) : 0.f;
+                ga[k] = gb[k] = 0.f;
+                za[k] = zb2[k] = 0u;
+                if constexpr (QJL) {
+                    const uint16_t* sz = reinterpret_cast<const uint16_t*>(st + L.z_off);
+                    const __half* sg = reinterpret_cast<const __half*>(st + L.gam_off);
+                    za[k] = zt ? sz[la[k] * zw + t] : 0u;
+                    zb2[k] = zt ? sz[lbb[k] * zw + t] : 0u;
+                    ga[k] = __half2float(sg[la[k]]);
+                    gb[k] = __half2float(sg[lbb[k]]);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < TPW; ++k) {
+                const size_t ra_g = unit_row + t0 + la[k], rb_g = unit_row + t0 + lbb[k];
+                kna[k] = va[k] ? half_bits_to_float(a.k_norms[ra_g]) : 0.f;
+                knb[k] = vb[k] ? half_bits_to_float(a.k_norms[rb_g]) : 0.f;
+                vn[k][0] = va[k] ? half_bits_to_float(a.v_norms[ra_g]) : 0.f;
+                vn[k][1] = vb[k] ? half_bits_to_float(a.v_norms[rb_g]) : 0.f;
+                ga[k] = gb[k] = 0.f;
+                za[k] = zb2[k] = 0u;
+                if constexpr (QJL) {
+                    const uint16_t* zr = reinterpret_cast<const uint16_t*>(a.k_qjl);
+                    za[k] = (va[k] && zt) ? zr[ra_g * zw + t] : 0u;
+                    zb2[k] = (vb[k] && zt) ? zr[rb_g * zw + t] : 0u;
+                    ga[k] = va[k] ? half_bits_to_float(a.k_gamma[ra_g]) : 0.f;
+                    gb[k] = vb[k] ? half_bits_to_float(a.k_gamma[rb_g]) : 0.f;
+                }
+            }
+        }
+        // ---- keys: the lane's 4*KB bytes of rows tau(g) and tau(g+8) of every tile
+        uint32_t sa[TPW][4], sb[TPW][4];
+        uint32_t ka[TPW][8], kb8[TPW][8];  // int8 keys: channels 32 t .. 32 t + 31 of rows tau(g), tau(g + 8)
+#pragma unroll
+        for (int k = 0; k < TPW; ++k) {
+            const uint32_t kst = sbase + L.k_off + (lb + TS * k) * VBK;
+            if constexpr (KB == INT8_BITS) {
+                // 128-byte rows all start at bank 0: lanes of odd g read their
+                // second 16 bytes first, so a quarter-warp (g = 2q, 2q + 1) hits
+                // 32 distinct banks
+                const uint32_t sw = (g & 1) * 16;
+                const uint4 x0 = ptx::lds128(kst + ra * VBK + 32 * t + sw);
+                const uint4 x1 = ptx::lds128(kst + ra * VBK + 32 * t + (sw ^ 16));
+                const uint4 y0 = ptx::lds128(kst + rb * VBK + 32 * t + sw);
+                const uint4 y1 = ptx::lds128(kst + rb * VBK + 32 * t + (sw ^ 16));
+                const bool odd = g & 1;
+                ka[k][0] = odd ? x1.x : x0.x; ka[k][1] = odd ? x1.y : x0.y; ka[k][2] = odd ? x1.z : x0.z; ka[k][3] = odd ? x1.w : x0.w;
+                ka[k][4] = odd ? x0.x : x1.x; ka[k][5] = odd ? x0.y : x1.y; ka[k][6] = odd ? x0.z : x1.z; ka[k][7] = odd ? x0.w : x1.w;
+                kb8[k][0] = odd ? y1.x : y0.x; kb8[k][1] = odd ? y1.y : y0.y; kb8[k][2] = odd ? y1.z : y0.z; kb8[k][3] = odd ? y1.w : y0.w;
+                kb8[k][4] = odd ? y0.x : y1.x; kb8[k][5] = odd ? y0.y : y1.y; kb8[k][6] = odd ? y0.z : y1.z; kb8[k][7] = odd ? y0.w : y1.w;
+            } else if constexpr (KB == 4) {
+                const uint4 x = ptx::lds128(kst + ra * VBK + 16 * t);
+                const uint4 y = ptx::lds128(kst + rb * VBK + 16 * t);
+                sa[k][0] = x.x; sa[k][1] = x.y; sa[k][2] = x.z; sa[k][3] = x.w;
+                sb[k][0] = y.x; sb[k][1] = y.y; sb[k][2] = y.z; sb[k][3] = y.w;
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) sa[k][q] = sb[k][q] = 0u;
+#pragma unroll
+                for (int q = 0; q < KB; ++q) {
+                    sa[k][q] = ptx::lds32(kst + ra * VBK + 4 * KB * t + 4 * q);
+                    sb[k][q] = ptx::lds32(kst + rb * VBK + 4 * KB * t + 4 * q);
+                }
+            }
+        }
+        // ---- scores: hi and lo query parts accumulate in separate chains
+        float cs[TPW][NT][4], cl[TPW][NT][4], cz[TPW][NT][4];
+#pragma unroll
+        for (int k = 0; k < TPW; ++k)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) cs[k][nt][e] = cl[k][nt][e] = cz[k][nt][e] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int k = 0; k < TPW; ++k) {
+                uint32_t a0, a1, a2, a3;
+                if constexpr (KB == INT8_BITS) {
+                    int8_pairs(ka[k][j], a0, a2);
+                    int8_pairs(kb8[k][j], a1, a3);
+                } else {
+                    a0 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sa[k], j, 0, laneoff));
+                    a1 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sb[k], j, 0, laneoff));
+                    a2 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sa[k], j, 1, laneoff));
+                    a3 = ptx::lds32_imm<WINDOW>(key_lut_addr<KB>(sb[k], j, 1, laneoff));
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    ptx::mma_16816(cs[k][nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
+                    ptx::mma_16816(cl[k][nt], a0, a1, a2, a3, bq[nt][j][2], bq[nt][j][3]);
+                }
+            }
+        if constexpr (QJL) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int k = 0; k < TPW; ++k) {
+                    // +-1 pairs from sign bits (bit set -> +1)
+                    const uint32_t xa = za[k] >> (4 * j), xb = zb2[k] >> (4 * j);
+                    const uint32_t a0 = 0xBC00BC00u ^ ((xa & 1u) << 15) ^ ((xa & 2u) << 30);
+                    const uint32_t a2 = 0xBC00BC00u ^ ((xa & 4u) << 13) ^ ((xa & 8u) << 28);
+                    const uint32_t a1 = 0xBC00BC00u ^ ((xb & 1u) << 15) ^ ((xb & 2u) << 30);
+                    const uint32_t a3 = 0xBC00BC00u ^ ((xb & 4u) << 13) ^ ((xb & 8u) << 28);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) ptx::mma_16816(cz[k][nt], a0, a1, a2, a3, bz[nt][j][0], bz[nt][j][1]);
+                }
+        }
+        float s[TPW][NT][4];
+#pragma unroll
+        for (int k = 0; k < TPW; ++k)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float v = (cs[k][nt][e] + cl[k][nt][e]) * f1[nt][e & 1];
+                    if constexpr (QJL) v = fmaf((e < 2 ? ga[k] : gb[k]) * cz[k][nt][e], f2[nt][e & 1], v);
+                    v *= e < 2 ? kna[k] : knb[k];
+                    if (MASK) v = (e < 2 ? va[k] : vb[k]) ? v : -INFINITY;
+                    s[k][nt][e] = v;
+                }
+
+        // ---- softmax: the reference max moves only when a score exceeds it by 2^LAZY
+        bool need = false;
+        float lm[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            lm[nt][0] = lm[nt][1] = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < TPW; ++k) {
+                lm[nt][0] = fmaxf(lm[nt][0], fmaxf(s[k][nt][0], s[k][nt][2]));
+                lm[nt][1] = fmaxf(lm[nt][1], fmaxf(s[k][nt][1], s[k][nt][3]));
+            }
+            need |= lm[nt][0] > S.m[nt][0] + LAZY || lm[nt][1] > S.m[nt][1] + LAZY;
+        }
+        float vmax = 0.f;
+#pragma unroll
+        for (int k = 0; k < TPW; ++k) vmax = fmaxf(vmax, fmaxf(vn[k][0], vn[k][1]));
+        need |= (S.vscale == 0.f && vmax > 0.f) || vmax * S.vscale > VRANGE;
+        if (__any_sync(kFullMask, need)) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) {
+                    lm[nt][0] = fmaxf(lm[nt][0], __shfl_xor_sync(kFullMask, lm[nt][0], o));
+                    lm[nt][1] = fmaxf(lm[nt][1], __shfl_xor_sync(kFullMask, lm[nt][1], o));
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float mn = fmaxf(S.m[nt][h], lm[nt][h]);
+                    if (mn > S.m[nt][h]) {
+                        const float c = ptx::ex2(S.m[nt][h] - mn);
+                        S.l[nt][h] *= c;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            S.acc[nt][i][h] *= c;
+                            S.acc[nt][i][h + 2] *= c;
+                        }
+                        S.m[nt][h] = mn;
+                    }
+                }
+            }
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFullMask, vmax, o));
+            if (vmax > 0.f && (S.vscale == 0.f || vmax * S.vscale > VRANGE)) {
+                const float target = exp2f(-ceilf(log2f(vmax)));  // vmax * target in (0.5, 1]
+                if (S.vscale > 0.f) {
+                    const float f = target / S.vscale;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) S.acc[nt][i][e] *= f;
+                }
+                S.vscale = target;
+            }
+        }
+
+        // ---- weights of every tile (Sparse V drops provably small ones)
+        float pv[TPW][NT][4];
+        bool any_v = false;
+#pragma unroll
+        for (int k = 0; k < TPW; ++k)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) pv[k][nt][e] = ptx::ex2(s[k][nt][e] - S.m[nt][e & 1]);
+                S.l[nt][0] += pv[k][nt][0] + pv[k][nt][2];
+                S.l[nt][1] += pv[k][nt][1] + pv[k][nt][3];
+            }
+        if (a.tau > 0.f) {
+            // Sparse V: the exact denominator relative to the reference is at
+            // least 1 (the reference is a seen score) and at least this lane's
+            // partial sum, so p / max(1, l) bounds the exact weight
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float th0 = a.tau * fmaxf(1.f, S.l[nt][0]), th1 = a.tau * fmaxf(1.f, S.l[nt][1]);
+#pragma unroll
+                for (int k = 0; k < TPW; ++k) {
+                    if (pv[k][nt][0] < th0) pv[k][nt][0] = 0.f;
+                    if (pv[k][nt][2] < th0) pv[k][nt][2] = 0.f;
+                    if (pv[k][nt][1] < th1) pv[k][nt][1] = 0.f;
+                    if (pv[k][nt][3] < th1) pv[k][nt][3] = 0.f;
+                    any_v |= (pv[k][nt][0] + pv[k][nt][1] + pv[k][nt][2] + pv[k][nt][3]) > 0.f;
+                }
+            }
+            // no weight of this warp's tiles left: their value products add nothing
+            if (!__any_sync(kFullMask, any_v)) return;
+        }
+        // ---- values: both tiles' products in one stretch (a tile past the
+        // item's end has zero weights and adds nothing)
+        uint32_t bv[TPW][NT][2];
+#pragma unroll
+        for (int k = 0; k < TPW; ++k) {
+            const float wa = vn[k][0] * S.vscale, wb = vn[k][1] * S.vscale;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                bv[k][nt][0] = ptx::movmatrix_trans(ptx::pack_half2(pv[k][nt][0] * wa, pv[k][nt][1] * wa));
+                bv[k][nt][1] = ptx::movmatrix_trans(ptx::pack_half2(pv[k][nt][2] * wb, pv[k][nt][3] * wb));
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < TPW; ++k) {
+            uint32_t A[8][4];
+            value_fragments<VB>(sbase + L.v_off + (lb + TS * k) * VBV, base, g, t, laneoff, A);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    ptx::mma_16816(S.acc[nt][i], A[i][0], A[i][1], A[i][2], A[i][3], bv[k][nt][0], bv[k][nt][1]);
+        }
+    }
+
+    // One chunk, tile after tile: the form for the register-heavy
+    // configurations (16-head groups, the QJL sketch), where holding both
+    // tiles' scores at once would spill.  MASK: the chunk may end before CHUNK
+    // tokens.
+    template <bool MASK>
+    __device__ void chunk_seq(const Item& w, const uint8_t* st, int t0, const uint32_t (&bq)[NT][8][4],
                           const uint32_t (&bz)[NT][4][2], const float (&f1)[NT][2], const float (&f2)[NT][2],
                           SoftState<NT>& S) {
         constexpr int VBK = 16 * KB, VBV = 16 * VB;
@@ -1177,6 +1480,14 @@ struct Consumer {
         }
     }
 
+    template <bool MASK>
+    __device__ void chunk(const Item& w, const uint8_t* st, int t0, const uint32_t (&bq)[NT][8][4],
+                          const uint32_t (&bz)[NT][4][2], const float (&f1)[NT][2], const float (&f2)[NT][2],
+                          SoftState<NT>& S) {
+        if constexpr (NT == 1 && !QJL) chunk_il<MASK>(w, st, t0, bq, bz, f1, f2, S);
+        else chunk_seq<MASK>(w, st, t0, bq, bz, f1, f2, S);
+    }
+
     __device__ float group_sum_g(float x) const {  // sum over the 8 lanes sharing t
         x += __shfl_xor_sync(kFullMask, x, 4);
         x += __shfl_xor_sync(kFullMask, x, 8);
@@ -1209,15 +1520,15 @@ struct Consumer {
                 for (int i = 0; i < 8; ++i) {
                     const int h0 = nt * 8 + 2 * t;  // heads h0, h0 + 1 of this lane's columns (same pass)
                     if (h0 < hb || h0 >= hb + GM) continue;
-                    float* mw = merge + (warp * GM + h0 - hb) * D;
-                    const int c_lo = 16 * g + 2 * i, c_hi = c_lo + 1;
+                    float* mw = merge + (warp * GM + h0 - hb) * MSTRIDE;
+                    const int c_lo = mslot(16 * g + 2 * i), c_hi = c_lo + 1;
                     if (h0 < G) {
                         mw[c_lo] = S.acc[nt][i][0] * unscale;
                         mw[c_hi] = S.acc[nt][i][2] * unscale;
                     }
                     if (h0 + 1 < G) {
-                        mw[D + c_lo] = S.acc[nt][i][1] * unscale;
-                        mw[D + c_hi] = S.acc[nt][i][3] * unscale;
+                        mw[MSTRIDE + c_lo] = S.acc[nt][i][1] * unscale;
+                        mw[MSTRIDE + c_hi] = S.acc[nt][i][3] * unscale;
                     }
                 }
             ptx::named_barrier(1, NUM_CONSUMERS);
@@ -1240,7 +1551,7 @@ struct Consumer {
                     const float2 mlw = ml[ww * 16 + h];
                     const float f = (mlw.y > 0.f && mx > -INFINITY) ? ptx::ex2(mlw.x - mx) : 0.f;
                     l = fmaf(mlw.y, f, l);
-                    const float4 v = m4[(ww * GM + hl) * (D / 4) + c4];
+                    const float4 v = m4[(ww * GM + hl) * (MSTRIDE / 4) + (c4 >> 2) * (MBLK / 4) + (c4 & 3)];
                     acc4.x = fmaf(v.x, f, acc4.x);
                     acc4.y = fmaf(v.y, f, acc4.y);
                     acc4.z = fmaf(v.z, f, acc4.z);
@@ -1260,54 +1571,72 @@ struct Consumer {
                                    static_cast<uint32_t>(nlive - 1);
         ptx::named_barrier(1, NUM_CONSUMERS);
         if (*last_flag) {
-            // Merge the splits: two warps per head, each lane two channels.  A
-            // warp's first batch of partial rows is requested before its split
-            // weights 2^(m_s - M) are formed (its own row of shared memory), so
-            // both reads overlap; the weighted sum runs in split order, so the
-            // result does not depend on timing.
+            // Merge the splits: two warps per head, each lane two channels.
+            // With at most 32 live splits (the usual case) every load, the
+            // partial rows and one (m, l) pair per lane, is issued before any
+            // is used, so the merge costs one round trip to L2; the weights
+            // 2^(m_s - M) are formed per lane and broadcast by shuffles.  Longer
+            // lists take batches.  Either way the weighted sum runs in split
+            // order, so the result does not depend on timing.
             float* o_s = merge;  // [G][D]
             const size_t ubase = static_cast<size_t>(w.unit) * a.n_split * G;
             const float2* src2 = reinterpret_cast<const float2*>(a.ws_acc + ubase * D);
-            float* wts = merge + G * D + warp * a.n_split;
-            constexpr int PB = 24;  // splits per batch of loads
+            // splits per batch of loads (at most one per lane for the weights); the
+            // register-heavy configurations take smaller batches
+            constexpr int PB = (NT == 1 && !QJL) ? 32 : 8;
             for (int u = warp; u < 2 * G; u += CW) {
                 const int h = u >> 1, c2 = (u & 1) * 32 + lane;  // float2 column
-                float2 v[PB];
-#pragma unroll
-                for (int j = 0; j < PB; ++j)
-                    v[j] = j < nlive ? __ldcg(src2 + (j * G + h) * (D / 2) + c2) : make_float2(0.f, 0.f);
-                float mx = -INFINITY;
-                for (int sp = lane; sp < nlive; sp += 32) {
-                    const float2 m2 = __ldcg(a.ws_ml + ubase + sp * G + h);
-                    if (m2.y > 0.f) mx = fmaxf(mx, m2.x);
-                }
-                mx = group_max<32>(mx);
-                float l = 0.f;
-                for (int sp = lane; sp < nlive; sp += 32) {
-                    const float2 m2 = __ldcg(a.ws_ml + ubase + sp * G + h);
-                    const float wgt = (m2.y > 0.f && mx > -INFINITY) ? ptx::ex2(m2.x - mx) : 0.f;
-                    wts[sp] = wgt;
-                    l = fmaf(m2.y, wgt, l);
-                }
-                l = group_sum<32>(l);
-                const float inv_l = l > 0.f ? 1.f / l : 0.f;
-                __syncwarp();
                 float2 acc = make_float2(0.f, 0.f);
-                for (int s0 = 0; s0 < nlive; s0 += PB) {
-                    if (s0 > 0) {
+                float l = 0.f;
+                if (nlive <= PB) {
+                    float2 v[PB];
+#pragma unroll
+                    for (int j = 0; j < PB; ++j)
+                        v[j] = j < nlive ? __ldcg(src2 + (j * G + h) * (D / 2) + c2) : make_float2(0.f, 0.f);
+                    const float2 m2 = lane < nlive ? __ldcg(a.ws_ml + ubase + lane * G + h) : make_float2(-INFINITY, 0.f);
+                    const float mx = group_max<32>(m2.y > 0.f ? m2.x : -INFINITY);
+                    const float wgt = (m2.y > 0.f && mx > -INFINITY) ? ptx::ex2(m2.x - mx) : 0.f;
+                    l = group_sum<32>(m2.y * wgt);
+#pragma unroll
+                    for (int j = 0; j < PB; ++j) {
+                        const float wj = __shfl_sync(kFullMask, wgt, j);
+                        if (j < nlive) {
+                            acc.x = fmaf(v[j].x, wj, acc.x);
+                            acc.y = fmaf(v[j].y, wj, acc.y);
+                        }
+                    }
+                } else {
+                    float* wts = merge + G * D + warp * a.n_split;
+                    float mx = -INFINITY;
+                    for (int sp = lane; sp < nlive; sp += 32) {
+                        const float2 m2 = __ldcg(a.ws_ml + ubase + sp * G + h);
+                        if (m2.y > 0.f) mx = fmaxf(mx, m2.x);
+                    }
+                    mx = group_max<32>(mx);
+                    for (int sp = lane; sp < nlive; sp += 32) {
+                        const float2 m2 = __ldcg(a.ws_ml + ubase + sp * G + h);
+                        const float wgt = (m2.y > 0.f && mx > -INFINITY) ? ptx::ex2(m2.x - mx) : 0.f;
+                        wts[sp] = wgt;
+                        l = fmaf(m2.y, wgt, l);
+                    }
+                    l = group_sum<32>(l);
+                    __syncwarp();
+                    for (int s0 = 0; s0 < nlive; s0 += PB) {
+                        float2 v[PB];
 #pragma unroll
                         for (int j = 0; j < PB; ++j)
                             v[j] = s0 + j < nlive ? __ldcg(src2 + ((s0 + j) * G + h) * (D / 2) + c2)
-                                                      : make_float2(0.f, 0.f);
-                    }
+                                                  : make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int j = 0; j < PB; ++j) {
-                        const float wgt = s0 + j < nlive ? wts[s0 + j] : 0.f;
-                        acc.x = fmaf(v[j].x, wgt, acc.x);
-                        acc.y = fmaf(v[j].y, wgt, acc.y);
+                        for (int j = 0; j < PB; ++j) {
+                            const float wgt = s0 + j < nlive ? wts[s0 + j] : 0.f;
+                            acc.x = fmaf(v[j].x, wgt, acc.x);
+                            acc.y = fmaf(v[j].y, wgt, acc.y);
+                        }
                     }
+                    __syncwarp();  // the weights row is rewritten by this warp's next unit
                 }
-                __syncwarp();  // the weights row is rewritten by this warp's next unit
+                const float inv_l = l > 0.f ? 1.f / l : 0.f;
                 *reinterpret_cast<float2*>(o_s + h * D + 2 * c2) = make_float2(acc.x * inv_l, acc.y * inv_l);
             }
             ptx::named_barrier(1, NUM_CONSUMERS);
@@ -1373,13 +1702,6 @@ struct Consumer {
             w.bad = false;
             const bool empty = h1.x & F_EMPTY, app = h1.x & F_APPEND;
             S.reset();
-            if (h1.x & F_DRAIN) {  // a stage filled before the item was known to be empty
-                const int slot = seq % a.stages, use = seq / a.stages;
-                if (!aborted() && !ptx::mbar_wait_bounded(full0 + 8 * slot, use & 1, WAIT_LIMIT)) set_abort();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(empty0 + 8 * slot);
-                ++seq;
-            }
             if (!empty) prologue(qseq, qseq == 0 && first_rotated, w, app, bq, bz, f1, f2);  // ends the slot's use
             else ptx::named_barrier(1, NUM_CONSUMERS);           // every warp has read the header
             if (tid == 0) ptx::mbar_arrive(qempty0 + 8 * (qseq & 1));  // query slot free
@@ -1402,6 +1724,15 @@ struct Consumer {
                     if (last) chunk<true>(w, st, t0, bq, bz, f1, f2, S);
                     else chunk<false>(w, st, t0, bq, bz, f1, f2, S);
                 }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(empty0 + 8 * slot);
+                ++seq;
+            }
+            // stages requested before the item's length was known and not
+            // needed after all: wait for their copies, release them unread
+            for (int dr = h1.x >> DRAIN_SHIFT; dr > 0; --dr) {
+                const int slot = seq % a.stages, use = seq / a.stages;
+                if (!aborted() && !ptx::mbar_wait_bounded(full0 + 8 * slot, use & 1, WAIT_LIMIT)) set_abort();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(empty0 + 8 * slot);
                 ++seq;

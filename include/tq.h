@@ -388,14 +388,15 @@ tq_status tq_append_decode_attention_paged(const tq_params* params, const tq_cod
  *     more scratch than the array holds (the launch plan for batch and
  *     max_seq_len on the current device decides; a workspace bound from
  *     tq_decode_workspace_bytes at or below the limit always fits).
- *   - The first call on a device looks up the array's address and queues a
- *     zero fill of it on `stream` ahead of its own kernels; make that first
- *     call before any stream capture.
+ *   - Every call looks up the array's address (a host query that allocates
+ *     nothing) and queues, on `stream` ahead of its kernels, a zero fill of
+ *     the counter words it uses ((batch * Hkv + 2) * 4 bytes at the front of
+ *     the array).  Only those words must be zero when a call starts, so a
+ *     call that ended with TQ_DEVERR_TIMEOUT leaves nothing behind that
+ *     harms the next one.
  *   - The array is shared by all calls on the device and keeps the last
- *     call's partials; only its counter words must be zero when a call
- *     starts, and every completed call leaves them zero.  Calls that overlap
- *     on the device (other streams, other threads) race on it: serialise
- *     them.
+ *     call's partials.  Calls that overlap on the device (other streams,
+ *     other threads) race on it: serialise them.
  */
 tq_status tq_decode_attention_static(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
                                      const void* d_q, tq_dtype q_dtype, const tq_cache* cache,

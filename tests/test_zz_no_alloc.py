@@ -14,18 +14,21 @@ from bit_kv_cache_tq_b200 import inputs, tq
 pytestmark = pytest.mark.gpu
 
 
-def _static(layer, q, cache, lens):
+def _static(layer, q, cache, lens, max_len=None, expect_word=0):
     lens_t = torch.as_tensor(np.asarray(lens), dtype=torch.int32).cuda()
     out = torch.empty(q.shape[0], layer.hq, layer.d, dtype=torch.float32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     tq.tq_decode_attention_static(layer.params, layer.kcb, layer.vcb, q.cuda().contiguous(), cache, lens_t,
-                                  int(max(lens)), out, err)
+                                  int(max_len or max(lens)), out, err)
     st, word = tq.tq_read_device_error(err)
-    assert st == tq.TQ_OK and word == 0
+    assert word == expect_word and st == (tq.TQ_OK if expect_word == 0 else tq.TQ_ERR_DEVICE), (st, word)
     return out.cpu().numpy()
 
 
 def test_static_scratch_matches_workspace_entry_point():
+    """Both entry points run the same deterministic launches, so the outputs
+    agree bit for bit: two calls in a row on one shape, then other batch
+    sizes and lengths."""
     layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=31)
     t = 3000
     k = inputs.lognormal_kv(3, t, 8, 128, seed=31, layer=31, which=inputs.K)
@@ -33,13 +36,31 @@ def test_static_scratch_matches_workspace_entry_point():
     q = inputs.queries(3, 32, 128, seed=31, layer=31)
     wide, _, _ = H.gpu_quantize(layer, k, v, t)
     narrow, _, _ = H.gpu_quantize(layer, k[:1], v[:1], t)
-    # two calls in a row on one shape, then other batch sizes and lengths
     for cache, qq, lens in [(wide, q, [t, 1999, 700]), (wide, q, [t, 1999, 700]), (narrow, q[:1], [t]),
                             (wide, q, [64, t, 1])]:
         want, st, word = H.gpu_decode(layer, qq, cache, lens)
         assert st == tq.TQ_OK and word == 0
         got = _static(layer, qq, cache, lens)
-        assert H.rel_l2_per_vector(got, want).max() <= H.ATTN_TOL, lens
+        assert np.array_equal(got, want), (lens, np.abs(got - want).max())
+
+
+def test_static_scratch_after_a_rejected_length():
+    """A call whose device-side length check fails (sequence 1 longer than
+    max_seq_len: TQ_DEVERR_SEQLEN, zeros for that sequence) leaves the shared
+    array fit for the next call, which again matches the workspace entry
+    point bit for bit."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=32)
+    t = 2500
+    k = inputs.lognormal_kv(2, t, 8, 128, seed=32, layer=32, which=inputs.K)
+    v = inputs.lognormal_kv(2, t, 8, 128, seed=32, layer=32, which=inputs.V)
+    q = inputs.queries(2, 32, 128, seed=32, layer=32)
+    cache, _, _ = H.gpu_quantize(layer, k, v, t)
+    bad = _static(layer, q, cache, [1000, t], max_len=2000, expect_word=tq.TQ_DEVERR_SEQLEN)
+    assert np.all(bad[1] == 0.0)
+    for lens in ([t, 1234], [t, 1234]):
+        want, st, word = H.gpu_decode(layer, q, cache, lens)
+        assert st == tq.TQ_OK and word == 0
+        assert np.array_equal(_static(layer, q, cache, lens), want), lens
 
 
 def test_static_scratch_rejects_calls_beyond_its_size():
