@@ -411,10 +411,14 @@ def decode_configs(dev, reps=10):
         assert st == tq.TQ_OK, (name, st, word)
         us = 1000.0 * e0.elapsed_time(e1) / reps
         extra = {}
-        if tau > 0:  # Sparse V's effect: the same call without skipping
+        if tau > 0:  # Sparse V's effect: the same call without skipping, and the positions it dropped
             dense = tq.make_params(D, hq, HKV, qjl_dims=m, seed=SEED, **modes)
             out_d = torch.empty_like(out)
-            tq.tq_decode_attention(p, kcb, vcb, q, caches[0], lens_t, tmax, out, ws, err)
+            mask = torch.zeros(bsz, hq, (tmax + 31) // 32, dtype=torch.int32, device=dev)
+            tq.tq_decode_attention(p, kcb, vcb, q, caches[0], lens_t, tmax, out, ws, err, skip_mask=mask)
+            words = mask.cpu().numpy().astype(np.uint32)
+            dropped = int(np.unpackbits(words.view(np.uint8)).sum())
+            extra["skip_fraction"] = dropped / float(hq * sum(lens))
             tq.tq_decode_attention(dense, kcb, vcb, q, caches[0], lens_t, tmax, out_d, ws, err)
             rel = ((out - out_d).norm(dim=-1) / out_d.norm(dim=-1)).max().item()
             d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -423,7 +427,8 @@ def decode_configs(dev, reps=10):
                 tq.tq_decode_attention(dense, kcb, vcb, q, caches[r % copies], lens_t, tmax, out_d, ws, err)
             d1.record()
             d1.synchronize()
-            extra = {"max_rel_l2_vs_no_skip": rel, "us_without_sparse_v": round(1000.0 * d0.elapsed_time(d1) / reps, 2)}
+            extra.update({"max_rel_l2_vs_no_skip": rel,
+                          "us_without_sparse_v": round(1000.0 * d0.elapsed_time(d1) / reps, 2)})
         per_tok = D * kb // 8 + 2 + (m // 8 + 2 if m else 0) + D * vb // 8 + 2
         nbytes = sum(lens) * HKV * per_tok
         res[name] = {"us_per_call": round(us, 2), "kv_tokens_per_s": round(sum(lens) / (us * 1e-6)),
@@ -638,7 +643,7 @@ def run_tq(args, world, rank, local):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
             "warmup": warmup, "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "vs_baseline": None, "dtype": "bf16-in/fp16-mma/fp32-acc", "data": "synthetic",
             "config": {"workload": WORKLOAD, "global_batch": BATCH * world, "seq_len": CONTEXT + 1,
                        "layers": LAYERS, "parallelism": "replicas%d" % world if world > 1 else "none",
                        "l2": "inputs larger than L2: 32 distinct layer caches, %.0f MB" %

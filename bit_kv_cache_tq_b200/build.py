@@ -53,18 +53,23 @@ def build(force=False, verbose=False):
     objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
     newest_header = max([os.path.getmtime(h) for h in _headers()] + [0.0])
-    objs = []
+    objs, jobs = [], []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         objs.append(obj)
         if not force and os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(src), newest_header):
             continue
         cmd = [nvcc(), "-c", src, "-o", obj, "-I", INCLUDE, "-I", CSRC] + NVCC_FLAGS
-        res = subprocess.run(cmd, capture_output=True, text=True)
-        if res.returncode != 0:
-            raise RuntimeError("nvcc failed for %s:\n%s\n%s" % (src, res.stdout, res.stderr))
-        if verbose:
-            sys.stderr.write(res.stderr)
+        jobs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)))
+    failed = []
+    for src, proc in jobs:  # the sources compile in parallel
+        out, err = proc.communicate()
+        if proc.returncode != 0:
+            failed.append("nvcc failed for %s:\n%s\n%s" % (src, out, err))
+        elif verbose:
+            sys.stderr.write(err)
+    if failed:
+        raise RuntimeError("\n".join(failed))
     tmp = LIB + ".tmp"
     cmd = [nvcc(), "-shared", "-o", tmp] + objs + ["-gencode", "arch=compute_100a,code=sm_100a", "-lcudart_static",
                                                    "-ldl", "-lrt", "-lpthread"]

@@ -53,6 +53,8 @@ struct DecodeArgs {
     uint32_t* err;
     int batch, hq, hkv, group, capacity, n_split, split_len;
     float sm_scale, tau;
+    uint32_t* skip_mask;  // Sparse V: [batch][hq][mask_words] bits of dropped positions, or null
+    int mask_words;
     uint32_t signs[8];
 };
 
@@ -182,6 +184,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_split_kernel(const _
             m_run[h] = m_new;
             // Sparse V: p / l_run is an upper bound on the exact weight
             const bool skip = a.tau > 0.0f && p < a.tau * l_run[h];
+            if (skip && a.skip_mask && lane == 0)
+                atomicOr(a.skip_mask + (static_cast<size_t>(b) * a.hq + kv * G + h) * a.mask_words + (t >> 5),
+                         1u << (t & 31));
             const float pv = skip ? 0.0f : p * v_norm;
 #pragma unroll
             for (int e = 0; e < V; ++e) acc[h][e] = fmaf(acc[h][e], corr, pv * kv_vals[e]);
@@ -297,7 +302,7 @@ cudaError_t launch_decode_mma(const tq_params& p, const tq_codebook* kcb, const 
                               const void* q, int q_dtype, const int32_t* seq_lens, int max_len, float* out,
                               const DecodePlan& plan, char* ws, uint32_t* err, int num_sms, cudaStream_t stream,
                               const void* k_new = nullptr, const void* v_new = nullptr, int new_dtype = 0,
-                              const PageMap* pm = nullptr);
+                              const PageMap* pm = nullptr, uint32_t* skip_mask = nullptr);
 
 }  // namespace tq
 
@@ -308,8 +313,8 @@ namespace tq {
 static tq_status decode_impl(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
                              const void* d_q, tq_dtype q_dtype, const tq_cache* cache, const int32_t* d_seq_lens,
                              int32_t max_seq_len, float* d_out, void* d_workspace, size_t workspace_bytes,
-                             uint32_t* d_error, void* stream, const void* k_new, const void* v_new,
-                             tq_dtype kv_dtype, const tq_block_table* table = nullptr) {
+                             uint32_t* d_skip_mask, uint32_t* d_error, void* stream, const void* k_new,
+                             const void* v_new, tq_dtype kv_dtype, const tq_block_table* table = nullptr) {
     tq_status st = validate_params(params);
     if (st != TQ_OK) return st;
     const tq_params& p = *params;
@@ -325,6 +330,7 @@ static tq_status decode_impl(const tq_params* params, const tq_codebook* kcb, co
     if (!d_q || !d_seq_lens || !d_out || !d_workspace || max_seq_len < 1) return TQ_ERR_INVALID_ARG;
     if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
     if (!aligned16(d_q) || !aligned16(d_out) || !aligned16(d_workspace)) return TQ_ERR_ALIGNMENT;
+    if (d_skip_mask && (reinterpret_cast<uintptr_t>(d_skip_mask) & 3u)) return TQ_ERR_ALIGNMENT;
     if (p.k_mode == TQ_MODE_TURBO && (st = validate_codebook(kcb, p.head_dim, p.k_bits)) != TQ_OK) return st;
     if (p.v_mode == TQ_MODE_TURBO && (st = validate_codebook(vcb, p.head_dim, p.v_bits)) != TQ_OK) return st;
     const bool append = k_new != nullptr;
@@ -342,7 +348,7 @@ static tq_status decode_impl(const tq_params* params, const tq_codebook* kcb, co
     if (decode_mma_supported(p)) {
         const cudaError_t e = launch_decode_mma(p, kcb, vcb, *cache, d_q, q_dtype, d_seq_lens, max_seq_len, d_out, plan,
                                                 static_cast<char*>(d_workspace), d_error, sms, s, k_new, v_new,
-                                                kv_dtype, pm);
+                                                kv_dtype, pm, d_skip_mask);
         if (e != cudaErrorNotSupported) return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
         // otherwise (shared memory too small for two stages, or a device whose
         // shared-memory window differs) take the general path
@@ -378,6 +384,8 @@ static tq_status decode_impl(const tq_params* params, const tq_codebook* kcb, co
     a.split_len = plan.split_len;
     a.sm_scale = p.sm_scale > 0.0f ? p.sm_scale : 1.0f / std::sqrt(static_cast<float>(p.head_dim));
     a.tau = p.sparse_v_threshold;
+    a.skip_mask = a.tau > 0.0f ? d_skip_mask : nullptr;
+    a.mask_words = (max_seq_len + 31) / 32;
     rotation_sign_bits(p.seed, p.head_dim, a.signs);
     cudaError_t e;
     switch (p.head_dim) {
@@ -392,21 +400,21 @@ static tq_status decode_impl(const tq_params* params, const tq_codebook* kcb, co
 extern "C" tq_status tq_decode_attention(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
                                          const void* d_q, tq_dtype q_dtype, const tq_cache* cache,
                                          const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
-                                         void* d_workspace, size_t workspace_bytes, uint32_t* d_error,
-                                         void* stream) {
+                                         void* d_workspace, size_t workspace_bytes, uint32_t* d_skip_mask,
+                                         uint32_t* d_error, void* stream) {
     return tq::decode_impl(params, kcb, vcb, d_q, q_dtype, cache, d_seq_lens, max_seq_len, d_out, d_workspace,
-                           workspace_bytes, d_error, stream, nullptr, nullptr, TQ_BF16);
+                           workspace_bytes, d_skip_mask, d_error, stream, nullptr, nullptr, TQ_BF16);
 }
 
 extern "C" tq_status tq_decode_attention_paged(const tq_params* params, const tq_codebook* kcb,
                                                const tq_codebook* vcb, const void* d_q, tq_dtype q_dtype,
                                                const tq_cache* pool, const tq_block_table* table,
                                                const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
-                                               void* d_workspace, size_t workspace_bytes, uint32_t* d_error,
-                                               void* stream) {
+                                               void* d_workspace, size_t workspace_bytes, uint32_t* d_skip_mask,
+                                               uint32_t* d_error, void* stream) {
     if (!table) return TQ_ERR_INVALID_ARG;
     return tq::decode_impl(params, kcb, vcb, d_q, q_dtype, pool, d_seq_lens, max_seq_len, d_out, d_workspace,
-                           workspace_bytes, d_error, stream, nullptr, nullptr, TQ_BF16, table);
+                           workspace_bytes, d_skip_mask, d_error, stream, nullptr, nullptr, TQ_BF16, table);
 }
 
 extern "C" tq_status tq_append_decode_attention_paged(const tq_params* params, const tq_codebook* kcb,
@@ -414,11 +422,11 @@ extern "C" tq_status tq_append_decode_attention_paged(const tq_params* params, c
                                                       tq_dtype kv_dtype, const void* d_q, tq_dtype q_dtype,
                                                       const tq_cache* pool, const tq_block_table* table,
                                                       const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
-                                                      void* d_workspace, size_t workspace_bytes, uint32_t* d_error,
-                                                      void* stream) {
+                                                      void* d_workspace, size_t workspace_bytes,
+                                                      uint32_t* d_skip_mask, uint32_t* d_error, void* stream) {
     if (!k_new || !v_new || !table) return TQ_ERR_INVALID_ARG;
     return tq::decode_impl(params, kcb, vcb, d_q, q_dtype, pool, d_seq_lens, max_seq_len, d_out, d_workspace,
-                           workspace_bytes, d_error, stream, k_new, v_new, kv_dtype, table);
+                           workspace_bytes, d_skip_mask, d_error, stream, k_new, v_new, kv_dtype, table);
 }
 
 extern "C" tq_status tq_append_decode_attention(const tq_params* params, const tq_codebook* kcb,
@@ -426,10 +434,11 @@ extern "C" tq_status tq_append_decode_attention(const tq_params* params, const t
                                                 tq_dtype kv_dtype, const void* d_q, tq_dtype q_dtype,
                                                 const tq_cache* cache, const int32_t* d_seq_lens,
                                                 int32_t max_seq_len, float* d_out, void* d_workspace,
-                                                size_t workspace_bytes, uint32_t* d_error, void* stream) {
+                                                size_t workspace_bytes, uint32_t* d_skip_mask, uint32_t* d_error,
+                                                void* stream) {
     if (!k_new || !v_new) return TQ_ERR_INVALID_ARG;
     return tq::decode_impl(params, kcb, vcb, d_q, q_dtype, cache, d_seq_lens, max_seq_len, d_out, d_workspace,
-                           workspace_bytes, d_error, stream, k_new, v_new, kv_dtype);
+                           workspace_bytes, d_skip_mask, d_error, stream, k_new, v_new, kv_dtype);
 }
 
 // ---------------------------------------------------------------------------
@@ -486,5 +495,5 @@ extern "C" tq_status tq_decode_attention_static(const tq_params* params, const t
     const long long units = static_cast<long long>(cache->batch) * params->num_kv_heads;
     if (static_scratch(&scratch, units, static_cast<cudaStream_t>(stream)) != cudaSuccess) return TQ_ERR_CUDA;
     return tq_decode_attention(params, kcb, vcb, d_q, q_dtype, cache, d_seq_lens, max_seq_len, d_out, scratch,
-                               TQ_DECODE_STATIC_SCRATCH_BYTES, d_error, stream);
+                               TQ_DECODE_STATIC_SCRATCH_BYTES, nullptr, d_error, stream);
 }

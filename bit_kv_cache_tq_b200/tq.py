@@ -89,11 +89,13 @@ _lib.tq_dequantize.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), 
                                ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
 _lib.tq_decode_attention.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p, ctypes.c_int,
                                      _P(tq_cache), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
-                                     ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+                                     ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_void_p]
 _lib.tq_append_decode_attention.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
                                             _P(tq_cache), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
-                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_void_p]
 _lib.tq_decode_attention_static.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
                                             ctypes.c_int, _P(tq_cache), ctypes.c_void_p, ctypes.c_int32,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
@@ -104,12 +106,12 @@ _lib.tq_quantize_append_paged.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_
 _lib.tq_decode_attention_paged.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
                                            ctypes.c_int, _P(tq_cache), _P(tq_block_table), ctypes.c_void_p,
                                            ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
-                                           ctypes.c_void_p, ctypes.c_void_p]
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
 _lib.tq_append_decode_attention_paged.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
                                                   ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
                                                   _P(tq_cache), _P(tq_block_table), ctypes.c_void_p, ctypes.c_int32,
                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
-                                                  ctypes.c_void_p]
+                                                  ctypes.c_void_p, ctypes.c_void_p]
 for _name in EXPORTED:
     if _name not in ("tq_status_string", "tq_abi_version"):
         getattr(_lib, _name).restype = ctypes.c_int
@@ -268,20 +270,22 @@ def tq_dequantize(params, kcb, vcb, cache, b, start, count, k_out=None, v_out=No
 
 
 def tq_decode_attention(params, kcb, vcb, q, cache, seq_lens, max_seq_len, out, workspace, error=None,
-                        stream=None):
-    """q: [batch, Hq, d] CUDA tensor; seq_lens int32 [batch]; out fp32 [batch, Hq, d]; workspace uint8."""
+                        stream=None, skip_mask=None):
+    """q: [batch, Hq, d] CUDA tensor; seq_lens int32 [batch]; out fp32 [batch, Hq, d]; workspace uint8;
+    skip_mask: zeroed int32 [batch, Hq, (max_seq_len + 31) // 32] CUDA tensor or None (Sparse V's dropped
+    positions, one bit each)."""
     assert q.is_contiguous() and out.is_contiguous() and out.dtype == torch.float32
     assert seq_lens.dtype == torch.int32 and seq_lens.is_cuda
     c = cache.struct()
     st = _lib.tq_decode_attention(ctypes.byref(params), kcb and ctypes.byref(kcb), vcb and ctypes.byref(vcb),
                                   _ptr(q), _dtype_code(q), ctypes.byref(c), _ptr(seq_lens), max_seq_len, _ptr(out),
-                                  _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(error),
-                                  _stream(stream))
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(skip_mask),
+                                  _ptr(error), _stream(stream))
     _check(st, "tq_decode_attention")
 
 
 def tq_append_decode_attention(params, kcb, vcb, k_new, v_new, q, cache, seq_lens, max_seq_len, out, workspace,
-                               error=None, stream=None):
+                               error=None, stream=None, skip_mask=None):
     """Append k_new/v_new ([batch, 1, Hkv, d]) at slot seq_lens-1, then decode attention over seq_lens tokens."""
     assert q.is_contiguous() and out.is_contiguous() and out.dtype == torch.float32
     assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.dtype == v_new.dtype
@@ -290,7 +294,8 @@ def tq_append_decode_attention(params, kcb, vcb, k_new, v_new, q, cache, seq_len
     st = _lib.tq_append_decode_attention(ctypes.byref(params), kcb and ctypes.byref(kcb), vcb and ctypes.byref(vcb),
                                          _ptr(k_new), _ptr(v_new), _dtype_code(k_new), _ptr(q), _dtype_code(q), ctypes.byref(c),
                                          _ptr(seq_lens), max_seq_len, _ptr(out), _ptr(workspace),
-                                         workspace.numel() * workspace.element_size(), _ptr(error), _stream(stream))
+                                         workspace.numel() * workspace.element_size(), _ptr(skip_mask), _ptr(error),
+                                         _stream(stream))
     _check(st, "tq_append_decode_attention")
 
 
@@ -319,7 +324,7 @@ def tq_quantize_append_paged(params, kcb, vcb, k_new, v_new, positions, pool, ta
 
 
 def tq_decode_attention_paged(params, kcb, vcb, q, pool, table, seq_lens, max_seq_len, out, workspace, error=None,
-                              stream=None):
+                              stream=None, skip_mask=None):
     """tq_decode_attention on a paged cache (see tq_quantize_append_paged)."""
     assert q.is_contiguous() and out.is_contiguous() and out.dtype == torch.float32
     assert seq_lens.dtype == torch.int32 and seq_lens.is_cuda
@@ -327,12 +332,13 @@ def tq_decode_attention_paged(params, kcb, vcb, q, pool, table, seq_lens, max_se
     st = _lib.tq_decode_attention_paged(ctypes.byref(params), kcb and ctypes.byref(kcb), vcb and ctypes.byref(vcb),
                                         _ptr(q), _dtype_code(q), ctypes.byref(c), ctypes.byref(bt), _ptr(seq_lens),
                                         max_seq_len, _ptr(out), _ptr(workspace),
-                                        workspace.numel() * workspace.element_size(), _ptr(error), _stream(stream))
+                                        workspace.numel() * workspace.element_size(), _ptr(skip_mask), _ptr(error),
+                                        _stream(stream))
     _check(st, "tq_decode_attention_paged")
 
 
 def tq_append_decode_attention_paged(params, kcb, vcb, k_new, v_new, q, pool, table, seq_lens, max_seq_len, out,
-                                     workspace, error=None, stream=None):
+                                     workspace, error=None, stream=None, skip_mask=None):
     """tq_append_decode_attention on a paged cache (see tq_quantize_append_paged)."""
     assert q.is_contiguous() and out.is_contiguous() and out.dtype == torch.float32
     assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.dtype == v_new.dtype
@@ -343,7 +349,7 @@ def tq_append_decode_attention_paged(params, kcb, vcb, k_new, v_new, q, pool, ta
                                                _dtype_code(k_new), _ptr(q), _dtype_code(q), ctypes.byref(c),
                                                ctypes.byref(bt), _ptr(seq_lens), max_seq_len, _ptr(out),
                                                _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                               _ptr(error), _stream(stream))
+                                               _ptr(skip_mask), _ptr(error), _stream(stream))
     _check(st, "tq_append_decode_attention_paged")
 
 

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 3
+#define TQ_ABI_VERSION 4
 
 typedef enum tq_status {
     TQ_OK = 0,
@@ -284,12 +284,19 @@ tq_status tq_dequantize(const tq_params* params, const tq_codebook* kcb, const t
  * the full denominator is at least l e^m, every dropped position has exact
  * weight p_i < tau.  Dropped positions stay in the denominator.  Which
  * positions are dropped depends on the launch configuration.
+ *   d_skip_mask    device uint32 [batch][Hq][(max_seq_len + 31) / 32], 4-byte
+ *                  aligned, zero-filled by the caller, or NULL.  With tau > 0
+ *                  the kernels set bit i % 32 of word i / 32 of row (b, h)
+ *                  for every position i the gate dropped from head h's V sum
+ *                  ([inferrs] "Sparse V：速度加成": the skipped low-weight V
+ *                  positions); nothing else is written.  Ignored when tau = 0.
  * An out-of-range seq_len sets TQ_DEVERR_SEQLEN and yields zeros for b.
  */
 tq_status tq_decode_attention(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
                               const void* d_q, tq_dtype q_dtype, const tq_cache* cache,
                               const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
-                              void* d_workspace, size_t workspace_bytes, uint32_t* d_error, void* stream);
+                              void* d_workspace, size_t workspace_bytes, uint32_t* d_skip_mask,
+                              uint32_t* d_error, void* stream);
 
 /*
  * One decode step of a layer in one call: append the step's new token of
@@ -300,7 +307,8 @@ tq_status tq_decode_attention(const tq_params* params, const tq_codebook* kcb, c
  *   d_seq_lens    lengths AFTER the append: sequence b's new token goes to
  *                 slot seq_lens[b] - 1 and attention covers seq_lens[b]
  *                 tokens.
- *   Other arguments as for tq_decode_attention (same workspace rules).
+ *   Other arguments as for tq_decode_attention (same workspace and skip-mask
+ *   rules).
  * The new token is encoded exactly as tq_quantize_append encodes it (the
  * cache afterwards holds what tq_quantize_append would have written, up to
  * codes within the boundary window).  On the tensor-core path (d = 128;
@@ -316,7 +324,7 @@ tq_status tq_append_decode_attention(const tq_params* params, const tq_codebook*
                                      const void* k_new, const void* v_new, tq_dtype kv_dtype, const void* d_q,
                                      tq_dtype q_dtype, const tq_cache* cache, const int32_t* d_seq_lens,
                                      int32_t max_seq_len, float* d_out, void* d_workspace, size_t workspace_bytes,
-                                     uint32_t* d_error, void* stream);
+                                     uint32_t* d_skip_mask, uint32_t* d_error, void* stream);
 
 /*
  * Paged cache.  [inferrs] manages its compressed cache with PagedAttention
@@ -364,15 +372,15 @@ tq_status tq_quantize_append_paged(const tq_params* params, const tq_codebook* k
 tq_status tq_decode_attention_paged(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
                                     const void* d_q, tq_dtype q_dtype, const tq_cache* pool,
                                     const tq_block_table* table, const int32_t* d_seq_lens, int32_t max_seq_len,
-                                    float* d_out, void* d_workspace, size_t workspace_bytes, uint32_t* d_error,
-                                    void* stream);
+                                    float* d_out, void* d_workspace, size_t workspace_bytes,
+                                    uint32_t* d_skip_mask, uint32_t* d_error, void* stream);
 tq_status tq_append_decode_attention_paged(const tq_params* params, const tq_codebook* kcb,
                                            const tq_codebook* vcb, const void* k_new, const void* v_new,
                                            tq_dtype kv_dtype, const void* d_q, tq_dtype q_dtype,
                                            const tq_cache* pool, const tq_block_table* table,
                                            const int32_t* d_seq_lens, int32_t max_seq_len, float* d_out,
-                                           void* d_workspace, size_t workspace_bytes, uint32_t* d_error,
-                                           void* stream);
+                                           void* d_workspace, size_t workspace_bytes, uint32_t* d_skip_mask,
+                                           uint32_t* d_error, void* stream);
 
 /* Bytes of the library's own decode scratch on each device. */
 #define TQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)16 << 20)

@@ -43,12 +43,18 @@ def _softmax(s):
     return e / np.sum(e)
 
 
-def decode_attention(q, k_hat, v_hat, lens, sm_scale=None, sparse_tau=0.0):
+def decode_attention(q, k_hat, v_hat, lens, sm_scale=None, sparse_tau=0.0, skip_mask=None):
     """q [B, Hq, d]; k_hat, v_hat [B, Hkv, L, d]; lens [B].
 
     Returns dict: ``out`` [B, Hq, d] (no skipping), and when sparse_tau > 0
     also ``lo``/``hi`` (the admissible interval above), ``exact_sparse``
     (skip set = E) and ``skip_fraction`` (|E| / len, averaged).
+
+    ``skip_mask`` (bool [B, Hq, >= max len], optional) is a skip set M per
+    (b, h): then ``masked`` [B, Hq, d] is sum_{i not in M} p_i v_i with the
+    denominator over every position, ``mask_max_weight`` [B, Hq] the largest
+    exact weight p_i among the positions in M (0 when M is empty) and
+    ``mask_count`` [B, Hq] the size of M below the length.
     """
     q = np.asarray(q, dtype=np.float64)
     bsz, hq, d = q.shape
@@ -60,6 +66,9 @@ def decode_attention(q, k_hat, v_hat, lens, sm_scale=None, sparse_tau=0.0):
     hi = np.zeros_like(out)
     exact = np.zeros_like(out)
     skipped = []
+    masked = np.zeros_like(out)
+    mask_max = np.zeros((bsz, hq))
+    mask_count = np.zeros((bsz, hq), dtype=np.int64)
     for b in range(bsz):
         n = int(lens[b])
         for h in range(hq):
@@ -68,6 +77,11 @@ def decode_attention(q, k_hat, v_hat, lens, sm_scale=None, sparse_tau=0.0):
             v = np.asarray(v_hat[b, kv, :n], dtype=np.float64)
             p = _softmax(scale * (k @ q[b, h]))
             out[b, h] = p @ v
+            if skip_mask is not None:
+                m = np.asarray(skip_mask[b, h, :n], dtype=bool)
+                masked[b, h] = p[~m] @ v[~m]
+                mask_max[b, h] = p[m].max() if m.any() else 0.0
+                mask_count[b, h] = int(m.sum())
             if sparse_tau > 0:
                 e = p < sparse_tau
                 contrib = p[e, None] * v[e]
@@ -76,6 +90,8 @@ def decode_attention(q, k_hat, v_hat, lens, sm_scale=None, sparse_tau=0.0):
                 exact[b, h] = p[~e] @ v[~e]
                 skipped.append(np.mean(e))
     res = {"out": out}
+    if skip_mask is not None:
+        res.update(masked=masked, mask_max_weight=mask_max, mask_count=mask_count)
     if sparse_tau > 0:
         res.update(lo=lo, hi=hi, exact_sparse=exact, skip_fraction=float(np.mean(skipped)))
     return res
@@ -95,3 +111,27 @@ def attention_rotated(q, signs, k_yhat, k_norm, v_yhat, v_norm, sm_scale=None):
     p = _softmax(s)
     acc = (p * np.asarray(v_norm, dtype=np.float64)) @ np.asarray(v_yhat, dtype=np.float64)
     return rotation.unrotate(acc, signs)
+
+
+def prefill_attention(q, k_hat, v_hat, start, sm_scale=None):
+    """Chunked prefill over a cache that already holds the chunk.
+
+    q [B, C, Hq, d] are the queries of C new tokens of each sequence;
+    k_hat, v_hat [B, Hkv, L, d] the reconstructed cache with the chunk at
+    positions start[b] .. start[b] + C - 1.  Query j of sequence b attends
+    causally to positions 0 .. start[b] + j (itself included), exactly as
+    a decode step over start[b] + j + 1 tokens would ([google] table "M5 Max
+    128GB 上的實測" and [inferrs] table "性能表现" measure prefill from the
+    compressed cache; the pages give no other rule, so the chunk attends to
+    its own tokens in compressed form, as the decode step attends to the
+    token it appended).  Returns out [B, C, Hq, d].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    bsz, c, hq, d = q.shape
+    out = np.zeros((bsz, c, hq, d))
+    for b in range(bsz):
+        for j in range(c):
+            r = decode_attention(q[b:b + 1, j], k_hat[b:b + 1], v_hat[b:b + 1], [int(start[b]) + j + 1], sm_scale)
+            out[b, j] = r["out"][0]
+    return out
+

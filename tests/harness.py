@@ -175,8 +175,9 @@ def gpu_quantize(layer, k, v, capacity, positions=None, cache=None):
     return cache, st, word
 
 
-def gpu_decode(layer, q, cache, lens, max_len=None, ws=None):
-    """Decode attention through the C ABI; a fresh zeroed workspace unless `ws` is given."""
+def gpu_decode(layer, q, cache, lens, max_len=None, ws=None, with_mask=False):
+    """Decode attention through the C ABI; a fresh zeroed workspace unless `ws` is given.
+    with_mask: also return the Sparse-V skip mask as bool [B, Hq, max_len]."""
     bsz = q.shape[0]
     lens_t = torch.as_tensor(np.asarray(lens), dtype=torch.int32).cuda()
     max_len = int(max(lens)) if max_len is None else max_len
@@ -184,10 +185,20 @@ def gpu_decode(layer, q, cache, lens, max_len=None, ws=None):
         ws = torch.zeros(tq.tq_decode_workspace_bytes(layer.params, bsz, max_len), dtype=torch.uint8, device="cuda")
     out = torch.empty(bsz, layer.hq, layer.d, dtype=torch.float32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mask = torch.zeros(bsz, layer.hq, (max_len + 31) // 32, dtype=torch.int32, device="cuda") if with_mask else None
     tq.tq_decode_attention(layer.params, layer.kcb, layer.vcb, q.cuda().contiguous(), cache, lens_t, max_len, out, ws,
-                           err)
+                           err, skip_mask=mask)
     st, word = tq.tq_read_device_error(err)
+    if with_mask:
+        return out.cpu().numpy(), st, word, unpack_mask(mask.cpu().numpy(), max_len)
     return out.cpu().numpy(), st, word
+
+
+def unpack_mask(words, n):
+    """int32 words [B, Hq, W] (bit i % 32 of word i / 32 = position i) -> bool [B, Hq, n]."""
+    w = words.astype(np.uint32)
+    bits = (w[..., :, None] >> np.arange(32, dtype=np.uint32)) & 1
+    return bits.reshape(w.shape[0], w.shape[1], -1)[..., :n].astype(bool)
 
 
 def stored_hat(layer, cache, b, h, n, which):
@@ -211,7 +222,7 @@ def stored_hat(layer, cache, b, h, n, which):
     return layer.oracle_decode(enc, which)
 
 
-def oracle_attention(layer, q, khat, vhat, lens, tau=0.0):
-    """q [B, Hq, d]; khat/vhat [B, Hkv, L, d] fp64."""
+def oracle_attention(layer, q, khat, vhat, lens, tau=0.0, skip_mask=None):
+    """q [B, Hq, d]; khat/vhat [B, Hkv, L, d] fp64; skip_mask bool [B, Hq, L] or None."""
     return oatt.decode_attention(np.asarray(q, dtype=np.float64), khat, vhat, lens,
-                                 layer.params.sm_scale or None, sparse_tau=tau)
+                                 layer.params.sm_scale or None, sparse_tau=tau, skip_mask=skip_mask)

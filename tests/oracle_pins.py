@@ -385,3 +385,63 @@ def pin_rotated_domain(att, q, cb, rng):
     k_y = ck[ek["codes"]] + (ek["gamma16"].astype(np.float64) * math.sqrt(math.pi / 2) / 64)[:, None] * ((2.0 * ek["qjl_bits"] - 1.0) @ sk)
     got = att.attention_rotated(qv, s, k_y, ek["norm16"], cv[ev["codes"]], ev["norm16"])
     assert np.allclose(got, ref, atol=1e-12, rtol=0)
+
+
+def pin_masked_sum(att):
+    """The sum with a given skip set (reading of [inferrs] "Sparse V：速度加成":
+    dropped positions leave the numerator, never the denominator): an empty
+    set gives full attention, the set E = {p_i < tau} gives the exact sparse
+    sum, the full set gives zero, and a two-token hand case with weights
+    3/4, 1/4 (score gap ln 3) dropping the second token gives 3/4 v_0."""
+    gen = np.random.default_rng(3)
+    q = gen.normal(size=(1, 2, 8))
+    k = gen.normal(size=(1, 1, 40, 8)) * 3.0
+    v = gen.normal(size=(1, 1, 40, 8))
+    none = np.zeros((1, 2, 40), dtype=bool)
+    r0 = att.decode_attention(q, k, v, [40], sparse_tau=0.05, skip_mask=none)
+    assert np.allclose(r0["masked"], r0["out"], rtol=0, atol=1e-14)
+    assert np.all(r0["mask_count"] == 0) and np.all(r0["mask_max_weight"] == 0)
+    s = np.einsum("hd,ld->hl", q[0], k[0, 0]) / math.sqrt(8)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    e = (p < 0.05)[None]
+    r1 = att.decode_attention(q, k, v, [40], sparse_tau=0.05, skip_mask=e)
+    assert np.allclose(r1["masked"], r1["exact_sparse"], rtol=0, atol=1e-14)
+    assert np.all(r1["mask_count"] == e.sum(axis=2)) and np.all(r1["mask_max_weight"] < 0.05)
+    r2 = att.decode_attention(q, k, v, [40], skip_mask=np.ones((1, 2, 40), dtype=bool))
+    assert np.all(r2["masked"] == 0.0)
+    # hand case: keys chosen so that the scores differ by ln 3
+    d = 4
+    qq = np.array([[[2.0, 0.0, 0.0, 0.0]]])
+    kk = np.zeros((1, 1, 2, d))
+    kk[0, 0, 0, 0] = math.log(3.0)  # scores ln 3 and 0 (sm_scale 1/2)
+    vv = np.array([[[[1.0, 2.0, 3.0, 4.0], [5.0, 6.0, 7.0, 8.0]]]])
+    r3 = att.decode_attention(qq, kk, vv, [2], skip_mask=np.array([[[False, True]]]))
+    assert np.allclose(r3["masked"][0, 0], 0.75 * vv[0, 0, 0], rtol=0, atol=1e-14)
+    assert abs(r3["mask_max_weight"][0, 0] - 0.25) < 1e-14
+
+
+def pin_prefill(att):
+    """Chunked prefill: a chunk of one query is one decode step over start + 1
+    positions; with identical keys (equal scores) query j's output is the
+    plain mean of v_0 .. v_{start+j} (the causal prefix, itself included),
+    which fixes the causal limit; with q = 0 the same holds for any keys."""
+    gen = np.random.default_rng(5)
+    d, hkv, hq, L = 16, 2, 4, 30
+    k = gen.normal(size=(1, hkv, L, d))
+    v = gen.normal(size=(1, hkv, L, d))
+    q = gen.normal(size=(1, 1, hq, d))
+    one = att.prefill_attention(q, k, v, [11])
+    dec = att.decode_attention(q[:, 0], k, v, [12])["out"]
+    assert np.allclose(one[:, 0], dec, rtol=0, atol=1e-14)
+    same = np.broadcast_to(k[:, :, :1], k.shape).copy()
+    qc = gen.normal(size=(1, 5, hq, d))
+    out = att.prefill_attention(qc, same, v, [20])
+    for j in range(5):
+        for h in range(hq):
+            want = v[0, h // (hq // hkv), :20 + j + 1].mean(axis=0)
+            assert np.allclose(out[0, j, h], want, rtol=0, atol=1e-12), (j, h)
+    zero = att.prefill_attention(np.zeros((1, 3, hq, d)), k, v, [7])
+    for j in range(3):
+        assert np.allclose(zero[0, j, 0], v[0, 0, :7 + j + 1].mean(axis=0), rtol=0, atol=1e-12)
+

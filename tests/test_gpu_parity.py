@@ -185,6 +185,41 @@ def test_sparse_v_within_admissible_interval():
     assert outside.max() < H.ATTN_TOL, outside.max()
 
 
+# A dropped position's weight as the kernel sees it is below tau; the
+# oracle's exact weight of the same position differs from the kernel's by the
+# kernel's score error (fp16 centroids and query terms, about 1e-3 in the
+# logit), so the oracle's weight stays below tau * (1 + 1e-2).
+MASK_SLACK = 1e-2
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_sparse_v_mask_is_admissible_and_exact(d):
+    """Sparse V with the kernel's skip mask (d = 128: tensor-core kernel, the
+    70B-shaped settings at small size; d = 64: the general kernels): every
+    dropped position has exact weight below tau, the output equals the
+    oracle's sum without exactly those positions (the denominator keeps
+    them), and the gate fires on log-normal data."""
+    if d == 128:
+        layer = H.Layer(128, 64, 8, k_bits=3, v_bits=2, qjl_dims=64, seed=9, tau=1e-6)
+    else:
+        layer = H.Layer(64, 16, 4, k_bits=3, v_bits=2, seed=9, tau=1e-6)
+    t = 2500
+    k = inputs.lognormal_kv(1, t, layer.hkv, d, seed=6, layer=9, which=inputs.K)
+    v = inputs.lognormal_kv(1, t, layer.hkv, d, seed=6, layer=9, which=inputs.V)
+    q = inputs.queries(1, layer.hq, d, seed=6, layer=9)
+    cache, st, _ = H.gpu_quantize(layer, k, v, t)
+    enc = _check_quantized(layer, cache, _to_np(k), _to_np(v))
+    khat = _oracle_hat(layer, enc[0], 0, (1, layer.hkv, t, d))
+    vhat = _oracle_hat(layer, enc[1], 1, (1, layer.hkv, t, d))
+    got, st, word, mask = H.gpu_decode(layer, q, cache, [t], with_mask=True)
+    assert st == tq.TQ_OK and word == 0
+    ref = H.oracle_attention(layer, _to_np(q), khat, vhat, [t], tau=1e-6, skip_mask=mask)
+    assert ref["mask_max_weight"].max() < 1e-6 * (1 + MASK_SLACK), ref["mask_max_weight"].max()
+    assert H.rel_l2_per_vector(got, ref["masked"]).max() < H.ATTN_TOL
+    frac = mask.sum() / mask.size
+    assert frac > 0.01, frac
+
+
 def test_sparse_v_exact_on_separated_scores():
     """Scores built so that the skip set is unambiguous: 4 of every 16
     positions are 'hot' (scores ~ +8), the rest 'cold' (~ -8, weight < 1e-6
@@ -211,10 +246,12 @@ def test_sparse_v_exact_on_separated_scores():
     vhat = layer.oracle_decode(enc[1], 1)[None, None]
     ref = H.oracle_attention(layer, _to_np(q), khat, vhat, [t], tau=1e-6)
     assert abs(ref["skip_fraction"] - 0.75) < 1e-9
-    got, st, _ = H.gpu_decode(layer, q, cache, [t])
+    got, st, _, mask = H.gpu_decode(layer, q, cache, [t], with_mask=True)
     assert st == tq.TQ_OK
     assert H.rel_l2_per_vector(got, ref["exact_sparse"]).max() < H.ATTN_TOL
     assert H.rel_l2_per_vector(ref["exact_sparse"], ref["out"]).min() > 10 * H.ATTN_TOL
+    # the kernel reports exactly the cold positions, for every head
+    assert np.array_equal(mask, np.broadcast_to((~hot).numpy(), mask.shape))
 
 
 @pytest.mark.parametrize("d", [128, 256])

@@ -53,7 +53,7 @@ def test_binding_declares_every_argument_type():
 
 
 def test_abi_version_and_status_strings():
-    assert tq.tq_abi_version() == 3
+    assert tq.tq_abi_version() == 4
     for st in range(8):
         assert tq.tq_status_string(st)
     assert tq.tq_status_string(99) == "unknown status"
@@ -206,12 +206,15 @@ def test_entry_points_reject_bad_arguments_before_launch():
     assert lib.tq_dequantize(*args, ctypes.byref(cache), 0, 60, 8, fake, fake, None) == tq.TQ_ERR_INVALID_ARG
     assert lib.tq_dequantize(*args, ctypes.byref(cache), 1, 0, 8, fake, fake, None) == tq.TQ_ERR_INVALID_ARG
     # decode: null workspace, bad max length, misaligned output
-    assert lib.tq_decode_attention(*args, fake, tq.TQ_BF16, ctypes.byref(cache), fake, 64, fake, None, 0, None,
+    assert lib.tq_decode_attention(*args, fake, tq.TQ_BF16, ctypes.byref(cache), fake, 64, fake, None, 0, None, None,
                                    None) == tq.TQ_ERR_INVALID_ARG
     assert lib.tq_decode_attention(*args, fake, tq.TQ_BF16, ctypes.byref(cache), fake, 0, fake, fake, 1 << 20, None,
-                                   None) == tq.TQ_ERR_INVALID_ARG
+                                   None, None) == tq.TQ_ERR_INVALID_ARG
     assert lib.tq_decode_attention(*args, fake, tq.TQ_BF16, ctypes.byref(cache), fake, 64, fake + 8, fake, 1 << 20,
-                                   None, None) == tq.TQ_ERR_ALIGNMENT
+                                   None, None, None) == tq.TQ_ERR_ALIGNMENT
+    # a skip mask that is not 4-byte aligned
+    assert lib.tq_decode_attention(*args, fake, tq.TQ_BF16, ctypes.byref(cache), fake, 64, fake, fake, 1 << 20,
+                                   fake + 2, None, None) == tq.TQ_ERR_ALIGNMENT
     # error-word reader
     word = ctypes.c_uint32()
     assert lib.tq_read_device_error(None, ctypes.byref(word), None, 10) == tq.TQ_ERR_INVALID_ARG
@@ -224,7 +227,7 @@ def test_append_decode_rejects_bad_arguments_before_launch():
     fake = 1 << 20
     cache = tq.tq_cache(1, 64, fake, fake, None, None, fake, fake, None)
     args = (ctypes.byref(p), ctypes.byref(kcb), ctypes.byref(vcb))
-    tail = (fake, tq.TQ_BF16, ctypes.byref(cache), fake, 64, fake, fake, 1 << 20, None, None)
+    tail = (fake, tq.TQ_BF16, ctypes.byref(cache), fake, 64, fake, fake, 1 << 20, None, None, None)
     assert lib.tq_append_decode_attention(*args, None, fake, tq.TQ_BF16, *tail) == tq.TQ_ERR_INVALID_ARG
     assert lib.tq_append_decode_attention(*args, fake, None, tq.TQ_BF16, *tail) == tq.TQ_ERR_INVALID_ARG
     assert lib.tq_append_decode_attention(*args, fake + 4, fake, tq.TQ_BF16, *tail) == tq.TQ_ERR_ALIGNMENT
@@ -248,7 +251,7 @@ def test_paged_entry_points_reject_bad_arguments_before_launch():
 
     def decode(pool_, table_):
         return lib.tq_decode_attention_paged(*args, fake, tq.TQ_BF16, ctypes.byref(pool_),
-                                             table_ and ctypes.byref(table_), fake, 64, fake, None, 0, None, None)
+                                             table_ and ctypes.byref(table_), fake, 64, fake, None, 0, None, None, None)
 
     assert append(pool, None) == tq.TQ_ERR_INVALID_ARG
     assert append(pool, tq.tq_block_table(None, 2, 4)) == tq.TQ_ERR_INVALID_ARG
@@ -263,7 +266,7 @@ def test_paged_entry_points_reject_bad_arguments_before_launch():
     assert decode(pool, table) == tq.TQ_ERR_INVALID_ARG
     assert lib.tq_append_decode_attention_paged(*args, None, fake, tq.TQ_BF16, fake, tq.TQ_BF16,
                                                 ctypes.byref(pool), ctypes.byref(table), fake, 64, fake, fake,
-                                                1 << 20, None, None) == tq.TQ_ERR_INVALID_ARG
+                                                1 << 20, None, None, None) == tq.TQ_ERR_INVALID_ARG
 
 
 def test_binding_constants_match_the_header():

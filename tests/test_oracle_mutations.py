@@ -205,3 +205,44 @@ def test_box_muller_control():
     r = R()
     r.qjl_matrix = lambda seed, m, d: _box_muller(seed, m, d)
     P.pin_first_qjl_pair(r)
+
+
+def test_masked_sum_drops_from_denominator(monkeypatch):
+    """Renormalising over the kept positions (dropping skipped positions from
+    the denominator too) must fail a pin."""
+    real = attention.decode_attention
+
+    def bad(q, k_hat, v_hat, lens, sm_scale=None, sparse_tau=0.0, skip_mask=None):
+        res = real(q, k_hat, v_hat, lens, sm_scale, sparse_tau, skip_mask)
+        if skip_mask is not None:
+            qd = np.asarray(q, dtype=np.float64)
+            g = qd.shape[1] // k_hat.shape[1]
+            scale = sm_scale or 1.0 / math.sqrt(qd.shape[-1])
+            for b in range(qd.shape[0]):
+                n = int(lens[b])
+                for h in range(qd.shape[1]):
+                    s = scale * (k_hat[b, h // g, :n] @ qd[b, h])
+                    p = np.exp(s - s.max())
+                    p /= p.sum()
+                    kept = p[~np.asarray(skip_mask[b, h, :n], dtype=bool)].sum()
+                    res["masked"][b, h] = res["masked"][b, h] / kept if kept > 0 else 0.0
+        return res
+    monkeypatch.setattr(attention, "decode_attention", bad)
+    _fails(P.pin_masked_sum, attention)
+
+
+@pytest.mark.parametrize("shift", [0, 2])
+def test_prefill_causal_limit_off_by_one(monkeypatch, shift):
+    """Query j seeing positions up to start + j - 1 (itself excluded) or up to
+    start + j + 1 (one token of the future) must fail a pin."""
+    def bad(q, k_hat, v_hat, start, sm_scale=None):
+        q = np.asarray(q, dtype=np.float64)
+        out = np.zeros(q.shape)
+        for b in range(q.shape[0]):
+            for j in range(q.shape[1]):
+                n = max(1, int(start[b]) + j + shift)
+                out[b, j] = attention.decode_attention(q[b:b + 1, j], k_hat[b:b + 1], v_hat[b:b + 1], [n],
+                                                       sm_scale)["out"][0]
+        return out
+    monkeypatch.setattr(attention, "prefill_attention", bad)
+    _fails(P.pin_prefill, attention)

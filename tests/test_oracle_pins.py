@@ -99,3 +99,12 @@ def test_rotated_domain_equals_original_domain():
 
 def test_oracle_package_exports():
     assert {"rng", "rotation", "codebook", "quantize", "attention"} <= set(dir(oracle))
+
+
+def test_masked_sparse_sum():
+    P.pin_masked_sum(attention)
+
+
+def test_prefill_causal_attention():
+    P.pin_prefill(attention)
+
