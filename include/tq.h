@@ -327,6 +327,32 @@ tq_status tq_append_decode_attention(const tq_params* params, const tq_codebook*
                                      uint32_t* d_skip_mask, uint32_t* d_error, void* stream);
 
 /*
+ * Chunked prefill from the compressed cache ([google] table "M5 Max 128GB
+ * 上的實測" and [inferrs] table "性能表现" measure prefill over TurboQuant
+ * caches): append n_new tokens of every sequence to the cache exactly as
+ * tq_quantize_append does (slots positions[b] .. positions[b] + n_new - 1),
+ * then attend causally with their queries: query j of sequence b attends to
+ * cache positions 0 .. positions[b] + j (itself included), the result of a
+ * decode step over positions[b] + j + 1 tokens.
+ *   k_new, v_new  device, [batch][n_new][Hkv][d] in kv_dtype, 16-byte aligned.
+ *   d_q           device, [batch][n_new][Hq][d] in q_dtype.
+ *   d_positions   device int32 [batch]: the chunk's first slot per sequence.
+ *   d_out         device, [batch][n_new][Hq][d] fp32.
+ * Supported: d = 128, TURBO keys and values (2, 3 or 4 bits), no QJL
+ * sketch, at most 16 query heads per kv head; other configurations return
+ * TQ_ERR_UNSUPPORTED before any launch.  The products Q K~^T and P V~ run on
+ * the tcgen05 tensor cores (fp16 operands, fp32 accumulation in tensor
+ * memory), 128 query rows (tokens x heads of a kv head's group) per block.
+ * A position out of range sets TQ_DEVERR_POSITION; that sequence gets no
+ * append and zero outputs.  Two kernels on `stream`: the append, then the
+ * attention.
+ */
+tq_status tq_prefill_attention(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
+                               const void* k_new, const void* v_new, tq_dtype kv_dtype, const void* d_q,
+                               tq_dtype q_dtype, int32_t n_new, const int32_t* d_positions, const tq_cache* cache,
+                               float* d_out, uint32_t* d_error, void* stream);
+
+/*
  * Paged cache.  [inferrs] manages its compressed cache with PagedAttention
  * ("二、inferrs：TurboQuant 轻量推理服务器"); the pages give no page format,
  * so this one follows the usual block-table scheme.  The pool is a tq_cache whose

@@ -1,0 +1,123 @@
+"""tq_prefill_attention (append a chunk of tokens, then causal attention of
+its queries over the compressed cache, on the tcgen05 tensor cores) against
+the oracle: the appended codes follow the code rules, and every output row
+matches the oracle's causal attention on the GPU's stored codes within 2e-3
+relative L2.  Chunks span several 128-row query blocks and several 64-key
+tiles with ragged ends."""
+
+import numpy as np
+import pytest
+import torch
+
+import harness as H
+from bit_kv_cache_tq_b200 import inputs, tq
+from oracle import attention as oatt
+
+pytestmark = pytest.mark.gpu
+
+
+def _prefill_case(layer, starts, n_new, seed, prefill_tokens=None):
+    """Cache pre-filled with `starts[b]` tokens per sequence (GPU quantise),
+    then one tq_prefill_attention call appending n_new fresh tokens."""
+    bsz, hkv, d = len(starts), layer.hkv, layer.d
+    cap = max(starts) + n_new + 40
+    pre = max(starts) if prefill_tokens is None else prefill_tokens
+    k0 = inputs.lognormal_kv(bsz, max(pre, 1), hkv, d, seed=seed, layer=3, which=inputs.K)
+    v0 = inputs.lognormal_kv(bsz, max(pre, 1), hkv, d, seed=seed, layer=3, which=inputs.V)
+    cache, st, word = H.gpu_quantize(layer, k0, v0, cap)
+    assert st == tq.TQ_OK and word == 0
+    kn = inputs.lognormal_kv(bsz, n_new, hkv, d, seed=seed, layer=3, which=inputs.K, token_offset_seed=5)
+    vn = inputs.lognormal_kv(bsz, n_new, hkv, d, seed=seed, layer=3, which=inputs.V, token_offset_seed=5)
+    q = torch.randn(bsz, n_new, layer.hq, d, generator=torch.Generator().manual_seed(seed)).to(torch.bfloat16)
+    pos = torch.tensor(starts, dtype=torch.int32, device="cuda")
+    out = torch.empty(bsz, n_new, layer.hq, d, dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.tq_prefill_attention(layer.params, layer.kcb, layer.vcb, kn.cuda(), vn.cuda(), q.cuda(), pos, cache, out, err)
+    st, word = tq.tq_read_device_error(err)
+    assert st == tq.TQ_OK and word == 0, (st, word)
+    return cache, out.cpu().numpy(), q, (kn, vn)
+
+
+def _check_rows(layer, cache, out, q, starts, rows=None):
+    """Oracle causal attention on the GPU's stored codes, row by row (all rows,
+    or the sampled (b, j) pairs given)."""
+    bsz, n_new = out.shape[0], out.shape[1]
+    worst = 0.0
+    for b in range(bsz):
+        n = starts[b] + n_new
+        khat = np.stack([H.stored_hat(layer, cache, b, h, n, 0) for h in range(layer.hkv)])[None]
+        vhat = np.stack([H.stored_hat(layer, cache, b, h, n, 1) for h in range(layer.hkv)])[None]
+        qb = q[b:b + 1].float().numpy().astype(np.float64)
+        js = range(n_new) if rows is None else [j for (bb, j) in rows if bb == b]
+        for j in js:
+            ref = oatt.decode_attention(qb[:, j], khat, vhat, [starts[b] + j + 1], layer.params.sm_scale or None)["out"]
+            rel = H.rel_l2_per_vector(out[b:b + 1, j], ref)
+            worst = max(worst, rel.max())
+    return worst
+
+
+def _check_appended_codes(layer, cache, starts, n_new, kn, vn):
+    for b, s0 in enumerate(starts):
+        for which, x, codes, norms in ((0, kn, cache.k_codes, cache.k_norms), (1, vn, cache.v_codes, cache.v_norms)):
+            for h in range(layer.hkv):
+                rows = x[b, :, h].float().numpy().astype(np.float64)
+                enc = layer.oracle_encode(rows, which)
+                got = codes[b, h, s0:s0 + n_new].cpu().numpy()
+                _, bits = layer.side(which)
+                _, t_or = H.oracle_codebook(layer.d, bits)
+                H.check_codes(got, enc, bits, layer.d, t_or)
+                H.check_norms(norms[b, h, s0:s0 + n_new].cpu().numpy().view(np.uint16), enc["norm16"])
+
+
+@pytest.mark.parametrize("hq,hkv,kb,vb", [(32, 8, 4, 2), (64, 8, 3, 2), (8, 8, 2, 4), (16, 1, 4, 3)])
+def test_prefill_matches_oracle(hq, hkv, kb, vb):
+    """Two sequences with different starts; 100 new tokens: several query
+    blocks (128 / G tokens each) and a ragged last one; ~13 key tiles."""
+    layer = H.Layer(128, hq, hkv, k_bits=kb, v_bits=vb, seed=21)
+    starts = [700, 333]
+    cache, out, q, (kn, vn) = _prefill_case(layer, starts, 100, seed=21)
+    _check_appended_codes(layer, cache, starts, 100, kn, vn)
+    worst = _check_rows(layer, cache, out, q, starts)
+    assert worst < H.ATTN_TOL, worst
+
+
+def test_prefill_chunk_of_one_is_a_decode_step():
+    """One new token: the same as tq_append_decode_attention over start + 1."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=22)
+    starts = [517]
+    cache, out, q, (kn, vn) = _prefill_case(layer, starts, 1, seed=22)
+    worst = _check_rows(layer, cache, out, q, starts)
+    assert worst < H.ATTN_TOL, worst
+
+
+def test_prefill_from_an_empty_cache():
+    """Start 0: the chunk attends only to itself (causal within the chunk)."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=23)
+    cache, out, q, _ = _prefill_case(layer, [0], 150, seed=23, prefill_tokens=1)
+    worst = _check_rows(layer, cache, out, q, [0])
+    assert worst < H.ATTN_TOL, worst
+
+
+@pytest.mark.slow
+def test_prefill_llama8b_32k_chunk_sampled_rows():
+    """Llama-3-8B-shaped layer, 32768 cached tokens, a 512-token chunk (the
+    benchmark's prefill workload), 16 sampled rows against the oracle."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=24)
+    starts = [32768]
+    cache, out, q, _ = _prefill_case(layer, starts, 512, seed=24)
+    gen = np.random.default_rng(24)
+    rows = [(0, int(j)) for j in sorted(gen.choice(512, size=16, replace=False))] + [(0, 0), (0, 511)]
+    worst = _check_rows(layer, cache, out, q, starts, rows=rows)
+    assert worst < H.ATTN_TOL, worst
+
+
+def test_prefill_rejects_unsupported_settings():
+    layer = H.Layer(128, 64, 8, k_bits=3, v_bits=2, qjl_dims=64, seed=25)
+    cache = tq.alloc_cache(layer.params, 1, 64)
+    x = torch.zeros(1, 4, 8, 128, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(1, 4, 64, 128, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(1, 4, 64, 128, device="cuda")
+    with pytest.raises(tq.TqError) as ei:
+        tq.tq_prefill_attention(layer.params, layer.kcb, layer.vcb, x, x, q, torch.zeros(1, dtype=torch.int32,
+                                device="cuda"), cache, out)
+    assert ei.value.status == tq.TQ_ERR_UNSUPPORTED
