@@ -487,6 +487,60 @@ def paged_decode(dev, reps=10, copies=4):
     return res
 
 
+PREFILL_CHUNK = 512
+
+
+def prefill_chunk(dev, reps=10):
+    """Chunked prefill from the compressed cache (tq_prefill_attention): the
+    Llama-3-8B-shaped layer (B=1, Hq=32, Hkv=8, d=128, K4/V2) with 32768
+    cached tokens and a 512-token chunk appended and attended causally.
+    Reports the call (append kernel + attention kernel) and the attention's
+    algorithmic tensor work: 4 d FLOPs per (query, head, visible key) for
+    Q K^T and P V, against the measured dense bf16 peak (fp16 operands have
+    the same nominal rate)."""
+    from bit_kv_cache_tq_b200 import inputs, tq
+    p = tq.make_params(D, HQ, HKV, K_BITS, V_BITS, seed=SEED)
+    kcb, vcb = tq.tq_codebook_init(D, K_BITS), tq.tq_codebook_init(D, V_BITS)
+    n_new, start = PREFILL_CHUNK, CONTEXT
+    cache = tq.alloc_cache(p, 1, start + n_new, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    k = inputs.lognormal_kv(1, start, HKV, D, SEED, 70, inputs.K, device=dev)
+    v = inputs.lognormal_kv(1, start, HKV, D, SEED, 70, inputs.V, device=dev)
+    tq.tq_quantize_append(p, kcb, vcb, k, v, torch.zeros(1, dtype=torch.int32, device=dev), cache, err)
+    del k, v
+    kn = inputs.lognormal_kv(1, n_new, HKV, D, SEED, 70, inputs.K, device=dev, token_offset_seed=3)
+    vn = inputs.lognormal_kv(1, n_new, HKV, D, SEED, 70, inputs.V, device=dev, token_offset_seed=3)
+    q = inputs.queries(1, n_new * HQ, D, SEED, layer=70, device=dev).view(1, n_new, HQ, D)
+    pos = torch.full((1,), start, dtype=torch.int32, device=dev)
+    out = torch.empty(1, n_new, HQ, D, dtype=torch.float32, device=dev)
+    for _ in range(3):
+        tq.tq_prefill_attention(p, kcb, vcb, kn, vn, q, pos, cache, out, err)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        tq.tq_prefill_attention(p, kcb, vcb, kn, vn, q, pos, cache, out, err)
+    e1.record()
+    e1.synchronize()
+    st, word = tq.tq_read_device_error(err)
+    assert st == tq.TQ_OK, ("prefill", st, word)
+    us = 1000.0 * e0.elapsed_time(e1) / reps
+    keys = sum(start + j + 1 for j in range(n_new))  # visible keys per (query, head), summed over the chunk
+    flops = 4.0 * D * HQ * keys
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            peak_tf, peak_kind = float(json.load(fh)["bf16_tflops"]), "measured bf16 burst"
+    except (OSError, KeyError, ValueError):
+        peak_tf, peak_kind = 1590.0, "fallback"
+    tflops = flops / (us * 1e-6) / 1e12
+    del cache
+    torch.cuda.empty_cache()
+    return {"workload": "llama3-8b-shaped layer, %d cached tokens + a %d-token chunk, K4/V2, causal" % (start, n_new),
+            "us_per_call": round(us, 2), "tokens_per_s": round(n_new / (us * 1e-6)),
+            "attention_tflops": round(tflops, 1), "peak_tflops": peak_tf, "peak_kind": peak_kind,
+            "frac_of_peak": round(tflops / peak_tf, 4), "algorithmic_flops": flops,
+            "kernels": "tq_prefill_attention: quantise-append of the chunk, then the tcgen05 attention kernel"}
+
+
 def run_tq(args, world, rank, local):
     from bit_kv_cache_tq_b200 import inputs, tq
     dev = torch.device("cuda", local)
@@ -665,6 +719,7 @@ def run_tq(args, world, rank, local):
             line["decode_configs"] = decode_configs(dev)
             line["paged_decode"] = {"workload": "llama3-8b-shaped layer, 32768 tokens, K4/V2, through a block "
                                                 "table (blocks in random order)", **paged_decode(dev)}
+            line["prefill"] = prefill_chunk(dev)
             peak_gbs = measured_peaks()[0]
             q = {"workload": "bulk prefill quantise: 262144 tokens x 8 kv heads, bf16, 32 layers (0, 1, 30, 31 "
                              "int8 per-vector absmax, others K4/V3 turbo), one input slab, 32 distinct outputs",
@@ -693,6 +748,18 @@ def run_profile_case(args):
     if args.profile == "quantize":
         for _ in range(args.warmup + args.steps):
             tq.tq_quantize_append(params, kcb, vcb, k, v, pos, cache, err)
+    elif args.profile == "prefill":
+        # a 512-token chunk after 32768 cached tokens (the prefill workload)
+        pcache = tq.alloc_cache(params, BATCH, CONTEXT + PREFILL_CHUNK, device=dev)
+        tq.tq_quantize_append(params, kcb, vcb, k[:, :CONTEXT].contiguous(), v[:, :CONTEXT].contiguous(), pos,
+                              pcache, err)
+        kn = inputs.lognormal_kv(BATCH, PREFILL_CHUNK, HKV, D, SEED, 0, inputs.K, device=dev, token_offset_seed=3)
+        vn = inputs.lognormal_kv(BATCH, PREFILL_CHUNK, HKV, D, SEED, 0, inputs.V, device=dev, token_offset_seed=3)
+        q = inputs.queries(BATCH, PREFILL_CHUNK * HQ, D, SEED, device=dev).view(BATCH, PREFILL_CHUNK, HQ, D)
+        start = torch.full((BATCH,), CONTEXT, dtype=torch.int32, device=dev)
+        out = torch.empty(BATCH, PREFILL_CHUNK, HQ, D, dtype=torch.float32, device=dev)
+        for _ in range(args.warmup + args.steps):
+            tq.tq_prefill_attention(params, kcb, vcb, kn, vn, q, start, pcache, out, err)
     else:
         tq.tq_quantize_append(params, kcb, vcb, k, v, pos, cache, err)
         q = inputs.queries(BATCH, HQ, D, SEED, device=dev)
@@ -704,7 +771,7 @@ def run_profile_case(args):
     torch.cuda.synchronize()
     st, word = tq.tq_read_device_error(err)
     assert st == tq.TQ_OK, (st, word)
-    print(json.dumps({"profile_case": args.profile, "launches": args.warmup + args.steps + (args.profile != "quantize")}))
+    print(json.dumps({"profile_case": args.profile, "launches": args.warmup + args.steps + (args.profile == "decode")}))
 
 
 def main():
@@ -716,7 +783,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true",
                     help="skip the bf16 baseline and the bulk prefill quantise measurement")
-    ap.add_argument("--profile", choices=["decode", "quantize"], default=None,
+    ap.add_argument("--profile", choices=["decode", "quantize", "prefill"], default=None,
                     help="run a small one-layer case for ncu instead of the benchmark")
     args = ap.parse_args()
     if args.profile:

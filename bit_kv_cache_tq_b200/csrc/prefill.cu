@@ -16,25 +16,39 @@
 //   out = R^-1( sum_i p_i ||v_i|| c[code_i] ).
 //
 // How: one thread block per (sequence, kv head, 128 query rows), a row being
-// one (query token, head of the GQA group).  The rotated query rows, scaled
-// to a largest magnitude of 1, enter as two fp16 terms (the rounded value
-// and its remainder, two MMAs into the same accumulator), so the scores keep
-// about 22 bits of the query.  Per 64-key tile the block
-// dequantises the packed codes into fp16 tiles in shared memory, laid out as
-// the tensor cores read them (K-major, 128-byte swizzle): K~ [64 keys x 128
-// channels] and V~^T [128 channels x 64 keys], centroids only (the norms
-// scale the scores and the softmax weights instead).  One thread issues
-// S = Q~ K~^T (M = 128, N = 64, K = 128) into tensor memory; each thread then
-// owns one query row: it reads its scores from tensor memory, applies the key
-// norms, the causal limit and the online softmax, and writes its weights
-// p_i ||v_i|| (fp16) back as the A operand of O_tile = P V~ (M = 128, N = 128,
-// K = 64), whose tensor-memory result it adds to its fp32 row accumulator.
-// The end divides by the softmax sum and applies the inverse rotation.  The
-// keys' fp16 centroids carry the codebook's fp16 scale (as in the decode
-// kernels), removed from the scores and the output.
+// one (query token, head of the GQA group), in warp-specialised roles that
+// overlap every stage of a 64-key tile with the tensor cores' work on others:
+//  * a producer thread bulk-copies each tile's packed codes and norms (1-D
+//    TMA copies, no multicast) into a ring of four stages;
+//  * four dequantising warps turn a stage into fp16 operand tiles in shared
+//    memory, laid out as the tensor cores read them (K-major, 128-byte
+//    swizzle), double-buffered, through tables that map a byte of codes to
+//    fp16 centroid pairs: K~ [64 keys x 128 channels], the centroids (the key
+//    norms multiply the fp32 scores instead: an fp16 product per element
+//    would add a rounding error that the exponential amplifies with the
+//    score), and V~ [64 keys x 128 channels], the centroids, in the same
+//    per-key layout, which the P V~ product reads as an MN-major operand;
+//    the tile's key and value norms go to small rings the softmax reads;
+//  * one thread issues the tcgen05 MMAs: S = (Q~hi + Q~lo) K~^T (M = 128,
+//    N = 64, K = 128, into one of two tensor-memory score buffers) for tile
+//    j + 1 before O += P V~ (M = 128, N = 128, K = 64, accumulated across
+//    tiles in tensor memory) for tile j, and signals completions through
+//    tcgen05.commit on mbarriers;
+//  * four softmax warps own one query row per thread: they rotate and stage
+//    the queries (two fp16 terms, rows scaled to a largest magnitude of 1, so
+//    the scores keep about 22 bits), then per tile read their scores from
+//    tensor memory, apply the causal limit and the online softmax with a lazy
+//    reference (the accumulator in tensor memory is rescaled only when a
+//    score passes the reference by more than 2^8), and write the weights
+//    times the value norms (scaled by 2^-8: with the reference headroom of
+//    2^8 no weight can leave the fp16 range) as the A operand of P V~.  The
+//    end divides by the softmax sum and applies the inverse rotation.
+// The keys' and values' fp16 centroids carry the codebook's fp16 scale (as in
+// the decode kernels), removed from the scores and the output.
 //
-// Every mbarrier wait is bounded (about a second; TQ_DEVERR_TIMEOUT, the
-// block stops issuing work and still frees its tensor memory).
+// Every mbarrier wait is bounded (about a second, then TQ_DEVERR_TIMEOUT; the
+// block stops issuing work, waits for its copies and MMAs, and frees its
+// tensor memory).
 
 #include <cuda_runtime.h>
 
@@ -51,27 +65,44 @@ namespace prefill {
 constexpr int D = 128;
 constexpr int BM = 128;                  // query rows per block
 constexpr int BK = 64;                   // keys per tile
-constexpr int NTHREADS = 128;            // one thread per query row
-constexpr uint32_t TMEM_COLS = 256;      // S at column 0 (64 columns), O at column 128 (128 columns)
-constexpr uint32_t TMEM_S = 0, TMEM_O = 128;
+constexpr int NS = 4;                    // code stages
+constexpr int SOFTMAX_WARPS = 4, DEQ_WARPS = 8;
+constexpr int DEQ0 = SOFTMAX_WARPS * 32;           // first dequantising thread
+constexpr int PRODUCER = DEQ0 + DEQ_WARPS * 32;    // producer thread (lane 0 of its warp)
+constexpr int MMA_WARP = PRODUCER / 32 + 1;        // MMA issuer warp (also allocates tensor memory)
+constexpr int NTHREADS = (MMA_WARP + 1) * 32;
+constexpr uint32_t TMEM_COLS = 256;      // S buffers at columns 0 and 64, O at 128
+constexpr uint32_t TMEM_O = 128;
 constexpr long long WAIT_LIMIT = 2000000000ll;  // clock cycles (~1 s)
+constexpr float NORM_FOLD = 1.0f / 256.0f;      // value norms enter the fp16 weights scaled by 2^-8
+constexpr float LAZY = 8.0f;                    // log2 headroom before the reference moves
 
 // shared-memory map (offsets from a 1024-byte aligned base)
-constexpr uint32_t SM_Q = 0;                     // fp16 [128 rows][128 ch], 2 column blocks of 16 KB
-constexpr uint32_t SM_QLO = SM_Q + BM * D * 2;   // fp16 remainder q~ - fp16(q~), same layout
-constexpr uint32_t SM_K = SM_QLO + BM * D * 2;   // fp16 [64 keys][128 ch], 2 column blocks of 8 KB
-constexpr uint32_t SM_VT = SM_K + BK * D * 2;    // fp16 [128 ch][64 keys], 1 column block
-constexpr uint32_t SM_P = SM_VT + D * BK * 2;    // fp16 [128 rows][64 keys], 1 column block
-constexpr uint32_t SM_KC = SM_P + BM * BK * 2;   // packed key codes of the tile [64][16 kb]
-constexpr uint32_t SM_VC = SM_KC + BK * 64;      // packed value codes of the tile [64][16 vb]
-constexpr uint32_t SM_KN = SM_VC + BK * 64;      // float key norms [64]
-constexpr uint32_t SM_VN = SM_KN + BK * 4;       // float value norms [64]
-constexpr uint32_t SM_CENT = SM_VN + BK * 4;     // fp16 key centroids [16], value centroids [16]
-constexpr uint32_t SM_BAR = SM_CENT + 64;        // mbarrier
-constexpr uint32_t SM_TMEM = SM_BAR + 8;         // tensor-memory address
-constexpr uint32_t SM_FLAG = SM_TMEM + 4;        // abort flag
+constexpr uint32_t SM_Q = 0;                       // fp16 [128 rows][128 ch], 2 column blocks of 16 KB
+constexpr uint32_t SM_QLO = SM_Q + BM * D * 2;     // fp16 remainder q~ - fp16(q~), same layout
+constexpr uint32_t SM_K = SM_QLO + BM * D * 2;     // 2 x fp16 [64 keys][128 ch] (2 column blocks of 8 KB each)
+constexpr uint32_t SM_VT = SM_K + 2 * BK * D * 2;  // 2 x fp16 V~ [64 keys][128 ch], the layout of K~
+constexpr uint32_t SM_P = SM_VT + 2 * D * BK * 2;  // 2 x fp16 [128 rows][64 keys]
+constexpr uint32_t STAGE_BYTES = BK * 64 + BK * 64 + BK * 2 + BK * 2;  // K codes, V codes, K norms, V norms
+constexpr uint32_t ST_KC = 0, ST_VC = BK * 64, ST_KN = 2 * BK * 64, ST_VN = 2 * BK * 64 + BK * 2;
+constexpr uint32_t SM_STAGE = SM_P + 2 * BM * BK * 2;
+constexpr uint32_t SM_KNR = SM_STAGE + NS * STAGE_BYTES;   // fp32 key norms of the last four tiles [4][64]
+constexpr uint32_t SM_VNR = SM_KNR + 4 * BK * 4;           // fp32 value norms x 2^-8 of the last four tiles [4][64]
+constexpr uint32_t SM_CENT = SM_VNR + 4 * BK * 4;          // fp16 key centroids [16], value centroids [16]
+constexpr uint32_t SM_KLUT = SM_CENT + 64;                 // byte of key codes -> fp16 centroids (2 KB)
+constexpr uint32_t SM_VLUT = SM_KLUT + 2048;               // byte of value codes -> fp16 centroids (2 KB)
+constexpr uint32_t SM_BAR = SM_VLUT + 2048;
+// mbarriers (8 bytes each)
+constexpr int B_FULL = 0, B_EMPTY = NS, B_KFULL = 2 * NS, B_KEMPTY = B_KFULL + 2, B_VFULL = B_KEMPTY + 2,
+              B_VEMPTY = B_VFULL + 2, B_SFULL = B_VEMPTY + 2, B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2,
+              B_PEMPTY = B_PFULL + 2, B_QREADY = B_PEMPTY + 2, B_FINAL = B_QREADY + 1, NBARS = B_FINAL + 1;
+// (B_PEMPTY[j % 2] also tells that every P V up to tile j is in the accumulator:
+// commits complete in order.  Waiting on it rather than on one shared
+// barrier keeps every wait within one phase of the barrier's state.)
+constexpr uint32_t SM_TMEM = SM_BAR + NBARS * 8;   // tensor-memory address
+constexpr uint32_t SM_FLAG = SM_TMEM + 4;          // abort flag
 constexpr uint32_t SM_BYTES = SM_FLAG + 4;
-constexpr uint32_t SM_ALLOC = SM_BYTES + 1024;   // room to align the base
+constexpr uint32_t SM_ALLOC = SM_BYTES + 1024;     // room to align the base
 
 struct Args {
     const uint8_t* k_codes;
@@ -82,9 +113,10 @@ struct Args {
     const int32_t* positions;
     float* out;              // [batch][n_new][hq][d]
     uint32_t* err;
-    int q_dtype, batch, hq, hkv, group, capacity, n_new, tok_per_tile, kb, vb;
+    int q_dtype, batch, hq, hkv, group, capacity, n_new, tok_per_tile;
+    int staged_norms;        // capacity % 8 == 0: norms ride in the bulk copies
     float score_scale;       // sm_scale * log2(e) / alpha_k
-    float inv_alpha_v;
+    float out_scale;         // 1 / (alpha_v * NORM_FOLD)
     uint32_t signs[4];
     uint16_t kcent[16];      // fp16 bits of alpha_k * key centroid
     uint16_t vcent[16];
@@ -106,293 +138,483 @@ __device__ __forceinline__ void fwht128(float (&x)[D]) {
 
 __device__ __forceinline__ uint32_t pack2(uint16_t lo, uint16_t hi) { return lo | (static_cast<uint32_t>(hi) << 16); }
 
-// code `i` of a packed row (LSB-first bitstream of `bits`-bit codes) held in
-// shared memory as 32-bit words
-__device__ __forceinline__ uint32_t code_at(const uint32_t* row, int i, int bits) {
-    const int bit = bits * i;
-    const uint32_t lo = row[bit >> 5];
-    const int sh = bit & 31;
-    uint32_t v = lo >> sh;
-    if (sh + bits > 32) v |= row[(bit >> 5) + 1] << (32 - sh);
-    return v & ((1u << bits) - 1u);
+// two fp16 bit patterns times an fp16 pair, as one fp16 pair
+__device__ __forceinline__ uint32_t hmul_pair(uint16_t lo, uint16_t hi, __half2 f) {
+    const __half2 c = __halves2half2(__ushort_as_half(lo), __ushort_as_half(hi));
+    const __half2 r = __hmul2(c, f);
+    return *reinterpret_cast<const uint32_t*>(&r);
 }
 
+struct Block {
+    int qt, kv, b, tok0, ntok, start, kend, ntiles;
+    bool bad;
+};
+
+// The 8 codes of channels 8 cg .. 8 cg + 7 of a packed row (KB bits each,
+// LSB-first) as one word, code e in bits [KB e, KB e + KB).
+template <int KB>
+__device__ __forceinline__ uint32_t eight_codes(const uint32_t* row, int cg) {
+    const int bit = 8 * KB * cg;
+    if constexpr (KB == 4) return row[cg];
+    if constexpr (KB == 2) return row[cg >> 1] >> (16 * (cg & 1));
+    const int w = bit >> 5, sh = bit & 31;  // 24 bits: may straddle two words
+    const uint32_t lo = row[w];
+    return sh <= 8 ? lo >> sh : __funnelshift_r(lo, row[w + 1], sh);
+}
+
+// Code tables: an index of codes -> their fp16 centroids, packed.  KB = 4: a
+// byte (2 codes) -> one pair; KB = 3: 6 bits (2 codes) -> one pair; KB = 2: a
+// byte (4 codes) -> two pairs.
+template <int BITS>
+__device__ void build_lut(uint32_t* lut, const uint16_t* cent, int t, int nthreads) {
+    if constexpr (BITS == 2) {
+        for (int e = t; e < 256; e += nthreads) {
+            lut[2 * e] = pack2(cent[e & 3], cent[(e >> 2) & 3]);
+            lut[2 * e + 1] = pack2(cent[(e >> 4) & 3], cent[e >> 6]);
+        }
+    } else {
+        constexpr int n = 1 << (2 * BITS), m = (1 << BITS) - 1;
+        for (int e = t; e < n; e += nthreads) lut[e] = pack2(cent[e & m], cent[e >> BITS]);
+    }
+}
+
+// fp16 centroids of 8 codes (channel order) through the table, as 4 pairs.
+template <int BITS>
+__device__ __forceinline__ uint4 dequant8(uint32_t c8, const uint32_t* lut) {
+    if constexpr (BITS == 4) {
+        return make_uint4(lut[c8 & 0xFFu], lut[(c8 >> 8) & 0xFFu], lut[(c8 >> 16) & 0xFFu], lut[c8 >> 24]);
+    } else if constexpr (BITS == 2) {
+        const uint2 a = reinterpret_cast<const uint2*>(lut)[c8 & 0xFFu];
+        const uint2 b = reinterpret_cast<const uint2*>(lut)[(c8 >> 8) & 0xFFu];
+        return make_uint4(a.x, a.y, b.x, b.y);
+    } else {
+        return make_uint4(lut[c8 & 63u], lut[(c8 >> 6) & 63u], lut[(c8 >> 12) & 63u], lut[(c8 >> 18) & 63u]);
+    }
+}
+
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t x, __half2 f) {
+    const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&x), f);
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+template <int KB, int VB>
 __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_constant__ Args a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = ptx::smem_addr(smem);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int qt = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
-    const int G = a.group, TT = a.tok_per_tile;
-    const int tok0 = qt * TT;
-    const uint32_t bar = sbase + SM_BAR;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t bars = sbase + SM_BAR;
+    auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM_FLAG);
+    auto fail = [&]() {
+        if (!*abort_flag && a.err) atomicOr(a.err, TQ_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+    };
+    // bounded wait on phase `parity` of mbarrier i; false (and the abort flag set) when it runs out
+    auto wait = [&](int i, uint32_t parity) -> bool {
+        if (*abort_flag) return false;
+        if (!ptx::mbar_wait_bounded(bar(i), parity, WAIT_LIMIT)) {
+            fail();
+            return false;
+        }
+        return true;
+    };
+
+    Block blk;
+    blk.qt = blockIdx.x;
+    blk.kv = blockIdx.y;
+    blk.b = blockIdx.z;
+    const int G = a.group, TT = a.tok_per_tile;
+    blk.tok0 = blk.qt * TT;
+    blk.start = a.positions[blk.b];
+    blk.bad = blk.start < 0 || blk.start > a.capacity - a.n_new;
+    blk.ntok = blk.bad ? 0 : min(TT, a.n_new - blk.tok0);
+    blk.kend = blk.ntok > 0 ? blk.start + blk.tok0 + blk.ntok : 0;  // keys [0, kend) are needed by some row
+    blk.ntiles = (blk.kend + BK - 1) / BK;
+    const int T = blk.ntiles;
 
     if (tid == 0) {
-        ptx::mbar_init(bar, 1);
+        for (int i = 0; i < NS; ++i) {
+            ptx::mbar_init(bar(B_FULL + i), 1);
+            ptx::mbar_init(bar(B_EMPTY + i), DEQ_WARPS);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(bar(B_KFULL + i), DEQ_WARPS);
+            ptx::mbar_init(bar(B_KEMPTY + i), 1);
+            ptx::mbar_init(bar(B_VFULL + i), DEQ_WARPS);
+            ptx::mbar_init(bar(B_VEMPTY + i), 1);
+            ptx::mbar_init(bar(B_SFULL + i), 1);
+            ptx::mbar_init(bar(B_SEMPTY + i), SOFTMAX_WARPS);
+            ptx::mbar_init(bar(B_PFULL + i), SOFTMAX_WARPS);
+            ptx::mbar_init(bar(B_PEMPTY + i), 1);
+        }
+        ptx::mbar_init(bar(B_QREADY), SOFTMAX_WARPS);
+        ptx::mbar_init(bar(B_FINAL), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    if (tid < 32) {
-        reinterpret_cast<uint16_t*>(smem + SM_CENT)[tid] = tid < 16 ? a.kcent[tid] : a.vcent[tid - 16];
-    }
-    if (warp == 0) {
+    if (tid < 32) reinterpret_cast<uint16_t*>(smem + SM_CENT)[tid] = tid < 16 ? a.kcent[tid] : a.vcent[tid - 16];
+    if (warp == MMA_WARP) {
         tc::tmem_alloc(sbase + SM_TMEM, TMEM_COLS);
         tc::tmem_relinquish();
     }
+    if (blk.bad && blk.qt == 0 && blk.kv == 0 && tid == 0 && a.err) atomicOr(a.err, TQ_DEVERR_POSITION);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + SM_TMEM);
-    const uint16_t* kcent = reinterpret_cast<const uint16_t*>(smem + SM_CENT);
-    const uint16_t* vcent = kcent + 16;
+    const size_t unit_row = (static_cast<size_t>(blk.b) * a.hkv + blk.kv) * a.capacity;
+    // the code tables, built by the dequantising warps (they alone read them;
+    // a named barrier among them publishes the tables)
+    constexpr int kbytes = 16 * KB, vbytes = 16 * VB;  // packed row sizes
 
-    // the chunk's first cache slot; an out-of-range start gives zeros
-    const int start = a.positions[b];
-    const bool bad = start < 0 || start > a.capacity - a.n_new;
-    if (bad && qt == 0 && kv == 0 && tid == 0 && a.err) atomicOr(a.err, TQ_DEVERR_POSITION);
-    const int ntok = bad ? 0 : min(TT, a.n_new - tok0);  // query tokens of this block
-
-    // ---- this thread's query row: token tok0 + r / G, head kv * G + r % G
-    const int r = tid;
-    const int rt = r / G, rh = r % G;
-    const bool row_ok = rt < ntok && rt * G + rh < BM;
-    float qscale = 0.f;  // largest |q~| of the row: the fp16 terms hold q~ / qscale
-    {
-        float x[D];
-        if (row_ok) {
-            const size_t qoff = ((static_cast<size_t>(b) * a.n_new + tok0 + rt) * a.hq + kv * G + rh) * D;
-#pragma unroll
-            for (int c = 0; c < D; c += 4) {
-                float v4[4];
-                load4(a.q, qoff + c, a.q_dtype, v4);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) x[c + e] = flip_sign(v4[e], (a.signs[(c + e) >> 5] >> ((c + e) & 31)) & 1u);
+    if (tid == PRODUCER) {
+        // ---------------------------------------------------------- producer
+        int issued = 0;
+        for (int j = 0; j < T; ++j) {
+            const int s = j % NS;
+            if (j >= NS && !wait(B_EMPTY + s, ((j - NS) / NS) & 1)) break;
+            const int key0 = j * BK, nk = min(BK, blk.kend - key0);
+            const uint32_t dst = sbase + SM_STAGE + s * STAGE_BYTES;
+            const int n8 = (nk + 7) & ~7;  // norms move in 16-byte pieces (8 keys)
+            const uint32_t bytes = nk * (kbytes + vbytes) + (a.staged_norms ? n8 * 4 : 0);
+            ptx::mbar_arrive_expect_tx(bar(B_FULL + s), bytes);
+            ptx::bulk_copy_g2s(dst + ST_KC, a.k_codes + (unit_row + key0) * kbytes, nk * kbytes, bar(B_FULL + s));
+            ptx::bulk_copy_g2s(dst + ST_VC, a.v_codes + (unit_row + key0) * vbytes, nk * vbytes, bar(B_FULL + s));
+            if (a.staged_norms) {
+                // capacity and key0 are multiples of 8: the rounded range stays inside the cache
+                ptx::bulk_copy_g2s(dst + ST_KN, a.k_norms + unit_row + key0, n8 * 2, bar(B_FULL + s));
+                ptx::bulk_copy_g2s(dst + ST_VN, a.v_norms + unit_row + key0, n8 * 2, bar(B_FULL + s));
             }
-            fwht128(x);
-        } else {
-#pragma unroll
-            for (int c = 0; c < D; ++c) x[c] = 0.f;
+            issued = j + 1;
         }
-        float amax = 0.f;
-#pragma unroll
-        for (int c = 0; c < D; ++c) amax = fmaxf(amax, fabsf(x[c]));
-        const float inv_sqrt_d = 0.08838834764831845f;
-        qscale = amax * inv_sqrt_d;
-        const float rs = amax > 0.f ? 1.f / amax : 0.f;
-#pragma unroll
-        for (int c = 0; c < D; c += 8) {
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float u0 = x[c + 2 * e] * rs, u1 = x[c + 2 * e + 1] * rs;
-                const __half h0 = __float2half_rn(u0), h1 = __float2half_rn(u1);
-                hw[e] = pack2(__half_as_ushort(h0), __half_as_ushort(h1));
-                lw[e] = pack2(__half_as_ushort(__float2half_rn(u0 - __half2float(h0))),
-                              __half_as_ushort(__float2half_rn(u1 - __half2float(h1))));
+        // every copy issued must land before the block may exit
+        for (int j = max(0, issued - NS); j < issued; ++j)
+            ptx::mbar_wait_bounded(bar(B_FULL + j % NS), (j / NS) & 1, WAIT_LIMIT);
+    } else if (warp >= DEQ0 / 32 && warp < PRODUCER / 32) {
+        // ------------------------------------------------------ dequantisers
+        const int dt = tid - DEQ0;  // 0 .. 127
+        const uint16_t* kcent = reinterpret_cast<const uint16_t*>(smem + SM_CENT);
+        const uint16_t* vcent = kcent + 16;
+        uint32_t* klut = reinterpret_cast<uint32_t*>(smem + SM_KLUT);
+        uint32_t* vlut = reinterpret_cast<uint32_t*>(smem + SM_VLUT);
+        build_lut<KB>(klut, kcent, dt, DEQ_WARPS * 32);
+        build_lut<VB>(vlut, vcent, dt, DEQ_WARPS * 32);
+        ptx::named_barrier(1, DEQ_WARPS * 32);
+        for (int j = 0; j < T; ++j) {
+            const int s = j % NS, bf = j & 1;
+            if (!wait(B_FULL + s, (j / NS) & 1)) break;
+            const uint8_t* st = smem + SM_STAGE + s * STAGE_BYTES;
+            const int key0 = j * BK, nk = min(BK, blk.kend - key0);
+            const uint16_t* skn = reinterpret_cast<const uint16_t*>(st + ST_KN);
+            const uint16_t* svn = reinterpret_cast<const uint16_t*>(st + ST_VN);
+            auto knorm = [&](int key) -> float {
+                if (key >= nk) return 0.f;
+                return half_bits_to_float(a.staged_norms ? skn[key] : a.k_norms[unit_row + key0 + key]);
+            };
+            auto vnorm = [&](int key) -> float {
+                if (key >= nk) return 0.f;
+                return half_bits_to_float(a.staged_norms ? svn[key] : a.v_norms[unit_row + key0 + key]);
+            };
+            // K~[bf]: 64 keys x 16 groups of 8 channels, centroids; the tile's
+            // key and value norms go to the softmax's rings (its tile j - 4 is
+            // done: this tile's K~ buffer was free only after S(j - 2), which
+            // needed the softmax to be through tile j - 4)
+            if (j >= 2 && !wait(B_KEMPTY + bf, ((j - 2) >> 1) & 1)) break;
+            if (dt < BK) {
+                reinterpret_cast<float*>(smem + SM_KNR)[(j & 3) * BK + dt] = knorm(dt);
+                reinterpret_cast<float*>(smem + SM_VNR)[(j & 3) * BK + dt] = vnorm(dt) * NORM_FOLD;
             }
-            *reinterpret_cast<uint4*>(smem + SM_Q + tc::sw128_offset(r, c, BM)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            *reinterpret_cast<uint4*>(smem + SM_QLO + tc::sw128_offset(r, c, BM)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        }
-    }
-    const float row_scale = qscale * a.score_scale;  // scores: S * ||k|| * row_scale (log2 units)
-    const int qpos = start + tok0 + rt;                       // this row's own position: the causal limit
-    const int kend = ntok > 0 ? start + tok0 + ntok : 0;      // keys [0, kend) are needed by some row
-    const int ntiles = (kend + BK - 1) / BK;
-    const int kbytes = 16 * a.kb, vbytes = 16 * a.vb;         // packed row sizes
-    const size_t unit_row = (static_cast<size_t>(b) * a.hkv + kv) * a.capacity;
-
-    float o[D];
-#pragma unroll
-    for (int c = 0; c < D; ++c) o[c] = 0.f;
-    float m = -INFINITY, l = 0.f;
-    uint32_t phase = 0;
-    const uint32_t idesc_s = tc::idesc_f16(BM, BK), idesc_o = tc::idesc_f16(BM, D);
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-
-    for (int tile = 0; tile < ntiles; ++tile) {
-        const int key0 = tile * BK;
-        const int nk = min(BK, kend - key0);  // keys of this tile below kend (all within the cache)
-        // ---- stage the tile's packed codes and norms (coalesced 16-byte loads)
-        {
-            const uint4* ksrc = reinterpret_cast<const uint4*>(a.k_codes + (unit_row + key0) * kbytes);
-            const uint4* vsrc = reinterpret_cast<const uint4*>(a.v_codes + (unit_row + key0) * vbytes);
-            uint4* kdst = reinterpret_cast<uint4*>(smem + SM_KC);
-            uint4* vdst = reinterpret_cast<uint4*>(smem + SM_VC);
-            const int kwords = nk * kbytes / 16, vwords = nk * vbytes / 16;
-            for (int i = tid; i < kwords; i += NTHREADS) kdst[i] = ksrc[i];
-            for (int i = tid; i < vwords; i += NTHREADS) vdst[i] = vsrc[i];
-            if (tid < BK) {
-                float* kn = reinterpret_cast<float*>(smem + SM_KN);
-                float* vn = reinterpret_cast<float*>(smem + SM_VN);
-                kn[tid] = tid < nk ? half_bits_to_float(a.k_norms[unit_row + key0 + tid]) : 0.f;
-                vn[tid] = tid < nk ? half_bits_to_float(a.v_norms[unit_row + key0 + tid]) : 0.f;
+            uint8_t* kt = smem + SM_K + bf * (BK * D * 2);
+#pragma unroll 4
+            for (int it = dt; it < BK * (D / 8); it += DEQ_WARPS * 32) {
+                const int key = it >> 4, cg = it & 15;
+                uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                if (key < nk)
+                    w = dequant8<KB>(eight_codes<KB>(reinterpret_cast<const uint32_t*>(st + ST_KC + key * kbytes), cg),
+                                     klut);
+                *reinterpret_cast<uint4*>(kt + tc::sw128_offset(key, 8 * cg, BK)) = w;
+            }
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(B_KFULL + bf));
+            // V~[bf]: the same per-key layout, centroids
+            if (j >= 2 && !wait(B_VEMPTY + bf, ((j - 2) >> 1) & 1)) break;
+            uint8_t* vt = smem + SM_VT + bf * (BK * D * 2);
+#pragma unroll 4
+            for (int it = dt; it < BK * (D / 8); it += DEQ_WARPS * 32) {
+                const int key = it >> 4, cg = it & 15;
+                uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                if (key < nk)
+                    w = dequant8<VB>(eight_codes<VB>(reinterpret_cast<const uint32_t*>(st + ST_VC + key * vbytes), cg),
+                                     vlut);
+                *reinterpret_cast<uint4*>(vt + tc::sw128_offset(key, 8 * cg, BK)) = w;
+            }
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(bar(B_VFULL + bf));
+                ptx::mbar_arrive(bar(B_EMPTY + s));  // the stage's codes and norms are used
             }
         }
-        __syncthreads();
-        // ---- dequantise: K~ [64 keys][128 ch] and V~^T [128 ch][64 keys]
-        for (int it = tid; it < BK * (D / 8); it += NTHREADS) {
-            const int key = it / (D / 8), cg = it % (D / 8);  // 8 channels 8 cg .. 8 cg + 7
-            uint4 w = make_uint4(0u, 0u, 0u, 0u);
-            if (key < nk) {
-                const uint32_t* row = reinterpret_cast<const uint32_t*>(smem + SM_KC + key * kbytes);
-                uint16_t h[8];
+    } else if (warp == MMA_WARP) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = tc::idesc_f16(BM, BK), idesc_o = tc::idesc_f16_bmn(BM, D);
+            bool ok = T == 0 || wait(B_QREADY, 0);
+            auto issue_s = [&](int j) -> bool {
+                const int bf = j & 1;
+                if (!wait(B_KFULL + bf, (j >> 1) & 1)) return false;
+                if (j >= 2 && !wait(B_SEMPTY + bf, ((j - 2) >> 1) & 1)) return false;
+                tc::fence_after_sync();
+                const uint32_t kt = sbase + SM_K + bf * (BK * D * 2);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) h[e] = kcent[code_at(row, 8 * cg + e, a.kb)];
-                w = make_uint4(pack2(h[0], h[1]), pack2(h[2], h[3]), pack2(h[4], h[5]), pack2(h[6], h[7]));
-            }
-            *reinterpret_cast<uint4*>(smem + SM_K + tc::sw128_offset(key, 8 * cg, BK)) = w;
-        }
-        for (int it = tid; it < D * (BK / 8); it += NTHREADS) {
-            const int ch = it % D, kg = it / D;  // channel ch of keys 8 kg .. 8 kg + 7
-            uint16_t h[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int key = 8 * kg + e;
-                h[e] = 0;
-                if (key < nk) {
-                    const uint32_t* row = reinterpret_cast<const uint32_t*>(smem + SM_VC + key * vbytes);
-                    h[e] = vcent[code_at(row, ch, a.vb)];
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t cb = ks >> 2, within = (ks & 3) * 32;
+                    const uint64_t bd = tc::sw128_desc(kt + cb * (BK * 128) + within);
+                    tc::mma_f16(tmem + BK * bf, tc::sw128_desc(sbase + SM_Q + cb * (BM * 128) + within), bd, idesc_s,
+                                ks > 0);
+                    tc::mma_f16(tmem + BK * bf, tc::sw128_desc(sbase + SM_QLO + cb * (BM * 128) + within), bd,
+                                idesc_s, true);
                 }
+                tc::commit(bar(B_SFULL + bf));
+                tc::commit(bar(B_KEMPTY + bf));
+                return true;
+            };
+            auto issue_pv = [&](int j) -> bool {
+                const int bf = j & 1;
+                if (!wait(B_PFULL + bf, (j >> 1) & 1)) return false;
+                if (!wait(B_VFULL + bf, (j >> 1) & 1)) return false;
+                tc::fence_after_sync();
+                const uint32_t pt = sbase + SM_P + bf * (BM * BK * 2), vt = sbase + SM_VT + bf * (BK * D * 2);
+                // V~ [64 keys][128 ch]: 16 keys per step = two 1024-byte K groups;
+                // the two 64-channel blocks lie 64 rows x 128 bytes apart
+#pragma unroll
+                for (int ks = 0; ks < BK / 16; ++ks)
+                    tc::mma_f16(tmem + TMEM_O, tc::sw128_desc(pt + ks * 32),
+                                tc::sw128_mn_desc(vt + ks * 2048, BK * 128, 1024), idesc_o, j > 0 || ks > 0);
+                tc::commit(bar(B_PEMPTY + bf));
+                tc::commit(bar(B_VEMPTY + bf));
+                return true;
+            };
+            if (ok && T > 0) ok = issue_s(0);
+            for (int j = 0; ok && j < T; ++j) {
+                if (j + 1 < T && !issue_s(j + 1)) break;
+                if (!issue_pv(j)) break;
             }
-            const uint4 w = make_uint4(pack2(h[0], h[1]), pack2(h[2], h[3]), pack2(h[4], h[5]), pack2(h[6], h[7]));
-            *reinterpret_cast<uint4*>(smem + SM_VT + tc::sw128_offset(ch, 8 * kg, D)) = w;
+            // every tensor-core operation issued completes before the block
+            // frees its tensor memory (bounded, also after an abort)
+            tc::commit(bar(B_FINAL));
+            ptx::mbar_wait_bounded(bar(B_FINAL), 0, WAIT_LIMIT);
+        }
+        __syncwarp();
+    } else if (warp < SOFTMAX_WARPS) {
+        // ---------------------------------------------------------- softmax
+        const int r = tid;
+        const int rt = r / G, rh = r % G;
+        const bool row_ok = rt < blk.ntok && rt * G + rh < BM;
+        float qscale = 0.f;  // largest |q~| of the row: the fp16 terms hold q~ / qscale
+        {
+            float x[D];
+            if (row_ok) {
+                const size_t qoff = ((static_cast<size_t>(blk.b) * a.n_new + blk.tok0 + rt) * a.hq + blk.kv * G + rh) * D;
+#pragma unroll
+                for (int c = 0; c < D; c += 4) {
+                    float v4[4];
+                    load4(a.q, qoff + c, a.q_dtype, v4);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        x[c + e] = flip_sign(v4[e], (a.signs[(c + e) >> 5] >> ((c + e) & 31)) & 1u);
+                }
+                fwht128(x);
+            } else {
+#pragma unroll
+                for (int c = 0; c < D; ++c) x[c] = 0.f;
+            }
+            float amax = 0.f;
+#pragma unroll
+            for (int c = 0; c < D; ++c) amax = fmaxf(amax, fabsf(x[c]));
+            const float inv_sqrt_d = 0.08838834764831845f;
+            qscale = amax * inv_sqrt_d;
+            const float rs = amax > 0.f ? 1.f / amax : 0.f;
+#pragma unroll
+            for (int c = 0; c < D; c += 8) {
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float u0 = x[c + 2 * e] * rs, u1 = x[c + 2 * e + 1] * rs;
+                    const __half h0 = __float2half_rn(u0), h1 = __float2half_rn(u1);
+                    hw[e] = pack2(__half_as_ushort(h0), __half_as_ushort(h1));
+                    lw[e] = pack2(__half_as_ushort(__float2half_rn(u0 - __half2float(h0))),
+                                  __half_as_ushort(__float2half_rn(u1 - __half2float(h1))));
+                }
+                *reinterpret_cast<uint4*>(smem + SM_Q + tc::sw128_offset(r, c, BM)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4*>(smem + SM_QLO + tc::sw128_offset(r, c, BM)) =
+                    make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
         }
         tc::fence_proxy_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-        tc::fence_after_sync();
-        // ---- S = (Q~hi + Q~lo) K~^T
-        if (tid == 0 && !*abort_flag) {
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const uint32_t blk = ks >> 2, within = (ks & 3) * 32;
-                const uint64_t bd = tc::sw128_desc(sbase + SM_K + blk * (BK * 128) + within);
-                tc::mma_f16(tmem + TMEM_S, tc::sw128_desc(sbase + SM_Q + blk * (BM * 128) + within), bd, idesc_s,
-                            ks > 0);
-                tc::mma_f16(tmem + TMEM_S, tc::sw128_desc(sbase + SM_QLO + blk * (BM * 128) + within), bd, idesc_s,
-                            true);
-            }
-            tc::commit(bar);
-        }
-        if (!*abort_flag && !ptx::mbar_wait_bounded(bar, phase & 1, WAIT_LIMIT)) {
-            if (a.err) atomicOr(a.err, TQ_DEVERR_TIMEOUT);
-            *abort_flag = 1;
-        }
-        ++phase;
-        tc::fence_after_sync();
-        // ---- online softmax of this row over the tile: one pass over the
-        // scores in tensor memory for the maximum, a second one for the
-        // weights (rereading tensor memory is cheaper than holding 64 scores)
-        {
-            float sv[32];
-            const float* kn = reinterpret_cast<const float*>(smem + SM_KN);
-            const float* vn = reinterpret_cast<const float*>(smem + SM_VN);
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(B_QREADY));
+        const float row_scale = qscale * a.score_scale;  // scores: S * row_scale, log2 units
+        const int qpos = blk.start + blk.tok0 + rt;      // this row's own position: the causal limit
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        float mref = -INFINITY, l = 0.f;
+        for (int j = 0; j < T; ++j) {
+            const int bf = j & 1, key0 = j * BK;
+            if (!wait(B_SFULL + bf, (j >> 1) & 1)) break;
+            tc::fence_after_sync();
+            float sv[2][32];
             float mt = -INFINITY;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tc::ld_32cols(tmem + lane_base + TMEM_S + 32 * half, sv);
-                tc::ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int key = key0 + 32 * half + j;
-                    if (row_ok && key <= qpos) mt = fmaxf(mt, sv[j] * kn[32 * half + j] * row_scale);
-                }
+            for (int h = 0; h < 2; ++h) {
+                tc::ld_32cols(tmem + lane_base + BK * bf + 32 * h, sv[h]);
             }
-            const float mn = fmaxf(m, mt);
-            const float corr = (m == -INFINITY) ? 0.f : ptx::ex2(m - mn);
+            tc::ld_wait();
+            const float* kn = reinterpret_cast<const float*>(smem + SM_KNR) + (j & 3) * BK;
+            if (key0 + BK - 1 <= blk.start + blk.tok0) {
+                // every row of the block sees every key of the tile (rows
+                // outside the chunk are never stored, so need no mask)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        sv[h][i] = sv[h][i] * kn[32 * h + i] * row_scale;
+                        mt = fmaxf(mt, sv[h][i]);
+                    }
+            } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int key = key0 + 32 * h + i;
+                        sv[h][i] = (row_ok && key <= qpos) ? sv[h][i] * kn[32 * h + i] * row_scale : -INFINITY;
+                        mt = fmaxf(mt, sv[h][i]);
+                    }
+            }
+            // lazy reference: moves (and the accumulator is rescaled) only when a
+            // score passes it by more than 2^LAZY; the weights stay below 2^LAZY
+            const bool need = mt > mref + LAZY;
+            if (__any_sync(0xffffffffu, need)) {
+                const float mnew = need ? mt : mref;
+                const float c = (need && mref > -INFINITY) ? ptx::ex2(mref - mnew) : 1.f;
+                if (j > 0) {
+                    // every P V of the earlier tiles is in the accumulator
+                    if (!wait(B_PEMPTY + ((j - 1) & 1), ((j - 1) >> 1) & 1)) break;
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        float ov[32];
+                        tc::ld_32cols(tmem + lane_base + TMEM_O + 32 * q4, ov);
+                        tc::ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) ov[i] *= c;
+                        tc::st_32cols(tmem + lane_base + TMEM_O + 32 * q4, ov);
+                    }
+                    tc::st_wait();
+                }
+                l *= c;
+                mref = mnew;
+            }
+            // weights of the tile, fp16, as the A operand of P V~
+            if (j >= 2 && !wait(B_PEMPTY + bf, ((j - 2) >> 1) & 1)) break;
+            uint8_t* pt = smem + SM_P + bf * (BM * BK * 2);
+            const float* vnr = reinterpret_cast<const float*>(smem + SM_VNR) + (j & 3) * BK;
             float ls = 0.f;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tc::ld_32cols(tmem + lane_base + TMEM_S + 32 * half, sv);
-                tc::ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int key = key0 + 32 * half + j;
-                    const float e = (row_ok && key <= qpos) ? ptx::ex2(sv[j] * kn[32 * half + j] * row_scale - mn)
-                                                            : 0.f;
-                    ls += e;
-                    sv[j] = e * vn[32 * half + j];
-                }
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int c = 0; c < 32; c += 8) {
-                    uint4 w;
-                    w.x = pack2(__half_as_ushort(__float2half_rn(sv[c])), __half_as_ushort(__float2half_rn(sv[c + 1])));
-                    w.y = pack2(__half_as_ushort(__float2half_rn(sv[c + 2])), __half_as_ushort(__float2half_rn(sv[c + 3])));
-                    w.z = pack2(__half_as_ushort(__float2half_rn(sv[c + 4])), __half_as_ushort(__float2half_rn(sv[c + 5])));
-                    w.w = pack2(__half_as_ushort(__float2half_rn(sv[c + 6])), __half_as_ushort(__float2half_rn(sv[c + 7])));
-                    *reinterpret_cast<uint4*>(smem + SM_P + tc::sw128_offset(r, 32 * half + c, BM)) = w;
+                    float e8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float pe = mref > -INFINITY ? ptx::ex2(sv[h][c + e] - mref) : 0.f;
+                        ls += pe;
+                        e8[e] = pe * vnr[32 * h + c + e];
+                    }
+                    const __half2 p0 = __floats2half2_rn(e8[0], e8[1]), p1 = __floats2half2_rn(e8[2], e8[3]);
+                    const __half2 p2 = __floats2half2_rn(e8[4], e8[5]), p3 = __floats2half2_rn(e8[6], e8[7]);
+                    *reinterpret_cast<uint4*>(pt + tc::sw128_offset(r, 32 * h + c, BM)) =
+                        make_uint4(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1),
+                                   *reinterpret_cast<const uint32_t*>(&p2), *reinterpret_cast<const uint32_t*>(&p3));
                 }
+            l += ls;
+            tc::fence_proxy_async_smem();
+            tc::fence_before_sync();
+            __syncwarp();
+            // the weights are written and the score buffer, the tile's norms
+            // and any accumulator rescale are done with
+            if (lane == 0) {
+                ptx::mbar_arrive(bar(B_SEMPTY + bf));
+                ptx::mbar_arrive(bar(B_PFULL + bf));
             }
-            l = l * corr + ls;
-            m = mn;
-#pragma unroll
-            for (int c = 0; c < D; ++c) o[c] *= corr;
         }
-        tc::fence_proxy_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
+        // ---- epilogue: wait for the last P V, normalise, inverse rotation
+        const bool done = T > 0 && wait(B_PEMPTY + ((T - 1) & 1), ((T - 1) >> 1) & 1);
         tc::fence_after_sync();
-        // ---- O_tile = P V~
-        if (tid == 0 && !*abort_flag) {
-#pragma unroll
-            for (int ks = 0; ks < BK / 16; ++ks) {
-                const uint64_t ad = tc::sw128_desc(sbase + SM_P + ks * 32);
-                const uint64_t bd = tc::sw128_desc(sbase + SM_VT + ks * 32);
-                tc::mma_f16(tmem + TMEM_O, ad, bd, idesc_o, ks > 0);
-            }
-            tc::commit(bar);
-        }
-        if (!*abort_flag && !ptx::mbar_wait_bounded(bar, phase & 1, WAIT_LIMIT)) {
-            if (a.err) atomicOr(a.err, TQ_DEVERR_TIMEOUT);
-            *abort_flag = 1;
-        }
-        ++phase;
-        tc::fence_after_sync();
-        {
-            float ov[32];
+        float o[D];
+        if (done) {
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
+                float ov[32];
                 tc::ld_32cols(tmem + lane_base + TMEM_O + 32 * q4, ov);
                 tc::ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) o[32 * q4 + j] += ov[j];
+                for (int i = 0; i < 32; ++i) o[32 * q4 + i] = ov[i];
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < D; ++c) o[c] = 0.f;
+        }
+        if (row_ok || (blk.bad && rt < min(TT, a.n_new - blk.tok0) && rt * G + rh < BM)) {
+            const float inv = (done && l > 0.f && !*abort_flag) ? a.out_scale / l : 0.f;
+#pragma unroll
+            for (int c = 0; c < D; ++c) o[c] *= inv;
+            fwht128(o);
+            const float inv_sqrt_d = 0.08838834764831845f;
+            float* dst = a.out + ((static_cast<size_t>(blk.b) * a.n_new + blk.tok0 + rt) * a.hq + blk.kv * G + rh) * D;
+#pragma unroll
+            for (int c = 0; c < D; c += 4) {
+                float4 v;
+                v.x = flip_sign(o[c] * inv_sqrt_d, (a.signs[c >> 5] >> (c & 31)) & 1u);
+                v.y = flip_sign(o[c + 1] * inv_sqrt_d, (a.signs[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u);
+                v.z = flip_sign(o[c + 2] * inv_sqrt_d, (a.signs[(c + 2) >> 5] >> ((c + 2) & 31)) & 1u);
+                v.w = flip_sign(o[c + 3] * inv_sqrt_d, (a.signs[(c + 3) >> 5] >> ((c + 3) & 31)) & 1u);
+                *reinterpret_cast<float4*>(dst + c) = v;
             }
         }
-        // every thread's tensor-memory reads and shared-memory uses of this
-        // tile are done before the next tile's operands and MMAs
-        tc::fence_before_sync();
-        if (__syncthreads_or(*abort_flag)) break;
-        tc::fence_after_sync();
-    }
-
-    // ---- epilogue: normalise, undo the value scale, inverse rotation
-    if (row_ok) {
-        const float inv = l > 0.f ? a.inv_alpha_v / l : 0.f;
-#pragma unroll
-        for (int c = 0; c < D; ++c) o[c] *= inv;
-        fwht128(o);
-        const float inv_sqrt_d = 0.08838834764831845f;
-        float* dst = a.out + ((static_cast<size_t>(b) * a.n_new + tok0 + rt) * a.hq + kv * G + rh) * D;
-#pragma unroll
-        for (int c = 0; c < D; c += 4) {
-            float4 v;
-            v.x = flip_sign(o[c] * inv_sqrt_d, (a.signs[c >> 5] >> (c & 31)) & 1u);
-            v.y = flip_sign(o[c + 1] * inv_sqrt_d, (a.signs[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u);
-            v.z = flip_sign(o[c + 2] * inv_sqrt_d, (a.signs[(c + 2) >> 5] >> ((c + 2) & 31)) & 1u);
-            v.w = flip_sign(o[c + 3] * inv_sqrt_d, (a.signs[(c + 3) >> 5] >> ((c + 3) & 31)) & 1u);
-            *reinterpret_cast<float4*>(dst + c) = v;
-        }
-    } else if (bad && rt < min(TT, a.n_new - tok0) && rt * G + rh < BM) {
-        // out-of-range start: zeros for every row of the block
-        float* dst = a.out + ((static_cast<size_t>(b) * a.n_new + tok0 + rt) * a.hq + kv * G + rh) * D;
-        for (int c = 0; c < D; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == MMA_WARP) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+template <int KB, int VB>
+static cudaError_t launch_typed(const Args& a, dim3 grid, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(SM_ALLOC));
+    if (e != cudaSuccess) return e;
+    prefill_kernel<KB, VB><<<grid, NTHREADS, SM_ALLOC, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int KB>
+static cudaError_t launch_k(int vb, const Args& a, dim3 grid, cudaStream_t s) {
+    switch (vb) {
+        case 2: return launch_typed<KB, 2>(a, grid, s);
+        case 3: return launch_typed<KB, 3>(a, grid, s);
+        default: return launch_typed<KB, 4>(a, grid, s);
+    }
+}
+
+static cudaError_t launch_kb(int kb, int vb, const Args& a, dim3 grid, cudaStream_t s) {
+    switch (kb) {
+        case 2: return launch_k<2>(vb, a, grid, s);
+        case 3: return launch_k<3>(vb, a, grid, s);
+        default: return launch_k<4>(vb, a, grid, s);
     }
 }
 
@@ -443,13 +665,12 @@ extern "C" tq_status tq_prefill_attention(const tq_params* params, const tq_code
     a.capacity = cache->capacity;
     a.n_new = n_new;
     a.tok_per_tile = prefill::BM / a.group;
-    a.kb = p.k_bits;
-    a.vb = p.v_bits;
+    a.staged_norms = (cache->capacity % 8) == 0;
     const double ak = kcb->fp16_scale > 0.0 ? kcb->fp16_scale : std::sqrt(128.0);
     const double av = vcb->fp16_scale > 0.0 ? vcb->fp16_scale : std::sqrt(128.0);
     const float sm = p.sm_scale > 0.0f ? p.sm_scale : 1.0f / std::sqrt(128.0f);
     a.score_scale = static_cast<float>(sm * 1.4426950408889634 / ak);
-    a.inv_alpha_v = static_cast<float>(1.0 / av);
+    a.out_scale = static_cast<float>(1.0 / (av * prefill::NORM_FOLD));
     for (int j = 0; j < 16; ++j) {
         const __half hk = __float2half_rn(j < (1 << p.k_bits) ? static_cast<float>(kcb->centroids[j] * ak) : 0.f);
         const __half hv = __float2half_rn(j < (1 << p.v_bits) ? static_cast<float>(vcb->centroids[j] * av) : 0.f);
@@ -461,9 +682,6 @@ extern "C" tq_status tq_prefill_attention(const tq_params* params, const tq_code
     for (int i = 0; i < 4; ++i) a.signs[i] = words[i];
     const dim3 grid((n_new + a.tok_per_tile - 1) / a.tok_per_tile, p.num_kv_heads, cache->batch);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaFuncSetAttribute(prefill::prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(prefill::SM_ALLOC));
-    if (e != cudaSuccess) return TQ_ERR_CUDA;
-    prefill::prefill_kernel<<<grid, prefill::NTHREADS, prefill::SM_ALLOC, s>>>(a);
-    return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+    const cudaError_t e = prefill::launch_kb(p.k_bits, p.v_bits, a, grid, s);
+    return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }

@@ -45,25 +45,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// As mbar_try_wait, but the thread may be suspended up to `ns` nanoseconds
-// while the phase is still open (it resumes as soon as the phase completes),
-// so a waiting warp leaves its scheduler to the others instead of polling.
-__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(ns)
-        : "memory");
-    return ok != 0;
-}
-
-// Wait for phase `parity` of an mbarrier, giving up after `limit` clock cycles
-// (each try suspends the thread for at most 20 us while the phase is open).
+// Wait for phase `parity` of an mbarrier, giving up after `limit` clock cycles.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long start = clock64();
-    while (!mbar_try_wait_suspend(bar, parity, 20000u)) {
+    while (!mbar_try_wait(bar, parity)) {
         if (clock64() - start > limit) return false;
     }
     return true;

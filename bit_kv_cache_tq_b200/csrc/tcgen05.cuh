@@ -68,6 +68,25 @@ __device__ __forceinline__ void ld_32cols(uint32_t taddr, float (&v)[32]) {
 }
 __device__ __forceinline__ void ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Store 32 consecutive fp32 columns of this thread's tensor-memory lane (the
+// lane layout of ld_32cols).  Wait with st_wait before the values are read by
+// the tensor cores.
+__device__ __forceinline__ void st_32cols(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
+        "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+        "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
+        "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+__device__ __forceinline__ void st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte
 // swizzled canonical layout: rows of 64 fp16 (128 bytes), eight rows to a
 // 1024-byte swizzle atom (16-byte chunk c of row r stored at chunk c ^ (r % 8)),
@@ -83,6 +102,21 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
     return d;
 }
 
+// Descriptor of an MN-major operand in the same 128-byte swizzled atoms:
+// rows along K (one per K index, 128 bytes = 64 MN elements), eight rows to a
+// 1024-byte atom; atoms of consecutive 8-row K groups `k_stride` bytes apart,
+// atoms of consecutive 64-element MN blocks `mn_stride` bytes apart.  A tile
+// stored [K rows][MN] in the K-major formula of sw128_offset (rows = K) is
+// this layout with k_stride = 1024 and mn_stride = rows * 128.
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t addr, uint32_t mn_stride, uint32_t k_stride) {
+    uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((mn_stride >> 4) & 0x3FFFu) << 16;  // leading byte offset: next MN block
+    d |= static_cast<uint64_t>((k_stride >> 4) & 0x3FFFu) << 32;   // stride byte offset: next K group
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
 // Instruction descriptor of kind::f16: fp16 A and B, both K-major, fp32 D,
 // shape M x N (M = 64 or 128, N a multiple of 8 up to 256 for M = 64, of 16
 // for M = 128).
@@ -92,6 +126,8 @@ __host__ __device__ constexpr uint32_t idesc_f16(int m, int n) {
            | (static_cast<uint32_t>(n >> 3) << 17)        // N / 8
            | (static_cast<uint32_t>(m >> 4) << 24);       // M / 16
 }
+// The same with B MN-major.
+__host__ __device__ constexpr uint32_t idesc_f16_bmn(int m, int n) { return idesc_f16(m, n) | (1u << 16); }
 
 // Byte offset of fp16 element (r, k) in a K-major 128-byte-swizzled tile of
 // `rows` rows: K is cut into 64-element column blocks of rows x 128 bytes.
