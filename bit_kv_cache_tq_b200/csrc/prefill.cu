@@ -138,13 +138,6 @@ __device__ __forceinline__ void fwht128(float (&x)[D]) {
 
 __device__ __forceinline__ uint32_t pack2(uint16_t lo, uint16_t hi) { return lo | (static_cast<uint32_t>(hi) << 16); }
 
-// two fp16 bit patterns times an fp16 pair, as one fp16 pair
-__device__ __forceinline__ uint32_t hmul_pair(uint16_t lo, uint16_t hi, __half2 f) {
-    const __half2 c = __halves2half2(__ushort_as_half(lo), __ushort_as_half(hi));
-    const __half2 r = __hmul2(c, f);
-    return *reinterpret_cast<const uint32_t*>(&r);
-}
-
 struct Block {
     int qt, kv, b, tok0, ntok, start, kend, ntiles;
     bool bad;
@@ -190,11 +183,6 @@ __device__ __forceinline__ uint4 dequant8(uint32_t c8, const uint32_t* lut) {
     } else {
         return make_uint4(lut[c8 & 63u], lut[(c8 >> 6) & 63u], lut[(c8 >> 12) & 63u], lut[(c8 >> 18) & 63u]);
     }
-}
-
-__device__ __forceinline__ uint32_t hmul2_bits(uint32_t x, __half2 f) {
-    const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&x), f);
-    return *reinterpret_cast<const uint32_t*>(&r);
 }
 
 template <int KB, int VB>
