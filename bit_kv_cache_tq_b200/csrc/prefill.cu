@@ -1,5 +1,6 @@
 // Chunked prefill attention from the compressed cache on the 5th-generation
-// tensor cores (sm_100a, tcgen05 with tensor-memory accumulators).
+// tensor cores (sm_100a, tcgen05 with tensor-memory operands and
+// accumulators).
 //
 // Pages (by title):
 //   [google]  "Google 最新極限壓縮算法，砸碎大模型本地部署的內存墻，8 倍提升！", table
@@ -17,34 +18,40 @@
 //
 // How: one thread block per (sequence, kv head, 128 query rows), a row being
 // one (query token, head of the GQA group), in warp-specialised roles that
-// overlap every stage of a 64-key tile with the tensor cores' work on others:
-//  * a producer thread bulk-copies each tile's packed codes and norms (1-D
+// overlap every stage of a 64-key tile with the tensor cores' work on others.
+// Shared memory carries only what the tensor cores must read from it (the
+// dequantised key and value tiles); the queries, the scores, the weights and
+// the output accumulator live in tensor memory:
+//  * a producer warp bulk-copies each tile's packed codes and norms (1-D
 //    TMA copies, no multicast) into a ring of four stages;
-//  * four dequantising warps turn a stage into fp16 operand tiles in shared
+//  * eight dequantising warps turn a stage into fp16 operand tiles in shared
 //    memory, laid out as the tensor cores read them (K-major, 128-byte
-//    swizzle), double-buffered, through tables that map a byte of codes to
-//    fp16 centroid pairs: K~ [64 keys x 128 channels], the centroids (the key
-//    norms multiply the fp32 scores instead: an fp16 product per element
-//    would add a rounding error that the exponential amplifies with the
-//    score), and V~ [64 keys x 128 channels], the centroids, in the same
-//    per-key layout, which the P V~ product reads as an MN-major operand;
-//    the tile's key and value norms go to small rings the softmax reads;
-//  * one thread issues the tcgen05 MMAs: S = (Q~hi + Q~lo) K~^T (M = 128,
-//    N = 64, K = 128, into one of two tensor-memory score buffers) for tile
-//    j + 1 before O += P V~ (M = 128, N = 128, K = 64, accumulated across
-//    tiles in tensor memory) for tile j, and signals completions through
+//    swizzle), double-buffered, through tables that map a field of two codes
+//    to a pair of fp16 centroids (one copy of each table per lane, so that the
+//    lookups of a warp never share a bank): K~ [64 keys x 128 channels], the
+//    centroids (the key norms multiply the fp32 scores instead: an fp16
+//    product per element would add a rounding error that the exponential
+//    amplifies with the score), and V~ [64 keys x 128 channels], the
+//    centroids times the value norms, in the same per-key layout, which the
+//    P V~ product reads as an MN-major operand; the tile's key norms go to a
+//    small ring the softmax reads;
+//  * one warp issues the tcgen05 MMAs (an elected lane), both with A in
+//    tensor memory:
+//    S = (Q~hi + Q~lo) K~^T (M = 128, N = 64, K = 128, into one of two score
+//    buffers) for tile j + 1 before O += P V~ (M = 128, N = 128, K = 64,
+//    accumulated across tiles) for tile j, and signals completions through
 //    tcgen05.commit on mbarriers;
-//  * four softmax warps own one query row per thread: they rotate and stage
-//    the queries (two fp16 terms, rows scaled to a largest magnitude of 1, so
-//    the scores keep about 22 bits), then per tile read their scores from
-//    tensor memory, apply the causal limit and the online softmax with a lazy
-//    reference (the accumulator in tensor memory is rescaled only when a
-//    score passes the reference by more than 2^8), and write the weights
-//    times the value norms (scaled by 2^-8: with the reference headroom of
-//    2^8 no weight can leave the fp16 range) as the A operand of P V~.  The
-//    end divides by the softmax sum and applies the inverse rotation.
+//  * four softmax warps own one query row per thread (the tensor-memory lane
+//    of the row): they rotate the queries and store them as two fp16 terms
+//    (rows scaled to a largest magnitude of 1, so the scores keep about 22
+//    bits), then per tile read their scores, apply the causal limit and the
+//    online softmax with a lazy reference (the accumulator is rescaled only
+//    when a score passes the reference by more than 2^8), and store the fp16
+//    weights (at most 2^8) as the A operand of P V~.  The end divides by the
+//    softmax sum and applies the inverse rotation.
 // The keys' and values' fp16 centroids carry the codebook's fp16 scale (as in
-// the decode kernels), removed from the scores and the output.
+// the decode kernels; the values' also a factor 2^-4 that keeps centroid x
+// norm inside the fp16 range), removed from the scores and the output.
 //
 // Every mbarrier wait is bounded (about a second, then TQ_DEVERR_TIMEOUT; the
 // block stops issuing work, waits for its copies and MMAs, and frees its
@@ -68,30 +75,30 @@ constexpr int BK = 64;                   // keys per tile
 constexpr int NS = 4;                    // code stages
 constexpr int SOFTMAX_WARPS = 4, DEQ_WARPS = 8;
 constexpr int DEQ0 = SOFTMAX_WARPS * 32;           // first dequantising thread
-constexpr int PRODUCER = DEQ0 + DEQ_WARPS * 32;    // producer thread (lane 0 of its warp)
+constexpr int PRODUCER = DEQ0 + DEQ_WARPS * 32;    // first thread of the producer warp
 constexpr int MMA_WARP = PRODUCER / 32 + 1;        // MMA issuer warp (also allocates tensor memory)
 constexpr int NTHREADS = (MMA_WARP + 1) * 32;
-constexpr uint32_t TMEM_COLS = 256;      // S buffers at columns 0 and 64, O at 128
-constexpr uint32_t TMEM_O = 128;
+// tensor-memory columns (32-bit; fp16 operands take two elements a column)
+constexpr uint32_t TM_QHI = 0;           // Q~ / qscale, fp16 [128 rows][128 ch]
+constexpr uint32_t TM_QLO = 64;          // its fp16 remainder
+constexpr uint32_t TM_S = 128;           // 2 x fp32 scores [128 rows][64 keys]
+constexpr uint32_t TM_P = 256;           // 2 x fp16 weights [128 rows][64 keys]
+constexpr uint32_t TM_O = 320;           // fp32 accumulator [128 rows][128 ch]
+constexpr uint32_t TMEM_COLS = 512;
 constexpr long long WAIT_LIMIT = 2000000000ll;  // clock cycles (~1 s)
-constexpr float NORM_FOLD = 1.0f / 256.0f;      // value norms enter the fp16 weights scaled by 2^-8
+constexpr float VFOLD = 1.0f / 16.0f;           // value centroids x norms enter V~ scaled by 2^-4
 constexpr float LAZY = 8.0f;                    // log2 headroom before the reference moves
 
-// shared-memory map (offsets from a 1024-byte aligned base)
-constexpr uint32_t SM_Q = 0;                       // fp16 [128 rows][128 ch], 2 column blocks of 16 KB
-constexpr uint32_t SM_QLO = SM_Q + BM * D * 2;     // fp16 remainder q~ - fp16(q~), same layout
-constexpr uint32_t SM_K = SM_QLO + BM * D * 2;     // 2 x fp16 [64 keys][128 ch] (2 column blocks of 8 KB each)
+// shared-memory map (offsets from a 1024-byte aligned base); the code tables'
+// sizes depend on the widths
+constexpr uint32_t SM_K = 0;                       // 2 x fp16 [64 keys][128 ch] (2 column blocks of 8 KB each)
 constexpr uint32_t SM_VT = SM_K + 2 * BK * D * 2;  // 2 x fp16 V~ [64 keys][128 ch], the layout of K~
-constexpr uint32_t SM_P = SM_VT + 2 * D * BK * 2;  // 2 x fp16 [128 rows][64 keys]
 constexpr uint32_t STAGE_BYTES = BK * 64 + BK * 64 + BK * 2 + BK * 2;  // K codes, V codes, K norms, V norms
 constexpr uint32_t ST_KC = 0, ST_VC = BK * 64, ST_KN = 2 * BK * 64, ST_VN = 2 * BK * 64 + BK * 2;
-constexpr uint32_t SM_STAGE = SM_P + 2 * BM * BK * 2;
+constexpr uint32_t SM_STAGE = SM_VT + 2 * D * BK * 2;
 constexpr uint32_t SM_KNR = SM_STAGE + NS * STAGE_BYTES;   // fp32 key norms of the last four tiles [4][64]
-constexpr uint32_t SM_VNR = SM_KNR + 4 * BK * 4;           // fp32 value norms x 2^-8 of the last four tiles [4][64]
-constexpr uint32_t SM_CENT = SM_VNR + 4 * BK * 4;          // fp16 key centroids [16], value centroids [16]
-constexpr uint32_t SM_KLUT = SM_CENT + 64;                 // byte of key codes -> fp16 centroids (2 KB)
-constexpr uint32_t SM_VLUT = SM_KLUT + 2048;               // byte of value codes -> fp16 centroids (2 KB)
-constexpr uint32_t SM_BAR = SM_VLUT + 2048;
+constexpr uint32_t SM_CENT = SM_KNR + 4 * BK * 4;          // fp16 key centroids [16], value centroids [16]
+constexpr uint32_t SM_BAR = SM_CENT + 64;
 // mbarriers (8 bytes each)
 constexpr int B_FULL = 0, B_EMPTY = NS, B_KFULL = 2 * NS, B_KEMPTY = B_KFULL + 2, B_VFULL = B_KEMPTY + 2,
               B_VEMPTY = B_VFULL + 2, B_SFULL = B_VEMPTY + 2, B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2,
@@ -101,8 +108,13 @@ constexpr int B_FULL = 0, B_EMPTY = NS, B_KFULL = 2 * NS, B_KEMPTY = B_KFULL + 2
 // barrier keeps every wait within one phase of the barrier's state.)
 constexpr uint32_t SM_TMEM = SM_BAR + NBARS * 8;   // tensor-memory address
 constexpr uint32_t SM_FLAG = SM_TMEM + 4;          // abort flag
-constexpr uint32_t SM_BYTES = SM_FLAG + 4;
-constexpr uint32_t SM_ALLOC = SM_BYTES + 1024;     // room to align the base
+constexpr uint32_t SM_KLUT = (SM_FLAG + 4 + 127) & ~127u;  // key code table, one copy per lane
+// A code table maps a field of two codes (2 BITS bits) to their fp16
+// centroids, packed, with 32 copies interleaved word by word: entry e of lane
+// l is word 32 e + l, so a warp's lookups fall in 32 distinct banks.
+__host__ __device__ constexpr uint32_t lut_bytes(int bits) { return 32u * 4u * (1u << (2 * bits)); }
+__host__ __device__ constexpr uint32_t sm_vlut(int kb) { return SM_KLUT + lut_bytes(kb); }
+__host__ __device__ constexpr uint32_t sm_alloc(int kb, int vb) { return sm_vlut(kb) + lut_bytes(vb) + 1024; }
 
 struct Args {
     const uint8_t* k_codes;
@@ -116,10 +128,10 @@ struct Args {
     int q_dtype, batch, hq, hkv, group, capacity, n_new, tok_per_tile;
     int staged_norms;        // capacity % 8 == 0: norms ride in the bulk copies
     float score_scale;       // sm_scale * log2(e) / alpha_k
-    float out_scale;         // 1 / (alpha_v * NORM_FOLD)
+    float out_scale;         // 1 / (alpha_v * VFOLD)
     uint32_t signs[4];
     uint16_t kcent[16];      // fp16 bits of alpha_k * key centroid
-    uint16_t vcent[16];
+    uint16_t vcent[16];      // fp16 bits of alpha_v * VFOLD * value centroid
 };
 
 // Unnormalised Walsh-Hadamard butterflies over the 128 values a thread holds
@@ -138,57 +150,94 @@ __device__ __forceinline__ void fwht128(float (&x)[D]) {
 
 __device__ __forceinline__ uint32_t pack2(uint16_t lo, uint16_t hi) { return lo | (static_cast<uint32_t>(hi) << 16); }
 
+__device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 struct Block {
     int qt, kv, b, tok0, ntok, start, kend, ntiles;
     bool bad;
 };
 
-// The 8 codes of channels 8 cg .. 8 cg + 7 of a packed row (KB bits each,
-// LSB-first) as one word, code e in bits [KB e, KB e + KB).
-template <int KB>
-__device__ __forceinline__ uint32_t eight_codes(const uint32_t* row, int cg) {
-    const int bit = 8 * KB * cg;
-    if constexpr (KB == 4) return row[cg];
-    if constexpr (KB == 2) return row[cg >> 1] >> (16 * (cg & 1));
-    const int w = bit >> 5, sh = bit & 31;  // 24 bits: may straddle two words
-    const uint32_t lo = row[w];
-    return sh <= 8 ? lo >> sh : __funnelshift_r(lo, row[w + 1], sh);
-}
-
-// Code tables: an index of codes -> their fp16 centroids, packed.  KB = 4: a
-// byte (2 codes) -> one pair; KB = 3: 6 bits (2 codes) -> one pair; KB = 2: a
-// byte (4 codes) -> two pairs.
+// The code table of BITS-bit codes: field e (code e & m, then code e >> BITS)
+// -> fp16 centroid pair, for every lane.
 template <int BITS>
 __device__ void build_lut(uint32_t* lut, const uint16_t* cent, int t, int nthreads) {
-    if constexpr (BITS == 2) {
-        for (int e = t; e < 256; e += nthreads) {
-            lut[2 * e] = pack2(cent[e & 3], cent[(e >> 2) & 3]);
-            lut[2 * e + 1] = pack2(cent[(e >> 4) & 3], cent[e >> 6]);
-        }
-    } else {
-        constexpr int n = 1 << (2 * BITS), m = (1 << BITS) - 1;
-        for (int e = t; e < n; e += nthreads) lut[e] = pack2(cent[e & m], cent[e >> BITS]);
+    constexpr int n = 32 << (2 * BITS), m = (1 << BITS) - 1;
+    for (int i = t; i < n; i += nthreads) {
+        const int e = i >> 5;
+        lut[i] = pack2(cent[e & m], cent[e >> BITS]);
     }
 }
 
-// fp16 centroids of 8 codes (channel order) through the table, as 4 pairs.
-template <int BITS>
-__device__ __forceinline__ uint4 dequant8(uint32_t c8, const uint32_t* lut) {
-    if constexpr (BITS == 4) {
-        return make_uint4(lut[c8 & 0xFFu], lut[(c8 >> 8) & 0xFFu], lut[(c8 >> 16) & 0xFFu], lut[c8 >> 24]);
-    } else if constexpr (BITS == 2) {
-        const uint2 a = reinterpret_cast<const uint2*>(lut)[c8 & 0xFFu];
-        const uint2 b = reinterpret_cast<const uint2*>(lut)[(c8 >> 8) & 0xFFu];
-        return make_uint4(a.x, a.y, b.x, b.y);
-    } else {
-        return make_uint4(lut[c8 & 63u], lut[(c8 >> 6) & 63u], lut[(c8 >> 12) & 63u], lut[(c8 >> 18) & 63u]);
+// One fp16 operand tile (64 keys x 128 channels, K-major, 128-byte swizzle)
+// from a stage's packed codes (rows of 16 BITS bytes, LSB-first): this
+// thread's share is channel group cg = dt % 16 (8 channels) of keys
+// dt / 16 + 16 i.  All shared addresses are 32-bit shared-window addresses;
+// `lut` is this lane's column of the code table.  The loads of the four
+// groups go out together, then the lookups, then the stores.  SCALE: times
+// the key's fp16 norm (from the stage, or from `gnorms` when the stage holds
+// none).  Keys at or past nk are written as zeros.
+template <int BITS, bool SCALE>
+__device__ __forceinline__ void dequant_tile(uint32_t tile, uint32_t codes, uint32_t lut, uint32_t snorms,
+                                             const uint16_t* gnorms, bool staged, int dt, int nk) {
+    constexpr int RB = 16 * BITS, W = 2 * BITS, IT = BK * (D / 8) / (DEQ_WARPS * 32);
+    constexpr uint32_t M = (1u << W) - 1;
+    const int cg = dt & 15, k0 = dt >> 4;
+    uint32_t c8[IT];
+#pragma unroll
+    for (int i = 0; i < IT; ++i) {
+        const uint32_t row = codes + (k0 + 16 * i) * RB;
+        if constexpr (BITS == 4) {
+            c8[i] = ptx::lds32(row + 4 * cg);
+        } else if constexpr (BITS == 2) {
+            c8[i] = ptx::lds32(row + 4 * (cg >> 1)) >> (16 * (cg & 1));
+        } else {  // 24 bits from bit 24 cg: may straddle two words
+            const int bit = 24 * cg, w = bit >> 5, sh = bit & 31;
+            const uint32_t lo = ptx::lds32(row + 4 * w), hi = ptx::lds32(row + 4 * min(w + 1, RB / 4 - 1));
+            c8[i] = sh <= 8 ? lo >> sh : __funnelshift_r(lo, hi, sh);
+        }
+    }
+    uint32_t n2[IT];
+    if constexpr (SCALE) {
+#pragma unroll
+        for (int i = 0; i < IT; ++i) {
+            const int key = k0 + 16 * i;
+            const uint16_t nb = staged ? ptx::lds16(snorms + 2 * key) : (key < nk ? gnorms[key] : uint16_t(0));
+            n2[i] = nb | (static_cast<uint32_t>(nb) << 16);
+        }
+    }
+    uint4 v[IT];
+#pragma unroll
+    for (int i = 0; i < IT; ++i) {
+        v[i].x = ptx::lds32(lut + 128u * (c8[i] & M));
+        v[i].y = ptx::lds32(lut + 128u * ((c8[i] >> W) & M));
+        v[i].z = ptx::lds32(lut + 128u * ((c8[i] >> (2 * W)) & M));
+        v[i].w = ptx::lds32(lut + 128u * ((c8[i] >> (3 * W)) & M));
+    }
+#pragma unroll
+    for (int i = 0; i < IT; ++i) {
+        const int key = k0 + 16 * i;
+        uint4 w = v[i];
+        if constexpr (SCALE) {
+            const __half2 f = *reinterpret_cast<const __half2*>(&n2[i]);
+            __half2* h = reinterpret_cast<__half2*>(&w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h[e] = __hmul2(h[e], f);
+        }
+        if (key >= nk) w = make_uint4(0u, 0u, 0u, 0u);
+        ptx::sts128(tile + tc::sw128_offset(key, 8 * cg, BK), w);
     }
 }
 
 template <int KB, int VB>
 __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_constant__ Args a) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, reached by pointer arithmetic on the shared
+    // array (a round trip through an integer would hide the address space and
+    // turn every access below into a generic load or store)
+    uint8_t* smem = smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = ptx::smem_addr(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t bars = sbase + SM_BAR;
@@ -252,28 +301,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + SM_TMEM);
     const size_t unit_row = (static_cast<size_t>(blk.b) * a.hkv + blk.kv) * a.capacity;
-    // the code tables, built by the dequantising warps (they alone read them;
-    // a named barrier among them publishes the tables)
     constexpr int kbytes = 16 * KB, vbytes = 16 * VB;  // packed row sizes
 
-    if (tid == PRODUCER) {
+    if (warp == PRODUCER / 32) {
         // ---------------------------------------------------------- producer
+        // the whole warp waits; one elected lane issues the copies
+        const bool leader = tc::elect_one();
         int issued = 0;
         for (int j = 0; j < T; ++j) {
             const int s = j % NS;
             if (j >= NS && !wait(B_EMPTY + s, ((j - NS) / NS) & 1)) break;
-            const int key0 = j * BK, nk = min(BK, blk.kend - key0);
-            const uint32_t dst = sbase + SM_STAGE + s * STAGE_BYTES;
-            const int n8 = (nk + 7) & ~7;  // norms move in 16-byte pieces (8 keys)
-            const uint32_t bytes = nk * (kbytes + vbytes) + (a.staged_norms ? n8 * 4 : 0);
-            ptx::mbar_arrive_expect_tx(bar(B_FULL + s), bytes);
-            ptx::bulk_copy_g2s(dst + ST_KC, a.k_codes + (unit_row + key0) * kbytes, nk * kbytes, bar(B_FULL + s));
-            ptx::bulk_copy_g2s(dst + ST_VC, a.v_codes + (unit_row + key0) * vbytes, nk * vbytes, bar(B_FULL + s));
-            if (a.staged_norms) {
-                // capacity and key0 are multiples of 8: the rounded range stays inside the cache
-                ptx::bulk_copy_g2s(dst + ST_KN, a.k_norms + unit_row + key0, n8 * 2, bar(B_FULL + s));
-                ptx::bulk_copy_g2s(dst + ST_VN, a.v_norms + unit_row + key0, n8 * 2, bar(B_FULL + s));
+            if (leader) {
+                const int key0 = j * BK, nk = min(BK, blk.kend - key0);
+                const uint32_t dst = sbase + SM_STAGE + s * STAGE_BYTES;
+                const int n8 = (nk + 7) & ~7;  // norms move in 16-byte pieces (8 keys)
+                const uint32_t bytes = nk * (kbytes + vbytes) + (a.staged_norms ? n8 * 4 : 0);
+                ptx::mbar_arrive_expect_tx(bar(B_FULL + s), bytes);
+                ptx::bulk_copy_g2s(dst + ST_KC, a.k_codes + (unit_row + key0) * kbytes, nk * kbytes, bar(B_FULL + s));
+                ptx::bulk_copy_g2s(dst + ST_VC, a.v_codes + (unit_row + key0) * vbytes, nk * vbytes, bar(B_FULL + s));
+                if (a.staged_norms) {
+                    // capacity and key0 are multiples of 8: the rounded range stays inside the cache
+                    ptx::bulk_copy_g2s(dst + ST_KN, a.k_norms + unit_row + key0, n8 * 2, bar(B_FULL + s));
+                    ptx::bulk_copy_g2s(dst + ST_VN, a.v_norms + unit_row + key0, n8 * 2, bar(B_FULL + s));
+                }
             }
+            __syncwarp();
             issued = j + 1;
         }
         // every copy issued must land before the block may exit
@@ -281,63 +333,38 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
             ptx::mbar_wait_bounded(bar(B_FULL + j % NS), (j / NS) & 1, WAIT_LIMIT);
     } else if (warp >= DEQ0 / 32 && warp < PRODUCER / 32) {
         // ------------------------------------------------------ dequantisers
-        const int dt = tid - DEQ0;  // 0 .. 127
+        const int dt = tid - DEQ0;  // 0 .. 255
         const uint16_t* kcent = reinterpret_cast<const uint16_t*>(smem + SM_CENT);
         const uint16_t* vcent = kcent + 16;
         uint32_t* klut = reinterpret_cast<uint32_t*>(smem + SM_KLUT);
-        uint32_t* vlut = reinterpret_cast<uint32_t*>(smem + SM_VLUT);
+        uint32_t* vlut = reinterpret_cast<uint32_t*>(smem + sm_vlut(KB));
         build_lut<KB>(klut, kcent, dt, DEQ_WARPS * 32);
         build_lut<VB>(vlut, vcent, dt, DEQ_WARPS * 32);
         ptx::named_barrier(1, DEQ_WARPS * 32);
+        const uint32_t klane = sbase + SM_KLUT + 4 * lane, vlane = sbase + sm_vlut(KB) + 4 * lane;
         for (int j = 0; j < T; ++j) {
             const int s = j % NS, bf = j & 1;
             if (!wait(B_FULL + s, (j / NS) & 1)) break;
             const uint8_t* st = smem + SM_STAGE + s * STAGE_BYTES;
+            const uint32_t sst = sbase + SM_STAGE + s * STAGE_BYTES;
             const int key0 = j * BK, nk = min(BK, blk.kend - key0);
             const uint16_t* skn = reinterpret_cast<const uint16_t*>(st + ST_KN);
-            const uint16_t* svn = reinterpret_cast<const uint16_t*>(st + ST_VN);
-            auto knorm = [&](int key) -> float {
-                if (key >= nk) return 0.f;
-                return half_bits_to_float(a.staged_norms ? skn[key] : a.k_norms[unit_row + key0 + key]);
-            };
-            auto vnorm = [&](int key) -> float {
-                if (key >= nk) return 0.f;
-                return half_bits_to_float(a.staged_norms ? svn[key] : a.v_norms[unit_row + key0 + key]);
-            };
             // K~[bf]: 64 keys x 16 groups of 8 channels, centroids; the tile's
-            // key and value norms go to the softmax's rings (its tile j - 4 is
-            // done: this tile's K~ buffer was free only after S(j - 2), which
-            // needed the softmax to be through tile j - 4)
+            // key norms go to the softmax's ring (its tile j - 4 is done: this
+            // tile's K~ buffer was free only after S(j - 2), which needed the
+            // softmax to be through tile j - 4)
             if (j >= 2 && !wait(B_KEMPTY + bf, ((j - 2) >> 1) & 1)) break;
-            if (dt < BK) {
-                reinterpret_cast<float*>(smem + SM_KNR)[(j & 3) * BK + dt] = knorm(dt);
-                reinterpret_cast<float*>(smem + SM_VNR)[(j & 3) * BK + dt] = vnorm(dt) * NORM_FOLD;
-            }
-            uint8_t* kt = smem + SM_K + bf * (BK * D * 2);
-#pragma unroll 4
-            for (int it = dt; it < BK * (D / 8); it += DEQ_WARPS * 32) {
-                const int key = it >> 4, cg = it & 15;
-                uint4 w = make_uint4(0u, 0u, 0u, 0u);
-                if (key < nk)
-                    w = dequant8<KB>(eight_codes<KB>(reinterpret_cast<const uint32_t*>(st + ST_KC + key * kbytes), cg),
-                                     klut);
-                *reinterpret_cast<uint4*>(kt + tc::sw128_offset(key, 8 * cg, BK)) = w;
-            }
+            if (dt < BK)
+                reinterpret_cast<float*>(smem + SM_KNR)[(j & 3) * BK + dt] =
+                    dt < nk ? half_bits_to_float(a.staged_norms ? skn[dt] : a.k_norms[unit_row + key0 + dt]) : 0.f;
+            dequant_tile<KB, false>(sbase + SM_K + bf * (BK * D * 2), sst + ST_KC, klane, 0u, nullptr, true, dt, nk);
             tc::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(bar(B_KFULL + bf));
-            // V~[bf]: the same per-key layout, centroids
+            // V~[bf]: the same per-key layout, centroids x norms
             if (j >= 2 && !wait(B_VEMPTY + bf, ((j - 2) >> 1) & 1)) break;
-            uint8_t* vt = smem + SM_VT + bf * (BK * D * 2);
-#pragma unroll 4
-            for (int it = dt; it < BK * (D / 8); it += DEQ_WARPS * 32) {
-                const int key = it >> 4, cg = it & 15;
-                uint4 w = make_uint4(0u, 0u, 0u, 0u);
-                if (key < nk)
-                    w = dequant8<VB>(eight_codes<VB>(reinterpret_cast<const uint32_t*>(st + ST_VC + key * vbytes), cg),
-                                     vlut);
-                *reinterpret_cast<uint4*>(vt + tc::sw128_offset(key, 8 * cg, BK)) = w;
-            }
+            dequant_tile<VB, true>(sbase + SM_VT + bf * (BK * D * 2), sst + ST_VC, vlane, sst + ST_VN,
+                                   a.v_norms + unit_row + key0, a.staged_norms != 0, dt, nk);
             tc::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -347,51 +374,63 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         }
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc_s = tc::idesc_f16(BM, BK), idesc_o = tc::idesc_f16_bmn(BM, D);
-            bool ok = T == 0 || wait(B_QREADY, 0);
-            auto issue_s = [&](int j) -> bool {
-                const int bf = j & 1;
-                if (!wait(B_KFULL + bf, (j >> 1) & 1)) return false;
-                if (j >= 2 && !wait(B_SEMPTY + bf, ((j - 2) >> 1) & 1)) return false;
-                tc::fence_after_sync();
-                const uint32_t kt = sbase + SM_K + bf * (BK * D * 2);
+        // the whole warp waits; one elected lane issues the MMAs and commits
+        const bool leader = tc::elect_one();
+        const uint32_t idesc_s = tc::idesc_f16(BM, BK), idesc_o = tc::idesc_f16_bmn(BM, D);
+        // descriptors are linear in the start address: the K slices and
+        // buffers are fixed offsets (in 16-byte units) from these
+        const uint64_t kdesc0 = tc::sw128_desc(sbase + SM_K);
+        const uint64_t vdesc0 = tc::sw128_mn_desc(sbase + SM_VT, BK * 128, 1024);
+        bool ok = T == 0 || wait(B_QREADY, 0);
+        auto issue_s = [&](int j) -> bool {
+            const int bf = j & 1;
+            if (!wait(B_KFULL + bf, (j >> 1) & 1)) return false;
+            if (j >= 2 && !wait(B_SEMPTY + bf, ((j - 2) >> 1) & 1)) return false;
+            tc::fence_after_sync();
+            if (leader) {
+                const uint64_t kd = kdesc0 + static_cast<uint64_t>(bf * (BK * D * 2) >> 4);
+                const uint32_t sd = tmem + TM_S + BK * bf;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t cb = ks >> 2, within = (ks & 3) * 32;
-                    const uint64_t bd = tc::sw128_desc(kt + cb * (BK * 128) + within);
-                    tc::mma_f16(tmem + BK * bf, tc::sw128_desc(sbase + SM_Q + cb * (BM * 128) + within), bd, idesc_s,
-                                ks > 0);
-                    tc::mma_f16(tmem + BK * bf, tc::sw128_desc(sbase + SM_QLO + cb * (BM * 128) + within), bd,
-                                idesc_s, true);
+                    // 16 channels per step: 32 bytes within a 64-channel block
+                    const uint64_t bd = kd + static_cast<uint64_t>(((ks >> 2) * (BK * 128) + (ks & 3) * 32) >> 4);
+                    tc::mma_f16_ts(sd, tmem + TM_QHI + 8 * ks, bd, idesc_s, ks > 0);
+                    tc::mma_f16_ts(sd, tmem + TM_QLO + 8 * ks, bd, idesc_s, true);
                 }
                 tc::commit(bar(B_SFULL + bf));
                 tc::commit(bar(B_KEMPTY + bf));
-                return true;
-            };
-            auto issue_pv = [&](int j) -> bool {
-                const int bf = j & 1;
-                if (!wait(B_PFULL + bf, (j >> 1) & 1)) return false;
-                if (!wait(B_VFULL + bf, (j >> 1) & 1)) return false;
-                tc::fence_after_sync();
-                const uint32_t pt = sbase + SM_P + bf * (BM * BK * 2), vt = sbase + SM_VT + bf * (BK * D * 2);
+            }
+            __syncwarp();
+            return true;
+        };
+        auto issue_pv = [&](int j) -> bool {
+            const int bf = j & 1;
+            if (!wait(B_PFULL + bf, (j >> 1) & 1)) return false;
+            if (!wait(B_VFULL + bf, (j >> 1) & 1)) return false;
+            tc::fence_after_sync();
+            if (leader) {
+                const uint64_t vd = vdesc0 + static_cast<uint64_t>(bf * (BK * D * 2) >> 4);
+                const uint32_t pa = tmem + TM_P + (BK / 2) * bf;
                 // V~ [64 keys][128 ch]: 16 keys per step = two 1024-byte K groups;
                 // the two 64-channel blocks lie 64 rows x 128 bytes apart
 #pragma unroll
                 for (int ks = 0; ks < BK / 16; ++ks)
-                    tc::mma_f16(tmem + TMEM_O, tc::sw128_desc(pt + ks * 32),
-                                tc::sw128_mn_desc(vt + ks * 2048, BK * 128, 1024), idesc_o, j > 0 || ks > 0);
+                    tc::mma_f16_ts(tmem + TM_O, pa + 8 * ks, vd + static_cast<uint64_t>(ks * 2048 >> 4), idesc_o,
+                                   j > 0 || ks > 0);
                 tc::commit(bar(B_PEMPTY + bf));
                 tc::commit(bar(B_VEMPTY + bf));
-                return true;
-            };
-            if (ok && T > 0) ok = issue_s(0);
-            for (int j = 0; ok && j < T; ++j) {
-                if (j + 1 < T && !issue_s(j + 1)) break;
-                if (!issue_pv(j)) break;
             }
-            // every tensor-core operation issued completes before the block
-            // frees its tensor memory (bounded, also after an abort)
+            __syncwarp();
+            return true;
+        };
+        if (ok && T > 0) ok = issue_s(0);
+        for (int j = 0; ok && j < T; ++j) {
+            if (j + 1 < T && !issue_s(j + 1)) break;
+            if (!issue_pv(j)) break;
+        }
+        // every tensor-core operation issued completes before the block
+        // frees its tensor memory (bounded, also after an abort)
+        if (leader) {
             tc::commit(bar(B_FINAL));
             ptx::mbar_wait_bounded(bar(B_FINAL), 0, WAIT_LIMIT);
         }
@@ -401,6 +440,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         const int r = tid;
         const int rt = r / G, rh = r % G;
         const bool row_ok = rt < blk.ntok && rt * G + rh < BM;
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
         float qscale = 0.f;  // largest |q~| of the row: the fp16 terms hold q~ / qscale
         {
             float x[D];
@@ -426,60 +466,68 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
             qscale = amax * inv_sqrt_d;
             const float rs = amax > 0.f ? 1.f / amax : 0.f;
 #pragma unroll
-            for (int c = 0; c < D; c += 8) {
-                uint32_t hw[4], lw[4];
+            for (int c = 0; c < D; c += 16) {
+                uint32_t hw[8], lw[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
+                for (int e = 0; e < 8; ++e) {
                     const float u0 = x[c + 2 * e] * rs, u1 = x[c + 2 * e + 1] * rs;
                     const __half h0 = __float2half_rn(u0), h1 = __float2half_rn(u1);
                     hw[e] = pack2(__half_as_ushort(h0), __half_as_ushort(h1));
-                    lw[e] = pack2(__half_as_ushort(__float2half_rn(u0 - __half2float(h0))),
-                                  __half_as_ushort(__float2half_rn(u1 - __half2float(h1))));
+                    lw[e] = half2_bits(u0 - __half2float(h0), u1 - __half2float(h1));
                 }
-                *reinterpret_cast<uint4*>(smem + SM_Q + tc::sw128_offset(r, c, BM)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4*>(smem + SM_QLO + tc::sw128_offset(r, c, BM)) =
-                    make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                tc::st_8cols(tmem + lane_base + TM_QHI + c / 2, hw);
+                tc::st_8cols(tmem + lane_base + TM_QLO + c / 2, lw);
             }
         }
-        tc::fence_proxy_async_smem();
+        tc::st_wait();
+        tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(B_QREADY));
-        const float row_scale = qscale * a.score_scale;  // scores: S * row_scale, log2 units
-        const int qpos = blk.start + blk.tok0 + rt;      // this row's own position: the causal limit
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        // scores in log2 units: S kn rs; a zero query row keeps rs > 0 so that a
+        // masked (-inf) score stays -inf
+        const float rs = fmaxf(qscale * a.score_scale, 1e-30f);
+        const int qpos = blk.start + blk.tok0 + rt;  // this row's own position: the causal limit
         float mref = -INFINITY, l = 0.f;
         for (int j = 0; j < T; ++j) {
             const int bf = j & 1, key0 = j * BK;
             if (!wait(B_SFULL + bf, (j >> 1) & 1)) break;
             tc::fence_after_sync();
-            float sv[2][32];
-            float mt = -INFINITY;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                tc::ld_32cols(tmem + lane_base + BK * bf + 32 * h, sv[h]);
+            float u[BK];
+            {
+                float (&u0)[32] = *reinterpret_cast<float (*)[32]>(&u[0]);
+                float (&u1)[32] = *reinterpret_cast<float (*)[32]>(&u[32]);
+                tc::ld_32cols(tmem + lane_base + TM_S + BK * bf, u0);
+                tc::ld_32cols(tmem + lane_base + TM_S + BK * bf + 32, u1);
             }
             tc::ld_wait();
-            const float* kn = reinterpret_cast<const float*>(smem + SM_KNR) + (j & 3) * BK;
-            if (key0 + BK - 1 <= blk.start + blk.tok0) {
-                // every row of the block sees every key of the tile (rows
-                // outside the chunk are never stored, so need no mask)
+            const float4* kn4 = reinterpret_cast<const float4*>(smem + SM_KNR + (j & 3) * BK * 4);
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        sv[h][i] = sv[h][i] * kn[32 * h + i] * row_scale;
-                        mt = fmaxf(mt, sv[h][i]);
-                    }
-            } else {
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int key = key0 + 32 * h + i;
-                        sv[h][i] = (row_ok && key <= qpos) ? sv[h][i] * kn[32 * h + i] * row_scale : -INFINITY;
-                        mt = fmaxf(mt, sv[h][i]);
-                    }
+            for (int i = 0; i < BK; i += 4) {
+                const float4 k4 = kn4[i / 4];
+                const float2 a01 = ptx::fmul2(make_float2(u[i], u[i + 1]), make_float2(k4.x, k4.y));
+                const float2 a23 = ptx::fmul2(make_float2(u[i + 2], u[i + 3]), make_float2(k4.z, k4.w));
+                u[i] = a01.x;
+                u[i + 1] = a01.y;
+                u[i + 2] = a23.x;
+                u[i + 3] = a23.y;
             }
+            if (key0 + BK - 1 > blk.start + blk.tok0) {
+                // a tile on the diagonal: keys past the row's own position drop
+                // out (rows outside the chunk are never stored; every key of an
+                // earlier tile is visible to every row of the block)
+#pragma unroll
+                for (int i = 0; i < BK; ++i)
+                    if (!row_ok || key0 + i > qpos) u[i] = -INFINITY;
+            }
+            float m4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float m = u[16 * q];
+#pragma unroll
+                for (int i = 1; i < 15; i += 2) m = ptx::fmax3(m, u[16 * q + i], u[16 * q + i + 1]);
+                m4[q] = fmaxf(m, u[16 * q + 15]);
+            }
+            const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * rs;
             // lazy reference: moves (and the accumulator is rescaled) only when a
             // score passes it by more than 2^LAZY; the weights stay below 2^LAZY
             const bool need = mt > mref + LAZY;
@@ -490,48 +538,47 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                     // every P V of the earlier tiles is in the accumulator
                     if (!wait(B_PEMPTY + ((j - 1) & 1), ((j - 1) >> 1) & 1)) break;
                     tc::fence_after_sync();
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        float ov[32];
-                        tc::ld_32cols(tmem + lane_base + TMEM_O + 32 * q4, ov);
+#pragma unroll 1
+                    for (int q8 = 0; q8 < 8; ++q8) {
+                        float ov[16];
+                        tc::ld_16cols(tmem + lane_base + TM_O + 16 * q8, ov);
                         tc::ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) ov[i] *= c;
-                        tc::st_32cols(tmem + lane_base + TMEM_O + 32 * q4, ov);
+                        for (int i = 0; i < 16; ++i) ov[i] *= c;
+                        tc::st_16cols(tmem + lane_base + TM_O + 16 * q8, ov);
                     }
-                    tc::st_wait();
                 }
                 l *= c;
                 mref = mnew;
             }
-            // weights of the tile, fp16, as the A operand of P V~
+            // weights of the tile, fp16, as the A operand of P V~ (stored in
+            // two halves of 32 keys)
             if (j >= 2 && !wait(B_PEMPTY + bf, ((j - 2) >> 1) & 1)) break;
-            uint8_t* pt = smem + SM_P + bf * (BM * BK * 2);
-            const float* vnr = reinterpret_cast<const float*>(smem + SM_VNR) + (j & 3) * BK;
-            float ls = 0.f;
+            const bool live = mref > -INFINITY;
+            const float2 rs2 = make_float2(rs, rs), nm2 = make_float2(-mref, -mref);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pw[16];
 #pragma unroll
-                for (int c = 0; c < 32; c += 8) {
-                    float e8[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float pe = mref > -INFINITY ? ptx::ex2(sv[h][c + e] - mref) : 0.f;
-                        ls += pe;
-                        e8[e] = pe * vnr[32 * h + c + e];
-                    }
-                    const __half2 p0 = __floats2half2_rn(e8[0], e8[1]), p1 = __floats2half2_rn(e8[2], e8[3]);
-                    const __half2 p2 = __floats2half2_rn(e8[4], e8[5]), p3 = __floats2half2_rn(e8[6], e8[7]);
-                    *reinterpret_cast<uint4*>(pt + tc::sw128_offset(r, 32 * h + c, BM)) =
-                        make_uint4(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1),
-                                   *reinterpret_cast<const uint32_t*>(&p2), *reinterpret_cast<const uint32_t*>(&p3));
+                for (int i = 0; i < 32; i += 4) {
+                    const float2 t0 = ptx::ffma2(make_float2(u[32 * h + i], u[32 * h + i + 1]), rs2, nm2);
+                    const float2 t1 = ptx::ffma2(make_float2(u[32 * h + i + 2], u[32 * h + i + 3]), rs2, nm2);
+                    const float2 p0 = make_float2(ptx::ex2(t0.x), ptx::ex2(t0.y));
+                    const float2 p1 = make_float2(ptx::ex2(t1.x), ptx::ex2(t1.y));
+                    acc0 = ptx::fadd2(acc0, p0);
+                    acc1 = ptx::fadd2(acc1, p1);
+                    pw[i / 2] = live ? half2_bits(p0.x, p0.y) : 0u;
+                    pw[i / 2 + 1] = live ? half2_bits(p1.x, p1.y) : 0u;
                 }
-            l += ls;
-            tc::fence_proxy_async_smem();
+                tc::st_16cols_u(tmem + lane_base + TM_P + (BK / 2) * bf + 16 * h, pw);
+            }
+            if (live) l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
+            tc::st_wait();
             tc::fence_before_sync();
             __syncwarp();
-            // the weights are written and the score buffer, the tile's norms
-            // and any accumulator rescale are done with
+            // the weights are stored and the score buffer, the tile's norms and
+            // any accumulator rescale are done with
             if (lane == 0) {
                 ptx::mbar_arrive(bar(B_SEMPTY + bf));
                 ptx::mbar_arrive(bar(B_PFULL + bf));
@@ -545,7 +592,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
                 float ov[32];
-                tc::ld_32cols(tmem + lane_base + TMEM_O + 32 * q4, ov);
+                tc::ld_32cols(tmem + lane_base + TM_O + 32 * q4, ov);
                 tc::ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[32 * q4 + i] = ov[i];
@@ -582,10 +629,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
 
 template <int KB, int VB>
 static cudaError_t launch_typed(const Args& a, dim3 grid, cudaStream_t s) {
+    constexpr uint32_t bytes = sm_alloc(KB, VB);
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(SM_ALLOC));
+                                         static_cast<int>(bytes));
     if (e != cudaSuccess) return e;
-    prefill_kernel<KB, VB><<<grid, NTHREADS, SM_ALLOC, s>>>(a);
+    prefill_kernel<KB, VB><<<grid, NTHREADS, bytes, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -658,10 +706,11 @@ extern "C" tq_status tq_prefill_attention(const tq_params* params, const tq_code
     const double av = vcb->fp16_scale > 0.0 ? vcb->fp16_scale : std::sqrt(128.0);
     const float sm = p.sm_scale > 0.0f ? p.sm_scale : 1.0f / std::sqrt(128.0f);
     a.score_scale = static_cast<float>(sm * 1.4426950408889634 / ak);
-    a.out_scale = static_cast<float>(1.0 / (av * prefill::NORM_FOLD));
+    a.out_scale = static_cast<float>(1.0 / (av * prefill::VFOLD));
     for (int j = 0; j < 16; ++j) {
         const __half hk = __float2half_rn(j < (1 << p.k_bits) ? static_cast<float>(kcb->centroids[j] * ak) : 0.f);
-        const __half hv = __float2half_rn(j < (1 << p.v_bits) ? static_cast<float>(vcb->centroids[j] * av) : 0.f);
+        const __half hv =
+            __float2half_rn(j < (1 << p.v_bits) ? static_cast<float>(vcb->centroids[j] * av * prefill::VFOLD) : 0.f);
         a.kcent[j] = __half_as_ushort(hk);
         a.vcent[j] = __half_as_ushort(hv);
     }
