@@ -139,36 +139,35 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
-# DRAM traffic of the decode kernel, taken from the committed ncu summary; it
-# applies only while the kernel's sources are the ones that were profiled.
-DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_mma_kernel_llama8b_layer_32k.md")
-DECODE_SOURCES = ("decode_mma.cu", "device_common.cuh", "ptx.cuh")
+# DRAM traffic per kernel from ncu captures, machine-read from
+# profiles/traffic.json: for each kernel the bytes (dram__bytes_read.sum +
+# dram__bytes_write.sum) of one captured launch, the units of work that launch
+# processed, and the sha256 of the sources it was built from.  A figure applies
+# only while those sources are unchanged.
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+CSRC = os.path.join(ROOT, "bit_kv_cache_tq_b200", "csrc")
 
 
-def decode_source_sha256():
+def sources_sha256(names):
     import hashlib
     h = hashlib.sha256()
-    for name in DECODE_SOURCES:
-        with open(os.path.join(ROOT, "bit_kv_cache_tq_b200", "csrc", name), "rb") as fh:
+    for name in names:
+        with open(os.path.join(CSRC, name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
 
 
-def profiled_traffic(tokens):
-    """DRAM bytes (read + write) of one decode launch over `tokens` tokens per
-    kv head, scaled from the profiled launch; None when the summary is missing
-    or the kernel changed since it was taken."""
-    fields = {}
+def profiled_traffic(kernel, units):
+    """DRAM bytes of one launch of `kernel` over `units` units of work, scaled
+    from the captured launch; None when no capture of the current sources is
+    recorded."""
     try:
-        with open(DECODE_PROFILE, encoding="utf-8") as fh:
-            for line in fh:
-                if line.startswith("- ") and ": " in line:
-                    key, val = line[2:].split(": ", 1)
-                    fields[key.strip()] = val.strip().strip("`")
-        if fields.get("kernel sources sha256") != decode_source_sha256():
+        with open(TRAFFIC_FILE, encoding="utf-8") as fh:
+            rec = json.load(fh)[kernel]
+        if rec["sources_sha256"] != sources_sha256(rec["sources"]):
             return None
-        return float(fields["dram bytes per launch"]) * tokens / float(fields["tokens per kv head"])
-    except (OSError, KeyError, ValueError):
+        return float(rec["dram_bytes_per_launch"]) * units / float(rec["units_per_launch"])
+    except (OSError, KeyError, ValueError, TypeError):
         return None
 
 
@@ -706,7 +705,8 @@ def run_tq(args, world, rank, local):
             "hbm_gbs": alg_bytes * LAYERS / (ms / steps * 1e-3) / 1e9,
             "pct_of_8tbs": 100.0 * alg_bytes * LAYERS / (ms / steps * 1e-3) / 8e12,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": profiled_traffic(seq), "peak_kind": peak_kind,
+                         "frac": achieved / peak, "traffic": profiled_traffic("decode_mma_kernel", seq),
+                         "peak_kind": peak_kind,
                          "kernel": "decode kernel timed alone (tq_decode_attention, no append), %.2f us per launch, %d B algorithmic"
                                    % (decode_us, alg_bytes)},
             "cpu_baseline": cpu_info,

@@ -216,19 +216,22 @@ __device__ __forceinline__ void dequant_tile(uint32_t tile, uint32_t codes, uint
         v[i].z = ptx::lds32(lut + 128u * ((c8[i] >> (2 * W)) & M));
         v[i].w = ptx::lds32(lut + 128u * ((c8[i] >> (3 * W)) & M));
     }
+    if constexpr (SCALE) {
 #pragma unroll
-    for (int i = 0; i < IT; ++i) {
-        const int key = k0 + 16 * i;
-        uint4 w = v[i];
-        if constexpr (SCALE) {
+        for (int i = 0; i < IT; ++i) {
             const __half2 f = *reinterpret_cast<const __half2*>(&n2[i]);
-            __half2* h = reinterpret_cast<__half2*>(&w);
+            __half2* h = reinterpret_cast<__half2*>(&v[i]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) h[e] = __hmul2(h[e], f);
         }
-        if (key >= nk) w = make_uint4(0u, 0u, 0u, 0u);
-        ptx::sts128(tile + tc::sw128_offset(key, 8 * cg, BK), w);
     }
+    if (nk < BK) {  // the last, partial tile only
+#pragma unroll
+        for (int i = 0; i < IT; ++i)
+            if (k0 + 16 * i >= nk) v[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < IT; ++i) ptx::sts128(tile + tc::sw128_offset(k0 + 16 * i, 8 * cg, BK), v[i]);
 }
 
 template <int KB, int VB>
@@ -250,7 +253,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
     // bounded wait on phase `parity` of mbarrier i; false (and the abort flag set) when it runs out
     auto wait = [&](int i, uint32_t parity) -> bool {
         if (*abort_flag) return false;
-        if (!ptx::mbar_wait_bounded(bar(i), parity, WAIT_LIMIT)) {
+        if (!ptx::mbar_wait_bounded_lean(bar(i), parity, WAIT_LIMIT)) {
             fail();
             return false;
         }
@@ -310,7 +313,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         int issued = 0;
         for (int j = 0; j < T; ++j) {
             const int s = j % NS;
-            if (j >= NS && !wait(B_EMPTY + s, ((j - NS) / NS) & 1)) break;
+            // (the ring is four tiles deep: the producer can poll slowly and
+            // leave the issue slots of its sub-partition to the working warps)
+            if (j >= NS) {
+                if (*abort_flag) break;
+                if (!ptx::mbar_wait_bounded_sleep(bar(B_EMPTY + s), ((j - NS) / NS) & 1, WAIT_LIMIT, 256)) {
+                    fail();
+                    break;
+                }
+            }
             if (leader) {
                 const int key0 = j * BK, nk = min(BK, blk.kend - key0);
                 const uint32_t dst = sbase + SM_STAGE + s * STAGE_BYTES;
@@ -568,8 +579,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                     const float2 p1 = make_float2(ptx::ex2(t1.x), ptx::ex2(t1.y));
                     acc0 = ptx::fadd2(acc0, p0);
                     acc1 = ptx::fadd2(acc1, p1);
-                    pw[i / 2] = live ? half2_bits(p0.x, p0.y) : 0u;
-                    pw[i / 2 + 1] = live ? half2_bits(p1.x, p1.y) : 0u;
+                    pw[i / 2] = half2_bits(p0.x, p0.y);
+                    pw[i / 2 + 1] = half2_bits(p1.x, p1.y);
+                }
+                if (!live) {  // no visible key yet (a row past the chunk): no weight
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) pw[i] = 0u;
                 }
                 tc::st_16cols_u(tmem + lane_base + TM_P + (BK / 2) * bf + 16 * h, pw);
             }

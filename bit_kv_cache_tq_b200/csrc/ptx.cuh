@@ -55,6 +55,20 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     return true;
 }
 
+// As mbar_wait_bounded, reading the clock once every 8 polls (a poll loop
+// that shares its sub-partition with working warps costs them fewer issue
+// slots).
+__device__ __forceinline__ bool mbar_wait_bounded_lean(uint32_t bar, uint32_t parity, long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long start = clock64();
+    for (;;) {
+#pragma unroll 1
+        for (int k = 0; k < 8; ++k)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (clock64() - start > limit) return false;
+    }
+}
+
 // As mbar_wait_bounded, sleeping `ns` nanoseconds between polls: for a thread
 // that waits most of the time and should leave its scheduler to other warps.
 __device__ __forceinline__ bool mbar_wait_bounded_sleep(uint32_t bar, uint32_t parity, long long limit, unsigned ns) {
