@@ -21,6 +21,8 @@
 
 #include <chrono>
 #include <cmath>
+#include <cstring>
+#include <algorithm>
 #include <thread>
 
 #include "device_common.cuh"
@@ -39,6 +41,15 @@ struct QuantSide {
     int mode, bits, vbytes, m;
     float centroids[16];
     float pos_boundaries[8];  // boundaries above zero, ascending (2^(bits-1) - 1 of them)
+    // Code grid (turbo mode; grid_inv_w = 0 when the table cannot hold the
+    // codebook): the rotated unit coordinate y is cut into cells of width w
+    // (no wider than the narrowest code cell, so a grid cell holds at most one
+    // boundary), cell c = round(y / w) covering [(c - 0.5) w, (c + 0.5) w).
+    // Entry c & 127 = {number of boundaries below the cell, the boundary
+    // inside it in cells (bits of an fp32; +inf when none)}: the code of y is
+    // the first plus (y / w > the second).  |y| <= 1 keeps c within +-63.
+    float grid_inv_w;
+    uint2 grid[128];
 };
 
 struct QuantArgs {
@@ -46,6 +57,8 @@ struct QuantArgs {
     const int32_t* positions;  // per sequence: first slot written, or (pos_from_lens) the length after the append
     uint32_t* err;
     int batch, n_new, hkv, capacity, pos_from_lens;  // capacity: tokens a sequence may hold
+    uint32_t total;                     // batch * n_new * hkv vectors (< 2^32)
+    uint64_t hkv_magic, n_new_magic;    // quotient multipliers: see div_magic
     // paged cache (table non-null): token t of sequence b is in block
     // table[b * max_blocks + t / block_size] of the pool
     const int32_t* table;
@@ -89,6 +102,123 @@ __device__ __forceinline__ uint32_t code_scaled(float x, const float (&ts)[7]) {
         m = a > ts[0];
     }
     return x > 0.0f ? static_cast<uint32_t>(half + m) : static_cast<uint32_t>(half - 1 - m);
+}
+
+// n / d for n < 2^32 as the high word of n * M, M = ceil(2^64 / d) (exact:
+// the product overshoots n / d by less than n / 2^64 < 1 / d); M = 0 stands
+// for d = 1.
+__device__ __forceinline__ uint32_t div_magic(uint32_t n, uint64_t m) {
+    return m == 0 ? n : static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(n), m));
+}
+
+// Walsh-Hadamard butterflies over a lane's 32 values, the stages of span 2
+// and more as packed fp32 pairs (the same additions, in the same order).
+__device__ __forceinline__ void fwht32_pairs(float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        const float a = v[i], b = v[i + 1];
+        v[i] = a + b;
+        v[i + 1] = a - b;
+    }
+#pragma unroll
+    for (int h = 2; h < 32; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+            if (!(i & h)) {
+                const float2 a = make_float2(v[i], v[i + 1]), b = make_float2(v[i + h], v[i + h + 1]);
+                const float2 s = ptx::fadd2(a, b), d = ptx::fsub2(a, b);
+                v[i] = s.x;
+                v[i + 1] = s.y;
+                v[i + h] = d.x;
+                v[i + h + 1] = d.y;
+            }
+}
+
+// fwht_lanes with the fused multiply-adds in packed pairs.
+template <int SPAN>
+__device__ __forceinline__ void fwht_lanes_pairs(float (&v)[32], int sub) {
+#pragma unroll
+    for (int m = 1; m < SPAN; m <<= 1) {
+        const float sg = (sub & m) ? -1.0f : 1.0f;  // upper lane: p - v, lower lane: v + p
+        const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+            const float2 p = make_float2(__shfl_xor_sync(kFullMask, v[i], m), __shfl_xor_sync(kFullMask, v[i + 1], m));
+            const float2 r = ptx::ffma2(make_float2(v[i], v[i + 1]), sg2, p);
+            v[i] = r.x;
+            v[i + 1] = r.y;
+        }
+    }
+}
+
+// Turbo encode through the code grid (shared copy `grid`); x holds the
+// lane's 32 coordinates with the rotation signs already applied.
+template <int D, int BITS>
+__device__ __forceinline__ void turbo_encode_grid(const QuantSide& s, const uint2* grid, float (&x)[32], int sub,
+                                                  size_t slot, bool valid) {
+    constexpr int LPV = D / 32;
+    float sumsq = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) sumsq = fmaf(x[j], x[j], sumsq);
+    fwht32_pairs(x);
+    fwht_lanes_pairs<LPV>(x, sub);
+    sumsq = group_sum<LPV>(sumsq);
+    const float n = sqrtf(sumsq);
+    const float scale = sqrtf(static_cast<float>(D)) * n;  // y_i = x_i / scale
+    const float inv = n > 0.0f ? s.grid_inv_w / scale : 0.0f;  // grid cells per unit of x
+    uint32_t packed[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        uint32_t acc = 0;
+#pragma unroll
+        for (int e = 7; e >= 0; --e) {
+            const float g = x[8 * k + e] * inv;
+            // round(g) in the low mantissa bits of g + 1.5 * 2^23 (|g| < 64)
+            const uint2 cell = grid[__float_as_uint(g + 12582912.0f) & 127u];
+            const uint32_t code = cell.x + (g > __uint_as_float(cell.y) ? 1u : 0u);
+            acc = acc * (1u << BITS) + code;
+        }
+        packed[k] = acc;
+    }
+    if (valid) {
+        uint8_t* row = s.codes + slot * static_cast<size_t>(s.vbytes);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) store_chunk_codes<BITS>(row, sub + LPV * k, packed[k]);
+        if (sub == 0) s.norms[slot] = float_to_half_bits(n);
+    }
+    if (s.m > 0) {  // QJL residual sketch (keys only)
+        const float rinv = n > 0.0f ? 1.0f / scale : 0.0f;
+        float g2 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const uint32_t code = (packed[i >> 3] >> (BITS * (i & 7))) & ((1u << BITS) - 1u);
+            x[i] = x[i] * rinv - s.centroids[code];  // residual r_i = y_i - c[code_i]
+            g2 = fmaf(x[i], x[i], g2);
+        }
+        g2 = group_sum<LPV>(g2);
+        uint32_t word = 0;
+        for (int r = 0; r < s.m; ++r) {
+            const float* row = s.sketch + static_cast<size_t>(r) * D;
+            float acc = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float4 a = __ldg(reinterpret_cast<const float4*>(row + 8 * (sub + LPV * k)));
+                const float4 b = __ldg(reinterpret_cast<const float4*>(row + 8 * (sub + LPV * k) + 4));
+                acc = fmaf(a.x, x[8 * k + 0], acc); acc = fmaf(a.y, x[8 * k + 1], acc);
+                acc = fmaf(a.z, x[8 * k + 2], acc); acc = fmaf(a.w, x[8 * k + 3], acc);
+                acc = fmaf(b.x, x[8 * k + 4], acc); acc = fmaf(b.y, x[8 * k + 5], acc);
+                acc = fmaf(b.z, x[8 * k + 6], acc); acc = fmaf(b.w, x[8 * k + 7], acc);
+            }
+            acc = group_sum<LPV>(acc);
+            word |= static_cast<uint32_t>(acc >= 0.0f) << (r & 31);
+            if ((r & 31) == 31) {
+                if (valid && sub == 0)
+                    reinterpret_cast<uint32_t*>(s.qjl + slot * static_cast<size_t>(s.m / 8))[r >> 5] = word;
+                word = 0;
+            }
+        }
+        if (valid && sub == 0) s.gamma[slot] = float_to_half_bits(sqrtf(g2));
+    }
 }
 
 // Rotation signs of this lane's 32 coordinates 8 (sub + LPV k) + e, as bit
@@ -200,26 +330,36 @@ __device__ __forceinline__ void int8_encode(const QuantSide& s, const float (&x)
 }
 
 template <int D, int DTYPE>
-__global__ void __launch_bounds__(256, 2) quantize_append_kernel(const __grid_constant__ QuantArgs a) {
+__global__ void __launch_bounds__(256, 3) quantize_append_kernel(const __grid_constant__ QuantArgs a) {
     constexpr int LPV = D / 32;  // lanes per vector
     constexpr int VPW = 32 / LPV;  // vectors per warp pass
+    __shared__ uint2 sgrid[128];
     const QuantSide& s = a.side[blockIdx.y];
+    const bool grid_path = s.mode == TQ_MODE_TURBO && s.grid_inv_w > 0.0f;
+    if (grid_path && threadIdx.x < 128) sgrid[threadIdx.x] = s.grid[threadIdx.x];
+    __syncthreads();
     ptx::launch_dependents();    // the next kernel may start launching
     ptx::wait_prerequisites();   // inputs and cache may come from the previous kernel
     const int lane = threadIdx.x & 31, sub = lane % LPV, grp = lane / LPV;
     const uint32_t smask = lane_sign_mask<D>(a.signs, sub);
-    const long long total = static_cast<long long>(a.batch) * a.n_new * a.hkv;
+    // bf16 inputs: the rotation signs of word i of chunk k (coordinates
+    // 8 k + 2 i and 8 k + 2 i + 1) at bits 15 and 31, applied to the raw words
+    uint32_t sw[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        sw[i] = (((smask >> (2 * i)) & 1u) << 15) | (((smask >> (2 * i + 1)) & 1u) << 31);
     const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
     for (long long base = (static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32) * VPW;
-         base < total; base += nwarps * VPW) {
-        const long long v = base + grp;
-        bool valid = v < total;
+         base < a.total; base += nwarps * VPW) {
+        const uint32_t v = static_cast<uint32_t>(base) + grp;
+        bool valid = v < a.total;
         size_t slot = 0;
         if (valid) {
-            const int h = static_cast<int>(v % a.hkv);
-            const long long bt = v / a.hkv;
-            const int t = static_cast<int>(bt % a.n_new);
-            const int b = static_cast<int>(bt / a.n_new);
+            const uint32_t bt = div_magic(v, a.hkv_magic);
+            const int h = static_cast<int>(v - bt * static_cast<uint32_t>(a.hkv));
+            const uint32_t b32 = div_magic(bt, a.n_new_magic);
+            const int t = static_cast<int>(bt - b32 * static_cast<uint32_t>(a.n_new));
+            const int b = static_cast<int>(b32);
             const int pos = a.positions[b] - (a.pos_from_lens ? a.n_new : 0);
             if (pos < 0 || pos > a.capacity - a.n_new) {
                 if (a.err && t == 0 && h == 0 && sub == 0 && blockIdx.y == 0) atomicOr(a.err, TQ_DEVERR_POSITION);
@@ -238,16 +378,42 @@ __global__ void __launch_bounds__(256, 2) quantize_append_kernel(const __grid_co
             }
         }
         float x[32];
-        if (v < total) {
+        if (DTYPE == 1 && grid_path) {
+            // raw bf16 words with the rotation signs flipped in place
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                load8_stream<DTYPE>(s.src, static_cast<size_t>(v) * D + 8 * (sub + LPV * k), &x[8 * k]);
+            for (int k = 0; k < 4; ++k) {
+                uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                if (v < a.total)
+                    w = __ldcs(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(s.src) +
+                                                              static_cast<size_t>(v) * D + 8 * (sub + LPV * k)));
+                const uint32_t ws[4] = {w.x ^ sw[4 * k], w.y ^ sw[4 * k + 1], w.z ^ sw[4 * k + 2], w.w ^ sw[4 * k + 3]};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    x[8 * k + 2 * i] = __uint_as_float(ws[i] << 16);
+                    x[8 * k + 2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
+                }
+            }
         } else {
+            if (v < a.total) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = 0.0f;
+                for (int k = 0; k < 4; ++k)
+                    load8_stream<DTYPE>(s.src, static_cast<size_t>(v) * D + 8 * (sub + LPV * k), &x[8 * k]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] = 0.0f;
+            }
+            if (grid_path) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    x[j] = __uint_as_float(__float_as_uint(x[j]) ^ ((smask << (31 - j)) & 0x80000000u));
+            }
         }
         if (s.mode == TQ_MODE_INT8) {
             int8_encode<D>(s, x, sub, slot, valid);
+        } else if (grid_path) {
+            if (s.bits == 4) turbo_encode_grid<D, 4>(s, sgrid, x, sub, slot, valid);
+            else if (s.bits == 3) turbo_encode_grid<D, 3>(s, sgrid, x, sub, slot, valid);
+            else turbo_encode_grid<D, 2>(s, sgrid, x, sub, slot, valid);
         } else if (s.bits == 4) {
             turbo_encode<D, 4>(s, x, sub, slot, valid, smask);
         } else if (s.bits == 3) {
@@ -349,12 +515,43 @@ static void fill_side(QuantSide& s, int mode, int bits, int d, const tq_codebook
     s.vbytes = vector_bytes(mode, bits, d);
     for (int j = 0; j < 16; ++j) s.centroids[j] = 0.0f;
     for (int j = 0; j < 8; ++j) s.pos_boundaries[j] = INFINITY;
+    s.grid_inv_w = 0.0f;
     if (mode == TQ_MODE_TURBO) {
         const int n = 1 << bits, half = n / 2;
         for (int j = 0; j < n; ++j) s.centroids[j] = static_cast<float>(cb->centroids[j]);
         for (int k = 0; k < half - 1; ++k) s.pos_boundaries[k] = static_cast<float>(cb->boundaries[half + k]);
+        // the code grid: cells no wider than the narrowest code cell; used
+        // only when |y| <= 1 stays within 62.5 cells of zero (else the binary
+        // search below serves)
+        double w = INFINITY;
+        for (int j = 0; j + 1 < n - 1; ++j) w = std::min(w, cb->boundaries[j + 1] - cb->boundaries[j]);
+        if (n == 2) w = 1.0;  // (not a width the codebooks produce: one boundary, at zero)
+        w *= 1.0 - 1e-6;
+        bool ok = 1.0 / w < 62.5;
+        for (int idx = 0; ok && idx < 128; ++idx) {
+            const int c = idx < 64 ? idx : idx - 128;
+            const double lo = (c - 0.5) * w, hi = (c + 0.5) * w;
+            uint32_t below = 0;
+            int inside = -1;
+            for (int j = 0; j < n - 1; ++j) {
+                const double t = cb->boundaries[j];
+                if (t < lo) ++below;
+                else if (t < hi) {
+                    if (inside >= 0) ok = false;  // two boundaries in a cell
+                    inside = j;
+                }
+            }
+            const float bnd = inside >= 0 ? static_cast<float>(cb->boundaries[inside] / w) : INFINITY;
+            uint32_t bits32;
+            std::memcpy(&bits32, &bnd, 4);
+            s.grid[idx] = make_uint2(below, bits32);
+        }
+        if (ok) s.grid_inv_w = static_cast<float>(1.0 / w);
     }
 }
+
+// ceil(2^64 / d) for the quotients of div_magic; 0 for d = 1.
+static uint64_t quotient_magic(uint32_t d) { return d <= 1 ? 0 : UINT64_MAX / d + 1; }
 
 int num_sms_current() {  // SM count of the current device, 0 if unknown
     int dev = 0, sms = 0;
@@ -366,7 +563,7 @@ int num_sms_current() {  // SM count of the current device, 0 if unknown
 template <int D, int DTYPE>
 static cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t stream) {
     constexpr int VPW = 32 / (D / 32);
-    const long long total = static_cast<long long>(a.batch) * a.n_new * a.hkv;
+    const long long total = a.total;
     const long long warps_needed = (total + VPW - 1) / VPW;
     const int sms = num_sms_current();
     long long blocks = (warps_needed + 7) / 8;
@@ -459,6 +656,13 @@ tq_status tq::quantize_append_impl(const tq_params* params, const tq_codebook* k
     a.batch = pm ? pm->batch : cache->batch;
     a.n_new = n_new;
     a.hkv = p.num_kv_heads;
+    {
+        const long long total = static_cast<long long>(a.batch) * n_new * p.num_kv_heads;
+        if (total >= (1ll << 32)) return TQ_ERR_INVALID_ARG;
+        a.total = static_cast<uint32_t>(total);
+        a.hkv_magic = quotient_magic(static_cast<uint32_t>(p.num_kv_heads));
+        a.n_new_magic = quotient_magic(static_cast<uint32_t>(n_new));
+    }
     a.capacity = capacity;
     if (pm) {
         a.table = pm->table;
