@@ -537,7 +537,18 @@ def prefill_chunk(dev, reps=10):
             "us_per_call": round(us, 2), "tokens_per_s": round(n_new / (us * 1e-6)),
             "attention_tflops": round(tflops, 1), "peak_tflops": peak_tf, "peak_kind": peak_kind,
             "frac_of_peak": round(tflops / peak_tf, 4), "algorithmic_flops": flops,
+            "traffic": profiled_traffic("prefill_kernel", 1),
             "kernels": "tq_prefill_attention: quantise-append of the chunk, then the tcgen05 attention kernel"}
+
+
+class EagerWork:
+    """Stands in for a captured CUDA graph: replay() enqueues the work."""
+
+    def __init__(self, fn):
+        self.fn = fn
+
+    def replay(self):
+        self.fn()
 
 
 def run_tq(args, world, rank, local):
@@ -589,17 +600,25 @@ def run_tq(args, world, rank, local):
                 tq.tq_append_decode_attention(params[l], kcb, vcb, k_new[l][:, i:i + 1], v_new[l][:, i:i + 1],
                                               qs[l][i], caches[l], lens[i], cap, outs[l], ws, err, stream=stream)
 
-    # one CUDA graph per step (the pointers of step i are baked in)
+    # one CUDA graph per step (the pointers of step i are baked in); --eager
+    # enqueues the same launches directly instead (for profilers that cannot
+    # follow graph kernel nodes)
     graphs = []
     with torch.cuda.stream(stream):
         for i in range(total_steps):
+            if args.eager:
+                graphs.append(EagerWork(lambda i=i: enqueue_step(i)))
+                continue
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 enqueue_step(i)
             graphs.append(g)
-        g_decode = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_decode, stream=stream):
-            enqueue_step(total_steps - 1, decode_only=True)
+        if args.eager:
+            g_decode = EagerWork(lambda: enqueue_step(total_steps - 1, decode_only=True))
+        else:
+            g_decode = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_decode, stream=stream):
+                enqueue_step(total_steps - 1, decode_only=True)
     torch.cuda.synchronize()
 
     for i in range(warmup):
@@ -665,12 +684,18 @@ def run_tq(args, world, rank, local):
     s_in = torch.empty(LAYERS * per_layer, dtype=torch.bfloat16, device=dev)
     s_k, s_v, s_q = layer_views(s_in)
     last = total_steps - 1
-    g_e2e = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        with torch.cuda.graph(g_e2e, stream=stream):
-            for l in range(LAYERS):
-                tq.tq_append_decode_attention(params[l], kcb, vcb, s_k[l], s_v[l], s_q[l], caches[l], lens[last], cap,
-                                              outs[l], ws, err, stream=stream)
+    def e2e_layers():
+        for l in range(LAYERS):
+            tq.tq_append_decode_attention(params[l], kcb, vcb, s_k[l], s_v[l], s_q[l], caches[l], lens[last], cap,
+                                          outs[l], ws, err, stream=stream)
+
+    if args.eager:
+        g_e2e = EagerWork(e2e_layers)
+    else:
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g_e2e, stream=stream):
+                e2e_layers()
     torch.cuda.synchronize()
     h2d = h_in.numel() * h_in.element_size()
     d2h = h_out.numel() * h_out.element_size()
@@ -701,7 +726,8 @@ def run_tq(args, world, rank, local):
                        "layers": LAYERS, "parallelism": "replicas%d" % world if world > 1 else "none",
                        "l2": "inputs larger than L2: 32 distinct layer caches, %.0f MB" %
                              (LAYERS * HKV * seq * bytes_per_token_head() / 1e6),
-                       "graphs": "one CUDA graph per step: 32 x tq_append_decode_attention (append + attend, one kernel per layer)"},
+                       "graphs": ("eager launches (--eager): " if args.eager else "one CUDA graph per step: ") +
+                                 "32 x tq_append_decode_attention (append + attend, one kernel per layer)"},
             "hbm_gbs": alg_bytes * LAYERS / (ms / steps * 1e-3) / 1e9,
             "pct_of_8tbs": 100.0 * alg_bytes * LAYERS / (ms / steps * 1e-3) / 8e12,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -760,6 +786,29 @@ def run_profile_case(args):
         out = torch.empty(BATCH, PREFILL_CHUNK, HQ, D, dtype=torch.float32, device=dev)
         for _ in range(args.warmup + args.steps):
             tq.tq_prefill_attention(params, kcb, vcb, kn, vn, q, start, pcache, out, err)
+    elif args.profile == "split":
+        # the split-and-combine decode kernels: d = 256 heads (B=1, Hq=32,
+        # Hkv=8, K4/V2), 8192 cached tokens
+        p256 = tq.make_params(256, HQ, HKV, K_BITS, V_BITS, seed=SEED)
+        kc2, vc2 = tq.tq_codebook_init(256, K_BITS), tq.tq_codebook_init(256, V_BITS)
+        t256 = 8192
+        c256 = tq.alloc_cache(p256, 1, t256 + 8, device=dev)
+        k2 = inputs.lognormal_kv(1, t256, HKV, 256, SEED, 0, inputs.K, device=dev)
+        v2 = inputs.lognormal_kv(1, t256, HKV, 256, SEED, 0, inputs.V, device=dev)
+        tq.tq_quantize_append(p256, kc2, vc2, k2, v2, pos[:1], c256, err)
+        q2 = inputs.queries(1, HQ, 256, SEED, device=dev)
+        lens2 = torch.full((1,), t256, dtype=torch.int32, device=dev)
+        ws2 = torch.zeros(tq.tq_decode_workspace_bytes(p256, 1, t256 + 8), dtype=torch.uint8, device=dev)
+        out2 = torch.empty(1, HQ, 256, dtype=torch.float32, device=dev)
+        for _ in range(args.warmup + args.steps):
+            tq.tq_decode_attention(p256, kc2, vc2, q2, c256, lens2, t256 + 8, out2, ws2, err)
+    elif args.profile == "dequantize":
+        # dequantise one sequence's 32768 cached tokens (all kv heads, K and V)
+        tq.tq_quantize_append(params, kcb, vcb, k, v, pos, cache, err)
+        ko = torch.empty(CONTEXT, HKV, D, dtype=torch.float32, device=dev)  # token-major
+        vo = torch.empty(CONTEXT, HKV, D, dtype=torch.float32, device=dev)
+        for _ in range(args.warmup + args.steps):
+            tq.tq_dequantize(params, kcb, vcb, cache, 0, 0, CONTEXT, ko, vo)
     else:
         tq.tq_quantize_append(params, kcb, vcb, k, v, pos, cache, err)
         q = inputs.queries(BATCH, HQ, D, SEED, device=dev)
@@ -781,9 +830,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="enqueue each step's launches directly instead of replaying CUDA graphs")
     ap.add_argument("--quick", action="store_true",
                     help="skip the bf16 baseline and the bulk prefill quantise measurement")
-    ap.add_argument("--profile", choices=["decode", "quantize", "prefill"], default=None,
+    ap.add_argument("--profile", choices=["decode", "quantize", "prefill", "split", "dequantize"], default=None,
                     help="run a small one-layer case for ncu instead of the benchmark")
     args = ap.parse_args()
     if args.profile:

@@ -341,7 +341,7 @@ static tq_status decode_impl(const tq_params* params, const tq_codebook* kcb, co
     }
     const int sms = num_sms_current();
     if (sms <= 0) return TQ_ERR_CUDA;
-    const DecodePlan plan = plan_decode(p, batch, max_seq_len, sms, workspace_bytes);
+    const DecodePlan plan = plan_decode(p, batch, max_seq_len, sms, workspace_bytes, !decode_mma_supported(p));
     if (workspace_bytes < plan.bytes) return TQ_ERR_CAPACITY;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -488,7 +488,8 @@ extern "C" tq_status tq_decode_attention_static(const tq_params* params, const t
     // Reject calls whose partials cannot fit before touching the device.
     const int sms = num_sms_current();
     if (sms <= 0) return TQ_ERR_CUDA;
-    if (plan_decode(*params, cache->batch, max_seq_len, sms, TQ_DECODE_STATIC_SCRATCH_BYTES).bytes >
+    if (plan_decode(*params, cache->batch, max_seq_len, sms, TQ_DECODE_STATIC_SCRATCH_BYTES,
+                    !decode_mma_supported(*params)).bytes >
         TQ_DECODE_STATIC_SCRATCH_BYTES)
         return TQ_ERR_CAPACITY;
     void* scratch = nullptr;

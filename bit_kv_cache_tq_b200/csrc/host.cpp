@@ -274,7 +274,8 @@ static void place_partials(DecodePlan& plan, size_t slots, int head_dim, size_t 
     plan.bytes = plan.off_acc + slots * head_dim * sizeof(float);
 }
 
-DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_sms, size_t workspace_bytes) {
+DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_sms, size_t workspace_bytes,
+                       bool general_kernel) {
     // Split count.  Few long sequences: one wave of equal items, one per SM,
     // when that keeps at least 85% of the SMs busy (every item then carries
     // one prologue and one merge); otherwise a multiple of the SM count where
@@ -298,6 +299,10 @@ DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_s
         n = (want + step - 1) / step * step;
         if (n > most) n = want;
     }
+    // The general split kernel (four warps a block, no persistent
+    // scheduling) hides its load latency only with many blocks: it takes the
+    // finest split the workspace bound allows.
+    if (general_kernel) n = most;
     if (n > most) n = most;
     if (n < 1) n = 1;
     long long len = (max_seq_len + n - 1) / n;

@@ -55,7 +55,10 @@ bool aligned16(const void* ptr);
 int vector_bytes(int mode, int bits, int head_dim);
 // Bytes of the counter region at the front of a workspace of this size.
 size_t counter_region_bytes(size_t workspace_bytes);
-DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_sms, size_t workspace_bytes);
+// general_kernel: the plan is for the general split kernel (not the
+// tensor-core decode kernel).
+DecodePlan plan_decode(const tq_params& p, int batch, int max_seq_len, int num_sms, size_t workspace_bytes,
+                       bool general_kernel);
 // Tensor-core decode path (decode_mma.cu): d = 128; TURBO or INT8 K; TURBO V,
 // or INT8 V beside INT8 K.
 bool decode_mma_supported(const tq_params& p);

@@ -45,11 +45,14 @@ struct QuantSide {
     // codebook): the rotated unit coordinate y is cut into cells of width w
     // (no wider than the narrowest code cell, so a grid cell holds at most one
     // boundary), cell c = round(y / w) covering [(c - 0.5) w, (c + 0.5) w).
-    // Entry c & 127 = {number of boundaries below the cell, the boundary
-    // inside it in cells (bits of an fp32; +inf when none)}: the code of y is
-    // the first plus (y / w > the second).  |y| <= 1 keeps c within +-63.
+    // Entry c & 127 is the fp32 bit pattern of the boundary inside the cell,
+    // in cells, with its 4 low mantissa bits replaced by the number of
+    // boundaries below the cell (the boundary moves by at most 15 ulps); a
+    // cell without a boundary holds +inf's pattern, a NaN once those bits are
+    // set, so it never compares below y.  The code of y is the count plus
+    // (y / w > the boundary).  |y| <= 1 keeps c within +-63.
     float grid_inv_w;
-    uint2 grid[128];
+    uint32_t grid[128];
 };
 
 struct QuantArgs {
@@ -154,7 +157,7 @@ __device__ __forceinline__ void fwht_lanes_pairs(float (&v)[32], int sub) {
 // Turbo encode through the code grid (shared copy `grid`); x holds the
 // lane's 32 coordinates with the rotation signs already applied.
 template <int D, int BITS>
-__device__ __forceinline__ void turbo_encode_grid(const QuantSide& s, const uint2* grid, float (&x)[32], int sub,
+__device__ __forceinline__ void turbo_encode_grid(const QuantSide& s, const uint32_t* grid, float (&x)[32], int sub,
                                                   size_t slot, bool valid) {
     constexpr int LPV = D / 32;
     float sumsq = 0.0f;
@@ -174,8 +177,8 @@ __device__ __forceinline__ void turbo_encode_grid(const QuantSide& s, const uint
         for (int e = 7; e >= 0; --e) {
             const float g = x[8 * k + e] * inv;
             // round(g) in the low mantissa bits of g + 1.5 * 2^23 (|g| < 64)
-            const uint2 cell = grid[__float_as_uint(g + 12582912.0f) & 127u];
-            const uint32_t code = cell.x + (g > __uint_as_float(cell.y) ? 1u : 0u);
+            const uint32_t cell = grid[__float_as_uint(g + 12582912.0f) & 127u];
+            const uint32_t code = (cell & 15u) + (g > __uint_as_float(cell) ? 1u : 0u);
             acc = acc * (1u << BITS) + code;
         }
         packed[k] = acc;
@@ -329,12 +332,13 @@ __device__ __forceinline__ void int8_encode(const QuantSide& s, const float (&x)
     if (sub == 0) s.norms[slot] = __half_as_ushort(scale16);
 }
 
-template <int D, int DTYPE>
-__global__ void __launch_bounds__(256, 3) quantize_append_kernel(const __grid_constant__ QuantArgs a) {
+// One side (K = 0, V = 1: blockIdx.y) of the quantise-append kernel; the side
+// is a template argument so that its fields are static parameter reads.
+template <int D, int DTYPE, int SIDE>
+__device__ __forceinline__ void quantize_side(const QuantArgs& a, uint32_t* sgrid) {
     constexpr int LPV = D / 32;  // lanes per vector
     constexpr int VPW = 32 / LPV;  // vectors per warp pass
-    __shared__ uint2 sgrid[128];
-    const QuantSide& s = a.side[blockIdx.y];
+    const QuantSide& s = a.side[SIDE];
     const bool grid_path = s.mode == TQ_MODE_TURBO && s.grid_inv_w > 0.0f;
     if (grid_path && threadIdx.x < 128) sgrid[threadIdx.x] = s.grid[threadIdx.x];
     __syncthreads();
@@ -422,6 +426,13 @@ __global__ void __launch_bounds__(256, 3) quantize_append_kernel(const __grid_co
             turbo_encode<D, 2>(s, x, sub, slot, valid, smask);
         }
     }
+}
+
+template <int D, int DTYPE>
+__global__ void __launch_bounds__(256, 3) quantize_append_kernel(const __grid_constant__ QuantArgs a) {
+    __shared__ uint32_t sgrid[128];
+    if (blockIdx.y == 0) quantize_side<D, DTYPE, 0>(a, sgrid);
+    else quantize_side<D, DTYPE, 1>(a, sgrid);
 }
 
 // ------------------------------------------------------------- dequantise
@@ -544,7 +555,7 @@ static void fill_side(QuantSide& s, int mode, int bits, int d, const tq_codebook
             const float bnd = inside >= 0 ? static_cast<float>(cb->boundaries[inside] / w) : INFINITY;
             uint32_t bits32;
             std::memcpy(&bits32, &bnd, 4);
-            s.grid[idx] = make_uint2(below, bits32);
+            s.grid[idx] = (bits32 & ~15u) | below;
         }
         if (ok) s.grid_inv_w = static_cast<float>(1.0 / w);
     }
