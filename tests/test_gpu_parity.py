@@ -268,6 +268,21 @@ def test_bulk_quantize_turbo_and_int8(d):
         _check_quantized(layer, cache, _to_np(k), _to_np(v))
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("kb,vb", [(2, 3), (3, 4), (4, 2)])
+def test_quantize_codes_every_width(d, kb, vb):
+    """Every (head size, code width) pair through the quantise kernel's code
+    grid: 333 tokens x 8 heads of bf16, K and V codes and norms against the
+    oracle's code rule (2, 3 and 4 bits on each of d = 64, 128, 256)."""
+    t = 333
+    k = inputs.lognormal_kv(1, t, 8, d, seed=9, layer=kb, which=inputs.K)
+    v = inputs.lognormal_kv(1, t, 8, d, seed=9, layer=vb, which=inputs.V)
+    layer = H.Layer(d, 8, 8, k_bits=kb, v_bits=vb, seed=3)
+    cache, st, word = H.gpu_quantize(layer, k, v, t)
+    assert st == tq.TQ_OK and word == 0
+    _check_quantized(layer, cache, _to_np(k), _to_np(v))
+
+
 def test_fp16_inputs_d64_group16():
     layer = H.Layer(64, 32, 2, k_bits=2, v_bits=4, seed=13)
     t = 700

@@ -16,25 +16,27 @@ from oracle import attention as oatt
 pytestmark = pytest.mark.gpu
 
 
-def _prefill_case(layer, starts, n_new, seed, prefill_tokens=None):
+def _prefill_case(layer, starts, n_new, seed, prefill_tokens=None, dtype=torch.bfloat16, expect_word=0,
+                  capacity=None):
     """Cache pre-filled with `starts[b]` tokens per sequence (GPU quantise),
-    then one tq_prefill_attention call appending n_new fresh tokens."""
+    then one tq_prefill_attention call appending n_new fresh tokens (chunk
+    and queries in `dtype`)."""
     bsz, hkv, d = len(starts), layer.hkv, layer.d
-    cap = max(starts) + n_new + 40
+    cap = max(starts) + n_new + 40 if capacity is None else capacity
     pre = max(starts) if prefill_tokens is None else prefill_tokens
     k0 = inputs.lognormal_kv(bsz, max(pre, 1), hkv, d, seed=seed, layer=3, which=inputs.K)
     v0 = inputs.lognormal_kv(bsz, max(pre, 1), hkv, d, seed=seed, layer=3, which=inputs.V)
     cache, st, word = H.gpu_quantize(layer, k0, v0, cap)
     assert st == tq.TQ_OK and word == 0
-    kn = inputs.lognormal_kv(bsz, n_new, hkv, d, seed=seed, layer=3, which=inputs.K, token_offset_seed=5)
-    vn = inputs.lognormal_kv(bsz, n_new, hkv, d, seed=seed, layer=3, which=inputs.V, token_offset_seed=5)
-    q = torch.randn(bsz, n_new, layer.hq, d, generator=torch.Generator().manual_seed(seed)).to(torch.bfloat16)
+    kn = inputs.lognormal_kv(bsz, n_new, hkv, d, seed=seed, layer=3, which=inputs.K, token_offset_seed=5).to(dtype)
+    vn = inputs.lognormal_kv(bsz, n_new, hkv, d, seed=seed, layer=3, which=inputs.V, token_offset_seed=5).to(dtype)
+    q = torch.randn(bsz, n_new, layer.hq, d, generator=torch.Generator().manual_seed(seed)).to(dtype)
     pos = torch.tensor(starts, dtype=torch.int32, device="cuda")
     out = torch.empty(bsz, n_new, layer.hq, d, dtype=torch.float32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     tq.tq_prefill_attention(layer.params, layer.kcb, layer.vcb, kn.cuda(), vn.cuda(), q.cuda(), pos, cache, out, err)
     st, word = tq.tq_read_device_error(err)
-    assert st == tq.TQ_OK and word == 0, (st, word)
+    assert word == expect_word and st == (tq.TQ_OK if expect_word == 0 else tq.TQ_ERR_DEVICE), (st, word)
     return cache, out.cpu().numpy(), q, (kn, vn)
 
 
@@ -95,6 +97,33 @@ def test_prefill_from_an_empty_cache():
     layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=23)
     cache, out, q, _ = _prefill_case(layer, [0], 150, seed=23, prefill_tokens=1)
     worst = _check_rows(layer, cache, out, q, [0])
+    assert worst < H.ATTN_TOL, worst
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16])
+def test_prefill_chunk_and_query_dtypes(dtype):
+    """fp32 and fp16 chunks and queries (the kernel converts on load)."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=26)
+    starts = [260]
+    cache, out, q, (kn, vn) = _prefill_case(layer, starts, 70, seed=26, dtype=dtype)
+    _check_appended_codes(layer, cache, starts, 70, kn, vn)
+    worst = _check_rows(layer, cache, out, q, starts)
+    assert worst < H.ATTN_TOL, worst
+
+
+def test_prefill_flags_a_chunk_past_the_capacity():
+    """A sequence whose chunk would end past the cache's capacity is refused
+    on the device (TQ_DEVERR_POSITION): nothing of it is appended and its
+    output rows are zero; the other sequence is unaffected."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=27)
+    n_new = 60
+    cap = 400 + n_new + 40
+    starts = [400, cap - n_new + 1]
+    cache, out, q, _ = _prefill_case(layer, starts, n_new, seed=27, prefill_tokens=400,
+                                     expect_word=tq.TQ_DEVERR_POSITION, capacity=cap)
+    assert np.all(out[1] == 0.0)
+    assert np.all(cache.k_norms[1, :, cap - n_new:].cpu().numpy().view(np.uint16) == 0)
+    worst = _check_rows(layer, cache, out[:1], q[:1], starts[:1])
     assert worst < H.ATTN_TOL, worst
 
 
