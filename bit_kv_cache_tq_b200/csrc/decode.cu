@@ -498,3 +498,15 @@ extern "C" tq_status tq_decode_attention_static(const tq_params* params, const t
     return tq_decode_attention(params, kcb, vcb, d_q, q_dtype, cache, d_seq_lens, max_seq_len, d_out, scratch,
                                TQ_DECODE_STATIC_SCRATCH_BYTES, nullptr, d_error, stream);
 }
+
+// Fill the counter region of the static array (the words a static call's
+// own zero fill covers, for any batch) with the byte `value`, on `stream`;
+// nothing is allocated.  0 is a full reset; other values stand for whatever
+// an interrupted call could leave there.
+extern "C" tq_status tq_decode_static_fill(uint8_t value, void* stream) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, tq::g_static_scratch) != cudaSuccess) return TQ_ERR_CUDA;
+    const size_t bytes = tq::counter_region_bytes(TQ_DECODE_STATIC_SCRATCH_BYTES);
+    return cudaMemsetAsync(ptr, value, bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess ? TQ_OK
+                                                                                              : TQ_ERR_CUDA;
+}

@@ -32,7 +32,7 @@ EXPORTED = (
     "tq_cache_bytes", "tq_decode_workspace_bytes", "tq_quantize_append", "tq_dequantize",
     "tq_decode_attention", "tq_append_decode_attention", "tq_decode_attention_static", "tq_read_device_error",
     "tq_quantize_append_paged", "tq_decode_attention_paged", "tq_append_decode_attention_paged",
-    "tq_prefill_attention",
+    "tq_prefill_attention", "tq_decode_static_fill",
 )
 
 # Bytes of the library's own decode scratch per device (tq_decode_attention_static).
@@ -97,6 +97,7 @@ _lib.tq_append_decode_attention.argtypes = [_P(tq_params), _P(tq_codebook), _P(t
                                             _P(tq_cache), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p,
                                             ctypes.c_void_p]
+_lib.tq_decode_static_fill.argtypes = [ctypes.c_uint8, ctypes.c_void_p]
 _lib.tq_decode_attention_static.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
                                             ctypes.c_int, _P(tq_cache), ctypes.c_void_p, ctypes.c_int32,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
@@ -302,6 +303,11 @@ def tq_append_decode_attention(params, kcb, vcb, k_new, v_new, q, cache, seq_len
                                          workspace.numel() * workspace.element_size(), _ptr(skip_mask), _ptr(error),
                                          _stream(stream))
     _check(st, "tq_append_decode_attention")
+
+
+def tq_decode_static_fill(value, stream=None):
+    """Fill the static decode array's counter region with the byte `value` (0: reset)."""
+    _check(_lib.tq_decode_static_fill(int(value) & 0xFF, _stream(stream)), "tq_decode_static_fill")
 
 
 def tq_decode_attention_static(params, kcb, vcb, q, cache, seq_lens, max_seq_len, out, error=None, stream=None):

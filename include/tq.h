@@ -438,6 +438,17 @@ tq_status tq_decode_attention_static(const tq_params* params, const tq_codebook*
                                      uint32_t* d_error, void* stream);
 
 /*
+ * Fill the counter region at the front of the static array (every counter
+ * word any tq_decode_attention_static call can use) with the byte `value`,
+ * queued on `stream`; allocates nothing.  0 resets the counters outright (for
+ * a caller that wants the array in a known state, e.g. after an error); any
+ * other value leaves them as an interrupted call could, which the next static
+ * call's own zero fill repairs.  Returns TQ_ERR_CUDA if the fill cannot be
+ * queued.  Races with static calls in flight on other streams.
+ */
+tq_status tq_decode_static_fill(uint8_t value, void* stream);
+
+/*
  * Copy the device error word to *out after the work queued on `stream` so
  * far, waiting at most timeout_ms milliseconds (polling, never blocking
  * indefinitely).  Returns TQ_ERR_TIMEOUT when the wait runs out,

@@ -63,6 +63,27 @@ def test_static_scratch_after_a_rejected_length():
         assert np.array_equal(_static(layer, q, cache, lens), want), lens
 
 
+def test_static_call_repairs_dirty_counters():
+    """Every counter word of the shared array set to 0xFFFFFFFF from the host
+    (the state an interrupted call could leave, made without faulting the
+    GPU): the next static call's own zero fill repairs what it uses, so two
+    calls in a row still match the workspace entry point bit for bit; a fill
+    with 0 resets the array outright."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=33)
+    t = 2200
+    k = inputs.lognormal_kv(2, t, 8, 128, seed=33, layer=33, which=inputs.K)
+    v = inputs.lognormal_kv(2, t, 8, 128, seed=33, layer=33, which=inputs.V)
+    q = inputs.queries(2, 32, 128, seed=33, layer=33)
+    cache, _, _ = H.gpu_quantize(layer, k, v, t)
+    want, st, word = H.gpu_decode(layer, q, cache, [t, 1500])
+    assert st == tq.TQ_OK and word == 0
+    tq.tq_decode_static_fill(0xFF)
+    for _ in range(2):
+        assert np.array_equal(_static(layer, q, cache, [t, 1500]), want)
+    tq.tq_decode_static_fill(0)
+    assert np.array_equal(_static(layer, q, cache, [t, 1500]), want)
+
+
 def test_static_scratch_rejects_calls_beyond_its_size():
     """1024 sequences x 64 query heads need more partials than the array holds;
     the call fails before any device work (the cache pointers are never read)."""
