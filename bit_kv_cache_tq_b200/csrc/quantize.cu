@@ -449,7 +449,12 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const __grid_constant__
     constexpr int VPW = 32 / LPV;
     const QuantSide& s = a.side[blockIdx.y];
     float* out = a.out[blockIdx.y];
-    if (!out) return;
+    if (!out) return;  // (the whole block: one side per block)
+    // the centroids in shared memory: a per-thread index into the kernel
+    // parameters would be served one address at a time
+    __shared__ float scen[16];
+    if (threadIdx.x < 16) scen[threadIdx.x] = s.centroids[threadIdx.x];
+    __syncthreads();
     const int lane = threadIdx.x & 31, sub = lane % LPV, grp = lane / LPV;
     const long long total = static_cast<long long>(a.count) * a.hkv;
     const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
@@ -482,7 +487,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const __grid_constant__
             for (int k = 0; k < 4; ++k) {
                 const uint32_t chunk = valid ? stream_bits(words, nwords, 8 * s.bits * (sub + LPV * k), 8 * s.bits) : 0u;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[8 * k + e] = s.centroids[(chunk >> (s.bits * e)) & mask];
+                for (int e = 0; e < 8; ++e) x[8 * k + e] = scen[(chunk >> (s.bits * e)) & mask];
             }
             if (s.m > 0 && valid) {
                 const float coef = half_bits_to_float(s.gamma[slot]) * sqrtf(0.5f * 3.14159265358979f) / s.m;
