@@ -680,38 +680,78 @@ def run_tq(args, world, rank, local):
         h_k[l].copy_(k_new[l][:, -1:])
         h_v[l].copy_(v_new[l][:, -1:])
         h_q[l].copy_(qs[l][-1])
-    h_out = torch.empty(LAYERS, BATCH, HQ, D, dtype=torch.float32).pin_memory()
-    s_in = torch.empty(LAYERS * per_layer, dtype=torch.bfloat16, device=dev)
-    s_k, s_v, s_q = layer_views(s_in)
+    # Two sets of device inputs and outputs (one CUDA graph each) so that the
+    # copies overlap the kernels: step i's inputs go up on one copy stream
+    # while step i - 1 computes, its outputs come down on another while step
+    # i + 1 computes.  Every step still moves its own inputs and outputs
+    # inside the timed region.
+    h_out = [torch.empty(LAYERS, BATCH, HQ, D, dtype=torch.float32).pin_memory() for _ in range(2)]
+    s_in = [torch.empty(LAYERS * per_layer, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    outs_e = [torch.empty(LAYERS, BATCH, HQ, D, dtype=torch.float32, device=dev) for _ in range(2)]
+    views = [layer_views(x) for x in s_in]
     last = total_steps - 1
-    def e2e_layers():
+
+    def e2e_layers(k):
+        s_k, s_v, s_q = views[k]
         for l in range(LAYERS):
             tq.tq_append_decode_attention(params[l], kcb, vcb, s_k[l], s_v[l], s_q[l], caches[l], lens[last], cap,
-                                          outs[l], ws, err, stream=stream)
+                                          outs_e[k][l], ws, err, stream=stream)
 
-    if args.eager:
-        g_e2e = EagerWork(e2e_layers)
-    else:
-        g_e2e = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
-            with torch.cuda.graph(g_e2e, stream=stream):
-                e2e_layers()
+    g_e2e = []
+    for k in range(2):
+        if args.eager:
+            g_e2e.append(EagerWork(lambda k=k: e2e_layers(k)))
+        else:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    e2e_layers(k)
+            g_e2e.append(g)
     torch.cuda.synchronize()
     h2d = h_in.numel() * h_in.element_size()
-    d2h = h_out.numel() * h_out.element_size()
+    d2h = h_out[0].numel() * h_out[0].element_size()
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    fetched = [torch.cuda.Event() for _ in range(2)]
     e2e_steps = steps
-    with torch.cuda.stream(stream):
-        for it in range(warmup + e2e_steps):
-            if it == warmup:
-                stream.synchronize()
-                f0 = torch.cuda.Event(enable_timing=True)
-                f1 = torch.cuda.Event(enable_timing=True)
-                f0.record(stream)
-            s_in.copy_(h_in, non_blocking=True)
-            g_e2e.replay()
-            h_out.copy_(outs, non_blocking=True)
-        f1.record(stream)
+    for it in range(warmup + e2e_steps):
+        k = it % 2
+        if it == warmup:
+            torch.cuda.synchronize()
+            f0 = torch.cuda.Event(enable_timing=True)
+            f1 = torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            up.wait_event(f0)
+        up.wait_event(computed[k])  # step it - 2 has read this input set
+        with torch.cuda.stream(up):
+            s_in[k].copy_(h_in, non_blocking=True)
+            in_ready[k].record(up)
+        stream.wait_event(in_ready[k])
+        stream.wait_event(fetched[k])  # step it - 2's outputs have left this output set
+        with torch.cuda.stream(stream):  # a graph replays on the current stream
+            g_e2e[k].replay()
+        computed[k].record(stream)
+        down.wait_event(computed[k])
+        with torch.cuda.stream(down):
+            h_out[k].copy_(outs_e[k], non_blocking=True)
+            fetched[k].record(down)
+    stream.wait_event(fetched[(warmup + e2e_steps - 1) % 2])
+    f1.record(stream)
     f1.synchronize()
+    # the same steps with every copy serialised with the kernels on one stream
+    # (reported beside the pipelined figure)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for it in range(e2e_steps):
+            s_in[0].copy_(h_in, non_blocking=True)
+            g_e2e[0].replay()
+            h_out[0].copy_(outs_e[0], non_blocking=True)
+        g1.record(stream)
+    g1.synchronize()
+    serial_ms = max_over_ranks(g0.elapsed_time(g1), world)
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
     e2e_value = world * LAYERS * BATCH * (last + CONTEXT + 1) * e2e_steps / (e2e_ms / 1000.0)
 
@@ -736,7 +776,11 @@ def run_tq(args, world, rank, local):
                          "kernel": "decode kernel timed alone (tq_decode_attention, no append), %.2f us per launch, %d B algorithmic"
                                    % (decode_us, alg_bytes)},
             "cpu_baseline": cpu_info,
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "copies": "every step uploads its inputs (one copy) and downloads its outputs (one copy) inside "
+                              "the timed region, on two copy streams that overlap the previous and next steps' "
+                              "kernels (two sets of device buffers)",
+                    "serial_value": world * LAYERS * BATCH * (last + CONTEXT + 1) * e2e_steps / (serial_ms / 1000.0)},
             "gpu_launches": launches_per_step * steps,
             "clocks": clocks.summary(),
         }
