@@ -489,6 +489,44 @@ def paged_decode(dev, reps=10, copies=4):
 PREFILL_CHUNK = 512
 
 
+def oracle_prefill_sample(seconds_target=8.0):
+    """The fp64 CPU oracle on a bounded sample of the prefill workload: one kv
+    head of the Llama-3-8B-shaped layer, 32768 cached tokens; each unit
+    encodes a 4-token chunk, dequantises the cache and runs the causal
+    attention of the chunk's 4 tokens x 4 query heads.  Returns a cpu_baseline
+    dict in attention GFLOP/s (4 d FLOPs per query head and visible key)."""
+    from oracle import attention as oatt
+    w = OracleDecode(units=1)
+    oq, c = w.oq, 4
+    from bit_kv_cache_tq_b200 import inputs
+    kn = inputs.lognormal_kv(1, c, 1, D, seed=SEED, layer=9, which=inputs.K).float().numpy()[0, :, 0]
+    vn = inputs.lognormal_kv(1, c, 1, D, seed=SEED, layer=9, which=inputs.V).float().numpy()[0, :, 0]
+    g = HQ // HKV
+    q = inputs.queries(1, c * g, D, seed=SEED, layer=9).float().numpy().astype(np.float64).reshape(1, c, g, D)
+    ek, ev = w.caches[0]
+
+    def unit():
+        nk = oq.encode_turbo(kn, w.signs, w.kc, w.kt, K_BITS)
+        nv = oq.encode_turbo(vn, w.signs, w.vc, w.vt, V_BITS)
+        khat = oq.dequantize_turbo(np.concatenate([ek["codes"], nk["codes"]]),
+                                   np.concatenate([ek["norm16"], nk["norm16"]]), w.signs, w.kc)
+        vhat = oq.dequantize_turbo(np.concatenate([ev["codes"], nv["codes"]]),
+                                   np.concatenate([ev["norm16"], nv["norm16"]]), w.signs, w.vc)
+        oatt.prefill_attention(q, khat[None, None], vhat[None, None], [w.context])
+
+    unit()  # warm-up
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds_target:
+        unit()
+        n += 1
+    dt = time.perf_counter() - t0
+    flops = 4.0 * D * g * sum(w.context + j + 1 for j in range(c))
+    val = n * flops / dt / 1e9
+    return {"kind": "oracle", "cores": w.cores(), "value": round(val, 3), "unit": "GFLOP/s",
+            "sample": "%d units, each: encode a %d-token chunk of one kv head, dequantise its %d cached tokens, "
+                      "causal attention of %d queries x %d heads (fp64 numpy); %.1f s" % (n, c, w.context, c, g, dt)}
+
+
 def prefill_chunk(dev, reps=10):
     """Chunked prefill from the compressed cache (tq_prefill_attention): the
     Llama-3-8B-shaped layer (B=1, Hq=32, Hkv=8, d=128, K4/V2) with 32768
@@ -790,6 +828,8 @@ def run_tq(args, world, rank, local):
             line["paged_decode"] = {"workload": "llama3-8b-shaped layer, 32768 tokens, K4/V2, through a block "
                                                 "table (blocks in random order)", **paged_decode(dev)}
             line["prefill"] = prefill_chunk(dev)
+            if not args.no_cpu_baseline:
+                line["prefill"]["cpu_baseline"] = oracle_prefill_sample()
             peak_gbs = measured_peaks()[0]
             q = {"workload": "bulk prefill quantise: 262144 tokens x 8 kv heads, bf16, 32 layers (0, 1, 30, 31 "
                              "int8 per-vector absmax, others K4/V3 turbo), one input slab, 32 distinct outputs",
