@@ -1,7 +1,8 @@
 // Hand-written inline-PTX wrappers for the 5th-generation tensor cores of
-// sm_100a (tcgen05): tensor-memory allocation, MMA from shared-memory
-// descriptors into tensor memory, completion through an mbarrier, and loads
-// from and stores to tensor memory.  Only the forms the prefill kernel uses.
+// sm_100a (tcgen05): tensor-memory allocation, MMA with A in tensor memory
+// and B from a shared-memory descriptor into tensor memory, completion
+// through an mbarrier, and loads from and stores to tensor memory.  Only the
+// forms the prefill kernel uses.
 #pragma once
 
 #include <cstdint>
@@ -42,20 +43,11 @@ __device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence
 // cores (the async proxy) before they read the operands.
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, fp16 inputs, fp32 accumulation; `accum`
-// false overwrites D.  One thread issues it.
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                        bool accum) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(static_cast<uint32_t>(accum))
-        : "memory");
-}
 
-// The same with A read from tensor memory at `a_tmem` (M = 128: row m in lane
-// m; fp16 element k of the row in column k / 2, even k in the low half, so a
-// 16-element K step spans 8 columns).
+// D[tmem] (+)= A[tmem] * B[smem]^T, fp16 inputs, fp32 accumulation; `accum`
+// false overwrites D.  One thread issues it.  A is read from tensor memory at
+// `a_tmem` (M = 128: row m in lane m; fp16 element k of the row in column
+// k / 2, even k in the low half, so a 16-element K step spans 8 columns).
 __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                            bool accum) {
     asm volatile(
@@ -91,24 +83,9 @@ __device__ __forceinline__ void ld_32cols(uint32_t taddr, float (&v)[32]) {
 }
 __device__ __forceinline__ void ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Store 32 consecutive fp32 columns of this thread's tensor-memory lane (the
-// lane layout of ld_32cols).  Wait with st_wait before the values are read by
-// the tensor cores.
-__device__ __forceinline__ void st_32cols(uint32_t taddr, const float (&v)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
-        "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-        "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
-        "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-        : "memory");
-}
-// Raw 32-bit words to 8 or 32 consecutive columns of this thread's lane.
+// Raw 32-bit words to 8 or 16 consecutive columns of this thread's lane (the
+// lane layout of ld_32cols); wait with st_wait before the tensor cores read
+// them.
 __device__ __forceinline__ void st_8cols(uint32_t taddr, const uint32_t (&v)[8]) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
                  "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
@@ -140,16 +117,6 @@ __device__ __forceinline__ void st_16cols(uint32_t taddr, const float (&v)[16]) 
 #pragma unroll
     for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(v[i]);
     st_16cols_u(taddr, r);
-}
-__device__ __forceinline__ void st_32cols_u(uint32_t taddr, const uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
-        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
-        "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
-        "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-        : "memory");
 }
 __device__ __forceinline__ void st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
