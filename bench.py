@@ -527,42 +527,55 @@ def oracle_prefill_sample(seconds_target=8.0):
                       "causal attention of %d queries x %d heads (fp64 numpy); %.1f s" % (n, c, w.context, c, g, dt)}
 
 
-def prefill_chunk(dev, reps=10):
+def prefill_chunk(dev, reps=100, warmup=10, smaller=(128, 32)):
     """Chunked prefill from the compressed cache (tq_prefill_attention): the
     Llama-3-8B-shaped layer (B=1, Hq=32, Hkv=8, d=128, K4/V2) with 32768
     cached tokens and a 512-token chunk appended and attended causally.
     Reports the call (append kernel + attention kernel) and the attention's
     algorithmic tensor work: 4 d FLOPs per (query, head, visible key) for
     Q K^T and P V, against the measured dense bf16 peak, burst (the call is
-    timed alone) and sustained (fp16 operands have the same nominal rate)."""
+    timed alone) and sustained (fp16 operands have the same nominal rate).
+    The smaller chunks after the same 32768 tokens (fewer units of 128 query
+    rows than SMs) are reported beside it."""
     from bit_kv_cache_tq_b200 import inputs, tq
     p = tq.make_params(D, HQ, HKV, K_BITS, V_BITS, seed=SEED)
     kcb, vcb = tq.tq_codebook_init(D, K_BITS), tq.tq_codebook_init(D, V_BITS)
-    n_new, start = PREFILL_CHUNK, CONTEXT
-    cache = tq.alloc_cache(p, 1, start + n_new, device=dev)
+    start = CONTEXT
+    cache = tq.alloc_cache(p, 1, start + PREFILL_CHUNK, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     k = inputs.lognormal_kv(1, start, HKV, D, SEED, 70, inputs.K, device=dev)
     v = inputs.lognormal_kv(1, start, HKV, D, SEED, 70, inputs.V, device=dev)
     tq.tq_quantize_append(p, kcb, vcb, k, v, torch.zeros(1, dtype=torch.int32, device=dev), cache, err)
     del k, v
-    kn = inputs.lognormal_kv(1, n_new, HKV, D, SEED, 70, inputs.K, device=dev, token_offset_seed=3)
-    vn = inputs.lognormal_kv(1, n_new, HKV, D, SEED, 70, inputs.V, device=dev, token_offset_seed=3)
-    q = inputs.queries(1, n_new * HQ, D, SEED, layer=70, device=dev).view(1, n_new, HQ, D)
-    pos = torch.full((1,), start, dtype=torch.int32, device=dev)
-    out = torch.empty(1, n_new, HQ, D, dtype=torch.float32, device=dev)
-    for _ in range(3):
-        tq.tq_prefill_attention(p, kcb, vcb, kn, vn, q, pos, cache, out, err)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        tq.tq_prefill_attention(p, kcb, vcb, kn, vn, q, pos, cache, out, err)
-    e1.record()
-    e1.synchronize()
-    st, word = tq.tq_read_device_error(err)
-    assert st == tq.TQ_OK, ("prefill", st, word)
-    us = 1000.0 * e0.elapsed_time(e1) / reps
-    keys = sum(start + j + 1 for j in range(n_new))  # visible keys per (query, head), summed over the chunk
-    flops = 4.0 * D * HQ * keys
+
+    def timed(n_new):
+        # (each call appends the chunk at the same slots, then attends)
+        kn = inputs.lognormal_kv(1, n_new, HKV, D, SEED, 70, inputs.K, device=dev, token_offset_seed=3)
+        vn = inputs.lognormal_kv(1, n_new, HKV, D, SEED, 70, inputs.V, device=dev, token_offset_seed=3)
+        q = inputs.queries(1, n_new * HQ, D, SEED, layer=70, device=dev).view(1, n_new, HQ, D)
+        pos = torch.full((1,), start, dtype=torch.int32, device=dev)
+        out = torch.empty(1, n_new, HQ, D, dtype=torch.float32, device=dev)
+        ws = torch.zeros(tq.tq_prefill_workspace_bytes(p, 1, n_new), dtype=torch.uint8, device=dev)
+        for _ in range(warmup):
+            tq.tq_prefill_attention(p, kcb, vcb, kn, vn, q, pos, cache, out, ws, err)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            tq.tq_prefill_attention(p, kcb, vcb, kn, vn, q, pos, cache, out, ws, err)
+        e1.record()
+        e1.synchronize()
+        st, word = tq.tq_read_device_error(err)
+        assert st == tq.TQ_OK, ("prefill", n_new, st, word)
+        us = 1000.0 * e0.elapsed_time(e1) / reps
+        keys = sum(start + j + 1 for j in range(n_new))  # visible keys per (query, head), summed over the chunk
+        flops = 4.0 * D * HQ * keys
+        return us, flops, flops / (us * 1e-6) / 1e12
+
+    us, flops, tflops = timed(PREFILL_CHUNK)
+    small = []
+    for n in smaller:
+        su, _, st = timed(n)
+        small.append({"chunk": n, "us_per_call": round(su, 2), "attention_tflops": round(st, 1)})
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
             peaks = json.load(fh)
@@ -570,16 +583,19 @@ def prefill_chunk(dev, reps=10):
         sustained_tf = float(peaks["bf16_tflops_sustained"])
     except (OSError, KeyError, ValueError):
         peak_tf, peak_kind, sustained_tf = 1590.0, "fallback", 1400.0
-    tflops = flops / (us * 1e-6) / 1e12
     del cache
     torch.cuda.empty_cache()
-    return {"workload": "llama3-8b-shaped layer, %d cached tokens + a %d-token chunk, K4/V2, causal" % (start, n_new),
-            "us_per_call": round(us, 2), "tokens_per_s": round(n_new / (us * 1e-6)),
+    return {"workload": "llama3-8b-shaped layer, %d cached tokens + a %d-token chunk, K4/V2, causal"
+                        % (start, PREFILL_CHUNK),
+            "us_per_call": round(us, 2), "tokens_per_s": round(PREFILL_CHUNK / (us * 1e-6)),
             "attention_tflops": round(tflops, 1), "peak_tflops": peak_tf, "peak_kind": peak_kind,
             "frac_of_peak": round(tflops / peak_tf, 4), "sustained_peak_tflops": sustained_tf,
             "frac_of_sustained_peak": round(tflops / sustained_tf, 4), "algorithmic_flops": flops,
             "traffic": profiled_traffic("prefill_kernel", 1),
-            "kernels": "tq_prefill_attention: quantise-append of the chunk, then the tcgen05 attention kernel"}
+            "timing": "%d calls after %d warm-up calls, CUDA events" % (reps, warmup),
+            "smaller_chunks": small,
+            "kernels": "tq_prefill_attention: quantise-append of the chunk, then the tcgen05 attention kernel "
+                       "(one block per SM sharing all units' key tiles)"}
 
 
 class EagerWork:
@@ -871,8 +887,9 @@ def run_profile_case(args):
         q = inputs.queries(BATCH, PREFILL_CHUNK * HQ, D, SEED, device=dev).view(BATCH, PREFILL_CHUNK, HQ, D)
         start = torch.full((BATCH,), CONTEXT, dtype=torch.int32, device=dev)
         out = torch.empty(BATCH, PREFILL_CHUNK, HQ, D, dtype=torch.float32, device=dev)
+        ws = torch.zeros(tq.tq_prefill_workspace_bytes(params, BATCH, PREFILL_CHUNK), dtype=torch.uint8, device=dev)
         for _ in range(args.warmup + args.steps):
-            tq.tq_prefill_attention(params, kcb, vcb, kn, vn, q, start, pcache, out, err)
+            tq.tq_prefill_attention(params, kcb, vcb, kn, vn, q, start, pcache, out, ws, err)
     elif args.profile == "split":
         # the split-and-combine decode kernels: d = 256 heads (B=1, Hq=32,
         # Hkv=8, K4/V2), 8192 cached tokens

@@ -16,9 +16,15 @@
 //   s_i = sm_scale ||k_i|| <q~, c[code_i]>,  p = softmax(s),
 //   out = R^-1( sum_i p_i ||v_i|| c[code_i] ).
 //
-// How: one thread block per (sequence, kv head, 128 query rows), a row being
-// one (query token, head of the GQA group), in warp-specialised roles that
-// overlap every stage of a 64-key tile with the tensor cores' work on others.
+// How: the work comes in units of (sequence, kv head, 128 query rows), a row
+// being one (query token, head of the GQA group), each unit a run of 64-key
+// tiles.  One thread block per SM takes an equal share of the sequence of
+// all units' tiles (so a unit can be cut between blocks: each piece's rows
+// go to the workspace as (O, m, l), and the last block to finish a piece of
+// the unit merges them by log-sum-exp); a block runs its share as
+// segments (unit, tile range) in warp-specialised roles that overlap every
+// stage of a tile with the tensor cores' work on others.  (With more units
+// than the schedule holds, each block takes one whole unit.)
 // Shared memory carries only what the tensor cores must read from it (the
 // dequantised key and value tiles); the queries, the scores, the weights and
 // the output accumulator live in tensor memory:
@@ -102,19 +108,32 @@ constexpr uint32_t SM_BAR = SM_CENT + 64;
 // mbarriers (8 bytes each)
 constexpr int B_FULL = 0, B_EMPTY = NS, B_KFULL = 2 * NS, B_KEMPTY = B_KFULL + 2, B_VFULL = B_KEMPTY + 2,
               B_VEMPTY = B_VFULL + 2, B_SFULL = B_VEMPTY + 2, B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2,
-              B_PEMPTY = B_PFULL + 2, B_QREADY = B_PEMPTY + 2, B_FINAL = B_QREADY + 1, NBARS = B_FINAL + 1;
+              B_PEMPTY = B_PFULL + 2, B_QREADY = B_PEMPTY + 2, B_FINAL = B_QREADY + 1, B_PART = B_FINAL + 1,
+              B_PFLAG = B_PART + 1, NBARS = B_PFLAG + 1;
+// (B_PART: the softmax warps have written a cut unit's partial rows;
+// B_PFLAG: thread 0 has published whether this block merges the unit.)
 // (B_PEMPTY[j % 2] also tells that every P V up to tile j is in the accumulator:
 // commits complete in order.  Waiting on it rather than on one shared
 // barrier keeps every wait within one phase of the barrier's state.)
 constexpr uint32_t SM_TMEM = SM_BAR + NBARS * 8;   // tensor-memory address
 constexpr uint32_t SM_FLAG = SM_TMEM + 4;          // abort flag
-constexpr uint32_t SM_KLUT = (SM_FLAG + 4 + 127) & ~127u;  // key code table, one copy per lane
+constexpr uint32_t SM_MFLAG = SM_FLAG + 4;         // "this block merges the unit's partials"
+constexpr uint32_t SM_SEG = (SM_MFLAG + 4 + 15) & ~15u;    // uint32 [4]: the block's g0, g1, g1x, C (spread mode)
+constexpr uint32_t SM_USTART = SM_SEG + 16;                // int: the block's first unit
+// uint32 [NTHREADS]: per-thread tile sums in the prologue, then each thread's
+// segment iterator (kept here, not in a register, through the tile loops)
+constexpr uint32_t SM_SCAN = SM_SEG + 32;
+constexpr uint32_t SM_NPART = SM_SCAN + NTHREADS * 4;      // uint32 [softmax threads]: cut units published
+constexpr int SCHED_MAX = 4096;                            // most units the shared schedule holds
+constexpr uint32_t SM_SCHED = SM_NPART + SOFTMAX_WARPS * 32 * 4;  // uint32 [units + 1]: tiles before each unit
+constexpr uint32_t SM_KLUT = (SM_SCHED + (SCHED_MAX + 1) * 4 + 127) & ~127u;  // key code table, one copy per lane
 // A code table maps a field of two codes (2 BITS bits) to their fp16
 // centroids, packed, with 32 copies interleaved word by word: entry e of lane
 // l is word 32 e + l, so a warp's lookups fall in 32 distinct banks.
 __host__ __device__ constexpr uint32_t lut_bytes(int bits) { return 32u * 4u * (1u << (2 * bits)); }
 __host__ __device__ constexpr uint32_t sm_vlut(int kb) { return SM_KLUT + lut_bytes(kb); }
 __host__ __device__ constexpr uint32_t sm_alloc(int kb, int vb) { return sm_vlut(kb) + lut_bytes(vb) + 1024; }
+static_assert(sm_alloc(4, 4) <= 227u * 1024u, "the largest code tables must fit a block's shared memory");
 
 struct Args {
     const uint8_t* k_codes;
@@ -127,6 +146,10 @@ struct Args {
     uint32_t* err;
     int q_dtype, batch, hq, hkv, group, capacity, n_new, tok_per_tile;
     int staged_norms;        // capacity % 8 == 0: norms ride in the bulk copies
+    int qtiles, units;       // query blocks per (sequence, kv head); units = batch * hkv * qtiles
+    int spread;              // 1: the blocks share the (unit, key tile) sequence evenly (see the kernel)
+    uint32_t* counters;      // [units] segments of a unit merged so far (zero between calls)
+    float* parts;            // [2 * gridDim.x][BM][D + 2] partial outputs of cut units
     float score_scale;       // sm_scale * log2(e) / alpha_k
     float out_scale;         // 1 / (alpha_v * VFOLD)
     uint32_t signs[4];
@@ -155,10 +178,83 @@ __device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-struct Block {
+// One unit of work: 128 query rows (TT tokens x G heads) of one (sequence,
+// kv head); units are numbered (b, kv, qt), qt fastest.
+struct Unit {
     int qt, kv, b, tok0, ntok, start, kend, ntiles;
-    bool bad;
+    bool bad;  // the sequence's chunk position is out of range: no tiles, zero rows
 };
+
+__device__ __forceinline__ Unit unit_of(const Args& a, int u) {
+    Unit x;
+    x.qt = u % a.qtiles;
+    const int bk = u / a.qtiles;
+    x.kv = bk % a.hkv;
+    x.b = bk / a.hkv;
+    x.tok0 = x.qt * a.tok_per_tile;
+    x.start = a.positions[x.b];
+    x.bad = x.start < 0 || x.start > a.capacity - a.n_new;
+    x.ntok = x.bad ? 0 : min(a.tok_per_tile, a.n_new - x.tok0);
+    x.kend = x.ntok > 0 ? x.start + x.tok0 + x.ntok : 0;  // keys [0, kend) are needed by some row
+    x.ntiles = (x.kend + BK - 1) / BK;
+    return x;
+}
+
+// The block's share of the work as segments (unit, key tiles [j0, j1)),
+// one per call.  The iterator (the first unit not yet visited) is the
+// shared word at `slot`, so that it takes no register through the tile
+// loops; segment_unit(slot) is the unit of the segment last returned.  Spread mode: the
+// units' tiles form one sequence (P[u] tiles before unit u); with
+// C = min(blocks, total) sharing, block c takes tiles
+// [c total / C, (c + 1) total / C) of it, so a unit can be cut between
+// blocks; a unit without tiles goes to the block whose range holds its
+// start (the last block for those at the very end).  Otherwise block c is
+// unit c, whole.
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// This block's key tiles [j0, j1) of unit u (one the block visits).
+__device__ __forceinline__ void segment_bounds(const Args& a, const uint8_t* smem, int u, int& j0, int& j1) {
+    if (!a.spread) {
+        j0 = 0;
+        j1 = unit_of(a, u).ntiles;
+        return;
+    }
+    const volatile uint32_t* seg = reinterpret_cast<const volatile uint32_t*>(smem + SM_SEG);
+    const volatile uint32_t* P = reinterpret_cast<const volatile uint32_t*>(smem + SM_SCHED);
+    const uint32_t pu = P[u], pn = P[u + 1], g0 = seg[0], g1 = seg[1];
+    j0 = static_cast<int>((pu > g0 ? pu : g0) - pu);
+    j1 = static_cast<int>((pn < g1 ? pn : g1) - pu);
+}
+
+__device__ __forceinline__ bool next_segment(const Args& a, const uint8_t* smem, uint32_t slot, int& j0, int& j1) {
+    const int it = static_cast<int>(ptx::lds32(slot));
+    if (it >= a.units || (!a.spread && it != static_cast<int>(blockIdx.x))) return false;
+    // (a unit starting at or past the range's end, g1x, belongs to a later block)
+    if (a.spread && reinterpret_cast<const volatile uint32_t*>(smem + SM_SCHED)[it] >=
+                        reinterpret_cast<const volatile uint32_t*>(smem + SM_SEG)[2])
+        return false;
+    segment_bounds(a, smem, it, j0, j1);
+    sts32(slot, static_cast<uint32_t>(it + 1));
+    return true;
+}
+
+// The unit of the segment that next_segment returned last.
+__device__ __forceinline__ int segment_unit(uint32_t slot) { return static_cast<int>(ptx::lds32(slot)) - 1; }
+
+// Whether unit u, which has tiles in this block, has some in another block too.
+__device__ __forceinline__ bool unit_is_cut(const Args& a, const uint8_t* smem, int u) {
+    if (!a.spread) return false;
+    const volatile uint32_t* seg = reinterpret_cast<const volatile uint32_t*>(smem + SM_SEG);
+    const volatile uint32_t* P = reinterpret_cast<const volatile uint32_t*>(smem + SM_SCHED);
+    return P[u] < seg[0] || P[u + 1] > seg[1];
+}
+
+// The block whose range holds global tile g (spread mode, g < total).
+__device__ __forceinline__ int block_of(uint32_t g, uint32_t total, uint32_t nblocks) {
+    return static_cast<int>(((static_cast<uint64_t>(g) + 1) * nblocks - 1) / total);
+}
 
 // The code table of BITS-bit codes: field e (code e & m, then code e >> BITS)
 // -> fp16 centroid pair, for every lane.
@@ -259,19 +355,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         }
         return true;
     };
-
-    Block blk;
-    blk.qt = blockIdx.x;
-    blk.kv = blockIdx.y;
-    blk.b = blockIdx.z;
     const int G = a.group, TT = a.tok_per_tile;
-    blk.tok0 = blk.qt * TT;
-    blk.start = a.positions[blk.b];
-    blk.bad = blk.start < 0 || blk.start > a.capacity - a.n_new;
-    blk.ntok = blk.bad ? 0 : min(TT, a.n_new - blk.tok0);
-    blk.kend = blk.ntok > 0 ? blk.start + blk.tok0 + blk.ntok : 0;  // keys [0, kend) are needed by some row
-    blk.ntiles = (blk.kend + BK - 1) / BK;
-    const int T = blk.ntiles;
 
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) {
@@ -290,6 +374,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         }
         ptx::mbar_init(bar(B_QREADY), SOFTMAX_WARPS);
         ptx::mbar_init(bar(B_FINAL), 1);
+        ptx::mbar_init(bar(B_PART), SOFTMAX_WARPS);
+        ptx::mbar_init(bar(B_PFLAG), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -298,53 +384,141 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         tc::tmem_alloc(sbase + SM_TMEM, TMEM_COLS);
         tc::tmem_relinquish();
     }
-    if (blk.bad && blk.qt == 0 && blk.kv == 0 && tid == 0 && a.err) atomicOr(a.err, TQ_DEVERR_POSITION);
+    // ---- the schedule (spread mode): P[u] = tiles of the units before u,
+    // from per-thread sums over contiguous runs of units and a scan of those
+    uint32_t* P = reinterpret_cast<uint32_t*>(smem + SM_SCHED);
+    uint32_t* scan = reinterpret_cast<uint32_t*>(smem + SM_SCAN);
+    const int U = a.units;
+    const int per = (U + NTHREADS - 1) / NTHREADS, u0 = tid * per, u1 = min(U, u0 + per);
+    if (a.spread) {
+        uint32_t sum = 0;
+        for (int u = u0; u < u1; ++u) sum += static_cast<uint32_t>(unit_of(a, u).ntiles);
+        scan[tid] = sum;
+    }
+    __syncthreads();
+    if (a.spread && warp == 0) {  // exclusive scan of the NTHREADS sums
+        constexpr int PER_LANE = NTHREADS / 32;
+        uint32_t v[PER_LANE], t = 0;
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i) {
+            v[i] = scan[lane * PER_LANE + i];
+            t += v[i];
+        }
+        uint32_t incl = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        uint32_t run = incl - t;
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i) {
+            scan[lane * PER_LANE + i] = run;
+            run += v[i];
+        }
+    }
+    __syncthreads();
+    if (a.spread) {
+        uint32_t run = scan[tid];
+        for (int u = u0; u < u1; ++u) {
+            P[u] = run;
+            run += static_cast<uint32_t>(unit_of(a, u).ntiles);
+        }
+        if (u1 == U && u0 < u1) P[U] = run;
+        if (U == 0 && tid == 0) P[0] = 0;
+    }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + SM_TMEM);
-    const size_t unit_row = (static_cast<size_t>(blk.b) * a.hkv + blk.kv) * a.capacity;
     constexpr int kbytes = 16 * KB, vbytes = 16 * VB;  // packed row sizes
+
+    // this block's range of the tile sequence, and its first unit
+    if (tid == 0) {
+        const int cb = static_cast<int>(blockIdx.x);
+        int ustart = cb;
+        if (a.spread) {
+            // (the host spreads only while the tile total fits 31 bits)
+            const uint32_t total = P[U];
+            // no more sharing blocks than tiles: each one's range then holds at
+            // least one tile, so a cut unit's pieces are in every block from its
+            // first to its last; the blocks past C take nothing
+            const uint32_t C = gridDim.x > total ? (total > 0 ? total : 1u) : gridDim.x;
+            uint32_t* seg = reinterpret_cast<uint32_t*>(smem + SM_SEG);
+            const uint32_t c = static_cast<uint32_t>(cb);
+            const uint32_t g0 = static_cast<uint32_t>(static_cast<uint64_t>(c) * total / C);
+            const uint32_t g1 = static_cast<uint32_t>(static_cast<uint64_t>(c + 1) * total / C);
+            seg[0] = g0;
+            seg[1] = g1;
+            seg[2] = c == C - 1 ? total + 1 : g1;
+            seg[3] = C;
+            if (c >= C) {
+                ustart = U;
+            } else {
+                int lo = 0, hi = U;  // first u with P[u + 1] > g0 or P[u] >= g0
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (P[mid + 1] > g0 || P[mid] >= g0) hi = mid;
+                    else lo = mid + 1;
+                }
+                ustart = lo;
+            }
+        }
+        *reinterpret_cast<int*>(smem + SM_USTART) = ustart;
+    }
+    __syncthreads();
+    // each thread's segment iterator (its prologue scan word is free now)
+    const uint32_t slot = sbase + SM_SCAN + 4u * static_cast<uint32_t>(tid);
+    sts32(slot, static_cast<uint32_t>(*reinterpret_cast<volatile int*>(smem + SM_USTART)));
 
     if (warp == PRODUCER / 32) {
         // ---------------------------------------------------------- producer
         // the whole warp waits; one elected lane issues the copies
         const bool leader = tc::elect_one();
-        int issued = 0;
-        for (int j = 0; j < T; ++j) {
-            const int s = j % NS;
-            // (the ring is four tiles deep: the producer can poll slowly and
-            // leave the issue slots of its sub-partition to the working warps)
-            if (j >= NS) {
-                if (*abort_flag) break;
-                if (!ptx::mbar_wait_bounded_sleep(bar(B_EMPTY + s), ((j - NS) / NS) & 1, WAIT_LIMIT, 256)) {
-                    fail();
-                    break;
+        int gi = 0;  // tiles issued so far (the ring position)
+        int j0, j1;
+        while (next_segment(a, smem, slot, j0, j1)) {
+            const Unit x = unit_of(a, segment_unit(slot));
+            // ring tile g holds the unit's keys from g BK - koff (koff = (gi - j0) BK)
+            const int koff = (gi - j0) * BK, kend = x.kend + koff;
+            const long long row0 = static_cast<long long>((static_cast<size_t>(x.b) * a.hkv + x.kv) * a.capacity) - koff;
+            for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
+                const int s = gi % NS;
+                // (the ring is four tiles deep: the producer can poll slowly and
+                // leave the issue slots of its sub-partition to the working warps)
+                if (gi >= NS) {
+                    if (*abort_flag) goto produced;
+                    if (!ptx::mbar_wait_bounded_sleep(bar(B_EMPTY + s), ((gi - NS) / NS) & 1, WAIT_LIMIT, 256)) {
+                        fail();
+                        goto produced;
+                    }
                 }
-            }
-            if (leader) {
-                const int key0 = j * BK, nk = min(BK, blk.kend - key0);
-                const uint32_t dst = sbase + SM_STAGE + s * STAGE_BYTES;
-                const int n8 = (nk + 7) & ~7;  // norms move in 16-byte pieces (8 keys)
-                const uint32_t bytes = nk * (kbytes + vbytes) + (a.staged_norms ? n8 * 4 : 0);
-                ptx::mbar_arrive_expect_tx(bar(B_FULL + s), bytes);
-                ptx::bulk_copy_g2s(dst + ST_KC, a.k_codes + (unit_row + key0) * kbytes, nk * kbytes, bar(B_FULL + s));
-                ptx::bulk_copy_g2s(dst + ST_VC, a.v_codes + (unit_row + key0) * vbytes, nk * vbytes, bar(B_FULL + s));
-                if (a.staged_norms) {
-                    // capacity and key0 are multiples of 8: the rounded range stays inside the cache
-                    ptx::bulk_copy_g2s(dst + ST_KN, a.k_norms + unit_row + key0, n8 * 2, bar(B_FULL + s));
-                    ptx::bulk_copy_g2s(dst + ST_VN, a.v_norms + unit_row + key0, n8 * 2, bar(B_FULL + s));
+                if (leader) {
+                    const int key0 = gi * BK, nk = min(BK, kend - key0);
+                    const size_t row = static_cast<size_t>(row0 + key0);
+                    const uint32_t dst = sbase + SM_STAGE + s * STAGE_BYTES;
+                    const int n8 = (nk + 7) & ~7;  // norms move in 16-byte pieces (8 keys)
+                    const uint32_t bytes = nk * (kbytes + vbytes) + (a.staged_norms ? n8 * 4 : 0);
+                    ptx::mbar_arrive_expect_tx(bar(B_FULL + s), bytes);
+                    ptx::bulk_copy_g2s(dst + ST_KC, a.k_codes + row * kbytes, nk * kbytes, bar(B_FULL + s));
+                    ptx::bulk_copy_g2s(dst + ST_VC, a.v_codes + row * vbytes, nk * vbytes, bar(B_FULL + s));
+                    if (a.staged_norms) {
+                        // capacity and the unit's key offset are multiples of 8: the
+                        // rounded range stays inside the cache
+                        ptx::bulk_copy_g2s(dst + ST_KN, a.k_norms + row, n8 * 2, bar(B_FULL + s));
+                        ptx::bulk_copy_g2s(dst + ST_VN, a.v_norms + row, n8 * 2, bar(B_FULL + s));
+                    }
                 }
+                __syncwarp();
             }
-            __syncwarp();
-            issued = j + 1;
         }
+    produced:
         // every copy issued must land before the block may exit
-        for (int j = max(0, issued - NS); j < issued; ++j)
-            ptx::mbar_wait_bounded(bar(B_FULL + j % NS), (j / NS) & 1, WAIT_LIMIT);
+        for (int k = max(0, gi - NS); k < gi; ++k)
+            ptx::mbar_wait_bounded(bar(B_FULL + k % NS), (k / NS) & 1, WAIT_LIMIT);
     } else if (warp >= DEQ0 / 32 && warp < PRODUCER / 32) {
         // ------------------------------------------------------ dequantisers
-        const int dt = tid - DEQ0;  // 0 .. 255
+        const int dt = tid - DEQ0;  // 0 .. 32 DEQ_WARPS - 1
         const uint16_t* kcent = reinterpret_cast<const uint16_t*>(smem + SM_CENT);
         const uint16_t* vcent = kcent + 16;
         uint32_t* klut = reinterpret_cast<uint32_t*>(smem + SM_KLUT);
@@ -353,36 +527,47 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         build_lut<VB>(vlut, vcent, dt, DEQ_WARPS * 32);
         ptx::named_barrier(1, DEQ_WARPS * 32);
         const uint32_t klane = sbase + SM_KLUT + 4 * lane, vlane = sbase + sm_vlut(KB) + 4 * lane;
-        for (int j = 0; j < T; ++j) {
-            const int s = j % NS, bf = j & 1;
-            if (!wait(B_FULL + s, (j / NS) & 1)) break;
-            const uint8_t* st = smem + SM_STAGE + s * STAGE_BYTES;
-            const uint32_t sst = sbase + SM_STAGE + s * STAGE_BYTES;
-            const int key0 = j * BK, nk = min(BK, blk.kend - key0);
-            const uint16_t* skn = reinterpret_cast<const uint16_t*>(st + ST_KN);
-            // K~[bf]: 64 keys x 16 groups of 8 channels, centroids; the tile's
-            // key norms go to the softmax's ring (its tile j - 4 is done: this
-            // tile's K~ buffer was free only after S(j - 2), which needed the
-            // softmax to be through tile j - 4)
-            if (j >= 2 && !wait(B_KEMPTY + bf, ((j - 2) >> 1) & 1)) break;
-            if (dt < BK)
-                reinterpret_cast<float*>(smem + SM_KNR)[(j & 3) * BK + dt] =
-                    dt < nk ? half_bits_to_float(a.staged_norms ? skn[dt] : a.k_norms[unit_row + key0 + dt]) : 0.f;
-            dequant_tile<KB, false>(sbase + SM_K + bf * (BK * D * 2), sst + ST_KC, klane, 0u, nullptr, true, dt, nk);
-            tc::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar(B_KFULL + bf));
-            // V~[bf]: the same per-key layout, centroids x norms
-            if (j >= 2 && !wait(B_VEMPTY + bf, ((j - 2) >> 1) & 1)) break;
-            dequant_tile<VB, true>(sbase + SM_VT + bf * (BK * D * 2), sst + ST_VC, vlane, sst + ST_VN,
-                                   a.v_norms + unit_row + key0, a.staged_norms != 0, dt, nk);
-            tc::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                ptx::mbar_arrive(bar(B_VFULL + bf));
-                ptx::mbar_arrive(bar(B_EMPTY + s));  // the stage's codes and norms are used
+        int gi = 0;
+        int j0, j1;
+        while (next_segment(a, smem, slot, j0, j1)) {
+            const Unit x = unit_of(a, segment_unit(slot));
+            // ring tile g holds the unit's keys from g BK - koff (as the producer's)
+            const int koff = (gi - j0) * BK, kend = x.kend + koff;
+            const long long row0 = static_cast<long long>((static_cast<size_t>(x.b) * a.hkv + x.kv) * a.capacity) - koff;
+            for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
+                const int s = gi % NS, bf = gi & 1;
+                if (!wait(B_FULL + s, (gi / NS) & 1)) goto dequantised;
+                const uint8_t* st = smem + SM_STAGE + s * STAGE_BYTES;
+                const uint32_t sst = sbase + SM_STAGE + s * STAGE_BYTES;
+                const int key0 = gi * BK, nk = min(BK, kend - key0);
+                const size_t row = static_cast<size_t>(row0 + key0);
+                const uint16_t* skn = reinterpret_cast<const uint16_t*>(st + ST_KN);
+                // K~[bf]: 64 keys x 16 groups of 8 channels, centroids; the tile's
+                // key norms go to the softmax's ring (its tile gi - 4 is done: this
+                // tile's K~ buffer was free only after S(gi - 2), which needed the
+                // softmax to be through tile gi - 4)
+                if (gi >= 2 && !wait(B_KEMPTY + bf, ((gi - 2) >> 1) & 1)) goto dequantised;
+                if (dt < BK)
+                    reinterpret_cast<float*>(smem + SM_KNR)[(gi & 3) * BK + dt] =
+                        dt < nk ? half_bits_to_float(a.staged_norms ? skn[dt] : a.k_norms[row + dt]) : 0.f;
+                dequant_tile<KB, false>(sbase + SM_K + bf * (BK * D * 2), sst + ST_KC, klane, 0u, nullptr, true, dt,
+                                        nk);
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(B_KFULL + bf));
+                // V~[bf]: the same per-key layout, centroids x norms
+                if (gi >= 2 && !wait(B_VEMPTY + bf, ((gi - 2) >> 1) & 1)) goto dequantised;
+                dequant_tile<VB, true>(sbase + SM_VT + bf * (BK * D * 2), sst + ST_VC, vlane, sst + ST_VN,
+                                       a.v_norms + row, a.staged_norms != 0, dt, nk);
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(bar(B_VFULL + bf));
+                    ptx::mbar_arrive(bar(B_EMPTY + s));  // the stage's codes and norms are used
+                }
             }
         }
+    dequantised:;
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------- MMA issuer
         // the whole warp waits; one elected lane issues the MMAs and commits
@@ -392,11 +577,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         // buffers are fixed offsets (in 16-byte units) from these
         const uint64_t kdesc0 = tc::sw128_desc(sbase + SM_K);
         const uint64_t vdesc0 = tc::sw128_mn_desc(sbase + SM_VT, BK * 128, 1024);
-        bool ok = T == 0 || wait(B_QREADY, 0);
-        auto issue_s = [&](int j) -> bool {
-            const int bf = j & 1;
-            if (!wait(B_KFULL + bf, (j >> 1) & 1)) return false;
-            if (j >= 2 && !wait(B_SEMPTY + bf, ((j - 2) >> 1) & 1)) return false;
+        auto issue_s = [&](int gi) -> bool {
+            const int bf = gi & 1;
+            if (!wait(B_KFULL + bf, (gi >> 1) & 1)) return false;
+            if (gi >= 2 && !wait(B_SEMPTY + bf, ((gi - 2) >> 1) & 1)) return false;
             tc::fence_after_sync();
             if (leader) {
                 const uint64_t kd = kdesc0 + static_cast<uint64_t>(bf * (BK * D * 2) >> 4);
@@ -414,10 +598,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
             __syncwarp();
             return true;
         };
-        auto issue_pv = [&](int j) -> bool {
-            const int bf = j & 1;
-            if (!wait(B_PFULL + bf, (j >> 1) & 1)) return false;
-            if (!wait(B_VFULL + bf, (j >> 1) & 1)) return false;
+        // first: the segment's first tile (the accumulator starts afresh)
+        auto issue_pv = [&](int gi, bool first) -> bool {
+            const int bf = gi & 1;
+            if (!wait(B_PFULL + bf, (gi >> 1) & 1)) return false;
+            if (!wait(B_VFULL + bf, (gi >> 1) & 1)) return false;
             tc::fence_after_sync();
             if (leader) {
                 const uint64_t vd = vdesc0 + static_cast<uint64_t>(bf * (BK * D * 2) >> 4);
@@ -427,18 +612,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
 #pragma unroll
                 for (int ks = 0; ks < BK / 16; ++ks)
                     tc::mma_f16_ts(tmem + TM_O, pa + 8 * ks, vd + static_cast<uint64_t>(ks * 2048 >> 4), idesc_o,
-                                   j > 0 || ks > 0);
+                                   !first || ks > 0);
                 tc::commit(bar(B_PEMPTY + bf));
                 tc::commit(bar(B_VEMPTY + bf));
             }
             __syncwarp();
             return true;
         };
-        if (ok && T > 0) ok = issue_s(0);
-        for (int j = 0; ok && j < T; ++j) {
-            if (j + 1 < T && !issue_s(j + 1)) break;
-            if (!issue_pv(j)) break;
+        int gi = 0, qs = 0;  // tiles issued, segments with tiles begun (the QREADY phase)
+        int j0, j1;
+        while (next_segment(a, smem, slot, j0, j1)) {
+            if (j1 <= j0) continue;  // no tiles: the softmax writes the unit's zero rows alone
+            // the segment's queries are in tensor memory (which also tells
+            // that the previous segment's output has been read)
+            if (!wait(B_QREADY, qs & 1)) break;
+            ++qs;
+            if (!issue_s(gi)) break;
+            const int gfirst = gi;
+            for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
+                if (gi + 1 < gend && !issue_s(gi + 1)) goto issued;
+                if (!issue_pv(gi, gi == gfirst)) goto issued;
+            }
         }
+    issued:
         // every tensor-core operation issued completes before the block
         // frees its tensor memory (bounded, also after an abort)
         if (leader) {
@@ -450,189 +646,296 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         // ---------------------------------------------------------- softmax
         const int r = tid;
         const int rt = r / G, rh = r % G;
-        const bool row_ok = rt < blk.ntok && rt * G + rh < BM;
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        float qscale = 0.f;  // largest |q~| of the row: the fp16 terms hold q~ / qscale
-        {
-            float x[D];
-            if (row_ok) {
-                const size_t qoff = ((static_cast<size_t>(blk.b) * a.n_new + blk.tok0 + rt) * a.hq + blk.kv * G + rh) * D;
-#pragma unroll
-                for (int c = 0; c < D; c += 4) {
-                    float v4[4];
-                    load4(a.q, qoff + c, a.q_dtype, v4);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        x[c + e] = flip_sign(v4[e], (a.signs[(c + e) >> 5] >> ((c + e) & 31)) & 1u);
-                }
-                fwht128(x);
-            } else {
-#pragma unroll
-                for (int c = 0; c < D; ++c) x[c] = 0.f;
-            }
-            float amax = 0.f;
-#pragma unroll
-            for (int c = 0; c < D; ++c) amax = fmaxf(amax, fabsf(x[c]));
-            const float inv_sqrt_d = 0.08838834764831845f;
-            qscale = amax * inv_sqrt_d;
-            const float rs = amax > 0.f ? 1.f / amax : 0.f;
-#pragma unroll
-            for (int c = 0; c < D; c += 16) {
-                uint32_t hw[8], lw[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float u0 = x[c + 2 * e] * rs, u1 = x[c + 2 * e + 1] * rs;
-                    const __half h0 = __float2half_rn(u0), h1 = __float2half_rn(u1);
-                    hw[e] = pack2(__half_as_ushort(h0), __half_as_ushort(h1));
-                    lw[e] = half2_bits(u0 - __half2float(h0), u1 - __half2float(h1));
-                }
-                tc::st_8cols(tmem + lane_base + TM_QHI + c / 2, hw);
-                tc::st_8cols(tmem + lane_base + TM_QLO + c / 2, lw);
-            }
-        }
-        tc::st_wait();
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(B_QREADY));
-        // scores in log2 units: S kn rs; a zero query row keeps rs > 0 so that a
-        // masked (-inf) score stays -inf
-        const float rs = fmaxf(qscale * a.score_scale, 1e-30f);
-        const int qpos = blk.start + blk.tok0 + rt;  // this row's own position: the causal limit
-        float mref = -INFINITY, l = 0.f;
-        for (int j = 0; j < T; ++j) {
-            const int bf = j & 1, key0 = j * BK;
-            if (!wait(B_SFULL + bf, (j >> 1) & 1)) break;
-            tc::fence_after_sync();
-            float u[BK];
+        const float inv_sqrt_d = 0.08838834764831845f;
+        // cut units this thread has published so far (the B_PART / B_PFLAG
+        // phase), in shared memory like the iterator
+        sts32(sbase + SM_NPART + 4u * static_cast<uint32_t>(tid), 0u);
+        int gi = 0;  // tiles done (the ring position)
+        int j0, j1;
+        // rows of a unit that exist in the output (all of them but the padding
+        // of a last, partial query block), and this thread's
+        auto out_row = [&](const Unit& x) -> float* {
+            const bool row_out = rt < min(TT, a.n_new - x.tok0) && rt * G + rh < BM;
+            return row_out ? a.out + ((static_cast<size_t>(x.b) * a.n_new + x.tok0 + rt) * a.hq + x.kv * G + rh) * D
+                           : nullptr;
+        };
+        while (next_segment(a, smem, slot, j0, j1)) {
+            // (what the tile loop needs is worked out again after the query's
+            // preparation, which holds a 128-value row: a value kept through
+            // it would be spilled, and reloaded at every tile)
+            float qscale = 0.f;  // largest |q~| of the row: the fp16 terms hold q~ / qscale
             {
-                float (&u0)[32] = *reinterpret_cast<float (*)[32]>(&u[0]);
-                float (&u1)[32] = *reinterpret_cast<float (*)[32]>(&u[32]);
-                tc::ld_32cols(tmem + lane_base + TM_S + BK * bf, u0);
-                tc::ld_32cols(tmem + lane_base + TM_S + BK * bf + 32, u1);
-            }
-            tc::ld_wait();
-            const float4* kn4 = reinterpret_cast<const float4*>(smem + SM_KNR + (j & 3) * BK * 4);
+                const Unit x = unit_of(a, segment_unit(slot));
+                const bool row_ok = rt < x.ntok && rt * G + rh < BM;
+                if (j1 <= j0) {
+                    // no tiles: a sequence whose chunk position was refused (zero rows)
+                    if (x.bad && x.qt == 0 && x.kv == 0 && tid == 0 && a.err) atomicOr(a.err, TQ_DEVERR_POSITION);
+                    float* dst = out_row(x);
+                    if (dst) {
 #pragma unroll
-            for (int i = 0; i < BK; i += 4) {
-                const float4 k4 = kn4[i / 4];
-                const float2 a01 = ptx::fmul2(make_float2(u[i], u[i + 1]), make_float2(k4.x, k4.y));
-                const float2 a23 = ptx::fmul2(make_float2(u[i + 2], u[i + 3]), make_float2(k4.z, k4.w));
-                u[i] = a01.x;
-                u[i + 1] = a01.y;
-                u[i + 2] = a23.x;
-                u[i + 3] = a23.y;
-            }
-            if (key0 + BK - 1 > blk.start + blk.tok0) {
-                // a tile on the diagonal: keys past the row's own position drop
-                // out (rows outside the chunk are never stored; every key of an
-                // earlier tile is visible to every row of the block)
-#pragma unroll
-                for (int i = 0; i < BK; ++i)
-                    if (!row_ok || key0 + i > qpos) u[i] = -INFINITY;
-            }
-            float m4[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float m = u[16 * q];
-#pragma unroll
-                for (int i = 1; i < 15; i += 2) m = ptx::fmax3(m, u[16 * q + i], u[16 * q + i + 1]);
-                m4[q] = fmaxf(m, u[16 * q + 15]);
-            }
-            const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * rs;
-            // lazy reference: moves (and the accumulator is rescaled) only when a
-            // score passes it by more than 2^LAZY; the weights stay below 2^LAZY
-            const bool need = mt > mref + LAZY;
-            if (__any_sync(0xffffffffu, need)) {
-                const float mnew = need ? mt : mref;
-                const float c = (need && mref > -INFINITY) ? ptx::ex2(mref - mnew) : 1.f;
-                if (j > 0) {
-                    // every P V of the earlier tiles is in the accumulator
-                    if (!wait(B_PEMPTY + ((j - 1) & 1), ((j - 1) >> 1) & 1)) break;
-                    tc::fence_after_sync();
-#pragma unroll 1
-                    for (int q8 = 0; q8 < 8; ++q8) {
-                        float ov[16];
-                        tc::ld_16cols(tmem + lane_base + TM_O + 16 * q8, ov);
-                        tc::ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) ov[i] *= c;
-                        tc::st_16cols(tmem + lane_base + TM_O + 16 * q8, ov);
+                        for (int c = 0; c < D; c += 4)
+                            *reinterpret_cast<float4*>(dst + c) = make_float4(0.f, 0.f, 0.f, 0.f);
                     }
+                    continue;
                 }
-                l *= c;
-                mref = mnew;
+                float xq[D];
+                if (row_ok) {
+                    const size_t qoff =
+                        ((static_cast<size_t>(x.b) * a.n_new + x.tok0 + rt) * a.hq + x.kv * G + rh) * D;
+#pragma unroll
+                    for (int c = 0; c < D; c += 4) {
+                        float v4[4];
+                        load4(a.q, qoff + c, a.q_dtype, v4);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            xq[c + e] = flip_sign(v4[e], (a.signs[(c + e) >> 5] >> ((c + e) & 31)) & 1u);
+                    }
+                    fwht128(xq);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < D; ++c) xq[c] = 0.f;
+                }
+                float amax = 0.f;
+#pragma unroll
+                for (int c = 0; c < D; ++c) amax = fmaxf(amax, fabsf(xq[c]));
+                qscale = amax * inv_sqrt_d;
+                const float rsq = amax > 0.f ? 1.f / amax : 0.f;
+#pragma unroll
+                for (int c = 0; c < D; c += 16) {
+                    uint32_t hw[8], lw[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float v0 = xq[c + 2 * e] * rsq, v1 = xq[c + 2 * e + 1] * rsq;
+                        const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
+                        hw[e] = pack2(__half_as_ushort(h0), __half_as_ushort(h1));
+                        lw[e] = half2_bits(v0 - __half2float(h0), v1 - __half2float(h1));
+                    }
+                    tc::st_8cols(tmem + lane_base + TM_QHI + c / 2, hw);
+                    tc::st_8cols(tmem + lane_base + TM_QLO + c / 2, lw);
+                }
             }
-            // weights of the tile, fp16, as the A operand of P V~ (stored in
-            // two halves of 32 keys)
-            if (j >= 2 && !wait(B_PEMPTY + bf, ((j - 2) >> 1) & 1)) break;
-            const bool live = mref > -INFINITY;
-            const float2 rs2 = make_float2(rs, rs), nm2 = make_float2(-mref, -mref);
-            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pw[16];
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const float2 t0 = ptx::ffma2(make_float2(u[32 * h + i], u[32 * h + i + 1]), rs2, nm2);
-                    const float2 t1 = ptx::ffma2(make_float2(u[32 * h + i + 2], u[32 * h + i + 3]), rs2, nm2);
-                    const float2 p0 = make_float2(ptx::ex2(t0.x), ptx::ex2(t0.y));
-                    const float2 p1 = make_float2(ptx::ex2(t1.x), ptx::ex2(t1.y));
-                    acc0 = ptx::fadd2(acc0, p0);
-                    acc1 = ptx::fadd2(acc1, p1);
-                    pw[i / 2] = half2_bits(p0.x, p0.y);
-                    pw[i / 2 + 1] = half2_bits(p1.x, p1.y);
-                }
-                if (!live) {  // no visible key yet (a row past the chunk): no weight
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) pw[i] = 0u;
-                }
-                tc::st_16cols_u(tmem + lane_base + TM_P + (BK / 2) * bf + 16 * h, pw);
-            }
-            if (live) l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
             tc::st_wait();
             tc::fence_before_sync();
             __syncwarp();
-            // the weights are stored and the score buffer, the tile's norms and
-            // any accumulator rescale are done with
-            if (lane == 0) {
-                ptx::mbar_arrive(bar(B_SEMPTY + bf));
-                ptx::mbar_arrive(bar(B_PFULL + bf));
-            }
-        }
-        // ---- epilogue: wait for the last P V, normalise, inverse rotation
-        const bool done = T > 0 && wait(B_PEMPTY + ((T - 1) & 1), ((T - 1) >> 1) & 1);
-        tc::fence_after_sync();
-        float o[D];
-        if (done) {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                float ov[32];
-                tc::ld_32cols(tmem + lane_base + TM_O + 32 * q4, ov);
+            if (lane == 0) ptx::mbar_arrive(bar(B_QREADY));
+            // scores in log2 units: S kn rs; a zero query row keeps rs > 0 so that a
+            // masked (-inf) score stays -inf
+            const float rs = fmaxf(qscale * a.score_scale, 1e-30f);
+            const Unit x = unit_of(a, segment_unit(slot));
+            const bool row_ok = rt < x.ntok && rt * G + rh < BM;
+            segment_bounds(a, smem, segment_unit(slot), j0, j1);
+            // the unit's first query position, in ring coordinates (ring tile g
+            // holds the unit's keys from g BK - (gi - j0) BK): keys past
+            // dlim + rt are past the row's own position
+            const int dlim = x.start + x.tok0 + (gi - j0) * BK;
+            float mref = -INFINITY, l = 0.f;
+            for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
+                const int bf = gi & 1, key0 = gi * BK;  // (ring coordinates)
+                if (!wait(B_SFULL + bf, (gi >> 1) & 1)) goto softmax_done;
+                tc::fence_after_sync();
+                float sc[BK];
+                {
+                    float (&sc0)[32] = *reinterpret_cast<float (*)[32]>(&sc[0]);
+                    float (&sc1)[32] = *reinterpret_cast<float (*)[32]>(&sc[32]);
+                    tc::ld_32cols(tmem + lane_base + TM_S + BK * bf, sc0);
+                    tc::ld_32cols(tmem + lane_base + TM_S + BK * bf + 32, sc1);
+                }
                 tc::ld_wait();
+                const float4* kn4 = reinterpret_cast<const float4*>(smem + SM_KNR + (gi & 3) * BK * 4);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) o[32 * q4 + i] = ov[i];
+                for (int i = 0; i < BK; i += 4) {
+                    const float4 k4 = kn4[i / 4];
+                    const float2 a01 = ptx::fmul2(make_float2(sc[i], sc[i + 1]), make_float2(k4.x, k4.y));
+                    const float2 a23 = ptx::fmul2(make_float2(sc[i + 2], sc[i + 3]), make_float2(k4.z, k4.w));
+                    sc[i] = a01.x;
+                    sc[i + 1] = a01.y;
+                    sc[i + 2] = a23.x;
+                    sc[i + 3] = a23.y;
+                }
+                if (key0 + BK - 1 > dlim) {
+                    // a tile on the diagonal: keys past the row's own position drop
+                    // out (rows outside the chunk are never stored; every key of an
+                    // earlier tile is visible to every row of the unit)
+                    const int qlim = dlim + rt;
+#pragma unroll
+                    for (int i = 0; i < BK; ++i)
+                        if (!row_ok || key0 + i > qlim) sc[i] = -INFINITY;
+                }
+                float m4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float m = sc[16 * q];
+#pragma unroll
+                    for (int i = 1; i < 15; i += 2) m = ptx::fmax3(m, sc[16 * q + i], sc[16 * q + i + 1]);
+                    m4[q] = fmaxf(m, sc[16 * q + 15]);
+                }
+                const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * rs;
+                // lazy reference: moves (and the accumulator is rescaled) only when a
+                // score passes it by more than 2^LAZY; the weights stay below 2^LAZY
+                const bool need = mt > mref + LAZY;
+                if (__any_sync(0xffffffffu, need)) {
+                    const float mnew = need ? mt : mref;
+                    const float c = (need && mref > -INFINITY) ? ptx::ex2(mref - mnew) : 1.f;
+                    if (__any_sync(0xffffffffu, mref > -INFINITY)) {
+                        // not the segment's first tile (where every reference is
+                        // still -inf and the accumulator holds nothing): every P V
+                        // of the segment's earlier tiles is in the accumulator
+                        if (!wait(B_PEMPTY + ((gi - 1) & 1), ((gi - 1) >> 1) & 1)) goto softmax_done;
+                        tc::fence_after_sync();
+#pragma unroll 1
+                        for (int q8 = 0; q8 < 8; ++q8) {
+                            float ov[16];
+                            tc::ld_16cols(tmem + lane_base + TM_O + 16 * q8, ov);
+                            tc::ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) ov[i] *= c;
+                            tc::st_16cols(tmem + lane_base + TM_O + 16 * q8, ov);
+                        }
+                    }
+                    l *= c;
+                    mref = mnew;
+                }
+                // weights of the tile, fp16, as the A operand of P V~ (stored in
+                // two halves of 32 keys)
+                if (gi >= 2 && !wait(B_PEMPTY + bf, ((gi - 2) >> 1) & 1)) goto softmax_done;
+                const bool live = mref > -INFINITY;
+                const float2 rs2 = make_float2(rs, rs), nm2 = make_float2(-mref, -mref);
+                float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pw[16];
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float2 t0 = ptx::ffma2(make_float2(sc[32 * h + i], sc[32 * h + i + 1]), rs2, nm2);
+                        const float2 t1 = ptx::ffma2(make_float2(sc[32 * h + i + 2], sc[32 * h + i + 3]), rs2, nm2);
+                        const float2 p0 = make_float2(ptx::ex2(t0.x), ptx::ex2(t0.y));
+                        const float2 p1 = make_float2(ptx::ex2(t1.x), ptx::ex2(t1.y));
+                        acc0 = ptx::fadd2(acc0, p0);
+                        acc1 = ptx::fadd2(acc1, p1);
+                        pw[i / 2] = half2_bits(p0.x, p0.y);
+                        pw[i / 2 + 1] = half2_bits(p1.x, p1.y);
+                    }
+                    if (!live) {  // no visible key yet (a row past the chunk): no weight
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) pw[i] = 0u;
+                    }
+                    tc::st_16cols_u(tmem + lane_base + TM_P + (BK / 2) * bf + 16 * h, pw);
+                }
+                if (live) l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
+                tc::st_wait();
+                tc::fence_before_sync();
+                __syncwarp();
+                // the weights are stored and the score buffer, the tile's norms and
+                // any accumulator rescale are done with
+                if (lane == 0) {
+                    ptx::mbar_arrive(bar(B_SEMPTY + bf));
+                    ptx::mbar_arrive(bar(B_PFULL + bf));
+                }
             }
-        } else {
+            // ---- the segment's end: wait for its last P V, read the accumulator
+            const bool done = wait(B_PEMPTY + ((gi - 1) & 1), ((gi - 1) >> 1) & 1);
+            tc::fence_after_sync();
+            float o[D];
+            if (done) {
 #pragma unroll
-            for (int c = 0; c < D; ++c) o[c] = 0.f;
-        }
-        if (row_ok || (blk.bad && rt < min(TT, a.n_new - blk.tok0) && rt * G + rh < BM)) {
-            const float inv = (done && l > 0.f && !*abort_flag) ? a.out_scale / l : 0.f;
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    float ov[32];
+                    tc::ld_32cols(tmem + lane_base + TM_O + 32 * q4, ov);
+                    tc::ld_wait();
 #pragma unroll
-            for (int c = 0; c < D; ++c) o[c] *= inv;
-            fwht128(o);
-            const float inv_sqrt_d = 0.08838834764831845f;
-            float* dst = a.out + ((static_cast<size_t>(blk.b) * a.n_new + blk.tok0 + rt) * a.hq + blk.kv * G + rh) * D;
+                    for (int i = 0; i < 32; ++i) o[32 * q4 + i] = ov[i];
+                }
+            } else {
 #pragma unroll
-            for (int c = 0; c < D; c += 4) {
-                float4 v;
-                v.x = flip_sign(o[c] * inv_sqrt_d, (a.signs[c >> 5] >> (c & 31)) & 1u);
-                v.y = flip_sign(o[c + 1] * inv_sqrt_d, (a.signs[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u);
-                v.z = flip_sign(o[c + 2] * inv_sqrt_d, (a.signs[(c + 2) >> 5] >> ((c + 2) & 31)) & 1u);
-                v.w = flip_sign(o[c + 3] * inv_sqrt_d, (a.signs[(c + 3) >> 5] >> ((c + 3) & 31)) & 1u);
-                *reinterpret_cast<float4*>(dst + c) = v;
+                for (int c = 0; c < D; ++c) o[c] = 0.f;
+            }
+            tc::fence_before_sync();
+            if (!done) goto softmax_done;
+            bool write = true;
+            const int u = segment_unit(slot);
+            if (unit_is_cut(a, smem, u)) {
+                // a unit cut between blocks: publish this segment's (O, m, l)
+                // rows; the last of the unit's blocks to do so merges them
+                const volatile uint32_t* seg = reinterpret_cast<const volatile uint32_t*>(smem + SM_SEG);
+                const volatile uint32_t* sched = reinterpret_cast<const volatile uint32_t*>(smem + SM_SCHED);
+                const uint32_t pu = sched[u], pn = sched[u + 1], total = sched[a.units], C = seg[3];
+                const int cb = static_cast<int>(blockIdx.x);
+                const int ca = block_of(pu, total, C), cz = block_of(pn - 1, total, C);
+                constexpr size_t PART = static_cast<size_t>(BM) * (D + 2);
+                float* mine = a.parts + static_cast<size_t>(2 * cb + (cb == ca ? 1 : 0)) * PART;
+#pragma unroll
+                for (int c = 0; c < D; c += 4)
+                    *reinterpret_cast<float4*>(mine + r * D + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+                mine[BM * D + r] = mref;
+                mine[BM * D + BM + r] = l;
+                // every row is written before thread 0's release; its acquire
+                // orders the merge's reads after the other blocks' rows (the
+                // waits are bounded: a warp that stopped early cannot hang the
+                // others)
+                __syncwarp();
+                volatile int* merge_flag = reinterpret_cast<volatile int*>(smem + SM_MFLAG);
+                const uint32_t npart = ptx::lds32(sbase + SM_NPART + 4u * static_cast<uint32_t>(tid));
+                const uint32_t ph = npart & 1u;
+                if (lane == 0) ptx::mbar_arrive(bar(B_PART));
+                if (tid == 0) {
+                    const bool all = wait(B_PART, ph);
+                    *merge_flag = all && ptx::atom_add_acq_rel_gpu(a.counters + u, 1u) ==
+                                             static_cast<uint32_t>(cz - ca);
+                    ptx::mbar_arrive(bar(B_PFLAG));
+                }
+                const bool published = wait(B_PFLAG, ph);
+                sts32(sbase + SM_NPART + 4u * static_cast<uint32_t>(tid), npart + 1u);
+                write = published && *merge_flag != 0;
+                if (write) {
+                    float mm = mref;
+                    for (int c2 = ca; c2 <= cz; ++c2)
+                        if (c2 != cb) {
+                            const float* other = a.parts + static_cast<size_t>(2 * c2 + (c2 == ca ? 1 : 0)) * PART;
+                            mm = fmaxf(mm, __ldcg(other + BM * D + r));
+                        }
+                    const float wme = (mref > -INFINITY && mm > -INFINITY) ? ptx::ex2(mref - mm) : 0.f;
+#pragma unroll
+                    for (int c = 0; c < D; ++c) o[c] *= wme;
+                    float lt = l * wme;
+                    for (int c2 = ca; c2 <= cz; ++c2) {
+                        if (c2 == cb) continue;
+                        const float* other = a.parts + static_cast<size_t>(2 * c2 + (c2 == ca ? 1 : 0)) * PART;
+                        const float mo = __ldcg(other + BM * D + r), lo = __ldcg(other + BM * D + BM + r);
+                        const float w = (mo > -INFINITY && mm > -INFINITY) ? ptx::ex2(mo - mm) : 0.f;
+                        lt = fmaf(lo, w, lt);
+#pragma unroll
+                        for (int c = 0; c < D; c += 4) {
+                            const float4 v = __ldcg(reinterpret_cast<const float4*>(other + r * D + c));
+                            o[c] = fmaf(v.x, w, o[c]);
+                            o[c + 1] = fmaf(v.y, w, o[c + 1]);
+                            o[c + 2] = fmaf(v.z, w, o[c + 2]);
+                            o[c + 3] = fmaf(v.w, w, o[c + 3]);
+                        }
+                    }
+                    l = lt;
+                    if (tid == 0) a.counters[u] = 0;  // ready for the next call
+                }
+            }
+            // ---- the unit's output: normalise, inverse rotation
+            float* dst = out_row(unit_of(a, u));
+            if (write && dst) {
+                const float inv = (row_ok && l > 0.f && !*abort_flag) ? a.out_scale / l : 0.f;
+#pragma unroll
+                for (int c = 0; c < D; ++c) o[c] *= inv;
+                fwht128(o);
+#pragma unroll
+                for (int c = 0; c < D; c += 4) {
+                    float4 v;
+                    v.x = flip_sign(o[c] * inv_sqrt_d, (a.signs[c >> 5] >> (c & 31)) & 1u);
+                    v.y = flip_sign(o[c + 1] * inv_sqrt_d, (a.signs[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u);
+                    v.z = flip_sign(o[c + 2] * inv_sqrt_d, (a.signs[(c + 2) >> 5] >> ((c + 2) & 31)) & 1u);
+                    v.w = flip_sign(o[c + 3] * inv_sqrt_d, (a.signs[(c + 3) >> 5] >> ((c + 3) & 31)) & 1u);
+                    *reinterpret_cast<float4*>(dst + c) = v;
+                }
             }
         }
+    softmax_done:;
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -676,12 +979,51 @@ bool prefill_supported(const tq_params& p) {
            p.num_q_heads / p.num_kv_heads <= 16;
 }
 
+namespace prefill {
+
+// Work layout of a call: units, whether the blocks share the tile sequence
+// (spread) and, if so, how many blocks and the workspace: the per-unit
+// counters, then two partial-output slots per block.
+struct Plan {
+    long long units;
+    int spread, blocks;
+    size_t counter_bytes, bytes;
+};
+
+static Plan plan(const tq_params& p, int batch, int n_new, int sms) {
+    Plan pl{};
+    const int tt = BM / (p.num_q_heads / p.num_kv_heads);
+    pl.units = static_cast<long long>(batch) * p.num_kv_heads * ((n_new + tt - 1) / tt);
+    pl.spread = pl.units <= SCHED_MAX && sms > 0;
+    pl.blocks = pl.spread ? sms : static_cast<int>(pl.units);
+    if (pl.spread) {
+        pl.counter_bytes = (static_cast<size_t>(pl.units) * 4 + 255) / 256 * 256;
+        pl.bytes = pl.counter_bytes + static_cast<size_t>(2 * pl.blocks) * BM * (D + 2) * sizeof(float);
+    }
+    return pl;
+}
+
+}  // namespace prefill
 }  // namespace tq
+
+extern "C" tq_status tq_prefill_workspace_bytes(const tq_params* params, int32_t batch, int32_t n_new,
+                                                size_t* bytes) {
+    using namespace tq;
+    tq_status st = validate_params(params);
+    if (st != TQ_OK) return st;
+    if (!bytes || batch < 1 || n_new < 1) return TQ_ERR_INVALID_ARG;
+    if (!prefill_supported(*params)) return TQ_ERR_UNSUPPORTED;
+    const int sms = num_sms_current();
+    if (sms <= 0) return TQ_ERR_CUDA;
+    *bytes = prefill::plan(*params, batch, n_new, sms).bytes;
+    return TQ_OK;
+}
 
 extern "C" tq_status tq_prefill_attention(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
                                           const void* k_new, const void* v_new, tq_dtype kv_dtype, const void* d_q,
                                           tq_dtype q_dtype, int32_t n_new, const int32_t* d_positions,
-                                          const tq_cache* cache, float* d_out, uint32_t* d_error, void* stream) {
+                                          const tq_cache* cache, float* d_out, void* d_workspace,
+                                          size_t workspace_bytes, uint32_t* d_error, void* stream) {
     using namespace tq;
     tq_status st = validate_params(params);
     if (st != TQ_OK) return st;
@@ -694,6 +1036,21 @@ extern "C" tq_status tq_prefill_attention(const tq_params* params, const tq_code
     if (n_new > cache->capacity) return TQ_ERR_CAPACITY;
     if ((st = validate_codebook(kcb, p.head_dim, p.k_bits)) != TQ_OK) return st;
     if ((st = validate_codebook(vcb, p.head_dim, p.v_bits)) != TQ_OK) return st;
+    const int sms = num_sms_current();
+    if (sms <= 0) return TQ_ERR_CUDA;
+    prefill::Plan pl = prefill::plan(p, cache->batch, n_new, sms);
+    if (pl.spread && pl.units * ((cache->capacity + prefill::BK - 1) / prefill::BK) >= (1LL << 31)) {
+        // the shared tile sequence is counted in 32 bits: a cache long enough
+        // to overflow it takes whole units per block instead
+        pl.spread = 0;
+        pl.blocks = static_cast<int>(pl.units);
+        pl.bytes = 0;
+    }
+    if (pl.bytes > 0) {
+        if (!d_workspace) return TQ_ERR_INVALID_ARG;
+        if (workspace_bytes < pl.bytes) return TQ_ERR_CAPACITY;
+        if (!aligned16(d_workspace)) return TQ_ERR_ALIGNMENT;
+    }
     // append the chunk (positions[b] .. positions[b] + n_new - 1), then attend
     st = quantize_append_impl(params, kcb, vcb, k_new, v_new, kv_dtype, n_new, d_positions, false, cache, d_error,
                               stream);
@@ -732,7 +1089,12 @@ extern "C" tq_status tq_prefill_attention(const tq_params* params, const tq_code
     uint32_t words[8];
     rotation_sign_bits(p.seed, 128, words);
     for (int i = 0; i < 4; ++i) a.signs[i] = words[i];
-    const dim3 grid((n_new + a.tok_per_tile - 1) / a.tok_per_tile, p.num_kv_heads, cache->batch);
+    a.qtiles = (n_new + a.tok_per_tile - 1) / a.tok_per_tile;
+    a.units = static_cast<int>(pl.units);
+    a.spread = pl.spread;
+    a.counters = pl.spread ? static_cast<uint32_t*>(d_workspace) : nullptr;
+    a.parts = pl.spread ? reinterpret_cast<float*>(static_cast<char*>(d_workspace) + pl.counter_bytes) : nullptr;
+    const dim3 grid(static_cast<unsigned>(pl.blocks));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const cudaError_t e = prefill::launch_kb(p.k_bits, p.v_bits, a, grid, s);
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;

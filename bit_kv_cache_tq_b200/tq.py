@@ -32,7 +32,7 @@ EXPORTED = (
     "tq_cache_bytes", "tq_decode_workspace_bytes", "tq_quantize_append", "tq_dequantize",
     "tq_decode_attention", "tq_append_decode_attention", "tq_decode_attention_static", "tq_read_device_error",
     "tq_quantize_append_paged", "tq_decode_attention_paged", "tq_append_decode_attention_paged",
-    "tq_prefill_attention", "tq_decode_static_fill",
+    "tq_prefill_attention", "tq_decode_static_fill", "tq_prefill_workspace_bytes",
 )
 
 # Bytes of the library's own decode scratch per device (tq_decode_attention_static).
@@ -117,7 +117,8 @@ _lib.tq_append_decode_attention_paged.argtypes = [_P(tq_params), _P(tq_codebook)
 _lib.tq_prefill_attention.argtypes = [_P(tq_params), _P(tq_codebook), _P(tq_codebook), ctypes.c_void_p,
                                       ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int32,
                                       ctypes.c_void_p, _P(tq_cache), ctypes.c_void_p, ctypes.c_void_p,
-                                      ctypes.c_void_p]
+                                      ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+_lib.tq_prefill_workspace_bytes.argtypes = [_P(tq_params), ctypes.c_int32, ctypes.c_int32, _P(ctypes.c_size_t)]
 for _name in EXPORTED:
     if _name not in ("tq_status_string", "tq_abi_version"):
         getattr(_lib, _name).restype = ctypes.c_int
@@ -321,17 +322,27 @@ def tq_decode_attention_static(params, kcb, vcb, q, cache, seq_lens, max_seq_len
     _check(st, "tq_decode_attention_static")
 
 
-def tq_prefill_attention(params, kcb, vcb, k_new, v_new, q, positions, cache, out, error=None, stream=None):
+def tq_prefill_workspace_bytes(params, batch, n_new):
+    n = ctypes.c_size_t(0)
+    _check(_lib.tq_prefill_workspace_bytes(ctypes.byref(params), batch, n_new, ctypes.byref(n)),
+           "tq_prefill_workspace_bytes")
+    return n.value
+
+
+def tq_prefill_attention(params, kcb, vcb, k_new, v_new, q, positions, cache, out, workspace, error=None,
+                         stream=None):
     """Append k_new/v_new ([batch, n_new, Hkv, d]) at slots positions[b] .., then causal attention of
-    q ([batch, n_new, Hq, d]) over the cache into out ([batch, n_new, Hq, d] fp32)."""
+    q ([batch, n_new, Hq, d]) over the cache into out ([batch, n_new, Hq, d] fp32); workspace: zeroed
+    uint8 CUDA tensor of tq_prefill_workspace_bytes(params, batch, n_new) bytes (or None when that is 0)."""
     assert q.is_contiguous() and out.is_contiguous() and out.dtype == torch.float32
     assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.dtype == v_new.dtype
     assert positions.dtype == torch.int32 and positions.is_cuda
     c = cache.struct()
     st = _lib.tq_prefill_attention(ctypes.byref(params), kcb and ctypes.byref(kcb), vcb and ctypes.byref(vcb),
                                    _ptr(k_new), _ptr(v_new), _dtype_code(k_new), _ptr(q), _dtype_code(q),
-                                   k_new.shape[1], _ptr(positions), ctypes.byref(c), _ptr(out), _ptr(error),
-                                   _stream(stream))
+                                   k_new.shape[1], _ptr(positions), ctypes.byref(c), _ptr(out), _ptr(workspace),
+                                   0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                   _ptr(error), _stream(stream))
     _check(st, "tq_prefill_attention")
 
 

@@ -34,7 +34,9 @@ def _prefill_case(layer, starts, n_new, seed, prefill_tokens=None, dtype=torch.b
     pos = torch.tensor(starts, dtype=torch.int32, device="cuda")
     out = torch.empty(bsz, n_new, layer.hq, d, dtype=torch.float32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    tq.tq_prefill_attention(layer.params, layer.kcb, layer.vcb, kn.cuda(), vn.cuda(), q.cuda(), pos, cache, out, err)
+    ws = torch.zeros(tq.tq_prefill_workspace_bytes(layer.params, bsz, n_new), dtype=torch.uint8, device="cuda")
+    tq.tq_prefill_attention(layer.params, layer.kcb, layer.vcb, kn.cuda(), vn.cuda(), q.cuda(), pos, cache, out, ws,
+                            err)
     st, word = tq.tq_read_device_error(err)
     assert word == expect_word and st == (tq.TQ_OK if expect_word == 0 else tq.TQ_ERR_DEVICE), (st, word)
     return cache, out.cpu().numpy(), q, (kn, vn)
@@ -127,6 +129,76 @@ def test_prefill_flags_a_chunk_past_the_capacity():
     assert worst < H.ATTN_TOL, worst
 
 
+def test_prefill_workspace_reused_across_chunks():
+    """Two chunks in a row on one workspace.  With 16 units of ~15 key tiles
+    over one block per SM, most units are cut between blocks; the block
+    that merges a unit resets its counter, so the counters are zero after
+    each call and the second call's merges are right as well."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=28)
+    start, n1, n2 = 900, 40, 56
+    cap = start + n1 + n2 + 40
+    k0 = inputs.lognormal_kv(1, start, 8, 128, seed=28, layer=3, which=inputs.K)
+    v0 = inputs.lognormal_kv(1, start, 8, 128, seed=28, layer=3, which=inputs.V)
+    cache, st, word = H.gpu_quantize(layer, k0, v0, cap)
+    assert st == tq.TQ_OK and word == 0
+    nbytes = max(tq.tq_prefill_workspace_bytes(layer.params, 1, n) for n in (n1, n2))
+    assert nbytes > 0
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    results = []
+    for at, n in ((start, n1), (start + n1, n2)):
+        kn = inputs.lognormal_kv(1, n, 8, 128, seed=28 + at, layer=3, which=inputs.K).cuda()
+        vn = inputs.lognormal_kv(1, n, 8, 128, seed=28 + at, layer=3, which=inputs.V).cuda()
+        q = torch.randn(1, n, 32, 128, generator=torch.Generator().manual_seed(at)).to(torch.bfloat16)
+        out = torch.empty(1, n, 32, 128, dtype=torch.float32, device="cuda")
+        pos = torch.tensor([at], dtype=torch.int32, device="cuda")
+        tq.tq_prefill_attention(layer.params, layer.kcb, layer.vcb, kn, vn, q.cuda(), pos, cache, out, ws, err)
+        st, word = tq.tq_read_device_error(err)
+        assert st == tq.TQ_OK and word == 0, (st, word)
+        units = 8 * ((n + 31) // 32)  # (32-token query blocks for a group of 4 heads)
+        assert not ws[:4 * units].any(), "unit counters left non-zero"
+        results.append((at, q, out.cpu().numpy()))
+    for at, q, out in results:
+        worst = _check_rows(layer, cache, out, q, [at])
+        assert worst < H.ATTN_TOL, (at, worst)
+
+
+def test_prefill_whole_units_past_the_schedule():
+    """More units than the shared schedule holds (a 16416-token chunk of 8
+    kv heads in 32-token query blocks: 4104 > 4096 units): each block takes
+    one whole unit and no workspace is needed; sampled rows against the
+    oracle, the first and last of query blocks among them."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=29)
+    n_new = 16416
+    assert tq.tq_prefill_workspace_bytes(layer.params, 1, n_new) == 0
+    cache, out, q, _ = _prefill_case(layer, [0], n_new, seed=29, prefill_tokens=1)
+    gen = np.random.default_rng(29)
+    rows = [(0, j) for j in (0, 31, 32, 8191, 8192, n_new - 1)]
+    rows += [(0, int(j)) for j in sorted(gen.choice(n_new, size=6, replace=False))]
+    worst = _check_rows(layer, cache, out, q, [0], rows=rows)
+    assert worst < H.ATTN_TOL, worst
+
+
+def test_prefill_workspace_argument_checks():
+    """A missing, short or misaligned workspace is refused before anything
+    is appended (the cache stays empty)."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=30)
+    n = 64
+    cache = tq.alloc_cache(layer.params, 1, 256)
+    x = torch.zeros(1, n, 8, 128, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(1, n, 32, 128, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(1, n, 32, 128, device="cuda")
+    pos = torch.zeros(1, dtype=torch.int32, device="cuda")
+    need = tq.tq_prefill_workspace_bytes(layer.params, 1, n)
+    big = torch.zeros(need + 16, dtype=torch.uint8, device="cuda")
+    for ws, status in ((None, tq.TQ_ERR_INVALID_ARG), (big[:need - 16], tq.TQ_ERR_CAPACITY),
+                       (big[1:need + 1], tq.TQ_ERR_ALIGNMENT)):
+        with pytest.raises(tq.TqError) as ei:
+            tq.tq_prefill_attention(layer.params, layer.kcb, layer.vcb, x, x, q, pos, cache, out, ws)
+        assert ei.value.status == status
+    assert not cache.k_norms.any()
+
+
 @pytest.mark.slow
 def test_prefill_llama8b_32k_chunk_sampled_rows():
     """Llama-3-8B-shaped layer, 32768 cached tokens, a 512-token chunk (the
@@ -148,5 +220,5 @@ def test_prefill_rejects_unsupported_settings():
     out = torch.empty(1, 4, 64, 128, device="cuda")
     with pytest.raises(tq.TqError) as ei:
         tq.tq_prefill_attention(layer.params, layer.kcb, layer.vcb, x, x, q, torch.zeros(1, dtype=torch.int32,
-                                device="cuda"), cache, out)
+                                device="cuda"), cache, out, None)
     assert ei.value.status == tq.TQ_ERR_UNSUPPORTED

@@ -53,7 +53,7 @@ def test_binding_declares_every_argument_type():
 
 
 def test_abi_version_and_status_strings():
-    assert tq.tq_abi_version() == 4
+    assert tq.tq_abi_version() == 5
     for st in range(8):
         assert tq.tq_status_string(st)
     assert tq.tq_status_string(99) == "unknown status"
