@@ -20,8 +20,8 @@
 // being one (query token, head of the GQA group), each unit a run of 64-key
 // tiles.  One thread block per SM takes an equal share of the sequence of
 // all units' tiles (so a unit can be cut between blocks: each piece's rows
-// go to the workspace as (O, m, l), and the last block to finish a piece of
-// the unit merges them by log-sum-exp); a block runs its share as
+// go to the workspace as (O, m, l), and a second kernel merges them by
+// log-sum-exp); a block runs its share as
 // segments (unit, tile range) in warp-specialised roles that overlap every
 // stage of a tile with the tensor cores' work on others.  (With more units
 // than the schedule holds, each block takes one whole unit.)
@@ -108,24 +108,19 @@ constexpr uint32_t SM_BAR = SM_CENT + 64;
 // mbarriers (8 bytes each)
 constexpr int B_FULL = 0, B_EMPTY = NS, B_KFULL = 2 * NS, B_KEMPTY = B_KFULL + 2, B_VFULL = B_KEMPTY + 2,
               B_VEMPTY = B_VFULL + 2, B_SFULL = B_VEMPTY + 2, B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2,
-              B_PEMPTY = B_PFULL + 2, B_QREADY = B_PEMPTY + 2, B_FINAL = B_QREADY + 1, B_PART = B_FINAL + 1,
-              B_PFLAG = B_PART + 1, NBARS = B_PFLAG + 1;
-// (B_PART: the softmax warps have written a cut unit's partial rows;
-// B_PFLAG: thread 0 has published whether this block merges the unit.)
+              B_PEMPTY = B_PFULL + 2, B_QREADY = B_PEMPTY + 2, B_FINAL = B_QREADY + 1, NBARS = B_FINAL + 1;
 // (B_PEMPTY[j % 2] also tells that every P V up to tile j is in the accumulator:
 // commits complete in order.  Waiting on it rather than on one shared
 // barrier keeps every wait within one phase of the barrier's state.)
 constexpr uint32_t SM_TMEM = SM_BAR + NBARS * 8;   // tensor-memory address
 constexpr uint32_t SM_FLAG = SM_TMEM + 4;          // abort flag
-constexpr uint32_t SM_MFLAG = SM_FLAG + 4;         // "this block merges the unit's partials"
-constexpr uint32_t SM_SEG = (SM_MFLAG + 4 + 15) & ~15u;    // uint32 [4]: the block's g0, g1, g1x, C (spread mode)
+constexpr uint32_t SM_SEG = (SM_FLAG + 4 + 15) & ~15u;     // uint32 [4]: the block's g0, g1, g1x, C (spread mode)
 constexpr uint32_t SM_USTART = SM_SEG + 16;                // int: the block's first unit
 // uint32 [NTHREADS]: per-thread tile sums in the prologue, then each thread's
 // segment iterator (kept here, not in a register, through the tile loops)
 constexpr uint32_t SM_SCAN = SM_SEG + 32;
-constexpr uint32_t SM_NPART = SM_SCAN + NTHREADS * 4;      // uint32 [softmax threads]: cut units published
 constexpr int SCHED_MAX = 4096;                            // most units the shared schedule holds
-constexpr uint32_t SM_SCHED = SM_NPART + SOFTMAX_WARPS * 32 * 4;  // uint32 [units + 1]: tiles before each unit
+constexpr uint32_t SM_SCHED = SM_SCAN + NTHREADS * 4;      // uint32 [units + 1]: tiles before each unit
 constexpr uint32_t SM_KLUT = (SM_SCHED + (SCHED_MAX + 1) * 4 + 127) & ~127u;  // key code table, one copy per lane
 // A code table maps a field of two codes (2 BITS bits) to their fp16
 // centroids, packed, with 32 copies interleaved word by word: entry e of lane
@@ -148,8 +143,8 @@ struct Args {
     int staged_norms;        // capacity % 8 == 0: norms ride in the bulk copies
     int qtiles, units;       // query blocks per (sequence, kv head); units = batch * hkv * qtiles
     int spread;              // 1: the blocks share the (unit, key tile) sequence evenly (see the kernel)
-    uint32_t* counters;      // [units] segments of a unit merged so far (zero between calls)
-    float* parts;            // [2 * gridDim.x][BM][D + 2] partial outputs of cut units
+    uint32_t* sched;         // [units + 1] the tile schedule, written by block 0 for the merge kernel
+    float* parts;            // [2 * blocks][BM][D + 2] partial outputs of cut units
     float score_scale;       // sm_scale * log2(e) / alpha_k
     float out_scale;         // 1 / (alpha_v * VFOLD)
     uint32_t signs[4];
@@ -255,6 +250,13 @@ __device__ __forceinline__ bool unit_is_cut(const Args& a, const uint8_t* smem, 
 __device__ __forceinline__ int block_of(uint32_t g, uint32_t total, uint32_t nblocks) {
     return static_cast<int>(((static_cast<uint64_t>(g) + 1) * nblocks - 1) / total);
 }
+
+// A block holds at most two pieces of cut units: the head of the unit its
+// range starts (the first block of that unit: slot 2c + 1) and a piece of a
+// unit begun earlier (slot 2c).  A slot is [BM][D] fp32 O rows, then the
+// rows' m and l.
+constexpr size_t PART_FLOATS = static_cast<size_t>(BM) * (D + 2);
+__device__ __forceinline__ int part_slot(int block, int first_block) { return 2 * block + (block == first_block); }
 
 // The code table of BITS-bit codes: field e (code e & m, then code e >> BITS)
 // -> fp16 centroid pair, for every lane.
@@ -374,8 +376,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         }
         ptx::mbar_init(bar(B_QREADY), SOFTMAX_WARPS);
         ptx::mbar_init(bar(B_FINAL), 1);
-        ptx::mbar_init(bar(B_PART), SOFTMAX_WARPS);
-        ptx::mbar_init(bar(B_PFLAG), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -419,13 +419,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
     }
     __syncthreads();
     if (a.spread) {
+        // (every block computes the same schedule; block 0 also leaves it in
+        // the workspace for the merge kernel)
+        const bool keep = blockIdx.x == 0;
         uint32_t run = scan[tid];
         for (int u = u0; u < u1; ++u) {
             P[u] = run;
+            if (keep) a.sched[u] = run;
             run += static_cast<uint32_t>(unit_of(a, u).ntiles);
         }
-        if (u1 == U && u0 < u1) P[U] = run;
-        if (U == 0 && tid == 0) P[0] = 0;
+        if (u1 == U && u0 < u1) {
+            P[U] = run;
+            if (keep) a.sched[U] = run;
+        }
+        if (U == 0 && tid == 0) {
+            P[0] = 0;
+            if (keep) a.sched[0] = 0;
+        }
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -648,9 +658,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         const int rt = r / G, rh = r % G;
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
         const float inv_sqrt_d = 0.08838834764831845f;
-        // cut units this thread has published so far (the B_PART / B_PFLAG
-        // phase), in shared memory like the iterator
-        sts32(sbase + SM_NPART + 4u * static_cast<uint32_t>(tid), 0u);
         int gi = 0;  // tiles done (the ring position)
         int j0, j1;
         // rows of a unit that exist in the output (all of them but the padding
@@ -855,67 +862,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
             bool write = true;
             const int u = segment_unit(slot);
             if (unit_is_cut(a, smem, u)) {
-                // a unit cut between blocks: publish this segment's (O, m, l)
-                // rows; the last of the unit's blocks to do so merges them
+                // a unit cut between blocks: this piece's (O, m, l) rows go to
+                // the workspace; the merge kernel that follows on the stream
+                // combines the pieces and writes the unit's output
                 const volatile uint32_t* seg = reinterpret_cast<const volatile uint32_t*>(smem + SM_SEG);
                 const volatile uint32_t* sched = reinterpret_cast<const volatile uint32_t*>(smem + SM_SCHED);
-                const uint32_t pu = sched[u], pn = sched[u + 1], total = sched[a.units], C = seg[3];
-                const int cb = static_cast<int>(blockIdx.x);
-                const int ca = block_of(pu, total, C), cz = block_of(pn - 1, total, C);
-                constexpr size_t PART = static_cast<size_t>(BM) * (D + 2);
-                float* mine = a.parts + static_cast<size_t>(2 * cb + (cb == ca ? 1 : 0)) * PART;
+                const uint32_t total = sched[a.units], C = seg[3];
+                const int cb = static_cast<int>(blockIdx.x), ca = block_of(sched[u], total, C);
+                float* mine = a.parts + static_cast<size_t>(part_slot(cb, ca)) * PART_FLOATS;
 #pragma unroll
                 for (int c = 0; c < D; c += 4)
                     *reinterpret_cast<float4*>(mine + r * D + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
                 mine[BM * D + r] = mref;
                 mine[BM * D + BM + r] = l;
-                // every row is written before thread 0's release; its acquire
-                // orders the merge's reads after the other blocks' rows (the
-                // waits are bounded: a warp that stopped early cannot hang the
-                // others)
-                __syncwarp();
-                volatile int* merge_flag = reinterpret_cast<volatile int*>(smem + SM_MFLAG);
-                const uint32_t npart = ptx::lds32(sbase + SM_NPART + 4u * static_cast<uint32_t>(tid));
-                const uint32_t ph = npart & 1u;
-                if (lane == 0) ptx::mbar_arrive(bar(B_PART));
-                if (tid == 0) {
-                    const bool all = wait(B_PART, ph);
-                    *merge_flag = all && ptx::atom_add_acq_rel_gpu(a.counters + u, 1u) ==
-                                             static_cast<uint32_t>(cz - ca);
-                    ptx::mbar_arrive(bar(B_PFLAG));
-                }
-                const bool published = wait(B_PFLAG, ph);
-                sts32(sbase + SM_NPART + 4u * static_cast<uint32_t>(tid), npart + 1u);
-                write = published && *merge_flag != 0;
-                if (write) {
-                    float mm = mref;
-                    for (int c2 = ca; c2 <= cz; ++c2)
-                        if (c2 != cb) {
-                            const float* other = a.parts + static_cast<size_t>(2 * c2 + (c2 == ca ? 1 : 0)) * PART;
-                            mm = fmaxf(mm, __ldcg(other + BM * D + r));
-                        }
-                    const float wme = (mref > -INFINITY && mm > -INFINITY) ? ptx::ex2(mref - mm) : 0.f;
-#pragma unroll
-                    for (int c = 0; c < D; ++c) o[c] *= wme;
-                    float lt = l * wme;
-                    for (int c2 = ca; c2 <= cz; ++c2) {
-                        if (c2 == cb) continue;
-                        const float* other = a.parts + static_cast<size_t>(2 * c2 + (c2 == ca ? 1 : 0)) * PART;
-                        const float mo = __ldcg(other + BM * D + r), lo = __ldcg(other + BM * D + BM + r);
-                        const float w = (mo > -INFINITY && mm > -INFINITY) ? ptx::ex2(mo - mm) : 0.f;
-                        lt = fmaf(lo, w, lt);
-#pragma unroll
-                        for (int c = 0; c < D; c += 4) {
-                            const float4 v = __ldcg(reinterpret_cast<const float4*>(other + r * D + c));
-                            o[c] = fmaf(v.x, w, o[c]);
-                            o[c + 1] = fmaf(v.y, w, o[c + 1]);
-                            o[c + 2] = fmaf(v.z, w, o[c + 2]);
-                            o[c + 3] = fmaf(v.w, w, o[c + 3]);
-                        }
-                    }
-                    l = lt;
-                    if (tid == 0) a.counters[u] = 0;  // ready for the next call
-                }
+                write = false;
             }
             // ---- the unit's output: normalise, inverse rotation
             float* dst = out_row(unit_of(a, u));
@@ -942,6 +902,110 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
     if (warp == MMA_WARP) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ merge
+// The output rows of the units cut between blocks, after the attention
+// kernel on the same stream.  Block (u, y) takes rows [32 y, 32 y + 32) of
+// unit u (nothing when the unit lies in one block, whose attention block
+// wrote it); eight threads per row, sixteen channels each.  Piece p of the
+// unit holds unnormalised rows O_p with their reference m_p (log2 units)
+// and sum l_p; the output is
+//   sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p,
+// then the inverse rotation with the butterflies of fwht128 in the same
+// order (strides 1 .. 8 within a thread, 16 .. 64 across its row's lanes).
+constexpr int MERGE_ROWS = 32, MERGE_THREADS = MERGE_ROWS * 8, MERGE_BATCH = 8;
+
+__global__ void __launch_bounds__(MERGE_THREADS) prefill_merge_kernel(const __grid_constant__ Args a, int nblocks) {
+    const uint32_t total = a.sched[a.units];
+    const int u = static_cast<int>(blockIdx.x);
+    const uint32_t pu = a.sched[u], pn = a.sched[u + 1];
+    if (total == 0 || pn <= pu) return;  // (a unit without tiles has zero rows, written by the attention kernel)
+    const uint32_t C = static_cast<uint32_t>(nblocks) > total ? total : static_cast<uint32_t>(nblocks);
+    const int ca = block_of(pu, total, C), cz = block_of(pn - 1, total, C);
+    if (ca == cz) return;
+    const int tid = static_cast<int>(threadIdx.x), sub = tid & 7;
+    const int r = static_cast<int>(blockIdx.y) * MERGE_ROWS + (tid >> 3);
+    const Unit x = unit_of(a, u);
+    const int G = a.group, rt = r / G, rh = r % G;
+    const bool row_ok = rt < x.ntok && rt * G + rh < BM;
+    const bool row_out = rt < min(a.tok_per_tile, a.n_new - x.tok0) && rt * G + rh < BM;
+    auto piece = [&](int c2) { return a.parts + static_cast<size_t>(part_slot(c2, ca)) * PART_FLOATS; };
+
+    float M = -INFINITY;
+    for (int c0 = ca; c0 <= cz; c0 += MERGE_BATCH) {
+        float mv[MERGE_BATCH];
+#pragma unroll
+        for (int k = 0; k < MERGE_BATCH; ++k) mv[k] = c0 + k <= cz ? __ldcg(piece(c0 + k) + BM * D + r) : -INFINITY;
+#pragma unroll
+        for (int k = 0; k < MERGE_BATCH; ++k) M = fmaxf(M, mv[k]);
+    }
+    float acc[16], L = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+    for (int c0 = ca; c0 <= cz; c0 += MERGE_BATCH) {
+        float4 v[MERGE_BATCH][4];
+        float mk[MERGE_BATCH], lk[MERGE_BATCH];
+#pragma unroll
+        for (int k = 0; k < MERGE_BATCH; ++k) {
+            const bool in = c0 + k <= cz;
+            const float* sp = piece(in ? c0 + k : ca);
+            const float4* row = reinterpret_cast<const float4*>(sp + r * D + 16 * sub);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) v[k][q] = in ? __ldcg(row + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            mk[k] = in ? __ldcg(sp + BM * D + r) : -INFINITY;
+            lk[k] = in ? __ldcg(sp + BM * D + BM + r) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < MERGE_BATCH; ++k) {
+            const float w = (mk[k] > -INFINITY && M > -INFINITY) ? ptx::ex2(mk[k] - M) : 0.f;
+            L = fmaf(lk[k], w, L);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                acc[4 * q] = fmaf(v[k][q].x, w, acc[4 * q]);
+                acc[4 * q + 1] = fmaf(v[k][q].y, w, acc[4 * q + 1]);
+                acc[4 * q + 2] = fmaf(v[k][q].z, w, acc[4 * q + 2]);
+                acc[4 * q + 3] = fmaf(v[k][q].w, w, acc[4 * q + 3]);
+            }
+        }
+    }
+    const float inv = (row_ok && L > 0.f) ? a.out_scale / L : 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] *= inv;
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if ((i & h) == 0) {
+                const float e0 = acc[i], e1 = acc[i + h];
+                acc[i] = e0 + e1;
+                acc[i + h] = e0 - e1;
+            }
+    // (every lane of the warp takes part: the four rows of a warp are all
+    // computed, padding rows included, and only the stores are skipped)
+#pragma unroll
+    for (int m = 1; m < 8; m <<= 1) {
+        const bool upper = (sub & m) != 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float o = __shfl_xor_sync(0xffffffffu, acc[i], m);
+            acc[i] = upper ? o - acc[i] : acc[i] + o;
+        }
+    }
+    if (row_out) {
+        const float inv_sqrt_d = 0.08838834764831845f;
+        float* dst = a.out + ((static_cast<size_t>(x.b) * a.n_new + x.tok0 + rt) * a.hq + x.kv * G + rh) * D;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int c = 16 * sub + 4 * q;
+            float4 v;
+            v.x = flip_sign(acc[4 * q] * inv_sqrt_d, (a.signs[c >> 5] >> (c & 31)) & 1u);
+            v.y = flip_sign(acc[4 * q + 1] * inv_sqrt_d, (a.signs[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u);
+            v.z = flip_sign(acc[4 * q + 2] * inv_sqrt_d, (a.signs[(c + 2) >> 5] >> ((c + 2) & 31)) & 1u);
+            v.w = flip_sign(acc[4 * q + 3] * inv_sqrt_d, (a.signs[(c + 3) >> 5] >> ((c + 3) & 31)) & 1u);
+            *reinterpret_cast<float4*>(dst + c) = v;
+        }
     }
 }
 
@@ -982,12 +1046,12 @@ bool prefill_supported(const tq_params& p) {
 namespace prefill {
 
 // Work layout of a call: units, whether the blocks share the tile sequence
-// (spread) and, if so, how many blocks and the workspace: the per-unit
-// counters, then two partial-output slots per block.
+// (spread) and, if so, how many blocks and the workspace: the schedule
+// (units + 1 words), then two partial-output slots per block.
 struct Plan {
     long long units;
     int spread, blocks;
-    size_t counter_bytes, bytes;
+    size_t sched_bytes, bytes;
 };
 
 static Plan plan(const tq_params& p, int batch, int n_new, int sms) {
@@ -997,8 +1061,8 @@ static Plan plan(const tq_params& p, int batch, int n_new, int sms) {
     pl.spread = pl.units <= SCHED_MAX && sms > 0;
     pl.blocks = pl.spread ? sms : static_cast<int>(pl.units);
     if (pl.spread) {
-        pl.counter_bytes = (static_cast<size_t>(pl.units) * 4 + 255) / 256 * 256;
-        pl.bytes = pl.counter_bytes + static_cast<size_t>(2 * pl.blocks) * BM * (D + 2) * sizeof(float);
+        pl.sched_bytes = (static_cast<size_t>(pl.units + 1) * 4 + 255) / 256 * 256;
+        pl.bytes = pl.sched_bytes + static_cast<size_t>(2 * pl.blocks) * PART_FLOATS * sizeof(float);
     }
     return pl;
 }
@@ -1092,10 +1156,16 @@ extern "C" tq_status tq_prefill_attention(const tq_params* params, const tq_code
     a.qtiles = (n_new + a.tok_per_tile - 1) / a.tok_per_tile;
     a.units = static_cast<int>(pl.units);
     a.spread = pl.spread;
-    a.counters = pl.spread ? static_cast<uint32_t*>(d_workspace) : nullptr;
-    a.parts = pl.spread ? reinterpret_cast<float*>(static_cast<char*>(d_workspace) + pl.counter_bytes) : nullptr;
+    a.sched = pl.spread ? static_cast<uint32_t*>(d_workspace) : nullptr;
+    a.parts = pl.spread ? reinterpret_cast<float*>(static_cast<char*>(d_workspace) + pl.sched_bytes) : nullptr;
     const dim3 grid(static_cast<unsigned>(pl.blocks));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const cudaError_t e = prefill::launch_kb(p.k_bits, p.v_bits, a, grid, s);
+    cudaError_t e = prefill::launch_kb(p.k_bits, p.v_bits, a, grid, s);
+    if (e == cudaSuccess && pl.spread) {
+        // the rows of the units cut between blocks
+        const dim3 mgrid(static_cast<unsigned>(pl.units), prefill::BM / prefill::MERGE_ROWS);
+        prefill::prefill_merge_kernel<<<mgrid, prefill::MERGE_THREADS, 0, s>>>(a, pl.blocks);
+        e = cudaGetLastError();
+    }
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }

@@ -332,8 +332,8 @@ def tq_prefill_workspace_bytes(params, batch, n_new):
 def tq_prefill_attention(params, kcb, vcb, k_new, v_new, q, positions, cache, out, workspace, error=None,
                          stream=None):
     """Append k_new/v_new ([batch, n_new, Hkv, d]) at slots positions[b] .., then causal attention of
-    q ([batch, n_new, Hq, d]) over the cache into out ([batch, n_new, Hq, d] fp32); workspace: zeroed
-    uint8 CUDA tensor of tq_prefill_workspace_bytes(params, batch, n_new) bytes (or None when that is 0)."""
+    q ([batch, n_new, Hq, d]) over the cache into out ([batch, n_new, Hq, d] fp32); workspace: a uint8
+    CUDA tensor of tq_prefill_workspace_bytes(params, batch, n_new) bytes, any contents (None when that is 0)."""
     assert q.is_contiguous() and out.is_contiguous() and out.dtype == torch.float32
     assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.dtype == v_new.dtype
     assert positions.dtype == torch.int32 and positions.is_cuda

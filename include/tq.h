@@ -344,24 +344,25 @@ tq_status tq_append_decode_attention(const tq_params* params, const tq_codebook*
  * the tcgen05 tensor cores (fp16 operands, fp32 accumulation in tensor
  * memory), 128 query rows (tokens x heads of a kv head's group) per block.
  * A position out of range sets TQ_DEVERR_POSITION; that sequence gets no
- * append and zero outputs.  Two kernels on `stream`: the append, then the
- * attention.
+ * append and zero outputs.  Kernels on `stream`: the append, the attention,
+ * then (when units are split, below) the merge.
  *   d_workspace, workspace_bytes  device scratch of at least
  *                 tq_prefill_workspace_bytes(params, cache->batch, n_new)
- *                 bytes (on the current device), 16-byte aligned, zero-filled
- *                 once before its first use; a call that completes leaves it
- *                 ready for the next (after TQ_DEVERR_TIMEOUT, zero it again).
- *                 Calls that overlap on one workspace race.  When that size
- *                 is 0 the workspace may be NULL.
+ *                 bytes (on the current device), 16-byte aligned; its
+ *                 contents need no initial value and mean nothing after the
+ *                 call.  Calls that overlap on one workspace race.  When that
+ *                 size is 0 the workspace may be NULL.
  * Work distribution: the units of 128 query rows (the (sequence, kv head)
  * pairs times the chunk's query blocks) are spread over one block per SM,
  * each block taking an equal share of the units' key tiles, so a unit's
- * tiles may be split between blocks; the block that finishes a split unit
- * last merges its partial outputs (log-sum-exp) from the workspace.  With
- * more than 4096 units, or when units x ceil(capacity / 64) reaches 2^31
- * (the tile sequence is counted in 32 bits), each block takes one whole
- * unit and the workspace is not used.  TQ_ERR_CAPACITY when workspace_bytes
- * is too small.
+ * tiles may be split between blocks; each piece of a split unit leaves its
+ * unnormalised rows with their softmax maximum and sum in the workspace,
+ * and the merge kernel combines them (log-sum-exp) into the unit's output.
+ * With more than 4096 units, or when units x ceil(capacity / 64) reaches
+ * 2^31 (the tile sequence is counted in 32 bits), each block takes one
+ * whole unit, the workspace is not used and no merge runs.  After
+ * TQ_DEVERR_TIMEOUT the outputs are not valid.  TQ_ERR_CAPACITY when
+ * workspace_bytes is too small.
  */
 tq_status tq_prefill_attention(const tq_params* params, const tq_codebook* kcb, const tq_codebook* vcb,
                                const void* k_new, const void* v_new, tq_dtype kv_dtype, const void* d_q,
@@ -371,9 +372,9 @@ tq_status tq_prefill_attention(const tq_params* params, const tq_codebook* kcb, 
 
 /*
  * Bytes of prefill workspace for `batch` sequences and chunks of n_new
- * tokens on the current device (its SM count decides): two partial outputs
- * of 128 rows per block plus one counter per unit; 0 when the call does not
- * need one.  TQ_ERR_UNSUPPORTED for configurations tq_prefill_attention
+ * tokens on the current device (its SM count decides): the tile schedule
+ * (one word per unit, plus one) and two partial outputs of 128 rows per
+ * block; 0 when the call does not need one.  TQ_ERR_UNSUPPORTED for configurations tq_prefill_attention
  * does not take.
  */
 tq_status tq_prefill_workspace_bytes(const tq_params* params, int32_t batch, int32_t n_new, size_t* bytes);

@@ -130,10 +130,9 @@ def test_prefill_flags_a_chunk_past_the_capacity():
 
 
 def test_prefill_workspace_reused_across_chunks():
-    """Two chunks in a row on one workspace.  With 16 units of ~15 key tiles
-    over one block per SM, most units are cut between blocks; the block
-    that merges a unit resets its counter, so the counters are zero after
-    each call and the second call's merges are right as well."""
+    """Two chunks in a row on one workspace that starts as arbitrary bytes.
+    With 16 units of ~15 key tiles over one block per SM, most units are
+    cut between blocks, so both calls go through the merge kernel."""
     layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=28)
     start, n1, n2 = 900, 40, 56
     cap = start + n1 + n2 + 40
@@ -143,7 +142,7 @@ def test_prefill_workspace_reused_across_chunks():
     assert st == tq.TQ_OK and word == 0
     nbytes = max(tq.tq_prefill_workspace_bytes(layer.params, 1, n) for n in (n1, n2))
     assert nbytes > 0
-    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    ws = torch.full((nbytes,), 0xAB, dtype=torch.uint8, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     results = []
     for at, n in ((start, n1), (start + n1, n2)):
@@ -155,8 +154,6 @@ def test_prefill_workspace_reused_across_chunks():
         tq.tq_prefill_attention(layer.params, layer.kcb, layer.vcb, kn, vn, q.cuda(), pos, cache, out, ws, err)
         st, word = tq.tq_read_device_error(err)
         assert st == tq.TQ_OK and word == 0, (st, word)
-        units = 8 * ((n + 31) // 32)  # (32-token query blocks for a group of 4 heads)
-        assert not ws[:4 * units].any(), "unit counters left non-zero"
         results.append((at, q, out.cpu().numpy()))
     for at, q, out in results:
         worst = _check_rows(layer, cache, out, q, [at])
