@@ -341,6 +341,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
     uint8_t* smem = smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = ptx::smem_addr(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // Launched as a programmatic dependent of the append kernel, which lets it
+    // start only after every earlier kernel has finished: everything but the
+    // chunk's own slots (codes and norms of positions[b] ..) is final here, and
+    // the producer waits for the append before it copies a tile holding any
+    // of them.  The merge kernel may start launching now (it waits for this
+    // one to finish).
+    ptx::launch_dependents();
     const uint32_t bars = sbase + SM_BAR;
     auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM_FLAG);
@@ -489,8 +496,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         int j0, j1;
         while (next_segment(a, smem, slot, j0, j1)) {
             const Unit x = unit_of(a, segment_unit(slot));
-            // ring tile g holds the unit's keys from g BK - koff (koff = (gi - j0) BK)
-            const int koff = (gi - j0) * BK, kend = x.kend + koff;
+            // ring tile g holds the unit's keys from g BK - koff (koff = (gi - j0) BK);
+            // knew: the chunk's first slot in those coordinates
+            const int koff = (gi - j0) * BK, kend = x.kend + koff, knew = x.start + koff;
             const long long row0 = static_cast<long long>((static_cast<size_t>(x.b) * a.hkv + x.kv) * a.capacity) - koff;
             for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
                 const int s = gi % NS;
@@ -505,6 +513,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                 }
                 if (leader) {
                     const int key0 = gi * BK, nk = min(BK, kend - key0);
+                    if (key0 + nk > knew) ptx::wait_prerequisites();  // the tile holds appended slots
                     const size_t row = static_cast<size_t>(row0 + key0);
                     const uint32_t dst = sbase + SM_STAGE + s * STAGE_BYTES;
                     const int n8 = (nk + 7) & ~7;  // norms move in 16-byte pieces (8 keys)
@@ -918,6 +927,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
 constexpr int MERGE_ROWS = 32, MERGE_THREADS = MERGE_ROWS * 8, MERGE_BATCH = 8;
 
 __global__ void __launch_bounds__(MERGE_THREADS) prefill_merge_kernel(const __grid_constant__ Args a, int nblocks) {
+    ptx::wait_prerequisites();  // launched as a programmatic dependent of the attention kernel
     const uint32_t total = a.sched[a.units];
     const int u = static_cast<int>(blockIdx.x);
     const uint32_t pu = a.sched[u], pn = a.sched[u + 1];
@@ -1009,14 +1019,33 @@ __global__ void __launch_bounds__(MERGE_THREADS) prefill_merge_kernel(const __gr
     }
 }
 
+// A launch that may start before the previous kernel on the stream finishes
+// (programmatic stream serialisation): the kernel waits for it with
+// griddepcontrol.wait where it first needs that kernel's results.
+template <typename... P, typename... T>
+static cudaError_t launch_dependent(void (*kernel)(P...), dim3 grid, dim3 block, uint32_t smem_bytes, cudaStream_t s,
+                                    T&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem_bytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<T&&>(args)...);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <int KB, int VB>
 static cudaError_t launch_typed(const Args& a, dim3 grid, cudaStream_t s) {
     constexpr uint32_t bytes = sm_alloc(KB, VB);
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(bytes));
     if (e != cudaSuccess) return e;
-    prefill_kernel<KB, VB><<<grid, NTHREADS, bytes, s>>>(a);
-    return cudaGetLastError();
+    return launch_dependent(prefill_kernel<KB, VB>, grid, dim3(NTHREADS), bytes, s, a);
 }
 
 template <int KB>
@@ -1164,8 +1193,8 @@ extern "C" tq_status tq_prefill_attention(const tq_params* params, const tq_code
     if (e == cudaSuccess && pl.spread) {
         // the rows of the units cut between blocks
         const dim3 mgrid(static_cast<unsigned>(pl.units), prefill::BM / prefill::MERGE_ROWS);
-        prefill::prefill_merge_kernel<<<mgrid, prefill::MERGE_THREADS, 0, s>>>(a, pl.blocks);
-        e = cudaGetLastError();
+        e = prefill::launch_dependent(prefill::prefill_merge_kernel, mgrid, dim3(prefill::MERGE_THREADS), 0u, s, a,
+                                      pl.blocks);
     }
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }

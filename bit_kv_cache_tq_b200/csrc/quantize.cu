@@ -342,8 +342,11 @@ __device__ __forceinline__ void quantize_side(const QuantArgs& a, uint32_t* sgri
     const bool grid_path = s.mode == TQ_MODE_TURBO && s.grid_inv_w > 0.0f;
     if (grid_path && threadIdx.x < 128) sgrid[threadIdx.x] = s.grid[threadIdx.x];
     __syncthreads();
-    ptx::launch_dependents();    // the next kernel may start launching
     ptx::wait_prerequisites();   // inputs and cache may come from the previous kernel
+    // the next kernel may start launching; as this comes after the wait, every
+    // kernel before this one has finished by then, so before its own wait the
+    // next kernel can read anything but what this one writes
+    ptx::launch_dependents();
     const int lane = threadIdx.x & 31, sub = lane % LPV, grp = lane / LPV;
     const uint32_t smask = lane_sign_mask<D>(a.signs, sub);
     // bf16 inputs: the rotation signs of word i of chunk k (coordinates
