@@ -160,6 +160,44 @@ def test_prefill_workspace_reused_across_chunks():
         assert worst < H.ATTN_TOL, (at, worst)
 
 
+def test_prefill_inputs_written_by_the_kernels_just_before():
+    """The chunk, the queries and the positions are produced on the stream by
+    GPU kernels immediately before the call, behind a long matmul.  The
+    attention and merge kernels start as programmatic dependents of the
+    kernel before them; they must still see these inputs (the append only
+    lets its dependent start after every earlier kernel has finished)."""
+    layer = H.Layer(128, 32, 8, k_bits=4, v_bits=2, seed=31)
+    start, n = 777, 48
+    k0 = inputs.lognormal_kv(1, start, 8, 128, seed=31, layer=3, which=inputs.K)
+    v0 = inputs.lognormal_kv(1, start, 8, 128, seed=31, layer=3, which=inputs.V)
+    cache, st, word = H.gpu_quantize(layer, k0, v0, start + n + 16)
+    assert st == tq.TQ_OK and word == 0
+    kn = inputs.lognormal_kv(1, n, 8, 128, seed=32, layer=3, which=inputs.K)
+    vn = inputs.lognormal_kv(1, n, 8, 128, seed=32, layer=3, which=inputs.V)
+    q = torch.randn(1, n, 32, 128, generator=torch.Generator().manual_seed(33)).to(torch.bfloat16)
+    # device copies of the inputs, scaled by zero until the kernels below fill them
+    kd, vd, qd = kn.cuda() * 0, vn.cuda() * 0, q.cuda() * 0
+    pos = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kc, vc, qc = kn.cuda(), vn.cuda(), q.cuda()
+    big = torch.randn(4096, 4096, device="cuda")
+    torch.cuda.synchronize()
+    for _ in range(3):
+        big = big @ big * (1.0 / 64.0)  # a few milliseconds of work ahead of the writes
+    kd.copy_(kc * 1.0)
+    vd.copy_(vc * 1.0)
+    qd.copy_(qc * 1.0)
+    pos.fill_(start)
+    out = torch.empty(1, n, 32, 128, dtype=torch.float32, device="cuda")
+    ws = torch.empty(tq.tq_prefill_workspace_bytes(layer.params, 1, n), dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.tq_prefill_attention(layer.params, layer.kcb, layer.vcb, kd, vd, qd, pos, cache, out, ws, err)
+    st, word = tq.tq_read_device_error(err)
+    assert st == tq.TQ_OK and word == 0, (st, word)
+    _check_appended_codes(layer, cache, [start], n, kn, vn)
+    worst = _check_rows(layer, cache, out.cpu().numpy(), q, [start])
+    assert worst < H.ATTN_TOL, worst
+
+
 def test_prefill_whole_units_past_the_schedule():
     """More units than the shared schedule holds (a 16416-token chunk of 8
     kv heads in 32-token query blocks: 4104 > 4096 units): each block takes
