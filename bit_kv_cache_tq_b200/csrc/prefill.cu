@@ -83,7 +83,17 @@ constexpr int SOFTMAX_WARPS = 4, DEQ_WARPS = 8;
 constexpr int DEQ0 = SOFTMAX_WARPS * 32;           // first dequantising thread
 constexpr int PRODUCER = DEQ0 + DEQ_WARPS * 32;    // first thread of the producer warp
 constexpr int MMA_WARP = PRODUCER / 32 + 1;        // MMA issuer warp (also allocates tensor memory)
-constexpr int NTHREADS = (MMA_WARP + 1) * 32;
+// Two idle warps complete the producer and MMA warps' warpgroup, so that the
+// block's registers can be moved between warpgroups (setmaxnreg works on
+// whole warpgroups): launched at 128 registers a thread (16 warps x 32 x 128
+// = the SM's 64 K), the softmax warpgroup takes 160 and the producer's gives
+// up to 96 (per sub-partition, one warp of each: +32 and -32).
+constexpr int NTHREADS = 16 * 32;
+constexpr int REGS_SOFTMAX = 160, REGS_LIGHT = 96;
+static_assert(MMA_WARP < NTHREADS / 32 && MMA_WARP / 4 == PRODUCER / 128 && PRODUCER / 128 == NTHREADS / 128 - 1,
+              "the producer and MMA warps share the last warpgroup");
+static_assert(SOFTMAX_WARPS == 4 && 4 * REGS_SOFTMAX + 8 * 128 + 4 * REGS_LIGHT == 16 * 128,
+              "the register split adds up to the launch's");
 // tensor-memory columns (32-bit; fp16 operands take two elements a column)
 constexpr uint32_t TM_QHI = 0;           // Q~ / qscale, fp16 [128 rows][128 ch]
 constexpr uint32_t TM_QLO = 64;          // its fp16 remainder
@@ -488,180 +498,138 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
     const uint32_t slot = sbase + SM_SCAN + 4u * static_cast<uint32_t>(tid);
     sts32(slot, static_cast<uint32_t>(*reinterpret_cast<volatile int*>(smem + SM_USTART)));
 
-    if (warp == PRODUCER / 32) {
-        // ---------------------------------------------------------- producer
-        // the whole warp waits; one elected lane issues the copies
-        const bool leader = tc::elect_one();
-        int gi = 0;  // tiles issued so far (the ring position)
-        int j0, j1;
-        while (next_segment(a, smem, slot, j0, j1)) {
-            const Unit x = unit_of(a, segment_unit(slot));
-            // ring tile g holds the unit's keys from g BK - koff (koff = (gi - j0) BK);
-            // knew: the chunk's first slot in those coordinates
-            const int koff = (gi - j0) * BK, kend = x.kend + koff, knew = x.start + koff;
-            const long long row0 = static_cast<long long>((static_cast<size_t>(x.b) * a.hkv + x.kv) * a.capacity) - koff;
-            for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
-                const int s = gi % NS;
-                // (the ring is four tiles deep: the producer can poll slowly and
-                // leave the issue slots of its sub-partition to the working warps)
-                if (gi >= NS) {
-                    if (*abort_flag) goto produced;
-                    if (!ptx::mbar_wait_bounded_sleep(bar(B_EMPTY + s), ((gi - NS) / NS) & 1, WAIT_LIMIT, 256)) {
-                        fail();
-                        goto produced;
+    // The register split (setmaxnreg works on whole warpgroups, each at one
+    // instruction): the last warpgroup (producer, MMA issuer, two idle warps)
+    // gives up registers, then the softmax warpgroup takes them; every role's
+    // code follows its own warpgroup's instruction, so the compiler allocates
+    // it within that warpgroup's count.  (The increase is covered by the
+    // decrease, so it cannot wait for ever.)
+    if (warp >= NTHREADS / 32 - 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_LIGHT));
+        if (warp == PRODUCER / 32) {
+            // ---------------------------------------------------------- producer
+            // the whole warp waits; one elected lane issues the copies
+            const bool leader = tc::elect_one();
+            int gi = 0;  // tiles issued so far (the ring position)
+            int j0, j1;
+            while (next_segment(a, smem, slot, j0, j1)) {
+                const Unit x = unit_of(a, segment_unit(slot));
+                // ring tile g holds the unit's keys from g BK - koff (koff = (gi - j0) BK);
+                // knew: the chunk's first slot in those coordinates
+                const int koff = (gi - j0) * BK, kend = x.kend + koff, knew = x.start + koff;
+                const long long row0 = static_cast<long long>((static_cast<size_t>(x.b) * a.hkv + x.kv) * a.capacity) - koff;
+                for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
+                    const int s = gi % NS;
+                    // (the ring is four tiles deep: the producer can poll slowly and
+                    // leave the issue slots of its sub-partition to the working warps)
+                    if (gi >= NS) {
+                        if (*abort_flag) goto produced;
+                        if (!ptx::mbar_wait_bounded_sleep(bar(B_EMPTY + s), ((gi - NS) / NS) & 1, WAIT_LIMIT, 256)) {
+                            fail();
+                            goto produced;
+                        }
                     }
+                    if (leader) {
+                        const int key0 = gi * BK, nk = min(BK, kend - key0);
+                        if (key0 + nk > knew) ptx::wait_prerequisites();  // the tile holds appended slots
+                        const size_t row = static_cast<size_t>(row0 + key0);
+                        const uint32_t dst = sbase + SM_STAGE + s * STAGE_BYTES;
+                        const int n8 = (nk + 7) & ~7;  // norms move in 16-byte pieces (8 keys)
+                        const uint32_t bytes = nk * (kbytes + vbytes) + (a.staged_norms ? n8 * 4 : 0);
+                        ptx::mbar_arrive_expect_tx(bar(B_FULL + s), bytes);
+                        ptx::bulk_copy_g2s(dst + ST_KC, a.k_codes + row * kbytes, nk * kbytes, bar(B_FULL + s));
+                        ptx::bulk_copy_g2s(dst + ST_VC, a.v_codes + row * vbytes, nk * vbytes, bar(B_FULL + s));
+                        if (a.staged_norms) {
+                            // capacity and the unit's key offset are multiples of 8: the
+                            // rounded range stays inside the cache
+                            ptx::bulk_copy_g2s(dst + ST_KN, a.k_norms + row, n8 * 2, bar(B_FULL + s));
+                            ptx::bulk_copy_g2s(dst + ST_VN, a.v_norms + row, n8 * 2, bar(B_FULL + s));
+                        }
+                    }
+                    __syncwarp();
                 }
+            }
+        produced:
+            // every copy issued must land before the block may exit
+            for (int k = max(0, gi - NS); k < gi; ++k)
+                ptx::mbar_wait_bounded(bar(B_FULL + k % NS), (k / NS) & 1, WAIT_LIMIT);
+        } else if (warp == MMA_WARP) {
+            // ------------------------------------------------------- MMA issuer
+            // the whole warp waits; one elected lane issues the MMAs and commits
+            const bool leader = tc::elect_one();
+            const uint32_t idesc_s = tc::idesc_f16(BM, BK), idesc_o = tc::idesc_f16_bmn(BM, D);
+            // descriptors are linear in the start address: the K slices and
+            // buffers are fixed offsets (in 16-byte units) from these
+            const uint64_t kdesc0 = tc::sw128_desc(sbase + SM_K);
+            const uint64_t vdesc0 = tc::sw128_mn_desc(sbase + SM_VT, BK * 128, 1024);
+            auto issue_s = [&](int gi) -> bool {
+                const int bf = gi & 1;
+                if (!wait(B_KFULL + bf, (gi >> 1) & 1)) return false;
+                if (gi >= 2 && !wait(B_SEMPTY + bf, ((gi - 2) >> 1) & 1)) return false;
+                tc::fence_after_sync();
                 if (leader) {
-                    const int key0 = gi * BK, nk = min(BK, kend - key0);
-                    if (key0 + nk > knew) ptx::wait_prerequisites();  // the tile holds appended slots
-                    const size_t row = static_cast<size_t>(row0 + key0);
-                    const uint32_t dst = sbase + SM_STAGE + s * STAGE_BYTES;
-                    const int n8 = (nk + 7) & ~7;  // norms move in 16-byte pieces (8 keys)
-                    const uint32_t bytes = nk * (kbytes + vbytes) + (a.staged_norms ? n8 * 4 : 0);
-                    ptx::mbar_arrive_expect_tx(bar(B_FULL + s), bytes);
-                    ptx::bulk_copy_g2s(dst + ST_KC, a.k_codes + row * kbytes, nk * kbytes, bar(B_FULL + s));
-                    ptx::bulk_copy_g2s(dst + ST_VC, a.v_codes + row * vbytes, nk * vbytes, bar(B_FULL + s));
-                    if (a.staged_norms) {
-                        // capacity and the unit's key offset are multiples of 8: the
-                        // rounded range stays inside the cache
-                        ptx::bulk_copy_g2s(dst + ST_KN, a.k_norms + row, n8 * 2, bar(B_FULL + s));
-                        ptx::bulk_copy_g2s(dst + ST_VN, a.v_norms + row, n8 * 2, bar(B_FULL + s));
+                    const uint64_t kd = kdesc0 + static_cast<uint64_t>(bf * (BK * D * 2) >> 4);
+                    const uint32_t sd = tmem + TM_S + BK * bf;
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        // 16 channels per step: 32 bytes within a 64-channel block
+                        const uint64_t bd = kd + static_cast<uint64_t>(((ks >> 2) * (BK * 128) + (ks & 3) * 32) >> 4);
+                        tc::mma_f16_ts(sd, tmem + TM_QHI + 8 * ks, bd, idesc_s, ks > 0);
+                        tc::mma_f16_ts(sd, tmem + TM_QLO + 8 * ks, bd, idesc_s, true);
                     }
+                    tc::commit(bar(B_SFULL + bf));
+                    tc::commit(bar(B_KEMPTY + bf));
                 }
                 __syncwarp();
-            }
-        }
-    produced:
-        // every copy issued must land before the block may exit
-        for (int k = max(0, gi - NS); k < gi; ++k)
-            ptx::mbar_wait_bounded(bar(B_FULL + k % NS), (k / NS) & 1, WAIT_LIMIT);
-    } else if (warp >= DEQ0 / 32 && warp < PRODUCER / 32) {
-        // ------------------------------------------------------ dequantisers
-        const int dt = tid - DEQ0;  // 0 .. 32 DEQ_WARPS - 1
-        const uint16_t* kcent = reinterpret_cast<const uint16_t*>(smem + SM_CENT);
-        const uint16_t* vcent = kcent + 16;
-        uint32_t* klut = reinterpret_cast<uint32_t*>(smem + SM_KLUT);
-        uint32_t* vlut = reinterpret_cast<uint32_t*>(smem + sm_vlut(KB));
-        build_lut<KB>(klut, kcent, dt, DEQ_WARPS * 32);
-        build_lut<VB>(vlut, vcent, dt, DEQ_WARPS * 32);
-        ptx::named_barrier(1, DEQ_WARPS * 32);
-        const uint32_t klane = sbase + SM_KLUT + 4 * lane, vlane = sbase + sm_vlut(KB) + 4 * lane;
-        int gi = 0;
-        int j0, j1;
-        while (next_segment(a, smem, slot, j0, j1)) {
-            const Unit x = unit_of(a, segment_unit(slot));
-            // ring tile g holds the unit's keys from g BK - koff (as the producer's)
-            const int koff = (gi - j0) * BK, kend = x.kend + koff;
-            const long long row0 = static_cast<long long>((static_cast<size_t>(x.b) * a.hkv + x.kv) * a.capacity) - koff;
-            for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
-                const int s = gi % NS, bf = gi & 1;
-                if (!wait(B_FULL + s, (gi / NS) & 1)) goto dequantised;
-                const uint8_t* st = smem + SM_STAGE + s * STAGE_BYTES;
-                const uint32_t sst = sbase + SM_STAGE + s * STAGE_BYTES;
-                const int key0 = gi * BK, nk = min(BK, kend - key0);
-                const size_t row = static_cast<size_t>(row0 + key0);
-                const uint16_t* skn = reinterpret_cast<const uint16_t*>(st + ST_KN);
-                // K~[bf]: 64 keys x 16 groups of 8 channels, centroids; the tile's
-                // key norms go to the softmax's ring (its tile gi - 4 is done: this
-                // tile's K~ buffer was free only after S(gi - 2), which needed the
-                // softmax to be through tile gi - 4)
-                if (gi >= 2 && !wait(B_KEMPTY + bf, ((gi - 2) >> 1) & 1)) goto dequantised;
-                if (dt < BK)
-                    reinterpret_cast<float*>(smem + SM_KNR)[(gi & 3) * BK + dt] =
-                        dt < nk ? half_bits_to_float(a.staged_norms ? skn[dt] : a.k_norms[row + dt]) : 0.f;
-                dequant_tile<KB, false>(sbase + SM_K + bf * (BK * D * 2), sst + ST_KC, klane, 0u, nullptr, true, dt,
-                                        nk);
-                tc::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(B_KFULL + bf));
-                // V~[bf]: the same per-key layout, centroids x norms
-                if (gi >= 2 && !wait(B_VEMPTY + bf, ((gi - 2) >> 1) & 1)) goto dequantised;
-                dequant_tile<VB, true>(sbase + SM_VT + bf * (BK * D * 2), sst + ST_VC, vlane, sst + ST_VN,
-                                       a.v_norms + row, a.staged_norms != 0, dt, nk);
-                tc::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    ptx::mbar_arrive(bar(B_VFULL + bf));
-                    ptx::mbar_arrive(bar(B_EMPTY + s));  // the stage's codes and norms are used
-                }
-            }
-        }
-    dequantised:;
-    } else if (warp == MMA_WARP) {
-        // ------------------------------------------------------- MMA issuer
-        // the whole warp waits; one elected lane issues the MMAs and commits
-        const bool leader = tc::elect_one();
-        const uint32_t idesc_s = tc::idesc_f16(BM, BK), idesc_o = tc::idesc_f16_bmn(BM, D);
-        // descriptors are linear in the start address: the K slices and
-        // buffers are fixed offsets (in 16-byte units) from these
-        const uint64_t kdesc0 = tc::sw128_desc(sbase + SM_K);
-        const uint64_t vdesc0 = tc::sw128_mn_desc(sbase + SM_VT, BK * 128, 1024);
-        auto issue_s = [&](int gi) -> bool {
-            const int bf = gi & 1;
-            if (!wait(B_KFULL + bf, (gi >> 1) & 1)) return false;
-            if (gi >= 2 && !wait(B_SEMPTY + bf, ((gi - 2) >> 1) & 1)) return false;
-            tc::fence_after_sync();
-            if (leader) {
-                const uint64_t kd = kdesc0 + static_cast<uint64_t>(bf * (BK * D * 2) >> 4);
-                const uint32_t sd = tmem + TM_S + BK * bf;
+                return true;
+            };
+            // first: the segment's first tile (the accumulator starts afresh)
+            auto issue_pv = [&](int gi, bool first) -> bool {
+                const int bf = gi & 1;
+                if (!wait(B_PFULL + bf, (gi >> 1) & 1)) return false;
+                if (!wait(B_VFULL + bf, (gi >> 1) & 1)) return false;
+                tc::fence_after_sync();
+                if (leader) {
+                    const uint64_t vd = vdesc0 + static_cast<uint64_t>(bf * (BK * D * 2) >> 4);
+                    const uint32_t pa = tmem + TM_P + (BK / 2) * bf;
+                    // V~ [64 keys][128 ch]: 16 keys per step = two 1024-byte K groups;
+                    // the two 64-channel blocks lie 64 rows x 128 bytes apart
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    // 16 channels per step: 32 bytes within a 64-channel block
-                    const uint64_t bd = kd + static_cast<uint64_t>(((ks >> 2) * (BK * 128) + (ks & 3) * 32) >> 4);
-                    tc::mma_f16_ts(sd, tmem + TM_QHI + 8 * ks, bd, idesc_s, ks > 0);
-                    tc::mma_f16_ts(sd, tmem + TM_QLO + 8 * ks, bd, idesc_s, true);
+                    for (int ks = 0; ks < BK / 16; ++ks)
+                        tc::mma_f16_ts(tmem + TM_O, pa + 8 * ks, vd + static_cast<uint64_t>(ks * 2048 >> 4), idesc_o,
+                                       !first || ks > 0);
+                    tc::commit(bar(B_PEMPTY + bf));
+                    tc::commit(bar(B_VEMPTY + bf));
                 }
-                tc::commit(bar(B_SFULL + bf));
-                tc::commit(bar(B_KEMPTY + bf));
+                __syncwarp();
+                return true;
+            };
+            int gi = 0, qs = 0;  // tiles issued, segments with tiles begun (the QREADY phase)
+            int j0, j1;
+            while (next_segment(a, smem, slot, j0, j1)) {
+                if (j1 <= j0) continue;  // no tiles: the softmax writes the unit's zero rows alone
+                // the segment's queries are in tensor memory (which also tells
+                // that the previous segment's output has been read)
+                if (!wait(B_QREADY, qs & 1)) break;
+                ++qs;
+                if (!issue_s(gi)) break;
+                const int gfirst = gi;
+                for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
+                    if (gi + 1 < gend && !issue_s(gi + 1)) goto issued;
+                    if (!issue_pv(gi, gi == gfirst)) goto issued;
+                }
+            }
+        issued:
+            // every tensor-core operation issued completes before the block
+            // frees its tensor memory (bounded, also after an abort)
+            if (leader) {
+                tc::commit(bar(B_FINAL));
+                ptx::mbar_wait_bounded(bar(B_FINAL), 0, WAIT_LIMIT);
             }
             __syncwarp();
-            return true;
-        };
-        // first: the segment's first tile (the accumulator starts afresh)
-        auto issue_pv = [&](int gi, bool first) -> bool {
-            const int bf = gi & 1;
-            if (!wait(B_PFULL + bf, (gi >> 1) & 1)) return false;
-            if (!wait(B_VFULL + bf, (gi >> 1) & 1)) return false;
-            tc::fence_after_sync();
-            if (leader) {
-                const uint64_t vd = vdesc0 + static_cast<uint64_t>(bf * (BK * D * 2) >> 4);
-                const uint32_t pa = tmem + TM_P + (BK / 2) * bf;
-                // V~ [64 keys][128 ch]: 16 keys per step = two 1024-byte K groups;
-                // the two 64-channel blocks lie 64 rows x 128 bytes apart
-#pragma unroll
-                for (int ks = 0; ks < BK / 16; ++ks)
-                    tc::mma_f16_ts(tmem + TM_O, pa + 8 * ks, vd + static_cast<uint64_t>(ks * 2048 >> 4), idesc_o,
-                                   !first || ks > 0);
-                tc::commit(bar(B_PEMPTY + bf));
-                tc::commit(bar(B_VEMPTY + bf));
-            }
-            __syncwarp();
-            return true;
-        };
-        int gi = 0, qs = 0;  // tiles issued, segments with tiles begun (the QREADY phase)
-        int j0, j1;
-        while (next_segment(a, smem, slot, j0, j1)) {
-            if (j1 <= j0) continue;  // no tiles: the softmax writes the unit's zero rows alone
-            // the segment's queries are in tensor memory (which also tells
-            // that the previous segment's output has been read)
-            if (!wait(B_QREADY, qs & 1)) break;
-            ++qs;
-            if (!issue_s(gi)) break;
-            const int gfirst = gi;
-            for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
-                if (gi + 1 < gend && !issue_s(gi + 1)) goto issued;
-                if (!issue_pv(gi, gi == gfirst)) goto issued;
-            }
         }
-    issued:
-        // every tensor-core operation issued completes before the block
-        // frees its tensor memory (bounded, also after an abort)
-        if (leader) {
-            tc::commit(bar(B_FINAL));
-            ptx::mbar_wait_bounded(bar(B_FINAL), 0, WAIT_LIMIT);
-        }
-        __syncwarp();
     } else if (warp < SOFTMAX_WARPS) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
         // ---------------------------------------------------------- softmax
         const int r = tid;
         const int rt = r / G, rh = r % G;
@@ -905,6 +873,58 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
             }
         }
     softmax_done:;
+    } else {
+        // ------------------------------------------------------ dequantisers
+        const int dt = tid - DEQ0;  // 0 .. 32 DEQ_WARPS - 1
+        const uint16_t* kcent = reinterpret_cast<const uint16_t*>(smem + SM_CENT);
+        const uint16_t* vcent = kcent + 16;
+        uint32_t* klut = reinterpret_cast<uint32_t*>(smem + SM_KLUT);
+        uint32_t* vlut = reinterpret_cast<uint32_t*>(smem + sm_vlut(KB));
+        build_lut<KB>(klut, kcent, dt, DEQ_WARPS * 32);
+        build_lut<VB>(vlut, vcent, dt, DEQ_WARPS * 32);
+        ptx::named_barrier(1, DEQ_WARPS * 32);
+        const uint32_t klane = sbase + SM_KLUT + 4 * lane, vlane = sbase + sm_vlut(KB) + 4 * lane;
+        int gi = 0;
+        int j0, j1;
+        while (next_segment(a, smem, slot, j0, j1)) {
+            const Unit x = unit_of(a, segment_unit(slot));
+            // ring tile g holds the unit's keys from g BK - koff (as the producer's)
+            const int koff = (gi - j0) * BK, kend = x.kend + koff;
+            const long long row0 = static_cast<long long>((static_cast<size_t>(x.b) * a.hkv + x.kv) * a.capacity) - koff;
+            for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
+                const int s = gi % NS, bf = gi & 1;
+                if (!wait(B_FULL + s, (gi / NS) & 1)) goto dequantised;
+                const uint8_t* st = smem + SM_STAGE + s * STAGE_BYTES;
+                const uint32_t sst = sbase + SM_STAGE + s * STAGE_BYTES;
+                const int key0 = gi * BK, nk = min(BK, kend - key0);
+                const size_t row = static_cast<size_t>(row0 + key0);
+                const uint16_t* skn = reinterpret_cast<const uint16_t*>(st + ST_KN);
+                // K~[bf]: 64 keys x 16 groups of 8 channels, centroids; the tile's
+                // key norms go to the softmax's ring (its tile gi - 4 is done: this
+                // tile's K~ buffer was free only after S(gi - 2), which needed the
+                // softmax to be through tile gi - 4)
+                if (gi >= 2 && !wait(B_KEMPTY + bf, ((gi - 2) >> 1) & 1)) goto dequantised;
+                if (dt < BK)
+                    reinterpret_cast<float*>(smem + SM_KNR)[(gi & 3) * BK + dt] =
+                        dt < nk ? half_bits_to_float(a.staged_norms ? skn[dt] : a.k_norms[row + dt]) : 0.f;
+                dequant_tile<KB, false>(sbase + SM_K + bf * (BK * D * 2), sst + ST_KC, klane, 0u, nullptr, true, dt,
+                                        nk);
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(B_KFULL + bf));
+                // V~[bf]: the same per-key layout, centroids x norms
+                if (gi >= 2 && !wait(B_VEMPTY + bf, ((gi - 2) >> 1) & 1)) goto dequantised;
+                dequant_tile<VB, true>(sbase + SM_VT + bf * (BK * D * 2), sst + ST_VC, vlane, sst + ST_VN,
+                                       a.v_norms + row, a.staged_norms != 0, dt, nk);
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(bar(B_VFULL + bf));
+                    ptx::mbar_arrive(bar(B_EMPTY + s));  // the stage's codes and norms are used
+                }
+            }
+        }
+    dequantised:;
     }
     tc::fence_before_sync();
     __syncthreads();
