@@ -178,6 +178,54 @@ __device__ __forceinline__ void fwht128(float (&x)[D]) {
 
 __device__ __forceinline__ uint32_t pack2(uint16_t lo, uint16_t hi) { return lo | (static_cast<uint32_t>(hi) << 16); }
 
+// One query row (D values of dtype 0 fp32, 1 bf16 or 2 fp16, 16-byte
+// aligned) into x: the dtype is chosen once and eight 16-byte loads are in
+// flight at a time (loads of four values with the dtype tested at each
+// came one after another, an L2 round trip apiece).
+__device__ __forceinline__ void load_row(const void* base, size_t off, int dtype, float (&x)[D]) {
+    if (dtype == 0) {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + off);
+#pragma unroll
+        for (int h = 0; h < D / 32; ++h) {
+            float4 v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = p[8 * h + i];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = 32 * h + 4 * i;
+                x[c] = v[i].x;
+                x[c + 1] = v[i].y;
+                x[c + 2] = v[i].z;
+                x[c + 3] = v[i].w;
+            }
+        }
+        return;
+    }
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + off);
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h) {
+        uint4 w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = p[8 * h + i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+            const int c = 64 * h + 8 * i;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (dtype == 1) {  // bf16: the upper half of an fp32
+                    x[c + 2 * k] = __uint_as_float(u[k] << 16);
+                    x[c + 2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
+                } else {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[k]));
+                    x[c + 2 * k] = f.x;
+                    x[c + 2 * k + 1] = f.y;
+                }
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
     const __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&h);
@@ -668,13 +716,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                     const size_t qoff =
                         ((static_cast<size_t>(x.b) * a.n_new + x.tok0 + rt) * a.hq + x.kv * G + rh) * D;
 #pragma unroll
-                    for (int c = 0; c < D; c += 4) {
-                        float v4[4];
-                        load4(a.q, qoff + c, a.q_dtype, v4);
+                    load_row(a.q, qoff, a.q_dtype, xq);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            xq[c + e] = flip_sign(v4[e], (a.signs[(c + e) >> 5] >> ((c + e) & 31)) & 1u);
-                    }
+                    for (int c = 0; c < D; ++c) xq[c] = flip_sign(xq[c], (a.signs[c >> 5] >> (c & 31)) & 1u);
                     fwht128(xq);
                 } else {
 #pragma unroll
