@@ -136,7 +136,17 @@ constexpr uint32_t SM_KLUT = (SM_SCHED + (SCHED_MAX + 1) * 4 + 127) & ~127u;  //
 // centroids, packed, with 32 copies interleaved word by word: entry e of lane
 // l is word 32 e + l, so a warp's lookups fall in 32 distinct banks.
 __host__ __device__ constexpr uint32_t lut_bytes(int bits) { return 32u * 4u * (1u << (2 * bits)); }
-__host__ __device__ constexpr uint32_t sm_vlut(int kb) { return SM_KLUT + lut_bytes(kb); }
+// The key table of 4-bit codes has 256-byte rows instead (entry e of lane l
+// at byte 256 e + 4 l, the upper half of each row unused), so that a lookup
+// address is one byte permute of the code word (code byte in bits 8-15, the
+// lane's offset below) and the load's immediate offset holds the table's
+// shared-window address: dynamic shared memory begins at window address
+// SMEM_WINDOW (the host checks the reserved size), where the kernel's
+// 1024-byte alignment leaves it.
+constexpr uint32_t SMEM_WINDOW = 1024;
+__host__ __device__ constexpr bool wide_klut(int kb) { return kb == 4; }
+__host__ __device__ constexpr uint32_t klut_bytes(int kb) { return wide_klut(kb) ? 65536u : lut_bytes(kb); }
+__host__ __device__ constexpr uint32_t sm_vlut(int kb) { return SM_KLUT + klut_bytes(kb); }
 __host__ __device__ constexpr uint32_t sm_alloc(int kb, int vb) { return sm_vlut(kb) + lut_bytes(vb) + 1024; }
 static_assert(sm_alloc(4, 4) <= 227u * 1024u, "the largest code tables must fit a block's shared memory");
 
@@ -318,12 +328,13 @@ __device__ __forceinline__ int part_slot(int block, int first_block) { return 2 
 
 // The code table of BITS-bit codes: field e (code e & m, then code e >> BITS)
 // -> fp16 centroid pair, for every lane.
-template <int BITS>
+// (ROW: words per entry, 32, or 64 for the 256-byte rows)
+template <int BITS, int ROW = 32>
 __device__ void build_lut(uint32_t* lut, const uint16_t* cent, int t, int nthreads) {
     constexpr int n = 32 << (2 * BITS), m = (1 << BITS) - 1;
     for (int i = t; i < n; i += nthreads) {
         const int e = i >> 5;
-        lut[i] = pack2(cent[e & m], cent[e >> BITS]);
+        lut[e * ROW + (i & 31)] = pack2(cent[e & m], cent[e >> BITS]);
     }
 }
 
@@ -335,9 +346,10 @@ __device__ void build_lut(uint32_t* lut, const uint16_t* cent, int t, int nthrea
 // groups go out together, then the lookups, then the stores.  SCALE: times
 // the key's fp16 norm (from the stage, or from `gnorms` when the stage holds
 // none).  Keys at or past nk are written as zeros.
-template <int BITS, bool SCALE>
+template <int BITS, bool SCALE, bool WIDE = false>
 __device__ __forceinline__ void dequant_tile(uint32_t tile, uint32_t codes, uint32_t lut, uint32_t snorms,
                                              const uint16_t* gnorms, bool staged, int dt, int nk) {
+    static_assert(!WIDE || BITS == 4, "the 256-byte-row table holds 4-bit code pairs");
     constexpr int RB = 16 * BITS, W = 2 * BITS, IT = BK * (D / 8) / (DEQ_WARPS * 32);
     constexpr uint32_t M = (1u << W) - 1;
     const int cg = dt & 15, k0 = dt >> 4;
@@ -365,12 +377,25 @@ __device__ __forceinline__ void dequant_tile(uint32_t tile, uint32_t codes, uint
         }
     }
     uint4 v[IT];
+    if constexpr (WIDE) {
+        // byte permute: bits 0-7 the lane's offset, bits 8-15 code byte j
+        const uint32_t l4 = 4u * static_cast<uint32_t>(dt & 31);
+        constexpr uint32_t T = SMEM_WINDOW + SM_KLUT;
 #pragma unroll
-    for (int i = 0; i < IT; ++i) {
-        v[i].x = ptx::lds32(lut + 128u * (c8[i] & M));
-        v[i].y = ptx::lds32(lut + 128u * ((c8[i] >> W) & M));
-        v[i].z = ptx::lds32(lut + 128u * ((c8[i] >> (2 * W)) & M));
-        v[i].w = ptx::lds32(lut + 128u * ((c8[i] >> (3 * W)) & M));
+        for (int i = 0; i < IT; ++i) {
+            v[i].x = ptx::lds32_imm<T>(__byte_perm(c8[i], l4, 0x7604));
+            v[i].y = ptx::lds32_imm<T>(__byte_perm(c8[i], l4, 0x7614));
+            v[i].z = ptx::lds32_imm<T>(__byte_perm(c8[i], l4, 0x7624));
+            v[i].w = ptx::lds32_imm<T>(__byte_perm(c8[i], l4, 0x7634));
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < IT; ++i) {
+            v[i].x = ptx::lds32(lut + 128u * (c8[i] & M));
+            v[i].y = ptx::lds32(lut + 128u * ((c8[i] >> W) & M));
+            v[i].z = ptx::lds32(lut + 128u * ((c8[i] >> (2 * W)) & M));
+            v[i].w = ptx::lds32(lut + 128u * ((c8[i] >> (3 * W)) & M));
+        }
     }
     if constexpr (SCALE) {
 #pragma unroll
@@ -924,7 +949,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         const uint16_t* vcent = kcent + 16;
         uint32_t* klut = reinterpret_cast<uint32_t*>(smem + SM_KLUT);
         uint32_t* vlut = reinterpret_cast<uint32_t*>(smem + sm_vlut(KB));
-        build_lut<KB>(klut, kcent, dt, DEQ_WARPS * 32);
+        build_lut<KB, wide_klut(KB) ? 64 : 32>(klut, kcent, dt, DEQ_WARPS * 32);
         build_lut<VB>(vlut, vcent, dt, DEQ_WARPS * 32);
         ptx::named_barrier(1, DEQ_WARPS * 32);
         const uint32_t klane = sbase + SM_KLUT + 4 * lane, vlane = sbase + sm_vlut(KB) + 4 * lane;
@@ -951,8 +976,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                 if (dt < BK)
                     reinterpret_cast<float*>(smem + SM_KNR)[(gi & 3) * BK + dt] =
                         dt < nk ? half_bits_to_float(a.staged_norms ? skn[dt] : a.k_norms[row + dt]) : 0.f;
-                dequant_tile<KB, false>(sbase + SM_K + bf * (BK * D * 2), sst + ST_KC, klane, 0u, nullptr, true, dt,
-                                        nk);
+                dequant_tile<KB, false, wide_klut(KB)>(sbase + SM_K + bf * (BK * D * 2), sst + ST_KC, klane, 0u, nullptr,
+                                                       true, dt, nk);
                 tc::fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bar(B_KFULL + bf));
@@ -1195,6 +1220,14 @@ extern "C" tq_status tq_prefill_attention(const tq_params* params, const tq_code
     if ((st = validate_codebook(vcb, p.head_dim, p.v_bits)) != TQ_OK) return st;
     const int sms = num_sms_current();
     if (sms <= 0) return TQ_ERR_CUDA;
+    if (prefill::wide_klut(p.k_bits)) {
+        // the 4-bit key table's lookups carry its shared-window address
+        int reserved = 0, dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+            return TQ_ERR_CUDA;
+        if (static_cast<uint32_t>(reserved) != prefill::SMEM_WINDOW) return TQ_ERR_UNSUPPORTED;
+    }
     prefill::Plan pl = prefill::plan(p, cache->batch, n_new, sms);
     if (pl.spread && pl.units * ((cache->capacity + prefill::BK - 1) / prefill::BK) >= (1LL << 31)) {
         // the shared tile sequence is counted in 32 bits: a cache long enough
