@@ -73,7 +73,8 @@ def _check_appended_codes(layer, cache, starts, n_new, kn, vn):
                 H.check_norms(norms[b, h, s0:s0 + n_new].cpu().numpy().view(np.uint16), enc["norm16"])
 
 
-@pytest.mark.parametrize("hq,hkv,kb,vb", [(32, 8, 4, 2), (64, 8, 3, 2), (8, 8, 2, 4), (16, 1, 4, 3)])
+@pytest.mark.parametrize("hq,hkv,kb,vb", [(32, 8, 4, 2), (64, 8, 3, 2), (8, 8, 2, 4), (16, 1, 4, 3), (32, 8, 4, 4),
+                                           (32, 8, 3, 3)])
 def test_prefill_matches_oracle(hq, hkv, kb, vb):
     """Two sequences with different starts; 100 new tokens: several query
     blocks (128 / G tokens each) and a ragged last one; ~13 key tiles."""
