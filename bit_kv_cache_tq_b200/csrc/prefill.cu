@@ -55,6 +55,12 @@
 //    when a score passes the reference by more than 2^8), and store the fp16
 //    weights (at most 2^8) as the A operand of P V~.  The end divides by the
 //    softmax sum and applies the inverse rotation.
+// Two idle warps complete the producer and MMA warps' warpgroup, so that the
+// block's registers can be moved between warpgroups (setmaxnreg): the
+// softmax warps run at 160 registers, the dequantising warps at 128, the
+// producer, MMA and idle warps at 96.  The attention kernel and the merge
+// kernel start as programmatic dependents of the kernel before them on the
+// stream.
 // The keys' and values' fp16 centroids carry the codebook's fp16 scale (as in
 // the decode kernels; the values' also a factor 2^-4 that keeps centroid x
 // norm inside the fp16 range), removed from the scores and the output.
