@@ -596,7 +596,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                 // ring tile g holds the unit's keys from g BK - koff (koff = (gi - j0) BK);
                 // knew: the chunk's first slot in those coordinates
                 const int koff = (gi - j0) * BK, kend = x.kend + koff, knew = x.start + koff;
-                const long long row0 = static_cast<long long>((static_cast<size_t>(x.b) * a.hkv + x.kv) * a.capacity) - koff;
+                const long long row0 =
+                    static_cast<long long>((static_cast<size_t>(x.b) * a.hkv + x.kv) * a.capacity) - koff;
                 for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
                     const int s = gi % NS;
                     // (the ring is four tiles deep: the producer can poll slowly and
@@ -965,7 +966,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
             const Unit x = unit_of(a, segment_unit(slot));
             // ring tile g holds the unit's keys from g BK - koff (as the producer's)
             const int koff = (gi - j0) * BK, kend = x.kend + koff;
-            const long long row0 = static_cast<long long>((static_cast<size_t>(x.b) * a.hkv + x.kv) * a.capacity) - koff;
+            const long long row0 =
+                static_cast<long long>((static_cast<size_t>(x.b) * a.hkv + x.kv) * a.capacity) - koff;
             for (const int gend = gi + (j1 - j0); gi < gend; ++gi) {
                 const int s = gi % NS, bf = gi & 1;
                 if (!wait(B_FULL + s, (gi / NS) & 1)) goto dequantised;
@@ -982,8 +984,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                 if (dt < BK)
                     reinterpret_cast<float*>(smem + SM_KNR)[(gi & 3) * BK + dt] =
                         dt < nk ? half_bits_to_float(a.staged_norms ? skn[dt] : a.k_norms[row + dt]) : 0.f;
-                dequant_tile<KB, false, wide_klut(KB)>(sbase + SM_K + bf * (BK * D * 2), sst + ST_KC, klane, 0u, nullptr,
-                                                       true, dt, nk);
+                dequant_tile<KB, false, wide_klut(KB)>(sbase + SM_K + bf * (BK * D * 2), sst + ST_KC, klane, 0u,
+                                                       nullptr, true, dt, nk);
                 tc::fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bar(B_KFULL + bf));
@@ -1019,6 +1021,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
 //   sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p,
 // then the inverse rotation with the butterflies of fwht128 in the same
 // order (strides 1 .. 8 within a thread, 16 .. 64 across its row's lanes).
+// (For few units, prefill_merge_rows_kernel below.)
 constexpr int MERGE_ROWS = 32, MERGE_THREADS = MERGE_ROWS * 8, MERGE_BATCH = 8;
 
 __global__ void __launch_bounds__(MERGE_THREADS) prefill_merge_kernel(const __grid_constant__ Args a, int nblocks) {
@@ -1111,6 +1114,110 @@ __global__ void __launch_bounds__(MERGE_THREADS) prefill_merge_kernel(const __gr
             v.w = flip_sign(acc[4 * q + 3] * inv_sqrt_d, (a.signs[(c + 3) >> 5] >> ((c + 3) & 31)) & 1u);
             *reinterpret_cast<float4*>(dst + c) = v;
         }
+    }
+}
+
+// The same merge for calls with few units, whose pieces are many (three or
+// more per unit): block (u, y) takes rows [8 y, 8 y + 8) of unit u, one warp
+// per row, four channels a lane.  Piece p of the unit
+// holds unnormalised rows O_p with their reference m_p (log2 units) and sum
+// l_p; the output is
+//   sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p,
+// then the inverse rotation with the butterflies of fwht128 in the same
+// order (strides 1 and 2 within a lane, 4 .. 64 across the row's lanes).
+// The pieces' (m, l) come in one lane-parallel round trip, their rows
+// RMERGE_BATCH at a time.
+constexpr int RMERGE_ROWS = 8, RMERGE_THREADS = RMERGE_ROWS * 32, RMERGE_BATCH = 16;
+constexpr long long RMERGE_MAX_UNITS = 48;  // at least three pieces a unit on 148 SMs
+
+__global__ void __launch_bounds__(RMERGE_THREADS)
+    prefill_merge_rows_kernel(const __grid_constant__ Args a, int nblocks) {
+    ptx::wait_prerequisites();  // launched as a programmatic dependent of the attention kernel
+    const uint32_t total = a.sched[a.units];
+    const int u = static_cast<int>(blockIdx.x);
+    const uint32_t pu = a.sched[u], pn = a.sched[u + 1];
+    if (total == 0 || pn <= pu) return;  // (a unit without tiles has zero rows, written by the attention kernel)
+    const uint32_t C = static_cast<uint32_t>(nblocks) > total ? total : static_cast<uint32_t>(nblocks);
+    const int ca = block_of(pu, total, C), cz = block_of(pn - 1, total, C);
+    if (ca == cz) return;
+    const int lane = static_cast<int>(threadIdx.x) & 31;
+    const int r = static_cast<int>(blockIdx.y) * RMERGE_ROWS + (static_cast<int>(threadIdx.x) >> 5);
+    const Unit x = unit_of(a, u);
+    const int G = a.group, rt = r / G, rh = r % G;
+    const bool row_ok = rt < x.ntok && rt * G + rh < BM;
+    const bool row_out = rt < min(a.tok_per_tile, a.n_new - x.tok0) && rt * G + rh < BM;
+    auto piece = [&](int c2) { return a.parts + static_cast<size_t>(part_slot(c2, ca)) * PART_FLOATS; };
+    const int np = cz - ca + 1;
+
+    // (m, l) of pieces lane, lane + 32, ...: the maximum, then each piece's
+    // weight 2^(m - M) kept by the lane that loaded it
+    float M = -INFINITY;
+    for (int j = lane; j < np; j += 32) M = fmaxf(M, __ldcg(piece(ca + j) + BM * D + r));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < np; j0 += 32) {
+        float w = 0.f;  // the weight of piece j0 + lane
+        if (j0 + lane < np) {
+            const float* sp = piece(ca + j0 + lane);
+            const float mk = __ldcg(sp + BM * D + r), lk = __ldcg(sp + BM * D + BM + r);
+            w = (mk > -INFINITY && M > -INFINITY) ? ptx::ex2(mk - M) : 0.f;
+            L = fmaf(lk, w, L);
+        }
+        const int nj = min(32, np - j0);
+        for (int b = 0; b < nj; b += RMERGE_BATCH) {
+            float4 v[RMERGE_BATCH];
+#pragma unroll
+            for (int k = 0; k < RMERGE_BATCH; ++k)
+                v[k] = b + k < nj ? __ldcg(reinterpret_cast<const float4*>(piece(ca + j0 + b + k) + r * D) + lane)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < RMERGE_BATCH; ++k) {
+                const float wk = __shfl_sync(0xffffffffu, w, (b + k) & 31);
+                if (b + k < nj) {
+                    acc.x = fmaf(v[k].x, wk, acc.x);
+                    acc.y = fmaf(v[k].y, wk, acc.y);
+                    acc.z = fmaf(v[k].z, wk, acc.z);
+                    acc.w = fmaf(v[k].w, wk, acc.w);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    const float inv = (row_ok && L > 0.f) ? a.out_scale / L : 0.f;
+    float e[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+    // strides 1 and 2 within the lane, then 4 .. 64 across lanes (bits 0 .. 4
+    // of the lane); every lane of the warp takes part (one row per warp)
+#pragma unroll
+    for (int h = 1; h < 4; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if ((i & h) == 0) {
+                const float e0 = e[i], e1 = e[i + h];
+                e[i] = e0 + e1;
+                e[i + h] = e0 - e1;
+            }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float o = __shfl_xor_sync(0xffffffffu, e[i], m);
+            e[i] = upper ? o - e[i] : e[i] + o;
+        }
+    }
+    if (row_out) {
+        const float inv_sqrt_d = 0.08838834764831845f;
+        float* dst = a.out + ((static_cast<size_t>(x.b) * a.n_new + x.tok0 + rt) * a.hq + x.kv * G + rh) * D;
+        const int c = 4 * lane;
+        float4 v;
+        v.x = flip_sign(e[0] * inv_sqrt_d, (a.signs[c >> 5] >> (c & 31)) & 1u);
+        v.y = flip_sign(e[1] * inv_sqrt_d, (a.signs[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u);
+        v.z = flip_sign(e[2] * inv_sqrt_d, (a.signs[(c + 2) >> 5] >> ((c + 2) & 31)) & 1u);
+        v.w = flip_sign(e[3] * inv_sqrt_d, (a.signs[(c + 3) >> 5] >> ((c + 3) & 31)) & 1u);
+        *reinterpret_cast<float4*>(dst + c) = v;
     }
 }
 
@@ -1295,9 +1402,18 @@ extern "C" tq_status tq_prefill_attention(const tq_params* params, const tq_code
     cudaError_t e = prefill::launch_kb(p.k_bits, p.v_bits, a, grid, s);
     if (e == cudaSuccess && pl.spread) {
         // the rows of the units cut between blocks
-        const dim3 mgrid(static_cast<unsigned>(pl.units), prefill::BM / prefill::MERGE_ROWS);
-        e = prefill::launch_dependent(prefill::prefill_merge_kernel, mgrid, dim3(prefill::MERGE_THREADS), 0u, s, a,
-                                      pl.blocks);
+        // (with few units each is cut into many pieces: a warp per row loads
+        // them with more parallelism; with many, pieces are few and the
+        // smaller grid of eight threads a row costs less)
+        if (pl.units <= prefill::RMERGE_MAX_UNITS) {
+            const dim3 mgrid(static_cast<unsigned>(pl.units), prefill::BM / prefill::RMERGE_ROWS);
+            e = prefill::launch_dependent(prefill::prefill_merge_rows_kernel, mgrid, dim3(prefill::RMERGE_THREADS), 0u,
+                                          s, a, pl.blocks);
+        } else {
+            const dim3 mgrid(static_cast<unsigned>(pl.units), prefill::BM / prefill::MERGE_ROWS);
+            e = prefill::launch_dependent(prefill::prefill_merge_kernel, mgrid, dim3(prefill::MERGE_THREADS), 0u, s, a,
+                                          pl.blocks);
+        }
     }
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
