@@ -595,7 +595,8 @@ def prefill_chunk(dev, reps=100, warmup=10, smaller=(128, 32)):
             "timing": "%d calls after %d warm-up calls, CUDA events" % (reps, warmup),
             "smaller_chunks": small,
             "kernels": "tq_prefill_attention: quantise-append of the chunk, then the tcgen05 attention kernel "
-                       "(one block per SM sharing all units' key tiles)"}
+                       "(one block per SM sharing all units' key tiles), then the merge kernel for units split "
+                       "between blocks"}
 
 
 class EagerWork:
