@@ -269,16 +269,7 @@ __device__ __forceinline__ Unit unit_of(const Args& a, int u) {
     return x;
 }
 
-// The block's share of the work as segments (unit, key tiles [j0, j1)),
-// one per call.  The iterator (the first unit not yet visited) is the
-// shared word at `slot`, so that it takes no register through the tile
-// loops; segment_unit(slot) is the unit of the segment last returned.  Spread mode: the
-// units' tiles form one sequence (P[u] tiles before unit u); with
-// C = min(blocks, total) sharing, block c takes tiles
-// [c total / C, (c + 1) total / C) of it, so a unit can be cut between
-// blocks; a unit without tiles goes to the block whose range holds its
-// start (the last block for those at the very end).  Otherwise block c is
-// unit c, whole.
+// A 32-bit store to a shared-window address.
 __device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
@@ -297,6 +288,16 @@ __device__ __forceinline__ void segment_bounds(const Args& a, const uint8_t* sme
     j1 = static_cast<int>((pn < g1 ? pn : g1) - pu);
 }
 
+// The block's share of the work as segments (unit, key tiles [j0, j1)),
+// one per call.  The iterator (the first unit not yet visited) is the
+// shared word at `slot`, so that it takes no register through the tile
+// loops; segment_unit(slot) is the unit of the segment last returned.
+// Spread mode: the units' tiles form one sequence (P[u] tiles before unit
+// u); with C = min(blocks, total) sharing, block c takes tiles
+// [c total / C, (c + 1) total / C) of it, so a unit can be cut between
+// blocks; a unit without tiles goes to the block whose range holds its
+// start (the last block for those at the very end).  Otherwise block c is
+// unit c, whole.
 __device__ __forceinline__ bool next_segment(const Args& a, const uint8_t* smem, uint32_t slot, int& j0, int& j1) {
     const int it = static_cast<int>(ptx::lds32(slot));
     if (it >= a.units || (!a.spread && it != static_cast<int>(blockIdx.x))) return false;
