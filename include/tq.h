@@ -340,7 +340,9 @@ tq_status tq_append_decode_attention(const tq_params* params, const tq_codebook*
  *   d_out         device, [batch][n_new][Hq][d] fp32.
  * Supported: d = 128, TURBO keys and values (2, 3 or 4 bits), no QJL
  * sketch, at most 16 query heads per kv head; other configurations return
- * TQ_ERR_UNSUPPORTED before any launch.  The products Q K~^T and P V~ run on
+ * TQ_ERR_UNSUPPORTED before any launch, as do 4-bit keys on a device whose
+ * reserved shared memory per block is not 1 KB (the key table's lookups
+ * carry its shared-window address; B200 reserves 1 KB).  The products Q K~^T and P V~ run on
  * the tcgen05 tensor cores (fp16 operands, fp32 accumulation in tensor
  * memory), 128 query rows (tokens x heads of a kv head's group) per block.
  * A position out of range sets TQ_DEVERR_POSITION; that sequence gets no
